@@ -1,0 +1,276 @@
+"""Pins for the oracle's attention, velocity and loop (CPU only).
+
+The velocity is checked against a second, loop-by-loop formulation on a micro
+workload, and the whole loop against closed forms (zero network, constant
+field), invariants (batch independence, GQA grouping) and exact FP8 cases.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import synthetic
+from oracle import oracle as O
+
+MICRO = synthetic.ActionExpertConfig("micro", L=2, D=8, Hq=4, Hkv=2, dh=4, F=6, H=3, A=2, B=2,
+                                     P=2, K=3, dtype="f32", time_dim=8)
+
+
+# ---------------------------------------------------------------- attention
+
+def _attention_loops(q, k, v):
+    """Scores, a running max, exp and normalisation as explicit scalar loops."""
+    Hq, n, dh = q.shape
+    Hkv, S, _ = k.shape
+    out = np.zeros((Hq, n, dh))
+    for j in range(Hq):
+        g = j // (Hq // Hkv)
+        for i in range(n):
+            sc = []
+            for s in range(S):
+                acc = 0.0
+                for d in range(dh):
+                    acc += q[j, i, d] * k[g, s, d]
+                sc.append(acc / math.sqrt(dh))
+            mx = max(sc)
+            ex = [math.exp(x - mx) for x in sc]
+            tot = sum(ex)
+            for d in range(dh):
+                out[j, i, d] = sum(ex[s] * v[g, s, d] for s in range(S)) / tot
+    return out
+
+
+def test_attention_brute_force():
+    rng = np.random.default_rng(3)
+    for Hq, Hkv, n, S, dh in ((4, 1, 3, 4, 4), (4, 2, 2, 3, 8), (2, 2, 4, 1, 2)):
+        q = rng.standard_normal((Hq, n, dh)) * 2
+        k = rng.standard_normal((Hkv, S, dh))
+        v = rng.standard_normal((Hkv, S, dh))
+        assert np.allclose(O.attention(q, k, v), _attention_loops(q, k, v), atol=1e-13)
+
+
+def test_attention_closed_forms():
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((2, 3, 8))
+    v = rng.standard_normal((1, 5, 8))
+    # all keys equal -> uniform weights -> mean of V
+    k = np.repeat(rng.standard_normal((1, 1, 8)), 5, axis=1)
+    assert np.allclose(O.attention(q, k, v), np.broadcast_to(v[0].mean(0), (2, 3, 8)), atol=1e-13)
+    # one dominant logit -> that row of V
+    k = np.zeros((1, 5, 8))
+    qd = np.zeros((1, 1, 8)); qd[0, 0, 0] = 1.0
+    k[0, 3, 0] = 1e4
+    assert np.allclose(O.attention(qd, k, v), v[0, 3], atol=1e-12)
+
+
+def test_attention_gqa_grouping_and_mha_reduction():
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((4, 3, 8))
+    k = rng.standard_normal((2, 6, 8))
+    v = rng.standard_normal((2, 6, 8))
+    o = O.attention(q, k, v)
+    # consecutive grouping: heads 0,1 read KV head 0 and heads 2,3 read KV head 1
+    kk = k[[0, 0, 1, 1]]
+    vv = v[[0, 0, 1, 1]]
+    assert np.allclose(O.attention(q, kk, vv), o, atol=1e-14)     # MHA with duplicated KV heads
+    for j, g in ((0, 0), (1, 0), (2, 1), (3, 1)):
+        assert np.allclose(O.attention(q[j:j + 1], k[g:g + 1], v[g:g + 1])[0], o[j], atol=1e-14)
+    # softmax rows sum to one
+    p = O.softmax(rng.standard_normal((5, 9)) * 30)
+    assert np.allclose(p.sum(-1), 1.0, atol=1e-14)
+
+
+# ---------------------------------------------------------------- velocity, second formulation
+
+def _matvec(W, x):
+    return [sum(W[n][c] * x[c] for c in range(len(x))) for n in range(len(W))]
+
+
+def _velocity_loops(cfg, w, x, t, pk, pv):
+    """One velocity of one sample with explicit loops (f32 workload, no rounding)."""
+    D, Hq, Hkv, dh, H, P = cfg.D, cfg.Hq, cfg.Hkv, cfg.dh, cfg.H, cfg.P
+    half_t = cfg.time_dim // 2
+    e = [math.sin(t * cfg.time_base ** (-i / half_t)) for i in range(half_t)] + \
+        [math.cos(t * cfg.time_base ** (-i / half_t)) for i in range(half_t)]
+    z1 = _matvec(w["w_t1"], e)
+    z1 = [z + b for z, b in zip(z1, w["b_t1"])]
+    z1 = [z / (1 + math.exp(-z)) for z in z1]
+    temb = [a + b for a, b in zip(_matvec(w["w_t2"], z1), w["b_t2"])]
+
+    def rms(vec, g):
+        ms = sum(a * a for a in vec) / len(vec)
+        return [a / math.sqrt(ms + cfg.eps) * gg for a, gg in zip(vec, g)]
+
+    def rot(vec, pos):
+        half = dh // 2
+        out = list(vec)
+        for j in range(half):
+            ang = pos * cfg.rope_theta ** (-2 * j / dh)
+            c, s = math.cos(ang), math.sin(ang)
+            out[j] = vec[j] * c - vec[j + half] * s
+            out[j + half] = vec[j] * s + vec[j + half] * c
+        return out
+
+    hs = []
+    for i in range(H):
+        hi = _matvec(w["w_in"], list(x[i]))
+        hs.append([a + b + c for a, b, c in zip(hi, w["b_in"], temb)])
+    for l, lw in enumerate(w["layers"]):
+        a = [rms(hs[i], lw["g1"]) for i in range(H)]
+        q = [_matvec(lw["wq"], a[i]) for i in range(H)]
+        k = [_matvec(lw["wk"], a[i]) for i in range(H)]
+        v = [_matvec(lw["wv"], a[i]) for i in range(H)]
+        new_h = []
+        for i in range(H):
+            o = []
+            for j in range(Hq):
+                g = j * Hkv // Hq
+                qi = rot(q[i][j * dh:(j + 1) * dh], P + i)
+                keys = [rot(list(pk[l][p][g]), p) for p in range(P)] + \
+                       [rot(k[r][g * dh:(g + 1) * dh], P + r) for r in range(H)]
+                vals = [list(pv[l][p][g]) for p in range(P)] + [v[r][g * dh:(g + 1) * dh] for r in range(H)]
+                sc = [sum(qi[d] * kk[d] for d in range(dh)) / math.sqrt(dh) for kk in keys]
+                mx = max(sc)
+                ex = [math.exp(s - mx) for s in sc]
+                tot = sum(ex)
+                o += [sum(ex[s] * vals[s][d] for s in range(len(vals))) / tot for d in range(dh)]
+            new_h.append([hh + oo for hh, oo in zip(hs[i], _matvec(lw["wo"], o))])
+        hs = new_h
+        for i in range(H):
+            a2 = rms(hs[i], lw["g2"])
+            gate = _matvec(lw["wg"], a2)
+            up = _matvec(lw["wu"], a2)
+            m = [0.5 * gg * (1 + math.tanh(math.sqrt(2 / math.pi) * (gg + 0.044715 * gg ** 3))) * uu
+                 for gg, uu in zip(gate, up)]
+            hs[i] = [hh + dd for hh, dd in zip(hs[i], _matvec(lw["wd"], m))]
+    out = []
+    for i in range(H):
+        f = rms(hs[i], w["g_f"])
+        out.append([a + b for a, b in zip(_matvec(w["w_out"], f), w["b_out"])])
+    return np.array(out)
+
+
+def _as_f64(w):
+    return {k: (v if k == "layers" else np.asarray(v, np.float64)) for k, v in w.items()}
+
+
+def test_velocity_matches_loop_formulation():
+    inp = synthetic.make_inputs(MICRO, seed=11)
+    w = inp["weights"]
+    # non-trivial gains and biases so that their placement is exercised
+    rng = np.random.default_rng(12)
+    for key in ("b_in", "b_out", "b_t1", "b_t2"):
+        w[key] = rng.standard_normal(w[key].shape).astype(np.float32)
+    w["g_f"] = (1 + 0.3 * rng.standard_normal(MICRO.D)).astype(np.float32)
+    for lw in w["layers"]:
+        lw["g1"] = (1 + 0.3 * rng.standard_normal(MICRO.D)).astype(np.float32)
+        lw["g2"] = (1 + 0.3 * rng.standard_normal(MICRO.D)).astype(np.float32)
+    model = O.PreparedModel(MICRO, w)
+    b = 1
+    kv_k, kv_v = O._sample_kv(model, inp["prefix_k"], inp["prefix_v"], b)
+    x = np.asarray(inp["x0"][b], np.float64)
+    for k_step, t in enumerate(O.time_grid(MICRO.K)[0]):
+        got = O.velocity(model, x, k_step, t, kv_k, kv_v)
+        want = _velocity_loops(MICRO, w, x, t, inp["prefix_k"][:, b], inp["prefix_v"][:, b])
+        # the oracle's RoPE tables are rounded to float32 once; the loops use float64 angles
+        assert np.allclose(got, want, rtol=1e-5, atol=1e-6), (got, want)
+
+
+# ---------------------------------------------------------------- loop closed forms
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "fp8"])
+def test_zero_network_leaves_x_unchanged(dtype):
+    cfg = MICRO.replace(dtype=dtype)
+    inp = synthetic.make_inputs(cfg, seed=2)
+    w = synthetic.zero_weights(cfg)
+    if dtype == "fp8":
+        # a zero tensor has no amax; give the scale a finite value to quantise with
+        for lw in w["layers"]:
+            for key in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
+                lw[key][0, 0] = 1e-30
+        scales = {(l, n): 1.0 for l in range(cfg.L) for n in O.PROJ_INPUTS}
+    else:
+        scales = None
+    out = O.denoise(cfg, w, inp["prefix_k"], inp["prefix_v"], inp["x0"], scales=scales)
+    assert np.array_equal(out, inp["x0"].astype(np.float64))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_constant_field_moves_x_by_minus_c(dtype):
+    cfg = MICRO.replace(dtype=dtype, K=10)
+    inp = synthetic.make_inputs(cfg, seed=2)
+    w = synthetic.zero_weights(cfg)
+    c = np.array([0.75, -1.5], np.float32)
+    w["b_out"] = c
+    out = O.denoise(cfg, w, inp["prefix_k"], inp["prefix_v"], inp["x0"])
+    assert np.allclose(out, inp["x0"] - c, atol=1e-13)          # K * dt * c = -c
+
+
+def test_time_only_field_integrates_the_time_mlp():
+    """Zero in-proj and layers: v = W_out RMS(temb(t_k)) + b_out depends on t only."""
+    cfg = MICRO.replace(K=4)
+    inp = synthetic.make_inputs(cfg, seed=5)
+    w = inp["weights"]
+    for lw in w["layers"]:
+        for key in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
+            lw[key][...] = 0.0
+    w["w_in"][...] = 0.0
+    rng = np.random.default_rng(9)
+    w["b_t1"] = rng.standard_normal(cfg.D).astype(np.float32)
+    out = O.denoise(cfg, w, inp["prefix_k"], inp["prefix_v"], inp["x0"])
+    model = O.PreparedModel(cfg, w)
+    ts, dt = O.time_grid(cfg.K)
+    shift = sum(dt * (O.rms_norm(model.temb(t), model.g_f, cfg.eps) @ model.w_out.T) for t in ts)
+    assert np.allclose(out, inp["x0"] + shift, atol=1e-12)
+    # every action token gets the same shift: temb is broadcast over the chunk
+    d = out - inp["x0"]
+    assert np.allclose(d, d[:, :1, :], atol=1e-12)
+
+
+def test_batch_samples_are_independent():
+    cfg = MICRO.replace(B=3, dtype="bf16")
+    inp = synthetic.make_inputs(cfg, seed=8)
+    full = O.denoise(cfg, inp["weights"], inp["prefix_k"], inp["prefix_v"], inp["x0"])
+    for b in range(3):
+        one = O.denoise(cfg, inp["weights"], inp["prefix_k"], inp["prefix_v"], inp["x0"], samples=[b])
+        assert np.array_equal(one[0], full[b])
+
+
+def test_bf16_workload_stays_close_to_f32():
+    cfg = MICRO.replace(D=32, F=64, dh=8, time_dim=16)
+    inp = synthetic.make_inputs(cfg, seed=4)
+    a = O.denoise(cfg, inp["weights"], inp["prefix_k"], inp["prefix_v"], inp["x0"])
+    b = O.denoise(cfg.replace(dtype="bf16"), inp["weights"], inp["prefix_k"], inp["prefix_v"], inp["x0"])
+    rel = np.linalg.norm(a - b) / np.linalg.norm(a)
+    assert 1e-5 < rel < 2e-2          # rounding is applied, and it is small
+
+
+def test_fp8_projection_exact_on_representable_operands():
+    cfg = MICRO.replace(dtype="fp8", L=1)
+    inp = synthetic.make_inputs(cfg, seed=6)
+    model = O.PreparedModel(cfg, inp["weights"])
+    lay = model.layers[0]
+    s_w = lay["sw_o"]
+    assert math.isclose(s_w, float(np.max(np.abs(inp["weights"]["layers"][0]["wo"]))) / 448.0)
+    codes = np.array([O.decode_e4m3(c) for c in range(0, 0x7E, 5)])
+    s_a = 0.037
+    a = codes[None, :cfg.Hq * cfg.dh] * s_a
+    (y,) = O._project(model, 0, "o", a, (lay["wo"],), {(0, "o"): s_a}, None)
+    assert np.allclose(y, a @ (lay["wo"] * s_w).T, rtol=1e-13)
+
+
+def test_calibration_scales_cover_every_projection_input():
+    cfg = MICRO.replace(dtype="fp8")
+    inp = synthetic.make_inputs(cfg, seed=1)
+    sc = O.calibrate(cfg, inp["weights"], inp["prefix_k"], inp["prefix_v"], inp["x0"])
+    assert set(sc) == {(l, n) for l in range(cfg.L) for n in O.PROJ_INPUTS}
+    assert all(v > 0 for v in sc.values())
+    # the normalised inputs of qkv/gu have |a| <= sqrt(D) (RMS = 1, unit gains)
+    for l in range(cfg.L):
+        assert sc[(l, "qkv")] * 448 <= math.sqrt(cfg.D) + 1e-12
+    arr = O.scales_to_array(cfg, sc)
+    assert O.array_to_scales(arr) == sc
+    out = O.denoise(cfg, inp["weights"], inp["prefix_k"], inp["prefix_v"], inp["x0"], scales=sc)
+    ref = O.denoise(cfg.replace(dtype="bf16"), inp["weights"], inp["prefix_k"], inp["prefix_v"], inp["x0"])
+    cos = np.sum(out * ref) / np.linalg.norm(out) / np.linalg.norm(ref)
+    assert cos > 0.99
