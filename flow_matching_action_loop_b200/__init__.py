@@ -1,0 +1,121 @@
+"""B200 flow-matching action-expert denoising loop.
+
+The compute path is libflowloop.so (CUDA kernels for sm_100a behind the C ABI
+in include/fr.h).  This package only marshals arguments: PyTorch supplies
+device memory and the current CUDA stream.  Importing it loads the library and
+fails loudly if it has not been built; there is no CPU fallback.
+
+    loop = ActionExpertLoop(cfg)            # fr_create
+    loop.load_weights(weights)              # fr_load_weights (host float32 arrays)
+    loop.set_prefix_kv(k, v)                # fr_set_prefix_kv (device tensors)
+    x_t0 = loop.denoise(x_t1)               # fr_denoise
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import numpy as np
+
+from ._abi import (  # noqa: F401
+    DTYPES, FR_DTYPE_BF16, FR_DTYPE_F32, FR_DTYPE_FP8, FR_ERR_ARG, FR_ERR_CUDA, FR_ERR_DEVICE, FR_ERR_SHAPE,
+    FR_ERR_STATE, FR_ERR_TIMEOUT, FR_ERR_UNSUPPORTED, FR_OK, FR_PATH_AUTO, FR_PATH_STEPWISE, FR_PATH_TENSOR,
+    FR_PREFIX_K_ROTATED, FrConfig, FrError, fr_calibrate, fr_create, fr_denoise, fr_destroy, fr_get_rope_tables,
+    fr_get_scales, fr_last_error, fr_launches_per_call, fr_load_weights, fr_path_name, fr_quantize_e4m3,
+    fr_read_kv, fr_rope_tables, fr_round_bf16, fr_set_prefix_kv, fr_set_scales, fr_sync_status, header_functions,
+    load_library, make_config,
+)
+
+load_library()
+
+__all__ = ["ActionExpertLoop", "FrError", "load_library", "make_config"]
+
+
+class ActionExpertLoop:
+    """One fr_handle on one GPU.  Device tensors are torch tensors; host weights are numpy arrays."""
+
+    def __init__(self, cfg, device: int = 0, B_max: Optional[int] = None, P_max: Optional[int] = None,
+                 path: int = FR_PATH_AUTO):
+        import torch
+        self._torch = torch
+        self.cfg = cfg
+        self.device = device
+        self.B_max = B_max or cfg.B
+        self.P_max = P_max or cfg.P
+        self.kv_dtype = torch.float32 if cfg.dtype == "f32" else torch.bfloat16
+        self.h = fr_create(make_config(cfg, self.B_max, self.P_max, path), device)
+
+    # -- plumbing
+    def _stream(self) -> int:
+        return self._torch.cuda.current_stream(self.device).cuda_stream
+
+    def _dev(self, t, dtype, shape, name):
+        torch = self._torch
+        if not isinstance(t, torch.Tensor) or t.device.type != "cuda" or t.dtype != dtype or not t.is_contiguous():
+            raise FrError(FR_ERR_ARG, name, f"expected a contiguous {dtype} CUDA tensor")
+        if tuple(t.shape) != tuple(shape):
+            raise FrError(FR_ERR_SHAPE, name, f"expected shape {tuple(shape)}, got {tuple(t.shape)}")
+        return t.data_ptr()
+
+    # -- the C ABI
+    @property
+    def path(self) -> str:
+        return fr_path_name(self.h)
+
+    def launches_per_call(self, B: Optional[int] = None) -> int:
+        return fr_launches_per_call(self.h, B or self.B_max)
+
+    def load_weights(self, weights: dict) -> None:
+        fr_load_weights(self.h, weights, self._stream())
+
+    def set_prefix_kv(self, k, v, rotated: bool = False) -> None:
+        c = self.cfg
+        L, B, P = k.shape[0], k.shape[1], k.shape[2]
+        shape = (L, B, P, c.Hkv, c.dh)
+        pk = self._dev(k, self.kv_dtype, shape, "fr_set_prefix_kv")
+        pv = self._dev(v, self.kv_dtype, shape, "fr_set_prefix_kv")
+        fr_set_prefix_kv(self.h, pk, pv, B, P, FR_PREFIX_K_ROTATED if rotated else 0, self._stream())
+
+    def calibrate(self, x0, k, v) -> None:
+        c = self.cfg
+        L, B, P = k.shape[0], k.shape[1], k.shape[2]
+        shape = (L, B, P, c.Hkv, c.dh)
+        fr_calibrate(self.h, self._dev(x0, self._torch.float32, (B, c.H, c.A), "fr_calibrate"),
+                     self._dev(k, self.kv_dtype, shape, "fr_calibrate"),
+                     self._dev(v, self.kv_dtype, shape, "fr_calibrate"), B, P, self._stream())
+
+    def denoise(self, x0, out=None):
+        c = self.cfg
+        B = x0.shape[0]
+        px = self._dev(x0, self._torch.float32, (B, c.H, c.A), "fr_denoise")
+        if out is None:
+            out = self._torch.empty_like(x0)
+        po = self._dev(out, self._torch.float32, (B, c.H, c.A), "fr_denoise")
+        fr_denoise(self.h, px, po, B, self._stream())
+        return out
+
+    def get_scales(self):
+        sa, sw = fr_get_scales(self.h, self.cfg.L * 4)
+        return sa.reshape(self.cfg.L, 4), sw.reshape(self.cfg.L, 4)
+
+    def set_scales(self, s_act) -> None:
+        fr_set_scales(self.h, np.asarray(s_act, np.float32).reshape(-1))
+
+    def sync_status(self) -> int:
+        return fr_sync_status(self.h, self._stream())
+
+    def read_kv(self, layer: int, b: int, n_slots: int):
+        return fr_read_kv(self.h, layer, b, n_slots, self.cfg.Hkv, self.cfg.dh, self.cfg.dtype != "f32")
+
+    def rope_tables(self, n_pos: int):
+        return fr_get_rope_tables(self.h, n_pos, self.cfg.dh)
+
+    def close(self) -> None:
+        if self.h:
+            fr_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,230 @@
+"""ctypes binding of include/fr.h: argument marshalling only.
+
+Every function here has the name of the C entry point it calls and raises
+FrError when the call returns a negative code.  Nothing of the method runs in
+Python: the loop, its kernels and the weight packer live in libflowloop.so.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import numpy as np
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libflowloop.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "fr.h")
+
+FR_OK = 0
+FR_ERR_ARG, FR_ERR_SHAPE, FR_ERR_STATE, FR_ERR_CUDA, FR_ERR_TIMEOUT, FR_ERR_DEVICE, FR_ERR_UNSUPPORTED = range(-1, -8, -1)
+FR_DTYPE_F32, FR_DTYPE_BF16, FR_DTYPE_FP8 = 0, 1, 2
+FR_PATH_AUTO, FR_PATH_STEPWISE, FR_PATH_TENSOR = 0, 1, 2
+FR_PREFIX_K_ROTATED = 1
+DTYPES = {"f32": FR_DTYPE_F32, "bf16": FR_DTYPE_BF16, "fp8": FR_DTYPE_FP8}
+ERR_NAMES = {FR_ERR_ARG: "FR_ERR_ARG", FR_ERR_SHAPE: "FR_ERR_SHAPE", FR_ERR_STATE: "FR_ERR_STATE",
+             FR_ERR_CUDA: "FR_ERR_CUDA", FR_ERR_TIMEOUT: "FR_ERR_TIMEOUT", FR_ERR_DEVICE: "FR_ERR_DEVICE",
+             FR_ERR_UNSUPPORTED: "FR_ERR_UNSUPPORTED"}
+
+
+class FrError(RuntimeError):
+    def __init__(self, code: int, func: str, msg: str):
+        super().__init__(f"{func} -> {ERR_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+class FrConfig(ctypes.Structure):
+    _fields_ = [("L", ctypes.c_int), ("D", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("dh", ctypes.c_int), ("F", ctypes.c_int), ("H", ctypes.c_int), ("A", ctypes.c_int),
+                ("B_max", ctypes.c_int), ("P_max", ctypes.c_int), ("K", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("path", ctypes.c_int), ("rope_theta", ctypes.c_float),
+                ("eps", ctypes.c_float), ("time_dim", ctypes.c_int), ("time_base", ctypes.c_float)]
+
+
+_FP = ctypes.POINTER(ctypes.c_float)
+
+
+class FrLayerWeights(ctypes.Structure):
+    _fields_ = [(n, _FP) for n in ("wq", "wk", "wv", "wo", "wg", "wu", "wd", "g1", "g2")]
+
+
+class FrWeights(ctypes.Structure):
+    _fields_ = [("layers", ctypes.POINTER(FrLayerWeights))] + \
+               [(n, _FP) for n in ("w_in", "b_in", "w_out", "b_out", "w_t1", "b_t1", "w_t2", "b_t2", "g_f")]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def header_functions():
+    """Names of the functions include/fr.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fr_[a-z0-9_]+)\s*\(", text)))
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libflowloop.so; raise if it has not been built (there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m flow_matching_action_loop_b200.build`")
+    lib = ctypes.CDLL(path)
+    c_int, c_void_p, c_uint, c_char_p = ctypes.c_int, ctypes.c_void_p, ctypes.c_uint, ctypes.c_char_p
+    H = c_void_p
+    sig = {
+        "fr_create": (c_int, [ctypes.POINTER(FrConfig), c_int, ctypes.POINTER(c_void_p)]),
+        "fr_load_weights": (c_int, [H, ctypes.POINTER(FrWeights), c_void_p]),
+        "fr_set_prefix_kv": (c_int, [H, c_void_p, c_void_p, c_int, c_int, c_uint, c_void_p]),
+        "fr_calibrate": (c_int, [H, c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p]),
+        "fr_denoise": (c_int, [H, c_void_p, c_void_p, c_int, c_void_p]),
+        "fr_get_scales": (c_int, [H, _FP, _FP, c_int]),
+        "fr_set_scales": (c_int, [H, _FP, c_int]),
+        "fr_sync_status": (c_int, [H, c_void_p]),
+        "fr_last_error": (c_char_p, []),
+        "fr_destroy": (None, [H]),
+        "fr_read_kv": (c_int, [H, c_int, c_int, c_void_p, c_void_p, c_int]),
+        "fr_get_rope_tables": (c_int, [H, _FP, _FP, c_int]),
+        "fr_path_name": (c_char_p, [H]),
+        "fr_launches_per_call": (c_int, [H, c_int]),
+        "fr_rope_tables": (c_int, [c_int, c_int, ctypes.c_double, _FP, _FP]),
+        "fr_round_bf16": (None, [_FP, ctypes.POINTER(ctypes.c_uint16), ctypes.c_size_t]),
+        "fr_quantize_e4m3": (None, [_FP, ctypes.POINTER(ctypes.c_uint8), ctypes.c_size_t, ctypes.c_double]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(rc: int, func: str) -> int:
+    if rc < 0:
+        raise FrError(rc, func, load_library().fr_last_error().decode())
+    return rc
+
+
+def _fptr(a: np.ndarray):
+    return a.ctypes.data_as(_FP)
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+def make_config(cfg, B_max: Optional[int] = None, P_max: Optional[int] = None, path: int = FR_PATH_AUTO) -> FrConfig:
+    """fr_config from any object with the action-expert size attributes."""
+    dtype = cfg.dtype if isinstance(cfg.dtype, int) else DTYPES[cfg.dtype]
+    return FrConfig(L=cfg.L, D=cfg.D, Hq=cfg.Hq, Hkv=cfg.Hkv, dh=cfg.dh, F=cfg.F, H=cfg.H, A=cfg.A,
+                    B_max=B_max or cfg.B, P_max=P_max or cfg.P, K=cfg.K, dtype=dtype, path=path,
+                    rope_theta=cfg.rope_theta, eps=cfg.eps, time_dim=cfg.time_dim, time_base=cfg.time_base)
+
+
+# ------------------------------------------------------------------ same-name wrappers
+
+def fr_create(cfg: FrConfig, device: int = 0) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(load_library().fr_create(ctypes.byref(cfg), device, ctypes.byref(h)), "fr_create")
+    return h
+
+
+def fr_load_weights(h, weights: dict, stream: int = 0) -> None:
+    """weights: the dict layout of host float32 arrays ({'layers': [...], 'w_in': ..., ...})."""
+    keep = []
+
+    def p(a):
+        a = _f32(a)
+        keep.append(a)
+        return _fptr(a)
+
+    layers = (FrLayerWeights * len(weights["layers"]))()
+    for i, lw in enumerate(weights["layers"]):
+        for n in ("wq", "wk", "wv", "wo", "wg", "wu", "wd", "g1", "g2"):
+            setattr(layers[i], n, p(lw[n]))
+    w = FrWeights(layers=layers, **{n: p(weights[n]) for n in
+                                    ("w_in", "b_in", "w_out", "b_out", "w_t1", "b_t1", "w_t2", "b_t2", "g_f")})
+    _check(load_library().fr_load_weights(h, ctypes.byref(w), stream), "fr_load_weights")
+
+
+def fr_set_prefix_kv(h, k_dev: int, v_dev: int, B: int, P: int, flags: int = 0, stream: int = 0) -> None:
+    _check(load_library().fr_set_prefix_kv(h, k_dev, v_dev, B, P, flags, stream), "fr_set_prefix_kv")
+
+
+def fr_calibrate(h, x0_dev: int, pk_dev: int, pv_dev: int, B: int, P: int, stream: int = 0) -> None:
+    _check(load_library().fr_calibrate(h, x0_dev, pk_dev, pv_dev, B, P, stream), "fr_calibrate")
+
+
+def fr_denoise(h, x0_dev: int, x_out_dev: int, B: int, stream: int = 0) -> None:
+    _check(load_library().fr_denoise(h, x0_dev, x_out_dev, B, stream), "fr_denoise")
+
+
+def fr_get_scales(h, n: int):
+    sa = np.zeros(n, np.float32)
+    sw = np.zeros(n, np.float32)
+    _check(load_library().fr_get_scales(h, _fptr(sa), _fptr(sw), n), "fr_get_scales")
+    return sa, sw
+
+
+def fr_set_scales(h, s_act) -> None:
+    s = _f32(s_act).ravel()
+    _check(load_library().fr_set_scales(h, _fptr(s), s.size), "fr_set_scales")
+
+
+def fr_sync_status(h, stream: int = 0) -> int:
+    return _check(load_library().fr_sync_status(h, stream), "fr_sync_status")
+
+
+def fr_last_error() -> str:
+    return load_library().fr_last_error().decode()
+
+
+def fr_destroy(h) -> None:
+    if h:
+        load_library().fr_destroy(h)
+
+
+def fr_read_kv(h, layer: int, b: int, n_slots: int, Hkv: int, dh: int, bf16: bool):
+    dt = np.uint16 if bf16 else np.float32
+    k = np.zeros((Hkv, n_slots, dh), dt)
+    v = np.zeros((Hkv, n_slots, dh), dt)
+    _check(load_library().fr_read_kv(h, layer, b, k.ctypes.data, v.ctypes.data, n_slots), "fr_read_kv")
+    return k, v
+
+
+def fr_get_rope_tables(h, n_pos: int, dh: int):
+    c = np.zeros((n_pos, dh // 2), np.float32)
+    s = np.zeros((n_pos, dh // 2), np.float32)
+    _check(load_library().fr_get_rope_tables(h, _fptr(c), _fptr(s), n_pos), "fr_get_rope_tables")
+    return c, s
+
+
+def fr_path_name(h) -> str:
+    return load_library().fr_path_name(h).decode()
+
+
+def fr_launches_per_call(h, B: int) -> int:
+    return load_library().fr_launches_per_call(h, B)
+
+
+def fr_rope_tables(n_pos: int, dh: int, theta: float):
+    c = np.zeros((n_pos, dh // 2), np.float32)
+    s = np.zeros((n_pos, dh // 2), np.float32)
+    _check(load_library().fr_rope_tables(n_pos, dh, theta, _fptr(c), _fptr(s)), "fr_rope_tables")
+    return c, s
+
+
+def fr_round_bf16(x) -> np.ndarray:
+    x = _f32(x)
+    out = np.zeros(x.shape, np.uint16)
+    load_library().fr_round_bf16(_fptr(x), out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)), x.size)
+    return out
+
+
+def fr_quantize_e4m3(x, scale: float) -> np.ndarray:
+    x = _f32(x)
+    out = np.zeros(x.shape, np.uint8)
+    load_library().fr_quantize_e4m3(_fptr(x), out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), x.size, scale)
+    return out

@@ -1,0 +1,656 @@
+// Runtime of the action-expert library: the handle, the weight packer and the
+// C ABI declared in fr.h.
+//
+// Design points taken from the pages (prior art, re-planned for one B200):
+//   - FlashRT walkthrough, "exec/: C ABI execution contract": named device
+//     buffers are the only state; cold start is separate from the hot call.
+//   - FlashRT walkthrough, component 7: the hot call takes pointers only and
+//     allocates nothing -- here every buffer is carved out of one allocation in
+//     fr_create.
+//   - APXInf page, section "一次跑得快，还要持续跑得稳": fixed execution path,
+//     memory allocated up front.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <algorithm>
+#include <cmath>
+#include <vector>
+
+#include "internal.h"
+#include "tensor_path.h"
+
+namespace fr {
+
+static thread_local char g_err[1024] = "";
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  set_error("CUDA error %d (%s) in %s", static_cast<int>(e), cudaGetErrorString(e), what);
+  return FR_ERR_CUDA;
+}
+
+}  // namespace fr
+
+using namespace fr;
+
+struct fr_handle {
+  fr_config cfg{};
+  int device = 0;
+  int S_max = 0;            // P_max + H KV slots per (layer, sample, kv head)
+  int n_qkv = 0, dq = 0;    // (Hq+2Hkv)dh, Hq dh
+  int wtype = W_F32;
+  size_t welem = 4;
+  int kv_bf = 0;
+  int path = FR_PATH_STEPWISE;
+  bool weights_loaded = false;
+  bool scales_set = false;
+  int prefix_B = 0, prefix_P = 0;
+
+  char* pool = nullptr;
+  size_t pool_bytes = 0;
+
+  std::vector<StepwiseWeights> lw;
+  float *w_in = nullptr, *b_in = nullptr, *w_out = nullptr, *b_out = nullptr;
+  float *w_t1 = nullptr, *b_t1 = nullptr, *w_t2 = nullptr, *b_t2 = nullptr, *g_f = nullptr;
+  float* temb = nullptr;                    // [K][D]
+  float *rope_cos = nullptr, *rope_sin = nullptr;   // [S_max][dh/2]
+  char *kv_k = nullptr, *kv_v = nullptr;    // [L][B_max][Hkv][S_max][dh]
+  size_t kv_layer_bytes = 0;
+  float *x = nullptr, *h = nullptr, *act = nullptr, *qkv = nullptr, *q = nullptr, *gu = nullptr;
+  float *s_a = nullptr, *s_w = nullptr, *alpha = nullptr;   // [L][4]
+  unsigned* amax = nullptr;                 // [L][4]
+  unsigned* status = nullptr;
+  std::vector<float> h_sw, h_sa;
+
+  TensorPath* tp = nullptr;                 // tensor-core kernel set (bf16/fp8)
+};
+
+namespace {
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Carver {
+  size_t off = 0;
+  template <typename T>
+  size_t take(size_t count, size_t align = 256) {
+    off = align_up(off, align);
+    const size_t o = off;
+    off += count * sizeof(T);
+    return o;
+  }
+};
+
+int validate(const fr_config& c) {
+  if (c.L < 1 || c.D < 1 || c.Hq < 1 || c.Hkv < 1 || c.dh < 2 || c.F < 1 || c.H < 1 || c.A < 1 ||
+      c.B_max < 1 || c.P_max < 1 || c.K < 1 || c.time_dim < 2) {
+    set_error("fr_create: every size must be positive");
+    return FR_ERR_ARG;
+  }
+  if (c.dtype < FR_DTYPE_F32 || c.dtype > FR_DTYPE_FP8 || c.path < FR_PATH_AUTO || c.path > FR_PATH_TENSOR) {
+    set_error("fr_create: bad dtype/path enum");
+    return FR_ERR_ARG;
+  }
+  if ((c.dh & 1) || (c.time_dim & 1) || (c.Hq % c.Hkv)) {
+    set_error("fr_create: dh and time_dim must be even and Hq a multiple of Hkv");
+    return FR_ERR_UNSUPPORTED;
+  }
+  if (c.A > 4096 || c.D > 16384 || c.time_dim > 4096 || c.P_max + c.H > 16384) {
+    set_error("fr_create: A <= 4096, D <= 16384, time_dim <= 4096, P_max+H <= 16384");
+    return FR_ERR_UNSUPPORTED;
+  }
+  if (c.path == FR_PATH_TENSOR && c.dtype == FR_DTYPE_F32) {
+    set_error("fr_create: the tensor-core path needs a bf16 or fp8 handle");
+    return FR_ERR_UNSUPPORTED;
+  }
+  return FR_OK;
+}
+
+int qmode_of(const fr_handle* h, bool measure) {
+  if (h->cfg.dtype == FR_DTYPE_F32) return Q_NONE;
+  if (h->cfg.dtype == FR_DTYPE_BF16) return Q_BF16;
+  return measure ? Q_MEASURE : Q_E4M3;
+}
+
+// Stepwise loop over all K steps for B samples (x already holds x0).
+void run_stepwise(fr_handle* h, int B, bool measure, cudaStream_t s) {
+  const fr_config& c = h->cfg;
+  const int T = B * c.H;
+  const int rb = c.dtype != FR_DTYPE_F32;
+  const int qm = qmode_of(h, measure);
+  const float dt = static_cast<float>(-1.0 / c.K);
+  const int P = h->prefix_P;
+  for (int k = 0; k < c.K; ++k) {
+    launch_inproj(h->x, h->w_in, h->b_in, h->temb + static_cast<size_t>(k) * c.D, h->h, T, c.D, c.A, rb, s);
+    for (int l = 0; l < c.L; ++l) {
+      const StepwiseWeights& w = h->lw[l];
+      void* kk = h->kv_k + l * h->kv_layer_bytes;
+      void* vv = h->kv_v + l * h->kv_layer_bytes;
+      const float* sa = h->s_a + l * PI_COUNT;
+      unsigned* am = h->amax + l * PI_COUNT;
+      auto alpha = [&](int i) -> const float* {
+        if (c.dtype != FR_DTYPE_FP8) return nullptr;
+        return (measure ? h->s_w : h->alpha) + l * PI_COUNT + i;
+      };
+      launch_rmsnorm_q(h->h, w.g1, h->act, T, c.D, c.eps, qm, sa + PI_QKV, am + PI_QKV, s);
+      launch_gemm(h->act, c.D, w.wqkv, h->wtype, alpha(PI_QKV), h->qkv, h->n_qkv, T, h->n_qkv, c.D, 0, s);
+      launch_rope_qkv(h->qkv, h->q, kk, vv, h->kv_bf, h->rope_cos, h->rope_sin, B, c.H, P, h->S_max,
+                      c.Hq, c.Hkv, c.dh, rb, s);
+      launch_attention(h->q, kk, vv, h->kv_bf, h->act, h->dq, B, c.H, P, h->S_max, c.Hq, c.Hkv, c.dh,
+                       qm, sa + PI_O, am + PI_O, s);
+      launch_gemm(h->act, h->dq, w.wo, h->wtype, alpha(PI_O), h->h, c.D, T, c.D, h->dq, 1, s);
+      launch_rmsnorm_q(h->h, w.g2, h->act, T, c.D, c.eps, qm, sa + PI_GU, am + PI_GU, s);
+      launch_gemm(h->act, c.D, w.wgu, h->wtype, alpha(PI_GU), h->gu, 2 * c.F, T, 2 * c.F, c.D, 0, s);
+      launch_gelu_mul(h->gu, h->act, T, c.F, qm, sa + PI_DOWN, am + PI_DOWN, s);
+      launch_gemm(h->act, c.F, w.wd, h->wtype, alpha(PI_DOWN), h->h, c.D, T, c.D, c.F, 1, s);
+    }
+    launch_final(h->h, h->g_f, h->w_out, h->b_out, h->x, T, c.D, c.A, c.eps, dt, rb, s);
+  }
+}
+
+int check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return FR_OK;
+}
+
+// Host packing helpers --------------------------------------------------------------
+void pack_rows(std::vector<uint8_t>& dst, size_t& off, const float* src, size_t n, int wtype, double scale) {
+  if (wtype == W_F32) {
+    std::memcpy(dst.data() + off, src, n * 4);
+    off += n * 4;
+  } else if (wtype == W_BF16) {
+    fr_round_bf16(src, reinterpret_cast<uint16_t*>(dst.data() + off), n);
+    off += n * 2;
+  } else {
+    fr_quantize_e4m3(src, dst.data() + off, n, scale);
+    off += n;
+  }
+}
+
+std::vector<float> rounded_f32(const float* src, size_t n, bool to_bf16) {
+  std::vector<float> out(src, src + n);
+  if (to_bf16) {
+    std::vector<uint16_t> b(n);
+    fr_round_bf16(src, b.data(), n);
+    for (size_t i = 0; i < n; ++i) {
+      const uint32_t u = static_cast<uint32_t>(b[i]) << 16;
+      std::memcpy(&out[i], &u, 4);
+    }
+  }
+  return out;
+}
+
+float max_abs(const float* p, size_t n) {
+  float m = 0.f;
+  for (size_t i = 0; i < n; ++i) m = std::max(m, std::fabs(p[i]));
+  return m;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fr_last_error(void) { return g_err; }
+
+int fr_create(const fr_config* cfg, int device, fr_handle** out) {
+  if (!cfg || !out) {
+    set_error("fr_create: NULL argument");
+    return FR_ERR_ARG;
+  }
+  *out = nullptr;
+  int rc = validate(*cfg);
+  if (rc) return rc;
+  FR_CUDA(cudaSetDevice(device));
+  fr_handle* h = new fr_handle();
+  h->cfg = *cfg;
+  h->device = device;
+  const fr_config& c = h->cfg;
+  h->S_max = c.P_max + c.H;
+  h->n_qkv = (c.Hq + 2 * c.Hkv) * c.dh;
+  h->dq = c.Hq * c.dh;
+  h->wtype = c.dtype == FR_DTYPE_F32 ? W_F32 : (c.dtype == FR_DTYPE_BF16 ? W_BF16 : W_E4M3);
+  h->welem = c.dtype == FR_DTYPE_F32 ? 4 : (c.dtype == FR_DTYPE_BF16 ? 2 : 1);
+  h->kv_bf = c.dtype != FR_DTYPE_F32;
+  h->path = c.path;
+  if (h->path == FR_PATH_AUTO) h->path = (c.dtype == FR_DTYPE_F32) ? FR_PATH_STEPWISE : FR_PATH_TENSOR;
+  if (h->path == FR_PATH_TENSOR && !tensor_path_supports(c)) {
+    if (c.path == FR_PATH_TENSOR) {
+      set_error("fr_create: sizes outside the tensor-core path (%s)", tensor_path_limits());
+      delete h;
+      return FR_ERR_UNSUPPORTED;
+    }
+    h->path = FR_PATH_STEPWISE;
+  }
+
+  const size_t T_max = static_cast<size_t>(c.B_max) * c.H;
+  const size_t D = c.D, F = c.F;
+  const size_t w_layer = (static_cast<size_t>(h->n_qkv) * D + D * h->dq + 2 * F * D + D * F);
+  const size_t act_w = std::max({D, F, static_cast<size_t>(h->dq)});
+  Carver cv;
+  std::vector<size_t> lw_off(c.L);
+  for (int l = 0; l < c.L; ++l) lw_off[l] = cv.take<uint8_t>(w_layer * h->welem);
+  const size_t o_gain = cv.take<float>(2 * D * c.L);
+  const size_t o_w_in = cv.take<float>(D * c.A), o_b_in = cv.take<float>(D);
+  const size_t o_w_out = cv.take<float>(c.A * D), o_b_out = cv.take<float>(c.A);
+  const size_t o_w_t1 = cv.take<float>(D * c.time_dim), o_b_t1 = cv.take<float>(D);
+  const size_t o_w_t2 = cv.take<float>(D * D), o_b_t2 = cv.take<float>(D), o_g_f = cv.take<float>(D);
+  const size_t o_temb = cv.take<float>(static_cast<size_t>(c.K) * D);
+  const size_t half = c.dh / 2;
+  const size_t o_cos = cv.take<float>(h->S_max * half), o_sin = cv.take<float>(h->S_max * half);
+  h->kv_layer_bytes = align_up(static_cast<size_t>(c.B_max) * c.Hkv * h->S_max * c.dh * (h->kv_bf ? 2 : 4), 256);
+  const size_t o_kvk = cv.take<uint8_t>(h->kv_layer_bytes * c.L), o_kvv = cv.take<uint8_t>(h->kv_layer_bytes * c.L);
+  const size_t o_x = cv.take<float>(T_max * c.A), o_h = cv.take<float>(T_max * D);
+  const size_t o_act = cv.take<float>(T_max * act_w), o_qkv = cv.take<float>(T_max * h->n_qkv);
+  const size_t o_q = cv.take<float>(T_max * h->dq), o_gu = cv.take<float>(T_max * 2 * F);
+  const size_t o_sa = cv.take<float>(c.L * PI_COUNT), o_sw = cv.take<float>(c.L * PI_COUNT);
+  const size_t o_alpha = cv.take<float>(c.L * PI_COUNT), o_amax = cv.take<unsigned>(c.L * PI_COUNT);
+  const size_t o_status = cv.take<unsigned>(4);
+  size_t tp_bytes = 0;
+  if (h->path == FR_PATH_TENSOR) tp_bytes = tensor_path_bytes(c);
+  const size_t o_tp = cv.take<uint8_t>(tp_bytes, 1024);
+  h->pool_bytes = align_up(cv.off, 1024);
+
+  cudaError_t e = cudaMalloc(&h->pool, h->pool_bytes);
+  if (e != cudaSuccess) {
+    delete h;
+    return cuda_fail(e, "cudaMalloc(handle pool)");
+  }
+  e = cudaMemset(h->pool, 0, h->pool_bytes);
+  if (e != cudaSuccess) {
+    cudaFree(h->pool);
+    delete h;
+    return cuda_fail(e, "cudaMemset(handle pool)");
+  }
+  char* p = h->pool;
+  h->lw.resize(c.L);
+  for (int l = 0; l < c.L; ++l) {
+    char* base = p + lw_off[l];
+    StepwiseWeights& w = h->lw[l];
+    w.wqkv = base;
+    w.wo = base + static_cast<size_t>(h->n_qkv) * D * h->welem;
+    w.wgu = static_cast<const char*>(w.wo) + D * h->dq * h->welem;
+    w.wd = static_cast<const char*>(w.wgu) + 2 * F * D * h->welem;
+    w.g1 = reinterpret_cast<float*>(p + o_gain) + 2 * D * l;
+    w.g2 = w.g1 + D;
+  }
+  h->w_in = reinterpret_cast<float*>(p + o_w_in);
+  h->b_in = reinterpret_cast<float*>(p + o_b_in);
+  h->w_out = reinterpret_cast<float*>(p + o_w_out);
+  h->b_out = reinterpret_cast<float*>(p + o_b_out);
+  h->w_t1 = reinterpret_cast<float*>(p + o_w_t1);
+  h->b_t1 = reinterpret_cast<float*>(p + o_b_t1);
+  h->w_t2 = reinterpret_cast<float*>(p + o_w_t2);
+  h->b_t2 = reinterpret_cast<float*>(p + o_b_t2);
+  h->g_f = reinterpret_cast<float*>(p + o_g_f);
+  h->temb = reinterpret_cast<float*>(p + o_temb);
+  h->rope_cos = reinterpret_cast<float*>(p + o_cos);
+  h->rope_sin = reinterpret_cast<float*>(p + o_sin);
+  h->kv_k = p + o_kvk;
+  h->kv_v = p + o_kvv;
+  h->x = reinterpret_cast<float*>(p + o_x);
+  h->h = reinterpret_cast<float*>(p + o_h);
+  h->act = reinterpret_cast<float*>(p + o_act);
+  h->qkv = reinterpret_cast<float*>(p + o_qkv);
+  h->q = reinterpret_cast<float*>(p + o_q);
+  h->gu = reinterpret_cast<float*>(p + o_gu);
+  h->s_a = reinterpret_cast<float*>(p + o_sa);
+  h->s_w = reinterpret_cast<float*>(p + o_sw);
+  h->alpha = reinterpret_cast<float*>(p + o_alpha);
+  h->amax = reinterpret_cast<unsigned*>(p + o_amax);
+  h->status = reinterpret_cast<unsigned*>(p + o_status);
+
+  // RoPE tables (R6): float64 math on the host, rounded once to float32.
+  std::vector<float> ct(h->S_max * half), st(h->S_max * half);
+  fr_rope_tables(h->S_max, c.dh, c.rope_theta, ct.data(), st.data());
+  e = cudaMemcpy(h->rope_cos, ct.data(), ct.size() * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(h->rope_sin, st.data(), st.size() * 4, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    fr_destroy(h);
+    return cuda_fail(e, "cudaMemcpy(rope tables)");
+  }
+  if (h->path == FR_PATH_TENSOR) {
+    TensorPathBuffers tb{};
+    tb.base = p + o_tp;
+    tb.bytes = tp_bytes;
+    tb.rope_cos = h->rope_cos;
+    tb.rope_sin = h->rope_sin;
+    tb.kv_k = h->kv_k;
+    tb.kv_v = h->kv_v;
+    tb.kv_layer_bytes = h->kv_layer_bytes;
+    tb.x = h->x;
+    tb.temb = h->temb;
+    tb.w_in = h->w_in;
+    tb.b_in = h->b_in;
+    tb.w_out = h->w_out;
+    tb.b_out = h->b_out;
+    tb.g_f = h->g_f;
+    tb.alpha = h->alpha;
+    tb.s_a = h->s_a;
+    tb.status = h->status;
+    rc = tensor_path_create(c, tb, &h->tp);
+    if (rc) {
+      fr_destroy(h);
+      return rc;
+    }
+  }
+  *out = h;
+  return FR_OK;
+}
+
+int fr_load_weights(fr_handle* h, const fr_weights* w, fr_stream_t stream) {
+  if (!h || !w || !w->layers || !w->w_in || !w->b_in || !w->w_out || !w->b_out || !w->w_t1 || !w->b_t1 ||
+      !w->w_t2 || !w->b_t2 || !w->g_f) {
+    set_error("fr_load_weights: NULL argument");
+    return FR_ERR_ARG;
+  }
+  const fr_config& c = h->cfg;
+  for (int l = 0; l < c.L; ++l) {
+    const fr_layer_weights& L = w->layers[l];
+    if (!L.wq || !L.wk || !L.wv || !L.wo || !L.wg || !L.wu || !L.wd || !L.g1 || !L.g2) {
+      set_error("fr_load_weights: NULL tensor in layer %d", l);
+      return FR_ERR_ARG;
+    }
+  }
+  FR_CUDA(cudaSetDevice(h->device));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t D = c.D, F = c.F, dq = h->dq, nkv = static_cast<size_t>(c.Hkv) * c.dh;
+  const bool rb = c.dtype != FR_DTYPE_F32;
+  h->h_sw.assign(static_cast<size_t>(c.L) * PI_COUNT, 1.f);
+  std::vector<uint8_t> buf;
+  std::vector<float> gains(2 * D * c.L);
+  for (int l = 0; l < c.L; ++l) {
+    const fr_layer_weights& L = w->layers[l];
+    const size_t bytes = (static_cast<size_t>(h->n_qkv) * D + D * dq + 2 * F * D + D * F) * h->welem;
+    buf.assign(bytes, 0);
+    size_t off = 0;
+    double sw[PI_COUNT] = {1, 1, 1, 1};
+    if (c.dtype == FR_DTYPE_FP8) {   // one scale per fused projection: s_w = max|w| / 448 (R11)
+      sw[PI_QKV] = std::max({max_abs(L.wq, dq * D), max_abs(L.wk, nkv * D), max_abs(L.wv, nkv * D)}) / 448.0;
+      sw[PI_O] = max_abs(L.wo, D * dq) / 448.0;
+      sw[PI_GU] = std::max(max_abs(L.wg, F * D), max_abs(L.wu, F * D)) / 448.0;
+      sw[PI_DOWN] = max_abs(L.wd, D * F) / 448.0;
+      for (int i = 0; i < PI_COUNT; ++i) {
+        if (!(sw[i] > 0)) sw[i] = 1.0;   // an all-zero tensor quantises to zero codes with any scale
+        h->h_sw[l * PI_COUNT + i] = static_cast<float>(sw[i]);
+      }
+    }
+    pack_rows(buf, off, L.wq, dq * D, h->wtype, sw[PI_QKV]);
+    pack_rows(buf, off, L.wk, nkv * D, h->wtype, sw[PI_QKV]);
+    pack_rows(buf, off, L.wv, nkv * D, h->wtype, sw[PI_QKV]);
+    pack_rows(buf, off, L.wo, D * dq, h->wtype, sw[PI_O]);
+    pack_rows(buf, off, L.wg, F * D, h->wtype, sw[PI_GU]);
+    pack_rows(buf, off, L.wu, F * D, h->wtype, sw[PI_GU]);
+    pack_rows(buf, off, L.wd, D * F, h->wtype, sw[PI_DOWN]);
+    FR_CUDA(cudaMemcpy(const_cast<void*>(h->lw[l].wqkv), buf.data(), bytes, cudaMemcpyHostToDevice));
+    std::memcpy(&gains[2 * D * l], L.g1, D * 4);
+    std::memcpy(&gains[2 * D * l + D], L.g2, D * 4);
+    if (h->tp) {
+      int rc = tensor_path_pack_layer(h->tp, l, L, sw);
+      if (rc) return rc;
+    }
+  }
+  FR_CUDA(cudaMemcpy(const_cast<float*>(h->lw[0].g1), gains.data(), gains.size() * 4, cudaMemcpyHostToDevice));
+  auto up = [&](float* dst, const float* src, size_t n, bool round) -> int {
+    std::vector<float> v = rounded_f32(src, n, round);
+    FR_CUDA(cudaMemcpy(dst, v.data(), n * 4, cudaMemcpyHostToDevice));
+    return FR_OK;
+  };
+  int rc = FR_OK;
+  if ((rc = up(h->w_in, w->w_in, D * c.A, rb))) return rc;
+  if ((rc = up(h->b_in, w->b_in, D, false))) return rc;
+  if ((rc = up(h->w_out, w->w_out, c.A * D, rb))) return rc;
+  if ((rc = up(h->b_out, w->b_out, c.A, false))) return rc;
+  if ((rc = up(h->w_t1, w->w_t1, D * c.time_dim, rb))) return rc;
+  if ((rc = up(h->b_t1, w->b_t1, D, false))) return rc;
+  if ((rc = up(h->w_t2, w->w_t2, D * D, rb))) return rc;
+  if ((rc = up(h->b_t2, w->b_t2, D, false))) return rc;
+  if ((rc = up(h->g_f, w->g_f, D, false))) return rc;
+  FR_CUDA(cudaMemcpy(h->s_w, h->h_sw.data(), h->h_sw.size() * 4, cudaMemcpyHostToDevice));
+  launch_temb(h->w_t1, h->b_t1, h->w_t2, h->b_t2, h->temb, c.D, c.time_dim, c.K, c.time_base, rb, s);
+  if ((rc = check_launch("time MLP kernel"))) return rc;
+  FR_CUDA(cudaStreamSynchronize(s));
+  if (h->tp) {
+    rc = tensor_path_finish_load(h->tp, s);
+    if (rc) return rc;
+  }
+  h->weights_loaded = true;
+  h->scales_set = false;
+  return FR_OK;
+}
+
+int fr_set_prefix_kv(fr_handle* h, const void* k_dev, const void* v_dev, int B, int P, unsigned flags,
+                     fr_stream_t stream) {
+  if (!h || !k_dev || !v_dev) {
+    set_error("fr_set_prefix_kv: NULL argument");
+    return FR_ERR_ARG;
+  }
+  const fr_config& c = h->cfg;
+  if (B < 1 || B > c.B_max || P < 1 || P > c.P_max) {
+    set_error("fr_set_prefix_kv: need 1 <= B <= %d and 1 <= P <= %d (got B=%d P=%d)", c.B_max, c.P_max, B, P);
+    return FR_ERR_SHAPE;
+  }
+  if (flags & ~FR_PREFIX_K_ROTATED) {
+    set_error("fr_set_prefix_kv: unknown flag bits 0x%x", flags);
+    return FR_ERR_ARG;
+  }
+  FR_CUDA(cudaSetDevice(h->device));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int rotate = (flags & FR_PREFIX_K_ROTATED) ? 0 : 1;
+  launch_prefix_ingest(k_dev, v_dev, h->kv_k, h->kv_v, h->kv_bf, h->rope_cos, h->rope_sin, c.L, B, c.B_max, P,
+                       h->S_max, c.Hkv, c.dh, rotate, s);
+  int rc = check_launch("prefix ingest kernel");
+  if (rc) return rc;
+  h->prefix_B = B;
+  h->prefix_P = P;
+  return FR_OK;
+}
+
+int fr_denoise(fr_handle* h, const float* x0_dev, float* x_out_dev, int B, fr_stream_t stream) {
+  if (!h || !x0_dev || !x_out_dev) {
+    set_error("fr_denoise: NULL argument");
+    return FR_ERR_ARG;
+  }
+  const fr_config& c = h->cfg;
+  if (B < 1 || B > c.B_max) {
+    set_error("fr_denoise: need 1 <= B <= %d (got %d)", c.B_max, B);
+    return FR_ERR_SHAPE;
+  }
+  if (!h->weights_loaded) {
+    set_error("fr_denoise: no weights loaded");
+    return FR_ERR_STATE;
+  }
+  if (h->prefix_B < B) {
+    set_error("fr_denoise: prefix KV set for %d samples, denoise asked for %d", h->prefix_B, B);
+    return FR_ERR_STATE;
+  }
+  if (c.dtype == FR_DTYPE_FP8 && !h->scales_set) {
+    set_error("fr_denoise: fp8 handle without activation scales (run fr_calibrate or fr_set_scales)");
+    return FR_ERR_STATE;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t xbytes = static_cast<size_t>(B) * c.H * c.A * sizeof(float);
+  if (h->path == FR_PATH_TENSOR) {
+    int rc = tensor_path_denoise(h->tp, x0_dev, x_out_dev, B, h->prefix_P, s);
+    if (rc) return rc;
+    return check_launch("tensor path");
+  }
+  FR_CUDA(cudaMemcpyAsync(h->x, x0_dev, xbytes, cudaMemcpyDeviceToDevice, s));
+  run_stepwise(h, B, false, s);
+  FR_CUDA(cudaMemcpyAsync(x_out_dev, h->x, xbytes, cudaMemcpyDeviceToDevice, s));
+  return check_launch("stepwise kernels");
+}
+
+int fr_calibrate(fr_handle* h, const float* x0_dev, const void* pk_dev, const void* pv_dev, int B, int P,
+                 fr_stream_t stream) {
+  if (!h || !x0_dev || !pk_dev || !pv_dev) {
+    set_error("fr_calibrate: NULL argument");
+    return FR_ERR_ARG;
+  }
+  const fr_config& c = h->cfg;
+  if (c.dtype != FR_DTYPE_FP8) {
+    set_error("fr_calibrate: only fp8 handles are calibrated");
+    return FR_ERR_STATE;
+  }
+  if (!h->weights_loaded) {
+    set_error("fr_calibrate: no weights loaded");
+    return FR_ERR_STATE;
+  }
+  int rc = fr_set_prefix_kv(h, pk_dev, pv_dev, B, P, 0, stream);
+  if (rc) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FR_CUDA(cudaMemsetAsync(h->amax, 0, c.L * PI_COUNT * sizeof(unsigned), s));
+  FR_CUDA(cudaMemcpyAsync(h->x, x0_dev, static_cast<size_t>(B) * c.H * c.A * 4, cudaMemcpyDeviceToDevice, s));
+  run_stepwise(h, B, true, s);
+  if ((rc = check_launch("calibration kernels"))) return rc;
+  std::vector<unsigned> am(c.L * PI_COUNT);
+  FR_CUDA(cudaMemcpyAsync(am.data(), h->amax, am.size() * 4, cudaMemcpyDeviceToHost, s));
+  FR_CUDA(cudaStreamSynchronize(s));
+  std::vector<float> sa(am.size());
+  for (size_t i = 0; i < am.size(); ++i) {
+    float a;
+    std::memcpy(&a, &am[i], 4);
+    sa[i] = a > 0.f ? a / 448.0f : 1.0f;
+  }
+  return fr_set_scales(h, sa.data(), static_cast<int>(sa.size()));
+}
+
+int fr_get_scales(const fr_handle* h, float* s_act, float* s_w, int n) {
+  if (!h || !s_act) {
+    set_error("fr_get_scales: NULL argument");
+    return FR_ERR_ARG;
+  }
+  if (h->cfg.dtype != FR_DTYPE_FP8 || !h->scales_set) {
+    set_error("fr_get_scales: not an fp8 handle or scales not set");
+    return FR_ERR_STATE;
+  }
+  if (n != h->cfg.L * PI_COUNT) {
+    set_error("fr_get_scales: n must be L*4 = %d", h->cfg.L * PI_COUNT);
+    return FR_ERR_SHAPE;
+  }
+  std::memcpy(s_act, h->h_sa.data(), n * 4);
+  if (s_w) std::memcpy(s_w, h->h_sw.data(), n * 4);
+  return FR_OK;
+}
+
+int fr_set_scales(fr_handle* h, const float* s_act, int n) {
+  if (!h || !s_act) {
+    set_error("fr_set_scales: NULL argument");
+    return FR_ERR_ARG;
+  }
+  const fr_config& c = h->cfg;
+  if (c.dtype != FR_DTYPE_FP8 || !h->weights_loaded) {
+    set_error("fr_set_scales: needs an fp8 handle with weights loaded");
+    return FR_ERR_STATE;
+  }
+  if (n != c.L * PI_COUNT) {
+    set_error("fr_set_scales: n must be L*4 = %d", c.L * PI_COUNT);
+    return FR_ERR_SHAPE;
+  }
+  for (int i = 0; i < n; ++i) {
+    if (!(s_act[i] > 0.f) || !std::isfinite(s_act[i])) {
+      set_error("fr_set_scales: scale %d is not a positive finite number", i);
+      return FR_ERR_ARG;
+    }
+  }
+  FR_CUDA(cudaSetDevice(h->device));
+  h->h_sa.assign(s_act, s_act + n);
+  std::vector<float> alpha(n);
+  for (int i = 0; i < n; ++i) alpha[i] = h->h_sa[i] * h->h_sw[i];   // alpha = act_scale x weight_scale
+  FR_CUDA(cudaMemcpy(h->s_a, h->h_sa.data(), n * 4, cudaMemcpyHostToDevice));
+  FR_CUDA(cudaMemcpy(h->alpha, alpha.data(), n * 4, cudaMemcpyHostToDevice));
+  if (h->tp) {
+    int rc = tensor_path_set_scales(h->tp, h->h_sa.data(), alpha.data());
+    if (rc) return rc;
+  }
+  h->scales_set = true;
+  return FR_OK;
+}
+
+int fr_sync_status(fr_handle* h, fr_stream_t stream) {
+  if (!h) {
+    set_error("fr_sync_status: NULL handle");
+    return FR_ERR_ARG;
+  }
+  FR_CUDA(cudaSetDevice(h->device));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned st[4] = {0, 0, 0, 0};
+  FR_CUDA(cudaMemcpyAsync(st, h->status, sizeof(st), cudaMemcpyDeviceToHost, s));
+  FR_CUDA(cudaStreamSynchronize(s));
+  FR_CUDA(cudaMemsetAsync(h->status, 0, sizeof(st), s));
+  FR_CUDA(cudaStreamSynchronize(s));
+  if (st[0] & ST_TIMEOUT) {
+    set_error("device wait gave up (phase word 0x%08x, block %u)", st[1], st[2]);
+    return FR_ERR_TIMEOUT;
+  }
+  if (st[0] & ST_BOUNDS) {
+    set_error("device bounds check failed (where 0x%08x, index %u)", st[1], st[2]);
+    return FR_ERR_DEVICE;
+  }
+  return FR_OK;
+}
+
+void fr_destroy(fr_handle* h) {
+  if (!h) return;
+  cudaSetDevice(h->device);
+  if (h->tp) tensor_path_destroy(h->tp);
+  if (h->pool) cudaFree(h->pool);
+  delete h;
+}
+
+int fr_read_kv(const fr_handle* h, int layer, int b, void* k_host, void* v_host, int n_slots) {
+  if (!h || !k_host || !v_host) {
+    set_error("fr_read_kv: NULL argument");
+    return FR_ERR_ARG;
+  }
+  const fr_config& c = h->cfg;
+  if (layer < 0 || layer >= c.L || b < 0 || b >= c.B_max || n_slots < 1 || n_slots > h->S_max) {
+    set_error("fr_read_kv: index out of range");
+    return FR_ERR_SHAPE;
+  }
+  FR_CUDA(cudaSetDevice(h->device));
+  FR_CUDA(cudaDeviceSynchronize());
+  const size_t el = h->kv_bf ? 2 : 4;
+  const size_t row = static_cast<size_t>(c.dh) * el;
+  for (int g = 0; g < c.Hkv; ++g) {
+    const size_t src = layer * h->kv_layer_bytes + ((static_cast<size_t>(b) * c.Hkv + g) * h->S_max) * row;
+    const size_t dst = static_cast<size_t>(g) * n_slots * row;
+    FR_CUDA(cudaMemcpy(static_cast<char*>(k_host) + dst, h->kv_k + src, n_slots * row, cudaMemcpyDeviceToHost));
+    FR_CUDA(cudaMemcpy(static_cast<char*>(v_host) + dst, h->kv_v + src, n_slots * row, cudaMemcpyDeviceToHost));
+  }
+  return FR_OK;
+}
+
+int fr_get_rope_tables(const fr_handle* h, float* cos_host, float* sin_host, int n_pos) {
+  if (!h || !cos_host || !sin_host) {
+    set_error("fr_get_rope_tables: NULL argument");
+    return FR_ERR_ARG;
+  }
+  if (n_pos < 1 || n_pos > h->S_max) {
+    set_error("fr_get_rope_tables: n_pos must be in [1, %d]", h->S_max);
+    return FR_ERR_SHAPE;
+  }
+  FR_CUDA(cudaSetDevice(h->device));
+  const size_t n = static_cast<size_t>(n_pos) * (h->cfg.dh / 2) * 4;
+  FR_CUDA(cudaMemcpy(cos_host, h->rope_cos, n, cudaMemcpyDeviceToHost));
+  FR_CUDA(cudaMemcpy(sin_host, h->rope_sin, n, cudaMemcpyDeviceToHost));
+  return FR_OK;
+}
+
+const char* fr_path_name(const fr_handle* h) {
+  if (!h) return "";
+  return h->path == FR_PATH_TENSOR ? "tensor" : "stepwise";
+}
+
+int fr_launches_per_call(const fr_handle* h, int B) {
+  if (!h) return 0;
+  if (h->path == FR_PATH_TENSOR) return tensor_path_launches(h->tp, B);
+  return h->cfg.K * (2 + 9 * h->cfg.L);
+}
+
+}  // extern "C"

@@ -1,0 +1,45 @@
+// Tensor-core kernel set of the action-expert library (bf16 / fp8 handles).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+
+#include "fr.h"
+
+namespace fr {
+
+// Handle-owned buffers the tensor path reads or writes (carved in fr_create).
+struct TensorPathBuffers {
+  char* base;                 // tensor_path_bytes(cfg) bytes for the path's own buffers
+  size_t bytes;
+  const float* rope_cos;      // [S_max][dh/2]
+  const float* rope_sin;
+  char* kv_k;                 // [L][B_max][Hkv][S_max][dh] bf16
+  char* kv_v;
+  size_t kv_layer_bytes;
+  float* x;                   // [B_max][H][A] state
+  const float* temb;          // [K][D]
+  const float* w_in;          // [D][A] (bf16-rounded values)
+  const float* b_in;
+  const float* w_out;         // [A][D]
+  const float* b_out;
+  const float* g_f;
+  const float* alpha;         // [L][4] fp8 GEMM epilogue scales
+  const float* s_a;           // [L][4] fp8 activation scales
+  unsigned* status;           // device status word
+};
+
+struct TensorPath;
+
+bool tensor_path_supports(const fr_config& c);
+const char* tensor_path_limits();
+size_t tensor_path_bytes(const fr_config& c);
+int tensor_path_create(const fr_config& c, const TensorPathBuffers& b, TensorPath** out);
+int tensor_path_pack_layer(TensorPath* tp, int layer, const fr_layer_weights& w, const double sw[4]);
+int tensor_path_finish_load(TensorPath* tp, cudaStream_t s);
+int tensor_path_set_scales(TensorPath* tp, const float* s_a, const float* alpha);
+int tensor_path_denoise(TensorPath* tp, const float* x0, float* x_out, int B, int P, cudaStream_t s);
+int tensor_path_launches(const TensorPath* tp, int B);
+void tensor_path_destroy(TensorPath* tp);
+
+}  // namespace fr

@@ -1,0 +1,233 @@
+/*
+ * fr.h -- C ABI of the B200 flow-matching action-expert denoising loop.
+ *
+ * The library runs the K-step Euler loop x <- x + dt * v(x, t) of a
+ * π0.5-style action expert on one GPU.  v comes from an L-layer gated
+ * transformer whose action tokens attend to a per-layer prefix KV cache that
+ * is written once and reused by every step.
+ *
+ * Shape of the boundary (sources):
+ *   - FlashRT walkthrough (m.lqnn.cn), component 7 "CUDA Graph capture": the
+ *     hot forward takes device pointers only and allocates nothing.
+ *   - same page, "exec/: C ABI execution contract": named device buffers are
+ *     the only state (KV cache, scales, noise); cold start (load, calibrate)
+ *     is separate from the hot call.
+ *   - same page, section comparing with TensorRT/vLLM/SGLang: the KV cache is a
+ *     static per-layer device buffer.
+ *   - APXInf page ("Thor 芯片上，Pi0.5推理被干到了26ms"), section "一次跑得快，
+ *     还要持续跑得稳": a fixed execution path with all memory allocated up front.
+ *
+ * Conventions
+ *   - Every call returns FR_OK (0) or a negative FR_ERR_* code and never throws.
+ *     The text of the last error of the calling thread is in fr_last_error().
+ *   - A handle is not thread-safe.  It owns every device buffer it allocates;
+ *     all device memory is allocated in fr_create and freed in fr_destroy.
+ *   - Pointers passed in are borrowed: host pointers for the duration of the
+ *     call, device pointers until the work queued on `stream` has finished.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     that take a stream are asynchronous unless stated otherwise.
+ *   - Device-side failures (a bounded wait that gave up, a device bounds check)
+ *     are latched in a device status word; fr_sync_status() reads and clears it.
+ */
+#ifndef FR_H_
+#define FR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fr_stream_t;   /* same type as cudaStream_t */
+typedef struct fr_handle fr_handle;
+
+enum {
+  FR_OK = 0,
+  FR_ERR_ARG = -1,          /* NULL pointer, negative size, bad enum */
+  FR_ERR_SHAPE = -2,        /* B > B_max, P > P_max, sizes that do not fit the config */
+  FR_ERR_STATE = -3,        /* e.g. denoise before weights / prefix, fp8 without scales */
+  FR_ERR_CUDA = -4,         /* a CUDA runtime call failed (message has the CUDA error) */
+  FR_ERR_TIMEOUT = -5,      /* a bounded device wait gave up */
+  FR_ERR_DEVICE = -6,       /* a device-side bounds check failed */
+  FR_ERR_UNSUPPORTED = -7   /* configuration outside what the kernels implement */
+};
+
+enum { FR_DTYPE_F32 = 0, FR_DTYPE_BF16 = 1, FR_DTYPE_FP8 = 2 };
+
+/* Kernel set used by fr_denoise.  FR_PATH_AUTO picks the tensor-core path for
+ * bf16/fp8 and the CUDA-core path for f32.  FR_PATH_STEPWISE forces the simple
+ * one-kernel-per-operation CUDA-core path (used by fp8 calibration as well). */
+enum { FR_PATH_AUTO = 0, FR_PATH_STEPWISE = 1, FR_PATH_TENSOR = 2 };
+
+/* Flags of fr_set_prefix_kv. */
+#define FR_PREFIX_K_ROTATED 1u   /* prefix K already carries RoPE at positions 0..P-1 */
+
+/*
+ * Sizes of one action expert.  Architecture per the workload descriptions:
+ * pre-norm RMSNorm (eps), fused QKV projection, grouped-query attention with
+ * rotate-half RoPE (rope_theta), merged gate|up projection with GeLU(tanh) on
+ * the gate, sinusoidal time embedding (time_dim, time_base) fed through
+ * Linear-SiLU-Linear and added to the in-projected action tokens.
+ */
+typedef struct fr_config {
+  int L;          /* layers */
+  int D;          /* width */
+  int Hq, Hkv;    /* query heads, key/value heads (Hq % Hkv == 0) */
+  int dh;         /* head dim (even) */
+  int F;          /* MLP width of gate and of up */
+  int H;          /* action tokens per chunk */
+  int A;          /* action dim */
+  int B_max;      /* largest batch fr_denoise will see */
+  int P_max;      /* largest prefix length */
+  int K;          /* Euler steps from t=1 to t=0, dt = -1/K */
+  int dtype;      /* FR_DTYPE_* of the layer projections */
+  int path;       /* FR_PATH_* */
+  float rope_theta;
+  float eps;
+  int time_dim;
+  float time_base;
+} fr_config;
+
+/* Host float32 weights of one layer, row-major [out][in] (the nn.Linear convention). */
+typedef struct fr_layer_weights {
+  const float* wq;   /* [Hq*dh][D]  */
+  const float* wk;   /* [Hkv*dh][D] */
+  const float* wv;   /* [Hkv*dh][D] */
+  const float* wo;   /* [D][Hq*dh]  */
+  const float* wg;   /* [F][D] gate */
+  const float* wu;   /* [F][D] up   */
+  const float* wd;   /* [D][F] down */
+  const float* g1;   /* [D] pre-attention RMSNorm gain */
+  const float* g2;   /* [D] pre-MLP RMSNorm gain */
+} fr_layer_weights;
+
+/* Host float32 weights of the action expert, by name. */
+typedef struct fr_weights {
+  const fr_layer_weights* layers;   /* L entries */
+  const float* w_in;   /* [D][A] */
+  const float* b_in;   /* [D] */
+  const float* w_out;  /* [A][D] */
+  const float* b_out;  /* [A] */
+  const float* w_t1;   /* [D][time_dim] */
+  const float* b_t1;   /* [D] */
+  const float* w_t2;   /* [D][D] */
+  const float* b_t2;   /* [D] */
+  const float* g_f;    /* [D] final RMSNorm gain */
+} fr_weights;
+
+/*
+ * fr_create -- validate the config, make `device` current and allocate ALL
+ * device memory of the handle: packed weights, the KV cache
+ * [L][B_max][Hkv][P_max+H][dh], activations, workspaces and status words.
+ * Errors: FR_ERR_ARG (NULL), FR_ERR_UNSUPPORTED (sizes the kernels do not
+ * implement), FR_ERR_CUDA (allocation).  *out is NULL on error.
+ */
+int fr_create(const fr_config* cfg, int device, fr_handle** out);
+
+/*
+ * fr_load_weights -- pack host float32 weights into the handle
+ * (PhyAI page, optimisation paragraph: Q/K/V fused into one GEMM, gate and up
+ * merged; FlashRT walkthrough, component 4: declarative weight loading with
+ * transpose/fuse/FP8-quantise transforms).  The packer concatenates
+ * W_qkv = [W_q; W_k; W_v] and W_gu = [W_gate; W_up], rounds to bf16 (RNE) or,
+ * for FR_DTYPE_FP8, quantises each fused projection to e4m3 with
+ * s_w = max|w| / 448, and precomputes the K time embeddings and the RoPE
+ * tables.  Synchronous with respect to the host pointers; the caller keeps
+ * ownership of `w`.  Errors: FR_ERR_ARG, FR_ERR_CUDA.
+ */
+int fr_load_weights(fr_handle* h, const fr_weights* w, fr_stream_t stream);
+
+/*
+ * fr_set_prefix_kv -- copy the per-layer prefix keys/values into the static KV
+ * cache (FlashRT walkthrough: static per-layer KV buffers, computed once and
+ * reused).  k_dev, v_dev: device [L][B][P][Hkv][dh], float32 for FR_DTYPE_F32
+ * handles and bf16 otherwise.  Unless FR_PREFIX_K_ROTATED is set, K is rotated
+ * at positions 0..P-1 on the way in.  The prefix stays until replaced.
+ * Errors: FR_ERR_ARG, FR_ERR_SHAPE (B > B_max, P > P_max, P < 1), FR_ERR_CUDA.
+ */
+int fr_set_prefix_kv(fr_handle* h, const void* k_dev, const void* v_dev, int B, int P,
+                     unsigned flags, fr_stream_t stream);
+
+/*
+ * fr_calibrate -- FP8 measure pass (FlashRT walkthrough, component 6, stage
+ * (a)): run the whole K-step loop once on (x0_dev, prefix) with e4m3 weights
+ * dequantised and projection inputs unquantised, record max|a| of each of the
+ * 4 projection inputs of every layer over all steps, tokens and samples, then
+ * set s_a = amax / 448 and alpha = s_a * s_w (stage (b)).  The calibration
+ * prefix replaces the handle's prefix KV: call fr_set_prefix_kv afterwards.
+ * Synchronises `stream`.  Errors: FR_ERR_STATE (not an fp8 handle, no
+ * weights), FR_ERR_SHAPE, FR_ERR_CUDA.
+ */
+int fr_calibrate(fr_handle* h, const float* x0_dev, const void* pk_dev, const void* pv_dev,
+                 int B, int P, fr_stream_t stream);
+
+/*
+ * fr_denoise -- the hot call: run K Euler steps on B chunks.
+ * x0_dev: device float32 [B][H][A] noise at t=1; x_out_dev: device float32
+ * [B][H][A] actions at t=0 (may alias x0_dev).  Asynchronous on `stream`,
+ * allocates nothing.  Errors: FR_ERR_ARG, FR_ERR_SHAPE (B > B_max or B < 1),
+ * FR_ERR_STATE (no weights, no prefix for these B samples, fp8 without
+ * scales), FR_ERR_CUDA.  Device-side failures surface in fr_sync_status.
+ */
+int fr_denoise(fr_handle* h, const float* x0_dev, float* x_out_dev, int B, fr_stream_t stream);
+
+/*
+ * fr_get_scales / fr_set_scales -- export/import FP8 calibration.
+ * s_act: host [L][4] activation scales in the order (qkv input, o input,
+ * gate|up input, down input); s_w: host [L][4] weight scales, same order
+ * (may be NULL).  n must be L*4.  fr_set_scales also recomputes alpha.
+ * Errors: FR_ERR_ARG, FR_ERR_STATE (not fp8, or scales not set for get).
+ */
+int fr_get_scales(const fr_handle* h, float* s_act, float* s_w, int n);
+int fr_set_scales(fr_handle* h, const float* s_act, int n);
+
+/*
+ * fr_sync_status -- synchronise `stream`, read and clear the device status
+ * word.  Returns FR_OK, FR_ERR_TIMEOUT or FR_ERR_DEVICE (message says where).
+ */
+int fr_sync_status(fr_handle* h, fr_stream_t stream);
+
+/* Text of the last error on the calling thread ("" if none).  Never NULL. */
+const char* fr_last_error(void);
+
+/* Free every device buffer of the handle.  NULL is a no-op. */
+void fr_destroy(fr_handle* h);
+
+/* ---- introspection (verification and tooling; not on the hot path) ---- */
+
+/*
+ * fr_read_kv -- copy layer `layer`, sample `b` of the KV cache to host:
+ * k_host, v_host receive [Hkv][n_slots][dh] in the cache's storage type
+ * (float32 for f32 handles, bf16 bits otherwise), n_slots = P + H (prefix
+ * slots first, then the action slots of the last step).  Synchronous.
+ */
+int fr_read_kv(const fr_handle* h, int layer, int b, void* k_host, void* v_host, int n_slots);
+
+/* Copy the handle's RoPE tables [n_pos][dh/2] to host (n_pos <= P_max + H). */
+int fr_get_rope_tables(const fr_handle* h, float* cos_host, float* sin_host, int n_pos);
+
+/* Name of the kernel set fr_denoise runs ("stepwise" or "tensor"). */
+const char* fr_path_name(const fr_handle* h);
+
+/* Number of kernel launches one fr_denoise call issues for batch B. */
+int fr_launches_per_call(const fr_handle* h, int B);
+
+/* ---- host number-format utilities used by the packer (no GPU needed) ---- */
+
+/* RoPE tables: cos/sin of pos * theta^(-2j/dh) for pos < n_pos, j < dh/2, float64
+ * math rounded once to float32 (rotate-half pairing (j, j + dh/2)). */
+int fr_rope_tables(int n_pos, int dh, double theta, float* cos_out, float* sin_out);
+
+/* float32 -> bf16 bits, round to nearest even (NaN stays NaN). */
+void fr_round_bf16(const float* in, uint16_t* out, size_t n);
+
+/* float32 -> e4m3 bytes of in[i] / scale computed in float64: saturate to +-448,
+ * round to nearest even (OCP E4M3, no infinities, NaN -> 0x7F). */
+void fr_quantize_e4m3(const float* in, uint8_t* out, size_t n, double scale);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FR_H_ */

@@ -1,0 +1,78 @@
+"""C-ABI library on the host (no GPU): it loads, exports every declared symbol,
+and its packer's number formats agree bit for bit with the oracle's own.
+"""
+import ctypes
+import subprocess
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from flow_matching_action_loop_b200 import _abi
+    _abi.load_library()
+    return _abi
+
+
+def test_every_header_function_is_exported(abi):
+    names = abi.header_functions()
+    assert len(names) >= 17
+    out = subprocess.run(["nm", "-D", "--defined-only", abi.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    lib = ctypes.CDLL(abi.LIB_PATH)
+    for n in names:
+        assert getattr(lib, n) is not None
+
+
+def test_rope_tables_byte_identical_to_oracle(abi):
+    for n_pos, dh, theta in ((866, 256, 1e4), (2148, 128, 1e4), (80, 64, 1e4), (7, 2, 500.0)):
+        c, s = abi.fr_rope_tables(n_pos, dh, theta)
+        oc, os_ = O.rope_tables(n_pos, dh, theta)
+        assert c.tobytes() == oc.tobytes() and s.tobytes() == os_.tobytes()
+
+
+def test_packer_bf16_matches_oracle_rounding(abi):
+    rng = np.random.default_rng(0)
+    x = (rng.standard_normal(300000) / 32).astype(np.float32)
+    bits = abi.fr_round_bf16(x)
+    vals = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.array_equal(vals, O.round_bf16(x.astype(np.float64)))
+
+
+def test_packer_e4m3_matches_oracle_quantiser(abi):
+    rng = np.random.default_rng(1)
+    w = (rng.standard_normal(200000) / 32).astype(np.float32)
+    s_w = float(np.max(np.abs(w.astype(np.float64)))) / 448.0
+    codes = abi.fr_quantize_e4m3(w, s_w)
+    decoded = np.array([O.decode_e4m3(int(c)) for c in range(256)])[codes]
+    assert np.array_equal(decoded, O.round_e4m3(w.astype(np.float64) / s_w))
+    # saturation, zero, and the NaN code
+    special = np.array([1e9, -1e9, 0.0, -0.0, np.nan], np.float32)
+    assert list(abi.fr_quantize_e4m3(special, 1.0)) == [0x7E, 0xFE, 0x00, 0x80, 0x7F]
+
+
+def test_invalid_configs_rejected_before_any_device_work(abi):
+    import synthetic
+    base = synthetic.CONFIGS["tiny_f32"]
+    bad = [
+        (abi.make_config(base.replace(dh=63)), abi.FR_ERR_UNSUPPORTED),
+        (abi.make_config(base.replace(Hq=3, Hkv=2)), abi.FR_ERR_UNSUPPORTED),
+        (abi.make_config(base.replace(L=0)), abi.FR_ERR_ARG),
+        (abi.make_config(base, path=7), abi.FR_ERR_ARG),
+        (abi.make_config(base, path=abi.FR_PATH_TENSOR), abi.FR_ERR_UNSUPPORTED),   # f32 has no tensor path
+    ]
+    for cfg, code in bad:
+        with pytest.raises(abi.FrError) as ei:
+            abi.fr_create(cfg, 0)
+        assert ei.value.code == code, abi.fr_last_error()
+    lib = abi.load_library()
+    h = ctypes.c_void_p()
+    assert lib.fr_create(None, 0, ctypes.byref(h)) == abi.FR_ERR_ARG
+    assert lib.fr_denoise(None, None, None, 1, None) == abi.FR_ERR_ARG
+    assert lib.fr_last_error() != b""
+    lib.fr_destroy(None)   # no-op
