@@ -1,20 +1,562 @@
-// Tensor-core kernel set: not built yet; every handle uses the stepwise kernels.
+// Host side of the tensor-core path: weight pre-tiling, launch plan, CUDA-graph capture.
+//
+// Prior art and what changes here: the PhyAI page (optimisation paragraph) replays the
+// ten-step Euler iteration of π0.5 from a CUDA graph and fuses the Q/K/V and gate/up
+// projections; the FlashRT walkthrough (component 7) captures a pointer-only forward.
+// This path captures every kernel of one call (K steps x L layers) into one graph whose
+// kernels are chained by programmatic dependent launch, so each GEMM kernel streams
+// its weights while its predecessor is still running.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <utility>
+#include <vector>
+
 #include "internal.h"
+#include "tc_kernels.h"
 #include "tensor_path.h"
 
 namespace fr {
 
-struct TensorPath {};
+using namespace fr::tc;
 
-bool tensor_path_supports(const fr_config&) { return false; }
-const char* tensor_path_limits() { return "tensor-core path not available"; }
-size_t tensor_path_bytes(const fr_config&) { return 0; }
-int tensor_path_create(const fr_config&, const TensorPathBuffers&, TensorPath**) { return FR_ERR_UNSUPPORTED; }
-int tensor_path_pack_layer(TensorPath*, int, const fr_layer_weights&, const double*) { return FR_ERR_UNSUPPORTED; }
-int tensor_path_finish_load(TensorPath*, cudaStream_t) { return FR_ERR_UNSUPPORTED; }
-int tensor_path_set_scales(TensorPath*, const float*, const float*) { return FR_ERR_UNSUPPORTED; }
-int tensor_path_denoise(TensorPath*, const float*, float*, int, int, cudaStream_t) { return FR_ERR_UNSUPPORTED; }
-int tensor_path_launches(const TensorPath*, int) { return 0; }
-void tensor_path_destroy(TensorPath*) {}
+namespace {
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+struct ProjLayout {
+  int rows = 0;      // output rows after permutation (padded to MB*BM)
+  int K = 0;         // input features
+  int MB = 0, NKC = 0;
+  size_t bytes = 0;  // tiled bytes per layer
+};
+
+ProjLayout make_layout(int rows, int K, int elem) {
+  ProjLayout p;
+  p.rows = rows;
+  p.K = K;
+  p.MB = ceil_div(rows, BM);
+  p.NKC = ceil_div(K * elem, KCB);
+  p.bytes = static_cast<size_t>(p.MB) * p.NKC * BM * KCB;
+  return p;
+}
+
+struct GemmPlan {
+  int S = 1, stages = 1;
+};
+
+struct StepPlan {
+  int B = 0, P = 0, T = 0, NT = 0, Nt = 0;
+  GemmPlan qkv, o, gu, dn;
+  int attn_C = 1, attn_KC = 64;
+};
+
+struct GraphEntry {
+  cudaGraphExec_t exec = nullptr;
+  std::vector<cudaGraphNode_t> x_in_nodes;   // nodes whose x input is the caller's x0
+  std::vector<cudaGraphNode_t> x_out_nodes;  // nodes whose output is the caller's x_out
+  const float* x0 = nullptr;
+  float* x_out = nullptr;
+  StepPlan plan;
+};
+
+}  // namespace
+
+struct TensorPath {
+  fr_config c{};
+  TensorPathBuffers tb{};
+  int nsm = 148;
+  int max_dyn = 0;
+  int fp8 = 0, elem = 2;
+  int T_max = 0, T_pad = 0, MBd = 0, MB_rot = 0;
+  ProjLayout qkv, o, gu, dn;
+  size_t layer_bytes = 0;
+  uint8_t* w = nullptr;          // [L][qkv|o|gu|dn] tiled weights
+  float* gains = nullptr;        // [L][2][D]
+  float* h = nullptr;            // [T_max][D]
+  float* ssq_a = nullptr;        // [MBd][T_pad]
+  float* ssq_b = nullptr;
+  __nv_bfloat16* qbuf = nullptr; // [B_max][Hq][H][dh]
+  uint8_t* obuf = nullptr;       // [T_max][Hq dh] bf16 / e4m3
+  uint8_t* ubuf = nullptr;       // [T_max][F]
+  float* xs = nullptr;           // [T_max][A] state between steps
+  cudaStream_t cap = nullptr;
+  std::map<std::pair<int, int>, GraphEntry> graphs;
+  std::vector<float> gains_host;
+};
+
+namespace {
+
+struct Carve {
+  char* base;         // nullptr: only measure
+  size_t off = 0;
+  template <typename T>
+  T* take(size_t count, size_t align = 256) {
+    off = align_up(off, align);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+void layouts(const fr_config& c, int elem, ProjLayout& qkv, ProjLayout& o, ProjLayout& gu, ProjLayout& dn) {
+  qkv = make_layout((c.Hq + 2 * c.Hkv) * c.dh, c.D, elem);
+  o = make_layout(c.D, c.Hq * c.dh, elem);
+  gu = make_layout(2 * c.F, c.D, elem);
+  dn = make_layout(c.D, c.F, elem);
+}
+
+size_t carve_all(TensorPath* tp, char* base) {
+  const fr_config& c = tp->c;
+  Carve cv{base};
+  tp->w = cv.take<uint8_t>(tp->layer_bytes * c.L, 1024);
+  tp->gains = cv.take<float>(static_cast<size_t>(c.L) * 2 * c.D);
+  tp->h = cv.take<float>(static_cast<size_t>(tp->T_max) * c.D);
+  tp->ssq_a = cv.take<float>(static_cast<size_t>(tp->MBd) * tp->T_pad);
+  tp->ssq_b = cv.take<float>(static_cast<size_t>(tp->MBd) * tp->T_pad);
+  tp->qbuf = cv.take<__nv_bfloat16>(static_cast<size_t>(c.B_max) * c.Hq * c.H * c.dh);
+  tp->obuf = cv.take<uint8_t>(static_cast<size_t>(tp->T_max) * c.Hq * c.dh * tp->elem);
+  tp->ubuf = cv.take<uint8_t>(static_cast<size_t>(tp->T_max) * c.F * tp->elem);
+  tp->xs = cv.take<float>(static_cast<size_t>(tp->T_max) * c.A);
+  return align_up(cv.off, 1024);
+}
+
+void init_sizes(TensorPath* tp, const fr_config& c) {
+  tp->c = c;
+  tp->fp8 = c.dtype == FR_DTYPE_FP8;
+  tp->elem = tp->fp8 ? 1 : 2;
+  tp->T_max = c.B_max * c.H;
+  tp->T_pad = static_cast<int>(align_up(tp->T_max, 16));
+  tp->MBd = ceil_div(c.D, BM);
+  tp->MB_rot = (c.Hq + c.Hkv) * c.dh / 2 / 64;
+  layouts(c, tp->elem, tp->qkv, tp->o, tp->gu, tp->dn);
+  tp->layer_bytes = tp->qkv.bytes + tp->o.bytes + tp->gu.bytes + tp->dn.bytes;
+}
+
+// Split-K / ring choice for one projection: a small cost model over S (cluster size).
+GemmPlan choose_plan(int tiles, int NKC, int Nt, int nsm, int max_dyn) {
+  const size_t slot = BM * KCB + static_cast<size_t>(Nt) * KCB;
+  const size_t red = static_cast<size_t>(Nt) * (BM + 4) * 4;
+  GemmPlan best;
+  double best_cost = 1e30;
+  for (int S = 1; S <= 16 && S <= NKC; ++S) {
+    const int chunks = ceil_div(NKC, S);
+    int stages = std::min(chunks, MAX_STAGES);
+    while (stages > 1 && std::max(stages * slot, red) > static_cast<size_t>(max_dyn)) --stages;
+    const size_t smem = std::max(stages * slot, red) + 2048;
+    const int per_sm = std::max(1, std::min(2, static_cast<int>((228 * 1024) / smem)));
+    const int waves = ceil_div(tiles * S, nsm * per_sm);
+    const double cost = waves * (chunks + 0.1 * S);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best.S = S;
+      best.stages = stages;
+    }
+  }
+  return best;
+}
+
+StepPlan make_plan(const TensorPath* tp, int B, int P) {
+  const fr_config& c = tp->c;
+  StepPlan p;
+  p.B = B;
+  p.P = P;
+  p.T = B * c.H;
+  p.NT = ceil_div(p.T, NT_MAX);
+  p.Nt = static_cast<int>(align_up(ceil_div(p.T, p.NT), 16));
+  p.qkv = choose_plan(tp->qkv.MB * p.NT, tp->qkv.NKC, p.Nt, tp->nsm, tp->max_dyn);
+  p.o = choose_plan(tp->o.MB * p.NT, tp->o.NKC, p.Nt, tp->nsm, tp->max_dyn);
+  p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, tp->nsm, tp->max_dyn);
+  p.dn = choose_plan(tp->dn.MB * p.NT, tp->dn.NKC, p.Nt, tp->nsm, tp->max_dyn);
+  const int S = P + c.H;
+  int C = std::min(16, ceil_div(S, ATTN_SUBK));
+  p.attn_KC = static_cast<int>(align_up(ceil_div(S, C), ATTN_SUBK));
+  p.attn_C = ceil_div(S, p.attn_KC);
+  return p;
+}
+
+// Pre-tile rows of one projection: rowsrc(r) gives the float32 row r (length K) or nullptr (zero row).
+template <typename RowFn>
+void tile_projection(const ProjLayout& L, int elem, double scale, RowFn rowsrc, std::vector<uint8_t>& out) {
+  out.assign(L.bytes, 0);
+  const int Kb = L.NKC * KCB;   // padded row bytes
+  std::vector<uint8_t> row(Kb);
+  std::vector<float> zero_pad;
+  for (int r = 0; r < L.MB * BM; ++r) {
+    const float* src = rowsrc(r);
+    std::fill(row.begin(), row.end(), 0);
+    if (src) {
+      if (elem == 2) fr_round_bf16(src, reinterpret_cast<uint16_t*>(row.data()), L.K);
+      else fr_quantize_e4m3(src, row.data(), L.K, scale);
+    }
+    const int mb = r / BM, rr = r % BM;
+    for (int kc = 0; kc < L.NKC; ++kc) {
+      uint8_t* blk = out.data() + (static_cast<size_t>(mb) * L.NKC + kc) * BM * KCB;
+      for (int j = 0; j < KCB / 16; ++j)
+        std::memcpy(blk + j * BM * 16 + (rr / 8) * 128 + (rr % 8) * 16, row.data() + kc * KCB + j * 16, 16);
+    }
+  }
+}
+
+GemmArgs base_args(const TensorPath* tp, const StepPlan& p, const ProjLayout& L, const GemmPlan& g, int layer,
+                   size_t w_off) {
+  const fr_config& c = tp->c;
+  GemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.W = tp->w + layer * tp->layer_bytes + w_off;
+  a.MB = L.MB;
+  a.NKC = L.NKC;
+  a.Nout = L.rows;
+  a.S = g.S;
+  a.stages = g.stages;
+  a.fp8 = tp->fp8;
+  a.T = p.T;
+  a.Nt = p.Nt;
+  a.Kdim = L.K;
+  a.eps = c.eps;
+  a.T_pad = tp->T_pad;
+  a.status = tp->tb.status;
+  return a;
+}
+
+int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out, cudaStream_t s) {
+  const fr_config& c = tp->c;
+  const float dt = static_cast<float>(-1.0 / c.K);
+  const size_t o_off = tp->qkv.bytes, gu_off = o_off + tp->o.bytes, dn_off = gu_off + tp->gu.bytes;
+  cudaError_t e;
+  for (int k = 0; k < c.K; ++k) {
+    const float* x_in = (k == 0) ? x0 : tp->xs;
+    float* x_nx = (k == c.K - 1) ? x_out : tp->xs;
+    InprojArgs ia{};
+    ia.x = x_in;
+    ia.w_in = tp->tb.w_in;
+    ia.b_in = tp->tb.b_in;
+    ia.temb = tp->tb.temb + static_cast<size_t>(k) * c.D;
+    ia.h = tp->h;
+    ia.ssq = tp->ssq_a;
+    ia.T = p.T;
+    ia.D = c.D;
+    ia.A = c.A;
+    ia.T_pad = tp->T_pad;
+    ia.round_bf16 = 1;
+    ia.first = (k == 0);
+    if ((e = launch_inproj_tc(ia, s, true)) != cudaSuccess) return cuda_fail(e, "in-proj kernel launch");
+    for (int l = 0; l < c.L; ++l) {
+      const float* sa = tp->tb.s_a ? tp->tb.s_a + l * PI_COUNT : nullptr;
+      const float* al = tp->tb.alpha ? tp->tb.alpha + l * PI_COUNT : nullptr;
+      __nv_bfloat16* kvk = reinterpret_cast<__nv_bfloat16*>(tp->tb.kv_k + l * tp->tb.kv_layer_bytes);
+      __nv_bfloat16* kvv = reinterpret_cast<__nv_bfloat16*>(tp->tb.kv_v + l * tp->tb.kv_layer_bytes);
+      const float* g1 = tp->gains + static_cast<size_t>(l) * 2 * c.D;
+      const float* g2 = g1 + c.D;
+      // QKV: RMSNorm fused into the B staging, split + RoPE fused into the epilogue
+      GemmArgs q = base_args(tp, p, tp->qkv, p.qkv, l, 0);
+      q.b_kind = B_NORM;
+      q.h = tp->h;
+      q.gamma = g1;
+      q.ssq = tp->ssq_a;
+      q.ssq_parts = tp->MBd;
+      q.s_a = tp->fp8 ? sa + PI_QKV : nullptr;
+      q.alpha = tp->fp8 ? al + PI_QKV : nullptr;
+      q.epi = EPI_QKV;
+      q.q_out = tp->qbuf;
+      q.kv_k = kvk;
+      q.kv_v = kvv;
+      q.rope_cos = tp->tb.rope_cos;
+      q.rope_sin = tp->tb.rope_sin;
+      q.H = c.H;
+      q.P = p.P;
+      q.S_max = c.P_max + c.H;
+      q.Hq = c.Hq;
+      q.Hkv = c.Hkv;
+      q.dh = c.dh;
+      q.MB_rot = tp->MB_rot;
+      if ((e = launch_gemm_tc(q, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "qkv GEMM launch");
+      // attention over [prefix; actions]
+      AttnArgs at{};
+      at.q = tp->qbuf;
+      at.kv_k = kvk;
+      at.kv_v = kvv;
+      at.o = tp->obuf;
+      at.s_a = tp->fp8 ? sa + PI_O : nullptr;
+      at.fp8 = tp->fp8;
+      at.H = c.H;
+      at.P = p.P;
+      at.S_max = c.P_max + c.H;
+      at.Hq = c.Hq;
+      at.Hkv = c.Hkv;
+      at.dh = c.dh;
+      at.C = p.attn_C;
+      at.KC = p.attn_KC;
+      at.scale = 1.0f / std::sqrt(static_cast<float>(c.dh));
+      if ((e = launch_attention_tc(at, p.B, s, true)) != cudaSuccess) return cuda_fail(e, "attention launch");
+      // O projection + residual (+ sum of squares for the pre-MLP norm)
+      GemmArgs og = base_args(tp, p, tp->o, p.o, l, o_off);
+      og.b_kind = B_ROWS;
+      og.act = tp->obuf;
+      og.act_ld = c.Hq * c.dh;
+      og.alpha = tp->fp8 ? al + PI_O : nullptr;
+      og.epi = EPI_RESID;
+      og.h_out = tp->h;
+      og.ssq_out = tp->ssq_b;
+      og.D = c.D;
+      if ((e = launch_gemm_tc(og, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "o GEMM launch");
+      // gate|up with RMSNorm fused, GeLU(gate)*up epilogue
+      GemmArgs gg = base_args(tp, p, tp->gu, p.gu, l, gu_off);
+      gg.b_kind = B_NORM;
+      gg.h = tp->h;
+      gg.gamma = g2;
+      gg.ssq = tp->ssq_b;
+      gg.ssq_parts = tp->MBd;
+      gg.s_a = tp->fp8 ? sa + PI_GU : nullptr;
+      gg.alpha = tp->fp8 ? al + PI_GU : nullptr;
+      gg.epi = EPI_GELU;
+      gg.u_out = tp->ubuf;
+      gg.s_a_out = tp->fp8 ? sa + PI_DOWN : nullptr;
+      gg.F = c.F;
+      if ((e = launch_gemm_tc(gg, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "gate|up GEMM launch");
+      // down projection + residual (+ sum of squares for the next norm)
+      GemmArgs dg = base_args(tp, p, tp->dn, p.dn, l, dn_off);
+      dg.b_kind = B_ROWS;
+      dg.act = tp->ubuf;
+      dg.act_ld = c.F;
+      dg.alpha = tp->fp8 ? al + PI_DOWN : nullptr;
+      dg.epi = EPI_RESID;
+      dg.h_out = tp->h;
+      dg.ssq_out = tp->ssq_a;
+      dg.D = c.D;
+      if ((e = launch_gemm_tc(dg, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "down GEMM launch");
+    }
+    FinalArgs fa{};
+    fa.h = tp->h;
+    fa.ssq = tp->ssq_a;
+    fa.ssq_parts = tp->MBd;
+    fa.g_f = tp->tb.g_f;
+    fa.w_out = tp->tb.w_out;
+    fa.b_out = tp->tb.b_out;
+    fa.x_in = x_in;
+    fa.x_out = x_nx;
+    fa.T = p.T;
+    fa.D = c.D;
+    fa.A = c.A;
+    fa.T_pad = tp->T_pad;
+    fa.eps = c.eps;
+    fa.dt = dt;
+    fa.first = (k == 0);
+    fa.last = (k == c.K - 1);
+    if ((e = launch_final_tc(fa, s, true)) != cudaSuccess) return cuda_fail(e, "final kernel launch");
+  }
+  return FR_OK;
+}
+
+int build_graph(TensorPath* tp, int B, int P, const float* x0, float* x_out, GraphEntry& ge) {
+  ge.plan = make_plan(tp, B, P);
+  cudaGraph_t g = nullptr;
+  FR_CUDA(cudaStreamBeginCapture(tp->cap, cudaStreamCaptureModeThreadLocal));
+  int rc = record_call(tp, ge.plan, x0, x_out, tp->cap);
+  cudaError_t e = cudaStreamEndCapture(tp->cap, &g);
+  if (rc) {
+    if (g) cudaGraphDestroy(g);
+    return rc;
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamEndCapture");
+  size_t n = 0;
+  FR_CUDA(cudaGraphGetNodes(g, nullptr, &n));
+  std::vector<cudaGraphNode_t> nodes(n);
+  FR_CUDA(cudaGraphGetNodes(g, nodes.data(), &n));
+  e = cudaGraphInstantiate(&ge.exec, g, 0);
+  if (e != cudaSuccess) {
+    cudaGraphDestroy(g);
+    return cuda_fail(e, "cudaGraphInstantiate");
+  }
+  for (cudaGraphNode_t nd : nodes) {
+    cudaGraphNodeType t;
+    FR_CUDA(cudaGraphNodeGetType(nd, &t));
+    if (t != cudaGraphNodeTypeKernel) continue;
+    cudaKernelNodeParams kp;
+    FR_CUDA(cudaGraphKernelNodeGetParams(nd, &kp));
+    if (kp.func == inproj_kernel_ptr()) {
+      if (static_cast<InprojArgs*>(kp.kernelParams[0])->first) ge.x_in_nodes.push_back(nd);
+    } else if (kp.func == final_kernel_ptr()) {
+      const FinalArgs* fa = static_cast<FinalArgs*>(kp.kernelParams[0]);
+      if (fa->first || fa->last) {
+        if (fa->first) ge.x_in_nodes.push_back(nd);
+        if (fa->last) ge.x_out_nodes.push_back(nd);
+      }
+    }
+  }
+  cudaGraphDestroy(g);
+  ge.x0 = x0;
+  ge.x_out = x_out;
+  return FR_OK;
+}
+
+// Point the graph's caller-facing nodes at this call's x0 / x_out.
+int retarget(TensorPath* tp, GraphEntry& ge, const float* x0, float* x_out) {
+  (void)tp;
+  if (ge.x0 == x0 && ge.x_out == x_out) return FR_OK;
+  std::vector<cudaGraphNode_t> all = ge.x_in_nodes;
+  for (cudaGraphNode_t nd : ge.x_out_nodes)
+    if (std::find(all.begin(), all.end(), nd) == all.end()) all.push_back(nd);
+  for (cudaGraphNode_t nd : all) {
+    cudaKernelNodeParams kp;
+    FR_CUDA(cudaGraphKernelNodeGetParams(nd, &kp));
+    if (kp.func == inproj_kernel_ptr()) {
+      InprojArgs ia = *static_cast<InprojArgs*>(kp.kernelParams[0]);
+      ia.x = x0;
+      void* args[] = {&ia};
+      kp.kernelParams = args;
+      FR_CUDA(cudaGraphExecKernelNodeSetParams(ge.exec, nd, &kp));
+    } else {
+      FinalArgs fa = *static_cast<FinalArgs*>(kp.kernelParams[0]);
+      if (fa.first) fa.x_in = x0;
+      if (fa.last) fa.x_out = x_out;
+      void* args[] = {&fa};
+      kp.kernelParams = args;
+      FR_CUDA(cudaGraphExecKernelNodeSetParams(ge.exec, nd, &kp));
+    }
+  }
+  ge.x0 = x0;
+  ge.x_out = x_out;
+  return FR_OK;
+}
+
+}  // namespace
+
+bool tensor_path_supports(const fr_config& c) {
+  if (c.dtype != FR_DTYPE_BF16 && c.dtype != FR_DTYPE_FP8) return false;
+  if (c.dh != 64 && c.dh != 128 && c.dh != 256) return false;
+  if (((c.Hq + c.Hkv) * c.dh / 2) % 64 != 0) return false;   // RoPE pairs fill whole m-blocks
+  if ((c.Hkv * c.dh) % BM != 0) return false;                // V rows fill whole m-blocks
+  if (c.F % 64 != 0) return false;                            // gate/up pairs fill whole m-blocks
+  if (c.H > 128) return false;                                // one attention row-group pass per warp
+  if (c.D % 16 != 0 || (c.Hq * c.dh) % 16 != 0) return false; // 16-byte operand rows
+  const int S = c.P_max + c.H;
+  const int C = std::min(16, ceil_div(S, ATTN_SUBK));
+  const int KC = static_cast<int>(align_up(ceil_div(S, C), ATTN_SUBK));
+  if (attn_smem_bytes(c.H, c.dh, KC) > 200 * 1024) return false;
+  return true;
+}
+
+const char* tensor_path_limits() {
+  return "bf16/fp8, dh in {64,128,256}, (Hq+Hkv)*dh/2 % 64 == 0, Hkv*dh % 128 == 0, F % 64 == 0, H <= 128, "
+         "D % 16 == 0, attention chunk fits shared memory";
+}
+
+size_t tensor_path_bytes(const fr_config& c) {
+  TensorPath tmp;
+  init_sizes(&tmp, c);
+  return carve_all(&tmp, nullptr);
+}
+
+int tensor_path_create(const fr_config& c, const TensorPathBuffers& b, TensorPath** out) {
+  TensorPath* tp = new TensorPath();
+  init_sizes(tp, c);
+  tp->tb = b;
+  if (c.dtype != FR_DTYPE_FP8) {
+    tp->tb.alpha = nullptr;
+    tp->tb.s_a = nullptr;
+  }
+  if (carve_all(tp, b.base) > b.bytes) {
+    delete tp;
+    set_error("tensor path: buffer carve exceeds its allocation");
+    return FR_ERR_CUDA;
+  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&tp->nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = tc_kernels_init();
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&tp->cap, cudaStreamNonBlocking);
+  if (e != cudaSuccess) {
+    delete tp;
+    return cuda_fail(e, "tensor path init");
+  }
+  tp->max_dyn = max_dynamic_smem();
+  tp->gains_host.assign(static_cast<size_t>(c.L) * 2 * c.D, 1.f);
+  *out = tp;
+  return FR_OK;
+}
+
+int tensor_path_pack_layer(TensorPath* tp, int l, const fr_layer_weights& w, const double sw[4]) {
+  const fr_config& c = tp->c;
+  const int D = c.D, dh = c.dh, half = dh / 2, F = c.F;
+  const int nq = c.Hq * dh, nk = c.Hkv * dh;
+  std::vector<uint8_t> buf;
+  uint8_t* dst = tp->w + l * tp->layer_bytes;
+  // QKV rows: m-blocks of 64 rotate-half pairs (lo rows 0-63, hi rows 64-127), then V rows
+  auto qkv_row = [&](int r) -> const float* {
+    const int mb = r / BM, rr = r % BM;
+    int cr;
+    if (mb < tp->MB_rot) {
+      const int pi = mb * 64 + (rr & 63);
+      const int head = pi / half, j = pi % half;
+      cr = head * dh + j + (rr >= 64 ? half : 0);
+    } else {
+      cr = nq + nk + (mb - tp->MB_rot) * BM + rr;
+      if (cr >= nq + 2 * nk) return nullptr;
+    }
+    if (cr < nq) return w.wq + static_cast<size_t>(cr) * D;
+    if (cr < nq + nk) return w.wk + static_cast<size_t>(cr - nq) * D;
+    return w.wv + static_cast<size_t>(cr - nq - nk) * D;
+  };
+  tile_projection(tp->qkv, tp->elem, sw[PI_QKV], qkv_row, buf);
+  FR_CUDA(cudaMemcpy(dst, buf.data(), buf.size(), cudaMemcpyHostToDevice));
+  dst += tp->qkv.bytes;
+  auto o_row = [&](int r) -> const float* { return r < D ? w.wo + static_cast<size_t>(r) * nq : nullptr; };
+  tile_projection(tp->o, tp->elem, sw[PI_O], o_row, buf);
+  FR_CUDA(cudaMemcpy(dst, buf.data(), buf.size(), cudaMemcpyHostToDevice));
+  dst += tp->o.bytes;
+  // gate|up rows: m-block mb holds gate features mb*64..+63 (rows 0-63) and the same up features (64-127)
+  auto gu_row = [&](int r) -> const float* {
+    const int mb = r / BM, rr = r % BM;
+    const int f = mb * 64 + (rr & 63);
+    if (f >= F) return nullptr;
+    return (rr < 64 ? w.wg : w.wu) + static_cast<size_t>(f) * D;
+  };
+  tile_projection(tp->gu, tp->elem, sw[PI_GU], gu_row, buf);
+  FR_CUDA(cudaMemcpy(dst, buf.data(), buf.size(), cudaMemcpyHostToDevice));
+  dst += tp->gu.bytes;
+  auto d_row = [&](int r) -> const float* { return r < D ? w.wd + static_cast<size_t>(r) * F : nullptr; };
+  tile_projection(tp->dn, tp->elem, sw[PI_DOWN], d_row, buf);
+  FR_CUDA(cudaMemcpy(dst, buf.data(), buf.size(), cudaMemcpyHostToDevice));
+  std::memcpy(&tp->gains_host[static_cast<size_t>(l) * 2 * D], w.g1, D * sizeof(float));
+  std::memcpy(&tp->gains_host[static_cast<size_t>(l) * 2 * D + D], w.g2, D * sizeof(float));
+  return FR_OK;
+}
+
+int tensor_path_finish_load(TensorPath* tp, cudaStream_t) {
+  FR_CUDA(cudaMemcpy(tp->gains, tp->gains_host.data(), tp->gains_host.size() * 4, cudaMemcpyHostToDevice));
+  return FR_OK;
+}
+
+int tensor_path_set_scales(TensorPath*, const float*, const float*) {
+  return FR_OK;   // kernels read the handle's device scale arrays directly
+}
+
+int tensor_path_denoise(TensorPath* tp, const float* x0, float* x_out, int B, int P, cudaStream_t s) {
+  auto key = std::make_pair(B, P);
+  auto it = tp->graphs.find(key);
+  if (it == tp->graphs.end()) {
+    GraphEntry ge;
+    int rc = build_graph(tp, B, P, x0, x_out, ge);
+    if (rc) return rc;
+    it = tp->graphs.emplace(key, ge).first;
+  }
+  int rc = retarget(tp, it->second, x0, x_out);
+  if (rc) return rc;
+  FR_CUDA(cudaGraphLaunch(it->second.exec, s));
+  return FR_OK;
+}
+
+int tensor_path_launches(const TensorPath* tp, int) { return tp->c.K * (2 + 5 * tp->c.L); }
+
+void tensor_path_destroy(TensorPath* tp) {
+  if (!tp) return;
+  for (auto& kv : tp->graphs)
+    if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
+  if (tp->cap) cudaStreamDestroy(tp->cap);
+  delete tp;
+}
 
 }  // namespace fr
