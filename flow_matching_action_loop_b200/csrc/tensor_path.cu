@@ -53,10 +53,18 @@ struct StepPlan {
   int attn_C = 1, attn_KC = 64;
 };
 
+struct RetargetNode {
+  cudaGraphNode_t node = nullptr;   // node of the captured graph (kept alive with the exec)
+  cudaKernelNodeParams kp{};
+  bool is_inproj = false;
+  InprojArgs ia{};
+  FinalArgs fa{};
+};
+
 struct GraphEntry {
+  cudaGraph_t graph = nullptr;      // owns the node handles used to retarget the exec
   cudaGraphExec_t exec = nullptr;
-  std::vector<cudaGraphNode_t> x_in_nodes;   // nodes whose x input is the caller's x0
-  std::vector<cudaGraphNode_t> x_out_nodes;  // nodes whose output is the caller's x_out
+  std::vector<RetargetNode> nodes;  // kernels reading the caller's x0 or writing the caller's x_out
   const float* x0 = nullptr;
   float* x_out = nullptr;
   StepPlan plan;
@@ -361,61 +369,57 @@ int build_graph(TensorPath* tp, int B, int P, const float* x0, float* x_out, Gra
     return rc;
   }
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamEndCapture");
+  ge.graph = g;
   size_t n = 0;
   FR_CUDA(cudaGraphGetNodes(g, nullptr, &n));
   std::vector<cudaGraphNode_t> nodes(n);
   FR_CUDA(cudaGraphGetNodes(g, nodes.data(), &n));
   e = cudaGraphInstantiate(&ge.exec, g, 0);
-  if (e != cudaSuccess) {
-    cudaGraphDestroy(g);
-    return cuda_fail(e, "cudaGraphInstantiate");
-  }
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGraphInstantiate");
   for (cudaGraphNode_t nd : nodes) {
     cudaGraphNodeType t;
     FR_CUDA(cudaGraphNodeGetType(nd, &t));
     if (t != cudaGraphNodeTypeKernel) continue;
     cudaKernelNodeParams kp;
     FR_CUDA(cudaGraphKernelNodeGetParams(nd, &kp));
+    RetargetNode rn;
+    rn.node = nd;
+    rn.kp = kp;
     if (kp.func == inproj_kernel_ptr()) {
-      if (static_cast<InprojArgs*>(kp.kernelParams[0])->first) ge.x_in_nodes.push_back(nd);
+      rn.ia = *static_cast<InprojArgs*>(kp.kernelParams[0]);
+      if (!rn.ia.first) continue;
+      rn.is_inproj = true;
     } else if (kp.func == final_kernel_ptr()) {
-      const FinalArgs* fa = static_cast<FinalArgs*>(kp.kernelParams[0]);
-      if (fa->first || fa->last) {
-        if (fa->first) ge.x_in_nodes.push_back(nd);
-        if (fa->last) ge.x_out_nodes.push_back(nd);
-      }
+      rn.fa = *static_cast<FinalArgs*>(kp.kernelParams[0]);
+      if (!rn.fa.first && !rn.fa.last) continue;
+    } else {
+      continue;
     }
+    rn.kp.kernelParams = nullptr;
+    rn.kp.extra = nullptr;
+    ge.nodes.push_back(rn);
   }
-  cudaGraphDestroy(g);
   ge.x0 = x0;
   ge.x_out = x_out;
   return FR_OK;
 }
 
 // Point the graph's caller-facing nodes at this call's x0 / x_out.
-int retarget(TensorPath* tp, GraphEntry& ge, const float* x0, float* x_out) {
-  (void)tp;
+int retarget(GraphEntry& ge, const float* x0, float* x_out) {
   if (ge.x0 == x0 && ge.x_out == x_out) return FR_OK;
-  std::vector<cudaGraphNode_t> all = ge.x_in_nodes;
-  for (cudaGraphNode_t nd : ge.x_out_nodes)
-    if (std::find(all.begin(), all.end(), nd) == all.end()) all.push_back(nd);
-  for (cudaGraphNode_t nd : all) {
-    cudaKernelNodeParams kp;
-    FR_CUDA(cudaGraphKernelNodeGetParams(nd, &kp));
-    if (kp.func == inproj_kernel_ptr()) {
-      InprojArgs ia = *static_cast<InprojArgs*>(kp.kernelParams[0]);
-      ia.x = x0;
-      void* args[] = {&ia};
-      kp.kernelParams = args;
-      FR_CUDA(cudaGraphExecKernelNodeSetParams(ge.exec, nd, &kp));
+  for (RetargetNode& rn : ge.nodes) {
+    cudaKernelNodeParams kp = rn.kp;
+    void* args[1];
+    if (rn.is_inproj) {
+      rn.ia.x = x0;
+      args[0] = &rn.ia;
     } else {
-      FinalArgs fa = *static_cast<FinalArgs*>(kp.kernelParams[0]);
-      if (fa.first) fa.x_in = x0;
-      if (fa.last) fa.x_out = x_out;
-      void* args[] = {&fa};
-      kp.kernelParams = args;
-      FR_CUDA(cudaGraphExecKernelNodeSetParams(ge.exec, nd, &kp));
+      if (rn.fa.first) rn.fa.x_in = x0;
+      if (rn.fa.last) rn.fa.x_out = x_out;
+      args[0] = &rn.fa;
     }
+    kp.kernelParams = args;
+    FR_CUDA(cudaGraphExecKernelNodeSetParams(ge.exec, rn.node, &kp));
   }
   ge.x0 = x0;
   ge.x_out = x_out;
@@ -540,10 +544,14 @@ int tensor_path_denoise(TensorPath* tp, const float* x0, float* x_out, int B, in
   if (it == tp->graphs.end()) {
     GraphEntry ge;
     int rc = build_graph(tp, B, P, x0, x_out, ge);
-    if (rc) return rc;
+    if (rc) {
+      if (ge.exec) cudaGraphExecDestroy(ge.exec);
+      if (ge.graph) cudaGraphDestroy(ge.graph);
+      return rc;
+    }
     it = tp->graphs.emplace(key, ge).first;
   }
-  int rc = retarget(tp, it->second, x0, x_out);
+  int rc = retarget(it->second, x0, x_out);
   if (rc) return rc;
   FR_CUDA(cudaGraphLaunch(it->second.exec, s));
   return FR_OK;
@@ -553,8 +561,10 @@ int tensor_path_launches(const TensorPath* tp, int) { return tp->c.K * (2 + 5 * 
 
 void tensor_path_destroy(TensorPath* tp) {
   if (!tp) return;
-  for (auto& kv : tp->graphs)
+  for (auto& kv : tp->graphs) {
     if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
+    if (kv.second.graph) cudaGraphDestroy(kv.second.graph);
+  }
   if (tp->cap) cudaStreamDestroy(tp->cap);
   delete tp;
 }
