@@ -1,24 +1,24 @@
 // Tensor-core kernels of the action-expert loop (sm_100a).
 //
-// GEMM (swap-AB): D[128 features x Nt tokens] = W_tile[128 x K] * act[Nt x K]^T
-//   on tcgen05 with the accumulator in tensor memory.  Weights are the A operand,
-//   pre-tiled by the packer so that each pipeline chunk (128 rows x 128 bytes of K)
-//   is one contiguous 16 KB block moved by a single bulk copy.  The B operand
-//   (activations) is staged by warps 2-7: RMSNorm (+ bf16/e4m3 quantisation) is
-//   fused into this staging for the QKV and gate|up projections (FlashRT
+// GEMM (swap-AB): D[128 features x Nt tokens] = W_tile[128 x K] * act[Nt x K]^T on tcgen05
+//   with the accumulator in tensor memory.  Both operands arrive by bulk copy (TMA
+//   engine): the weight chunks (pre-tiled by the packer, one 16 KB block per chunk) are
+//   issued before the kernel waits on its predecessor; the activation chunks after it.
+//   For the QKV and gate|up projections the activation is the raw fp32 residual h and
+//   warps 2-7 turn it into RMSNorm(h)*gamma (bf16 or e4m3) in shared memory (FlashRT
 //   walkthrough, component 8: norm and residual+norm+quant fusion).  Split-K is a
-//   thread-block cluster: partial tiles are summed over distributed shared memory
-//   in rank order, then a fused epilogue runs:
+//   thread-block cluster: each CTA pushes the token slices of its partial tile to their
+//   owners with bulk shared-to-shared copies, and each owner sums its slices in rank
+//   order (deterministic).  Fused epilogues:
 //     EPI_QKV   QKV split + rotate-half RoPE, q to its buffer, k/v into the KV cache
 //     EPI_RESID residual add into h and the per-token sum of squares of the new h
-//     EPI_GELU  GeLU(tanh)(gate) * up, quantised for the down projection
+//     EPI_GELU  GeLU(tanh)(gate) * up, quantised, written as the down projection's operand
 //   (PhyAI page, optimisation paragraph: fused QKV and merged gate|up GEMMs.)
 //
-// Attention: one cluster per (sample, query head), one CTA per key chunk.  Warp-level
-//   bf16 MMA computes scores and P*V with an online softmax over 64-key sub-chunks;
-//   the key chunks are merged with their log-sum-exp weights over distributed shared
-//   memory in rank order (flash-decoding split over keys).
-#include <cooperative_groups.h>
+// Attention: one cluster per (sample, query head), one CTA per key chunk (flash-decoding
+//   split over keys).  Warp-level bf16 MMA computes scores and P*V with an online softmax
+//   over 64-key sub-chunks; the chunks' (O, max, sum) rows are pushed to their owner CTA by
+//   bulk copies and merged with log-sum-exp weights in rank order.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <math.h>
@@ -27,15 +27,14 @@
 #include "sm100.h"
 #include "tc_kernels.h"
 
-namespace cg = cooperative_groups;
-
 namespace fr {
 namespace tc {
 namespace {
 
 using namespace fr::sm100;
 
-constexpr int RED_LD = BM + 4;   // row stride (floats) of the epilogue reduction buffer
+constexpr int CONV_THREADS = 192;                                  // warps 2-7
+constexpr int CONV_ITEMS = (NT_MAX * 8 + CONV_THREADS - 1) / CONV_THREADS;
 
 __device__ __forceinline__ void report_timeout(unsigned* status, uint32_t where) {
   if (status) {
@@ -59,43 +58,73 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  return static_cast<uint32_t>(to_e4m3(a)) | (static_cast<uint32_t>(to_e4m3(b)) << 8) |
+         (static_cast<uint32_t>(to_e4m3(c)) << 16) | (static_cast<uint32_t>(to_e4m3(d)) << 24);
+}
+
+__device__ __forceinline__ void conv_sync() { asm volatile("bar.sync 1, 192;" ::: "memory"); }
+
 // ================================================================== GEMM
 
 struct GemmSmem {
   uint64_t full_a[MAX_STAGES];
   uint64_t full_b[MAX_STAGES];
+  uint64_t raw_b[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
   uint64_t done;
+  uint64_t recv_bar;
   uint32_t tmem_base;
-  int abort_flag;
   float rstd[NT_MAX];
   float ssq_part[2][4];
 };
+
+struct GemmGeom {
+  uint32_t a_bytes, breg, slot, raw_bytes, ring, gamma_off, recv_off;
+  int TS;
+};
+
+__host__ __device__ __forceinline__ GemmGeom gemm_geom(int Nt, int stages, int b_kind, int fp8, int S, int nk) {
+  GemmGeom g;
+  g.a_bytes = BM * KCB;
+  g.raw_bytes = (b_kind == B_NORM) ? static_cast<uint32_t>(Nt) * 256u * (fp8 ? 2u : 1u) : 0u;
+  const uint32_t tile = static_cast<uint32_t>(Nt) * KCB;
+  g.breg = tile > g.raw_bytes ? tile : g.raw_bytes;
+  g.slot = g.a_bytes + g.breg;
+  g.ring = g.slot * static_cast<uint32_t>(stages);
+  g.gamma_off = g.ring;   // B_NORM: gamma of this CTA's k-range (nk * kel floats)
+  g.TS = (Nt + S - 1) / S;
+  g.recv_off = ((static_cast<uint32_t>(Nt) * RED_LD * 4u) + 1023u) & ~1023u;
+  return g;
+}
 
 __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_constant__ GemmArgs a) {
   extern __shared__ __align__(1024) uint8_t dsm[];
   __shared__ GemmSmem sh;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int ks = blockIdx.x;            // split-K rank (cluster rank)
+  const int ks = blockIdx.x;            // split-K rank (= cluster rank)
   const int mb = blockIdx.y;            // m-block
   const int nt = blockIdx.z;            // n-tile
   const int Nt = a.Nt;
-  const int n0 = nt * Nt;               // first token of this tile
-  const int kc0 = ks * a.NKC / a.S, kc1 = (ks + 1) * a.NKC / a.S;
+  const int n0 = nt * Nt;
+  const int S = a.S;
+  const int kc0 = ks * a.NKC / S, kc1 = (ks + 1) * a.NKC / S;
   const int nk = kc1 - kc0;
   const int stages = a.stages;
-  const uint32_t A_BYTES = BM * KCB;
-  const uint32_t B_BYTES = static_cast<uint32_t>(Nt) * KCB;
-  const uint32_t SLOT = A_BYTES + B_BYTES;
+  const int norm = a.b_kind == B_NORM;
+  const int kel = a.fp8 ? KCB : KCB / 2;            // K elements per chunk
+  const GemmGeom gm = gemm_geom(Nt, stages, a.b_kind, a.fp8, S, nk);
+  float* gsm = reinterpret_cast<float*>(dsm + gm.gamma_off);
 
   if (tid == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&sh.full_a[s], 1);
-      mbar_init(&sh.full_b[s], 192);
+      mbar_init(&sh.full_b[s], norm ? CONV_THREADS : 1);
+      mbar_init(&sh.raw_b[s], 1);
       mbar_init(&sh.empty[s], 1);
     }
     mbar_init(&sh.done, 1);
-    sh.abort_flag = 0;
+    mbar_init(&sh.recv_bar, 1);
     fence_mbar_init();
   }
   uint32_t ncols = 32;
@@ -107,28 +136,52 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  grid_dep_launch();   // the next kernel may start its own weight prefetch now
+  grid_dep_launch();   // the next kernel may start its own prefetch now
   const uint32_t tacc = sh.tmem_base;
 
   if (warp == 0) {
-    // ---------------- A producer: weight chunks by bulk copy (independent of the previous kernel)
+    // ---------------- bulk-copy producer
     if (lane == 0) {
-      const uint8_t* wsrc = a.W + (static_cast<size_t>(mb) * a.NKC + kc0) * A_BYTES;
-      int issued = 0;
-      for (int i = 0; i < nk; ++i) {
+      const uint8_t* wsrc = a.W + (static_cast<size_t>(mb) * a.NKC + kc0) * gm.a_bytes;
+      auto issue_b = [&](int i) {
         const int s = i % stages;
-        if (i >= stages && !mbar_wait(&sh.empty[s], ((i / stages) - 1) & 1, WAIT_LIMIT_NS)) {
+        uint8_t* bdst = dsm + s * gm.slot + gm.a_bytes;
+        if (norm) {
+          const int kb = (kc0 + i) * (a.fp8 ? 2 : 1);
+          mbar_arrive_expect_tx(&sh.raw_b[s], gm.raw_bytes);
+          bulk_g2s(bdst, a.h + (static_cast<size_t>(nt) * a.KB + kb) * Nt * 64, gm.raw_bytes, &sh.raw_b[s]);
+        } else {
+          const uint32_t tb = static_cast<uint32_t>(Nt) * KCB;
+          mbar_arrive_expect_tx(&sh.full_b[s], tb);
+          bulk_g2s(bdst, a.act + (static_cast<size_t>(nt) * a.NKC + kc0 + i) * tb, tb, &sh.full_b[s]);
+        }
+      };
+      const int pre = nk < stages ? nk : stages;
+      for (int i = 0; i < pre; ++i) {   // weights first: they do not depend on the previous kernel
+        mbar_arrive_expect_tx(&sh.full_a[i], gm.a_bytes);
+        bulk_g2s(dsm + i * gm.slot, wsrc + static_cast<size_t>(i) * gm.a_bytes, gm.a_bytes, &sh.full_a[i]);
+      }
+      grid_dep_wait();
+      for (int i = 0; i < pre; ++i) issue_b(i);
+      int issued = pre;
+      for (int i = pre; i < nk; ++i) {
+        const int s = i % stages;
+        if (!mbar_wait(&sh.empty[s], ((i / stages) - 1) & 1, WAIT_LIMIT_NS)) {
           report_timeout(a.status, 0x100);
-          sh.abort_flag = 1;
           break;
         }
-        mbar_arrive_expect_tx(&sh.full_a[s], A_BYTES);
-        bulk_g2s(dsm + s * SLOT, wsrc + static_cast<size_t>(i) * A_BYTES, A_BYTES, &sh.full_a[s]);
+        mbar_arrive_expect_tx(&sh.full_a[s], gm.a_bytes);
+        bulk_g2s(dsm + s * gm.slot, wsrc + static_cast<size_t>(i) * gm.a_bytes, gm.a_bytes, &sh.full_a[s]);
+        issue_b(i);
         issued = i + 1;
       }
-      // drain: every copy issued into this CTA's shared memory has landed before it is reused
-      for (int i = (issued > stages ? issued - stages : 0); i < issued; ++i)
-        mbar_wait(&sh.full_a[i % stages], (i / stages) & 1, WAIT_LIMIT_NS);
+      // drain: the copies issued into this CTA's shared memory have landed before it is reused
+      for (int i = (issued > stages ? issued - stages : 0); i < issued; ++i) {
+        const int s = i % stages;
+        const uint32_t par = (i / stages) & 1;
+        mbar_wait(&sh.full_a[s], par, WAIT_LIMIT_NS);
+        mbar_wait(norm ? &sh.raw_b[s] : &sh.full_b[s], par, WAIT_LIMIT_NS);
+      }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
@@ -139,11 +192,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         const uint32_t par = (i / stages) & 1;
         if (!mbar_wait(&sh.full_a[s], par, WAIT_LIMIT_NS) || !mbar_wait(&sh.full_b[s], par, WAIT_LIMIT_NS)) {
           report_timeout(a.status, 0x200);
-          sh.abort_flag = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t a0 = smem_u32(dsm + s * SLOT), b0 = a0 + A_BYTES;
+        const uint32_t a0 = smem_u32(dsm + s * gm.slot), b0 = a0 + gm.a_bytes;
 #pragma unroll
         for (int k = 0; k < KCB / 32; ++k) {
           const uint64_t ad = smem_desc(a0 + k * 2 * BM * 16, BM * 16, 128);
@@ -155,68 +207,81 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       }
       mma_commit(&sh.done);
     }
-  } else {
-    // ---------------- B staging (warps 2-7): activations of this n-tile into the ring
-    grid_dep_wait();
-    const int st = tid - 64;   // 0..191
-    if (a.b_kind == B_NORM) {
-      for (int r = st; r < Nt; r += 192) {
-        const int t = n0 + r;
-        float ss = 0.f;
-        if (t < a.T)
-          for (int p = 0; p < a.ssq_parts; ++p) ss += a.ssq[p * a.T_pad + t];
-        sh.rstd[r] = 1.0f / sqrtf(ss / a.Kdim + a.eps);
-      }
-      asm volatile("bar.sync 1, 192;" ::: "memory");
+  } else if (norm) {
+    // ---------------- B conversion (warps 2-7): RMSNorm(h)*gamma -> bf16 / e4m3 operand tile
+    const int st = tid - 64;
+    for (int idx = st; idx < nk * kel; idx += CONV_THREADS) {   // static: before the dependency wait
+      const int k = kc0 * kel + idx;
+      gsm[idx] = k < a.D ? a.gamma[k] : 0.f;                      // padded K: zero
     }
-    const float inv_sa = (a.fp8 && a.b_kind == B_NORM) ? 1.0f / *a.s_a : 1.0f;
-    const int elem = a.fp8 ? 1 : 2;
-    const int kel = KCB / elem;                 // K elements per chunk
+    grid_dep_wait();
+    for (int r = st; r < Nt; r += CONV_THREADS) {
+      const int t = n0 + r;
+      float rs = 0.f;
+      if (t < a.T) {
+        const float4* sp = reinterpret_cast<const float4*>(a.ssq + static_cast<size_t>(t) * a.ssq_ld);
+        float4 v[4];
+        const int nv = a.ssq_ld >> 2;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (q < nv) v[q] = sp[q];
+        float ss = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (q < nv) ss += ((v[q].x + v[q].y) + v[q].z) + v[q].w;
+        rs = 1.0f / sqrtf(ss / a.D + a.eps);
+      }
+      sh.rstd[r] = rs;   // padded tokens become zero
+    }
+    conv_sync();
+    const float inv_sa = a.fp8 ? 1.0f / *a.s_a : 1.0f;
     for (int i = 0; i < nk; ++i) {
       const int s = i % stages;
-      if (i >= stages && !mbar_wait(&sh.empty[s], ((i / stages) - 1) & 1, WAIT_LIMIT_NS)) {
+      if (!mbar_wait(&sh.raw_b[s], (i / stages) & 1, WAIT_LIMIT_NS)) {
         report_timeout(a.status, 0x300);
-        sh.abort_flag = 1;
         break;
       }
-      uint8_t* bdst = dsm + s * SLOT + A_BYTES;
-      const int k0 = (kc0 + i) * kel;
-      // item = one 16-byte row segment (slab j of token row r)
-      for (int it = st; it < Nt * 8; it += 192) {
-        const int r = it >> 3, j = it & 7;
-        const int t = n0 + r;
-        const int kk = k0 + j * (16 / elem);
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (t < a.T && kk < a.Kdim) {
-          if (a.b_kind == B_ROWS) {
-            val = *reinterpret_cast<const uint4*>(a.act + (static_cast<size_t>(t) * a.act_ld + kk) * elem);
-          } else {
-            const float* hp = a.h + static_cast<size_t>(t) * a.Kdim + kk;
-            const float* gp = a.gamma + kk;
-            const float rs = sh.rstd[r];
-            if (!a.fp8) {
-              const float4 h0 = *reinterpret_cast<const float4*>(hp), h1 = *reinterpret_cast<const float4*>(hp + 4);
-              const float4 g0 = *reinterpret_cast<const float4*>(gp), g1 = *reinterpret_cast<const float4*>(gp + 4);
-              val.x = pack_bf16x2(h0.x * rs * g0.x, h0.y * rs * g0.y);
-              val.y = pack_bf16x2(h0.z * rs * g0.z, h0.w * rs * g0.w);
-              val.z = pack_bf16x2(h1.x * rs * g1.x, h1.y * rs * g1.y);
-              val.w = pack_bf16x2(h1.z * rs * g1.z, h1.w * rs * g1.w);
-            } else {
-              uint32_t wds[4];
+      uint8_t* breg = dsm + s * gm.slot + gm.a_bytes;
+      const float* raw = reinterpret_cast<const float*>(breg);
+      const float* gch = gsm + i * kel;
+      uint4 res[CONV_ITEMS];
 #pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4) {
-                const float4 hv = *reinterpret_cast<const float4*>(hp + 4 * q4);
-                const float4 gv = *reinterpret_cast<const float4*>(gp + 4 * q4);
-                wds[q4] = static_cast<uint32_t>(to_e4m3(hv.x * rs * gv.x * inv_sa)) |
-                          (static_cast<uint32_t>(to_e4m3(hv.y * rs * gv.y * inv_sa)) << 8) |
-                          (static_cast<uint32_t>(to_e4m3(hv.z * rs * gv.z * inv_sa)) << 16) |
-                          (static_cast<uint32_t>(to_e4m3(hv.w * rs * gv.w * inv_sa)) << 24);
-              }
-              val = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+      for (int q = 0; q < CONV_ITEMS; ++q) {
+        const int it = st + q * CONV_THREADS;
+        if (it < Nt * 8) {
+          const int r = it >> 3, j = it & 7;
+          const float rs = sh.rstd[r];
+          if (!a.fp8) {
+            const float* p = raw + static_cast<size_t>(r) * 64 + j * 8;
+            const float4 h0 = *reinterpret_cast<const float4*>(p), h1 = *reinterpret_cast<const float4*>(p + 4);
+            const float4 g0 = *reinterpret_cast<const float4*>(gch + j * 8);
+            const float4 g1 = *reinterpret_cast<const float4*>(gch + j * 8 + 4);
+            res[q] = make_uint4(pack_bf16x2(h0.x * rs * g0.x, h0.y * rs * g0.y),
+                                pack_bf16x2(h0.z * rs * g0.z, h0.w * rs * g0.w),
+                                pack_bf16x2(h1.x * rs * g1.x, h1.y * rs * g1.y),
+                                pack_bf16x2(h1.z * rs * g1.z, h1.w * rs * g1.w));
+          } else {
+            const float* p = raw + (static_cast<size_t>(j >> 2) * Nt + r) * 64 + (j & 3) * 16;
+            uint32_t w4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float4 hv = *reinterpret_cast<const float4*>(p + 4 * u);
+              const float4 gv = *reinterpret_cast<const float4*>(gch + j * 16 + 4 * u);
+              const float m = rs * inv_sa;
+              w4[u] = pack_e4m3x4(hv.x * gv.x * m, hv.y * gv.y * m, hv.z * gv.z * m, hv.w * gv.w * m);
             }
+            res[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
-        *reinterpret_cast<uint4*>(bdst + j * Nt * 16 + (r >> 3) * 128 + (r & 7) * 16) = val;
+      }
+      conv_sync();   // every raw value of this slot has been read before the tile overwrites it
+#pragma unroll
+      for (int q = 0; q < CONV_ITEMS; ++q) {
+        const int it = st + q * CONV_THREADS;
+        if (it < Nt * 8) {
+          const int r = it >> 3, j = it & 7;
+          *reinterpret_cast<uint4*>(breg + j * Nt * 16 + (r >> 3) * 128 + (r & 7) * 16) = res[q];
+        }
       }
       fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core (async proxy)
       mbar_arrive(&sh.full_b[s]);
@@ -225,13 +290,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
 
   // ---------------- epilogue
   grid_dep_wait();
-  if (!mbar_wait(&sh.done, 0, WAIT_LIMIT_NS)) {
-    report_timeout(a.status, 0x400);
-    sh.abort_flag = 1;
-  }
+  if (!mbar_wait(&sh.done, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0x400);
   tc_fence_after();
   __syncthreads();
-  float* red = reinterpret_cast<float*>(dsm);          // [Nt][RED_LD], aliases the drained ring
+  float* red = reinterpret_cast<float*>(dsm);   // [Nt][RED_LD], aliases the drained ring
   if (warp >= 4) {
     const int q = warp & 3;
     const int row = q * 32 + lane;
@@ -243,18 +305,35 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
     }
   }
   tc_fence_before();
-  __syncthreads();
-  cg::cluster_group cluster = cg::this_cluster();
-  if (a.S > 1) cluster.sync();
+  const int tok0 = ks * Nt / S, tok1 = (ks + 1) * Nt / S;
+  float* recv = reinterpret_cast<float*>(dsm + gm.recv_off);   // [S][TS][RED_LD]
+  if (S > 1) {
+    if (tid == 0) mbar_arrive_expect_tx(&sh.recv_bar, static_cast<uint32_t>(S * (tok1 - tok0) * RED_LD * 4));
+    fence_proxy_async_smem();
+    __syncthreads();
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    if (tid == 0) {
+      for (int d = 0; d < S; ++d) {
+        const int d0 = d * Nt / S, d1 = (d + 1) * Nt / S;
+        const uint32_t dst = mapa_shared(recv + static_cast<size_t>(ks) * gm.TS * RED_LD, d);
+        bulk_s2cluster(dst, red + static_cast<size_t>(d0) * RED_LD, static_cast<uint32_t>((d1 - d0) * RED_LD * 4),
+                       mapa_shared(&sh.recv_bar, d));
+      }
+      bulk_commit();
+    }
+    if (!mbar_wait(&sh.recv_bar, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0x500);
+  } else {
+    __syncthreads();
+  }
 
   const float al = a.alpha ? *a.alpha : 1.0f;
-  const int tok0 = ks * Nt / a.S, tok1 = (ks + 1) * Nt / a.S;
   // split-K sum of one accumulator element over the cluster, in rank order (deterministic)
-  auto gather = [&](int tok, int row) -> float {
-    const int idx = tok * RED_LD + row;
-    if (a.S == 1) return red[idx] * al;
+  auto val = [&](int tok, int row) -> float {
+    if (S == 1) return red[tok * RED_LD + row] * al;
     float v = 0.f;
-    for (int s = 0; s < a.S; ++s) v += cluster.map_shared_rank(red, s)[idx];
+    const float* p = recv + static_cast<size_t>(tok - tok0) * RED_LD + row;
+    for (int s = 0; s < S; ++s) v += p[static_cast<size_t>(s) * gm.TS * RED_LD];
     return v * al;
   };
 
@@ -266,17 +345,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       const int t = n0 + tok;
       float sq = 0.f;
       if (tok < tok1 && t < a.T && f < a.Nout) {
-        float* hp = a.h_out + static_cast<size_t>(t) * a.D + f;
-        const float hv = *hp + gather(tok, row);
+        float* hp = a.h_out + htile_offset(t, f, Nt, a.KB);
+        const float hv = *hp + val(tok, row);
         *hp = hv;
         sq = hv * hv;
       }
       for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
       if (lane == 0) sh.ssq_part[sub][(tid >> 5) & 3] = sq;
       __syncthreads();
-      if (row == 0 && tok < tok1 && t < a.T_pad)
-        a.ssq_out[mb * a.T_pad + t] = ((sh.ssq_part[sub][0] + sh.ssq_part[sub][1]) + sh.ssq_part[sub][2]) +
-                                      sh.ssq_part[sub][3];
+      if (row == 0 && tok < tok1 && t < a.T)
+        a.ssq_out[static_cast<size_t>(t) * a.ssq_ld + mb] =
+            ((sh.ssq_part[sub][0] + sh.ssq_part[sub][1]) + sh.ssq_part[sub][2]) + sh.ssq_part[sub][3];
       __syncthreads();
     }
   } else if (a.epi == EPI_GELU) {
@@ -286,9 +365,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
     for (int tok = tok0 + sub; tok < tok1; tok += 4) {
       const int t = n0 + tok;
       if (t >= a.T || f >= a.F) continue;
-      const float u = gelu_tanh(gather(tok, p)) * gather(tok, p + 64);
-      if (a.fp8) a.u_out[static_cast<size_t>(t) * a.F + f] = to_e4m3(u * inv);
-      else reinterpret_cast<__nv_bfloat16*>(a.u_out)[static_cast<size_t>(t) * a.F + f] = __float2bfloat16_rn(u);
+      const float u = gelu_tanh(val(tok, p)) * val(tok, p + 64);
+      if (a.fp8) {
+        a.u_out[btile_offset(t, f, Nt, a.NKC_u)] = to_e4m3(u * inv);
+      } else {
+        *reinterpret_cast<__nv_bfloat16*>(a.u_out + btile_offset(t, 2 * f, Nt, a.NKC_u)) = __float2bfloat16_rn(u);
+      }
     }
   } else {   // EPI_QKV
     const int half = a.dh >> 1;
@@ -300,7 +382,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         const int t = n0 + tok;
         if (t >= a.T) continue;
         const int b = t / a.H, i = t % a.H, pos = a.P + i;
-        const float lo = gather(tok, p), hi = gather(tok, p + 64);
+        const float lo = val(tok, p), hi = val(tok, p + 64);
         const float c = a.rope_cos[pos * half + j], sn = a.rope_sin[pos * half + j];
         const float r0 = lo * c - hi * sn, r1 = lo * sn + hi * c;
         __nv_bfloat16* dst;
@@ -317,11 +399,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         const int t = n0 + tok;
         if (t >= a.T) continue;
         const int b = t / a.H, i = t % a.H, pos = a.P + i;
-        a.kv_v[((static_cast<size_t>(b) * a.Hkv + g) * a.S_max + pos) * a.dh + d] = __float2bfloat16_rn(gather(tok, row));
+        a.kv_v[((static_cast<size_t>(b) * a.Hkv + g) * a.S_max + pos) * a.dh + d] = __float2bfloat16_rn(val(tok, row));
       }
     }
   }
-  if (a.S > 1) cluster.sync();   // peers have finished reading this CTA's partial tile
+  if (S > 1 && tid == 0) bulk_wait_read_all();   // peers have read this CTA's slices
   __syncthreads();
   if (warp == 1) {
     __syncwarp();
@@ -332,7 +414,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
 
 // ================================================================== attention
 
-constexpr int SUBK = 64;          // keys per online-softmax step (the key chunk is a multiple of it)
 constexpr int ATT_PAD = 8;        // bf16 elements of row padding (16 bytes) against bank conflicts
 
 __device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc, bool valid) {
@@ -361,25 +442,55 @@ __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uin
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+struct AttnGeom {
+  uint32_t q_bytes, kv_bytes, obuf_bytes, recv_off, rowb;
+  int R;   // rows per owner (max)
+};
+
+__host__ __device__ __forceinline__ AttnGeom attn_geom(int H, int dh, int KC, int C) {
+  AttnGeom g;
+  const int Hp = (H + 15) & ~15;
+  const int LD = dh + ATT_PAD;
+  g.q_bytes = static_cast<uint32_t>(Hp) * LD * 2;
+  g.kv_bytes = 2u * static_cast<uint32_t>(KC) * LD * 2;
+  g.rowb = static_cast<uint32_t>(dh + 4) * 4;                  // O row + (max, sum) + pad
+  g.obuf_bytes = static_cast<uint32_t>(Hp) * g.rowb;
+  const uint32_t compute = g.q_bytes + g.kv_bytes;
+  const uint32_t a0 = compute > g.obuf_bytes ? compute : g.obuf_bytes;
+  g.recv_off = (a0 + 127u) & ~127u;
+  g.R = (H + C - 1) / C;
+  return g;
+}
+
 template <int DH>
 __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArgs a) {
   extern __shared__ __align__(128) uint8_t dsm[];
-  __shared__ float m_sh[256], l_sh[256];
-  __shared__ float w_sh[16][32];
+  __shared__ uint64_t recv_bar;
+  __shared__ float w_sh[16][16];
+  __shared__ float inv_den[16];
   constexpr int LD = DH + ATT_PAD;       // bf16 row stride in shared memory
+  constexpr int OLD = DH + 4;            // fp32 row stride of the partial-O rows
   const int c = blockIdx.x, j = blockIdx.y, b = blockIdx.z;
   const int g = (j * a.Hkv) / a.Hq;      // consecutive query-head groups share a KV head
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
   const int H = a.H, Hp = (H + 15) & ~15;
   const int S = a.P + H;
+  const int C = a.C;
   const int key0 = c * a.KC;
   const int nkeys = min(a.KC, S - key0);
+  const AttnGeom gm = attn_geom(H, DH, a.KC, C);
   __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(dsm);
-  __nv_bfloat16* Ks = Qs + Hp * LD;
+  __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(dsm + gm.q_bytes);
   __nv_bfloat16* Vs = Ks + a.KC * LD;
+  float* Obuf = reinterpret_cast<float*>(dsm);                  // after compute: [Hp][OLD]
+  float* recv = reinterpret_cast<float*>(dsm + gm.recv_off);    // [C][R][OLD]
   const __nv_bfloat16* kg = a.kv_k + ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max) * DH;
   const __nv_bfloat16* vg = a.kv_v + ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max) * DH;
   constexpr int VPR = DH / 8;            // 16-byte vectors per row
+  if (tid == 0) {
+    mbar_init(&recv_bar, 1);
+    fence_mbar_init();
+  }
   grid_dep_launch();
   // prefix keys/values do not depend on the previous kernel: start their loads first
   for (int it = tid; it < a.KC * VPR; it += blockDim.x) {
@@ -412,209 +523,262 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
 
   const int gq = lane >> 2, tq = lane & 3;
   const float sl2 = a.scale * 1.4426950408889634f;   // scores in log2 units
-  float* Obuf = reinterpret_cast<float*>(Ks);         // [Hp][DH] fp32, reused after the keys are consumed
-  const int n_rg = Hp / 16;
-  // each warp owns row groups rg = warp, warp + nw, ...
+  const int n_rg = Hp / 16;                           // one pass: n_rg <= number of warps
+  const int rg = warp;
+  const bool active = rg < n_rg;
   float oacc[DH / 8][4];
-  float mrow[2], lrow[2];
-  for (int rg0 = 0; rg0 < n_rg; rg0 += nw) {
-    const int rg = rg0 + warp;
-    const bool active = rg < n_rg;
-    if (active) {
+  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+  if (active) {
 #pragma unroll
-      for (int n = 0; n < DH / 8; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
-      mrow[0] = mrow[1] = -INFINITY;
-      lrow[0] = lrow[1] = 0.f;
-      const uint32_t qa = smem_u32(Qs + (rg * 16 + (lane & 15)) * LD + (lane >> 4) * 8);
-      for (int kb = 0; kb < nkeys; kb += SUBK) {
-        float sacc[SUBK / 8][4];
+    for (int n = 0; n < DH / 8; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
+    const uint32_t qa = smem_u32(Qs + (rg * 16 + (lane & 15)) * LD + (lane >> 4) * 8);
+    for (int kb = 0; kb < nkeys; kb += ATTN_SUBK) {
+      float sacc[ATTN_SUBK / 8][4];
 #pragma unroll
-        for (int n = 0; n < SUBK / 8; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+      for (int n = 0; n < ATTN_SUBK / 8; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(qa + kk * 32, a0, a1, a2, a3);
+      for (int kk = 0; kk < DH / 16; ++kk) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(qa + kk * 32, a0, a1, a2, a3);
 #pragma unroll
-          for (int n = 0; n < SUBK / 8; ++n) {
-            uint32_t b0, b1;
-            const uint32_t ka = smem_u32(Ks + (kb + n * 8 + (lane & 7)) * LD + kk * 16 + ((lane >> 3) & 1) * 8);
-            ldsm_x2(ka, b0, b1);
-            mma16816(sacc[n], a0, a1, a2, a3, b0, b1);
-          }
-        }
-        // scale, mask, online softmax
-        float mnew[2] = {mrow[0], mrow[1]};
-#pragma unroll
-        for (int n = 0; n < SUBK / 8; ++n) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int key = kb + n * 8 + tq * 2 + (e & 1);
-            float v = sacc[n][e] * sl2;
-            if (key >= nkeys) v = -INFINITY;
-            sacc[n][e] = v;
-            mnew[e >> 1] = fmaxf(mnew[e >> 1], v);
-          }
-        }
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          mnew[h2] = fmaxf(mnew[h2], __shfl_xor_sync(0xffffffffu, mnew[h2], 1));
-          mnew[h2] = fmaxf(mnew[h2], __shfl_xor_sync(0xffffffffu, mnew[h2], 2));
-        }
-        float corr[2], psum[2] = {0.f, 0.f};
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) corr[h2] = exp2f(mrow[h2] - mnew[h2]);
-#pragma unroll
-        for (int n = 0; n < SUBK / 8; ++n) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p = exp2f(sacc[n][e] - mnew[e >> 1]);
-            sacc[n][e] = p;
-            psum[e >> 1] += p;
-          }
-        }
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          psum[h2] += __shfl_xor_sync(0xffffffffu, psum[h2], 1);
-          psum[h2] += __shfl_xor_sync(0xffffffffu, psum[h2], 2);
-          lrow[h2] = lrow[h2] * corr[h2] + psum[h2];
-          mrow[h2] = mnew[h2];
-        }
-#pragma unroll
-        for (int n = 0; n < DH / 8; ++n) {
-          oacc[n][0] *= corr[0];
-          oacc[n][1] *= corr[0];
-          oacc[n][2] *= corr[1];
-          oacc[n][3] *= corr[1];
-        }
-        // O += P V
-#pragma unroll
-        for (int kk = 0; kk < SUBK / 16; ++kk) {
-          const uint32_t p0 = pack_bf16x2(sacc[2 * kk][0], sacc[2 * kk][1]);
-          const uint32_t p1 = pack_bf16x2(sacc[2 * kk][2], sacc[2 * kk][3]);
-          const uint32_t p2 = pack_bf16x2(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1]);
-          const uint32_t p3 = pack_bf16x2(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3]);
-          const uint32_t va0 = smem_u32(Vs + (kb + kk * 16 + (lane & 15)) * LD);
-#pragma unroll
-          for (int n = 0; n < DH / 8; ++n) {
-            uint32_t b0, b1;
-            ldsm_x2_t(va0 + n * 16, b0, b1);
-            mma16816(oacc[n], p0, p1, p2, p3, b0, b1);
-          }
+        for (int n = 0; n < ATTN_SUBK / 8; ++n) {
+          uint32_t b0, b1;
+          const uint32_t ka = smem_u32(Ks + (kb + n * 8 + (lane & 7)) * LD + kk * 16 + ((lane >> 3) & 1) * 8);
+          ldsm_x2(ka, b0, b1);
+          mma16816(sacc[n], a0, a1, a2, a3, b0, b1);
         }
       }
-    }
-    __syncthreads();   // all warps are done with Ks/Vs of this pass before Obuf overwrites them
-    if (active) {
-      const int r0 = rg * 16 + gq;
+      float mnew[2] = {mrow[0], mrow[1]};
+#pragma unroll
+      for (int n = 0; n < ATTN_SUBK / 8; ++n) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = kb + n * 8 + tq * 2 + (e & 1);
+          float v = sacc[n][e] * sl2;
+          if (key >= nkeys) v = -INFINITY;
+          sacc[n][e] = v;
+          mnew[e >> 1] = fmaxf(mnew[e >> 1], v);
+        }
+      }
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        mnew[h2] = fmaxf(mnew[h2], __shfl_xor_sync(0xffffffffu, mnew[h2], 1));
+        mnew[h2] = fmaxf(mnew[h2], __shfl_xor_sync(0xffffffffu, mnew[h2], 2));
+      }
+      float corr[2], psum[2] = {0.f, 0.f};
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) corr[h2] = exp2f(mrow[h2] - mnew[h2]);
+#pragma unroll
+      for (int n = 0; n < ATTN_SUBK / 8; ++n) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p = exp2f(sacc[n][e] - mnew[e >> 1]);
+          sacc[n][e] = p;
+          psum[e >> 1] += p;
+        }
+      }
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        psum[h2] += __shfl_xor_sync(0xffffffffu, psum[h2], 1);
+        psum[h2] += __shfl_xor_sync(0xffffffffu, psum[h2], 2);
+        lrow[h2] = lrow[h2] * corr[h2] + psum[h2];
+        mrow[h2] = mnew[h2];
+      }
 #pragma unroll
       for (int n = 0; n < DH / 8; ++n) {
-        const int col = n * 8 + tq * 2;
-        Obuf[r0 * DH + col] = oacc[n][0];
-        Obuf[r0 * DH + col + 1] = oacc[n][1];
-        Obuf[(r0 + 8) * DH + col] = oacc[n][2];
-        Obuf[(r0 + 8) * DH + col + 1] = oacc[n][3];
+        oacc[n][0] *= corr[0];
+        oacc[n][1] *= corr[0];
+        oacc[n][2] *= corr[1];
+        oacc[n][3] *= corr[1];
       }
-      if (tq == 0) {
-        m_sh[r0] = mrow[0];
-        l_sh[r0] = lrow[0];
-        m_sh[r0 + 8] = mrow[1];
-        l_sh[r0 + 8] = lrow[1];
+#pragma unroll
+      for (int kk = 0; kk < ATTN_SUBK / 16; ++kk) {
+        const uint32_t p0 = pack_bf16x2(sacc[2 * kk][0], sacc[2 * kk][1]);
+        const uint32_t p1 = pack_bf16x2(sacc[2 * kk][2], sacc[2 * kk][3]);
+        const uint32_t p2 = pack_bf16x2(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1]);
+        const uint32_t p3 = pack_bf16x2(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3]);
+        const uint32_t va0 = smem_u32(Vs + (kb + kk * 16 + (lane & 15)) * LD);
+#pragma unroll
+        for (int n = 0; n < DH / 8; ++n) {
+          uint32_t b0, b1;
+          ldsm_x2_t(va0 + n * 16, b0, b1);
+          mma16816(oacc[n], p0, p1, p2, p3, b0, b1);
+        }
       }
     }
+  }
+  __syncthreads();   // every warp is done with Q/K/V before the partial rows overwrite them
+  if (active) {
+    const int r0 = rg * 16 + gq;
+#pragma unroll
+    for (int n = 0; n < DH / 8; ++n) {
+      const int col = n * 8 + tq * 2;
+      Obuf[r0 * OLD + col] = oacc[n][0];
+      Obuf[r0 * OLD + col + 1] = oacc[n][1];
+      Obuf[(r0 + 8) * OLD + col] = oacc[n][2];
+      Obuf[(r0 + 8) * OLD + col + 1] = oacc[n][3];
+    }
+    if (tq == 0) {
+      Obuf[r0 * OLD + DH] = mrow[0];
+      Obuf[r0 * OLD + DH + 1] = lrow[0];
+      Obuf[(r0 + 8) * OLD + DH] = mrow[1];
+      Obuf[(r0 + 8) * OLD + DH + 1] = lrow[1];
+    }
+  }
+  // ---------------- push each owner its rows, merge the rows this CTA owns (rank order)
+  const int r_lo = c * H / C, r_hi = (c + 1) * H / C;
+  if (tid == 0) mbar_arrive_expect_tx(&recv_bar, static_cast<uint32_t>(C * (r_hi - r_lo)) * gm.rowb);
+  fence_proxy_async_smem();
+  __syncthreads();
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  if (tid == 0) {
+    for (int d = 0; d < C; ++d) {
+      const int d0 = d * H / C, d1 = (d + 1) * H / C;
+      if (d1 > d0)
+        bulk_s2cluster(mapa_shared(recv + static_cast<size_t>(c) * gm.R * OLD, d), Obuf + static_cast<size_t>(d0) * OLD,
+                       static_cast<uint32_t>(d1 - d0) * gm.rowb, mapa_shared(&recv_bar, d));
+    }
+    bulk_commit();
+  }
+  mbar_wait(&recv_bar, 0, WAIT_LIMIT_NS);
+  const int nr = r_hi - r_lo;   // <= 16 (host keeps H <= 16 C)
+  if (tid < nr) {
+    float M = -INFINITY;
+    for (int s = 0; s < C; ++s) M = fmaxf(M, recv[(static_cast<size_t>(s) * gm.R + tid) * OLD + DH]);
+    float den = 0.f;
+    for (int s = 0; s < C; ++s) {
+      const float* row = recv + (static_cast<size_t>(s) * gm.R + tid) * OLD;
+      const float e = exp2f(row[DH] - M);
+      w_sh[s][tid] = e;
+      den += e * row[DH + 1];
+    }
+    inv_den[tid] = 1.0f / den;
   }
   __syncthreads();
-  // ---------------- merge the key chunks of this (sample, head) over the cluster, in rank order
-  cg::cluster_group cluster = cg::this_cluster();
-  cluster.sync();
-  const int C = a.C;
-  const int r_lo = c * H / C, r_hi = (c + 1) * H / C;   // this CTA writes rows [r_lo, r_hi)
   const float inv_sa = (a.fp8 && a.s_a) ? 1.0f / *a.s_a : 1.0f;
-  for (int rb = r_lo; rb < r_hi; rb += 16) {
-    const int nr = min(16, r_hi - rb);
-    // weights of each chunk for these rows: w_s = 2^(m_s - M) / sum_s 2^(m_s - M) l_s
-    if (tid < nr) {
-      const int r = rb + tid;
-      float M = -INFINITY;
-      for (int s = 0; s < C; ++s) M = fmaxf(M, cluster.map_shared_rank(m_sh, s)[r]);
-      float den = 0.f;
-      for (int s = 0; s < C; ++s) {
-        const float e = exp2f(cluster.map_shared_rank(m_sh, s)[r] - M);
-        w_sh[s][tid] = e;
-        den += e * cluster.map_shared_rank(l_sh, s)[r];
-      }
-      const float inv = 1.0f / den;
-      for (int s = 0; s < C; ++s) w_sh[s][tid] *= inv;
-    }
-    __syncthreads();
-    for (int it = tid; it < nr * DH; it += blockDim.x) {
-      const int rr = it / DH, d = it % DH;
-      const int r = rb + rr;
-      float acc = 0.f;
-      for (int s = 0; s < C; ++s) acc += w_sh[s][rr] * cluster.map_shared_rank(Obuf, s)[r * DH + d];
-      const size_t oi = (static_cast<size_t>(b) * H + r) * (a.Hq * DH) + static_cast<size_t>(j) * DH + d;
-      if (a.fp8) a.o[oi] = to_e4m3(acc * inv_sa);
-      else reinterpret_cast<__nv_bfloat16*>(a.o)[oi] = __float2bfloat16_rn(acc);
-    }
-    __syncthreads();
+  for (int it = tid; it < nr * DH; it += blockDim.x) {
+    const int rr = it / DH, d = it % DH;
+    float acc = 0.f;
+    for (int s = 0; s < C; ++s) acc += w_sh[s][rr] * recv[(static_cast<size_t>(s) * gm.R + rr) * OLD + d];
+    acc *= inv_den[rr];
+    const int t = b * H + r_lo + rr;
+    const int kidx = j * DH + d;
+    if (a.fp8) a.o[btile_offset(t, kidx, a.Nt, a.NKC_o)] = to_e4m3(acc * inv_sa);
+    else *reinterpret_cast<__nv_bfloat16*>(a.o + btile_offset(t, 2 * kidx, a.Nt, a.NKC_o)) = __float2bfloat16_rn(acc);
   }
-  cluster.sync();   // peers have finished reading this CTA's partials
+  if (tid == 0) bulk_wait_read_all();   // peers have read this CTA's rows
+  __syncthreads();
 }
 
 // ================================================================== in-proj and final
 
-__global__ void __launch_bounds__(128) k_inproj_tc(const __grid_constant__ InprojArgs a) {
-  extern __shared__ float xs[];
-  __shared__ float wpart[4];
-  grid_dep_launch();
-  grid_dep_wait();
+__global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ InprojArgs a) {
+  extern __shared__ __align__(128) uint8_t dsm[];
+  __shared__ uint64_t wbar;
+  __shared__ float xs[64];
+  __shared__ float part[16][4];
+  __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(dsm);   // [D][A]
   const int t = blockIdx.x, tid = threadIdx.x;
-  for (int i = tid; i < a.A; i += blockDim.x) {
-    const float v = a.x[static_cast<size_t>(t) * a.A + i];
-    xs[i] = a.round_bf16 ? __bfloat162float(__float2bfloat16_rn(v)) : v;
+  const uint32_t wbytes = static_cast<uint32_t>(a.D) * a.A * 2;
+  if (tid == 0) {
+    mbar_init(&wbar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&wbar, wbytes);
+    bulk_g2s(wsm, a.w_in, wbytes, &wbar);   // static weights: before the dependency wait
   }
+  grid_dep_launch();
+  constexpr int QMAX = 16;                 // D <= 4096
+  float base[QMAX];
+#pragma unroll
+  for (int q = 0; q < QMAX; ++q) {
+    const int n = tid + q * 256;
+    base[q] = n < a.D ? a.b_in[n] + a.temb[n] : 0.f;
+  }
+  grid_dep_wait();
+  if (tid < a.A) xs[tid] = __bfloat162float(__float2bfloat16_rn(a.x[static_cast<size_t>(t) * a.A + tid]));
   __syncthreads();
-  const int nmb = (a.D + BM - 1) / BM;
-  for (int m = 0; m < nmb; ++m) {
-    const int n = m * BM + tid;
+  mbar_wait(&wbar, 0, WAIT_LIMIT_NS);
+  const int warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+  for (int q = 0; q < QMAX; ++q) {
+    const int n = tid + q * 256;
+    if (q * 256 >= a.D) break;
     float hv = 0.f;
     if (n < a.D) {
-      const float* wr = a.w_in + static_cast<size_t>(n) * a.A;
+      const __nv_bfloat16* wr = wsm + static_cast<size_t>(n) * a.A;
       float acc = 0.f;
-      for (int i = 0; i < a.A; ++i) acc = fmaf(wr[i], xs[i], acc);
-      hv = acc + a.b_in[n] + a.temb[n];
-      a.h[static_cast<size_t>(t) * a.D + n] = hv;
+      for (int i = 0; i < a.A; ++i) acc = fmaf(__bfloat162float(wr[i]), xs[i], acc);
+      hv = acc + base[q];
+      a.h[htile_offset(t, n, a.Nt, a.KB)] = hv;
     }
     float sq = hv * hv;
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    if ((tid & 31) == 0) wpart[tid >> 5] = sq;
-    __syncthreads();
-    if (tid == 0) a.ssq[m * a.T_pad + t] = ((wpart[0] + wpart[1]) + wpart[2]) + wpart[3];
-    __syncthreads();
+    if (lane == 0) part[2 * q + (warp >> 2)][warp & 3] = sq;
   }
+  __syncthreads();
+  const int nmb = (a.D + BM - 1) / BM;
+  if (tid < nmb) a.ssq[static_cast<size_t>(t) * a.ssq_ld + tid] = ((part[tid][0] + part[tid][1]) + part[tid][2]) + part[tid][3];
 }
 
-__global__ void __launch_bounds__(128) k_final_tc(const __grid_constant__ FinalArgs a) {
-  extern __shared__ float hn[];
-  grid_dep_launch();
-  grid_dep_wait();
+__global__ void __launch_bounds__(256) k_final_tc(const __grid_constant__ FinalArgs a) {
+  extern __shared__ __align__(128) uint8_t dsm[];
+  __shared__ uint64_t wbar;
+  __shared__ float ssq_sh[16];
+  __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(dsm);                     // [A][D]
+  float* hn = reinterpret_cast<float*>(dsm + ((static_cast<size_t>(a.A) * a.D * 2 + 127) & ~size_t(127)));
   const int t = blockIdx.x, tid = threadIdx.x;
-  float ss = 0.f;
-  for (int p = 0; p < a.ssq_parts; ++p) ss += a.ssq[p * a.T_pad + t];
-  const float r = 1.0f / sqrtf(ss / a.D + a.eps);
-  for (int k = tid; k < a.D; k += blockDim.x)
-    hn[k] = __bfloat162float(__float2bfloat16_rn(a.h[static_cast<size_t>(t) * a.D + k] * r * a.g_f[k]));
+  const uint32_t wbytes = static_cast<uint32_t>(a.A) * a.D * 2;
+  if (tid == 0) {
+    mbar_init(&wbar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&wbar, wbytes);
+    bulk_g2s(wsm, a.w_out, wbytes, &wbar);   // static weights: before the dependency wait
+  }
+  grid_dep_launch();
+  constexpr int QMAX = 16;
+  float gf[QMAX];
+#pragma unroll
+  for (int q = 0; q < QMAX; ++q) {
+    const int k = tid + q * 256;
+    gf[q] = k < a.D ? a.g_f[k] : 0.f;
+  }
+  grid_dep_wait();
+  float hv[QMAX];
+#pragma unroll
+  for (int q = 0; q < QMAX; ++q) {
+    const int k = tid + q * 256;
+    hv[q] = k < a.D ? a.h[htile_offset(t, k, a.Nt, a.KB)] : 0.f;
+  }
+  if (tid < a.ssq_parts) ssq_sh[tid] = a.ssq[static_cast<size_t>(t) * a.ssq_ld + tid];
   __syncthreads();
-  const int warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
-  for (int i = warp; i < a.A; i += nw) {
-    const float* wr = a.w_out + static_cast<size_t>(i) * a.D;
+  float ss = 0.f;
+  for (int p = 0; p < a.ssq_parts; ++p) ss += ssq_sh[p];
+  const float r = 1.0f / sqrtf(ss / a.D + a.eps);
+#pragma unroll
+  for (int q = 0; q < QMAX; ++q) {
+    const int k = tid + q * 256;
+    if (k < a.D) hn[k] = __bfloat162float(__float2bfloat16_rn(hv[q] * r * gf[q]));
+  }
+  __syncthreads();
+  mbar_wait(&wbar, 0, WAIT_LIMIT_NS);
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int i = warp; i < a.A; i += 8) {
+    const __nv_bfloat16* wr = wsm + static_cast<size_t>(i) * a.D;
     float acc = 0.f;
-    for (int k = lane; k < a.D; k += 32) acc = fmaf(wr[k], hn[k], acc);
+    for (int k = lane; k < a.D; k += 32) acc = fmaf(__bfloat162float(wr[k]), hn[k], acc);
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) {
       const size_t xi = static_cast<size_t>(t) * a.A + i;
       a.x_out[xi] = a.x_in[xi] + a.dt * (acc + a.b_out[i]);
     }
   }
+}
+
+__global__ void k_to_bf16(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    dst[i] = __float2bfloat16_rn(src[i]);
 }
 
 // ================================================================== launch helpers
@@ -647,17 +811,18 @@ cudaError_t launch_ex(const void* func, dim3 grid, dim3 block, size_t smem, cuda
 
 }  // namespace
 
-size_t gemm_smem_bytes(int Nt, int stages) {
-  const size_t ring = static_cast<size_t>(stages) * (BM * KCB + static_cast<size_t>(Nt) * KCB);
-  const size_t red = static_cast<size_t>(Nt) * RED_LD * sizeof(float);
-  return ring > red ? ring : red;
+size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk) {
+  const GemmGeom g = gemm_geom(Nt, stages, b_kind, fp8, S, nk);
+  const size_t kel = fp8 ? KCB : KCB / 2;
+  const size_t main = g.ring + (b_kind == B_NORM ? static_cast<size_t>(nk) * kel * 4 : 0);
+  const size_t red = static_cast<size_t>(Nt) * RED_LD * 4;
+  const size_t epi = S > 1 ? g.recv_off + static_cast<size_t>(S) * g.TS * RED_LD * 4 : red;
+  return main > epi ? main : epi;
 }
 
-size_t attn_smem_bytes(int H, int dh, int KC) {
-  const int Hp = (H + 15) & ~15;
-  const size_t qkv = (static_cast<size_t>(Hp) + 2 * KC) * (dh + ATT_PAD) * 2;
-  const size_t obuf = static_cast<size_t>(Hp) * dh * 4 + static_cast<size_t>(Hp) * (dh + ATT_PAD) * 2;
-  return qkv > obuf ? qkv : obuf;
+size_t attn_smem_bytes(int H, int dh, int KC, int C) {
+  const AttnGeom g = attn_geom(H, dh, KC, C);
+  return g.recv_off + static_cast<size_t>(C) * g.R * g.rowb;
 }
 
 cudaError_t tc_kernels_init() {
@@ -666,12 +831,16 @@ cudaError_t tc_kernels_init() {
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
   const void* fns[] = {reinterpret_cast<const void*>(k_gemm_tc), reinterpret_cast<const void*>(k_attn_tc<64>),
-                       reinterpret_cast<const void*>(k_attn_tc<128>), reinterpret_cast<const void*>(k_attn_tc<256>)};
+                       reinterpret_cast<const void*>(k_attn_tc<128>), reinterpret_cast<const void*>(k_attn_tc<256>),
+                       reinterpret_cast<const void*>(k_inproj_tc), reinterpret_cast<const void*>(k_final_tc)};
   for (const void* f : fns) {
     cudaFuncAttributes fa;
     if ((e = cudaFuncGetAttributes(&fa, f)) != cudaSuccess) return e;
     const int dyn = optin - static_cast<int>(fa.sharedSizeBytes);
     if ((e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared)) !=
+        cudaSuccess)
+      return e;
     if ((e = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -689,8 +858,9 @@ int max_dynamic_smem() {
 cudaError_t launch_gemm_tc(const GemmArgs& a, int n_tiles, cudaStream_t s, bool pdl) {
   GemmArgs copy = a;
   void* args[] = {&copy};
+  const int nk_max = (a.NKC + a.S - 1) / a.S;
   return launch_ex(reinterpret_cast<const void*>(k_gemm_tc), dim3(a.S, a.MB, n_tiles), dim3(GEMM_THREADS),
-                   gemm_smem_bytes(a.Nt, a.stages), s, pdl, a.S, args);
+                   gemm_smem_bytes(a.Nt, a.stages, a.b_kind, a.fp8, a.S, nk_max), s, pdl, a.S, args);
 }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, int B, cudaStream_t s, bool pdl) {
@@ -701,21 +871,26 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int B, cudaStream_t s, bool p
   const void* f = a.dh == 64 ? reinterpret_cast<const void*>(k_attn_tc<64>)
                 : a.dh == 128 ? reinterpret_cast<const void*>(k_attn_tc<128>)
                               : reinterpret_cast<const void*>(k_attn_tc<256>);
-  return launch_ex(f, dim3(a.C, a.Hq, B), dim3(32 * nw), attn_smem_bytes(a.H, a.dh, a.KC), s, pdl, a.C, args);
+  return launch_ex(f, dim3(a.C, a.Hq, B), dim3(32 * nw), attn_smem_bytes(a.H, a.dh, a.KC, a.C), s, pdl, a.C, args);
 }
 
 cudaError_t launch_inproj_tc(const InprojArgs& a, cudaStream_t s, bool pdl) {
   InprojArgs copy = a;
   void* args[] = {&copy};
-  return launch_ex(reinterpret_cast<const void*>(k_inproj_tc), dim3(a.T), dim3(128), a.A * sizeof(float), s, pdl, 1,
-                   args);
+  return launch_ex(reinterpret_cast<const void*>(k_inproj_tc), dim3(a.T), dim3(256),
+                   static_cast<size_t>(a.D) * a.A * 2, s, pdl, 1, args);
 }
 
 cudaError_t launch_final_tc(const FinalArgs& a, cudaStream_t s, bool pdl) {
   FinalArgs copy = a;
   void* args[] = {&copy};
-  return launch_ex(reinterpret_cast<const void*>(k_final_tc), dim3(a.T), dim3(128), a.D * sizeof(float), s, pdl, 1,
-                   args);
+  const size_t smem = ((static_cast<size_t>(a.A) * a.D * 2 + 127) & ~size_t(127)) + static_cast<size_t>(a.D) * 4;
+  return launch_ex(reinterpret_cast<const void*>(k_final_tc), dim3(a.T), dim3(256), smem, s, pdl, 1, args);
+}
+
+cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s) {
+  k_to_bf16<<<static_cast<unsigned>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0, s>>>(src, dst, n);
+  return cudaGetLastError();
 }
 
 const void* inproj_kernel_ptr() { return reinterpret_cast<const void*>(k_inproj_tc); }

@@ -43,6 +43,13 @@ ProjLayout make_layout(int rows, int K, int elem) {
   return p;
 }
 
+// Key chunks of the split-KV attention: at most 16 (one cluster), a multiple of the 64-key step.
+void attn_chunks(int S, int& C, int& KC) {
+  C = std::min(16, ceil_div(S, ATTN_SUBK));
+  KC = static_cast<int>(align_up(ceil_div(S, C), ATTN_SUBK));
+  C = ceil_div(S, KC);
+}
+
 struct GemmPlan {
   int S = 1, stages = 1;
 };
@@ -79,17 +86,22 @@ struct TensorPath {
   int max_dyn = 0;
   int fp8 = 0, elem = 2;
   int T_max = 0, T_pad = 0, MBd = 0, MB_rot = 0;
+  int KB = 0;                    // 64-feature blocks of h per n-tile (D rounded up to 128)
+  int ssq_ld = 0;                // columns of the Σh² partials (MBd rounded up to 4)
+  int tok_alloc = 0;             // token rows of the tiled buffers (covers NT * Nt for every batch)
   ProjLayout qkv, o, gu, dn;
   size_t layer_bytes = 0;
   uint8_t* w = nullptr;          // [L][qkv|o|gu|dn] tiled weights
   float* gains = nullptr;        // [L][2][D]
-  float* h = nullptr;            // [T_max][D]
-  float* ssq_a = nullptr;        // [MBd][T_pad]
+  float* h = nullptr;            // tiled [NT][KB][Nt][64]
+  float* ssq_a = nullptr;        // [T_pad][ssq_ld]
   float* ssq_b = nullptr;
   __nv_bfloat16* qbuf = nullptr; // [B_max][Hq][H][dh]
-  uint8_t* obuf = nullptr;       // [T_max][Hq dh] bf16 / e4m3
-  uint8_t* ubuf = nullptr;       // [T_max][F]
+  uint8_t* obuf = nullptr;       // tiled [NT][NKC_o][Nt x 128] bf16 / e4m3
+  uint8_t* ubuf = nullptr;       // tiled [NT][NKC_u][Nt x 128]
   float* xs = nullptr;           // [T_max][A] state between steps
+  __nv_bfloat16* w_in_bf = nullptr;   // [D][A]
+  __nv_bfloat16* w_out_bf = nullptr;  // [A][D]
   cudaStream_t cap = nullptr;
   std::map<std::pair<int, int>, GraphEntry> graphs;
   std::vector<float> gains_host;
@@ -121,13 +133,15 @@ size_t carve_all(TensorPath* tp, char* base) {
   Carve cv{base};
   tp->w = cv.take<uint8_t>(tp->layer_bytes * c.L, 1024);
   tp->gains = cv.take<float>(static_cast<size_t>(c.L) * 2 * c.D);
-  tp->h = cv.take<float>(static_cast<size_t>(tp->T_max) * c.D);
-  tp->ssq_a = cv.take<float>(static_cast<size_t>(tp->MBd) * tp->T_pad);
-  tp->ssq_b = cv.take<float>(static_cast<size_t>(tp->MBd) * tp->T_pad);
+  tp->h = cv.take<float>(static_cast<size_t>(tp->tok_alloc) * tp->KB * 64);
+  tp->ssq_a = cv.take<float>(static_cast<size_t>(tp->T_pad) * tp->ssq_ld);
+  tp->ssq_b = cv.take<float>(static_cast<size_t>(tp->T_pad) * tp->ssq_ld);
   tp->qbuf = cv.take<__nv_bfloat16>(static_cast<size_t>(c.B_max) * c.Hq * c.H * c.dh);
-  tp->obuf = cv.take<uint8_t>(static_cast<size_t>(tp->T_max) * c.Hq * c.dh * tp->elem);
-  tp->ubuf = cv.take<uint8_t>(static_cast<size_t>(tp->T_max) * c.F * tp->elem);
+  tp->obuf = cv.take<uint8_t>(static_cast<size_t>(tp->tok_alloc) * tp->o.NKC * KCB);
+  tp->ubuf = cv.take<uint8_t>(static_cast<size_t>(tp->tok_alloc) * tp->dn.NKC * KCB);
   tp->xs = cv.take<float>(static_cast<size_t>(tp->T_max) * c.A);
+  tp->w_in_bf = cv.take<__nv_bfloat16>(static_cast<size_t>(c.D) * c.A);
+  tp->w_out_bf = cv.take<__nv_bfloat16>(static_cast<size_t>(c.A) * c.D);
   return align_up(cv.off, 1024);
 }
 
@@ -139,22 +153,25 @@ void init_sizes(TensorPath* tp, const fr_config& c) {
   tp->T_pad = static_cast<int>(align_up(tp->T_max, 16));
   tp->MBd = ceil_div(c.D, BM);
   tp->MB_rot = (c.Hq + c.Hkv) * c.dh / 2 / 64;
+  tp->KB = ceil_div(c.D, BM) * 2;
+  tp->ssq_ld = static_cast<int>(align_up(tp->MBd, 4));
+  const int nt_max = ceil_div(tp->T_max, NT_MAX);
+  tp->tok_alloc = tp->T_max + 16 * nt_max;
   layouts(c, tp->elem, tp->qkv, tp->o, tp->gu, tp->dn);
   tp->layer_bytes = tp->qkv.bytes + tp->o.bytes + tp->gu.bytes + tp->dn.bytes;
 }
 
 // Split-K / ring choice for one projection: a small cost model over S (cluster size).
-GemmPlan choose_plan(int tiles, int NKC, int Nt, int nsm, int max_dyn) {
-  const size_t slot = BM * KCB + static_cast<size_t>(Nt) * KCB;
-  const size_t red = static_cast<size_t>(Nt) * (BM + 4) * 4;
+GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int nsm, int max_dyn) {
   GemmPlan best;
   double best_cost = 1e30;
   for (int S = 1; S <= 16 && S <= NKC; ++S) {
     const int chunks = ceil_div(NKC, S);
     int stages = std::min(chunks, MAX_STAGES);
-    while (stages > 1 && std::max(stages * slot, red) > static_cast<size_t>(max_dyn)) --stages;
-    const size_t smem = std::max(stages * slot, red) + 2048;
-    const int per_sm = std::max(1, std::min(2, static_cast<int>((228 * 1024) / smem)));
+    while (stages > 1 && gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks) > static_cast<size_t>(max_dyn)) --stages;
+    const size_t smem = gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks);
+    if (smem > static_cast<size_t>(max_dyn)) continue;
+    const int per_sm = std::max(1, std::min(2, static_cast<int>((228 * 1024) / (smem + 4096))));
     const int waves = ceil_div(tiles * S, nsm * per_sm);
     const double cost = waves * (chunks + 0.1 * S);
     if (cost < best_cost - 1e-9) {
@@ -174,14 +191,11 @@ StepPlan make_plan(const TensorPath* tp, int B, int P) {
   p.T = B * c.H;
   p.NT = ceil_div(p.T, NT_MAX);
   p.Nt = static_cast<int>(align_up(ceil_div(p.T, p.NT), 16));
-  p.qkv = choose_plan(tp->qkv.MB * p.NT, tp->qkv.NKC, p.Nt, tp->nsm, tp->max_dyn);
-  p.o = choose_plan(tp->o.MB * p.NT, tp->o.NKC, p.Nt, tp->nsm, tp->max_dyn);
-  p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, tp->nsm, tp->max_dyn);
-  p.dn = choose_plan(tp->dn.MB * p.NT, tp->dn.NKC, p.Nt, tp->nsm, tp->max_dyn);
-  const int S = P + c.H;
-  int C = std::min(16, ceil_div(S, ATTN_SUBK));
-  p.attn_KC = static_cast<int>(align_up(ceil_div(S, C), ATTN_SUBK));
-  p.attn_C = ceil_div(S, p.attn_KC);
+  p.qkv = choose_plan(tp->qkv.MB * p.NT, tp->qkv.NKC, p.Nt, B_NORM, tp->fp8, tp->nsm, tp->max_dyn);
+  p.o = choose_plan(tp->o.MB * p.NT, tp->o.NKC, p.Nt, B_ROWS, tp->fp8, tp->nsm, tp->max_dyn);
+  p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, B_NORM, tp->fp8, tp->nsm, tp->max_dyn);
+  p.dn = choose_plan(tp->dn.MB * p.NT, tp->dn.NKC, p.Nt, B_ROWS, tp->fp8, tp->nsm, tp->max_dyn);
+  attn_chunks(P + c.H, p.attn_C, p.attn_KC);
   return p;
 }
 
@@ -222,9 +236,11 @@ GemmArgs base_args(const TensorPath* tp, const StepPlan& p, const ProjLayout& L,
   a.fp8 = tp->fp8;
   a.T = p.T;
   a.Nt = p.Nt;
-  a.Kdim = L.K;
+  a.KB = tp->KB;
+  a.D = c.D;
   a.eps = c.eps;
-  a.T_pad = tp->T_pad;
+  a.ssq_ld = tp->ssq_ld;
+  a.ssq_parts = tp->MBd;
   a.status = tp->tb.status;
   return a;
 }
@@ -239,7 +255,7 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
     float* x_nx = (k == c.K - 1) ? x_out : tp->xs;
     InprojArgs ia{};
     ia.x = x_in;
-    ia.w_in = tp->tb.w_in;
+    ia.w_in = tp->w_in_bf;
     ia.b_in = tp->tb.b_in;
     ia.temb = tp->tb.temb + static_cast<size_t>(k) * c.D;
     ia.h = tp->h;
@@ -247,8 +263,9 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
     ia.T = p.T;
     ia.D = c.D;
     ia.A = c.A;
-    ia.T_pad = tp->T_pad;
-    ia.round_bf16 = 1;
+    ia.Nt = p.Nt;
+    ia.KB = tp->KB;
+    ia.ssq_ld = tp->ssq_ld;
     ia.first = (k == 0);
     if ((e = launch_inproj_tc(ia, s, true)) != cudaSuccess) return cuda_fail(e, "in-proj kernel launch");
     for (int l = 0; l < c.L; ++l) {
@@ -264,7 +281,6 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       q.h = tp->h;
       q.gamma = g1;
       q.ssq = tp->ssq_a;
-      q.ssq_parts = tp->MBd;
       q.s_a = tp->fp8 ? sa + PI_QKV : nullptr;
       q.alpha = tp->fp8 ? al + PI_QKV : nullptr;
       q.epi = EPI_QKV;
@@ -287,6 +303,8 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       at.kv_k = kvk;
       at.kv_v = kvv;
       at.o = tp->obuf;
+      at.Nt = p.Nt;
+      at.NKC_o = tp->o.NKC;
       at.s_a = tp->fp8 ? sa + PI_O : nullptr;
       at.fp8 = tp->fp8;
       at.H = c.H;
@@ -303,12 +321,10 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       GemmArgs og = base_args(tp, p, tp->o, p.o, l, o_off);
       og.b_kind = B_ROWS;
       og.act = tp->obuf;
-      og.act_ld = c.Hq * c.dh;
       og.alpha = tp->fp8 ? al + PI_O : nullptr;
       og.epi = EPI_RESID;
       og.h_out = tp->h;
       og.ssq_out = tp->ssq_b;
-      og.D = c.D;
       if ((e = launch_gemm_tc(og, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "o GEMM launch");
       // gate|up with RMSNorm fused, GeLU(gate)*up epilogue
       GemmArgs gg = base_args(tp, p, tp->gu, p.gu, l, gu_off);
@@ -316,11 +332,11 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       gg.h = tp->h;
       gg.gamma = g2;
       gg.ssq = tp->ssq_b;
-      gg.ssq_parts = tp->MBd;
       gg.s_a = tp->fp8 ? sa + PI_GU : nullptr;
       gg.alpha = tp->fp8 ? al + PI_GU : nullptr;
       gg.epi = EPI_GELU;
       gg.u_out = tp->ubuf;
+      gg.NKC_u = tp->dn.NKC;
       gg.s_a_out = tp->fp8 ? sa + PI_DOWN : nullptr;
       gg.F = c.F;
       if ((e = launch_gemm_tc(gg, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "gate|up GEMM launch");
@@ -328,27 +344,27 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       GemmArgs dg = base_args(tp, p, tp->dn, p.dn, l, dn_off);
       dg.b_kind = B_ROWS;
       dg.act = tp->ubuf;
-      dg.act_ld = c.F;
       dg.alpha = tp->fp8 ? al + PI_DOWN : nullptr;
       dg.epi = EPI_RESID;
       dg.h_out = tp->h;
       dg.ssq_out = tp->ssq_a;
-      dg.D = c.D;
       if ((e = launch_gemm_tc(dg, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "down GEMM launch");
     }
     FinalArgs fa{};
     fa.h = tp->h;
     fa.ssq = tp->ssq_a;
+    fa.ssq_ld = tp->ssq_ld;
     fa.ssq_parts = tp->MBd;
     fa.g_f = tp->tb.g_f;
-    fa.w_out = tp->tb.w_out;
+    fa.w_out = tp->w_out_bf;
     fa.b_out = tp->tb.b_out;
     fa.x_in = x_in;
     fa.x_out = x_nx;
     fa.T = p.T;
     fa.D = c.D;
     fa.A = c.A;
-    fa.T_pad = tp->T_pad;
+    fa.Nt = p.Nt;
+    fa.KB = tp->KB;
     fa.eps = c.eps;
     fa.dt = dt;
     fa.first = (k == 0);
@@ -436,16 +452,17 @@ bool tensor_path_supports(const fr_config& c) {
   if (c.F % 64 != 0) return false;                            // gate/up pairs fill whole m-blocks
   if (c.H > 128) return false;                                // one attention row-group pass per warp
   if (c.D % 16 != 0 || (c.Hq * c.dh) % 16 != 0) return false; // 16-byte operand rows
-  const int S = c.P_max + c.H;
-  const int C = std::min(16, ceil_div(S, ATTN_SUBK));
-  const int KC = static_cast<int>(align_up(ceil_div(S, C), ATTN_SUBK));
-  if (attn_smem_bytes(c.H, c.dh, KC) > 200 * 1024) return false;
+  if (c.D > 2048 || c.A > 64) return false;                     // per-token kernels keep a row in registers
+  if (static_cast<size_t>(c.D) * c.A * 2 > 160 * 1024) return false;   // in/out-proj weights fit shared memory
+  int C = 1, KC = 64;
+  attn_chunks(c.P_max + c.H, C, KC);
+  if (attn_smem_bytes(c.H, c.dh, KC, C) > 200 * 1024) return false;
   return true;
 }
 
 const char* tensor_path_limits() {
   return "bf16/fp8, dh in {64,128,256}, (Hq+Hkv)*dh/2 % 64 == 0, Hkv*dh % 128 == 0, F % 64 == 0, H <= 128, "
-         "D % 16 == 0, attention chunk fits shared memory";
+         "D % 16 == 0, D <= 2048, A <= 64, attention chunk fits shared memory";
 }
 
 size_t tensor_path_bytes(const fr_config& c) {
@@ -529,8 +546,13 @@ int tensor_path_pack_layer(TensorPath* tp, int l, const fr_layer_weights& w, con
   return FR_OK;
 }
 
-int tensor_path_finish_load(TensorPath* tp, cudaStream_t) {
+int tensor_path_finish_load(TensorPath* tp, cudaStream_t s) {
+  const fr_config& c = tp->c;
   FR_CUDA(cudaMemcpy(tp->gains, tp->gains_host.data(), tp->gains_host.size() * 4, cudaMemcpyHostToDevice));
+  // in/out-proj weights hold bf16-rounded values already: the conversion is exact
+  FR_CUDA(launch_to_bf16(tp->tb.w_in, tp->w_in_bf, static_cast<size_t>(c.D) * c.A, s));
+  FR_CUDA(launch_to_bf16(tp->tb.w_out, tp->w_out_bf, static_cast<size_t>(c.A) * c.D, s));
+  FR_CUDA(cudaStreamSynchronize(s));
   return FR_OK;
 }
 
