@@ -455,9 +455,7 @@ __host__ __device__ __forceinline__ AttnGeom attn_geom(int H, int dh, int KC, in
   g.kv_bytes = 2u * static_cast<uint32_t>(KC) * LD * 2;
   g.rowb = static_cast<uint32_t>(dh + 4) * 4;                  // O row + (max, sum) + pad
   g.obuf_bytes = static_cast<uint32_t>(Hp) * g.rowb;
-  const uint32_t compute = g.q_bytes + g.kv_bytes;
-  const uint32_t a0 = compute > g.obuf_bytes ? compute : g.obuf_bytes;
-  g.recv_off = (a0 + 127u) & ~127u;
+  g.recv_off = (g.obuf_bytes + 127u) & ~127u;                  // Obuf and recv both overlay the dead Q/K/V
   g.R = (H + C - 1) / C;
   return g;
 }
@@ -466,8 +464,8 @@ template <int DH>
 __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArgs a) {
   extern __shared__ __align__(128) uint8_t dsm[];
   __shared__ uint64_t recv_bar;
-  __shared__ float w_sh[16][16];
-  __shared__ float inv_den[16];
+  __shared__ float w_sh[16][128];   // merge weight of chunk s for owned row rr (C <= 16, rows <= H <= 128)
+  __shared__ float inv_den[128];
   constexpr int LD = DH + ATT_PAD;       // bf16 row stride in shared memory
   constexpr int OLD = DH + 4;            // fp32 row stride of the partial-O rows
   const int c = blockIdx.x, j = blockIdx.y, b = blockIdx.z;
@@ -627,28 +625,39 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
   }
   // ---------------- push each owner its rows, merge the rows this CTA owns (rank order)
   const int r_lo = c * H / C, r_hi = (c + 1) * H / C;
-  if (tid == 0) mbar_arrive_expect_tx(&recv_bar, static_cast<uint32_t>(C * (r_hi - r_lo)) * gm.rowb);
-  fence_proxy_async_smem();
-  __syncthreads();
-  cluster_arrive_release();
-  cluster_wait_acquire();
-  if (tid == 0) {
-    for (int d = 0; d < C; ++d) {
-      const int d0 = d * H / C, d1 = (d + 1) * H / C;
-      if (d1 > d0)
-        bulk_s2cluster(mapa_shared(recv + static_cast<size_t>(c) * gm.R * OLD, d), Obuf + static_cast<size_t>(d0) * OLD,
-                       static_cast<uint32_t>(d1 - d0) * gm.rowb, mapa_shared(&recv_bar, d));
+  const float* src;        // row rr of chunk s at src + (s * rstride + rr) * OLD
+  size_t rstride;
+  if (C > 1) {
+    if (tid == 0) mbar_arrive_expect_tx(&recv_bar, static_cast<uint32_t>(C * (r_hi - r_lo)) * gm.rowb);
+    fence_proxy_async_smem();
+    __syncthreads();
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    if (tid == 0) {
+      for (int d = 0; d < C; ++d) {
+        const int d0 = d * H / C, d1 = (d + 1) * H / C;
+        if (d1 > d0)
+          bulk_s2cluster(mapa_shared(recv + static_cast<size_t>(c) * gm.R * OLD, d),
+                         Obuf + static_cast<size_t>(d0) * OLD, static_cast<uint32_t>(d1 - d0) * gm.rowb,
+                         mapa_shared(&recv_bar, d));
+      }
+      bulk_commit();
     }
-    bulk_commit();
+    mbar_wait(&recv_bar, 0, WAIT_LIMIT_NS);
+    src = recv;
+    rstride = gm.R;
+  } else {   // a single key chunk: no cluster, the CTA's own rows are final
+    __syncthreads();
+    src = Obuf;
+    rstride = 0;
   }
-  mbar_wait(&recv_bar, 0, WAIT_LIMIT_NS);
-  const int nr = r_hi - r_lo;   // <= 16 (host keeps H <= 16 C)
+  const int nr = r_hi - r_lo;
   if (tid < nr) {
     float M = -INFINITY;
-    for (int s = 0; s < C; ++s) M = fmaxf(M, recv[(static_cast<size_t>(s) * gm.R + tid) * OLD + DH]);
+    for (int s = 0; s < C; ++s) M = fmaxf(M, src[(static_cast<size_t>(s) * rstride + tid) * OLD + DH]);
     float den = 0.f;
     for (int s = 0; s < C; ++s) {
-      const float* row = recv + (static_cast<size_t>(s) * gm.R + tid) * OLD;
+      const float* row = src + (static_cast<size_t>(s) * rstride + tid) * OLD;
       const float e = exp2f(row[DH] - M);
       w_sh[s][tid] = e;
       den += e * row[DH + 1];
@@ -660,14 +669,14 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
   for (int it = tid; it < nr * DH; it += blockDim.x) {
     const int rr = it / DH, d = it % DH;
     float acc = 0.f;
-    for (int s = 0; s < C; ++s) acc += w_sh[s][rr] * recv[(static_cast<size_t>(s) * gm.R + rr) * OLD + d];
+    for (int s = 0; s < C; ++s) acc += w_sh[s][rr] * src[(static_cast<size_t>(s) * rstride + rr) * OLD + d];
     acc *= inv_den[rr];
     const int t = b * H + r_lo + rr;
     const int kidx = j * DH + d;
     if (a.fp8) a.o[btile_offset(t, kidx, a.Nt, a.NKC_o)] = to_e4m3(acc * inv_sa);
     else *reinterpret_cast<__nv_bfloat16*>(a.o + btile_offset(t, 2 * kidx, a.Nt, a.NKC_o)) = __float2bfloat16_rn(acc);
   }
-  if (tid == 0) bulk_wait_read_all();   // peers have read this CTA's rows
+  if (C > 1 && tid == 0) bulk_wait_read_all();   // peers have read this CTA's rows
   __syncthreads();
 }
 
@@ -703,7 +712,7 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
 #pragma unroll
   for (int q = 0; q < QMAX; ++q) {
     const int n = tid + q * 256;
-    if (q * 256 >= a.D) break;
+    if (q * 256 >= a.D) continue;   // uniform across the block
     float hv = 0.f;
     if (n < a.D) {
       const __nv_bfloat16* wr = wsm + static_cast<size_t>(n) * a.A;
@@ -822,7 +831,9 @@ size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk) {
 
 size_t attn_smem_bytes(int H, int dh, int KC, int C) {
   const AttnGeom g = attn_geom(H, dh, KC, C);
-  return g.recv_off + static_cast<size_t>(C) * g.R * g.rowb;
+  const size_t compute = static_cast<size_t>(g.q_bytes) + g.kv_bytes;
+  const size_t merge = C > 1 ? g.recv_off + static_cast<size_t>(C) * g.R * g.rowb : g.obuf_bytes;
+  return compute > merge ? compute : merge;
 }
 
 cudaError_t tc_kernels_init() {
