@@ -33,6 +33,34 @@ namespace {
 
 using namespace fr::sm100;
 
+// Optional phase timestamps (globaltimer per CTA), compiled in only with -DFR_TIMELINE for
+// performance analysis; the product build has none of this code.
+#ifdef FR_TIMELINE
+__device__ unsigned long long* g_tl = nullptr;   // [cap][8]: kind, cta, t0..t5
+__device__ unsigned g_tl_count = 0;
+__device__ unsigned g_tl_cap = 0;
+#define TL_DECL __shared__ unsigned tl_slot_;
+#define TL_BEGIN(kind)                                                                          \
+  do {                                                                                          \
+    if (threadIdx.x == 0) {                                                                     \
+      tl_slot_ = g_tl ? atomicAdd(&g_tl_count, 1u) : 0xFFFFFFFFu;                               \
+      if (tl_slot_ < g_tl_cap) {                                                                \
+        g_tl[tl_slot_ * 8 + 0] = (kind);                                                        \
+        g_tl[tl_slot_ * 8 + 1] = blockIdx.x | (blockIdx.y << 10) | (blockIdx.z << 20);          \
+        g_tl[tl_slot_ * 8 + 2] = fr::sm100::globaltimer();                                      \
+      }                                                                                         \
+    }                                                                                           \
+  } while (0)
+#define TL(k)                                                                                   \
+  do {                                                                                          \
+    if (tl_slot_ < g_tl_cap) g_tl[tl_slot_ * 8 + 2 + (k)] = fr::sm100::globaltimer();          \
+  } while (0)
+#else
+#define TL_DECL
+#define TL_BEGIN(kind) do {} while (0)
+#define TL(k) do {} while (0)
+#endif
+
 constexpr int CONV_THREADS = 192;                                  // warps 2-7
 constexpr int CONV_ITEMS = (NT_MAX * 8 + CONV_THREADS - 1) / CONV_THREADS;
 
@@ -101,7 +129,9 @@ __host__ __device__ __forceinline__ GemmGeom gemm_geom(int Nt, int stages, int b
 __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_constant__ GemmArgs a) {
   extern __shared__ __align__(1024) uint8_t dsm[];
   __shared__ GemmSmem sh;
+  TL_DECL
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  TL_BEGIN(10 + a.epi);
   const int ks = blockIdx.x;            // split-K rank (= cluster rank)
   const int mb = blockIdx.y;            // m-block
   const int nt = blockIdx.z;            // n-tile
@@ -162,6 +192,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         bulk_g2s(dsm + i * gm.slot, wsrc + static_cast<size_t>(i) * gm.a_bytes, gm.a_bytes, &sh.full_a[i]);
       }
       grid_dep_wait();
+      TL(1);
       for (int i = 0; i < pre; ++i) issue_b(i);
       int issued = pre;
       for (int i = pre; i < nk; ++i) {
@@ -206,13 +237,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         mma_commit(&sh.empty[s]);
       }
       mma_commit(&sh.done);
+      TL(2);
     }
-  } else if (norm) {
-    // ---------------- B conversion (warps 2-7): RMSNorm(h)*gamma -> bf16 / e4m3 operand tile
+  } else if (norm || a.rscale) {
+    // ---------------- warps 2-7: per-token rstd; for B_NORM also RMSNorm(h)*gamma -> e4m3 / bf16 tile
     const int st = tid - 64;
-    for (int idx = st; idx < nk * kel; idx += CONV_THREADS) {   // static: before the dependency wait
-      const int k = kc0 * kel + idx;
-      gsm[idx] = k < a.D ? a.gamma[k] : 0.f;                      // padded K: zero
+    if (norm) {
+      for (int idx = st; idx < nk * kel; idx += CONV_THREADS) {   // static: before the dependency wait
+        const int k = kc0 * kel + idx;
+        gsm[idx] = k < a.D ? a.gamma[k] : 0.f;                      // padded K: zero
+      }
     }
     grid_dep_wait();
     for (int r = st; r < Nt; r += CONV_THREADS) {
@@ -234,8 +268,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       sh.rstd[r] = rs;   // padded tokens become zero
     }
     conv_sync();
-    const float inv_sa = a.fp8 ? 1.0f / *a.s_a : 1.0f;
-    for (int i = 0; i < nk; ++i) {
+    const float inv_sa = (norm && a.fp8) ? 1.0f / *a.s_a : 1.0f;
+    for (int i = 0; i < (norm ? nk : 0); ++i) {
       const int s = i % stages;
       if (!mbar_wait(&sh.raw_b[s], (i / stages) & 1, WAIT_LIMIT_NS)) {
         report_timeout(a.status, 0x300);
@@ -293,15 +327,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   if (!mbar_wait(&sh.done, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0x400);
   tc_fence_after();
   __syncthreads();
+  if (tid == 0) TL(3);
   float* red = reinterpret_cast<float*>(dsm);   // [Nt][RED_LD], aliases the drained ring
   if (warp >= 4) {
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    for (int c0 = 0; c0 < Nt; c0 += 16) {
-      float v[16];
-      tmem_ld16(tacc + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
+    for (int c0 = 0; c0 < Nt; c0 += 64) {   // up to 4 loads in flight, one wait
+      uint32_t v[4][16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) red[(c0 + j) * RED_LD + row] = v[j];
+      for (int u = 0; u < 4; ++u)
+        if (c0 + 16 * u < Nt) tmem_ld16_nowait(tacc + (static_cast<uint32_t>(q * 32) << 16) + c0 + 16 * u, v[u]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c0 + 16 * u < Nt)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) red[(c0 + 16 * u + j) * RED_LD + row] = __uint_as_float(v[u][j]);
     }
   }
   tc_fence_before();
@@ -326,15 +367,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   } else {
     __syncthreads();
   }
+  if (tid == 0) TL(4);
 
   const float al = a.alpha ? *a.alpha : 1.0f;
   // split-K sum of one accumulator element over the cluster, in rank order (deterministic)
   auto val = [&](int tok, int row) -> float {
-    if (S == 1) return red[tok * RED_LD + row] * al;
-    float v = 0.f;
+    const float sc = a.rscale ? al * sh.rstd[tok] : al;
+    if (S == 1) return red[tok * RED_LD + row] * sc;
     const float* p = recv + static_cast<size_t>(tok - tok0) * RED_LD + row;
-    for (int s = 0; s < S; ++s) v += p[static_cast<size_t>(s) * gm.TS * RED_LD];
-    return v * al;
+    const size_t stride = static_cast<size_t>(gm.TS) * RED_LD;
+    float v[16];
+#pragma unroll
+    for (int s = 0; s < 16; ++s) v[s] = s < S ? p[s * stride] : 0.f;   // independent loads
+    float acc = 0.f;
+#pragma unroll
+    for (int s = 0; s < 16; ++s) acc += v[s];                          // rank order
+    return acc * sc;
   };
 
   if (a.epi == EPI_RESID) {
@@ -349,6 +397,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         const float hv = *hp + val(tok, row);
         *hp = hv;
         sq = hv * hv;
+        if (a.xb_out)
+          *reinterpret_cast<__nv_bfloat16*>(a.xb_out + btile_offset(t, 2 * f, Nt, a.NKC_x)) =
+              __float2bfloat16_rn(hv * a.xb_gamma[f]);
       }
       for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
       if (lane == 0) sh.ssq_part[sub][(tid >> 5) & 3] = sq;
@@ -405,6 +456,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   }
   if (S > 1 && tid == 0) bulk_wait_read_all();   // peers have read this CTA's slices
   __syncthreads();
+  if (tid == 0) TL(5);
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -466,6 +518,8 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
   __shared__ uint64_t recv_bar;
   __shared__ float w_sh[16][128];   // merge weight of chunk s for owned row rr (C <= 16, rows <= H <= 128)
   __shared__ float inv_den[128];
+  TL_DECL
+  TL_BEGIN(20);
   constexpr int LD = DH + ATT_PAD;       // bf16 row stride in shared memory
   constexpr int OLD = DH + 4;            // fp32 row stride of the partial-O rows
   const int c = blockIdx.x, j = blockIdx.y, b = blockIdx.z;
@@ -502,6 +556,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
   }
   cp_async_commit();
   grid_dep_wait();
+  if (tid == 0) TL(1);
   for (int it = tid; it < a.KC * VPR; it += blockDim.x) {
     const int r = it / VPR, v = it % VPR;
     const int key = key0 + r;
@@ -518,6 +573,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
   cp_async_commit();
   cp_async_wait_all();
   __syncthreads();
+  if (tid == 0) TL(2);
 
   const int gq = lane >> 2, tq = lane & 3;
   const float sl2 = a.scale * 1.4426950408889634f;   // scores in log2 units
@@ -606,6 +662,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
     }
   }
   __syncthreads();   // every warp is done with Q/K/V before the partial rows overwrite them
+  if (tid == 0) TL(3);
   if (active) {
     const int r0 = rg * 16 + gq;
 #pragma unroll
@@ -651,6 +708,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
     src = Obuf;
     rstride = 0;
   }
+  if (tid == 0) TL(4);
   const int nr = r_hi - r_lo;
   if (tid < nr) {
     float M = -INFINITY;
@@ -668,8 +726,13 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
   const float inv_sa = (a.fp8 && a.s_a) ? 1.0f / *a.s_a : 1.0f;
   for (int it = tid; it < nr * DH; it += blockDim.x) {
     const int rr = it / DH, d = it % DH;
+    float v[16];
+#pragma unroll
+    for (int s = 0; s < 16; ++s) v[s] = s < C ? src[(static_cast<size_t>(s) * rstride + rr) * OLD + d] : 0.f;
     float acc = 0.f;
-    for (int s = 0; s < C; ++s) acc += w_sh[s][rr] * src[(static_cast<size_t>(s) * rstride + rr) * OLD + d];
+#pragma unroll
+    for (int s = 0; s < 16; ++s)
+      if (s < C) acc += w_sh[s][rr] * v[s];                                 // rank order
     acc *= inv_den[rr];
     const int t = b * H + r_lo + rr;
     const int kidx = j * DH + d;
@@ -678,6 +741,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
   }
   if (C > 1 && tid == 0) bulk_wait_read_all();   // peers have read this CTA's rows
   __syncthreads();
+  if (tid == 0) TL(5);
 }
 
 // ================================================================== in-proj and final
@@ -687,6 +751,8 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
   __shared__ uint64_t wbar;
   __shared__ float xs[64];
   __shared__ float part[16][4];
+  TL_DECL
+  TL_BEGIN(1);
   __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(dsm);   // [D][A]
   const int t = blockIdx.x, tid = threadIdx.x;
   const uint32_t wbytes = static_cast<uint32_t>(a.D) * a.A * 2;
@@ -705,6 +771,7 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
     base[q] = n < a.D ? a.b_in[n] + a.temb[n] : 0.f;
   }
   grid_dep_wait();
+  if (tid == 0) TL(1);
   if (tid < a.A) xs[tid] = __bfloat162float(__float2bfloat16_rn(a.x[static_cast<size_t>(t) * a.A + tid]));
   __syncthreads();
   mbar_wait(&wbar, 0, WAIT_LIMIT_NS);
@@ -720,6 +787,9 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
       for (int i = 0; i < a.A; ++i) acc = fmaf(__bfloat162float(wr[i]), xs[i], acc);
       hv = acc + base[q];
       a.h[htile_offset(t, n, a.Nt, a.KB)] = hv;
+      if (a.xb)
+        *reinterpret_cast<__nv_bfloat16*>(a.xb + btile_offset(t, 2 * n, a.Nt, a.NKC_x)) =
+            __float2bfloat16_rn(hv * a.xb_gamma[n]);
     }
     float sq = hv * hv;
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
@@ -728,12 +798,15 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
   __syncthreads();
   const int nmb = (a.D + BM - 1) / BM;
   if (tid < nmb) a.ssq[static_cast<size_t>(t) * a.ssq_ld + tid] = ((part[tid][0] + part[tid][1]) + part[tid][2]) + part[tid][3];
+  if (tid == 0) TL(5);
 }
 
 __global__ void __launch_bounds__(256) k_final_tc(const __grid_constant__ FinalArgs a) {
   extern __shared__ __align__(128) uint8_t dsm[];
   __shared__ uint64_t wbar;
   __shared__ float ssq_sh[16];
+  TL_DECL
+  TL_BEGIN(2);
   __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(dsm);                     // [A][D]
   float* hn = reinterpret_cast<float*>(dsm + ((static_cast<size_t>(a.A) * a.D * 2 + 127) & ~size_t(127)));
   const int t = blockIdx.x, tid = threadIdx.x;
@@ -753,6 +826,7 @@ __global__ void __launch_bounds__(256) k_final_tc(const __grid_constant__ FinalA
     gf[q] = k < a.D ? a.g_f[k] : 0.f;
   }
   grid_dep_wait();
+  if (threadIdx.x == 0) TL(1);
   float hv[QMAX];
 #pragma unroll
   for (int q = 0; q < QMAX; ++q) {
@@ -782,6 +856,8 @@ __global__ void __launch_bounds__(256) k_final_tc(const __grid_constant__ FinalA
       a.x_out[xi] = a.x_in[xi] + a.dt * (acc + a.b_out[i]);
     }
   }
+  __syncthreads();
+  if (tid == 0) TL(5);
 }
 
 __global__ void k_to_bf16(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, size_t n) {
@@ -909,3 +985,17 @@ const void* final_kernel_ptr() { return reinterpret_cast<const void*>(k_final_tc
 
 }  // namespace tc
 }  // namespace fr
+
+#ifdef FR_TIMELINE
+extern "C" int fr_debug_timeline(unsigned long long* dev_buf, unsigned cap, unsigned* count_out) {
+  unsigned zero = 0;
+  if (count_out) {
+    cudaDeviceSynchronize();
+    cudaMemcpyFromSymbol(count_out, fr::tc::g_tl_count, sizeof(unsigned));
+  }
+  cudaMemcpyToSymbol(fr::tc::g_tl, &dev_buf, sizeof(dev_buf));
+  cudaMemcpyToSymbol(fr::tc::g_tl_cap, &cap, sizeof(cap));
+  cudaMemcpyToSymbol(fr::tc::g_tl_count, &zero, sizeof(zero));
+  return cudaDeviceSynchronize() == cudaSuccess ? 0 : -4;
+}
+#endif

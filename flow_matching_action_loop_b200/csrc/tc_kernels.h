@@ -74,6 +74,7 @@ struct GemmArgs {
   const float* s_a;        // fp8: activation scale of this projection input (device scalar)
   // B_ROWS: already-quantised activation in the tiled operand layout
   const uint8_t* act;      // [NT][NKC][Nt x 128]
+  int rscale;              // 1: B_ROWS holds bf16(h*gamma); the epilogue scales token t by rstd_t (from ssq)
   // epilogue
   int epi;
   const float* alpha;      // fp8: dequantisation scale s_a * s_w (device scalar), else nullptr
@@ -87,6 +88,9 @@ struct GemmArgs {
   // EPI_RESID
   float* h_out;            // tiled h (+=)
   float* ssq_out;          // [T_pad][ssq_ld], column mb
+  uint8_t* xb_out;         // bf16(h_new * xb_gamma) in the tiled operand layout of the next norm's GEMM, or nullptr
+  const float* xb_gamma;   // gain of the next RMSNorm
+  int NKC_x;
   // EPI_GELU
   uint8_t* u_out;          // tiled [NT][NKC_u][Nt x 128]
   int NKC_u;
@@ -116,6 +120,9 @@ struct InprojArgs {
   const float* temb;           // [D] of this step
   float* h;                    // tiled h
   float* ssq;                  // [T_pad][ssq_ld]
+  uint8_t* xb;                 // bf16(h * gamma1 of layer 0), tiled operand layout, or nullptr
+  const float* xb_gamma;
+  int NKC_x;
   int T, D, A, Nt, KB, ssq_ld;
   int first;                   // x is the caller's x0 (graph node lookup)
 };

@@ -99,6 +99,7 @@ struct TensorPath {
   __nv_bfloat16* qbuf = nullptr; // [B_max][Hq][H][dh]
   uint8_t* obuf = nullptr;       // tiled [NT][NKC_o][Nt x 128] bf16 / e4m3
   uint8_t* ubuf = nullptr;       // tiled [NT][NKC_u][Nt x 128]
+  uint8_t* xbuf = nullptr;       // bf16: tiled bf16(h * gamma) of the next RMSNorm, [NT][NKC_x][Nt x 128]
   float* xs = nullptr;           // [T_max][A] state between steps
   __nv_bfloat16* w_in_bf = nullptr;   // [D][A]
   __nv_bfloat16* w_out_bf = nullptr;  // [A][D]
@@ -139,6 +140,7 @@ size_t carve_all(TensorPath* tp, char* base) {
   tp->qbuf = cv.take<__nv_bfloat16>(static_cast<size_t>(c.B_max) * c.Hq * c.H * c.dh);
   tp->obuf = cv.take<uint8_t>(static_cast<size_t>(tp->tok_alloc) * tp->o.NKC * KCB);
   tp->ubuf = cv.take<uint8_t>(static_cast<size_t>(tp->tok_alloc) * tp->dn.NKC * KCB);
+  tp->xbuf = cv.take<uint8_t>(tp->fp8 ? 0 : static_cast<size_t>(tp->tok_alloc) * tp->qkv.NKC * KCB);
   tp->xs = cv.take<float>(static_cast<size_t>(tp->T_max) * c.A);
   tp->w_in_bf = cv.take<__nv_bfloat16>(static_cast<size_t>(c.D) * c.A);
   tp->w_out_bf = cv.take<__nv_bfloat16>(static_cast<size_t>(c.A) * c.D);
@@ -191,9 +193,10 @@ StepPlan make_plan(const TensorPath* tp, int B, int P) {
   p.T = B * c.H;
   p.NT = ceil_div(p.T, NT_MAX);
   p.Nt = static_cast<int>(align_up(ceil_div(p.T, p.NT), 16));
-  p.qkv = choose_plan(tp->qkv.MB * p.NT, tp->qkv.NKC, p.Nt, B_NORM, tp->fp8, tp->nsm, tp->max_dyn);
+  const int norm_kind = tp->fp8 ? B_NORM : B_ROWS;   // bf16: the producer wrote bf16(h*gamma) already
+  p.qkv = choose_plan(tp->qkv.MB * p.NT, tp->qkv.NKC, p.Nt, norm_kind, tp->fp8, tp->nsm, tp->max_dyn);
   p.o = choose_plan(tp->o.MB * p.NT, tp->o.NKC, p.Nt, B_ROWS, tp->fp8, tp->nsm, tp->max_dyn);
-  p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, B_NORM, tp->fp8, tp->nsm, tp->max_dyn);
+  p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, norm_kind, tp->fp8, tp->nsm, tp->max_dyn);
   p.dn = choose_plan(tp->dn.MB * p.NT, tp->dn.NKC, p.Nt, B_ROWS, tp->fp8, tp->nsm, tp->max_dyn);
   attn_chunks(P + c.H, p.attn_C, p.attn_KC);
   return p;
@@ -266,6 +269,9 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
     ia.Nt = p.Nt;
     ia.KB = tp->KB;
     ia.ssq_ld = tp->ssq_ld;
+    ia.xb = tp->fp8 ? nullptr : tp->xbuf;
+    ia.xb_gamma = tp->gains;   // gamma1 of layer 0
+    ia.NKC_x = tp->qkv.NKC;
     ia.first = (k == 0);
     if ((e = launch_inproj_tc(ia, s, true)) != cudaSuccess) return cuda_fail(e, "in-proj kernel launch");
     for (int l = 0; l < c.L; ++l) {
@@ -277,7 +283,13 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       const float* g2 = g1 + c.D;
       // QKV: RMSNorm fused into the B staging, split + RoPE fused into the epilogue
       GemmArgs q = base_args(tp, p, tp->qkv, p.qkv, l, 0);
-      q.b_kind = B_NORM;
+      if (tp->fp8) {
+        q.b_kind = B_NORM;
+      } else {
+        q.b_kind = B_ROWS;
+        q.act = tp->xbuf;
+        q.rscale = 1;
+      }
       q.h = tp->h;
       q.gamma = g1;
       q.ssq = tp->ssq_a;
@@ -325,10 +337,19 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       og.epi = EPI_RESID;
       og.h_out = tp->h;
       og.ssq_out = tp->ssq_b;
+      og.xb_out = tp->fp8 ? nullptr : tp->xbuf;
+      og.xb_gamma = g2;
+      og.NKC_x = tp->qkv.NKC;
       if ((e = launch_gemm_tc(og, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "o GEMM launch");
       // gate|up with RMSNorm fused, GeLU(gate)*up epilogue
       GemmArgs gg = base_args(tp, p, tp->gu, p.gu, l, gu_off);
-      gg.b_kind = B_NORM;
+      if (tp->fp8) {
+        gg.b_kind = B_NORM;
+      } else {
+        gg.b_kind = B_ROWS;
+        gg.act = tp->xbuf;
+        gg.rscale = 1;
+      }
       gg.h = tp->h;
       gg.gamma = g2;
       gg.ssq = tp->ssq_b;
@@ -348,6 +369,9 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       dg.epi = EPI_RESID;
       dg.h_out = tp->h;
       dg.ssq_out = tp->ssq_a;
+      dg.xb_out = (tp->fp8 || l == c.L - 1) ? nullptr : tp->xbuf;
+      dg.xb_gamma = g1 + 2 * c.D;   // gamma1 of layer l+1
+      dg.NKC_x = tp->qkv.NKC;
       if ((e = launch_gemm_tc(dg, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "down GEMM launch");
     }
     FinalArgs fa{};
