@@ -101,7 +101,6 @@ struct GemmSmem {
   uint64_t raw_b[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
   uint64_t done;
-  uint64_t recv_bar;
   uint32_t tmem_base;
   float rstd[NT_MAX];
   float ssq_part[2][4];
@@ -122,7 +121,7 @@ __host__ __device__ __forceinline__ GemmGeom gemm_geom(int Nt, int stages, int b
   g.ring = g.slot * static_cast<uint32_t>(stages);
   g.gamma_off = g.ring;   // B_NORM: gamma of this CTA's k-range (nk * kel floats)
   g.TS = (Nt + S - 1) / S;
-  g.recv_off = ((static_cast<uint32_t>(Nt) * RED_LD * 4u) + 1023u) & ~1023u;
+  g.recv_off = 0;
   return g;
 }
 
@@ -154,7 +153,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       mbar_init(&sh.empty[s], 1);
     }
     mbar_init(&sh.done, 1);
-    mbar_init(&sh.recv_bar, 1);
     fence_mbar_init();
   }
   uint32_t ncols = 32;
@@ -328,7 +326,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   tc_fence_after();
   __syncthreads();
   if (tid == 0) TL(3);
-  float* red = reinterpret_cast<float*>(dsm);   // [Nt][RED_LD], aliases the drained ring
+  float* red = reinterpret_cast<float*>(dsm);   // S == 1: [Nt][RED_LD], aliases the drained ring
+  float* xs = (S > 1) ? a.xscratch + (static_cast<size_t>(nt) * a.MB + mb) * S * Nt * BM : nullptr;
+  const int t_hi = min(Nt, a.T - n0);           // valid tokens of this n-tile
   if (warp >= 4) {
     const int q = warp & 3;
     const int row = q * 32 + lane;
@@ -342,28 +342,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       for (int u = 0; u < 4; ++u)
         if (c0 + 16 * u < Nt)
 #pragma unroll
-          for (int j = 0; j < 16; ++j) red[(c0 + 16 * u + j) * RED_LD + row] = __uint_as_float(v[u][j]);
+          for (int j = 0; j < 16; ++j) {
+            const int tok = c0 + 16 * u + j;
+            if (S == 1) red[tok * RED_LD + row] = __uint_as_float(v[u][j]);
+            else if (tok < t_hi) xs[(static_cast<size_t>(ks) * Nt + tok) * BM + row] = __uint_as_float(v[u][j]);
+          }
     }
   }
   tc_fence_before();
   const int tok0 = ks * Nt / S, tok1 = (ks + 1) * Nt / S;
-  float* recv = reinterpret_cast<float*>(dsm + gm.recv_off);   // [S][TS][RED_LD]
   if (S > 1) {
-    if (tid == 0) mbar_arrive_expect_tx(&sh.recv_bar, static_cast<uint32_t>(S * (tok1 - tok0) * RED_LD * 4));
-    fence_proxy_async_smem();
-    __syncthreads();
-    cluster_arrive_release();
+    cluster_arrive_release();   // the partial tiles in scratch are visible to the cluster after this barrier
     cluster_wait_acquire();
-    if (tid == 0) {
-      for (int d = 0; d < S; ++d) {
-        const int d0 = d * Nt / S, d1 = (d + 1) * Nt / S;
-        const uint32_t dst = mapa_shared(recv + static_cast<size_t>(ks) * gm.TS * RED_LD, d);
-        bulk_s2cluster(dst, red + static_cast<size_t>(d0) * RED_LD, static_cast<uint32_t>((d1 - d0) * RED_LD * 4),
-                       mapa_shared(&sh.recv_bar, d));
-      }
-      bulk_commit();
-    }
-    if (!mbar_wait(&sh.recv_bar, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0x500);
   } else {
     __syncthreads();
   }
@@ -374,11 +364,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   auto val = [&](int tok, int row) -> float {
     const float sc = a.rscale ? al * sh.rstd[tok] : al;
     if (S == 1) return red[tok * RED_LD + row] * sc;
-    const float* p = recv + static_cast<size_t>(tok - tok0) * RED_LD + row;
-    const size_t stride = static_cast<size_t>(gm.TS) * RED_LD;
+    const float* p = xs + static_cast<size_t>(tok) * BM + row;
+    const size_t stride = static_cast<size_t>(Nt) * BM;
     float v[16];
 #pragma unroll
-    for (int s = 0; s < 16; ++s) v[s] = s < S ? p[s * stride] : 0.f;   // independent loads
+    for (int s = 0; s < 16; ++s) v[s] = s < S ? __ldcg(p + s * stride) : 0.f;   // independent L2 loads
     float acc = 0.f;
 #pragma unroll
     for (int s = 0; s < 16; ++s) acc += v[s];                          // rank order
@@ -454,7 +444,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       }
     }
   }
-  if (S > 1 && tid == 0) bulk_wait_read_all();   // peers have read this CTA's slices
   __syncthreads();
   if (tid == 0) TL(5);
   if (warp == 1) {
@@ -506,16 +495,15 @@ __host__ __device__ __forceinline__ AttnGeom attn_geom(int H, int dh, int KC, in
   g.q_bytes = static_cast<uint32_t>(Hp) * LD * 2;
   g.kv_bytes = 2u * static_cast<uint32_t>(KC) * LD * 2;
   g.rowb = static_cast<uint32_t>(dh + 4) * 4;                  // O row + (max, sum) + pad
-  g.obuf_bytes = static_cast<uint32_t>(Hp) * g.rowb;
-  g.recv_off = (g.obuf_bytes + 127u) & ~127u;                  // Obuf and recv both overlay the dead Q/K/V
+  g.obuf_bytes = static_cast<uint32_t>(Hp) * g.rowb;          // single-chunk case only, overlays Q/K/V
+  g.recv_off = 0;
   g.R = (H + C - 1) / C;
   return g;
 }
 
 template <int DH>
 __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArgs a) {
-  extern __shared__ __align__(128) uint8_t dsm[];
-  __shared__ uint64_t recv_bar;
+  extern __shared__ __align__(1024) uint8_t dsm[];
   __shared__ float w_sh[16][128];   // merge weight of chunk s for owned row rr (C <= 16, rows <= H <= 128)
   __shared__ float inv_den[128];
   TL_DECL
@@ -524,7 +512,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
   constexpr int OLD = DH + 4;            // fp32 row stride of the partial-O rows
   const int c = blockIdx.x, j = blockIdx.y, b = blockIdx.z;
   const int g = (j * a.Hkv) / a.Hq;      // consecutive query-head groups share a KV head
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, Hp = (H + 15) & ~15;
   const int S = a.P + H;
   const int C = a.C;
@@ -534,15 +522,12 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
   __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(dsm);
   __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(dsm + gm.q_bytes);
   __nv_bfloat16* Vs = Ks + a.KC * LD;
-  float* Obuf = reinterpret_cast<float*>(dsm);                  // after compute: [Hp][OLD]
-  float* recv = reinterpret_cast<float*>(dsm + gm.recv_off);    // [C][R][OLD]
+  float* Obuf = reinterpret_cast<float*>(dsm);                  // C == 1, after compute: [Hp][OLD]
+  // C > 1: this CTA's partial rows in the L2 scratch, [C][H][OLD] per (sample, head)
+  float* xs = (C > 1) ? a.xscratch + (static_cast<size_t>(b) * a.Hq + j) * C * H * OLD : nullptr;
   const __nv_bfloat16* kg = a.kv_k + ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max) * DH;
   const __nv_bfloat16* vg = a.kv_v + ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max) * DH;
   constexpr int VPR = DH / 8;            // 16-byte vectors per row
-  if (tid == 0) {
-    mbar_init(&recv_bar, 1);
-    fence_mbar_init();
-  }
   grid_dep_launch();
   // prefix keys/values do not depend on the previous kernel: start their loads first
   for (int it = tid; it < a.KC * VPR; it += blockDim.x) {
@@ -661,64 +646,84 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
       }
     }
   }
-  __syncthreads();   // every warp is done with Q/K/V before the partial rows overwrite them
-  if (tid == 0) TL(3);
-  if (active) {
-    const int r0 = rg * 16 + gq;
-#pragma unroll
-    for (int n = 0; n < DH / 8; ++n) {
-      const int col = n * 8 + tq * 2;
-      Obuf[r0 * OLD + col] = oacc[n][0];
-      Obuf[r0 * OLD + col + 1] = oacc[n][1];
-      Obuf[(r0 + 8) * OLD + col] = oacc[n][2];
-      Obuf[(r0 + 8) * OLD + col + 1] = oacc[n][3];
-    }
-    if (tq == 0) {
-      Obuf[r0 * OLD + DH] = mrow[0];
-      Obuf[r0 * OLD + DH + 1] = lrow[0];
-      Obuf[(r0 + 8) * OLD + DH] = mrow[1];
-      Obuf[(r0 + 8) * OLD + DH + 1] = lrow[1];
-    }
-  }
-  // ---------------- push each owner its rows, merge the rows this CTA owns (rank order)
-  const int r_lo = c * H / C, r_hi = (c + 1) * H / C;
-  const float* src;        // row rr of chunk s at src + (s * rstride + rr) * OLD
-  size_t rstride;
   if (C > 1) {
-    if (tid == 0) mbar_arrive_expect_tx(&recv_bar, static_cast<uint32_t>(C * (r_hi - r_lo)) * gm.rowb);
-    fence_proxy_async_smem();
-    __syncthreads();
+    // partial rows straight from registers to the scratch; then one cluster barrier
+    if (active) {
+      const int r0 = rg * 16 + gq;
+      float* x0 = xs + (static_cast<size_t>(c) * H + r0) * OLD;
+      float* x8 = x0 + 8 * OLD;
+#pragma unroll
+      for (int n = 0; n < DH / 8; ++n) {
+        const int col = n * 8 + tq * 2;
+        if (r0 < H) *reinterpret_cast<float2*>(x0 + col) = make_float2(oacc[n][0], oacc[n][1]);
+        if (r0 + 8 < H) *reinterpret_cast<float2*>(x8 + col) = make_float2(oacc[n][2], oacc[n][3]);
+      }
+      if (tq == 0) {
+        if (r0 < H) *reinterpret_cast<float2*>(x0 + DH) = make_float2(mrow[0], lrow[0]);
+        if (r0 + 8 < H) *reinterpret_cast<float2*>(x8 + DH) = make_float2(mrow[1], lrow[1]);
+      }
+    }
+    if (tid == 0) TL(3);
     cluster_arrive_release();
     cluster_wait_acquire();
-    if (tid == 0) {
-      for (int d = 0; d < C; ++d) {
-        const int d0 = d * H / C, d1 = (d + 1) * H / C;
-        if (d1 > d0)
-          bulk_s2cluster(mapa_shared(recv + static_cast<size_t>(c) * gm.R * OLD, d),
-                         Obuf + static_cast<size_t>(d0) * OLD, static_cast<uint32_t>(d1 - d0) * gm.rowb,
-                         mapa_shared(&recv_bar, d));
+  } else {
+    __syncthreads();   // every warp is done with Q/K/V before the partial rows overwrite them
+    if (tid == 0) TL(3);
+    if (active) {
+      const int r0 = rg * 16 + gq;
+#pragma unroll
+      for (int n = 0; n < DH / 8; ++n) {
+        const int col = n * 8 + tq * 2;
+        Obuf[r0 * OLD + col] = oacc[n][0];
+        Obuf[r0 * OLD + col + 1] = oacc[n][1];
+        Obuf[(r0 + 8) * OLD + col] = oacc[n][2];
+        Obuf[(r0 + 8) * OLD + col + 1] = oacc[n][3];
       }
-      bulk_commit();
+      if (tq == 0) {
+        Obuf[r0 * OLD + DH] = mrow[0];
+        Obuf[r0 * OLD + DH + 1] = lrow[0];
+        Obuf[(r0 + 8) * OLD + DH] = mrow[1];
+        Obuf[(r0 + 8) * OLD + DH + 1] = lrow[1];
+      }
     }
-    mbar_wait(&recv_bar, 0, WAIT_LIMIT_NS);
-    src = recv;
-    rstride = gm.R;
-  } else {   // a single key chunk: no cluster, the CTA's own rows are final
     __syncthreads();
-    src = Obuf;
-    rstride = 0;
   }
+  // ---------------- merge the rows this CTA owns over the key chunks, in rank order
+  const int r_lo = c * H / C, r_hi = (c + 1) * H / C;
+  // row rr (relative to r_lo) of chunk s: src + (s * sstride + r_lo + rr) * OLD
+  const float* src = (C > 1) ? xs : Obuf;
+  const size_t sstride = (C > 1) ? static_cast<size_t>(H) : 0;
+  // the scratch is read through L2 only (written by other CTAs); the single-chunk rows are in shared memory
+  auto ld1 = [&](const float* p) -> float { return C > 1 ? __ldcg(p) : *p; };
+  auto ld2 = [&](const float* p) -> float2 {
+    return C > 1 ? __ldcg(reinterpret_cast<const float2*>(p)) : *reinterpret_cast<const float2*>(p);
+  };
   if (tid == 0) TL(4);
   const int nr = r_hi - r_lo;
   if (tid < nr) {
+    float mv[16], lv[16];
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+      if (s < C) {
+        const float2 ml = ld2(src + (s * sstride + r_lo + tid) * OLD + DH);
+        mv[s] = ml.x;
+        lv[s] = ml.y;
+      } else {
+        mv[s] = -INFINITY;
+        lv[s] = 0.f;
+      }
+    }
     float M = -INFINITY;
-    for (int s = 0; s < C; ++s) M = fmaxf(M, src[(static_cast<size_t>(s) * rstride + tid) * OLD + DH]);
+#pragma unroll
+    for (int s = 0; s < 16; ++s) M = fmaxf(M, mv[s]);
     float den = 0.f;
-    for (int s = 0; s < C; ++s) {
-      const float* row = src + (static_cast<size_t>(s) * rstride + tid) * OLD;
-      const float e = exp2f(row[DH] - M);
-      w_sh[s][tid] = e;
-      den += e * row[DH + 1];
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+      if (s < C) {
+        const float e = exp2f(mv[s] - M);
+        w_sh[s][tid] = e;
+        den += e * lv[s];
+      }
     }
     inv_den[tid] = 1.0f / den;
   }
@@ -728,7 +733,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
     const int rr = it / DH, d = it % DH;
     float v[16];
 #pragma unroll
-    for (int s = 0; s < 16; ++s) v[s] = s < C ? src[(static_cast<size_t>(s) * rstride + rr) * OLD + d] : 0.f;
+    for (int s = 0; s < 16; ++s) v[s] = s < C ? ld1(src + (s * sstride + r_lo + rr) * OLD + d) : 0.f;
     float acc = 0.f;
 #pragma unroll
     for (int s = 0; s < 16; ++s)
@@ -739,7 +744,6 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
     if (a.fp8) a.o[btile_offset(t, kidx, a.Nt, a.NKC_o)] = to_e4m3(acc * inv_sa);
     else *reinterpret_cast<__nv_bfloat16*>(a.o + btile_offset(t, 2 * kidx, a.Nt, a.NKC_o)) = __float2bfloat16_rn(acc);
   }
-  if (C > 1 && tid == 0) bulk_wait_read_all();   // peers have read this CTA's rows
   __syncthreads();
   if (tid == 0) TL(5);
 }
@@ -747,7 +751,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
 // ================================================================== in-proj and final
 
 __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ InprojArgs a) {
-  extern __shared__ __align__(128) uint8_t dsm[];
+  extern __shared__ __align__(1024) uint8_t dsm[];
   __shared__ uint64_t wbar;
   __shared__ float xs[64];
   __shared__ float part[16][4];
@@ -802,7 +806,7 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
 }
 
 __global__ void __launch_bounds__(256) k_final_tc(const __grid_constant__ FinalArgs a) {
-  extern __shared__ __align__(128) uint8_t dsm[];
+  extern __shared__ __align__(1024) uint8_t dsm[];
   __shared__ uint64_t wbar;
   __shared__ float ssq_sh[16];
   TL_DECL
@@ -900,15 +904,22 @@ size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk) {
   const GemmGeom g = gemm_geom(Nt, stages, b_kind, fp8, S, nk);
   const size_t kel = fp8 ? KCB : KCB / 2;
   const size_t main = g.ring + (b_kind == B_NORM ? static_cast<size_t>(nk) * kel * 4 : 0);
-  const size_t red = static_cast<size_t>(Nt) * RED_LD * 4;
-  const size_t epi = S > 1 ? g.recv_off + static_cast<size_t>(S) * g.TS * RED_LD * 4 : red;
+  const size_t epi = S > 1 ? 0 : static_cast<size_t>(Nt) * RED_LD * 4;
   return main > epi ? main : epi;
+}
+
+size_t gemm_scratch_bytes(int NT, int MB, int S, int Nt) {
+  return S > 1 ? static_cast<size_t>(NT) * MB * S * Nt * BM * 4 : 0;
+}
+
+size_t attn_scratch_bytes(int B, int Hq, int C, int H, int dh) {
+  return C > 1 ? static_cast<size_t>(B) * Hq * C * H * (dh + 4) * 4 : 0;
 }
 
 size_t attn_smem_bytes(int H, int dh, int KC, int C) {
   const AttnGeom g = attn_geom(H, dh, KC, C);
   const size_t compute = static_cast<size_t>(g.q_bytes) + g.kv_bytes;
-  const size_t merge = C > 1 ? g.recv_off + static_cast<size_t>(C) * g.R * g.rowb : g.obuf_bytes;
+  const size_t merge = C > 1 ? 0 : g.obuf_bytes;
   return compute > merge ? compute : merge;
 }
 

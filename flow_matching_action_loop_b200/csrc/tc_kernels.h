@@ -5,10 +5,12 @@
 //   inproj -> per layer { qkv GEMM -> attention -> o GEMM -> gate|up GEMM -> down GEMM } -> final
 // Every kernel fetches what does not depend on its predecessor (weights, prefix
 // keys/values) before it waits on it, so those loads overlap the previous kernel.
-// Loads on the dependent side are asynchronous bulk copies issued up front; split-K
+// Loads on the dependent side are asynchronous bulk copies issued up front.  Split-K
 // partial tiles and attention key-chunk partials are exchanged inside a thread-block
-// cluster by bulk copies between shared memories and summed in rank order
-// (deterministic).
+// cluster through an L2-resident scratch buffer (stored straight from registers, one
+// cluster barrier with release/acquire semantics, then read by their owner CTA) and
+// summed in rank order (deterministic).  On this part the L2 moves these partials
+// several times faster than distributed shared memory does.
 //
 // Activation layouts (all per call, n-tile of Nt tokens, nt = t / Nt, r = t % Nt):
 //   h (residual, fp32)   [NT][D/64][Nt][64]          -- a 64-feature chunk of an n-tile is contiguous
@@ -96,6 +98,8 @@ struct GemmArgs {
   int NKC_u;
   const float* s_a_out;    // fp8: scale of the down-projection input
   int F;
+  // split-K exchange (S > 1): fp32 partial tiles [NT][MB][S][Nt][128], L2-resident scratch
+  float* xscratch;
   unsigned* status;
 };
 
@@ -111,6 +115,7 @@ struct AttnArgs {
   int C;                       // key chunks = cluster size
   int KC;                      // keys per chunk (multiple of ATTN_SUBK)
   float scale;                 // 1/sqrt(dh)
+  float* xscratch;             // C > 1: partial rows [B][Hq][C][H][dh + 4] (O, max, sum), L2-resident scratch
 };
 
 struct InprojArgs {
@@ -149,6 +154,8 @@ cudaError_t launch_inproj_tc(const InprojArgs& a, cudaStream_t s, bool pdl);
 cudaError_t launch_final_tc(const FinalArgs& a, cudaStream_t s, bool pdl);
 cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s);
 size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk);
+size_t gemm_scratch_bytes(int NT, int MB, int S, int Nt);
+size_t attn_scratch_bytes(int B, int Hq, int C, int H, int dh);
 size_t attn_smem_bytes(int H, int dh, int KC, int C);
 const void* inproj_kernel_ptr();
 const void* final_kernel_ptr();

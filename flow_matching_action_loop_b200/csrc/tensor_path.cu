@@ -100,6 +100,8 @@ struct TensorPath {
   uint8_t* obuf = nullptr;       // tiled [NT][NKC_o][Nt x 128] bf16 / e4m3
   uint8_t* ubuf = nullptr;       // tiled [NT][NKC_u][Nt x 128]
   uint8_t* xbuf = nullptr;       // bf16: tiled bf16(h * gamma) of the next RMSNorm, [NT][NKC_x][Nt x 128]
+  float* xscratch = nullptr;     // split-K / key-chunk exchange scratch (L2-resident), shared by all kernels
+  size_t xscratch_bytes = 0;
   float* xs = nullptr;           // [T_max][A] state between steps
   __nv_bfloat16* w_in_bf = nullptr;   // [D][A]
   __nv_bfloat16* w_out_bf = nullptr;  // [A][D]
@@ -142,6 +144,7 @@ size_t carve_all(TensorPath* tp, char* base) {
   tp->ubuf = cv.take<uint8_t>(static_cast<size_t>(tp->tok_alloc) * tp->dn.NKC * KCB);
   tp->xbuf = cv.take<uint8_t>(tp->fp8 ? 0 : static_cast<size_t>(tp->tok_alloc) * tp->qkv.NKC * KCB);
   tp->xs = cv.take<float>(static_cast<size_t>(tp->T_max) * c.A);
+  tp->xscratch = cv.take<float>(tp->xscratch_bytes / sizeof(float) + 64);
   tp->w_in_bf = cv.take<__nv_bfloat16>(static_cast<size_t>(c.D) * c.A);
   tp->w_out_bf = cv.take<__nv_bfloat16>(static_cast<size_t>(c.A) * c.D);
   return align_up(cv.off, 1024);
@@ -163,19 +166,30 @@ void init_sizes(TensorPath* tp, const fr_config& c) {
   tp->layer_bytes = tp->qkv.bytes + tp->o.bytes + tp->gu.bytes + tp->dn.bytes;
 }
 
-// Split-K / ring choice for one projection: a small cost model over S (cluster size).
+// Split-K / ring choice for one projection.  Batch-1-like tiles (Nt <= 64) are latency-bound:
+// at most one CTA per SM (so the next kernel's CTAs can become resident and prefetch their
+// weights next to it) and at most ~120 KB of shared memory; the cost counts waves, the split-K
+// exchange, and weight chunks that must stream after the dependency wait.  Wider tiles are
+// throughput-bound: no split-K unless the tiles leave most SMs idle.
 GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int nsm, int max_dyn) {
   GemmPlan best;
+  if (Nt > 64) {
+    best.S = (tiles * 2 <= nsm && NKC >= 2) ? 2 : 1;
+    const int chunks = ceil_div(NKC, best.S);
+    best.stages = std::min(chunks, MAX_STAGES);
+    while (best.stages > 1 && gemm_smem_bytes(Nt, best.stages, b_kind, fp8, best.S, chunks) > static_cast<size_t>(max_dyn))
+      --best.stages;
+    return best;
+  }
+  const size_t cap = std::min<size_t>(static_cast<size_t>(max_dyn), 120 * 1024);
   double best_cost = 1e30;
   for (int S = 1; S <= 16 && S <= NKC; ++S) {
     const int chunks = ceil_div(NKC, S);
     int stages = std::min(chunks, MAX_STAGES);
-    while (stages > 1 && gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks) > static_cast<size_t>(max_dyn)) --stages;
-    const size_t smem = gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks);
-    if (smem > static_cast<size_t>(max_dyn)) continue;
-    const int per_sm = std::max(1, std::min(2, static_cast<int>((228 * 1024) / (smem + 4096))));
-    const int waves = ceil_div(tiles * S, nsm * per_sm);
-    const double cost = waves * (chunks + 0.1 * S);
+    while (stages > 1 && gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks) > cap) --stages;
+    if (gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks) > static_cast<size_t>(max_dyn)) continue;
+    const int waves = ceil_div(tiles * S, nsm);
+    const double cost = waves * (1.0 + (S > 1 ? 1.0 : 0.0) + 0.3 * (chunks - stages) + 0.05 * chunks);
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best.S = S;
@@ -244,6 +258,7 @@ GemmArgs base_args(const TensorPath* tp, const StepPlan& p, const ProjLayout& L,
   a.eps = c.eps;
   a.ssq_ld = tp->ssq_ld;
   a.ssq_parts = tp->MBd;
+  a.xscratch = tp->xscratch;
   a.status = tp->tb.status;
   return a;
 }
@@ -328,6 +343,7 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       at.C = p.attn_C;
       at.KC = p.attn_KC;
       at.scale = 1.0f / std::sqrt(static_cast<float>(c.dh));
+      at.xscratch = tp->xscratch;
       if ((e = launch_attention_tc(at, p.B, s, true)) != cudaSuccess) return cuda_fail(e, "attention launch");
       // O projection + residual (+ sum of squares for the pre-MLP norm)
       GemmArgs og = base_args(tp, p, tp->o, p.o, l, o_off);
@@ -489,15 +505,46 @@ const char* tensor_path_limits() {
          "D % 16 == 0, D <= 2048, A <= 64, attention chunk fits shared memory";
 }
 
+// Exchange scratch needed by any batch size up to B_max and any prefix length up to P_max.
+size_t exchange_scratch_bytes(TensorPath* tp) {
+  const fr_config& c = tp->c;
+  size_t mx = 0;
+  for (int B = 1; B <= c.B_max; ++B) {
+    const StepPlan p = make_plan(tp, B, c.P_max);
+    const ProjLayout* L[4] = {&tp->qkv, &tp->o, &tp->gu, &tp->dn};
+    const GemmPlan* G[4] = {&p.qkv, &p.o, &p.gu, &p.dn};
+    for (int i = 0; i < 4; ++i) mx = std::max(mx, gemm_scratch_bytes(p.NT, L[i]->MB, G[i]->S, p.Nt));
+  }
+  int cmax = 1;
+  for (int P = 1; P <= c.P_max; ++P) {   // key chunks of every prefix length the handle accepts
+    int C = 1, KC = 64;
+    attn_chunks(P + c.H, C, KC);
+    cmax = std::max(cmax, C);
+  }
+  mx = std::max(mx, attn_scratch_bytes(c.B_max, c.Hq, cmax, c.H, c.dh));
+  return mx;
+}
+
+void device_params(TensorPath* tp) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&tp->nsm, cudaDevAttrMultiProcessorCount, dev);
+  tc_kernels_init();
+  tp->max_dyn = max_dynamic_smem();
+}
+
 size_t tensor_path_bytes(const fr_config& c) {
   TensorPath tmp;
   init_sizes(&tmp, c);
+  device_params(&tmp);
+  tmp.xscratch_bytes = exchange_scratch_bytes(&tmp);
   return carve_all(&tmp, nullptr);
 }
 
 int tensor_path_create(const fr_config& c, const TensorPathBuffers& b, TensorPath** out) {
   TensorPath* tp = new TensorPath();
   init_sizes(tp, c);
+  device_params(tp);
+  tp->xscratch_bytes = exchange_scratch_bytes(tp);
   tp->tb = b;
   if (c.dtype != FR_DTYPE_FP8) {
     tp->tb.alpha = nullptr;
