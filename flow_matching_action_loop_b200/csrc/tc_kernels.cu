@@ -19,6 +19,7 @@
 //   split over keys).  Warp-level bf16 MMA computes scores and P*V with an online softmax
 //   over 64-key sub-chunks; the chunks' (O, max, sum) rows are pushed to their owner CTA by
 //   bulk copies and merged with log-sum-exp weights in rank order.
+#include <algorithm>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <math.h>
@@ -101,6 +102,8 @@ struct GemmSmem {
   uint64_t raw_b[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
   uint64_t done;
+  uint64_t hbar;      // residual rows of this CTA's tokens (EPI_RESID, S > 1)
+  uint64_t xbar;      // split-K slices of this CTA's tokens (S > 1)
   uint32_t tmem_base;
   float rstd[NT_MAX];
   float ssq_part[2][4];
@@ -121,7 +124,11 @@ __host__ __device__ __forceinline__ GemmGeom gemm_geom(int Nt, int stages, int b
   g.ring = g.slot * static_cast<uint32_t>(stages);
   g.gamma_off = g.ring;   // B_NORM: gamma of this CTA's k-range (nk * kel floats)
   g.TS = (Nt + S - 1) / S;
-  g.recv_off = 0;
+  // S > 1: residual rows (2 x TS x 64 floats) live past the ring and the gamma slice, because
+  // they land while the ring is still in use; the split-K slices (S x TS x 128 floats) land
+  // after the MMAs and overlay the ring.
+  const uint32_t kel = fp8 ? KCB : KCB / 2;
+  g.recv_off = (g.ring + (b_kind == B_NORM ? static_cast<uint32_t>(nk) * kel * 4u : 0u) + 1023u) & ~1023u;
   return g;
 }
 
@@ -153,6 +160,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       mbar_init(&sh.empty[s], 1);
     }
     mbar_init(&sh.done, 1);
+    mbar_init(&sh.hbar, 1);
+    mbar_init(&sh.xbar, 1);
     fence_mbar_init();
   }
   uint32_t ncols = 32;
@@ -192,6 +201,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       grid_dep_wait();
       TL(1);
       for (int i = 0; i < pre; ++i) issue_b(i);
+      if (S > 1 && a.epi == EPI_RESID) {   // residual rows of this CTA's tokens, for the epilogue
+        const int r0 = ks * Nt / S, r1 = (ks + 1) * Nt / S;
+        const uint32_t rb = static_cast<uint32_t>(r1 - r0) * 256u;
+        float* hst = reinterpret_cast<float*>(dsm + gm.recv_off);
+        mbar_arrive_expect_tx(&sh.hbar, 2 * rb);
+        for (int u = 0; u < 2; ++u)
+          bulk_g2s(hst + static_cast<size_t>(u) * gm.TS * 64,
+                   a.h_out + ((static_cast<size_t>(nt) * a.KB + 2 * mb + u) * Nt + r0) * 64, rb, &sh.hbar);
+      }
       int issued = pre;
       for (int i = pre; i < nk; ++i) {
         const int s = i % stages;
@@ -351,9 +369,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   }
   tc_fence_before();
   const int tok0 = ks * Nt / S, tok1 = (ks + 1) * Nt / S;
+  float* xst = reinterpret_cast<float*>(dsm);   // S > 1: [S][TS][128] slices of this CTA's tokens
   if (S > 1) {
     cluster_arrive_release();   // the partial tiles in scratch are visible to the cluster after this barrier
     cluster_wait_acquire();
+    if (tid == 0) {             // one round trip: every slice of this CTA's tokens by bulk copy
+      const uint32_t sb = static_cast<uint32_t>(tok1 - tok0) * BM * 4u;
+      mbar_arrive_expect_tx(&sh.xbar, S * sb);
+      for (int s2 = 0; s2 < S; ++s2)
+        bulk_g2s(xst + static_cast<size_t>(s2) * gm.TS * BM, xs + (static_cast<size_t>(s2) * Nt + tok0) * BM, sb,
+                 &sh.xbar);
+    }
+    if (!mbar_wait(&sh.xbar, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0x500);
   } else {
     __syncthreads();
   }
@@ -364,11 +391,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   auto val = [&](int tok, int row) -> float {
     const float sc = a.rscale ? al * sh.rstd[tok] : al;
     if (S == 1) return red[tok * RED_LD + row] * sc;
-    const float* p = xs + static_cast<size_t>(tok) * BM + row;
-    const size_t stride = static_cast<size_t>(Nt) * BM;
+    const float* p = xst + static_cast<size_t>(tok - tok0) * BM + row;
+    const size_t stride = static_cast<size_t>(gm.TS) * BM;
     float v[16];
 #pragma unroll
-    for (int s = 0; s < 16; ++s) v[s] = s < S ? __ldcg(p + s * stride) : 0.f;   // independent L2 loads
+    for (int s = 0; s < 16; ++s) v[s] = s < S ? p[s * stride] : 0.f;
     float acc = 0.f;
 #pragma unroll
     for (int s = 0; s < 16; ++s) acc += v[s];                          // rank order
@@ -378,13 +405,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   if (a.epi == EPI_RESID) {
     const int row = tid & 127, sub = tid >> 7;
     const int f = mb * BM + row;
+    const float* hst = reinterpret_cast<const float*>(dsm + gm.recv_off);   // [2][TS][64]
+    if (S > 1 && !mbar_wait(&sh.hbar, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0x600);
     for (int tb = tok0; tb < tok1; tb += 2) {
       const int tok = tb + sub;
       const int t = n0 + tok;
       float sq = 0.f;
       if (tok < tok1 && t < a.T && f < a.Nout) {
         float* hp = a.h_out + htile_offset(t, f, Nt, a.KB);
-        const float hv = *hp + val(tok, row);
+        const float hold = (S > 1) ? hst[((row >> 6) * gm.TS + (tok - tok0)) * 64 + (row & 63)] : *hp;
+        const float hv = hold + val(tok, row);
         *hp = hv;
         sq = hv * hv;
         if (a.xb_out)
@@ -504,6 +534,7 @@ __host__ __device__ __forceinline__ AttnGeom attn_geom(int H, int dh, int KC, in
 template <int DH>
 __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t dsm[];
+  __shared__ uint64_t stage_bar;
   __shared__ float w_sh[16][128];   // merge weight of chunk s for owned row rr (C <= 16, rows <= H <= 128)
   __shared__ float inv_den[128];
   TL_DECL
@@ -528,6 +559,10 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
   const __nv_bfloat16* kg = a.kv_k + ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max) * DH;
   const __nv_bfloat16* vg = a.kv_v + ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max) * DH;
   constexpr int VPR = DH / 8;            // 16-byte vectors per row
+  if (tid == 0) {
+    mbar_init(&stage_bar, 1);
+    fence_mbar_init();
+  }
   grid_dep_launch();
   // prefix keys/values do not depend on the previous kernel: start their loads first
   for (int it = tid; it < a.KC * VPR; it += blockDim.x) {
@@ -664,6 +699,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
       }
     }
     if (tid == 0) TL(3);
+    __syncthreads();   // Q/K/V are dead in every warp: the slices below overlay them
     cluster_arrive_release();
     cluster_wait_acquire();
   } else {
@@ -691,13 +727,25 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
   // ---------------- merge the rows this CTA owns over the key chunks, in rank order
   const int r_lo = c * H / C, r_hi = (c + 1) * H / C;
   // row rr (relative to r_lo) of chunk s: src + (s * sstride + r_lo + rr) * OLD
-  const float* src = (C > 1) ? xs : Obuf;
-  const size_t sstride = (C > 1) ? static_cast<size_t>(H) : 0;
-  // the scratch is read through L2 only (written by other CTAs); the single-chunk rows are in shared memory
-  auto ld1 = [&](const float* p) -> float { return C > 1 ? __ldcg(p) : *p; };
-  auto ld2 = [&](const float* p) -> float2 {
-    return C > 1 ? __ldcg(reinterpret_cast<const float2*>(p)) : *reinterpret_cast<const float2*>(p);
-  };
+  // C > 1: one round trip brings this CTA's rows of every chunk into shared memory, [C][R][OLD]
+  float* stage = reinterpret_cast<float*>(dsm);
+  if (C > 1) {
+    if (tid == 0) {
+      const uint32_t sb = static_cast<uint32_t>(r_hi - r_lo) * gm.rowb;
+      mbar_arrive_expect_tx(&stage_bar, C * sb);
+      if (sb)
+        for (int s2 = 0; s2 < C; ++s2)
+          bulk_g2s(stage + static_cast<size_t>(s2) * gm.R * OLD, xs + (static_cast<size_t>(s2) * H + r_lo) * OLD, sb,
+                   &stage_bar);
+    }
+    mbar_wait(&stage_bar, 0, WAIT_LIMIT_NS);
+  }
+  // row rr of chunk s: src + (s * sstride + roff + rr) * OLD
+  const float* src = (C > 1) ? stage : Obuf;
+  const size_t sstride = (C > 1) ? static_cast<size_t>(gm.R) : 0;
+  const int roff = (C > 1) ? 0 : r_lo;
+  auto ld1 = [&](const float* p) -> float { return *p; };
+  auto ld2 = [&](const float* p) -> float2 { return *reinterpret_cast<const float2*>(p); };
   if (tid == 0) TL(4);
   const int nr = r_hi - r_lo;
   if (tid < nr) {
@@ -705,7 +753,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
 #pragma unroll
     for (int s = 0; s < 16; ++s) {
       if (s < C) {
-        const float2 ml = ld2(src + (s * sstride + r_lo + tid) * OLD + DH);
+        const float2 ml = ld2(src + (s * sstride + roff + tid) * OLD + DH);
         mv[s] = ml.x;
         lv[s] = ml.y;
       } else {
@@ -733,7 +781,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
     const int rr = it / DH, d = it % DH;
     float v[16];
 #pragma unroll
-    for (int s = 0; s < 16; ++s) v[s] = s < C ? ld1(src + (s * sstride + r_lo + rr) * OLD + d) : 0.f;
+    for (int s = 0; s < 16; ++s) v[s] = s < C ? ld1(src + (s * sstride + roff + rr) * OLD + d) : 0.f;
     float acc = 0.f;
 #pragma unroll
     for (int s = 0; s < 16; ++s)
@@ -904,7 +952,9 @@ size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk) {
   const GemmGeom g = gemm_geom(Nt, stages, b_kind, fp8, S, nk);
   const size_t kel = fp8 ? KCB : KCB / 2;
   const size_t main = g.ring + (b_kind == B_NORM ? static_cast<size_t>(nk) * kel * 4 : 0);
-  const size_t epi = S > 1 ? 0 : static_cast<size_t>(Nt) * RED_LD * 4;
+  const size_t TS = (Nt + S - 1) / S;
+  const size_t epi = S > 1 ? std::max<size_t>(static_cast<size_t>(S) * TS * BM * 4, g.recv_off + 2 * TS * 64 * 4)
+                           : static_cast<size_t>(Nt) * RED_LD * 4;
   return main > epi ? main : epi;
 }
 
@@ -919,7 +969,7 @@ size_t attn_scratch_bytes(int B, int Hq, int C, int H, int dh) {
 size_t attn_smem_bytes(int H, int dh, int KC, int C) {
   const AttnGeom g = attn_geom(H, dh, KC, C);
   const size_t compute = static_cast<size_t>(g.q_bytes) + g.kv_bytes;
-  const size_t merge = C > 1 ? 0 : g.obuf_bytes;
+  const size_t merge = C > 1 ? static_cast<size_t>(C) * g.R * g.rowb : g.obuf_bytes;
   return compute > merge ? compute : merge;
 }
 
