@@ -90,6 +90,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fr_path_name": (c_char_p, [H]),
         "fr_launches_per_call": (c_int, [H, c_int]),
         "fr_rope_tables": (c_int, [c_int, c_int, ctypes.c_double, _FP, _FP]),
+        "fr_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
+                                 c_void_p, ctypes.c_size_t, c_void_p]),
+        "fr_attention_scratch_bytes": (ctypes.c_size_t, [c_int, c_int, c_int, c_int, c_int]),
         "fr_round_bf16": (None, [_FP, ctypes.POINTER(ctypes.c_uint16), ctypes.c_size_t]),
         "fr_quantize_e4m3": (None, [_FP, ctypes.POINTER(ctypes.c_uint8), ctypes.c_size_t, ctypes.c_double]),
     }
@@ -207,6 +210,16 @@ def fr_path_name(h) -> str:
 
 def fr_launches_per_call(h, B: int) -> int:
     return load_library().fr_launches_per_call(h, B)
+
+
+def fr_attention(q: int, k: int, v: int, o: int, B: int, Hq: int, Hkv: int, H: int, S_keys: int, dh: int,
+                 scratch: int = 0, scratch_bytes: int = 0, stream: int = 0) -> None:
+    _check(load_library().fr_attention(q, k, v, o, B, Hq, Hkv, H, S_keys, dh, scratch, scratch_bytes, stream),
+           "fr_attention")
+
+
+def fr_attention_scratch_bytes(B: int, Hq: int, H: int, S_keys: int, dh: int) -> int:
+    return load_library().fr_attention_scratch_bytes(B, Hq, H, S_keys, dh)
 
 
 def fr_rope_tables(n_pos: int, dh: int, theta: float):

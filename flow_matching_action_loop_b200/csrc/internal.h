@@ -74,4 +74,7 @@ void launch_final(const float* h, const float* g_f, const float* w_out, const fl
 
 enum WType : int { W_F32 = 0, W_BF16 = 1, W_E4M3 = 2 };
 
+// Kernel attributes of the tensor-core kernels, set once per device (ops.cu).
+cudaError_t ensure_tc_kernels(int* dev_out);
+
 }  // namespace fr

@@ -1,0 +1,109 @@
+// Kernel-library entry points: one op of the loop on caller-owned device buffers.
+//
+// FlashRT walkthrough, component 8: the kernel library exposes its ops through a stable
+// ABI, separate from the per-model pipeline.  Here that is the split-KV grouped-query
+// attention of the action tokens over [prefix; actions] (component 5: the Pi0.5 decoder
+// attention site), the same kernel fr_denoise runs for every layer.
+#include <cmath>
+#include <mutex>
+
+#include "internal.h"
+#include "tc_kernels.h"
+
+namespace fr {
+namespace {
+
+constexpr int MAX_DEVICES = 64;
+std::once_flag g_init_once[MAX_DEVICES];
+cudaError_t g_init_err[MAX_DEVICES];
+
+}  // namespace
+
+// Kernel attributes are per device; set them once on each device the ops run on.
+cudaError_t ensure_tc_kernels(int* dev_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
+  std::call_once(g_init_once[dev], [dev] { g_init_err[dev] = tc::tc_kernels_init(); });
+  if (dev_out) *dev_out = dev;
+  return g_init_err[dev];
+}
+
+namespace {
+
+}  // namespace
+
+int check_attention(const void* q, const void* k, const void* v, const void* o, int B, int Hq, int Hkv, int H,
+                    int S_keys, int dh) {
+  if (!q || !k || !v || !o) {
+    set_error("fr_attention: NULL tensor");
+    return FR_ERR_ARG;
+  }
+  if (B < 1 || Hq < 1 || Hkv < 1 || H < 1 || S_keys < 1) {
+    set_error("fr_attention: sizes must be positive");
+    return FR_ERR_ARG;
+  }
+  if ((dh != 64 && dh != 128 && dh != 256) || Hq % Hkv != 0 || H > 128 || H > S_keys || S_keys > 32768) {
+    set_error("fr_attention: needs dh in {64,128,256}, Hq %% Hkv == 0, H <= 128, H <= S_keys <= 32768");
+    return FR_ERR_UNSUPPORTED;
+  }
+  int C = 1, KC = 64;
+  tc::attn_chunks(S_keys, C, KC);
+  if (tc::attn_smem_bytes(H, dh, KC, C) > 200 * 1024) {
+    set_error("fr_attention: a key chunk of %d keys does not fit shared memory", KC);
+    return FR_ERR_UNSUPPORTED;
+  }
+  return FR_OK;
+}
+
+tc::AttnArgs attention_args(const void* q, const void* k, const void* v, void* o, int Hq, int Hkv, int H,
+                            int S_keys, int dh, float* scratch) {
+  tc::AttnArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.kv_k = static_cast<const __nv_bfloat16*>(k);
+  a.kv_v = static_cast<const __nv_bfloat16*>(v);
+  a.o = static_cast<uint8_t*>(o);
+  a.o_rowmajor = 1;
+  a.fp8 = 0;
+  a.H = H;
+  a.P = S_keys - H;
+  a.S_max = S_keys;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.dh = dh;
+  tc::attn_chunks(S_keys, a.C, a.KC);
+  a.scale = 1.0f / std::sqrt(static_cast<float>(dh));
+  a.xscratch = scratch;
+  return a;
+}
+
+}  // namespace fr
+
+using namespace fr;
+
+extern "C" {
+
+size_t fr_attention_scratch_bytes(int B, int Hq, int H, int S_keys, int dh) {
+  if (B < 1 || Hq < 1 || H < 1 || S_keys < 1 || dh < 1) return 0;
+  int C = 1, KC = 64;
+  tc::attn_chunks(S_keys, C, KC);
+  return tc::attn_scratch_bytes(B, Hq, C, H, dh);
+}
+
+int fr_attention(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int H, int S_keys,
+                 int dh, void* scratch, size_t scratch_bytes, fr_stream_t stream) {
+  int rc = check_attention(q, k, v, o, B, Hq, Hkv, H, S_keys, dh);
+  if (rc) return rc;
+  const size_t need = fr_attention_scratch_bytes(B, Hq, H, S_keys, dh);
+  if (need > 0 && (!scratch || scratch_bytes < need)) {
+    set_error("fr_attention: scratch of %zu bytes needed, %zu given", need, scratch ? scratch_bytes : size_t(0));
+    return FR_ERR_SHAPE;
+  }
+  FR_CUDA(ensure_tc_kernels(nullptr));
+  const tc::AttnArgs a = attention_args(q, k, v, o, Hq, Hkv, H, S_keys, dh, static_cast<float*>(scratch));
+  FR_CUDA(tc::launch_attention_tc(a, B, reinterpret_cast<cudaStream_t>(stream), false));
+  return FR_OK;
+}
+
+}  // extern "C"

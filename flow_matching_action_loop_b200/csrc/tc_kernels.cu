@@ -124,11 +124,13 @@ __host__ __device__ __forceinline__ GemmGeom gemm_geom(int Nt, int stages, int b
   g.ring = g.slot * static_cast<uint32_t>(stages);
   g.gamma_off = g.ring;   // B_NORM: gamma of this CTA's k-range (nk * kel floats)
   g.TS = (Nt + S - 1) / S;
-  // S > 1: residual rows (2 x TS x 64 floats) live past the ring and the gamma slice, because
-  // they land while the ring is still in use; the split-K slices (S x TS x 128 floats) land
-  // after the MMAs and overlay the ring.
+  // S > 1: residual rows (2 x TS x 64 floats) live past the ring, the gamma slice and the
+  // split-K slices: they land while the ring is still in use and are read after the split-K
+  // slices (S x TS x 128 floats, overlaying the ring from offset 0) have landed.
   const uint32_t kel = fp8 ? KCB : KCB / 2;
-  g.recv_off = (g.ring + (b_kind == B_NORM ? static_cast<uint32_t>(nk) * kel * 4u : 0u) + 1023u) & ~1023u;
+  const uint32_t main_end = g.ring + (b_kind == B_NORM ? static_cast<uint32_t>(nk) * kel * 4u : 0u);
+  const uint32_t slices_end = S > 1 ? static_cast<uint32_t>(S) * g.TS * BM * 4u : 0u;
+  g.recv_off = ((main_end > slices_end ? main_end : slices_end) + 1023u) & ~1023u;
   return g;
 }
 
@@ -789,7 +791,9 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
     acc *= inv_den[rr];
     const int t = b * H + r_lo + rr;
     const int kidx = j * DH + d;
-    if (a.fp8) a.o[btile_offset(t, kidx, a.Nt, a.NKC_o)] = to_e4m3(acc * inv_sa);
+    if (a.o_rowmajor)
+      reinterpret_cast<__nv_bfloat16*>(a.o)[static_cast<size_t>(t) * a.Hq * DH + kidx] = __float2bfloat16_rn(acc);
+    else if (a.fp8) a.o[btile_offset(t, kidx, a.Nt, a.NKC_o)] = to_e4m3(acc * inv_sa);
     else *reinterpret_cast<__nv_bfloat16*>(a.o + btile_offset(t, 2 * kidx, a.Nt, a.NKC_o)) = __float2bfloat16_rn(acc);
   }
   __syncthreads();

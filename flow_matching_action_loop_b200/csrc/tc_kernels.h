@@ -116,7 +116,17 @@ struct AttnArgs {
   int KC;                      // keys per chunk (multiple of ATTN_SUBK)
   float scale;                 // 1/sqrt(dh)
   float* xscratch;             // C > 1: partial rows [B][Hq][C][H][dh + 4] (O, max, sum), L2-resident scratch
+  int o_rowmajor;              // 1: o is bf16 [B][H][Hq*dh] row-major instead of the tiled operand layout
 };
+
+// Key chunks of the split-KV attention over S keys: at most 16 (one cluster), each a multiple
+// of the 64-key online-softmax step.
+inline void attn_chunks(int S, int& C, int& KC) {
+  C = S < 16 * ATTN_SUBK ? (S + ATTN_SUBK - 1) / ATTN_SUBK : 16;
+  const int per = (S + C - 1) / C;
+  KC = (per + ATTN_SUBK - 1) / ATTN_SUBK * ATTN_SUBK;
+  C = (S + KC - 1) / KC;
+}
 
 struct InprojArgs {
   const float* x;              // [T][A] state at the start of the step

@@ -43,13 +43,6 @@ ProjLayout make_layout(int rows, int K, int elem) {
   return p;
 }
 
-// Key chunks of the split-KV attention: at most 16 (one cluster), a multiple of the 64-key step.
-void attn_chunks(int S, int& C, int& KC) {
-  C = std::min(16, ceil_div(S, ATTN_SUBK));
-  KC = static_cast<int>(align_up(ceil_div(S, C), ATTN_SUBK));
-  C = ceil_div(S, KC);
-}
-
 struct GemmPlan {
   int S = 1, stages = 1;
 };

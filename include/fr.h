@@ -213,6 +213,29 @@ const char* fr_path_name(const fr_handle* h);
 /* Number of kernel launches one fr_denoise call issues for batch B. */
 int fr_launches_per_call(const fr_handle* h, int B);
 
+/* ---- kernel library: one op on caller buffers (no handle) ---- */
+
+/*
+ * fr_attention -- the loop's split-KV grouped-query attention as a stand-alone op
+ * (FlashRT walkthrough, component 5: the Pi0.5 decoder attention site; component 8:
+ * a kernel library with a stable op ABI).  For every sample b, query head j and query
+ * row i:  o = softmax(q k^T / sqrt(dh)) v  over all S_keys keys of KV head
+ * floor(j * Hkv / Hq); no mask.
+ * q: device bf16 [B][Hq][H][dh]; k, v: device bf16 [B][Hkv][S_keys][dh] (keys already
+ * rotated); o: device bf16 [B][H][Hq*dh] (row-major, the O-projection input layout).
+ * Keys are split into up to 16 chunks of a multiple of 64 keys; the chunks' partial rows
+ * are merged through `scratch`, a device buffer of fr_attention_scratch_bytes() bytes
+ * owned by the caller (NULL when that size is 0).  Asynchronous on `stream`.
+ * Limits: dh in {64, 128, 256}, Hq % Hkv == 0, 1 <= H <= 128, H <= S_keys <= 32768.
+ * Errors: FR_ERR_ARG (NULL pointer, bad size), FR_ERR_UNSUPPORTED (limits),
+ * FR_ERR_SHAPE (scratch smaller than needed), FR_ERR_CUDA.
+ */
+int fr_attention(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int H, int S_keys,
+                 int dh, void* scratch, size_t scratch_bytes, fr_stream_t stream);
+
+/* Bytes of scratch fr_attention needs for these sizes (0 if the keys fit one chunk). */
+size_t fr_attention_scratch_bytes(int B, int Hq, int H, int S_keys, int dh);
+
 /* ---- host number-format utilities used by the packer (no GPU needed) ---- */
 
 /* RoPE tables: cos/sin of pos * theta^(-2j/dh) for pos < n_pos, j < dh/2, float64

@@ -76,3 +76,21 @@ def test_invalid_configs_rejected_before_any_device_work(abi):
     assert lib.fr_denoise(None, None, None, 1, None) == abi.FR_ERR_ARG
     assert lib.fr_last_error() != b""
     lib.fr_destroy(None)   # no-op
+
+
+def test_attention_op_sizes_and_validation(abi):
+    # one key chunk needs no scratch; more chunks need [B][Hq][C][H][dh+4] floats
+    assert abi.fr_attention_scratch_bytes(1, 2, 1, 60, 128) == 0
+    assert abi.fr_attention_scratch_bytes(1, 8, 50, 866, 256) == 8 * 14 * 50 * (256 + 4) * 4
+    assert abi.fr_attention_scratch_bytes(3, 16, 100, 2148, 128) == 3 * 16 * 12 * 100 * (128 + 4) * 4
+    p = 1  # any non-NULL value: validation fails before any device access
+    bad = [((None, p, p, p, 1, 8, 1, 50, 866, 256), abi.FR_ERR_ARG),
+           ((p, p, p, p, 1, 8, 3, 50, 866, 256), abi.FR_ERR_UNSUPPORTED),   # Hq % Hkv
+           ((p, p, p, p, 1, 8, 1, 50, 866, 96), abi.FR_ERR_UNSUPPORTED),    # dh
+           ((p, p, p, p, 1, 8, 1, 129, 866, 256), abi.FR_ERR_UNSUPPORTED),  # H > 128
+           ((p, p, p, p, 1, 8, 1, 50, 40, 256), abi.FR_ERR_UNSUPPORTED),    # H > S_keys
+           ((p, p, p, p, 0, 8, 1, 50, 866, 256), abi.FR_ERR_ARG),
+           ((p, p, p, p, 1, 8, 1, 50, 866, 256), abi.FR_ERR_SHAPE)]         # no scratch given
+    lib = abi.load_library()
+    for args, code in bad:
+        assert lib.fr_attention(*args, None, 0, None) == code, (args, abi.fr_last_error())
