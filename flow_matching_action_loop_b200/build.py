@@ -1,6 +1,6 @@
 """Build the action-expert shared library in-tree for sm_100a.
 
-    python -m flow_matching_action_loop_b200.build [--force] [-v]
+    python flow_matching_action_loop_b200/build.py [--force] [-v]
 
 Compiles every csrc/*.cu and csrc/*.cpp with nvcc into _build/ and links
 libflowloop.so next to this file (CUDA runtime linked statically).
