@@ -70,7 +70,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     if _lib is not None:
         return _lib
     if not os.path.exists(path):
-        raise ImportError(f"{path} is missing: build it with `python -m flow_matching_action_loop_b200.build`")
+        raise ImportError(f"{path} is missing: build it with `python flow_matching_action_loop_b200/build.py`")
     lib = ctypes.CDLL(path)
     c_int, c_void_p, c_uint, c_char_p = ctypes.c_int, ctypes.c_void_p, ctypes.c_uint, ctypes.c_char_p
     H = c_void_p
@@ -93,6 +93,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fr_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                  c_void_p, ctypes.c_size_t, c_void_p]),
         "fr_attention_scratch_bytes": (ctypes.c_size_t, [c_int, c_int, c_int, c_int, c_int]),
+        "fr_attention_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
+                                         c_int, c_void_p]),
         "fr_round_bf16": (None, [_FP, ctypes.POINTER(ctypes.c_uint16), ctypes.c_size_t]),
         "fr_quantize_e4m3": (None, [_FP, ctypes.POINTER(ctypes.c_uint8), ctypes.c_size_t, ctypes.c_double]),
     }
@@ -220,6 +222,15 @@ def fr_attention(q: int, k: int, v: int, o: int, B: int, Hq: int, Hkv: int, H: i
 
 def fr_attention_scratch_bytes(B: int, Hq: int, H: int, S_keys: int, dh: int) -> int:
     return load_library().fr_attention_scratch_bytes(B, Hq, H, S_keys, dh)
+
+
+FR_ATTENTION_NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def fr_attention_noalloc(q: int, k: int, v: int, o: int, B: int, Hq: int, Hkv: int, H: int, S_keys: int, dh: int,
+                         stream: int = 0) -> None:
+    _check(load_library().fr_attention_noalloc(q, k, v, o, B, Hq, Hkv, H, S_keys, dh, stream),
+           "fr_attention_noalloc")
 
 
 def fr_rope_tables(n_pos: int, dh: int, theta: float):

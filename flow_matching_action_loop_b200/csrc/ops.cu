@@ -107,3 +107,44 @@ int fr_attention(const void* q, const void* k, const void* v, void* o, int B, in
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- fr_attention_noalloc
+// The same kernel with its chunk-merge scratch in a fixed array of this library's device
+// image instead of a caller buffer.  Every device the library runs on holds its own copy
+// of the array (module globals are per context); its address is looked up once per device.
+namespace {
+
+constexpr size_t NOALLOC_SCRATCH_BYTES = FR_ATTENTION_NOALLOC_SCRATCH_BYTES;
+static_assert(NOALLOC_SCRATCH_BYTES % 256 == 0, "scratch array size");
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+std::once_flag g_noalloc_once[MAX_DEVICES];
+void* g_noalloc_ptr[MAX_DEVICES];
+cudaError_t g_noalloc_err[MAX_DEVICES];
+
+}  // namespace
+
+extern "C" int fr_attention_noalloc(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv,
+                                    int H, int S_keys, int dh, fr_stream_t stream) {
+  int rc = check_attention(q, k, v, o, B, Hq, Hkv, H, S_keys, dh);
+  if (rc) return rc;
+  const size_t need = fr_attention_scratch_bytes(B, Hq, H, S_keys, dh);
+  if (need > NOALLOC_SCRATCH_BYTES) {
+    set_error("fr_attention_noalloc: these sizes need %zu bytes of scratch; the built-in array holds %zu "
+              "(call fr_attention with a caller-owned buffer instead)", need, NOALLOC_SCRATCH_BYTES);
+    return FR_ERR_UNSUPPORTED;
+  }
+  int dev = 0;
+  FR_CUDA(ensure_tc_kernels(&dev));
+  // once per device, with that device current: the array's device address
+  std::call_once(g_noalloc_once[dev], [dev] {
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
+  });
+  if (g_noalloc_err[dev] != cudaSuccess) return cuda_fail(g_noalloc_err[dev], "cudaGetSymbolAddress(scratch)");
+  // every scratch word the kernel reads is written earlier in the same launch: nothing to clear
+  const tc::AttnArgs a =
+      attention_args(q, k, v, o, Hq, Hkv, H, S_keys, dh, static_cast<float*>(g_noalloc_ptr[dev]));
+  FR_CUDA(tc::launch_attention_tc(a, B, reinterpret_cast<cudaStream_t>(stream), false));
+  return FR_OK;
+}

@@ -236,6 +236,31 @@ int fr_attention(const void* q, const void* k, const void* v, void* o, int B, in
 /* Bytes of scratch fr_attention needs for these sizes (0 if the keys fit one chunk). */
 size_t fr_attention_scratch_bytes(int B, int Hq, int H, int S_keys, int dh);
 
+/* Bytes of the scratch array built into the library for fr_attention_noalloc. */
+#define FR_ATTENTION_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/*
+ * fr_attention_noalloc -- fr_attention without a scratch argument.  The paper has no
+ * counterpart: it is a convenience of this library.  It serves callers that cannot
+ * allocate or own a device buffer: a control loop that must not enter an allocator once it
+ * runs (cudaMalloc may synchronise the device and takes unbounded time), a plug-in handed
+ * tensors but no workspace by its host framework, or code that must not change its device
+ * memory footprint after start-up.  For them the chunk-merge scratch is one fixed device
+ * array inside the library, FR_ATTENTION_NOALLOC_SCRATCH_BYTES (8 MiB) per device; this
+ * function allocates nothing.
+ * Arguments, layouts, limits and errors are those of fr_attention; in addition sizes whose
+ * fr_attention_scratch_bytes() exceeds the array are rejected with FR_ERR_UNSUPPORTED
+ * (the π0.5 layer shape, B=1 Hq=8 H=50 S_keys=866 dh=256, needs 5.8 MB).
+ * The first call on a device looks up the array's address on that device (and sets the
+ * kernel attributes); make that first call before any stream capture that should contain
+ * later calls.  All calls on one device share the one array: two calls whose kernels can
+ * overlap in time (different streams, or different host threads without ordering) race
+ * on it and may return wrong results; calls ordered on one stream are safe.  The array
+ * needs no clearing: each launch writes every word it reads before reading it.
+ */
+int fr_attention_noalloc(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int H,
+                         int S_keys, int dh, fr_stream_t stream);
+
 /* ---- host number-format utilities used by the packer (no GPU needed) ---- */
 
 /* RoPE tables: cos/sin of pos * theta^(-2j/dh) for pos < n_pos, j < dh/2, float64

@@ -94,3 +94,13 @@ def test_attention_op_sizes_and_validation(abi):
     lib = abi.load_library()
     for args, code in bad:
         assert lib.fr_attention(*args, None, 0, None) == code, (args, abi.fr_last_error())
+
+
+def test_noalloc_attention_rejects_before_device_work(abi):
+    lib = abi.load_library()
+    p = 1
+    # the π0.5 layer fits the built-in 8 MiB array; two samples of it do not
+    assert abi.fr_attention_scratch_bytes(1, 8, 50, 866, 256) <= abi.FR_ATTENTION_NOALLOC_SCRATCH_BYTES
+    assert lib.fr_attention_noalloc(p, p, p, p, 2, 8, 1, 50, 866, 256, None) == abi.FR_ERR_UNSUPPORTED
+    assert b"scratch" in lib.fr_last_error()
+    assert lib.fr_attention_noalloc(None, p, p, p, 1, 8, 1, 50, 866, 256, None) == abi.FR_ERR_ARG
