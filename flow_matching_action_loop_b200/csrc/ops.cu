@@ -48,16 +48,10 @@ int check_attention(const void* q, const void* k, const void* v, const void* o, 
     set_error("fr_attention: needs dh in {64,128,256}, Hq %% Hkv == 0, H <= 128, H <= S_keys <= 32768");
     return FR_ERR_UNSUPPORTED;
   }
-  int C = 1, KC = 64;
-  tc::attn_chunks(S_keys, C, KC);
-  if (tc::attn_smem_bytes(H, dh, KC, C) > 200 * 1024) {
-    set_error("fr_attention: a key chunk of %d keys does not fit shared memory", KC);
-    return FR_ERR_UNSUPPORTED;
-  }
   return FR_OK;
 }
 
-tc::AttnArgs attention_args(const void* q, const void* k, const void* v, void* o, int Hq, int Hkv, int H,
+tc::AttnArgs attention_args(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int H,
                             int S_keys, int dh, float* scratch) {
   tc::AttnArgs a{};
   a.q = static_cast<const __nv_bfloat16*>(q);
@@ -72,7 +66,9 @@ tc::AttnArgs attention_args(const void* q, const void* k, const void* v, void* o
   a.Hq = Hq;
   a.Hkv = Hkv;
   a.dh = dh;
-  tc::attn_chunks(S_keys, a.C, a.KC);
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  tc::attn_plan(S_keys, tc::attn_tiles(B, Hq, Hkv, H), nsm, a.C, a.KC);
   a.scale = 1.0f / std::sqrt(static_cast<float>(dh));
   a.xscratch = scratch;
   return a;
@@ -101,7 +97,7 @@ int fr_attention(const void* q, const void* k, const void* v, void* o, int B, in
     return FR_ERR_SHAPE;
   }
   FR_CUDA(ensure_tc_kernels(nullptr));
-  const tc::AttnArgs a = attention_args(q, k, v, o, Hq, Hkv, H, S_keys, dh, static_cast<float*>(scratch));
+  const tc::AttnArgs a = attention_args(q, k, v, o, B, Hq, Hkv, H, S_keys, dh, static_cast<float*>(scratch));
   FR_CUDA(tc::launch_attention_tc(a, B, reinterpret_cast<cudaStream_t>(stream), false));
   return FR_OK;
 }

@@ -20,6 +20,7 @@
 //   over 64-key sub-chunks; the chunks' (O, max, sum) rows are pushed to their owner CTA by
 //   bulk copies and merged with log-sum-exp weights in rank order.
 #include <algorithm>
+#include <type_traits>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <math.h>
@@ -37,7 +38,7 @@ using namespace fr::sm100;
 // Optional phase timestamps (globaltimer per CTA), compiled in only with -DFR_TIMELINE for
 // performance analysis; the product build has none of this code.
 #ifdef FR_TIMELINE
-__device__ unsigned long long* g_tl = nullptr;   // [cap][8]: kind, cta, t0..t5
+__device__ unsigned long long* g_tl = nullptr;   // [cap][16]: kind, cta, t0..t13
 __device__ unsigned g_tl_count = 0;
 __device__ unsigned g_tl_cap = 0;
 #define TL_DECL __shared__ unsigned tl_slot_;
@@ -46,15 +47,15 @@ __device__ unsigned g_tl_cap = 0;
     if (threadIdx.x == 0) {                                                                     \
       tl_slot_ = g_tl ? atomicAdd(&g_tl_count, 1u) : 0xFFFFFFFFu;                               \
       if (tl_slot_ < g_tl_cap) {                                                                \
-        g_tl[tl_slot_ * 8 + 0] = (kind);                                                        \
-        g_tl[tl_slot_ * 8 + 1] = blockIdx.x | (blockIdx.y << 10) | (blockIdx.z << 20);          \
-        g_tl[tl_slot_ * 8 + 2] = fr::sm100::globaltimer();                                      \
+        g_tl[tl_slot_ * 16 + 0] = (kind);                                                        \
+        g_tl[tl_slot_ * 16 + 1] = blockIdx.x | (blockIdx.y << 10) | (blockIdx.z << 20);          \
+        g_tl[tl_slot_ * 16 + 2] = fr::sm100::globaltimer();                                      \
       }                                                                                         \
     }                                                                                           \
   } while (0)
 #define TL(k)                                                                                   \
   do {                                                                                          \
-    if (tl_slot_ < g_tl_cap) g_tl[tl_slot_ * 8 + 2 + (k)] = fr::sm100::globaltimer();          \
+    if (tl_slot_ < g_tl_cap) g_tl[tl_slot_ * 16 + 2 + (k)] = fr::sm100::globaltimer();          \
   } while (0)
 #else
 #define TL_DECL
@@ -244,6 +245,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
           break;
         }
         tc_fence_after();
+        if (i == 0) TL(6);
         const uint32_t a0 = smem_u32(dsm + s * gm.slot), b0 = a0 + gm.a_bytes;
 #pragma unroll
         for (int k = 0; k < KCB / 32; ++k) {
@@ -349,18 +351,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   float* red = reinterpret_cast<float*>(dsm);   // S == 1: [Nt][RED_LD], aliases the drained ring
   float* xs = (S > 1) ? a.xscratch + (static_cast<size_t>(nt) * a.MB + mb) * S * Nt * BM : nullptr;
   const int t_hi = min(Nt, a.T - n0);           // valid tokens of this n-tile
-  if (warp >= 4) {
+  {
+    // TMEM -> red (S == 1) or the scratch (S > 1) by all eight warps: warp w reads the lane
+    // quadrant w % 4; warps 0-3 take the first half of the token columns, warps 4-7 the rest
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    for (int c0 = 0; c0 < Nt; c0 += 64) {   // up to 4 loads in flight, one wait
+    const int hc = ((Nt >> 4) + 1) / 2 * 16;
+    const int cbeg = warp < 4 ? 0 : hc, cend = warp < 4 ? min(hc, Nt) : Nt;
+    for (int c0 = cbeg; c0 < cend; c0 += 64) {   // up to 4 loads in flight, one wait
       uint32_t v[4][16];
 #pragma unroll
       for (int u = 0; u < 4; ++u)
-        if (c0 + 16 * u < Nt) tmem_ld16_nowait(tacc + (static_cast<uint32_t>(q * 32) << 16) + c0 + 16 * u, v[u]);
+        if (c0 + 16 * u < cend) tmem_ld16_nowait(tacc + (static_cast<uint32_t>(q * 32) << 16) + c0 + 16 * u, v[u]);
       tmem_wait_ld();
 #pragma unroll
       for (int u = 0; u < 4; ++u)
-        if (c0 + 16 * u < Nt)
+        if (c0 + 16 * u < cend)
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int tok = c0 + 16 * u + j;
@@ -369,12 +375,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
           }
     }
   }
+  if (tid == 128) TL(7);
   tc_fence_before();
   const int tok0 = ks * Nt / S, tok1 = (ks + 1) * Nt / S;
   float* xst = reinterpret_cast<float*>(dsm);   // S > 1: [S][TS][128] slices of this CTA's tokens
   if (S > 1) {
     cluster_arrive_release();   // the partial tiles in scratch are visible to the cluster after this barrier
     cluster_wait_acquire();
+    if (tid == 0) TL(8);
     if (tid == 0) {             // one round trip: every slice of this CTA's tokens by bulk copy
       const uint32_t sb = static_cast<uint32_t>(tok1 - tok0) * BM * 4u;
       mbar_arrive_expect_tx(&sh.xbar, S * sb);
@@ -389,93 +397,147 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   if (tid == 0) TL(4);
 
   const float al = a.alpha ? *a.alpha : 1.0f;
-  // split-K sum of one accumulator element over the cluster, in rank order (deterministic)
-  auto val = [&](int tok, int row) -> float {
+  // Split-K sums of N (2 or 4) consecutive accumulator rows of one token over the cluster, in
+  // rank order (deterministic), times the dequantisation / deferred-rstd scale.
+  auto vals = [&](int tok, int row, float* out, auto n_tag) {
+    constexpr int N = decltype(n_tag)::value;
     const float sc = a.rscale ? al * sh.rstd[tok] : al;
-    if (S == 1) return red[tok * RED_LD + row] * sc;
-    const float* p = xst + static_cast<size_t>(tok - tok0) * BM + row;
+    float acc[N];
+#pragma unroll
+    for (int e = 0; e < N; ++e) acc[e] = 0.f;
+    const float* p = (S == 1) ? red + tok * RED_LD + row : xst + static_cast<size_t>(tok - tok0) * BM + row;
     const size_t stride = static_cast<size_t>(gm.TS) * BM;
-    float v[16];
+    const int ns = (S == 1) ? 1 : S;
 #pragma unroll
-    for (int s = 0; s < 16; ++s) v[s] = s < S ? p[s * stride] : 0.f;
-    float acc = 0.f;
+    for (int s2 = 0; s2 < 16; ++s2)
+      if (s2 < ns) {
+        if constexpr (N == 4) {
+          const float4 v = *reinterpret_cast<const float4*>(p + s2 * stride);
+          acc[0] += v.x;   // rank order
+          acc[1] += v.y;
+          acc[2] += v.z;
+          acc[3] += v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2*>(p + s2 * stride);
+          acc[0] += v.x;
+          acc[1] += v.y;
+        }
+      }
 #pragma unroll
-    for (int s = 0; s < 16; ++s) acc += v[s];                          // rank order
-    return acc * sc;
+    for (int e = 0; e < N; ++e) out[e] = acc[e] * sc;
   };
+  using Two = std::integral_constant<int, 2>;
+  using Four = std::integral_constant<int, 4>;
+  // Each warp takes whole tokens (tok0 + warp, + 8, ...), each lane 2 or 4 consecutive
+  // features; EPU tokens per warp have their independent loads issued before any is used.
+  constexpr int EPU = 4;
 
   if (a.epi == EPI_RESID) {
-    const int row = tid & 127, sub = tid >> 7;
+    const int row = lane * 4;
     const int f = mb * BM + row;
+    const bool fok = f < a.Nout;   // Nout is a multiple of 16
     const float* hst = reinterpret_cast<const float*>(dsm + gm.recv_off);   // [2][TS][64]
     if (S > 1 && !mbar_wait(&sh.hbar, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0x600);
-    for (int tb = tok0; tb < tok1; tb += 2) {
-      const int tok = tb + sub;
-      const int t = n0 + tok;
-      float sq = 0.f;
-      if (tok < tok1 && t < a.T && f < a.Nout) {
-        float* hp = a.h_out + htile_offset(t, f, Nt, a.KB);
-        const float hold = (S > 1) ? hst[((row >> 6) * gm.TS + (tok - tok0)) * 64 + (row & 63)] : *hp;
-        const float hv = hold + val(tok, row);
-        *hp = hv;
-        sq = hv * hv;
-        if (a.xb_out)
-          *reinterpret_cast<__nv_bfloat16*>(a.xb_out + btile_offset(t, 2 * f, Nt, a.NKC_x)) =
-              __float2bfloat16_rn(hv * a.xb_gamma[f]);
+    float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (a.xb_out && fok) g4 = *reinterpret_cast<const float4*>(a.xb_gamma + f);
+    for (int tb = tok0 + warp; tb < tok1; tb += 8 * EPU) {
+      float4 hold[EPU];
+      float acc[EPU][4];
+#pragma unroll
+      for (int u = 0; u < EPU; ++u) {
+        const int tok = tb + 8 * u, t = n0 + tok;
+        if (tok < tok1 && t < a.T && fok) {
+          hold[u] = (S > 1) ? *reinterpret_cast<const float4*>(hst + ((row >> 6) * gm.TS + (tok - tok0)) * 64 + (row & 63))
+                            : *reinterpret_cast<const float4*>(a.h_out + htile_offset(t, f, Nt, a.KB));
+          vals(tok, row, acc[u], Four{});
+        }
       }
-      for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-      if (lane == 0) sh.ssq_part[sub][(tid >> 5) & 3] = sq;
-      __syncthreads();
-      if (row == 0 && tok < tok1 && t < a.T)
-        a.ssq_out[static_cast<size_t>(t) * a.ssq_ld + mb] =
-            ((sh.ssq_part[sub][0] + sh.ssq_part[sub][1]) + sh.ssq_part[sub][2]) + sh.ssq_part[sub][3];
-      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < EPU; ++u) {
+        const int tok = tb + 8 * u, t = n0 + tok;
+        if (tok >= tok1 || t >= a.T) break;   // warp-uniform
+        float sq = 0.f;
+        if (fok) {
+          const float4 hv = make_float4(hold[u].x + acc[u][0], hold[u].y + acc[u][1], hold[u].z + acc[u][2],
+                                        hold[u].w + acc[u][3]);
+          *reinterpret_cast<float4*>(a.h_out + htile_offset(t, f, Nt, a.KB)) = hv;
+          sq = ((hv.x * hv.x + hv.y * hv.y) + hv.z * hv.z) + hv.w * hv.w;
+          if (a.xb_out)
+            *reinterpret_cast<uint2*>(a.xb_out + btile_offset(t, 2 * f, Nt, a.NKC_x)) =
+                make_uint2(pack_bf16x2(hv.x * g4.x, hv.y * g4.y), pack_bf16x2(hv.z * g4.z, hv.w * g4.w));
+        }
+        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        if (lane == 0) a.ssq_out[static_cast<size_t>(t) * a.ssq_ld + mb] = sq;
+      }
     }
   } else if (a.epi == EPI_GELU) {
-    const int p = tid & 63, sub = tid >> 6;
-    const int f = mb * 64 + p;
+    const int p = lane * 2;
+    const int f = mb * 64 + p;   // F is a multiple of 64
     const float inv = (a.fp8 && a.s_a_out) ? 1.0f / *a.s_a_out : 1.0f;
-    for (int tok = tok0 + sub; tok < tok1; tok += 4) {
+    for (int tok = tok0 + warp; tok < tok1; tok += 8) {
       const int t = n0 + tok;
-      if (t >= a.T || f >= a.F) continue;
-      const float u = gelu_tanh(val(tok, p)) * val(tok, p + 64);
+      if (t >= a.T || f >= a.F) break;
+      float g[2], up[2];
+      vals(tok, p, g, Two{});
+      vals(tok, p + 64, up, Two{});
+      const float u0 = gelu_tanh(g[0]) * up[0], u1 = gelu_tanh(g[1]) * up[1];
       if (a.fp8) {
-        a.u_out[btile_offset(t, f, Nt, a.NKC_u)] = to_e4m3(u * inv);
+        *reinterpret_cast<uint16_t*>(a.u_out + btile_offset(t, f, Nt, a.NKC_u)) =
+            static_cast<uint16_t>(to_e4m3(u0 * inv) | (static_cast<uint32_t>(to_e4m3(u1 * inv)) << 8));
       } else {
-        *reinterpret_cast<__nv_bfloat16*>(a.u_out + btile_offset(t, 2 * f, Nt, a.NKC_u)) = __float2bfloat16_rn(u);
+        *reinterpret_cast<uint32_t*>(a.u_out + btile_offset(t, 2 * f, Nt, a.NKC_u)) = pack_bf16x2(u0, u1);
       }
     }
   } else {   // EPI_QKV
     const int half = a.dh >> 1;
     if (mb < a.MB_rot) {
-      const int p = tid & 63, sub = tid >> 6;
+      const int p = lane * 2;                 // rotate-half pairs p, p+1 (same head: half is even)
       const int pi = mb * 64 + p;
       const int head = pi / half, j = pi % half;
-      for (int tok = tok0 + sub; tok < tok1; tok += 4) {
-        const int t = n0 + tok;
-        if (t >= a.T) continue;
-        const int b = t / a.H, i = t % a.H, pos = a.P + i;
-        const float lo = val(tok, p), hi = val(tok, p + 64);
-        const float c = a.rope_cos[pos * half + j], sn = a.rope_sin[pos * half + j];
-        const float r0 = lo * c - hi * sn, r1 = lo * sn + hi * c;
-        __nv_bfloat16* dst;
-        if (head < a.Hq) dst = a.q_out + ((static_cast<size_t>(b) * a.Hq + head) * a.H + i) * a.dh;
-        else dst = a.kv_k + ((static_cast<size_t>(b) * a.Hkv + (head - a.Hq)) * a.S_max + pos) * a.dh;
-        dst[j] = __float2bfloat16_rn(r0);
-        dst[j + half] = __float2bfloat16_rn(r1);
+      for (int tb = tok0 + warp; tb < tok1; tb += 8 * EPU) {
+        float2 cs[EPU], sn[EPU];
+#pragma unroll
+        for (int u = 0; u < EPU; ++u) {
+          const int tok = tb + 8 * u, t = n0 + tok;
+          if (tok < tok1 && t < a.T) {
+            const int pos = a.P + t % a.H;
+            cs[u] = *reinterpret_cast<const float2*>(a.rope_cos + pos * half + j);
+            sn[u] = *reinterpret_cast<const float2*>(a.rope_sin + pos * half + j);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < EPU; ++u) {
+          const int tok = tb + 8 * u, t = n0 + tok;
+          if (tok >= tok1 || t >= a.T) break;
+          const int b = t / a.H, i = t % a.H, pos = a.P + i;
+          float lo[2], hi[2];
+          vals(tok, p, lo, Two{});
+          vals(tok, p + 64, hi, Two{});
+          const float r00 = lo[0] * cs[u].x - hi[0] * sn[u].x, r10 = lo[0] * sn[u].x + hi[0] * cs[u].x;
+          const float r01 = lo[1] * cs[u].y - hi[1] * sn[u].y, r11 = lo[1] * sn[u].y + hi[1] * cs[u].y;
+          __nv_bfloat16* dst;
+          if (head < a.Hq) dst = a.q_out + ((static_cast<size_t>(b) * a.Hq + head) * a.H + i) * a.dh;
+          else dst = a.kv_k + ((static_cast<size_t>(b) * a.Hkv + (head - a.Hq)) * a.S_max + pos) * a.dh;
+          *reinterpret_cast<uint32_t*>(dst + j) = pack_bf16x2(r00, r01);
+          *reinterpret_cast<uint32_t*>(dst + j + half) = pack_bf16x2(r10, r11);
+        }
       }
     } else {
-      const int row = tid & 127, sub = tid >> 7;
+      const int row = lane * 4;
       const int idx = (mb - a.MB_rot) * BM + row;
       const int g = idx / a.dh, d = idx % a.dh;
-      for (int tok = tok0 + sub; tok < tok1; tok += 2) {
+      for (int tok = tok0 + warp; tok < tok1; tok += 8) {
         const int t = n0 + tok;
-        if (t >= a.T) continue;
+        if (t >= a.T) break;
         const int b = t / a.H, i = t % a.H, pos = a.P + i;
-        a.kv_v[((static_cast<size_t>(b) * a.Hkv + g) * a.S_max + pos) * a.dh + d] = __float2bfloat16_rn(val(tok, row));
+        float v4[4];
+        vals(tok, row, v4, Four{});
+        *reinterpret_cast<uint2*>(a.kv_v + ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max + pos) * a.dh + d) =
+            make_uint2(pack_bf16x2(v4[0], v4[1]), pack_bf16x2(v4[2], v4[3]));
       }
     }
   }
+  if (tid == 0) TL(9);
   __syncthreads();
   if (tid == 0) TL(5);
   if (warp == 1) {
@@ -704,6 +766,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
     __syncthreads();   // Q/K/V are dead in every warp: the slices below overlay them
     cluster_arrive_release();
     cluster_wait_acquire();
+    if (tid == 0) TL(6);
   } else {
     __syncthreads();   // every warp is done with Q/K/V before the partial rows overwrite them
     if (tid == 0) TL(3);
@@ -778,6 +841,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
     inv_den[tid] = 1.0f / den;
   }
   __syncthreads();
+  if (tid == 0) TL(7);
   const float inv_sa = (a.fp8 && a.s_a) ? 1.0f / *a.s_a : 1.0f;
   for (int it = tid; it < nr * DH; it += blockDim.x) {
     const int rr = it / DH, d = it % DH;
@@ -795,6 +859,402 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
       reinterpret_cast<__nv_bfloat16*>(a.o)[static_cast<size_t>(t) * a.Hq * DH + kidx] = __float2bfloat16_rn(acc);
     else if (a.fp8) a.o[btile_offset(t, kidx, a.Nt, a.NKC_o)] = to_e4m3(acc * inv_sa);
     else *reinterpret_cast<__nv_bfloat16*>(a.o + btile_offset(t, 2 * kidx, a.Nt, a.NKC_o)) = __float2bfloat16_rn(acc);
+  }
+  __syncthreads();
+  if (tid == 0) TL(5);
+}
+
+// ================================================================== attention on tcgen05
+//
+// One CTA per (sample b, KV head g, tile of 128 query rows, key chunk c); the rows of a tile
+// are the (query head, action row) pairs of every query head that reads KV head g, so the
+// chunk's K and V are staged once for the whole group.  Per 64-key sub-chunk:
+//   S = Q K^T          tcgen05 (M = 128 rows, N = 64 keys, K = dh), fp32 in tensor memory
+//   online softmax     one thread per row: S row from tensor memory, running max / sum,
+//                      P = 2^(s - m) in bf16 into shared memory, O rescaled in tensor memory
+//   O += P V           tcgen05 (M = 128, N = dh, K = 64 keys), V read MN-major as stored
+// Chunks (a cluster when C > 1) are merged over (O, max, sum) rows in the L2 scratch with the
+// same rank-order log-sum-exp weights as the flash-decoding merge.
+
+constexpr int UA_SUB = 64;        // keys per sub-chunk
+constexpr int UA_THREADS = 128;   // one thread per query row of the tile
+
+struct UAttnGeom {
+  uint32_t q_off, k_off0, k_off1, v_off0, v_off1, p_off, total, tcols, o_col;
+};
+
+__host__ __device__ __forceinline__ UAttnGeom uattn_geom(int dh) {
+  UAttnGeom g;
+  const uint32_t q = 128u * dh * 2u, kv = static_cast<uint32_t>(UA_SUB) * dh * 2u;
+  g.q_off = 0;
+  g.k_off0 = q;
+  g.v_off0 = q + kv;
+  g.k_off1 = q + 2 * kv;
+  g.v_off1 = q + 3 * kv;
+  g.p_off = q + 4 * kv;
+  g.total = g.p_off + 128u * UA_SUB * 2u;
+  g.tcols = dh == 256 ? 512u : (dh == 128 ? 256u : 128u);   // S at column 0, O at o_col
+  g.o_col = dh == 256 ? 256u : (dh == 128 ? 128u : 64u);
+  return g;
+}
+
+template <int DH>
+__global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_constant__ AttnArgs a) {
+  extern __shared__ __align__(1024) uint8_t dsm[];
+  __shared__ uint64_t bar_s, bar_o, stage_bar;
+  __shared__ uint32_t tmem_base;
+  __shared__ float w_sh[16][128];   // merge weight of chunk s for owned row rr (C <= 16)
+  __shared__ float inv_den[128];
+  TL_DECL
+  TL_BEGIN(20);
+  constexpr int OLD = DH + 4;            // fp32 row stride of the partial-O rows
+  constexpr int VPR = DH / 8;            // 16-byte vectors per K/V/Q row
+  constexpr uint32_t IDESC_S = idesc_f32acc(FMT_BF16, 128, UA_SUB);
+  constexpr uint32_t IDESC_O = idesc_f32acc(FMT_BF16, 128, DH) | IDESC_B_MN_MAJOR;
+  const UAttnGeom gm = uattn_geom(DH);
+  const int c = blockIdx.x, y = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.Hq / a.Hkv;            // query heads per KV head (consecutive heads)
+  const int R = G * a.H;                 // query rows of one KV group
+  const int MT = (R + 127) >> 7;
+  const int g = y / MT, row0 = (y - g * MT) * 128;
+  const int Rv = min(128, R - row0);     // valid rows of this tile
+  const int S = a.P + a.H;
+  const int C = a.C;
+  const int key0 = c * a.KC;
+  const int nkeys = min(a.KC, S - key0);
+  const int nsub = (nkeys + UA_SUB - 1) / UA_SUB;
+  const __nv_bfloat16* kg = a.kv_k + ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max) * DH;
+  const __nv_bfloat16* vg = a.kv_v + ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max) * DH;
+  // the group's query rows are contiguous: heads g*G.. of sample b, H rows each
+  const __nv_bfloat16* qg = a.q + ((static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G) * a.H + row0) * DH;
+
+  if (tid == 0) {
+    mbar_init(&bar_s, 1);
+    mbar_init(&bar_o, 1);
+    mbar_init(&stage_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_base, gm.tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  grid_dep_launch();
+  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t tS = tmem_base, tO = tmem_base + gm.o_col;
+
+  // K rows of sub-chunk sc into a K-major operand tile [64 keys x DH] (16-byte core columns
+  // of 64 x 16 B); which: 0 = prefix keys (and zero rows past the chunk), 1 = action keys, 2 = all.
+  auto load_k = [&](int sc, uint8_t* Kb, int which) {
+    const int kb0 = key0 + sc * UA_SUB;
+    for (int it = tid; it < UA_SUB * VPR; it += UA_THREADS) {
+      const int n = it % UA_SUB, j = it / UA_SUB;   // consecutive threads: consecutive keys
+      const int key = kb0 + n;
+      const bool valid = sc * UA_SUB + n < nkeys;
+      const bool mine = which == 2 || (which == 0 ? (key < a.P || !valid) : (key >= a.P && valid));
+      if (mine)
+        cp_async16(Kb + j * (UA_SUB * 16) + (n >> 3) * 128 + (n & 7) * 16,
+                   kg + static_cast<size_t>(valid ? key : 0) * DH + j * 8, valid);
+    }
+  };
+  // V rows of sub-chunk sc as stored ([key][DH], DH contiguous): the MN-major B operand of
+  // O += P V, core matrices of 8 keys x 16 B; 8-key groups DH*16 bytes apart.
+  auto load_v = [&](int sc, uint8_t* Vb, int which) {
+    const int kb0 = key0 + sc * UA_SUB;
+    for (int it = tid; it < UA_SUB * VPR; it += UA_THREADS) {
+      const int k8 = it & 7, j = (it >> 3) % VPR, kq = (it >> 3) / VPR;
+      const int n = kq * 8 + k8;
+      const int key = kb0 + n;
+      const bool valid = sc * UA_SUB + n < nkeys;
+      const bool mine = which == 2 || (which == 0 ? (key < a.P || !valid) : (key >= a.P && valid));
+      if (mine)
+        cp_async16(Vb + kq * (DH * 16) + j * 128 + k8 * 16, vg + static_cast<size_t>(valid ? key : 0) * DH + j * 8,
+                   valid);
+    }
+  };
+  auto Kbuf = [&](int bf) { return dsm + (bf ? gm.k_off1 : gm.k_off0); };
+  auto Vbuf = [&](int bf) { return dsm + (bf ? gm.v_off1 : gm.v_off0); };
+
+  // prefix keys do not depend on the previous kernel: their loads go first
+  load_k(0, Kbuf(0), 0);
+  load_v(0, Vbuf(0), 0);
+  if (nsub > 1) {
+    load_k(1, Kbuf(1), 0);
+    load_v(1, Vbuf(1), 0);
+  }
+  cp_async_commit();
+  grid_dep_wait();
+  if (tid == 0) TL(1);
+  load_k(0, Kbuf(0), 1);
+  load_v(0, Vbuf(0), 1);
+  if (nsub > 1) {
+    load_k(1, Kbuf(1), 1);
+    load_v(1, Vbuf(1), 1);
+  }
+  for (int it = tid; it < 128 * VPR; it += UA_THREADS) {   // Q tile, K-major [128 rows x DH]
+    const int r = it & 127, j = it >> 7;
+    cp_async16(dsm + gm.q_off + j * 2048 + (r >> 3) * 128 + (r & 7) * 16,
+               qg + static_cast<size_t>(r < Rv ? r : 0) * DH + j * 8, r < Rv);
+  }
+  cp_async_commit();
+  cp_async_wait_all();
+  fence_proxy_async_smem();   // cp.async writes -> visible to the tensor core
+  __syncthreads();
+  if (tid == 0) TL(2);
+
+  const float sl2 = a.scale * 1.4426950408889634f;   // scores in log2 units
+  float m_run = -INFINITY, l_run = 0.f;
+  bool failed = false;
+  for (int sc = 0; sc < nsub; ++sc) {
+    const int bf = sc & 1;
+    if (sc >= 2) {   // K(sc) and V(sc) were issued in the two previous sub-chunks
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      __syncthreads();
+    }
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t qa = smem_u32(dsm + gm.q_off), ka = smem_u32(Kbuf(bf));
+#pragma unroll
+      for (int k = 0; k < DH / 16; ++k)
+        mma_bf16(tS, smem_desc(qa + k * 2 * 2048, 2048, 128), smem_desc(ka + k * 2 * (UA_SUB * 16), UA_SUB * 16, 128),
+                 IDESC_S, k > 0);
+      mma_commit(&bar_s);
+    }
+    const bool got_s = mbar_wait(&bar_s, sc & 1, WAIT_LIMIT_NS);
+    if (__syncthreads_or(!got_s)) {
+      if (tid == 0) report_timeout(a.status, 0x700);
+      failed = true;
+      break;
+    }
+    tc_fence_after();
+    if (sc + 2 < nsub) {   // K buffer bf is free once S(sc) is done
+      load_k(sc + 2, Kbuf(bf), 2);
+      cp_async_commit();
+    }
+    uint32_t sv[UA_SUB];
+#pragma unroll
+    for (int u = 0; u < UA_SUB / 16; ++u) tmem_ld16_nowait(tS + lane_base + 16 * u, sv + 16 * u);
+    tmem_wait_ld();
+    const int kb = sc * UA_SUB;
+    float mx = m_run;
+#pragma unroll
+    for (int jj = 0; jj < UA_SUB; ++jj) {
+      float v = __uint_as_float(sv[jj]) * sl2;
+      if (kb + jj >= nkeys) v = -INFINITY;
+      sv[jj] = __float_as_uint(v);
+      mx = fmaxf(mx, v);
+    }
+    if (sc > 0) {   // O(sc-1) complete: P may be overwritten and O rescaled
+      const bool got_o = mbar_wait(&bar_o, (sc - 1) & 1, WAIT_LIMIT_NS);
+      if (__syncthreads_or(!got_o)) {
+        if (tid == 0) report_timeout(a.status, 0x701);
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+      if (sc + 1 < nsub) {   // V buffer of sub-chunk sc-1 is free: V(sc+1) goes there
+        load_v(sc + 1, Vbuf((sc + 1) & 1), 2);
+        cp_async_commit();
+      }
+    }
+    const float corr = exp2f(m_run - mx);
+    float psum = 0.f;
+    uint8_t* prow = dsm + gm.p_off + (tid >> 3) * 128 + (tid & 7) * 16;   // P row, K-major [128 x 64]
+#pragma unroll
+    for (int kk = 0; kk < UA_SUB / 8; ++kk) {
+      float p[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        p[e] = exp2f(__uint_as_float(sv[kk * 8 + e]) - mx);
+        psum += p[e];
+      }
+      *reinterpret_cast<uint4*>(prow + kk * 2048) =
+          make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
+    }
+    l_run = l_run * corr + psum;
+    m_run = mx;
+    if (sc > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
+#pragma unroll 1
+      for (int c0 = 0; c0 < DH; c0 += 16) {
+        uint32_t ov[16];
+        tmem_ld16_nowait(tO + lane_base + c0, ov);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+        tmem_st16(tO + lane_base + c0, ov);
+      }
+      tmem_wait_st();
+    }
+    fence_proxy_async_smem();   // P (generic-proxy stores) -> visible to the tensor core
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t pa = smem_u32(dsm + gm.p_off), va = smem_u32(Vbuf(bf));
+#pragma unroll
+      for (int k = 0; k < UA_SUB / 16; ++k)
+        mma_bf16(tO, smem_desc(pa + k * 2 * 2048, 2048, 128), smem_desc(va + k * 2 * (DH * 16), DH * 16, 128), IDESC_O,
+                 (sc > 0 || k > 0) ? 1u : 0u);
+      mma_commit(&bar_o);
+    }
+  }
+  if (!failed) {
+    const bool got = mbar_wait(&bar_o, (nsub - 1) & 1, WAIT_LIMIT_NS);
+    if (__syncthreads_or(!got)) {
+      if (tid == 0) report_timeout(a.status, 0x702);
+      failed = true;
+    }
+  }
+  cp_async_wait_all();
+  tc_fence_after();
+  if (tid == 0) TL(3);
+
+  const int rr = row0 + tid;                         // this thread's row of the group
+  const bool rv = tid < Rv && !failed;
+  const int jq = g * G + rr / a.H, iq = rr % a.H;    // query head, action row
+  const float inv_sa = (a.fp8 && a.s_a) ? 1.0f / *a.s_a : 1.0f;
+  // writes 16 consecutive output features d0.. of row (token t, head jq)
+  auto store16 = [&](int t, int jh, int d0, const float* v) {
+    const int kidx = jh * DH + d0;
+    if (a.o_rowmajor) {
+      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + static_cast<size_t>(t) * a.Hq * DH + kidx);
+      dst[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+      dst[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                          pack_bf16x2(v[14], v[15]));
+    } else if (a.fp8) {
+      *reinterpret_cast<uint4*>(a.o + btile_offset(t, kidx, a.Nt, a.NKC_o)) =
+          make_uint4(pack_e4m3x4(v[0] * inv_sa, v[1] * inv_sa, v[2] * inv_sa, v[3] * inv_sa),
+                     pack_e4m3x4(v[4] * inv_sa, v[5] * inv_sa, v[6] * inv_sa, v[7] * inv_sa),
+                     pack_e4m3x4(v[8] * inv_sa, v[9] * inv_sa, v[10] * inv_sa, v[11] * inv_sa),
+                     pack_e4m3x4(v[12] * inv_sa, v[13] * inv_sa, v[14] * inv_sa, v[15] * inv_sa));
+    } else {
+      *reinterpret_cast<uint4*>(a.o + btile_offset(t, 2 * kidx, a.Nt, a.NKC_o)) =
+          make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+      *reinterpret_cast<uint4*>(a.o + btile_offset(t, 2 * kidx + 16, a.Nt, a.NKC_o)) =
+          make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                     pack_bf16x2(v[14], v[15]));
+    }
+  };
+
+  if (C == 1) {
+    const float inv = 1.0f / l_run;
+#pragma unroll 1
+    for (int c0 = 0; c0 < DH; c0 += 16) {
+      uint32_t ov[16];
+      tmem_ld16_nowait(tO + lane_base + c0, ov);
+      tmem_wait_ld();
+      float v[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(ov[e]) * inv;
+      if (rv) store16(b * a.H + iq, jq, c0, v);
+    }
+  } else {
+    // this chunk's (O, max, sum) row into the scratch, [B][Hq][C][H][OLD]
+    float* xrow = a.xscratch + ((static_cast<size_t>(b) * a.Hq + jq) * C + c) * a.H * OLD + static_cast<size_t>(iq) * OLD;
+#pragma unroll 1
+    for (int c0 = 0; c0 < DH; c0 += 16) {
+      uint32_t ov[16];
+      tmem_ld16_nowait(tO + lane_base + c0, ov);
+      tmem_wait_ld();
+      if (rv)
+#pragma unroll
+        for (int e = 0; e < 16; e += 4)
+          *reinterpret_cast<float4*>(xrow + c0 + e) = make_float4(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1]),
+                                                                  __uint_as_float(ov[e + 2]), __uint_as_float(ov[e + 3]));
+    }
+    if (rv) *reinterpret_cast<float4*>(xrow + DH) = make_float4(m_run, l_run, 0.f, 0.f);
+  }
+  tc_fence_before();
+  fence_proxy_async_smem();   // the staging below overwrites Q/K/V/P by bulk copy
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, gm.tcols);
+  }
+  if (C == 1) {
+    if (tid == 0) TL(5);
+    return;
+  }
+  cluster_arrive_release();   // every chunk's rows are in the scratch after this barrier
+  cluster_wait_acquire();
+  if (tid == 0) TL(6);
+  // ---------------- merge the rows this CTA owns over the key chunks, in rank order
+  const int r_lo = c * Rv / C, r_hi = (c + 1) * Rv / C;
+  const int RM = (128 + C - 1) / C;                  // staged rows per chunk (upper bound of r_hi - r_lo)
+  float* stage = reinterpret_cast<float*>(dsm);      // [C][RM][OLD]
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&stage_bar, static_cast<uint32_t>(r_hi - r_lo) * OLD * 4u * C);
+    for (int r = r_lo; r < r_hi;) {                  // runs of rows within one query head
+      const int gr = row0 + r, jh = g * G + gr / a.H, ih = gr % a.H;
+      const int run = min(r_hi - r, a.H - ih);
+      for (int s2 = 0; s2 < C; ++s2)
+        bulk_g2s(stage + (static_cast<size_t>(s2) * RM + (r - r_lo)) * OLD,
+                 a.xscratch + ((static_cast<size_t>(b) * a.Hq + jh) * C + s2) * a.H * OLD + static_cast<size_t>(ih) * OLD,
+                 static_cast<uint32_t>(run) * OLD * 4u, &stage_bar);
+      r += run;
+    }
+  }
+  if (!mbar_wait(&stage_bar, 0, WAIT_LIMIT_NS) && tid == 0) report_timeout(a.status, 0x703);
+  if (tid == 0) TL(4);
+  const int nr = r_hi - r_lo;
+  if (tid < nr) {
+    float mv[16], lv[16];
+#pragma unroll
+    for (int s2 = 0; s2 < 16; ++s2) {
+      if (s2 < C) {
+        const float2 ml = *reinterpret_cast<const float2*>(stage + (static_cast<size_t>(s2) * RM + tid) * OLD + DH);
+        mv[s2] = ml.x;
+        lv[s2] = ml.y;
+      } else {
+        mv[s2] = -INFINITY;
+        lv[s2] = 0.f;
+      }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int s2 = 0; s2 < 16; ++s2) M = fmaxf(M, mv[s2]);
+    float den = 0.f;
+#pragma unroll
+    for (int s2 = 0; s2 < 16; ++s2) {
+      if (s2 < C) {
+        const float e = exp2f(mv[s2] - M);
+        w_sh[s2][tid] = e;
+        den += e * lv[s2];
+      }
+    }
+    inv_den[tid] = 1.0f / den;
+  }
+  __syncthreads();
+  if (tid == 0) TL(7);
+  // 16 output features per work item: (owned row, 16-feature group)
+  for (int it = tid; it < nr * (DH / 16); it += UA_THREADS) {
+    const int rq = it / (DH / 16), d0 = (it % (DH / 16)) * 16;
+    const int gr = row0 + r_lo + rq, jh = g * G + gr / a.H, ih = gr % a.H;
+    float acc[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int s2 = 0; s2 < 16; ++s2)
+      if (s2 < C) {
+        const float w = w_sh[s2][rq];
+        const float* src = stage + (static_cast<size_t>(s2) * RM + rq) * OLD + d0;
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(src + e);
+          acc[e] += w * v.x;   // rank order
+          acc[e + 1] += w * v.y;
+          acc[e + 2] += w * v.z;
+          acc[e + 3] += w * v.w;
+        }
+      }
+    const float id = inv_den[rq];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[e] *= id;
+    store16(b * a.H + ih, jh, d0, acc);
   }
   __syncthreads();
   if (tid == 0) TL(5);
@@ -971,10 +1431,10 @@ size_t attn_scratch_bytes(int B, int Hq, int C, int H, int dh) {
 }
 
 size_t attn_smem_bytes(int H, int dh, int KC, int C) {
-  const AttnGeom g = attn_geom(H, dh, KC, C);
-  const size_t compute = static_cast<size_t>(g.q_bytes) + g.kv_bytes;
-  const size_t merge = C > 1 ? static_cast<size_t>(C) * g.R * g.rowb : g.obuf_bytes;
-  return compute > merge ? compute : merge;
+  (void)H;
+  (void)KC;
+  (void)C;
+  return uattn_geom(dh).total;   // the merge stage (<= 144 rows x (dh + 4) floats) overlays it
 }
 
 cudaError_t tc_kernels_init() {
@@ -982,8 +1442,8 @@ cudaError_t tc_kernels_init() {
   int dev = 0, optin = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
-  const void* fns[] = {reinterpret_cast<const void*>(k_gemm_tc), reinterpret_cast<const void*>(k_attn_tc<64>),
-                       reinterpret_cast<const void*>(k_attn_tc<128>), reinterpret_cast<const void*>(k_attn_tc<256>),
+  const void* fns[] = {reinterpret_cast<const void*>(k_gemm_tc), reinterpret_cast<const void*>(k_attn_umma<64>),
+                       reinterpret_cast<const void*>(k_attn_umma<128>), reinterpret_cast<const void*>(k_attn_umma<256>),
                        reinterpret_cast<const void*>(k_inproj_tc), reinterpret_cast<const void*>(k_final_tc)};
   for (const void* f : fns) {
     cudaFuncAttributes fa;
@@ -1018,12 +1478,12 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int n_tiles, cudaStream_t s, bool 
 cudaError_t launch_attention_tc(const AttnArgs& a, int B, cudaStream_t s, bool pdl) {
   AttnArgs copy = a;
   void* args[] = {&copy};
-  const int Hp = (a.H + 15) & ~15;
-  const int nw = min(8, max(4, Hp / 16));
-  const void* f = a.dh == 64 ? reinterpret_cast<const void*>(k_attn_tc<64>)
-                : a.dh == 128 ? reinterpret_cast<const void*>(k_attn_tc<128>)
-                              : reinterpret_cast<const void*>(k_attn_tc<256>);
-  return launch_ex(f, dim3(a.C, a.Hq, B), dim3(32 * nw), attn_smem_bytes(a.H, a.dh, a.KC, a.C), s, pdl, a.C, args);
+  const void* f = a.dh == 64 ? reinterpret_cast<const void*>(k_attn_umma<64>)
+                : a.dh == 128 ? reinterpret_cast<const void*>(k_attn_umma<128>)
+                              : reinterpret_cast<const void*>(k_attn_umma<256>);
+  const int tiles = (a.Hq / a.Hkv * a.H + 127) / 128;
+  return launch_ex(f, dim3(a.C, a.Hkv * tiles, B), dim3(UA_THREADS), attn_smem_bytes(a.H, a.dh, a.KC, a.C), s, pdl,
+                   a.C, args);
 }
 
 cudaError_t launch_inproj_tc(const InprojArgs& a, cudaStream_t s, bool pdl) {

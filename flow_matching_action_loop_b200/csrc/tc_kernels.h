@@ -117,13 +117,29 @@ struct AttnArgs {
   float scale;                 // 1/sqrt(dh)
   float* xscratch;             // C > 1: partial rows [B][Hq][C][H][dh + 4] (O, max, sum), L2-resident scratch
   int o_rowmajor;              // 1: o is bf16 [B][H][Hq*dh] row-major instead of the tiled operand layout
+  unsigned* status;            // device status word (timeouts), or nullptr
 };
 
 // Key chunks of the split-KV attention over S keys: at most 16 (one cluster), each a multiple
-// of the 64-key online-softmax step.
+// of the 64-key sub-chunk.  This is the largest split; it sizes the merge scratch.
 inline void attn_chunks(int S, int& C, int& KC) {
   C = S < 16 * ATTN_SUBK ? (S + ATTN_SUBK - 1) / ATTN_SUBK : 16;
   const int per = (S + C - 1) / C;
+  KC = (per + ATTN_SUBK - 1) / ATTN_SUBK * ATTN_SUBK;
+  C = (S + KC - 1) / KC;
+}
+
+// Query-row tiles of the attention kernel: 128 rows of (query head, action row) per KV head.
+inline int attn_tiles(int B, int Hq, int Hkv, int H) { return B * Hkv * ((Hq / Hkv * H + 127) / 128); }
+
+// Key split actually launched: enough chunks to give every SM a CTA, never more than
+// attn_chunks allows (so its scratch bound holds).
+inline void attn_plan(int S, int tiles, int nsm, int& C, int& KC) {
+  int cmax = 1, kc = 64;
+  attn_chunks(S, cmax, kc);
+  int want = nsm / (tiles > 0 ? tiles : 1);
+  want = want < 1 ? 1 : (want > cmax ? cmax : want);
+  const int per = (S + want - 1) / want;
   KC = (per + ATTN_SUBK - 1) / ATTN_SUBK * ATTN_SUBK;
   C = (S + KC - 1) / KC;
 }

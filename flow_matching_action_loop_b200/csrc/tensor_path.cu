@@ -205,7 +205,7 @@ StepPlan make_plan(const TensorPath* tp, int B, int P) {
   p.o = choose_plan(tp->o.MB * p.NT, tp->o.NKC, p.Nt, B_ROWS, tp->fp8, tp->nsm, tp->max_dyn);
   p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, norm_kind, tp->fp8, tp->nsm, tp->max_dyn);
   p.dn = choose_plan(tp->dn.MB * p.NT, tp->dn.NKC, p.Nt, B_ROWS, tp->fp8, tp->nsm, tp->max_dyn);
-  attn_chunks(P + c.H, p.attn_C, p.attn_KC);
+  attn_plan(P + c.H, attn_tiles(B, c.Hq, c.Hkv, c.H), tp->nsm, p.attn_C, p.attn_KC);
   return p;
 }
 
@@ -337,6 +337,7 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       at.KC = p.attn_KC;
       at.scale = 1.0f / std::sqrt(static_cast<float>(c.dh));
       at.xscratch = tp->xscratch;
+      at.status = tp->tb.status;
       if ((e = launch_attention_tc(at, p.B, s, true)) != cudaSuccess) return cuda_fail(e, "attention launch");
       // O projection + residual (+ sum of squares for the pre-MLP norm)
       GemmArgs og = base_args(tp, p, tp->o, p.o, l, o_off);
