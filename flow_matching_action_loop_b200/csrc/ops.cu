@@ -140,7 +140,7 @@ extern "C" int fr_attention_noalloc(const void* q, const void* k, const void* v,
   if (g_noalloc_err[dev] != cudaSuccess) return cuda_fail(g_noalloc_err[dev], "cudaGetSymbolAddress(scratch)");
   // every scratch word the kernel reads is written earlier in the same launch: nothing to clear
   const tc::AttnArgs a =
-      attention_args(q, k, v, o, Hq, Hkv, H, S_keys, dh, static_cast<float*>(g_noalloc_ptr[dev]));
+      attention_args(q, k, v, o, B, Hq, Hkv, H, S_keys, dh, static_cast<float*>(g_noalloc_ptr[dev]));
   FR_CUDA(tc::launch_attention_tc(a, B, reinterpret_cast<cudaStream_t>(stream), false));
   return FR_OK;
 }
