@@ -218,6 +218,8 @@ def main(argv=None):
 
     inp = synthetic.make_inputs(cfg, 0)
     loop = ActionExpertLoop(cfg, device=local, path=args.path)
+    if args.path == 0 and cfg.dtype != "f32" and loop.path != "tensor":
+        raise SystemExit(f"{cfg.name}: the automatic kernel set is {loop.path!r}, expected the tensor path")
     loop.load_weights(inp["weights"])
     if cfg.dtype == "fp8":
         obs = synthetic.make_observation(cfg, 1)

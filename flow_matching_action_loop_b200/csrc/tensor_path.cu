@@ -488,15 +488,13 @@ bool tensor_path_supports(const fr_config& c) {
   if (c.D % 16 != 0 || (c.Hq * c.dh) % 16 != 0) return false; // 16-byte operand rows
   if (c.D > 2048 || c.A > 64) return false;                     // per-token kernels keep a row in registers
   if (static_cast<size_t>(c.D) * c.A * 2 > 160 * 1024) return false;   // in/out-proj weights fit shared memory
-  int C = 1, KC = 64;
-  attn_chunks(c.P_max + c.H, C, KC);
-  if (attn_smem_bytes(c.H, c.dh, KC, C) > 200 * 1024) return false;
+  if (attn_smem_bytes(c.H, c.dh, 64, 1) > 218 * 1024) return false;   // B200: 227 KB less the static part
   return true;
 }
 
 const char* tensor_path_limits() {
   return "bf16/fp8, dh in {64,128,256}, (Hq+Hkv)*dh/2 % 64 == 0, Hkv*dh % 128 == 0, F % 64 == 0, H <= 128, "
-         "D % 16 == 0, D <= 2048, A <= 64, attention chunk fits shared memory";
+         "D % 16 == 0, D <= 2048, A <= 64";
 }
 
 // Exchange scratch needed by any batch size up to B_max and any prefix length up to P_max.

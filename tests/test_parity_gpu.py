@@ -34,7 +34,9 @@ def _assert_close(cfg, got, want, label=""):
 
 
 def _paths(cfg):
-    return [FR_PATH_STEPWISE] if cfg.dtype == "f32" else [FR_PATH_STEPWISE, FR_PATH_AUTO]
+    # bf16/fp8 handles run both kernel sets; the tensor path is requested explicitly so that a
+    # configuration it does not support fails instead of silently running the stepwise kernels
+    return [FR_PATH_STEPWISE] if cfg.dtype == "f32" else [FR_PATH_STEPWISE, FR_PATH_TENSOR]
 
 
 SMALL = ["tiny_f32", "ragged_f32", "ragged_bf16", "mha_bf16", "minimal_bf16"]
@@ -209,6 +211,13 @@ def test_smaller_batch_and_prefix_than_the_handle_maximum():
     for path in _paths(cfg):
         got, loop = C.run_library(small, inp, path=path, B_max=cfg.B, P_max=cfg.P)
         _assert_close(small, got, want, f"path={loop.path}")
+        loop.close()
+
+
+def test_automatic_path_is_the_tensor_path_for_bf16_and_fp8():
+    for name in ("pi05_bf16_b1", "pi05_fp8_b1", "pi05_bf16_b32", "stress_bf16_b4", "ragged_bf16", "mha_bf16"):
+        loop = ActionExpertLoop(C.get_config(name), path=FR_PATH_AUTO)
+        assert loop.path == "tensor", (name, loop.path)
         loop.close()
 
 
