@@ -48,6 +48,12 @@ int check_attention(const void* q, const void* k, const void* v, const void* o, 
     set_error("fr_attention: needs dh in {64,128,256}, Hq %% Hkv == 0, H <= 128, H <= S_keys <= 32768");
     return FR_ERR_UNSUPPORTED;
   }
+  int C = 1, KC = 64;
+  tc::attn_chunks(S_keys, C, KC);
+  if (tc::attn_smem_bytes(H, dh, KC, C, 0) > 200 * 1024) {
+    set_error("fr_attention: a key chunk of %d keys does not fit shared memory", KC);
+    return FR_ERR_UNSUPPORTED;
+  }
   return FR_OK;
 }
 
@@ -68,7 +74,7 @@ tc::AttnArgs attention_args(const void* q, const void* k, const void* v, void* o
   a.dh = dh;
   int dev = 0, nsm = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  tc::attn_plan(S_keys, tc::attn_tiles(B, Hq, Hkv, H), nsm, a.C, a.KC);
+  a.umma = tc::attn_plan(S_keys, tc::attn_tiles(B, Hq, Hkv, H), nsm, a.C, a.KC);
   a.scale = 1.0f / std::sqrt(static_cast<float>(dh));
   a.xscratch = scratch;
   return a;

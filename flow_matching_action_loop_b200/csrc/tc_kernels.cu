@@ -1430,11 +1430,12 @@ size_t attn_scratch_bytes(int B, int Hq, int C, int H, int dh) {
   return C > 1 ? static_cast<size_t>(B) * Hq * C * H * (dh + 4) * 4 : 0;
 }
 
-size_t attn_smem_bytes(int H, int dh, int KC, int C) {
-  (void)H;
-  (void)KC;
-  (void)C;
-  return uattn_geom(dh).total;   // the merge stage (<= 144 rows x (dh + 4) floats) overlays it
+size_t attn_smem_bytes(int H, int dh, int KC, int C, int umma) {
+  if (umma) return uattn_geom(dh).total;   // the merge stage (<= 144 rows x (dh + 4) floats) overlays it
+  const AttnGeom g = attn_geom(H, dh, KC, C);
+  const size_t compute = static_cast<size_t>(g.q_bytes) + g.kv_bytes;
+  const size_t merge = C > 1 ? static_cast<size_t>(C) * g.R * g.rowb : g.obuf_bytes;
+  return compute > merge ? compute : merge;
 }
 
 cudaError_t tc_kernels_init() {
@@ -1442,7 +1443,9 @@ cudaError_t tc_kernels_init() {
   int dev = 0, optin = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
-  const void* fns[] = {reinterpret_cast<const void*>(k_gemm_tc), reinterpret_cast<const void*>(k_attn_umma<64>),
+  const void* fns[] = {reinterpret_cast<const void*>(k_gemm_tc), reinterpret_cast<const void*>(k_attn_tc<64>),
+                       reinterpret_cast<const void*>(k_attn_tc<128>), reinterpret_cast<const void*>(k_attn_tc<256>),
+                       reinterpret_cast<const void*>(k_attn_umma<64>),
                        reinterpret_cast<const void*>(k_attn_umma<128>), reinterpret_cast<const void*>(k_attn_umma<256>),
                        reinterpret_cast<const void*>(k_inproj_tc), reinterpret_cast<const void*>(k_final_tc)};
   for (const void* f : fns) {
@@ -1478,12 +1481,20 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int n_tiles, cudaStream_t s, bool 
 cudaError_t launch_attention_tc(const AttnArgs& a, int B, cudaStream_t s, bool pdl) {
   AttnArgs copy = a;
   void* args[] = {&copy};
-  const void* f = a.dh == 64 ? reinterpret_cast<const void*>(k_attn_umma<64>)
-                : a.dh == 128 ? reinterpret_cast<const void*>(k_attn_umma<128>)
-                              : reinterpret_cast<const void*>(k_attn_umma<256>);
-  const int tiles = (a.Hq / a.Hkv * a.H + 127) / 128;
-  return launch_ex(f, dim3(a.C, a.Hkv * tiles, B), dim3(UA_THREADS), attn_smem_bytes(a.H, a.dh, a.KC, a.C), s, pdl,
-                   a.C, args);
+  const size_t smem = attn_smem_bytes(a.H, a.dh, a.KC, a.C, a.umma);
+  if (a.umma) {
+    const void* f = a.dh == 64 ? reinterpret_cast<const void*>(k_attn_umma<64>)
+                  : a.dh == 128 ? reinterpret_cast<const void*>(k_attn_umma<128>)
+                                : reinterpret_cast<const void*>(k_attn_umma<256>);
+    const int tiles = (a.Hq / a.Hkv * a.H + 127) / 128;
+    return launch_ex(f, dim3(a.C, a.Hkv * tiles, B), dim3(UA_THREADS), smem, s, pdl, a.C, args);
+  }
+  const int Hp = (a.H + 15) & ~15;
+  const int nw = min(8, max(4, Hp / 16));
+  const void* f = a.dh == 64 ? reinterpret_cast<const void*>(k_attn_tc<64>)
+                : a.dh == 128 ? reinterpret_cast<const void*>(k_attn_tc<128>)
+                              : reinterpret_cast<const void*>(k_attn_tc<256>);
+  return launch_ex(f, dim3(a.C, a.Hq, B), dim3(32 * nw), smem, s, pdl, a.C, args);
 }
 
 cudaError_t launch_inproj_tc(const InprojArgs& a, cudaStream_t s, bool pdl) {

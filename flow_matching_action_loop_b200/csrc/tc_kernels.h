@@ -118,6 +118,7 @@ struct AttnArgs {
   float* xscratch;             // C > 1: partial rows [B][Hq][C][H][dh + 4] (O, max, sum), L2-resident scratch
   int o_rowmajor;              // 1: o is bf16 [B][H][Hq*dh] row-major instead of the tiled operand layout
   unsigned* status;            // device status word (timeouts), or nullptr
+  int umma;                    // 1: tcgen05 kernel over GQA-group tiles; 0: warp-MMA kernel per query head
 };
 
 // Key chunks of the split-KV attention over S keys: at most 16 (one cluster), each a multiple
@@ -132,16 +133,24 @@ inline void attn_chunks(int S, int& C, int& KC) {
 // Query-row tiles of the attention kernel: 128 rows of (query head, action row) per KV head.
 inline int attn_tiles(int B, int Hq, int Hkv, int H) { return B * Hkv * ((Hq / Hkv * H + 127) / 128); }
 
-// Key split actually launched: enough chunks to give every SM a CTA, never more than
-// attn_chunks allows (so its scratch bound holds).
-inline void attn_plan(int S, int tiles, int nsm, int& C, int& KC) {
+// Attention kernel and key split.  When even the largest split leaves SMs idle (batch-1 sizes)
+// the warp-MMA kernel runs, one CTA per (key chunk, query head), with attn_chunks' split;
+// otherwise the tcgen05 kernel runs with enough chunks to give every SM a CTA.  Either way
+// C <= attn_chunks' C, so the scratch bound holds.  Returns 1 for the tcgen05 kernel.
+inline int attn_plan(int S, int tiles, int nsm, int& C, int& KC) {
   int cmax = 1, kc = 64;
   attn_chunks(S, cmax, kc);
+  if (tiles * cmax < nsm) {
+    C = cmax;
+    KC = kc;
+    return 0;
+  }
   int want = nsm / (tiles > 0 ? tiles : 1);
   want = want < 1 ? 1 : (want > cmax ? cmax : want);
   const int per = (S + want - 1) / want;
   KC = (per + ATTN_SUBK - 1) / ATTN_SUBK * ATTN_SUBK;
   C = (S + KC - 1) / KC;
+  return 1;
 }
 
 struct InprojArgs {
@@ -182,7 +191,7 @@ cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaS
 size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk);
 size_t gemm_scratch_bytes(int NT, int MB, int S, int Nt);
 size_t attn_scratch_bytes(int B, int Hq, int C, int H, int dh);
-size_t attn_smem_bytes(int H, int dh, int KC, int C);
+size_t attn_smem_bytes(int H, int dh, int KC, int C, int umma);
 const void* inproj_kernel_ptr();
 const void* final_kernel_ptr();
 cudaError_t tc_kernels_init();    // function attributes (smem opt-in, carveout, non-portable clusters)

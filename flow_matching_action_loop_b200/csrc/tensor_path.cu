@@ -50,7 +50,7 @@ struct GemmPlan {
 struct StepPlan {
   int B = 0, P = 0, T = 0, NT = 0, Nt = 0;
   GemmPlan qkv, o, gu, dn;
-  int attn_C = 1, attn_KC = 64;
+  int attn_C = 1, attn_KC = 64, attn_umma = 0;
 };
 
 struct RetargetNode {
@@ -205,7 +205,7 @@ StepPlan make_plan(const TensorPath* tp, int B, int P) {
   p.o = choose_plan(tp->o.MB * p.NT, tp->o.NKC, p.Nt, B_ROWS, tp->fp8, tp->nsm, tp->max_dyn);
   p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, norm_kind, tp->fp8, tp->nsm, tp->max_dyn);
   p.dn = choose_plan(tp->dn.MB * p.NT, tp->dn.NKC, p.Nt, B_ROWS, tp->fp8, tp->nsm, tp->max_dyn);
-  attn_plan(P + c.H, attn_tiles(B, c.Hq, c.Hkv, c.H), tp->nsm, p.attn_C, p.attn_KC);
+  p.attn_umma = attn_plan(P + c.H, attn_tiles(B, c.Hq, c.Hkv, c.H), tp->nsm, p.attn_C, p.attn_KC);
   return p;
 }
 
@@ -338,6 +338,7 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       at.scale = 1.0f / std::sqrt(static_cast<float>(c.dh));
       at.xscratch = tp->xscratch;
       at.status = tp->tb.status;
+      at.umma = p.attn_umma;
       if ((e = launch_attention_tc(at, p.B, s, true)) != cudaSuccess) return cuda_fail(e, "attention launch");
       // O projection + residual (+ sum of squares for the pre-MLP norm)
       GemmArgs og = base_args(tp, p, tp->o, p.o, l, o_off);
@@ -488,13 +489,16 @@ bool tensor_path_supports(const fr_config& c) {
   if (c.D % 16 != 0 || (c.Hq * c.dh) % 16 != 0) return false; // 16-byte operand rows
   if (c.D > 2048 || c.A > 64) return false;                     // per-token kernels keep a row in registers
   if (static_cast<size_t>(c.D) * c.A * 2 > 160 * 1024) return false;   // in/out-proj weights fit shared memory
-  if (attn_smem_bytes(c.H, c.dh, 64, 1) > 218 * 1024) return false;   // B200: 227 KB less the static part
+  if (attn_smem_bytes(c.H, c.dh, 64, 1, 1) > 218 * 1024) return false;   // B200: 227 KB less the static part
+  int C = 1, KC = 64;
+  attn_chunks(c.P_max + c.H, C, KC);
+  if (attn_smem_bytes(c.H, c.dh, KC, C, 0) > 200 * 1024) return false;
   return true;
 }
 
 const char* tensor_path_limits() {
   return "bf16/fp8, dh in {64,128,256}, (Hq+Hkv)*dh/2 % 64 == 0, Hkv*dh % 128 == 0, F % 64 == 0, H <= 128, "
-         "D % 16 == 0, D <= 2048, A <= 64";
+         "D % 16 == 0, D <= 2048, A <= 64, attention chunk fits shared memory";
 }
 
 // Exchange scratch needed by any batch size up to B_max and any prefix length up to P_max.

@@ -1,4 +1,4 @@
-"""The split-KV attention kernel on its own (fr_attention) against the oracle's attention.
+"""The split-KV attention kernels on their own (fr_attention) against the oracle's attention.
 
 Tolerance per (sample, query head): relative L2 <= 1e-2 and cosine >= 0.9999 -- the output is
 rounded to bf16 and P is rounded to bf16 inside the kernel (flash-attention practice).
@@ -25,6 +25,9 @@ CASES = [
     (3, 16, 2, 100, 2148, 128), # stress shapes: 12 chunks of 192
     (1, 1, 1, 1, 2, 128),       # one query row, one chunk (no cluster)
     (1, 4, 1, 128, 900, 64),    # largest query count
+    # batched shapes run the tcgen05 kernel (query tiles x key chunks fill the SMs)
+    (40, 2, 2, 50, 66, 128),    # one chunk of two sub-chunks, the second of 2 keys
+    (12, 8, 1, 50, 866, 256),   # 3 chunks of 5 sub-chunks: online softmax, O rescale, merge
 ]
 
 
