@@ -48,6 +48,13 @@ Readings where the pages are silent (each listed in the design notes):
       input per layer, from a calibration amax over all steps and tokens,
       s_a = amax/448); y = (s_a*s_w) * sum(a_q*w_q).  Everything else is as bf16.
   R12 f32 workloads round nothing.
+  R16 w4a16 workload (PhyAI page, optimisation paragraph: W4A16 among the
+      offline quantisation schemes; the pages give no group size): each of the
+      four layer projections is stored per output row in groups of 128
+      consecutive input features as 4-bit integers q in [-7, 7] with one bf16
+      scale per group, s = bf16(max|w| / 7), q = clamp(round-half-even(w / s));
+      the tensor-core operand is the dequantised weight bf16(q * s).
+      Projection inputs are bf16 as in R10; everything else is as bf16.
 """
 from __future__ import annotations
 
@@ -57,6 +64,8 @@ from typing import Callable, Dict, List, Optional
 import numpy as np
 
 E4M3_MAX = 448.0
+W4_GROUP = 128     # input features per 4-bit scale group (R16)
+W4_QMAX = 7        # symmetric 4-bit range [-7, 7] (R16)
 PROJ_INPUTS = ("qkv", "o", "gu", "down")   # the four FP8 projection inputs per layer
 
 
@@ -85,6 +94,35 @@ def round_e4m3(x) -> np.ndarray:
     lead = np.maximum(e - 1, -6)             # exponent of the leading bit, subnormals at -6
     quantum = np.ldexp(1.0, lead - 3)        # 3 fraction bits
     return np.sign(x) * np.rint(ax / quantum) * quantum
+
+
+def quantize_w4(w, group: int = W4_GROUP):
+    """4-bit group quantisation of a [rows][cols] weight (R16).
+
+    Per row and per group of `group` consecutive columns: s = bf16(max|w| / 7) and
+    q = clamp(round-half-even(w / s), -7, 7); an all-zero group has s = 0, q = 0.
+    Returns q (int8 [rows][cols]) and s (float64 [rows][ceil(cols / group)]).
+    """
+    w = np.asarray(w, dtype=np.float64)
+    rows, cols = w.shape
+    ng = -(-cols // group)
+    q = np.zeros((rows, cols), dtype=np.int8)
+    s = np.zeros((rows, ng), dtype=np.float64)
+    for g in range(ng):
+        blk = w[:, g * group:(g + 1) * group]
+        sg = round_bf16(np.max(np.abs(blk), axis=1) / W4_QMAX)
+        s[:, g] = sg
+        safe = np.where(sg > 0, sg, 1.0)[:, None]
+        r = np.where(sg[:, None] > 0, blk / safe, 0.0)
+        q[:, g * group:(g + 1) * group] = np.clip(np.rint(r), -W4_QMAX, W4_QMAX).astype(np.int8)
+    return q, s
+
+
+def dequantize_w4(q, s, group: int = W4_GROUP):
+    """The tensor-core operand of a 4-bit weight: bf16(q * s) per element (R16)."""
+    q = np.asarray(q, dtype=np.float64)
+    rep = np.repeat(np.asarray(s, dtype=np.float64), group, axis=1)[:, :q.shape[1]]
+    return round_bf16(q * rep)
 
 
 def decode_e4m3(code: int) -> float:
@@ -231,6 +269,7 @@ class PreparedModel:
     four layer projections are additionally held as e4m3 values w_q on the grid
     of w / s_w with one s_w per fused projection (PhyAI page: fused QKV, merged
     gate/up; FlashRT walkthrough, component 4: FP8 quantisation with scales).
+    For w4a16 they are held as their dequantised 4-bit values bf16(q * s) (R16).
     """
 
     def __init__(self, cfg, weights: dict):
@@ -258,6 +297,9 @@ class PreparedModel:
                     d["sw_" + name] = s_w
                     for p in parts:
                         d[p] = round_e4m3(np.asarray(lw[p], np.float64) / s_w)   # codes' values
+            elif cfg.dtype == "w4a16":
+                for p in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
+                    d[p] = dequantize_w4(*quantize_w4(lw[p]))
             else:
                 for p in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
                     d[p] = rnd(lw[p])

@@ -35,8 +35,9 @@ __all__ = ["ActionExpertConfig", "CONFIGS", "make_inputs", "make_noise", "make_p
 class ActionExpertConfig:
     """Sizes of one action-expert workload.
 
-    dtype is the arithmetic format of the layer projections: "f32", "bf16" or
-    "fp8" (e4m3 weights and projection inputs).
+    dtype is the arithmetic format of the layer projections: "f32", "bf16",
+    "fp8" (e4m3 weights and projection inputs) or "w4a16" (4-bit weights with a
+    scale per group of input features, bf16 projection inputs).
     """
 
     name: str
@@ -82,6 +83,9 @@ CONFIGS: Dict[str, ActionExpertConfig] = {
     # throughput regime: 32 independent chunks
     "pi05_bf16_b32": ActionExpertConfig("pi05_bf16_b32", L=18, D=1024, Hq=8, Hkv=1, dh=256,
                                         F=4096, H=50, A=32, B=32, P=816, K=10, dtype="bf16"),
+    # same with 4-bit weights (group scales) and bf16 projection inputs
+    "pi05_w4a16_b1": ActionExpertConfig("pi05_w4a16_b1", L=18, D=1024, Hq=8, Hkv=1, dh=256,
+                                        F=4096, H=50, A=32, B=1, P=816, K=10, dtype="w4a16"),
     # larger stress variant
     "stress_bf16_b4": ActionExpertConfig("stress_bf16_b4", L=18, D=2048, Hq=16, Hkv=2, dh=128,
                                          F=8192, H=100, A=32, B=4, P=2048, K=10, dtype="bf16"),

@@ -178,7 +178,7 @@ def test_velocity_matches_loop_formulation():
 
 # ---------------------------------------------------------------- loop closed forms
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "fp8", "w4a16"])
 def test_zero_network_leaves_x_unchanged(dtype):
     cfg = MICRO.replace(dtype=dtype)
     inp = synthetic.make_inputs(cfg, seed=2)
@@ -195,7 +195,7 @@ def test_zero_network_leaves_x_unchanged(dtype):
     assert np.array_equal(out, inp["x0"].astype(np.float64))
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "w4a16"])
 def test_constant_field_moves_x_by_minus_c(dtype):
     cfg = MICRO.replace(dtype=dtype, K=10)
     inp = synthetic.make_inputs(cfg, seed=2)
@@ -257,6 +257,31 @@ def test_fp8_projection_exact_on_representable_operands():
     a = codes[None, :cfg.Hq * cfg.dh] * s_a
     (y,) = O._project(model, 0, "o", a, (lay["wo"],), {(0, "o"): s_a}, None)
     assert np.allclose(y, a @ (lay["wo"] * s_w).T, rtol=1e-13)
+
+
+def test_w4a16_on_grid_weights_reduce_to_the_bf16_workload():
+    """Layer weights already on the 4-bit grid (power-of-two group scales, a +-7 code in every
+    group) dequantise to themselves, so the w4a16 loop must equal the bf16 loop bit for bit."""
+    cfg = MICRO.replace(D=16, F=16, dh=4, Hq=4, Hkv=2, time_dim=8, dtype="bf16")
+    inp = synthetic.make_inputs(cfg, seed=11)
+    w = inp["weights"]
+    rng = np.random.default_rng(12)
+    for lw in w["layers"]:
+        for key in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
+            rows, cols = lw[key].shape
+            k = rng.integers(-7, 8, size=(rows, cols))
+            k[:, 0] = 7                                              # max |k| = 7 in each (single) group
+            scale = 2.0 ** rng.integers(-8, -3, size=(rows, 1))
+            lw[key] = (k * scale).astype(np.float32)
+    a = O.denoise(cfg, w, inp["prefix_k"], inp["prefix_v"], inp["x0"])
+    b = O.denoise(cfg.replace(dtype="w4a16"), w, inp["prefix_k"], inp["prefix_v"], inp["x0"])
+    assert np.array_equal(a, b)
+    # and off the grid the two differ, by about the 4-bit step
+    w2 = synthetic.make_inputs(cfg, seed=11)["weights"]
+    a2 = O.denoise(cfg, w2, inp["prefix_k"], inp["prefix_v"], inp["x0"])
+    b2 = O.denoise(cfg.replace(dtype="w4a16"), w2, inp["prefix_k"], inp["prefix_v"], inp["x0"])
+    rel = np.linalg.norm(a2 - b2) / np.linalg.norm(a2 - inp["x0"])
+    assert 1e-3 < rel < 0.5
 
 
 def test_calibration_scales_cover_every_projection_input():

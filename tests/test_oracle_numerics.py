@@ -217,3 +217,61 @@ def test_rope_tables_float32_rounding_once():
     # a position with a large angle still matches float64 math rounded once
     inv = 1e4 ** (-2 * 3 / 256)
     assert c[865, 3] == np.float32(math.cos(865 * inv))
+
+
+# ---------------------------------------------------------------- 4-bit group weights (R16)
+
+def test_w4_quantiser_closed_forms():
+    rng = np.random.default_rng(7)
+    w = (rng.standard_normal((6, 300)) / 17.0).astype(np.float32)   # ragged last group: 300 = 2 x 128 + 44
+    q, s = O.quantize_w4(w)
+    assert q.dtype == np.int8 and s.shape == (6, 3)
+    assert q.min() >= -7 and q.max() <= 7
+    for r in range(6):
+        for g in range(3):
+            blk = w[r, g * 128:(g + 1) * 128].astype(np.float64)
+            amax = np.max(np.abs(blk))
+            # the scale is amax / 7 rounded to bf16 (torch's RNE conversion, an independent rounding)
+            assert s[r, g] == torch.tensor(amax / 7.0, dtype=torch.float64).to(torch.bfloat16).double().item()
+            qb = q[r, g * 128:(g + 1) * 128].astype(np.float64)
+            # every code is the nearest integer to w / s (ties to even), clamped: |w/s - q| <= 1/2 inside the range
+            ratio = blk / s[r, g]
+            inside = np.abs(ratio) <= 7.0
+            assert np.all(np.abs(ratio[inside] - qb[inside]) <= 0.5)
+            assert np.all(np.abs(qb[~inside]) == 7)
+            # the largest magnitude lands at +-7: amax / s = 7 / (1 +- 2^-9) rounds to 7
+            k = int(np.argmax(np.abs(blk)))
+            assert abs(int(q[r, g * 128 + k])) == 7
+
+
+def test_w4_quantiser_special_cases():
+    # an all-zero group: zero scale, zero codes, zero operand
+    w = np.zeros((2, 256), np.float32)
+    w[1, 128:] = 1.0
+    q, s = O.quantize_w4(w)
+    assert s[0, 0] == 0 and s[0, 1] == 0 and s[1, 0] == 0 and not q[0].any() and not q[1, :128].any()
+    # a group of one repeated value v: s = bf16(v / 7); the codes all equal round(v / s) = 7
+    assert s[1, 1] == torch.tensor(1.0 / 7.0, dtype=torch.float64).to(torch.bfloat16).double().item()
+    assert np.all(q[1, 128:] == 7)
+    # exact grid: w = k * s0 with a power-of-two s0 and integer k in [-7, 7] comes back exactly
+    s0 = 2.0 ** -5
+    ks = np.tile(np.arange(-7, 8), 10)[:128]
+    ks[0] = 7                                   # make max|w| = 7 s0 so that s = s0 exactly
+    w = (ks * s0).astype(np.float32)[None, :]
+    q, s = O.quantize_w4(w)
+    assert s[0, 0] == s0 and np.array_equal(q[0], ks)
+    assert np.array_equal(O.dequantize_w4(q, s)[0], ks * s0)
+
+
+def test_w4_dequantised_operand_is_bf16_of_the_exact_product():
+    rng = np.random.default_rng(8)
+    w = (rng.standard_normal((4, 256)) * 0.05).astype(np.float32)
+    q, s = O.quantize_w4(w)
+    deq = O.dequantize_w4(q, s)
+    # q * s (3 magnitude bits times an 8-bit bf16 significand) is exact in float32, so torch's
+    # float32 -> bf16 conversion of the float32 product is the same single rounding
+    prod32 = torch.from_numpy(q.astype(np.float32)) * torch.from_numpy(np.repeat(s, 128, axis=1).astype(np.float32))
+    assert np.array_equal(deq, prod32.to(torch.bfloat16).double().numpy())
+    # and the operand stays within half a code step plus one bf16 rounding of w
+    step = np.repeat(s, 128, axis=1)
+    assert np.all(np.abs(deq - w) <= 0.5 * step + np.abs(deq) * 2.0 ** -8 + 1e-30)
