@@ -34,11 +34,15 @@ UNIT = "us/chunk"
 
 def workload_bytes(cfg) -> dict:
     """Algorithmic bytes of one chunk: weights streamed once per Euler step plus the KV read per step."""
-    wb = {"f32": 4, "bf16": 2, "fp8": 1}[cfg.dtype]
     D, F, dq, nkv = cfg.D, cfg.F, cfg.Hq * cfg.dh, cfg.Hkv * cfg.dh
     layer_w = (dq + 2 * nkv) * D + D * dq + 2 * F * D + D * F
+    if cfg.dtype == "w4a16":   # half a byte per weight plus a bf16 scale per 128 inputs of each row
+        rows_k = [((dq + 2 * nkv), D), (D, dq), (2 * F, D), (D, F)]
+        layer_bytes = layer_w // 2 + sum(r * -(-k // 128) * 2 for r, k in rows_k)
+    else:
+        layer_bytes = layer_w * {"f32": 4, "bf16": 2, "fp8": 1}[cfg.dtype]
     small = 2 * (cfg.D * cfg.A * 2 + 3 * cfg.D * 4) + cfg.A * 4   # in/out-proj (bf16) + gains/biases
-    w_step = cfg.L * (layer_w * wb + 2 * D * 4) + small
+    w_step = cfg.L * (layer_bytes + 2 * D * 4) + small
     kv_step = cfg.L * cfg.B * cfg.Hkv * (cfg.P + cfg.H) * cfg.dh * 2 * (4 if cfg.dtype == "f32" else 2)
     return {"weights_per_step": w_step, "kv_per_step": kv_step, "per_chunk": cfg.K * (w_step + kv_step),
             "weights_per_chunk": cfg.K * w_step}

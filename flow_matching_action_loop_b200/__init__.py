@@ -17,12 +17,12 @@ from typing import Optional
 import numpy as np
 
 from ._abi import (  # noqa: F401
-    DTYPES, FR_DTYPE_BF16, FR_DTYPE_F32, FR_DTYPE_FP8, FR_ERR_ARG, FR_ERR_CUDA, FR_ERR_DEVICE, FR_ERR_SHAPE,
+    DTYPES, FR_DTYPE_BF16, FR_DTYPE_F32, FR_DTYPE_FP8, FR_DTYPE_W4A16, FR_ERR_ARG, FR_ERR_CUDA, FR_ERR_DEVICE, FR_ERR_SHAPE,
     FR_ERR_STATE, FR_ERR_TIMEOUT, FR_ERR_UNSUPPORTED, FR_OK, FR_PATH_AUTO, FR_PATH_STEPWISE, FR_PATH_TENSOR,
     FR_ATTENTION_NOALLOC_SCRATCH_BYTES, FR_PREFIX_K_ROTATED, FrConfig, FrError, fr_attention,
     fr_attention_noalloc, fr_attention_scratch_bytes, fr_calibrate, fr_create,
     fr_denoise, fr_destroy, fr_get_rope_tables,
-    fr_get_scales, fr_last_error, fr_launches_per_call, fr_load_weights, fr_path_name, fr_quantize_e4m3,
+    fr_get_scales, fr_last_error, fr_launches_per_call, fr_load_weights, fr_path_name, fr_quantize_e4m3, fr_quantize_w4,
     fr_read_kv, fr_rope_tables, fr_round_bf16, fr_set_prefix_kv, fr_set_scales, fr_sync_status, header_functions,
     load_library, make_config,
 )

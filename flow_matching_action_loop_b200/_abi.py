@@ -19,10 +19,11 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "fr.h")
 
 FR_OK = 0
 FR_ERR_ARG, FR_ERR_SHAPE, FR_ERR_STATE, FR_ERR_CUDA, FR_ERR_TIMEOUT, FR_ERR_DEVICE, FR_ERR_UNSUPPORTED = range(-1, -8, -1)
-FR_DTYPE_F32, FR_DTYPE_BF16, FR_DTYPE_FP8 = 0, 1, 2
+FR_DTYPE_F32, FR_DTYPE_BF16, FR_DTYPE_FP8, FR_DTYPE_W4A16 = 0, 1, 2, 3
+FR_W4_GROUP = 128
 FR_PATH_AUTO, FR_PATH_STEPWISE, FR_PATH_TENSOR = 0, 1, 2
 FR_PREFIX_K_ROTATED = 1
-DTYPES = {"f32": FR_DTYPE_F32, "bf16": FR_DTYPE_BF16, "fp8": FR_DTYPE_FP8}
+DTYPES = {"f32": FR_DTYPE_F32, "bf16": FR_DTYPE_BF16, "fp8": FR_DTYPE_FP8, "w4a16": FR_DTYPE_W4A16}
 ERR_NAMES = {FR_ERR_ARG: "FR_ERR_ARG", FR_ERR_SHAPE: "FR_ERR_SHAPE", FR_ERR_STATE: "FR_ERR_STATE",
              FR_ERR_CUDA: "FR_ERR_CUDA", FR_ERR_TIMEOUT: "FR_ERR_TIMEOUT", FR_ERR_DEVICE: "FR_ERR_DEVICE",
              FR_ERR_UNSUPPORTED: "FR_ERR_UNSUPPORTED"}
@@ -97,6 +98,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                          c_int, c_void_p]),
         "fr_round_bf16": (None, [_FP, ctypes.POINTER(ctypes.c_uint16), ctypes.c_size_t]),
         "fr_quantize_e4m3": (None, [_FP, ctypes.POINTER(ctypes.c_uint8), ctypes.c_size_t, ctypes.c_double]),
+        "fr_quantize_w4": (c_int, [_FP, c_int, c_int, ctypes.POINTER(ctypes.c_int8), ctypes.POINTER(ctypes.c_uint16)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -252,3 +254,14 @@ def fr_quantize_e4m3(x, scale: float) -> np.ndarray:
     out = np.zeros(x.shape, np.uint8)
     load_library().fr_quantize_e4m3(_fptr(x), out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), x.size, scale)
     return out
+
+
+def fr_quantize_w4(w):
+    """4-bit codes [rows][cols] (int8) and bf16 scale bits [rows][groups] (uint16) of a 2-D weight."""
+    w = np.ascontiguousarray(np.asarray(w, np.float32))
+    rows, cols = w.shape
+    q = np.zeros((rows, cols), np.int8)
+    sb = np.zeros((rows, -(-cols // FR_W4_GROUP)), np.uint16)
+    _check(load_library().fr_quantize_w4(_fptr(w), rows, cols, q.ctypes.data_as(ctypes.POINTER(ctypes.c_int8)),
+                                          sb.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16))), "fr_quantize_w4")
+    return q, sb

@@ -92,7 +92,7 @@ int validate(const fr_config& c) {
     set_error("fr_create: every size must be positive");
     return FR_ERR_ARG;
   }
-  if (c.dtype < FR_DTYPE_F32 || c.dtype > FR_DTYPE_FP8 || c.path < FR_PATH_AUTO || c.path > FR_PATH_TENSOR) {
+  if (c.dtype < FR_DTYPE_F32 || c.dtype > FR_DTYPE_W4A16 || c.path < FR_PATH_AUTO || c.path > FR_PATH_TENSOR) {
     set_error("fr_create: bad dtype/path enum");
     return FR_ERR_ARG;
   }
@@ -105,7 +105,7 @@ int validate(const fr_config& c) {
     return FR_ERR_UNSUPPORTED;
   }
   if (c.path == FR_PATH_TENSOR && c.dtype == FR_DTYPE_F32) {
-    set_error("fr_create: the tensor-core path needs a bf16 or fp8 handle");
+    set_error("fr_create: the tensor-core path needs a bf16, fp8 or w4a16 handle");
     return FR_ERR_UNSUPPORTED;
   }
   return FR_OK;
@@ -113,7 +113,7 @@ int validate(const fr_config& c) {
 
 int qmode_of(const fr_handle* h, bool measure) {
   if (h->cfg.dtype == FR_DTYPE_F32) return Q_NONE;
-  if (h->cfg.dtype == FR_DTYPE_BF16) return Q_BF16;
+  if (h->cfg.dtype == FR_DTYPE_BF16 || h->cfg.dtype == FR_DTYPE_W4A16) return Q_BF16;
   return measure ? Q_MEASURE : Q_E4M3;
 }
 
@@ -173,6 +173,25 @@ void pack_rows(std::vector<uint8_t>& dst, size_t& off, const float* src, size_t 
   }
 }
 
+// w4a16: the 4-bit codes and scales of a [rows][cols] weight, then bf16(q * s) per element
+// (q * s is exact in float32: 3 magnitude bits times an 8-bit significand).
+void pack_w4_dequant(std::vector<uint8_t>& dst, size_t& off, const float* src, int rows, int cols) {
+  const int ng = (cols + FR_W4_GROUP - 1) / FR_W4_GROUP;
+  std::vector<int8_t> q(static_cast<size_t>(rows) * cols);
+  std::vector<uint16_t> sb(static_cast<size_t>(rows) * ng);
+  fr_quantize_w4(src, rows, cols, q.data(), sb.data());
+  std::vector<float> deq(q.size());
+  for (int r = 0; r < rows; ++r)
+    for (int c = 0; c < cols; ++c) {
+      const uint32_t u = static_cast<uint32_t>(sb[static_cast<size_t>(r) * ng + c / FR_W4_GROUP]) << 16;
+      float sv;
+      std::memcpy(&sv, &u, 4);
+      deq[static_cast<size_t>(r) * cols + c] = static_cast<float>(q[static_cast<size_t>(r) * cols + c]) * sv;
+    }
+  fr_round_bf16(deq.data(), reinterpret_cast<uint16_t*>(dst.data() + off), deq.size());
+  off += deq.size() * 2;
+}
+
 std::vector<float> rounded_f32(const float* src, size_t n, bool to_bf16) {
   std::vector<float> out(src, src + n);
   if (to_bf16) {
@@ -214,8 +233,9 @@ int fr_create(const fr_config* cfg, int device, fr_handle** out) {
   h->S_max = c.P_max + c.H;
   h->n_qkv = (c.Hq + 2 * c.Hkv) * c.dh;
   h->dq = c.Hq * c.dh;
-  h->wtype = c.dtype == FR_DTYPE_F32 ? W_F32 : (c.dtype == FR_DTYPE_BF16 ? W_BF16 : W_E4M3);
-  h->welem = c.dtype == FR_DTYPE_F32 ? 4 : (c.dtype == FR_DTYPE_BF16 ? 2 : 1);
+  // w4a16: the stepwise kernels read the dequantised operand bf16(q * s)
+  h->wtype = c.dtype == FR_DTYPE_F32 ? W_F32 : (c.dtype == FR_DTYPE_FP8 ? W_E4M3 : W_BF16);
+  h->welem = c.dtype == FR_DTYPE_F32 ? 4 : (c.dtype == FR_DTYPE_FP8 ? 1 : 2);
   h->kv_bf = c.dtype != FR_DTYPE_F32;
   h->path = c.path;
   if (h->path == FR_PATH_AUTO) h->path = (c.dtype == FR_DTYPE_F32) ? FR_PATH_STEPWISE : FR_PATH_TENSOR;
@@ -380,13 +400,24 @@ int fr_load_weights(fr_handle* h, const fr_weights* w, fr_stream_t stream) {
         h->h_sw[l * PI_COUNT + i] = static_cast<float>(sw[i]);
       }
     }
-    pack_rows(buf, off, L.wq, dq * D, h->wtype, sw[PI_QKV]);
-    pack_rows(buf, off, L.wk, nkv * D, h->wtype, sw[PI_QKV]);
-    pack_rows(buf, off, L.wv, nkv * D, h->wtype, sw[PI_QKV]);
-    pack_rows(buf, off, L.wo, D * dq, h->wtype, sw[PI_O]);
-    pack_rows(buf, off, L.wg, F * D, h->wtype, sw[PI_GU]);
-    pack_rows(buf, off, L.wu, F * D, h->wtype, sw[PI_GU]);
-    pack_rows(buf, off, L.wd, D * F, h->wtype, sw[PI_DOWN]);
+    if (c.dtype == FR_DTYPE_W4A16) {
+      const int iD = c.D, iF = c.F, idq = static_cast<int>(dq), inkv = static_cast<int>(nkv);
+      pack_w4_dequant(buf, off, L.wq, idq, iD);
+      pack_w4_dequant(buf, off, L.wk, inkv, iD);
+      pack_w4_dequant(buf, off, L.wv, inkv, iD);
+      pack_w4_dequant(buf, off, L.wo, iD, idq);
+      pack_w4_dequant(buf, off, L.wg, iF, iD);
+      pack_w4_dequant(buf, off, L.wu, iF, iD);
+      pack_w4_dequant(buf, off, L.wd, iD, iF);
+    } else {
+      pack_rows(buf, off, L.wq, dq * D, h->wtype, sw[PI_QKV]);
+      pack_rows(buf, off, L.wk, nkv * D, h->wtype, sw[PI_QKV]);
+      pack_rows(buf, off, L.wv, nkv * D, h->wtype, sw[PI_QKV]);
+      pack_rows(buf, off, L.wo, D * dq, h->wtype, sw[PI_O]);
+      pack_rows(buf, off, L.wg, F * D, h->wtype, sw[PI_GU]);
+      pack_rows(buf, off, L.wu, F * D, h->wtype, sw[PI_GU]);
+      pack_rows(buf, off, L.wd, D * F, h->wtype, sw[PI_DOWN]);
+    }
     FR_CUDA(cudaMemcpy(const_cast<void*>(h->lw[l].wqkv), buf.data(), bytes, cudaMemcpyHostToDevice));
     std::memcpy(&gains[2 * D * l], L.g1, D * 4);
     std::memcpy(&gains[2 * D * l + D], L.g2, D * 4);

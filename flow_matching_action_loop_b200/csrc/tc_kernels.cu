@@ -105,6 +105,8 @@ struct GemmSmem {
   uint64_t done;
   uint64_t hbar;      // residual rows of this CTA's tokens (EPI_RESID, S > 1)
   uint64_t xbar;      // split-K slices of this CTA's tokens (S > 1)
+  uint64_t raw_a[MAX_STAGES];   // w4: raw 4-bit chunk landed
+  uint64_t sbar;      // w4: the scales of this CTA's k-range landed
   uint32_t tmem_base;
   float rstd[NT_MAX];
   float ssq_part[2][4];
@@ -112,10 +114,17 @@ struct GemmSmem {
 
 struct GemmGeom {
   uint32_t a_bytes, breg, slot, raw_bytes, ring, gamma_off, recv_off;
+  uint32_t rawa_off, scl_off;   // w4: raw 4-bit chunks [stages][4 KB], bf16 scales [groups][128]
   int TS;
 };
 
-__host__ __device__ __forceinline__ GemmGeom gemm_geom(int Nt, int stages, int b_kind, int fp8, int S, int nk) {
+constexpr uint32_t W4_CHUNK = BM * KCB / 4;   // 4-bit codes of one 128 x 64 weight chunk (4 KB)
+
+// 4-bit scale groups (128 inputs = two 64-element chunks) touched by chunks kc0 .. kc0+nk-1
+__host__ __device__ __forceinline__ int w4_groups(int kc0, int nk) { return nk > 0 ? (kc0 + nk - 1) / 2 - kc0 / 2 + 1 : 0; }
+
+__host__ __device__ __forceinline__ GemmGeom gemm_geom(int Nt, int stages, int b_kind, int fp8, int S, int nk,
+                                                       int w4 = 0, int kc0 = 0) {
   GemmGeom g;
   g.a_bytes = BM * KCB;
   g.raw_bytes = (b_kind == B_NORM) ? static_cast<uint32_t>(Nt) * 256u * (fp8 ? 2u : 1u) : 0u;
@@ -123,24 +132,29 @@ __host__ __device__ __forceinline__ GemmGeom gemm_geom(int Nt, int stages, int b
   g.breg = tile > g.raw_bytes ? tile : g.raw_bytes;
   g.slot = g.a_bytes + g.breg;
   g.ring = g.slot * static_cast<uint32_t>(stages);
-  g.gamma_off = g.ring;   // B_NORM: gamma of this CTA's k-range (nk * kel floats)
   g.TS = (Nt + S - 1) / S;
   // S > 1: residual rows (2 x TS x 64 floats) live past the ring, the gamma slice and the
   // split-K slices: they land while the ring is still in use and are read after the split-K
   // slices (S x TS x 128 floats, overlaying the ring from offset 0) have landed.
   const uint32_t kel = fp8 ? KCB : KCB / 2;
-  const uint32_t main_end = g.ring + (b_kind == B_NORM ? static_cast<uint32_t>(nk) * kel * 4u : 0u);
+  g.rawa_off = g.ring;
+  g.scl_off = g.rawa_off + (w4 ? static_cast<uint32_t>(stages) * W4_CHUNK : 0u);
+  // scale groups of any k-range of nk chunks: at most nk/2 + 1 (one more when kc0 is odd)
+  const uint32_t scl_bytes = w4 ? static_cast<uint32_t>(w4_groups(kc0, nk) > nk / 2 + 1 ? w4_groups(kc0, nk) : nk / 2 + 1) * BM * 2u : 0u;
+  g.gamma_off = (g.scl_off + scl_bytes + 15u) & ~15u;
+  const uint32_t main_end = g.gamma_off + (b_kind == B_NORM ? static_cast<uint32_t>(nk) * kel * 4u : 0u);
   const uint32_t slices_end = S > 1 ? static_cast<uint32_t>(S) * g.TS * BM * 4u : 0u;
   g.recv_off = ((main_end > slices_end ? main_end : slices_end) + 1023u) & ~1023u;
   return g;
 }
 
+template <int EPI, int FP8, int NORM, int W4>
 __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_constant__ GemmArgs a) {
   extern __shared__ __align__(1024) uint8_t dsm[];
   __shared__ GemmSmem sh;
   TL_DECL
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  TL_BEGIN(10 + a.epi);
+  TL_BEGIN(10 + EPI);
   const int ks = blockIdx.x;            // split-K rank (= cluster rank)
   const int mb = blockIdx.y;            // m-block
   const int nt = blockIdx.z;            // n-tile
@@ -150,14 +164,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   const int kc0 = ks * a.NKC / S, kc1 = (ks + 1) * a.NKC / S;
   const int nk = kc1 - kc0;
   const int stages = a.stages;
-  const int norm = a.b_kind == B_NORM;
-  const int kel = a.fp8 ? KCB : KCB / 2;            // K elements per chunk
-  const GemmGeom gm = gemm_geom(Nt, stages, a.b_kind, a.fp8, S, nk);
+  constexpr int norm = NORM;
+  const int kel = FP8 ? KCB : KCB / 2;            // K elements per chunk
+  const GemmGeom gm = gemm_geom(Nt, stages, NORM ? B_NORM : B_ROWS, FP8, S, nk, W4, kc0);
+  const int g0 = kc0 / 2;                          // w4: first scale group of this CTA's k-range
   float* gsm = reinterpret_cast<float*>(dsm + gm.gamma_off);
 
   if (tid == 0) {
     for (int s = 0; s < stages; ++s) {
-      mbar_init(&sh.full_a[s], 1);
+      mbar_init(&sh.full_a[s], W4 ? CONV_THREADS : 1);   // w4: the converters hand each chunk over
+      mbar_init(&sh.raw_a[s], 1);
       mbar_init(&sh.full_b[s], norm ? CONV_THREADS : 1);
       mbar_init(&sh.raw_b[s], 1);
       mbar_init(&sh.empty[s], 1);
@@ -165,6 +181,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
     mbar_init(&sh.done, 1);
     mbar_init(&sh.hbar, 1);
     mbar_init(&sh.xbar, 1);
+    mbar_init(&sh.sbar, 1);
     fence_mbar_init();
   }
   uint32_t ncols = 32;
@@ -187,7 +204,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         const int s = i % stages;
         uint8_t* bdst = dsm + s * gm.slot + gm.a_bytes;
         if (norm) {
-          const int kb = (kc0 + i) * (a.fp8 ? 2 : 1);
+          const int kb = (kc0 + i) * (FP8 ? 2 : 1);
           mbar_arrive_expect_tx(&sh.raw_b[s], gm.raw_bytes);
           bulk_g2s(bdst, a.h + (static_cast<size_t>(nt) * a.KB + kb) * Nt * 64, gm.raw_bytes, &sh.raw_b[s]);
         } else {
@@ -196,15 +213,28 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
           bulk_g2s(bdst, a.act + (static_cast<size_t>(nt) * a.NKC + kc0 + i) * tb, tb, &sh.full_b[s]);
         }
       };
+      const uint8_t* w4src = a.W + (static_cast<size_t>(mb) * a.NKC + kc0) * W4_CHUNK;
+      auto issue_a = [&](int i) {
+        const int s = i % stages;
+        if (W4) {
+          mbar_arrive_expect_tx(&sh.raw_a[s], W4_CHUNK);
+          bulk_g2s(dsm + gm.rawa_off + s * W4_CHUNK, w4src + static_cast<size_t>(i) * W4_CHUNK, W4_CHUNK, &sh.raw_a[s]);
+        } else {
+          mbar_arrive_expect_tx(&sh.full_a[s], gm.a_bytes);
+          bulk_g2s(dsm + s * gm.slot, wsrc + static_cast<size_t>(i) * gm.a_bytes, gm.a_bytes, &sh.full_a[s]);
+        }
+      };
       const int pre = nk < stages ? nk : stages;
-      for (int i = 0; i < pre; ++i) {   // weights first: they do not depend on the previous kernel
-        mbar_arrive_expect_tx(&sh.full_a[i], gm.a_bytes);
-        bulk_g2s(dsm + i * gm.slot, wsrc + static_cast<size_t>(i) * gm.a_bytes, gm.a_bytes, &sh.full_a[i]);
+      if (W4) {   // the scales of this CTA's groups, one copy
+        const uint32_t sb = static_cast<uint32_t>(w4_groups(kc0, nk)) * BM * 2u;
+        mbar_arrive_expect_tx(&sh.sbar, sb);
+        bulk_g2s(dsm + gm.scl_off, a.Wscale + (static_cast<size_t>(mb) * ((a.NKC + 1) / 2) + g0) * BM, sb, &sh.sbar);
       }
+      for (int i = 0; i < pre; ++i) issue_a(i);   // weights first: they do not depend on the previous kernel
       grid_dep_wait();
       TL(1);
       for (int i = 0; i < pre; ++i) issue_b(i);
-      if (S > 1 && a.epi == EPI_RESID) {   // residual rows of this CTA's tokens, for the epilogue
+      if (S > 1 && EPI == EPI_RESID) {   // residual rows of this CTA's tokens, for the epilogue
         const int r0 = ks * Nt / S, r1 = (ks + 1) * Nt / S;
         const uint32_t rb = static_cast<uint32_t>(r1 - r0) * 256u;
         float* hst = reinterpret_cast<float*>(dsm + gm.recv_off);
@@ -220,8 +250,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
           report_timeout(a.status, 0x100);
           break;
         }
-        mbar_arrive_expect_tx(&sh.full_a[s], gm.a_bytes);
-        bulk_g2s(dsm + s * gm.slot, wsrc + static_cast<size_t>(i) * gm.a_bytes, gm.a_bytes, &sh.full_a[s]);
+        issue_a(i);
         issue_b(i);
         issued = i + 1;
       }
@@ -229,14 +258,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       for (int i = (issued > stages ? issued - stages : 0); i < issued; ++i) {
         const int s = i % stages;
         const uint32_t par = (i / stages) & 1;
-        mbar_wait(&sh.full_a[s], par, WAIT_LIMIT_NS);
+        mbar_wait(W4 ? &sh.raw_a[s] : &sh.full_a[s], par, WAIT_LIMIT_NS);
         mbar_wait(norm ? &sh.raw_b[s] : &sh.full_b[s], par, WAIT_LIMIT_NS);
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_f32acc(a.fp8 ? FMT_E4M3 : FMT_BF16, BM, Nt);
+      const uint32_t idesc = idesc_f32acc(FP8 ? FMT_E4M3 : FMT_BF16, BM, Nt);
       for (int i = 0; i < nk; ++i) {
         const int s = i % stages;
         const uint32_t par = (i / stages) & 1;
@@ -251,7 +280,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         for (int k = 0; k < KCB / 32; ++k) {
           const uint64_t ad = smem_desc(a0 + k * 2 * BM * 16, BM * 16, 128);
           const uint64_t bd = smem_desc(b0 + k * 2 * Nt * 16, Nt * 16, 128);
-          if (a.fp8) mma_e4m3(tacc, ad, bd, idesc, (i | k) != 0);
+          if (FP8) mma_e4m3(tacc, ad, bd, idesc, (i | k) != 0);
           else mma_bf16(tacc, ad, bd, idesc, (i | k) != 0);
         }
         mma_commit(&sh.empty[s]);
@@ -259,9 +288,39 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       mma_commit(&sh.done);
       TL(2);
     }
-  } else if (norm || a.rscale) {
-    // ---------------- warps 2-7: per-token rstd; for B_NORM also RMSNorm(h)*gamma -> e4m3 / bf16 tile
+  } else if (norm || a.rscale || W4) {
+    // ---------------- warps 2-7: per-token rstd; for B_NORM also RMSNorm(h)*gamma -> e4m3 / bf16 tile;
+    // for 4-bit weights the A operand bf16(q * s) of every chunk
     const int st = tid - 64;
+    // w4: chunk i's codes (slab j, row r: 8 codes in 4 B) -> bf16(q * s) in the K-major A slot
+    auto convert_a = [&](int i) {
+      const int s = i % stages;
+      if (!mbar_wait(&sh.raw_a[s], (i / stages) & 1, WAIT_LIMIT_NS)) report_timeout(a.status, 0x310);
+      const uint32_t* raw = reinterpret_cast<const uint32_t*>(dsm + gm.rawa_off + s * W4_CHUNK);
+      const __nv_bfloat16* scl =
+          reinterpret_cast<const __nv_bfloat16*>(dsm + gm.scl_off) + ((kc0 + i) / 2 - g0) * BM;
+      uint8_t* adst = dsm + s * gm.slot;
+      for (int it = st; it < 8 * BM; it += CONV_THREADS) {
+        const int j = it >> 7, r = it & (BM - 1);     // consecutive threads: consecutive rows
+        const uint32_t wv = raw[it];
+        const float sc = __bfloat162float(scl[r]);
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float lo = static_cast<float>(static_cast<int>(wv << (28 - 8 * e)) >> 28) * sc;
+          const float hi = static_cast<float>(static_cast<int>(wv << (24 - 8 * e)) >> 28) * sc;
+          o[e] = pack_bf16x2(lo, hi);
+        }
+        *reinterpret_cast<uint4*>(adst + j * (BM * 16) + (r >> 3) * 128 + (r & 7) * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core
+      mbar_arrive(&sh.full_a[s]);
+    };
+    const int pre_a = nk < stages ? nk : stages;
+    if (W4) {   // static weights: convert what is resident before the dependency wait
+      if (!mbar_wait(&sh.sbar, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0x311);
+      for (int i = 0; i < pre_a; ++i) convert_a(i);
+    }
     if (norm) {
       for (int idx = st; idx < nk * kel; idx += CONV_THREADS) {   // static: before the dependency wait
         const int k = kc0 * kel + idx;
@@ -269,7 +328,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       }
     }
     grid_dep_wait();
-    for (int r = st; r < Nt; r += CONV_THREADS) {
+    for (int r = st; r < ((norm || a.rscale) ? Nt : 0); r += CONV_THREADS) {
       const int t = n0 + r;
       float rs = 0.f;
       if (t < a.T) {
@@ -288,7 +347,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       sh.rstd[r] = rs;   // padded tokens become zero
     }
     conv_sync();
-    const float inv_sa = (norm && a.fp8) ? 1.0f / *a.s_a : 1.0f;
+    if (W4)
+      for (int i = pre_a; i < nk; ++i) convert_a(i);
+    const float inv_sa = (norm && FP8) ? 1.0f / *a.s_a : 1.0f;
     for (int i = 0; i < (norm ? nk : 0); ++i) {
       const int s = i % stages;
       if (!mbar_wait(&sh.raw_b[s], (i / stages) & 1, WAIT_LIMIT_NS)) {
@@ -305,7 +366,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         if (it < Nt * 8) {
           const int r = it >> 3, j = it & 7;
           const float rs = sh.rstd[r];
-          if (!a.fp8) {
+          if (!FP8) {
             const float* p = raw + static_cast<size_t>(r) * 64 + j * 8;
             const float4 h0 = *reinterpret_cast<const float4*>(p), h1 = *reinterpret_cast<const float4*>(p + 4);
             const float4 g0 = *reinterpret_cast<const float4*>(gch + j * 8);
@@ -432,7 +493,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   // features; EPU tokens per warp have their independent loads issued before any is used.
   constexpr int EPU = 4;
 
-  if (a.epi == EPI_RESID) {
+  if (EPI == EPI_RESID) {
     const int row = lane * 4;
     const int f = mb * BM + row;
     const bool fok = f < a.Nout;   // Nout is a multiple of 16
@@ -470,10 +531,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         if (lane == 0) a.ssq_out[static_cast<size_t>(t) * a.ssq_ld + mb] = sq;
       }
     }
-  } else if (a.epi == EPI_GELU) {
+  } else if (EPI == EPI_GELU) {
     const int p = lane * 2;
     const int f = mb * 64 + p;   // F is a multiple of 64
-    const float inv = (a.fp8 && a.s_a_out) ? 1.0f / *a.s_a_out : 1.0f;
+    const float inv = (FP8 && a.s_a_out) ? 1.0f / *a.s_a_out : 1.0f;
     for (int tok = tok0 + warp; tok < tok1; tok += 8) {
       const int t = n0 + tok;
       if (t >= a.T || f >= a.F) break;
@@ -481,7 +542,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       vals(tok, p, g, Two{});
       vals(tok, p + 64, up, Two{});
       const float u0 = gelu_tanh(g[0]) * up[0], u1 = gelu_tanh(g[1]) * up[1];
-      if (a.fp8) {
+      if (FP8) {
         *reinterpret_cast<uint16_t*>(a.u_out + btile_offset(t, f, Nt, a.NKC_u)) =
             static_cast<uint16_t>(to_e4m3(u0 * inv) | (static_cast<uint32_t>(to_e4m3(u1 * inv)) << 8));
       } else {
@@ -1412,10 +1473,10 @@ cudaError_t launch_ex(const void* func, dim3 grid, dim3 block, size_t smem, cuda
 
 }  // namespace
 
-size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk) {
-  const GemmGeom g = gemm_geom(Nt, stages, b_kind, fp8, S, nk);
+size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4) {
+  const GemmGeom g = gemm_geom(Nt, stages, b_kind, fp8, S, nk, w4, 1);   // kc0 odd: the larger group count
   const size_t kel = fp8 ? KCB : KCB / 2;
-  const size_t main = g.ring + (b_kind == B_NORM ? static_cast<size_t>(nk) * kel * 4 : 0);
+  const size_t main = g.gamma_off + (b_kind == B_NORM ? static_cast<size_t>(nk) * kel * 4 : 0);
   const size_t TS = (Nt + S - 1) / S;
   const size_t epi = S > 1 ? std::max<size_t>(static_cast<size_t>(S) * TS * BM * 4, g.recv_off + 2 * TS * 64 * 4)
                            : static_cast<size_t>(Nt) * RED_LD * 4;
@@ -1438,12 +1499,17 @@ size_t attn_smem_bytes(int H, int dh, int KC, int C, int umma) {
   return compute > merge ? compute : merge;
 }
 
+const void* gemm_kernel(int epi, int fp8, int norm, int w4);
+
 cudaError_t tc_kernels_init() {
   cudaError_t e;
   int dev = 0, optin = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
-  const void* fns[] = {reinterpret_cast<const void*>(k_gemm_tc), reinterpret_cast<const void*>(k_attn_tc<64>),
+  const void* fns[] = {gemm_kernel(EPI_QKV, 0, 0, 0), gemm_kernel(EPI_RESID, 0, 0, 0), gemm_kernel(EPI_GELU, 0, 0, 0),
+                       gemm_kernel(EPI_QKV, 1, 1, 0), gemm_kernel(EPI_GELU, 1, 1, 0), gemm_kernel(EPI_RESID, 1, 0, 0),
+                       gemm_kernel(EPI_QKV, 0, 0, 1), gemm_kernel(EPI_RESID, 0, 0, 1), gemm_kernel(EPI_GELU, 0, 0, 1),
+                       reinterpret_cast<const void*>(k_attn_tc<64>),
                        reinterpret_cast<const void*>(k_attn_tc<128>), reinterpret_cast<const void*>(k_attn_tc<256>),
                        reinterpret_cast<const void*>(k_attn_umma<64>),
                        reinterpret_cast<const void*>(k_attn_umma<128>), reinterpret_cast<const void*>(k_attn_umma<256>),
@@ -1466,16 +1532,38 @@ int max_dynamic_smem() {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   cudaFuncAttributes fa;
-  cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(k_gemm_tc));
+  cudaFuncGetAttributes(&fa, gemm_kernel(EPI_RESID, 0, 0, 0));
   return optin - static_cast<int>(fa.sharedSizeBytes);
+}
+
+// One instantiation per (epilogue, operand type, B-operand kind, 4-bit weights) in use.
+const void* gemm_kernel(int epi, int fp8, int norm, int w4) {
+  if (w4) {
+    if (fp8 || norm) return nullptr;
+    if (epi == EPI_QKV) return reinterpret_cast<const void*>(k_gemm_tc<EPI_QKV, 0, 0, 1>);
+    if (epi == EPI_RESID) return reinterpret_cast<const void*>(k_gemm_tc<EPI_RESID, 0, 0, 1>);
+    if (epi == EPI_GELU) return reinterpret_cast<const void*>(k_gemm_tc<EPI_GELU, 0, 0, 1>);
+  } else if (!fp8 && !norm) {
+    if (epi == EPI_QKV) return reinterpret_cast<const void*>(k_gemm_tc<EPI_QKV, 0, 0, 0>);
+    if (epi == EPI_RESID) return reinterpret_cast<const void*>(k_gemm_tc<EPI_RESID, 0, 0, 0>);
+    if (epi == EPI_GELU) return reinterpret_cast<const void*>(k_gemm_tc<EPI_GELU, 0, 0, 0>);
+  } else if (fp8 && norm) {
+    if (epi == EPI_QKV) return reinterpret_cast<const void*>(k_gemm_tc<EPI_QKV, 1, 1, 0>);
+    if (epi == EPI_GELU) return reinterpret_cast<const void*>(k_gemm_tc<EPI_GELU, 1, 1, 0>);
+  } else if (fp8 && !norm) {
+    if (epi == EPI_RESID) return reinterpret_cast<const void*>(k_gemm_tc<EPI_RESID, 1, 0, 0>);
+  }
+  return nullptr;
 }
 
 cudaError_t launch_gemm_tc(const GemmArgs& a, int n_tiles, cudaStream_t s, bool pdl) {
   GemmArgs copy = a;
   void* args[] = {&copy};
   const int nk_max = (a.NKC + a.S - 1) / a.S;
-  return launch_ex(reinterpret_cast<const void*>(k_gemm_tc), dim3(a.S, a.MB, n_tiles), dim3(GEMM_THREADS),
-                   gemm_smem_bytes(a.Nt, a.stages, a.b_kind, a.fp8, a.S, nk_max), s, pdl, a.S, args);
+  const void* f = gemm_kernel(a.epi, a.fp8, a.b_kind == B_NORM, a.w4);
+  if (!f) return cudaErrorInvalidValue;
+  return launch_ex(f, dim3(a.S, a.MB, n_tiles), dim3(GEMM_THREADS),
+                   gemm_smem_bytes(a.Nt, a.stages, a.b_kind, a.fp8, a.S, nk_max, a.w4), s, pdl, a.S, args);
 }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, int B, cudaStream_t s, bool pdl) {

@@ -57,7 +57,9 @@ __host__ __device__ __forceinline__ size_t htile_offset(int t, int f, int Nt, in
 
 struct GemmArgs {
   // A operand: weights pre-tiled by the packer, [MB][NKC][BM rows x KCB bytes] core-matrix slabs
-  const uint8_t* W;
+  const uint8_t* W;           // w4: 4-bit codes [MB][NKC][8 slabs][128 rows][4 B] (8 codes per 4 B, low nibble first)
+  const uint16_t* Wscale;     // w4: bf16 scales [MB][NG][128 rows], one per 128 inputs (two chunks)
+  int w4;                     // 1: 4-bit weights, dequantised to bf16(q * s) in shared memory
   int MB, NKC;             // m-blocks, k-chunks
   int Nout;                // valid output rows (features) over all m-blocks
   int S;                   // split-K factor = cluster size along x
@@ -188,7 +190,7 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int B, cudaStream_t s, bool p
 cudaError_t launch_inproj_tc(const InprojArgs& a, cudaStream_t s, bool pdl);
 cudaError_t launch_final_tc(const FinalArgs& a, cudaStream_t s, bool pdl);
 cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s);
-size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk);
+size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4 = 0);
 size_t gemm_scratch_bytes(int NT, int MB, int S, int Nt);
 size_t attn_scratch_bytes(int B, int Hq, int C, int H, int dh);
 size_t attn_smem_bytes(int H, int dh, int KC, int C, int umma);

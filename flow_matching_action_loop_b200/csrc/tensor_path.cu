@@ -30,16 +30,26 @@ struct ProjLayout {
   int rows = 0;      // output rows after permutation (padded to MB*BM)
   int K = 0;         // input features
   int MB = 0, NKC = 0;
+  int NG = 0;        // w4: scale groups of 128 inputs
+  size_t sc_off = 0; // w4: byte offset of the scales after the 4-bit codes
   size_t bytes = 0;  // tiled bytes per layer
 };
 
-ProjLayout make_layout(int rows, int K, int elem) {
+// bf16 / e4m3: [MB][NKC][128 rows x 128 B] core-matrix slabs.  w4 (chunks of 64 inputs, as bf16):
+// codes [MB][NKC][8 slabs][128 rows][4 B], then bf16 scales [MB][NG][128 rows].
+ProjLayout make_layout(int rows, int K, int elem, int w4) {
   ProjLayout p;
   p.rows = rows;
   p.K = K;
   p.MB = ceil_div(rows, BM);
   p.NKC = ceil_div(K * elem, KCB);
-  p.bytes = static_cast<size_t>(p.MB) * p.NKC * BM * KCB;
+  if (w4) {
+    p.NG = ceil_div(p.NKC, 2);
+    p.sc_off = static_cast<size_t>(p.MB) * p.NKC * (BM * KCB / 4);
+    p.bytes = align_up(p.sc_off + static_cast<size_t>(p.MB) * p.NG * BM * 2, 1024);
+  } else {
+    p.bytes = static_cast<size_t>(p.MB) * p.NKC * BM * KCB;
+  }
   return p;
 }
 
@@ -78,6 +88,7 @@ struct TensorPath {
   int nsm = 148;
   int max_dyn = 0;
   int fp8 = 0, elem = 2;
+  int w4 = 0;                    // 4-bit weights dequantised in the GEMM (activations as bf16)
   int T_max = 0, T_pad = 0, MBd = 0, MB_rot = 0;
   int KB = 0;                    // 64-feature blocks of h per n-tile (D rounded up to 128)
   int ssq_ld = 0;                // columns of the Σh² partials (MBd rounded up to 4)
@@ -117,11 +128,11 @@ struct Carve {
   }
 };
 
-void layouts(const fr_config& c, int elem, ProjLayout& qkv, ProjLayout& o, ProjLayout& gu, ProjLayout& dn) {
-  qkv = make_layout((c.Hq + 2 * c.Hkv) * c.dh, c.D, elem);
-  o = make_layout(c.D, c.Hq * c.dh, elem);
-  gu = make_layout(2 * c.F, c.D, elem);
-  dn = make_layout(c.D, c.F, elem);
+void layouts(const fr_config& c, int elem, int w4, ProjLayout& qkv, ProjLayout& o, ProjLayout& gu, ProjLayout& dn) {
+  qkv = make_layout((c.Hq + 2 * c.Hkv) * c.dh, c.D, elem, w4);
+  o = make_layout(c.D, c.Hq * c.dh, elem, w4);
+  gu = make_layout(2 * c.F, c.D, elem, w4);
+  dn = make_layout(c.D, c.F, elem, w4);
 }
 
 size_t carve_all(TensorPath* tp, char* base) {
@@ -146,6 +157,7 @@ size_t carve_all(TensorPath* tp, char* base) {
 void init_sizes(TensorPath* tp, const fr_config& c) {
   tp->c = c;
   tp->fp8 = c.dtype == FR_DTYPE_FP8;
+  tp->w4 = c.dtype == FR_DTYPE_W4A16;
   tp->elem = tp->fp8 ? 1 : 2;
   tp->T_max = c.B_max * c.H;
   tp->T_pad = static_cast<int>(align_up(tp->T_max, 16));
@@ -155,7 +167,7 @@ void init_sizes(TensorPath* tp, const fr_config& c) {
   tp->ssq_ld = static_cast<int>(align_up(tp->MBd, 4));
   const int nt_max = ceil_div(tp->T_max, NT_MAX);
   tp->tok_alloc = tp->T_max + 16 * nt_max;
-  layouts(c, tp->elem, tp->qkv, tp->o, tp->gu, tp->dn);
+  layouts(c, tp->elem, tp->w4, tp->qkv, tp->o, tp->gu, tp->dn);
   tp->layer_bytes = tp->qkv.bytes + tp->o.bytes + tp->gu.bytes + tp->dn.bytes;
 }
 
@@ -164,13 +176,13 @@ void init_sizes(TensorPath* tp, const fr_config& c) {
 // weights next to it) and at most ~120 KB of shared memory; the cost counts waves, the split-K
 // exchange, and weight chunks that must stream after the dependency wait.  Wider tiles are
 // throughput-bound: no split-K unless the tiles leave most SMs idle.
-GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int nsm, int max_dyn) {
+GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, int nsm, int max_dyn) {
   GemmPlan best;
   if (Nt > 64) {
     best.S = (tiles * 2 <= nsm && NKC >= 2) ? 2 : 1;
     const int chunks = ceil_div(NKC, best.S);
     best.stages = std::min(chunks, MAX_STAGES);
-    while (best.stages > 1 && gemm_smem_bytes(Nt, best.stages, b_kind, fp8, best.S, chunks) > static_cast<size_t>(max_dyn))
+    while (best.stages > 1 && gemm_smem_bytes(Nt, best.stages, b_kind, fp8, best.S, chunks, w4) > static_cast<size_t>(max_dyn))
       --best.stages;
     return best;
   }
@@ -179,8 +191,8 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int nsm, i
   for (int S = 1; S <= 16 && S <= NKC; ++S) {
     const int chunks = ceil_div(NKC, S);
     int stages = std::min(chunks, MAX_STAGES);
-    while (stages > 1 && gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks) > cap) --stages;
-    if (gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks) > static_cast<size_t>(max_dyn)) continue;
+    while (stages > 1 && gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4) > cap) --stages;
+    if (gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4) > static_cast<size_t>(max_dyn)) continue;
     const int waves = ceil_div(tiles * S, nsm);
     const double cost = waves * (1.0 + (S > 1 ? 1.0 : 0.0) + 0.3 * (chunks - stages) + 0.05 * chunks);
     if (cost < best_cost - 1e-9) {
@@ -201,10 +213,10 @@ StepPlan make_plan(const TensorPath* tp, int B, int P) {
   p.NT = ceil_div(p.T, NT_MAX);
   p.Nt = static_cast<int>(align_up(ceil_div(p.T, p.NT), 16));
   const int norm_kind = tp->fp8 ? B_NORM : B_ROWS;   // bf16: the producer wrote bf16(h*gamma) already
-  p.qkv = choose_plan(tp->qkv.MB * p.NT, tp->qkv.NKC, p.Nt, norm_kind, tp->fp8, tp->nsm, tp->max_dyn);
-  p.o = choose_plan(tp->o.MB * p.NT, tp->o.NKC, p.Nt, B_ROWS, tp->fp8, tp->nsm, tp->max_dyn);
-  p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, norm_kind, tp->fp8, tp->nsm, tp->max_dyn);
-  p.dn = choose_plan(tp->dn.MB * p.NT, tp->dn.NKC, p.Nt, B_ROWS, tp->fp8, tp->nsm, tp->max_dyn);
+  p.qkv = choose_plan(tp->qkv.MB * p.NT, tp->qkv.NKC, p.Nt, norm_kind, tp->fp8, tp->w4, tp->nsm, tp->max_dyn);
+  p.o = choose_plan(tp->o.MB * p.NT, tp->o.NKC, p.Nt, B_ROWS, tp->fp8, tp->w4, tp->nsm, tp->max_dyn);
+  p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, norm_kind, tp->fp8, tp->w4, tp->nsm, tp->max_dyn);
+  p.dn = choose_plan(tp->dn.MB * p.NT, tp->dn.NKC, p.Nt, B_ROWS, tp->fp8, tp->w4, tp->nsm, tp->max_dyn);
   p.attn_umma = attn_plan(P + c.H, attn_tiles(B, c.Hq, c.Hkv, c.H), tp->nsm, p.attn_C, p.attn_KC);
   return p;
 }
@@ -232,6 +244,27 @@ void tile_projection(const ProjLayout& L, int elem, double scale, RowFn rowsrc, 
   }
 }
 
+// 4-bit codes and scales of one projection (fr_quantize_w4 per source row, groups along K).
+template <typename RowFn>
+void tile_projection_w4(const ProjLayout& L, RowFn rowsrc, std::vector<uint8_t>& out) {
+  out.assign(L.bytes, 0);
+  std::vector<int8_t> q(L.K);
+  std::vector<uint16_t> sb(L.NG);
+  uint16_t* scales = reinterpret_cast<uint16_t*>(out.data() + L.sc_off);
+  for (int r = 0; r < L.MB * BM; ++r) {
+    const float* src = rowsrc(r);
+    if (!src) continue;   // padding rows: zero codes, zero scales
+    fr_quantize_w4(src, 1, L.K, q.data(), sb.data());
+    const int mb = r / BM, rr = r % BM;
+    for (int g = 0; g < L.NG; ++g) scales[(static_cast<size_t>(mb) * L.NG + g) * BM + rr] = sb[g];
+    for (int k = 0; k < L.K; ++k) {
+      const int kc = k / 64, j = (k % 64) / 8, e = k % 8;
+      uint8_t* word = out.data() + ((static_cast<size_t>(mb) * L.NKC + kc) * 8 + j) * BM * 4 + rr * 4;
+      word[e >> 1] |= static_cast<uint8_t>((static_cast<uint8_t>(q[k]) & 0xF) << (4 * (e & 1)));
+    }
+  }
+}
+
 GemmArgs base_args(const TensorPath* tp, const StepPlan& p, const ProjLayout& L, const GemmPlan& g, int layer,
                    size_t w_off) {
   const fr_config& c = tp->c;
@@ -244,6 +277,8 @@ GemmArgs base_args(const TensorPath* tp, const StepPlan& p, const ProjLayout& L,
   a.S = g.S;
   a.stages = g.stages;
   a.fp8 = tp->fp8;
+  a.w4 = tp->w4;
+  a.Wscale = tp->w4 ? reinterpret_cast<const uint16_t*>(a.W + L.sc_off) : nullptr;
   a.T = p.T;
   a.Nt = p.Nt;
   a.KB = tp->KB;
@@ -480,7 +515,7 @@ int retarget(GraphEntry& ge, const float* x0, float* x_out) {
 }  // namespace
 
 bool tensor_path_supports(const fr_config& c) {
-  if (c.dtype != FR_DTYPE_BF16 && c.dtype != FR_DTYPE_FP8) return false;
+  if (c.dtype != FR_DTYPE_BF16 && c.dtype != FR_DTYPE_FP8 && c.dtype != FR_DTYPE_W4A16) return false;
   if (c.dh != 64 && c.dh != 128 && c.dh != 256) return false;
   if (((c.Hq + c.Hkv) * c.dh / 2) % 64 != 0) return false;   // RoPE pairs fill whole m-blocks
   if ((c.Hkv * c.dh) % BM != 0) return false;                // V rows fill whole m-blocks
@@ -497,7 +532,7 @@ bool tensor_path_supports(const fr_config& c) {
 }
 
 const char* tensor_path_limits() {
-  return "bf16/fp8, dh in {64,128,256}, (Hq+Hkv)*dh/2 % 64 == 0, Hkv*dh % 128 == 0, F % 64 == 0, H <= 128, "
+  return "bf16/fp8/w4a16, dh in {64,128,256}, (Hq+Hkv)*dh/2 % 64 == 0, Hkv*dh % 128 == 0, F % 64 == 0, H <= 128, "
          "D % 16 == 0, D <= 2048, A <= 64, attention chunk fits shared memory";
 }
 
@@ -588,11 +623,13 @@ int tensor_path_pack_layer(TensorPath* tp, int l, const fr_layer_weights& w, con
     if (cr < nq + nk) return w.wk + static_cast<size_t>(cr - nq) * D;
     return w.wv + static_cast<size_t>(cr - nq - nk) * D;
   };
-  tile_projection(tp->qkv, tp->elem, sw[PI_QKV], qkv_row, buf);
+  if (tp->w4) tile_projection_w4(tp->qkv, qkv_row, buf);
+  else tile_projection(tp->qkv, tp->elem, sw[PI_QKV], qkv_row, buf);
   FR_CUDA(cudaMemcpy(dst, buf.data(), buf.size(), cudaMemcpyHostToDevice));
   dst += tp->qkv.bytes;
   auto o_row = [&](int r) -> const float* { return r < D ? w.wo + static_cast<size_t>(r) * nq : nullptr; };
-  tile_projection(tp->o, tp->elem, sw[PI_O], o_row, buf);
+  if (tp->w4) tile_projection_w4(tp->o, o_row, buf);
+  else tile_projection(tp->o, tp->elem, sw[PI_O], o_row, buf);
   FR_CUDA(cudaMemcpy(dst, buf.data(), buf.size(), cudaMemcpyHostToDevice));
   dst += tp->o.bytes;
   // gate|up rows: m-block mb holds gate features mb*64..+63 (rows 0-63) and the same up features (64-127)
@@ -602,11 +639,13 @@ int tensor_path_pack_layer(TensorPath* tp, int l, const fr_layer_weights& w, con
     if (f >= F) return nullptr;
     return (rr < 64 ? w.wg : w.wu) + static_cast<size_t>(f) * D;
   };
-  tile_projection(tp->gu, tp->elem, sw[PI_GU], gu_row, buf);
+  if (tp->w4) tile_projection_w4(tp->gu, gu_row, buf);
+  else tile_projection(tp->gu, tp->elem, sw[PI_GU], gu_row, buf);
   FR_CUDA(cudaMemcpy(dst, buf.data(), buf.size(), cudaMemcpyHostToDevice));
   dst += tp->gu.bytes;
   auto d_row = [&](int r) -> const float* { return r < D ? w.wd + static_cast<size_t>(r) * F : nullptr; };
-  tile_projection(tp->dn, tp->elem, sw[PI_DOWN], d_row, buf);
+  if (tp->w4) tile_projection_w4(tp->dn, d_row, buf);
+  else tile_projection(tp->dn, tp->elem, sw[PI_DOWN], d_row, buf);
   FR_CUDA(cudaMemcpy(dst, buf.data(), buf.size(), cudaMemcpyHostToDevice));
   std::memcpy(&tp->gains_host[static_cast<size_t>(l) * 2 * D], w.g1, D * sizeof(float));
   std::memcpy(&tp->gains_host[static_cast<size_t>(l) * 2 * D + D], w.g2, D * sizeof(float));

@@ -53,7 +53,10 @@ enum {
   FR_ERR_UNSUPPORTED = -7   /* configuration outside what the kernels implement */
 };
 
-enum { FR_DTYPE_F32 = 0, FR_DTYPE_BF16 = 1, FR_DTYPE_FP8 = 2 };
+enum { FR_DTYPE_F32 = 0, FR_DTYPE_BF16 = 1, FR_DTYPE_FP8 = 2, FR_DTYPE_W4A16 = 3 };
+
+/* Input features per scale group of the 4-bit weights of FR_DTYPE_W4A16. */
+#define FR_W4_GROUP 128
 
 /* Kernel set used by fr_denoise.  FR_PATH_AUTO picks the tensor-core path for
  * bf16/fp8 and the CUDA-core path for f32.  FR_PATH_STEPWISE forces the simple
@@ -132,8 +135,9 @@ int fr_create(const fr_config* cfg, int device, fr_handle** out);
  * transpose/fuse/FP8-quantise transforms).  The packer concatenates
  * W_qkv = [W_q; W_k; W_v] and W_gu = [W_gate; W_up], rounds to bf16 (RNE) or,
  * for FR_DTYPE_FP8, quantises each fused projection to e4m3 with
- * s_w = max|w| / 448, and precomputes the K time embeddings and the RoPE
- * tables.  Synchronous with respect to the host pointers; the caller keeps
+ * s_w = max|w| / 448, or, for FR_DTYPE_W4A16, quantises every layer projection
+ * to 4-bit codes with a bf16 scale per FR_W4_GROUP inputs (fr_quantize_w4), and
+ * precomputes the K time embeddings and the RoPE tables.  Synchronous with respect to the host pointers; the caller keeps
  * ownership of `w`.  Errors: FR_ERR_ARG, FR_ERR_CUDA.
  */
 int fr_load_weights(fr_handle* h, const fr_weights* w, fr_stream_t stream);
@@ -269,6 +273,14 @@ int fr_rope_tables(int n_pos, int dh, double theta, float* cos_out, float* sin_o
 
 /* float32 -> bf16 bits, round to nearest even (NaN stays NaN). */
 void fr_round_bf16(const float* in, uint16_t* out, size_t n);
+
+/* 4-bit group quantisation of a row-major [rows][cols] float32 weight (FR_DTYPE_W4A16;
+ * PhyAI page, optimisation paragraph: W4A16; the group size is this library's reading).
+ * Per row and per group of FR_W4_GROUP consecutive columns: scale s = bf16(max|w| / 7),
+ * one rounding from float64, returned as bf16 bits in scale_bits [rows][ceil(cols/128)];
+ * codes q = round-half-even(w / s) clamped to [-7, 7] in q [rows][cols]; an all-zero group
+ * has s = 0 and q = 0.  The projection uses bf16(q * s).  FR_ERR_ARG on NULL or negative sizes. */
+int fr_quantize_w4(const float* w, int rows, int cols, int8_t* q, uint16_t* scale_bits);
 
 /* float32 -> e4m3 bytes of in[i] / scale computed in float64: saturate to +-448,
  * round to nearest even (OCP E4M3, no infinities, NaN -> 0x7F). */

@@ -22,6 +22,8 @@ RAGGED = {
                                                 A=7, B=3, P=75, K=3, dtype="bf16"),
     "ragged_fp8": synthetic.ActionExpertConfig("ragged_fp8", L=2, D=320, Hq=4, Hkv=2, dh=64, F=704, H=37,
                                                A=7, B=3, P=75, K=3, dtype="fp8"),
+    "ragged_w4a16": synthetic.ActionExpertConfig("ragged_w4a16", L=2, D=320, Hq=4, Hkv=2, dh=64, F=704, H=37,
+                                                 A=7, B=3, P=75, K=3, dtype="w4a16"),
     "ragged_f32": synthetic.ActionExpertConfig("ragged_f32", L=2, D=192, Hq=6, Hkv=3, dh=32, F=200, H=21,
                                                A=5, B=2, P=33, K=2, dtype="f32"),
     "mha_bf16": synthetic.ActionExpertConfig("mha_bf16", L=1, D=256, Hq=2, Hkv=2, dh=128, F=512, H=50,

@@ -104,3 +104,16 @@ def test_noalloc_attention_rejects_before_device_work(abi):
     assert lib.fr_attention_noalloc(p, p, p, p, 2, 8, 1, 50, 866, 256, None) == abi.FR_ERR_UNSUPPORTED
     assert b"scratch" in lib.fr_last_error()
     assert lib.fr_attention_noalloc(None, p, p, p, 1, 8, 1, 50, 866, 256, None) == abi.FR_ERR_ARG
+
+
+def test_packer_w4_matches_oracle_quantiser(abi):
+    rng = np.random.default_rng(5)
+    w = (rng.standard_normal((37, 300)) / 19).astype(np.float32)   # ragged last group (300 = 2 x 128 + 44)
+    w[3, :128] = 0.0                                                 # an all-zero group
+    w[4, 128:256] = 0.25                                             # a constant group
+    q, sb = abi.fr_quantize_w4(w)
+    oq, os_ = O.quantize_w4(w)
+    assert np.array_equal(q, oq)
+    sv = (sb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.array_equal(sv, os_)
+    assert abi.load_library().fr_quantize_w4(None, 1, 1, None, None) == abi.FR_ERR_ARG

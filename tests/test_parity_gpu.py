@@ -26,7 +26,7 @@ def _assert_close(cfg, got, want, label=""):
     rel, cos = C.chunk_metrics(got, want)
     if cfg.dtype == "f32":
         assert np.all(rel <= C.TOL_F32_REL_L2), (label, rel)
-    elif cfg.dtype == "bf16":
+    elif cfg.dtype in ("bf16", "w4a16"):   # w4a16: both sides use the same dequantised bf16 operands
         assert np.all(rel <= C.TOL_BF16_REL_L2) and np.all(cos >= C.TOL_BF16_COS), (label, rel, cos)
     else:
         assert np.all(cos >= C.TOL_FP8_COS), (label, rel, cos)
@@ -39,7 +39,7 @@ def _paths(cfg):
     return [FR_PATH_STEPWISE] if cfg.dtype == "f32" else [FR_PATH_STEPWISE, FR_PATH_TENSOR]
 
 
-SMALL = ["tiny_f32", "ragged_f32", "ragged_bf16", "mha_bf16", "minimal_bf16"]
+SMALL = ["tiny_f32", "ragged_f32", "ragged_bf16", "mha_bf16", "minimal_bf16", "ragged_w4a16"]
 
 
 @pytest.mark.parametrize("name", SMALL)
@@ -100,6 +100,18 @@ def test_parity_pi05_fp8_batch1():
         assert np.allclose(sa, O.scales_to_array(cfg, sc), rtol=C.TOL_CALIB_REL, atol=0)
         rel, cos = _assert_close(cfg, got, want, f"own calibration, path={loop.path}")
         print(f"pi05_fp8_b1 {loop.path}: rel-L2 {rel.max():.3e} cos {cos.min():.6f}")
+        loop.close()
+
+
+@pytest.mark.slow
+def test_parity_pi05_w4a16_batch1():
+    cfg = synthetic.CONFIGS["pi05_w4a16_b1"]
+    inp = C.inputs("pi05_w4a16_b1")
+    want = O.denoise(cfg, inp["weights"], inp["prefix_k"], inp["prefix_v"], inp["x0"])
+    for path in _paths(cfg):
+        got, loop = C.run_library(cfg, inp, path=path)
+        rel, cos = _assert_close(cfg, got, want, f"path={loop.path}")
+        print(f"pi05_w4a16_b1 {loop.path}: rel-L2 {rel.max():.3e} cos {cos.min():.6f}")
         loop.close()
 
 
@@ -215,7 +227,8 @@ def test_smaller_batch_and_prefix_than_the_handle_maximum():
 
 
 def test_automatic_path_is_the_tensor_path_for_bf16_and_fp8():
-    for name in ("pi05_bf16_b1", "pi05_fp8_b1", "pi05_bf16_b32", "stress_bf16_b4", "ragged_bf16", "mha_bf16"):
+    for name in ("pi05_bf16_b1", "pi05_fp8_b1", "pi05_w4a16_b1", "pi05_bf16_b32", "stress_bf16_b4", "ragged_bf16",
+                 "mha_bf16", "ragged_w4a16"):
         loop = ActionExpertLoop(C.get_config(name), path=FR_PATH_AUTO)
         assert loop.path == "tensor", (name, loop.path)
         loop.close()
