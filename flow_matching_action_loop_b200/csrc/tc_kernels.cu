@@ -41,21 +41,29 @@ using namespace fr::sm100;
 __device__ unsigned long long* g_tl = nullptr;   // [cap][16]: kind, cta, t0..t13
 __device__ unsigned g_tl_count = 0;
 __device__ unsigned g_tl_cap = 0;
-#define TL_DECL __shared__ unsigned tl_slot_;
+// The record pointer is resolved once per CTA into shared memory, so that a timestamp costs a
+// clock read and a store, not a global load ahead of the clock read.
+#define TL_DECL __shared__ unsigned long long* tl_rec_;
 #define TL_BEGIN(kind)                                                                          \
   do {                                                                                          \
     if (threadIdx.x == 0) {                                                                     \
-      tl_slot_ = g_tl ? atomicAdd(&g_tl_count, 1u) : 0xFFFFFFFFu;                               \
-      if (tl_slot_ < g_tl_cap) {                                                                \
-        g_tl[tl_slot_ * 16 + 0] = (kind);                                                        \
-        g_tl[tl_slot_ * 16 + 1] = blockIdx.x | (blockIdx.y << 10) | (blockIdx.z << 20);          \
-        g_tl[tl_slot_ * 16 + 2] = fr::sm100::globaltimer();                                      \
+      const unsigned long long t0_ = fr::sm100::globaltimer();                                 \
+      unsigned long long* base_ = g_tl;                                                         \
+      const unsigned slot_ = base_ ? atomicAdd(&g_tl_count, 1u) : 0xFFFFFFFFu;                 \
+      tl_rec_ = (base_ && slot_ < g_tl_cap) ? base_ + static_cast<size_t>(slot_) * 16 : nullptr; \
+      if (tl_rec_) {                                                                            \
+        tl_rec_[0] = (kind);                                                                    \
+        tl_rec_[1] = blockIdx.x | (blockIdx.y << 10) | (blockIdx.z << 20);                      \
+        tl_rec_[2] = t0_;                                                                       \
       }                                                                                         \
     }                                                                                           \
+    __syncthreads();                                                                            \
   } while (0)
 #define TL(k)                                                                                   \
   do {                                                                                          \
-    if (tl_slot_ < g_tl_cap) g_tl[tl_slot_ * 16 + 2 + (k)] = fr::sm100::globaltimer();          \
+    const unsigned long long t_ = fr::sm100::globaltimer();                                     \
+    unsigned long long* r_ = tl_rec_;                                                           \
+    if (r_) r_[2 + (k)] = t_;                                                                   \
   } while (0)
 #else
 #define TL_DECL
@@ -148,6 +156,22 @@ __host__ __device__ __forceinline__ GemmGeom gemm_geom(int Nt, int stages, int b
   return g;
 }
 
+// Largest chunk count of any split-K rank: the shared-memory layout is the same in every CTA.
+__host__ __device__ __forceinline__ int nk_max_of(const GemmArgs& a) { return (a.NKC + a.S - 1) / a.S; }
+
+// Bytes of the main loop and epilogue regions; the QKV epilogue's RoPE stage ([H][64] (cos, sin)
+// pairs of the m-block) follows them.
+__host__ __device__ __forceinline__ uint32_t gemm_rope_off(int Nt, int stages, int b_kind, int fp8, int S, int nk,
+                                                          int w4) {
+  const GemmGeom g = gemm_geom(Nt, stages, b_kind, fp8, S, nk, w4, 1);   // kc0 odd: the larger group count
+  const uint32_t kel = fp8 ? KCB : KCB / 2;
+  const uint32_t main = g.gamma_off + (b_kind == B_NORM ? static_cast<uint32_t>(nk) * kel * 4u : 0u);
+  const uint32_t TS = (Nt + S - 1) / S;
+  uint32_t epi = S > 1 ? static_cast<uint32_t>(S) * TS * BM * 4u : static_cast<uint32_t>(Nt) * RED_LD * 4u;
+  if (S > 1 && g.recv_off + 2u * TS * 64u * 4u > epi) epi = g.recv_off + 2u * TS * 64u * 4u;
+  return ((main > epi ? main : epi) + 15u) & ~15u;
+}
+
 template <int EPI, int FP8, int NORM, int W4>
 __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_constant__ GemmArgs a) {
   extern __shared__ __align__(1024) uint8_t dsm[];
@@ -195,6 +219,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   tc_fence_after();
   grid_dep_launch();   // the next kernel may start its own prefetch now
   const uint32_t tacc = sh.tmem_base;
+  // QKV: (cos, sin) of this m-block's 64 rotate-half pairs at every action position, staged while
+  // the previous kernel runs (the tables are static); read by the epilogue after the main loop
+  float2* rope_sh = reinterpret_cast<float2*>(dsm + gemm_rope_off(Nt, stages, NORM ? B_NORM : B_ROWS, FP8, S, nk_max_of(a), W4));
+  if (EPI == EPI_QKV && mb < a.MB_rot && warp >= 2) {   // warps 2-7: the producer and MMA warps go on
+    const int half = a.dh >> 1;
+    for (int idx = tid - 64; idx < a.H * 64; idx += GEMM_THREADS - 64) {
+      const int i = idx >> 6, p = idx & 63;
+      const int j = (mb * 64 + p) % half, pos = a.P + i;
+      rope_sh[idx] = make_float2(a.rope_cos[pos * half + j], a.rope_sin[pos * half + j]);
+    }
+  }
 
   if (warp == 0) {
     // ---------------- bulk-copy producer
@@ -561,9 +596,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         for (int u = 0; u < EPU; ++u) {
           const int tok = tb + 8 * u, t = n0 + tok;
           if (tok < tok1 && t < a.T) {
-            const int pos = a.P + t % a.H;
-            cs[u] = *reinterpret_cast<const float2*>(a.rope_cos + pos * half + j);
-            sn[u] = *reinterpret_cast<const float2*>(a.rope_sin + pos * half + j);
+            const float4 r4 = *reinterpret_cast<const float4*>(rope_sh + (t % a.H) * 64 + p);   // pairs p, p+1
+            cs[u] = make_float2(r4.x, r4.z);
+            sn[u] = make_float2(r4.y, r4.w);
           }
         }
 #pragma unroll
@@ -1331,7 +1366,7 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
   TL_DECL
   TL_BEGIN(1);
   __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(dsm);   // [D][A]
-  const int t = blockIdx.x, tid = threadIdx.x;
+  const int tid = threadIdx.x;
   const uint32_t wbytes = static_cast<uint32_t>(a.D) * a.A * 2;
   if (tid == 0) {
     mbar_init(&wbar, 1);
@@ -1349,10 +1384,11 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
   }
   grid_dep_wait();
   if (tid == 0) TL(1);
-  if (tid < a.A) xs[tid] = __bfloat162float(__float2bfloat16_rn(a.x[static_cast<size_t>(t) * a.A + tid]));
-  __syncthreads();
   mbar_wait(&wbar, 0, WAIT_LIMIT_NS);
   const int warp = tid >> 5, lane = tid & 31;
+  for (int t = blockIdx.x; t < a.T; t += gridDim.x) {   // the weights are staged once per CTA
+  if (tid < a.A) xs[tid] = __bfloat162float(__float2bfloat16_rn(a.x[static_cast<size_t>(t) * a.A + tid]));
+  __syncthreads();
 #pragma unroll
   for (int q = 0; q < QMAX; ++q) {
     const int n = tid + q * 256;
@@ -1375,6 +1411,8 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
   __syncthreads();
   const int nmb = (a.D + BM - 1) / BM;
   if (tid < nmb) a.ssq[static_cast<size_t>(t) * a.ssq_ld + tid] = ((part[tid][0] + part[tid][1]) + part[tid][2]) + part[tid][3];
+  __syncthreads();   // xs and part are rewritten by the next token
+  }
   if (tid == 0) TL(5);
 }
 
@@ -1386,7 +1424,7 @@ __global__ void __launch_bounds__(256) k_final_tc(const __grid_constant__ FinalA
   TL_BEGIN(2);
   __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(dsm);                     // [A][D]
   float* hn = reinterpret_cast<float*>(dsm + ((static_cast<size_t>(a.A) * a.D * 2 + 127) & ~size_t(127)));
-  const int t = blockIdx.x, tid = threadIdx.x;
+  const int tid = threadIdx.x;
   const uint32_t wbytes = static_cast<uint32_t>(a.A) * a.D * 2;
   if (tid == 0) {
     mbar_init(&wbar, 1);
@@ -1404,6 +1442,7 @@ __global__ void __launch_bounds__(256) k_final_tc(const __grid_constant__ FinalA
   }
   grid_dep_wait();
   if (threadIdx.x == 0) TL(1);
+  for (int t = blockIdx.x; t < a.T; t += gridDim.x) {   // the weights are staged once per CTA
   float hv[QMAX];
 #pragma unroll
   for (int q = 0; q < QMAX; ++q) {
@@ -1433,7 +1472,8 @@ __global__ void __launch_bounds__(256) k_final_tc(const __grid_constant__ FinalA
       a.x_out[xi] = a.x_in[xi] + a.dt * (acc + a.b_out[i]);
     }
   }
-  __syncthreads();
+  __syncthreads();   // hn and ssq_sh are rewritten by the next token
+  }
   if (tid == 0) TL(5);
 }
 
@@ -1473,14 +1513,8 @@ cudaError_t launch_ex(const void* func, dim3 grid, dim3 block, size_t smem, cuda
 
 }  // namespace
 
-size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4) {
-  const GemmGeom g = gemm_geom(Nt, stages, b_kind, fp8, S, nk, w4, 1);   // kc0 odd: the larger group count
-  const size_t kel = fp8 ? KCB : KCB / 2;
-  const size_t main = g.gamma_off + (b_kind == B_NORM ? static_cast<size_t>(nk) * kel * 4 : 0);
-  const size_t TS = (Nt + S - 1) / S;
-  const size_t epi = S > 1 ? std::max<size_t>(static_cast<size_t>(S) * TS * BM * 4, g.recv_off + 2 * TS * 64 * 4)
-                           : static_cast<size_t>(Nt) * RED_LD * 4;
-  return main > epi ? main : epi;
+size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4, int rope_rows) {
+  return gemm_rope_off(Nt, stages, b_kind, fp8, S, nk, w4) + static_cast<size_t>(rope_rows) * 64 * 8;
 }
 
 size_t gemm_scratch_bytes(int NT, int MB, int S, int Nt) {
@@ -1563,7 +1597,8 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int n_tiles, cudaStream_t s, bool 
   const void* f = gemm_kernel(a.epi, a.fp8, a.b_kind == B_NORM, a.w4);
   if (!f) return cudaErrorInvalidValue;
   return launch_ex(f, dim3(a.S, a.MB, n_tiles), dim3(GEMM_THREADS),
-                   gemm_smem_bytes(a.Nt, a.stages, a.b_kind, a.fp8, a.S, nk_max, a.w4), s, pdl, a.S, args);
+                   gemm_smem_bytes(a.Nt, a.stages, a.b_kind, a.fp8, a.S, nk_max, a.w4, a.epi == EPI_QKV ? a.H : 0), s,
+                   pdl, a.S, args);
 }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, int B, cudaStream_t s, bool pdl) {
@@ -1588,7 +1623,7 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int B, cudaStream_t s, bool p
 cudaError_t launch_inproj_tc(const InprojArgs& a, cudaStream_t s, bool pdl) {
   InprojArgs copy = a;
   void* args[] = {&copy};
-  return launch_ex(reinterpret_cast<const void*>(k_inproj_tc), dim3(a.T), dim3(256),
+  return launch_ex(reinterpret_cast<const void*>(k_inproj_tc), dim3(a.max_ctas > 0 && a.max_ctas < a.T ? a.max_ctas : a.T), dim3(256),
                    static_cast<size_t>(a.D) * a.A * 2, s, pdl, 1, args);
 }
 
@@ -1596,7 +1631,8 @@ cudaError_t launch_final_tc(const FinalArgs& a, cudaStream_t s, bool pdl) {
   FinalArgs copy = a;
   void* args[] = {&copy};
   const size_t smem = ((static_cast<size_t>(a.A) * a.D * 2 + 127) & ~size_t(127)) + static_cast<size_t>(a.D) * 4;
-  return launch_ex(reinterpret_cast<const void*>(k_final_tc), dim3(a.T), dim3(256), smem, s, pdl, 1, args);
+  return launch_ex(reinterpret_cast<const void*>(k_final_tc), dim3(a.max_ctas > 0 && a.max_ctas < a.T ? a.max_ctas : a.T),
+                   dim3(256), smem, s, pdl, 1, args);
 }
 
 cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s) {
