@@ -83,6 +83,15 @@ __device__ __forceinline__ void bulk_s2cluster(uint32_t dst_cluster, const void*
       "r"(smem_u32(src_smem)), "r"(bytes), "r"(bar_cluster)
       : "memory");
 }
+// shared (this CTA) -> global, tracked by the bulk async-group of this thread.
+__device__ __forceinline__ void bulk_s2g(void* gdst, const void* src_smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(src_smem)),
+               "r"(bytes)
+               : "memory");
+}
+// Wait until every committed bulk copy of this thread has completed (writes performed).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until the sources of every committed bulk copy of this thread have been read.
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }

@@ -467,8 +467,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
           for (int j = 0; j < 16; ++j) {
             const int tok = c0 + 16 * u + j;
             if (S == 1) red[tok * RED_LD + row] = __uint_as_float(v[u][j]);
-            else if (tok < t_hi) xs[(static_cast<size_t>(ks) * Nt + tok) * BM + row] = __uint_as_float(v[u][j]);
+            else if (tok < t_hi) red[tok * BM + row] = __uint_as_float(v[u][j]);   // staged for one bulk store
           }
+    }
+  }
+  if (S > 1) {   // the partial tile (valid tokens) into the scratch with one bulk store
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      bulk_s2g(xs + static_cast<size_t>(ks) * Nt * BM, red, static_cast<uint32_t>(t_hi) * BM * 4u);
+      bulk_commit();
+      bulk_wait_all();
+      fence_proxy_async_global();
     }
   }
   if (tid == 128) TL(7);
