@@ -156,19 +156,32 @@ __host__ __device__ __forceinline__ GemmGeom gemm_geom(int Nt, int stages, int b
   return g;
 }
 
+// Bytes of the epilogue stage that follows the main-loop and exchange regions: the QKV epilogue's
+// RoPE (cos, sin) pairs.  (Staging the other epilogues' outputs for bulk stores was measured slower
+// than direct stores: the kernel would have to wait for its stores before exiting.)
+__host__ __device__ __forceinline__ uint32_t gemm_stage_bytes(int epi, int fp8, int Nt, int S, int H, int xb) {
+  (void)fp8;
+  (void)Nt;
+  (void)S;
+  (void)xb;
+  return epi == EPI_QKV ? static_cast<uint32_t>(H) * 64u * 8u : 0u;
+}
+
 // Largest chunk count of any split-K rank: the shared-memory layout is the same in every CTA.
 __host__ __device__ __forceinline__ int nk_max_of(const GemmArgs& a) { return (a.NKC + a.S - 1) / a.S; }
 
 // Bytes of the main loop and epilogue regions; the QKV epilogue's RoPE stage ([H][64] (cos, sin)
 // pairs of the m-block) follows them.
 __host__ __device__ __forceinline__ uint32_t gemm_rope_off(int Nt, int stages, int b_kind, int fp8, int S, int nk,
-                                                          int w4) {
+                                                          int w4, int epi_kind) {
   const GemmGeom g = gemm_geom(Nt, stages, b_kind, fp8, S, nk, w4, 1);   // kc0 odd: the larger group count
   const uint32_t kel = fp8 ? KCB : KCB / 2;
   const uint32_t main = g.gamma_off + (b_kind == B_NORM ? static_cast<uint32_t>(nk) * kel * 4u : 0u);
   const uint32_t TS = (Nt + S - 1) / S;
+  // split-K slices (S > 1) or the S == 1 accumulator rows overlay the ring; the residual epilogue's
+  // prefetched h rows (S > 1) follow at recv_off
   uint32_t epi = S > 1 ? static_cast<uint32_t>(S) * TS * BM * 4u : static_cast<uint32_t>(Nt) * RED_LD * 4u;
-  if (S > 1 && g.recv_off + 2u * TS * 64u * 4u > epi) epi = g.recv_off + 2u * TS * 64u * 4u;
+  if (S > 1 && epi_kind == EPI_RESID && g.recv_off + 2u * TS * 64u * 4u > epi) epi = g.recv_off + 2u * TS * 64u * 4u;
   return ((main > epi ? main : epi) + 15u) & ~15u;
 }
 
@@ -221,7 +234,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   const uint32_t tacc = sh.tmem_base;
   // QKV: (cos, sin) of this m-block's 64 rotate-half pairs at every action position, staged while
   // the previous kernel runs (the tables are static); read by the epilogue after the main loop
-  float2* rope_sh = reinterpret_cast<float2*>(dsm + gemm_rope_off(Nt, stages, NORM ? B_NORM : B_ROWS, FP8, S, nk_max_of(a), W4));
+  float2* rope_sh = reinterpret_cast<float2*>(dsm + gemm_rope_off(Nt, stages, NORM ? B_NORM : B_ROWS, FP8, S, nk_max_of(a), W4, EPI));
   if (EPI == EPI_QKV && mb < a.MB_rot && warp >= 2) {   // warps 2-7: the producer and MMA warps go on
     const int half = a.dh >> 1;
     for (int idx = tid - 64; idx < a.H * 64; idx += GEMM_THREADS - 64) {
@@ -566,8 +579,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         if (fok) {
           const float4 hv = make_float4(hold[u].x + acc[u][0], hold[u].y + acc[u][1], hold[u].z + acc[u][2],
                                         hold[u].w + acc[u][3]);
-          *reinterpret_cast<float4*>(a.h_out + htile_offset(t, f, Nt, a.KB)) = hv;
           sq = ((hv.x * hv.x + hv.y * hv.y) + hv.z * hv.z) + hv.w * hv.w;
+          *reinterpret_cast<float4*>(a.h_out + htile_offset(t, f, Nt, a.KB)) = hv;
           if (a.xb_out)
             *reinterpret_cast<uint2*>(a.xb_out + btile_offset(t, 2 * f, Nt, a.NKC_x)) =
                 make_uint2(pack_bf16x2(hv.x * g4.x, hv.y * g4.y), pack_bf16x2(hv.z * g4.z, hv.w * g4.w));
@@ -695,7 +708,7 @@ __host__ __device__ __forceinline__ AttnGeom attn_geom(int H, int dh, int KC, in
   g.q_bytes = static_cast<uint32_t>(Hp) * LD * 2;
   g.kv_bytes = 2u * static_cast<uint32_t>(KC) * LD * 2;
   g.rowb = static_cast<uint32_t>(dh + 4) * 4;                  // O row + (max, sum) + pad
-  g.obuf_bytes = static_cast<uint32_t>(Hp) * g.rowb;          // single-chunk case only, overlays Q/K/V
+  g.obuf_bytes = static_cast<uint32_t>(Hp) * g.rowb;          // partial rows of this chunk, overlays Q/K/V
   g.recv_off = 0;
   g.R = (H + C - 1) / C;
   return g;
@@ -852,24 +865,31 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
     }
   }
   if (C > 1) {
-    // partial rows straight from registers to the scratch; then one cluster barrier
+    // partial rows staged in shared memory (over the dead Q/K/V), one bulk store into the
+    // scratch, then one cluster barrier
+    __syncthreads();   // every warp is done with Q/K/V
     if (active) {
       const int r0 = rg * 16 + gq;
-      float* x0 = xs + (static_cast<size_t>(c) * H + r0) * OLD;
-      float* x8 = x0 + 8 * OLD;
 #pragma unroll
       for (int n = 0; n < DH / 8; ++n) {
         const int col = n * 8 + tq * 2;
-        if (r0 < H) *reinterpret_cast<float2*>(x0 + col) = make_float2(oacc[n][0], oacc[n][1]);
-        if (r0 + 8 < H) *reinterpret_cast<float2*>(x8 + col) = make_float2(oacc[n][2], oacc[n][3]);
+        *reinterpret_cast<float2*>(Obuf + r0 * OLD + col) = make_float2(oacc[n][0], oacc[n][1]);
+        *reinterpret_cast<float2*>(Obuf + (r0 + 8) * OLD + col) = make_float2(oacc[n][2], oacc[n][3]);
       }
       if (tq == 0) {
-        if (r0 < H) *reinterpret_cast<float2*>(x0 + DH) = make_float2(mrow[0], lrow[0]);
-        if (r0 + 8 < H) *reinterpret_cast<float2*>(x8 + DH) = make_float2(mrow[1], lrow[1]);
+        *reinterpret_cast<float2*>(Obuf + r0 * OLD + DH) = make_float2(mrow[0], lrow[0]);
+        *reinterpret_cast<float2*>(Obuf + (r0 + 8) * OLD + DH) = make_float2(mrow[1], lrow[1]);
       }
     }
-    if (tid == 0) TL(3);
-    __syncthreads();   // Q/K/V are dead in every warp: the slices below overlay them
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      bulk_s2g(xs + static_cast<size_t>(c) * H * OLD, Obuf, static_cast<uint32_t>(H) * OLD * 4u);
+      bulk_commit();
+      bulk_wait_all();
+      fence_proxy_async_global();
+      TL(3);
+    }
     cluster_arrive_release();
     cluster_wait_acquire();
     if (tid == 0) TL(6);
@@ -1523,8 +1543,8 @@ cudaError_t launch_ex(const void* func, dim3 grid, dim3 block, size_t smem, cuda
 
 }  // namespace
 
-size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4, int rope_rows) {
-  return gemm_rope_off(Nt, stages, b_kind, fp8, S, nk, w4) + static_cast<size_t>(rope_rows) * 64 * 8;
+size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4, int epi, int H, int xb) {
+  return gemm_rope_off(Nt, stages, b_kind, fp8, S, nk, w4, epi) + gemm_stage_bytes(epi, fp8, Nt, S, H, xb);
 }
 
 size_t gemm_scratch_bytes(int NT, int MB, int S, int Nt) {
@@ -1539,7 +1559,8 @@ size_t attn_smem_bytes(int H, int dh, int KC, int C, int umma) {
   if (umma) return uattn_geom(dh).total;   // the merge stage (<= 144 rows x (dh + 4) floats) overlays it
   const AttnGeom g = attn_geom(H, dh, KC, C);
   const size_t compute = static_cast<size_t>(g.q_bytes) + g.kv_bytes;
-  const size_t merge = C > 1 ? static_cast<size_t>(C) * g.R * g.rowb : g.obuf_bytes;
+  // the partial rows are staged over Q/K/V (obuf) before the merge stage overlays them
+  const size_t merge = std::max<size_t>(g.obuf_bytes, C > 1 ? static_cast<size_t>(C) * g.R * g.rowb : 0);
   return compute > merge ? compute : merge;
 }
 
@@ -1607,7 +1628,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int n_tiles, cudaStream_t s, bool 
   const void* f = gemm_kernel(a.epi, a.fp8, a.b_kind == B_NORM, a.w4);
   if (!f) return cudaErrorInvalidValue;
   return launch_ex(f, dim3(a.S, a.MB, n_tiles), dim3(GEMM_THREADS),
-                   gemm_smem_bytes(a.Nt, a.stages, a.b_kind, a.fp8, a.S, nk_max, a.w4, a.epi == EPI_QKV ? a.H : 0), s,
+                   gemm_smem_bytes(a.Nt, a.stages, a.b_kind, a.fp8, a.S, nk_max, a.w4, a.epi, a.H, a.xb_out != nullptr), s,
                    pdl, a.S, args);
 }
 

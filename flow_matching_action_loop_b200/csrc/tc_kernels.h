@@ -192,7 +192,7 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int B, cudaStream_t s, bool p
 cudaError_t launch_inproj_tc(const InprojArgs& a, cudaStream_t s, bool pdl);
 cudaError_t launch_final_tc(const FinalArgs& a, cudaStream_t s, bool pdl);
 cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s);
-size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4 = 0, int rope_rows = 0);
+size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4, int epi, int H, int xb);
 size_t gemm_scratch_bytes(int NT, int MB, int S, int Nt);
 size_t attn_scratch_bytes(int B, int Hq, int C, int H, int dh);
 size_t attn_smem_bytes(int H, int dh, int KC, int C, int umma);

@@ -176,23 +176,32 @@ void init_sizes(TensorPath* tp, const fr_config& c) {
 // weights next to it) and at most ~120 KB of shared memory; the cost counts waves, the split-K
 // exchange, and weight chunks that must stream after the dependency wait.  Wider tiles are
 // throughput-bound: no split-K unless the tiles leave most SMs idle.
-GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, int rope_rows, int nsm, int max_dyn) {
+GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, int epi, int H, int xb, int nsm,
+                     int max_dyn) {
   GemmPlan best;
   if (Nt > 64) {
-    best.S = (tiles * 2 <= nsm && NKC >= 2) ? 2 : 1;
-    const int chunks = ceil_div(NKC, best.S);
-    best.stages = std::min(chunks, MAX_STAGES);
-    while (best.stages > 1 && gemm_smem_bytes(Nt, best.stages, b_kind, fp8, best.S, chunks, w4, rope_rows) > static_cast<size_t>(max_dyn))
-      --best.stages;
-    return best;
+    // throughput-bound tiles: split K in two only when the tiles leave most SMs idle; fall back to
+    // the other split when the preferred one does not fit shared memory
+    const int pref = (tiles * 2 <= nsm && NKC >= 2) ? 2 : 1;
+    for (int S : {pref, 3 - pref}) {
+      if (S > NKC) continue;
+      const int chunks = ceil_div(NKC, S);
+      int stages = std::min(chunks, MAX_STAGES);
+      while (stages > 1 && gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, epi, H, xb) > static_cast<size_t>(max_dyn))
+        --stages;
+      best.S = S;
+      best.stages = stages;
+      if (gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, epi, H, xb) <= static_cast<size_t>(max_dyn)) return best;
+    }
+    return best;   // nothing fits: the launch reports it
   }
   const size_t cap = std::min<size_t>(static_cast<size_t>(max_dyn), 120 * 1024);
   double best_cost = 1e30;
   for (int S = 1; S <= 16 && S <= NKC; ++S) {
     const int chunks = ceil_div(NKC, S);
     int stages = std::min(chunks, MAX_STAGES);
-    while (stages > 1 && gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, rope_rows) > cap) --stages;
-    if (gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, rope_rows) > static_cast<size_t>(max_dyn)) continue;
+    while (stages > 1 && gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, epi, H, xb) > cap) --stages;
+    if (gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, epi, H, xb) > static_cast<size_t>(max_dyn)) continue;
     const int waves = ceil_div(tiles * S, nsm);
     const double cost = waves * (1.0 + (S > 1 ? 1.0 : 0.0) + 0.3 * (chunks - stages) + 0.05 * chunks);
     if (cost < best_cost - 1e-9) {
@@ -213,10 +222,14 @@ StepPlan make_plan(const TensorPath* tp, int B, int P) {
   p.NT = ceil_div(p.T, NT_MAX);
   p.Nt = static_cast<int>(align_up(ceil_div(p.T, p.NT), 16));
   const int norm_kind = tp->fp8 ? B_NORM : B_ROWS;   // bf16: the producer wrote bf16(h*gamma) already
-  p.qkv = choose_plan(tp->qkv.MB * p.NT, tp->qkv.NKC, p.Nt, norm_kind, tp->fp8, tp->w4, c.H, tp->nsm, tp->max_dyn);
-  p.o = choose_plan(tp->o.MB * p.NT, tp->o.NKC, p.Nt, B_ROWS, tp->fp8, tp->w4, 0, tp->nsm, tp->max_dyn);
-  p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, norm_kind, tp->fp8, tp->w4, 0, tp->nsm, tp->max_dyn);
-  p.dn = choose_plan(tp->dn.MB * p.NT, tp->dn.NKC, p.Nt, B_ROWS, tp->fp8, tp->w4, 0, tp->nsm, tp->max_dyn);
+  p.qkv = choose_plan(tp->qkv.MB * p.NT, tp->qkv.NKC, p.Nt, norm_kind, tp->fp8, tp->w4, EPI_QKV, c.H, 0, tp->nsm,
+                      tp->max_dyn);
+  p.o = choose_plan(tp->o.MB * p.NT, tp->o.NKC, p.Nt, B_ROWS, tp->fp8, tp->w4, EPI_RESID, c.H, !tp->fp8, tp->nsm,
+                    tp->max_dyn);
+  p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, norm_kind, tp->fp8, tp->w4, EPI_GELU, c.H, 0, tp->nsm,
+                     tp->max_dyn);
+  p.dn = choose_plan(tp->dn.MB * p.NT, tp->dn.NKC, p.Nt, B_ROWS, tp->fp8, tp->w4, EPI_RESID, c.H, !tp->fp8, tp->nsm,
+                     tp->max_dyn);
   p.attn_umma = attn_plan(P + c.H, attn_tiles(B, c.Hq, c.Hkv, c.H), tp->nsm, p.attn_C, p.attn_KC);
   return p;
 }
