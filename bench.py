@@ -32,6 +32,12 @@ METRIC = "µs per 10-step action chunk (batch 1); achieved HBM GB/s vs 8 TB/s"
 UNIT = "us/chunk"
 
 
+# DRAM bytes (read + written) of one whole chunk, summed over the launch list of one ncu capture of
+# this build's kernels (profiles/launches_pi05_bf16_b1.md gives the command).  Reported as the roofline
+# traffic for the workload it was taken on; other workloads report null.
+MEASURED_TRAFFIC = {"pi05_bf16_b1": 6.384e9 + 0.2001e9}
+
+
 def workload_bytes(cfg) -> dict:
     """Algorithmic bytes of one chunk: weights streamed once per Euler step plus the KV read per step."""
     D, F, dq, nkv = cfg.D, cfg.F, cfg.Hq * cfg.dh, cfg.Hkv * cfg.dh
@@ -293,7 +299,7 @@ def main(argv=None):
     # dominant kernel: the path's kernel set per chunk; per-launch algorithmic bytes over its device time
     achieved_gbs = wb["per_chunk"] / (ms_per_step * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved_gbs / hbm, 4), "traffic": None,
+                "frac": round(achieved_gbs / hbm, 4), "traffic": MEASURED_TRAFFIC.get(cfg.name),
                 "peak_kind": f"{peak_kind} HBM copy", "kernel": f"{loop.path} path, whole chunk",
                 "bytes_per_launch": wb["per_chunk"]}
     line = {
