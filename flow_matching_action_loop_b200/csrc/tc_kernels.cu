@@ -1395,7 +1395,7 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
   __shared__ float part[16][4];
   TL_DECL
   TL_BEGIN(1);
-  __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(dsm);   // [D][A]
+  __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(dsm);   // [A][D]: consecutive threads read consecutive n
   const int tid = threadIdx.x;
   const uint32_t wbytes = static_cast<uint32_t>(a.D) * a.A * 2;
   if (tid == 0) {
@@ -1425,9 +1425,8 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
     if (q * 256 >= a.D) continue;   // uniform across the block
     float hv = 0.f;
     if (n < a.D) {
-      const __nv_bfloat16* wr = wsm + static_cast<size_t>(n) * a.A;
       float acc = 0.f;
-      for (int i = 0; i < a.A; ++i) acc = fmaf(__bfloat162float(wr[i]), xs[i], acc);
+      for (int i = 0; i < a.A; ++i) acc = fmaf(__bfloat162float(wsm[static_cast<size_t>(i) * a.D + n]), xs[i], acc);
       hv = acc + base[q];
       a.h[htile_offset(t, n, a.Nt, a.KB)] = hv;
       if (a.xb)
@@ -1505,6 +1504,16 @@ __global__ void __launch_bounds__(256) k_final_tc(const __grid_constant__ FinalA
   __syncthreads();   // hn and ssq_sh are rewritten by the next token
   }
   if (tid == 0) TL(5);
+}
+
+// [rows][cols] float32 -> [cols][rows] bf16
+__global__ void k_to_bf16_t(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, int rows, int cols) {
+  const size_t n = static_cast<size_t>(rows) * cols;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t c = i / rows, r = i % rows;   // dst index i = c * rows + r
+    dst[i] = __float2bfloat16_rn(src[r * cols + c]);
+  }
 }
 
 __global__ void k_to_bf16(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, size_t n) {
@@ -1668,6 +1677,12 @@ cudaError_t launch_final_tc(const FinalArgs& a, cudaStream_t s, bool pdl) {
 
 cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s) {
   k_to_bf16<<<static_cast<unsigned>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0, s>>>(src, dst, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_to_bf16_t(const float* src, __nv_bfloat16* dst, int rows, int cols, cudaStream_t s) {
+  const size_t n = static_cast<size_t>(rows) * cols;
+  k_to_bf16_t<<<static_cast<unsigned>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0, s>>>(src, dst, rows, cols);
   return cudaGetLastError();
 }
 

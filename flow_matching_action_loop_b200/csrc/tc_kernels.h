@@ -158,7 +158,7 @@ inline int attn_plan(int S, int tiles, int nsm, int& C, int& KC) {
 struct InprojArgs {
   int max_ctas;                // grid cap (tokens are strided over the CTAs); 0: one CTA per token
   const float* x;              // [T][A] state at the start of the step
-  const __nv_bfloat16* w_in;   // [D][A]
+  const __nv_bfloat16* w_in;   // [A][D] (transposed by the loader)
   const float* b_in;
   const float* temb;           // [D] of this step
   float* h;                    // tiled h
@@ -192,6 +192,7 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int B, cudaStream_t s, bool p
 cudaError_t launch_inproj_tc(const InprojArgs& a, cudaStream_t s, bool pdl);
 cudaError_t launch_final_tc(const FinalArgs& a, cudaStream_t s, bool pdl);
 cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s);
+cudaError_t launch_to_bf16_t(const float* src, __nv_bfloat16* dst, int rows, int cols, cudaStream_t s);
 size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4, int epi, int H, int xb);
 size_t gemm_scratch_bytes(int NT, int MB, int S, int Nt);
 size_t attn_scratch_bytes(int B, int Hq, int C, int H, int dh);

@@ -107,7 +107,7 @@ struct TensorPath {
   float* xscratch = nullptr;     // split-K / key-chunk exchange scratch (L2-resident), shared by all kernels
   size_t xscratch_bytes = 0;
   float* xs = nullptr;           // [T_max][A] state between steps
-  __nv_bfloat16* w_in_bf = nullptr;   // [D][A]
+  __nv_bfloat16* w_in_bf = nullptr;   // [A][D]
   __nv_bfloat16* w_out_bf = nullptr;  // [A][D]
   cudaStream_t cap = nullptr;
   std::map<std::pair<int, int>, GraphEntry> graphs;
@@ -671,7 +671,7 @@ int tensor_path_finish_load(TensorPath* tp, cudaStream_t s) {
   const fr_config& c = tp->c;
   FR_CUDA(cudaMemcpy(tp->gains, tp->gains_host.data(), tp->gains_host.size() * 4, cudaMemcpyHostToDevice));
   // in/out-proj weights hold bf16-rounded values already: the conversion is exact
-  FR_CUDA(launch_to_bf16(tp->tb.w_in, tp->w_in_bf, static_cast<size_t>(c.D) * c.A, s));
+  FR_CUDA(launch_to_bf16_t(tp->tb.w_in, tp->w_in_bf, c.D, c.A, s));
   FR_CUDA(launch_to_bf16(tp->tb.w_out, tp->w_out_bf, static_cast<size_t>(c.A) * c.D, s));
   FR_CUDA(cudaStreamSynchronize(s));
   return FR_OK;
