@@ -1,0 +1,52 @@
+"""bench.py's multi-rank host logic on CPU: two gloo ranks, as torchrun would launch them.
+
+The timing all-reduce returns the maximum over the ranks on every rank, and the whole-job time per
+chunk counts the chunks of all ranks (replicas, weak scaling).
+"""
+import os
+import socket
+
+import pytest
+
+torch = pytest.importorskip("torch")
+import torch.distributed as dist  # noqa: E402
+import torch.multiprocessing as mp  # noqa: E402
+
+import bench  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        got = bench.max_over_ranks(10.0 + rank, world)
+        bench.barrier(world)
+        q.put((rank, got))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_timing_is_the_max_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = dict(q.get(timeout=5) for _ in range(2))
+    assert got == {0: 11.0, 1: 11.0}
+
+
+def test_whole_job_time_per_chunk_counts_every_rank():
+    # 2 ranks x 50 calls x 32 chunks in 1000 ms -> 1e6 us / 3200 chunks
+    assert bench.job_us_per_chunk(1000.0, 2, 50, 32) == pytest.approx(312.5)
+    assert bench.job_us_per_chunk(9.0, 1, 1, 1) == pytest.approx(9000.0)
