@@ -205,6 +205,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   const int kel = FP8 ? KCB : KCB / 2;            // K elements per chunk
   const GemmGeom gm = gemm_geom(Nt, stages, NORM ? B_NORM : B_ROWS, FP8, S, nk, W4, kc0);
   const int g0 = kc0 / 2;                          // w4: first scale group of this CTA's k-range
+  // ring slot addresses: B_NORM interleaves [A | raw h] per slot; otherwise the A slots come first and
+  // the B slots follow contiguously, so that the B chunks resident before the main loop arrive in one copy
+  auto a_slot = [&](int s) -> uint8_t* { return dsm + (NORM ? s * gm.slot : s * gm.a_bytes); };
+  auto b_slot = [&](int s) -> uint8_t* {
+    return dsm + (NORM ? s * gm.slot + gm.a_bytes : stages * gm.a_bytes + s * (gm.slot - gm.a_bytes));
+  };
   float* gsm = reinterpret_cast<float*>(dsm + gm.gamma_off);
 
   if (tid == 0) {
@@ -250,7 +256,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       const uint8_t* wsrc = a.W + (static_cast<size_t>(mb) * a.NKC + kc0) * gm.a_bytes;
       auto issue_b = [&](int i) {
         const int s = i % stages;
-        uint8_t* bdst = dsm + s * gm.slot + gm.a_bytes;
+        uint8_t* bdst = b_slot(s);
         if (norm) {
           const int kb = (kc0 + i) * (FP8 ? 2 : 1);
           mbar_arrive_expect_tx(&sh.raw_b[s], gm.raw_bytes);
@@ -269,7 +275,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
           bulk_g2s(dsm + gm.rawa_off + s * W4_CHUNK, w4src + static_cast<size_t>(i) * W4_CHUNK, W4_CHUNK, &sh.raw_a[s]);
         } else {
           mbar_arrive_expect_tx(&sh.full_a[s], gm.a_bytes);
-          bulk_g2s(dsm + s * gm.slot, wsrc + static_cast<size_t>(i) * gm.a_bytes, gm.a_bytes, &sh.full_a[s]);
+          bulk_g2s(a_slot(s), wsrc + static_cast<size_t>(i) * gm.a_bytes, gm.a_bytes, &sh.full_a[s]);
         }
       };
       const int pre = nk < stages ? nk : stages;
@@ -281,7 +287,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       for (int i = 0; i < pre; ++i) issue_a(i);   // weights first: they do not depend on the previous kernel
       grid_dep_wait();
       TL(1);
-      for (int i = 0; i < pre; ++i) issue_b(i);
+      if (!NORM && Nt <= 64) {   // batch-1 tiles: B chunks 0..pre-1 are contiguous in global and in shared memory: one copy
+        const uint32_t tb = static_cast<uint32_t>(Nt) * KCB;
+        mbar_arrive_expect_tx(&sh.full_b[0], pre * tb);
+        bulk_g2s(b_slot(0), a.act + (static_cast<size_t>(nt) * a.NKC + kc0) * tb, pre * tb, &sh.full_b[0]);
+        for (int i = 1; i < pre; ++i) mbar_arrive(&sh.full_b[i]);   // round 0 of these slots is covered by slot 0
+      } else {
+        for (int i = 0; i < pre; ++i) issue_b(i);
+      }
       if (S > 1 && EPI == EPI_RESID) {   // residual rows of this CTA's tokens, for the epilogue
         const int r0 = ks * Nt / S, r1 = (ks + 1) * Nt / S;
         const uint32_t rb = static_cast<uint32_t>(r1 - r0) * 256u;
@@ -317,13 +330,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       for (int i = 0; i < nk; ++i) {
         const int s = i % stages;
         const uint32_t par = (i / stages) & 1;
-        if (!mbar_wait(&sh.full_a[s], par, WAIT_LIMIT_NS) || !mbar_wait(&sh.full_b[s], par, WAIT_LIMIT_NS)) {
+        // round 0 of batch-1 tiles without B_NORM: one copy brought every resident B chunk and completes
+        // slot 0; the chunks after it need no wait of their own
+        const bool wait_b = NORM || Nt > 64 || i >= stages || i == 0;
+        if (!mbar_wait(&sh.full_a[s], par, WAIT_LIMIT_NS) || (wait_b && !mbar_wait(&sh.full_b[s], par, WAIT_LIMIT_NS))) {
           report_timeout(a.status, 0x200);
           break;
         }
         tc_fence_after();
         if (i == 0) TL(6);
-        const uint32_t a0 = smem_u32(dsm + s * gm.slot), b0 = a0 + gm.a_bytes;
+        const uint32_t a0 = smem_u32(a_slot(s)), b0 = smem_u32(b_slot(s));
 #pragma unroll
         for (int k = 0; k < KCB / 32; ++k) {
           const uint64_t ad = smem_desc(a0 + k * 2 * BM * 16, BM * 16, 128);
@@ -347,7 +363,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       const uint32_t* raw = reinterpret_cast<const uint32_t*>(dsm + gm.rawa_off + s * W4_CHUNK);
       const __nv_bfloat16* scl =
           reinterpret_cast<const __nv_bfloat16*>(dsm + gm.scl_off) + ((kc0 + i) / 2 - g0) * BM;
-      uint8_t* adst = dsm + s * gm.slot;
+      uint8_t* adst = a_slot(s);
       for (int it = st; it < 8 * BM; it += CONV_THREADS) {
         const int j = it >> 7, r = it & (BM - 1);     // consecutive threads: consecutive rows
         const uint32_t wv = raw[it];
@@ -404,7 +420,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         report_timeout(a.status, 0x300);
         break;
       }
-      uint8_t* breg = dsm + s * gm.slot + gm.a_bytes;
+      uint8_t* breg = b_slot(s);
       const float* raw = reinterpret_cast<const float*>(breg);
       const float* gch = gsm + i * kel;
       uint4 res[CONV_ITEMS];
@@ -935,7 +951,6 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
   const float* src = (C > 1) ? stage : Obuf;
   const size_t sstride = (C > 1) ? static_cast<size_t>(gm.R) : 0;
   const int roff = (C > 1) ? 0 : r_lo;
-  auto ld1 = [&](const float* p) -> float { return *p; };
   auto ld2 = [&](const float* p) -> float2 { return *reinterpret_cast<const float2*>(p); };
   if (tid == 0) TL(4);
   const int nr = r_hi - r_lo;
@@ -969,22 +984,45 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
   __syncthreads();
   if (tid == 0) TL(7);
   const float inv_sa = (a.fp8 && a.s_a) ? 1.0f / *a.s_a : 1.0f;
-  for (int it = tid; it < nr * DH; it += blockDim.x) {
-    const int rr = it / DH, d = it % DH;
-    float v[16];
+  // eight consecutive features per work item: one 16-byte (bf16) or 8-byte (e4m3) store
+  for (int it = tid; it < nr * (DH / 8); it += blockDim.x) {
+    const int rr = it / (DH / 8), d0 = (it % (DH / 8)) * 8;
+    float acc[8];
 #pragma unroll
-    for (int s = 0; s < 16; ++s) v[s] = s < C ? ld1(src + (s * sstride + roff + rr) * OLD + d) : 0.f;
-    float acc = 0.f;
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
     for (int s = 0; s < 16; ++s)
-      if (s < C) acc += w_sh[s][rr] * v[s];                                 // rank order
-    acc *= inv_den[rr];
+      if (s < C) {
+        const float w = w_sh[s][rr];
+        const float* p = src + (s * sstride + roff + rr) * OLD + d0;
+        const float4 v0 = *reinterpret_cast<const float4*>(p), v1 = *reinterpret_cast<const float4*>(p + 4);
+        acc[0] += w * v0.x;   // rank order
+        acc[1] += w * v0.y;
+        acc[2] += w * v0.z;
+        acc[3] += w * v0.w;
+        acc[4] += w * v1.x;
+        acc[5] += w * v1.y;
+        acc[6] += w * v1.z;
+        acc[7] += w * v1.w;
+      }
+    const float id = inv_den[rr];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] *= id;
     const int t = b * H + r_lo + rr;
-    const int kidx = j * DH + d;
-    if (a.o_rowmajor)
-      reinterpret_cast<__nv_bfloat16*>(a.o)[static_cast<size_t>(t) * a.Hq * DH + kidx] = __float2bfloat16_rn(acc);
-    else if (a.fp8) a.o[btile_offset(t, kidx, a.Nt, a.NKC_o)] = to_e4m3(acc * inv_sa);
-    else *reinterpret_cast<__nv_bfloat16*>(a.o + btile_offset(t, 2 * kidx, a.Nt, a.NKC_o)) = __float2bfloat16_rn(acc);
+    const int kidx = j * DH + d0;
+    if (a.o_rowmajor) {
+      *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + static_cast<size_t>(t) * a.Hq * DH + kidx) =
+          make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                     pack_bf16x2(acc[6], acc[7]));
+    } else if (a.fp8) {
+      *reinterpret_cast<uint2*>(a.o + btile_offset(t, kidx, a.Nt, a.NKC_o)) =
+          make_uint2(pack_e4m3x4(acc[0] * inv_sa, acc[1] * inv_sa, acc[2] * inv_sa, acc[3] * inv_sa),
+                     pack_e4m3x4(acc[4] * inv_sa, acc[5] * inv_sa, acc[6] * inv_sa, acc[7] * inv_sa));
+    } else {
+      *reinterpret_cast<uint4*>(a.o + btile_offset(t, 2 * kidx, a.Nt, a.NKC_o)) =
+          make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                     pack_bf16x2(acc[6], acc[7]));
+    }
   }
   __syncthreads();
   if (tid == 0) TL(5);
