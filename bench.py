@@ -35,7 +35,7 @@ UNIT = "us/chunk"
 # DRAM bytes (read + written) of one whole chunk, summed over the launch list of one ncu capture of
 # this build's kernels (profiles/launches_pi05_bf16_b1.md gives the command).  Reported as the roofline
 # traffic for the workload it was taken on; other workloads report null.
-MEASURED_TRAFFIC = {"pi05_bf16_b1": 6.384e9 + 0.2001e9}
+MEASURED_TRAFFIC = {"pi05_bf16_b1": 6.384e9 + 0.1956e9}
 
 
 def workload_bytes(cfg) -> dict:
