@@ -19,12 +19,13 @@ import numpy as np
 from ._abi import (  # noqa: F401
     DTYPES, FR_DTYPE_BF16, FR_DTYPE_F32, FR_DTYPE_FP8, FR_DTYPE_W4A16, FR_ERR_ARG, FR_ERR_CUDA, FR_ERR_DEVICE, FR_ERR_SHAPE,
     FR_ERR_STATE, FR_ERR_TIMEOUT, FR_ERR_UNSUPPORTED, FR_OK, FR_PATH_AUTO, FR_PATH_STEPWISE, FR_PATH_TENSOR,
-    FR_ATTENTION_NOALLOC_SCRATCH_BYTES, FR_PREFIX_K_ROTATED, FrConfig, FrError, fr_attention,
-    fr_attention_noalloc, fr_attention_scratch_bytes, fr_calibrate, fr_create,
-    fr_denoise, fr_destroy, fr_get_rope_tables,
-    fr_get_scales, fr_last_error, fr_launches_per_call, fr_load_weights, fr_path_name, fr_quantize_e4m3, fr_quantize_w4,
-    fr_read_kv, fr_rope_tables, fr_round_bf16, fr_set_prefix_kv, fr_set_scales, fr_sync_status, header_functions,
-    load_library, make_config,
+    FR_ATTENTION_NOALLOC_SCRATCH_BYTES, FR_CAPSULE_MAGIC, FR_PREFIX_K_ROTATED, FrCapsule, FrConfig, FrError,
+    fr_attention, fr_attention_noalloc, fr_attention_scratch_bytes, fr_calibrate, fr_capsule_bytes,
+    fr_capsule_restore, fr_capsule_save, fr_create, fr_denoise, fr_destroy, fr_get_buffer, fr_get_rope_tables,
+    fr_get_scales, fr_graph_count, fr_last_error, fr_launches_per_call, fr_load_weights, fr_path_name,
+    fr_quantize_e4m3, fr_quantize_w4, fr_read_kv, fr_refresh_prefix_kv, fr_rope_tables, fr_round_bf16,
+    fr_set_graph_capacity, fr_set_prefix_kv, fr_set_scales, fr_sync_status, header_functions, load_library,
+    make_config,
 )
 
 load_library()
@@ -76,6 +77,7 @@ class ActionExpertLoop:
         pk = self._dev(k, self.kv_dtype, shape, "fr_set_prefix_kv")
         pv = self._dev(v, self.kv_dtype, shape, "fr_set_prefix_kv")
         fr_set_prefix_kv(self.h, pk, pv, B, P, FR_PREFIX_K_ROTATED if rotated else 0, self._stream())
+        self._P = P
 
     def calibrate(self, x0, k, v) -> None:
         c = self.cfg
@@ -84,6 +86,7 @@ class ActionExpertLoop:
         fr_calibrate(self.h, self._dev(x0, self._torch.float32, (B, c.H, c.A), "fr_calibrate"),
                      self._dev(k, self.kv_dtype, shape, "fr_calibrate"),
                      self._dev(v, self.kv_dtype, shape, "fr_calibrate"), B, P, self._stream())
+        self._P = P   # the calibration prefix is now the cached one
 
     def denoise(self, x0, out=None):
         c = self.cfg
@@ -94,6 +97,53 @@ class ActionExpertLoop:
         po = self._dev(out, self._torch.float32, (B, c.H, c.A), "fr_denoise")
         fr_denoise(self.h, px, po, B, self._stream())
         return out
+
+    # -- execution contract across chunks
+    def refresh_prefix_kv(self, k, v, slots, rotated: bool = False) -> None:
+        """Replace the prefix of batch slots `slots` (k, v: [L][len(slots)][P][Hkv][dh])."""
+        c = self.cfg
+        L, n, P = k.shape[0], k.shape[1], k.shape[2]
+        shape = (L, n, P, c.Hkv, c.dh)
+        fr_refresh_prefix_kv(self.h, self._dev(k, self.kv_dtype, shape, "fr_refresh_prefix_kv"),
+                             self._dev(v, self.kv_dtype, shape, "fr_refresh_prefix_kv"), list(slots), P,
+                             FR_PREFIX_K_ROTATED if rotated else 0, self._stream())
+
+    def buffer(self, name: str):
+        """(device address, bytes) of the handle's named buffer `name`."""
+        return fr_get_buffer(self.h, name)
+
+    def save_capsule(self, B: int, x=None):
+        """Snapshot slots 0..B-1 (and x [B][H][A] if given) into a new device buffer: (buffer, description)."""
+        torch = self._torch
+        c = self.cfg
+        n = fr_capsule_bytes(make_config(c, self.B_max, self.P_max), B, self._prefix_P(), x is not None)
+        if n == 0:
+            raise FrError(FR_ERR_SHAPE, "fr_capsule_bytes", f"no capsule size for B={B}")
+        buf = torch.empty(n, dtype=torch.uint8, device=f"cuda:{self.device}")
+        px = self._dev(x, torch.float32, (B, c.H, c.A), "fr_capsule_save") if x is not None else 0
+        desc = fr_capsule_save(self.h, buf.data_ptr(), n, B, px, self._stream())
+        return buf, desc
+
+    def restore_capsule(self, capsule, B: Optional[int] = None, sample_map=None, x_out=None) -> None:
+        """Make (buffer, description) the prefix state; sample_map forks or reorders its samples."""
+        buf, desc = capsule
+        c = self.cfg
+        B = B or (len(sample_map) if sample_map is not None else desc.B)
+        px = self._dev(x_out, self._torch.float32, (B, c.H, c.A), "fr_capsule_restore") if x_out is not None else 0
+        fr_capsule_restore(self.h, buf.data_ptr(), desc, B, sample_map, px, self._stream())
+        self._P = desc.P
+
+    def set_graph_capacity(self, capacity: int) -> None:
+        fr_set_graph_capacity(self.h, capacity)
+
+    def graph_count(self) -> int:
+        return fr_graph_count(self.h)
+
+    def _prefix_P(self) -> int:
+        P = getattr(self, "_P", None)
+        if P is None:
+            raise FrError(FR_ERR_STATE, "fr_capsule_save", "no prefix set")
+        return P
 
     def get_scales(self):
         sa, sw = fr_get_scales(self.h, self.cfg.L * 4)

@@ -55,6 +55,15 @@ class FrWeights(ctypes.Structure):
                [(n, _FP) for n in ("w_in", "b_in", "w_out", "b_out", "w_t1", "b_t1", "w_t2", "b_t2", "g_f")]
 
 
+FR_CAPSULE_MAGIC = 0x46524350
+
+
+class FrCapsule(ctypes.Structure):
+    _fields_ = [("magic", ctypes.c_uint32), ("L", ctypes.c_int), ("Hkv", ctypes.c_int), ("dh", ctypes.c_int),
+                ("kv_bytes_per_elem", ctypes.c_int), ("H", ctypes.c_int), ("A", ctypes.c_int),
+                ("B", ctypes.c_int), ("P", ctypes.c_int), ("has_x", ctypes.c_int), ("bytes", ctypes.c_size_t)]
+
+
 _lib: Optional[ctypes.CDLL] = None
 
 
@@ -96,6 +105,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fr_attention_scratch_bytes": (ctypes.c_size_t, [c_int, c_int, c_int, c_int, c_int]),
         "fr_attention_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
                                          c_int, c_void_p]),
+        "fr_refresh_prefix_kv": (c_int, [H, c_void_p, c_void_p, ctypes.POINTER(c_int), c_int, c_int, c_uint,
+                                         c_void_p]),
+        "fr_get_buffer": (c_int, [H, c_char_p, ctypes.POINTER(c_void_p), ctypes.POINTER(ctypes.c_size_t)]),
+        "fr_capsule_bytes": (ctypes.c_size_t, [ctypes.POINTER(FrConfig), c_int, c_int, c_int]),
+        "fr_capsule_save": (c_int, [H, c_void_p, ctypes.c_size_t, c_int, c_void_p, ctypes.POINTER(FrCapsule),
+                                    c_void_p]),
+        "fr_capsule_restore": (c_int, [H, c_void_p, ctypes.POINTER(FrCapsule), ctypes.POINTER(c_int), c_int,
+                                       c_void_p, c_void_p]),
+        "fr_set_graph_capacity": (c_int, [H, c_int]),
+        "fr_graph_count": (c_int, [H]),
         "fr_round_bf16": (None, [_FP, ctypes.POINTER(ctypes.c_uint16), ctypes.c_size_t]),
         "fr_quantize_e4m3": (None, [_FP, ctypes.POINTER(ctypes.c_uint8), ctypes.c_size_t, ctypes.c_double]),
         "fr_quantize_w4": (c_int, [_FP, c_int, c_int, ctypes.POINTER(ctypes.c_int8), ctypes.POINTER(ctypes.c_uint16)]),
@@ -214,6 +233,51 @@ def fr_path_name(h) -> str:
 
 def fr_launches_per_call(h, B: int) -> int:
     return load_library().fr_launches_per_call(h, B)
+
+
+def _ints(values):
+    a = (ctypes.c_int * len(values))(*[int(v) for v in values])
+    return a
+
+
+def fr_refresh_prefix_kv(h, k_dev: int, v_dev: int, slots, P: int, flags: int = 0, stream: int = 0) -> None:
+    sl = _ints(slots)
+    _check(load_library().fr_refresh_prefix_kv(h, k_dev, v_dev, sl, len(sl), P, flags, stream),
+           "fr_refresh_prefix_kv")
+
+
+def fr_get_buffer(h, name: str):
+    """(device address, bytes) of a named buffer of the handle."""
+    p = ctypes.c_void_p()
+    n = ctypes.c_size_t()
+    _check(load_library().fr_get_buffer(h, name.encode(), ctypes.byref(p), ctypes.byref(n)), "fr_get_buffer")
+    return p.value or 0, n.value
+
+
+def fr_capsule_bytes(cfg: FrConfig, B: int, P: int, with_x: bool) -> int:
+    return load_library().fr_capsule_bytes(ctypes.byref(cfg), B, P, 1 if with_x else 0)
+
+
+def fr_capsule_save(h, cap_dev: int, cap_bytes: int, B: int, x_dev: int = 0, stream: int = 0) -> FrCapsule:
+    d = FrCapsule()
+    _check(load_library().fr_capsule_save(h, cap_dev, cap_bytes, B, x_dev or None, ctypes.byref(d), stream),
+           "fr_capsule_save")
+    return d
+
+
+def fr_capsule_restore(h, cap_dev: int, desc: FrCapsule, B: int, sample_map=None, x_dev: int = 0,
+                       stream: int = 0) -> None:
+    m = _ints(sample_map) if sample_map is not None else None
+    _check(load_library().fr_capsule_restore(h, cap_dev, ctypes.byref(desc), m, B, x_dev or None, stream),
+           "fr_capsule_restore")
+
+
+def fr_set_graph_capacity(h, capacity: int) -> None:
+    _check(load_library().fr_set_graph_capacity(h, capacity), "fr_set_graph_capacity")
+
+
+def fr_graph_count(h) -> int:
+    return _check(load_library().fr_graph_count(h), "fr_graph_count")
 
 
 def fr_attention(q: int, k: int, v: int, o: int, B: int, Hq: int, Hkv: int, H: int, S_keys: int, dh: int,

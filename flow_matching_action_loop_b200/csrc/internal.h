@@ -61,9 +61,18 @@ void launch_gemm(const float* A, int lda, const void* W, int wtype, const float*
 void launch_rope_qkv(const float* qkv, float* q, void* kv_k, void* kv_v, int kv_bf16,
                      const float* cos_t, const float* sin_t, int B, int H, int P, int S_max,
                      int Hq, int Hkv, int dh, int round_bf16, cudaStream_t s);
+// Batch slots written by one prefix-ingest launch: source sample b0 + i goes to slot slot[i]
+// (n == 0: slot b0 + i).
+constexpr int SLOT_MAP_MAX = 64;
+struct SlotMap {
+  int n;
+  int slot[SLOT_MAP_MAX];
+};
+// in [L][B_src][P][Hkv][dh] samples b0 .. b0+nb-1 -> cache [L][B_max][Hkv][S_max][dh]
 void launch_prefix_ingest(const void* k_in, const void* v_in, void* kv_k, void* kv_v, int kv_bf16,
-                          const float* cos_t, const float* sin_t, int L, int B, int B_max, int P,
-                          int S_max, int Hkv, int dh, int rotate, cudaStream_t s);
+                          const float* cos_t, const float* sin_t, int L, int B_src, int b0, int nb,
+                          const SlotMap& map, int B_max, int P, int S_max, int Hkv, int dh, int rotate,
+                          cudaStream_t s);
 void launch_attention(const float* q, const void* kv_k, const void* kv_v, int kv_bf16, float* act,
                       int ld_act, int B, int H, int P, int S_max, int Hq, int Hkv, int dh,
                       int qmode, const float* s_a, unsigned* amax, cudaStream_t s);
@@ -73,6 +82,23 @@ void launch_final(const float* h, const float* g_f, const float* w_out, const fl
                   float* x, int T, int D, int A, float eps, float dt, int round_bf16, cudaStream_t s);
 
 enum WType : int { W_F32 = 0, W_BF16 = 1, W_E4M3 = 2 };
+
+// ------------------------------------------------------------------ state copies (state.cu)
+// Rows (outer, sample, mid, row) of row_bytes (a multiple of 4) copied for each of `parts`
+// (src, dst) pairs; destination sample b (b < n_sample <= SLOT_MAP_MAX) reads source sample
+// map[b].  Strides are in bytes.
+struct RowCopy {
+  const char* src[2];
+  char* dst[2];
+  int parts;
+  long long n_outer, n_sample, n_mid, n_row;
+  long long s_outer, s_sample, s_mid, s_row;
+  long long d_outer, d_sample, d_mid, d_row;
+  long long row_bytes;
+  int row_words;   // set by the launcher
+  int map[SLOT_MAP_MAX];
+};
+void launch_state_copy(RowCopy c, cudaStream_t s);
 
 // Kernel attributes of the tensor-core kernels, set once per device (ops.cu).
 cudaError_t ensure_tc_kernels(int* dev_out);

@@ -473,13 +473,287 @@ int fr_set_prefix_kv(fr_handle* h, const void* k_dev, const void* v_dev, int B, 
   FR_CUDA(cudaSetDevice(h->device));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int rotate = (flags & FR_PREFIX_K_ROTATED) ? 0 : 1;
-  launch_prefix_ingest(k_dev, v_dev, h->kv_k, h->kv_v, h->kv_bf, h->rope_cos, h->rope_sin, c.L, B, c.B_max, P,
-                       h->S_max, c.Hkv, c.dh, rotate, s);
+  SlotMap identity{};
+  launch_prefix_ingest(k_dev, v_dev, h->kv_k, h->kv_v, h->kv_bf, h->rope_cos, h->rope_sin, c.L, B, 0, B, identity,
+                       c.B_max, P, h->S_max, c.Hkv, c.dh, rotate, s);
   int rc = check_launch("prefix ingest kernel");
   if (rc) return rc;
   h->prefix_B = B;
   h->prefix_P = P;
   return FR_OK;
+}
+
+// ------------------------------------------------------------------ execution contract across chunks
+
+int fr_refresh_prefix_kv(fr_handle* h, const void* k_dev, const void* v_dev, const int* slots, int n, int P,
+                         unsigned flags, fr_stream_t stream) {
+  if (!h || !k_dev || !v_dev || !slots || n < 1) {
+    set_error("fr_refresh_prefix_kv: NULL argument or n < 1");
+    return FR_ERR_ARG;
+  }
+  if (flags & ~FR_PREFIX_K_ROTATED) {
+    set_error("fr_refresh_prefix_kv: unknown flag bits 0x%x", flags);
+    return FR_ERR_ARG;
+  }
+  if (h->prefix_B < 1) {
+    set_error("fr_refresh_prefix_kv: no prefix set (call fr_set_prefix_kv or fr_capsule_restore first)");
+    return FR_ERR_STATE;
+  }
+  if (P != h->prefix_P) {
+    set_error("fr_refresh_prefix_kv: P=%d differs from the cached prefix length %d", P, h->prefix_P);
+    return FR_ERR_SHAPE;
+  }
+  std::vector<char> seen(h->prefix_B, 0);
+  for (int i = 0; i < n; ++i) {
+    if (slots[i] < 0 || slots[i] >= h->prefix_B) {
+      set_error("fr_refresh_prefix_kv: slot %d outside the %d cached samples", slots[i], h->prefix_B);
+      return FR_ERR_SHAPE;
+    }
+    if (seen[slots[i]]) {
+      set_error("fr_refresh_prefix_kv: slot %d given twice", slots[i]);
+      return FR_ERR_ARG;
+    }
+    seen[slots[i]] = 1;
+  }
+  const fr_config& c = h->cfg;
+  FR_CUDA(cudaSetDevice(h->device));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int rotate = (flags & FR_PREFIX_K_ROTATED) ? 0 : 1;
+  for (int b0 = 0; b0 < n; b0 += SLOT_MAP_MAX) {
+    SlotMap m{};
+    m.n = std::min(SLOT_MAP_MAX, n - b0);
+    for (int i = 0; i < m.n; ++i) m.slot[i] = slots[b0 + i];
+    launch_prefix_ingest(k_dev, v_dev, h->kv_k, h->kv_v, h->kv_bf, h->rope_cos, h->rope_sin, c.L, n, b0, m.n, m,
+                         c.B_max, P, h->S_max, c.Hkv, c.dh, rotate, s);
+    int rc = check_launch("prefix ingest kernel");
+    if (rc) return rc;
+  }
+  return FR_OK;
+}
+
+int fr_get_buffer(const fr_handle* h, const char* name, void** dev, size_t* bytes) {
+  if (!h || !name || !dev || !bytes) {
+    set_error("fr_get_buffer: NULL argument");
+    return FR_ERR_ARG;
+  }
+  const fr_config& c = h->cfg;
+  const size_t rope = static_cast<size_t>(h->S_max) * (c.dh / 2) * sizeof(float);
+  struct Named {
+    const char* name;
+    void* p;
+    size_t n;
+  };
+  const Named table[] = {
+      {"kv_k", h->kv_k, h->kv_layer_bytes * c.L},
+      {"kv_v", h->kv_v, h->kv_layer_bytes * c.L},
+      {"rope_cos", h->rope_cos, rope},
+      {"rope_sin", h->rope_sin, rope},
+      {"temb", h->temb, static_cast<size_t>(c.K) * c.D * sizeof(float)},
+      {"s_act", h->s_a, static_cast<size_t>(c.L) * PI_COUNT * sizeof(float)},
+      {"status", h->status, sizeof(unsigned)},
+  };
+  for (const Named& e : table)
+    if (std::strcmp(e.name, name) == 0) {
+      *dev = e.p;
+      *bytes = e.n;
+      return FR_OK;
+    }
+  set_error("fr_get_buffer: no buffer named '%s'", name);
+  return FR_ERR_ARG;
+}
+
+namespace {
+
+struct CapsuleLayout {
+  size_t kv_bytes = 0;   // one of K or V: [L][B][Hkv][P][dh]
+  size_t v_off = 0, x_off = 0, total = 0;
+};
+
+CapsuleLayout capsule_layout(const fr_config& c, int B, int P, int with_x) {
+  CapsuleLayout l;
+  const size_t elem = c.dtype == FR_DTYPE_F32 ? 4 : 2;
+  l.kv_bytes = static_cast<size_t>(c.L) * B * c.Hkv * P * c.dh * elem;
+  l.v_off = align_up(l.kv_bytes, 256);
+  l.x_off = l.v_off + align_up(l.kv_bytes, 256);
+  l.total = l.x_off + (with_x ? align_up(static_cast<size_t>(B) * c.H * c.A * sizeof(float), 256) : 0);
+  return l;
+}
+
+// Rows of the prefix KV between the handle's cache and a capsule's [L][B][Hkv][P][dh] layout.
+// to_capsule: cache slot map[b] -> capsule sample b; otherwise capsule sample map[b] -> slot b.
+int copy_prefix(const fr_handle* h, char* cap, int B_cap, int P, const int* map, int n, bool to_capsule,
+                cudaStream_t s) {
+  const fr_config& c = h->cfg;
+  const long long rowb = static_cast<long long>(c.dh) * (h->kv_bf ? 2 : 4);
+  const CapsuleLayout lay = capsule_layout(c, B_cap, P, 0);
+  const long long cache[4] = {static_cast<long long>(h->kv_layer_bytes), c.Hkv * h->S_max * rowb, h->S_max * rowb, rowb};
+  const long long capsule[4] = {static_cast<long long>(B_cap) * c.Hkv * P * rowb, c.Hkv * P * rowb, P * rowb, rowb};
+  const long long* src = to_capsule ? cache : capsule;
+  const long long* dst = to_capsule ? capsule : cache;
+  char* cache_k = h->kv_k;
+  char* cache_v = h->kv_v;
+  char* cap_k = cap;
+  char* cap_v = cap + lay.v_off;
+  for (int b0 = 0; b0 < n; b0 += SLOT_MAP_MAX) {
+    RowCopy rc{};
+    rc.parts = 2;
+    rc.src[0] = to_capsule ? cache_k : cap_k;
+    rc.src[1] = to_capsule ? cache_v : cap_v;
+    rc.dst[0] = (to_capsule ? cap_k : cache_k) + b0 * dst[1];
+    rc.dst[1] = (to_capsule ? cap_v : cache_v) + b0 * dst[1];
+    rc.n_outer = c.L;
+    rc.n_sample = std::min(SLOT_MAP_MAX, n - b0);
+    rc.n_mid = c.Hkv;
+    rc.n_row = P;
+    rc.s_outer = src[0], rc.s_sample = src[1], rc.s_mid = src[2], rc.s_row = src[3];
+    rc.d_outer = dst[0], rc.d_sample = dst[1], rc.d_mid = dst[2], rc.d_row = dst[3];
+    rc.row_bytes = rowb;
+    for (int i = 0; i < rc.n_sample; ++i) rc.map[i] = map[b0 + i];
+    launch_state_copy(rc, s);
+    int r = check_launch("state copy kernel");
+    if (r) return r;
+  }
+  return FR_OK;
+}
+
+// x [B][H][A] float32 rows: dst sample b <- src sample map[b].
+int copy_x(const fr_config& c, const float* src, float* dst, const int* map, int n, cudaStream_t s) {
+  const long long xb = static_cast<long long>(c.H) * c.A * sizeof(float);
+  for (int b0 = 0; b0 < n; b0 += SLOT_MAP_MAX) {
+    RowCopy rc{};
+    rc.parts = 1;
+    rc.src[0] = reinterpret_cast<const char*>(src);
+    rc.dst[0] = reinterpret_cast<char*>(dst) + b0 * xb;
+    rc.n_outer = rc.n_mid = rc.n_row = 1;
+    rc.n_sample = std::min(SLOT_MAP_MAX, n - b0);
+    rc.s_sample = rc.d_sample = xb;
+    rc.row_bytes = xb;
+    for (int i = 0; i < rc.n_sample; ++i) rc.map[i] = map[b0 + i];
+    launch_state_copy(rc, s);
+    int r = check_launch("state copy kernel");
+    if (r) return r;
+  }
+  return FR_OK;
+}
+
+}  // namespace
+
+size_t fr_capsule_bytes(const fr_config* cfg, int B, int P, int with_x) {
+  if (!cfg || validate(*cfg) != FR_OK || B < 1 || B > cfg->B_max || P < 1 || P > cfg->P_max) return 0;
+  return capsule_layout(*cfg, B, P, with_x ? 1 : 0).total;
+}
+
+int fr_capsule_save(const fr_handle* h, void* cap_dev, size_t cap_bytes, int B, const float* x_dev,
+                    fr_capsule* desc, fr_stream_t stream) {
+  if (!h || !cap_dev || !desc) {
+    set_error("fr_capsule_save: NULL argument");
+    return FR_ERR_ARG;
+  }
+  if (h->prefix_B < 1) {
+    set_error("fr_capsule_save: no prefix set");
+    return FR_ERR_STATE;
+  }
+  if (B < 1 || B > h->prefix_B) {
+    set_error("fr_capsule_save: need 1 <= B <= %d cached samples (got %d)", h->prefix_B, B);
+    return FR_ERR_SHAPE;
+  }
+  const fr_config& c = h->cfg;
+  const int P = h->prefix_P;
+  const CapsuleLayout lay = capsule_layout(c, B, P, x_dev != nullptr);
+  if (cap_bytes < lay.total) {
+    set_error("fr_capsule_save: capsule buffer of %zu bytes, %zu needed", cap_bytes, lay.total);
+    return FR_ERR_SHAPE;
+  }
+  FR_CUDA(cudaSetDevice(h->device));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  std::vector<int> identity(B);
+  for (int b = 0; b < B; ++b) identity[b] = b;
+  char* cap = static_cast<char*>(cap_dev);
+  int rc = copy_prefix(h, cap, B, P, identity.data(), B, true, s);
+  if (rc) return rc;
+  if (x_dev) {
+    rc = copy_x(c, x_dev, reinterpret_cast<float*>(cap + lay.x_off), identity.data(), B, s);
+    if (rc) return rc;
+  }
+  fr_capsule d{};
+  d.magic = FR_CAPSULE_MAGIC;
+  d.L = c.L, d.Hkv = c.Hkv, d.dh = c.dh, d.kv_bytes_per_elem = h->kv_bf ? 2 : 4;
+  d.H = c.H, d.A = c.A;
+  d.B = B, d.P = P;
+  d.has_x = x_dev != nullptr;
+  d.bytes = lay.total;
+  *desc = d;
+  return FR_OK;
+}
+
+int fr_capsule_restore(fr_handle* h, const void* cap_dev, const fr_capsule* desc, const int* map, int B,
+                       float* x_dev, fr_stream_t stream) {
+  if (!h || !cap_dev || !desc) {
+    set_error("fr_capsule_restore: NULL argument");
+    return FR_ERR_ARG;
+  }
+  const fr_config& c = h->cfg;
+  if (desc->magic != FR_CAPSULE_MAGIC || desc->B < 1 || desc->P < 1) {
+    set_error("fr_capsule_restore: not a capsule description (magic 0x%x, B=%d, P=%d)", desc->magic, desc->B,
+              desc->P);
+    return FR_ERR_ARG;
+  }
+  if (desc->L != c.L || desc->Hkv != c.Hkv || desc->dh != c.dh || desc->kv_bytes_per_elem != (h->kv_bf ? 2 : 4) ||
+      desc->H != c.H || desc->A != c.A) {
+    set_error("fr_capsule_restore: capsule written by a handle of another shape");
+    return FR_ERR_SHAPE;
+  }
+  if (B < 1 || B > c.B_max || desc->P > c.P_max) {
+    set_error("fr_capsule_restore: need 1 <= B <= %d and P <= %d (got B=%d, capsule P=%d)", c.B_max, c.P_max, B,
+              desc->P);
+    return FR_ERR_SHAPE;
+  }
+  std::vector<int> m(B);
+  for (int b = 0; b < B; ++b) {
+    m[b] = map ? map[b] : b;
+    if (m[b] < 0 || m[b] >= desc->B) {
+      if (!map) {
+        set_error("fr_capsule_restore: B=%d without a map, the capsule holds %d samples", B, desc->B);
+        return FR_ERR_SHAPE;
+      }
+      set_error("fr_capsule_restore: map[%d]=%d outside the capsule's %d samples", b, m[b], desc->B);
+      return FR_ERR_ARG;
+    }
+  }
+  if (x_dev && !desc->has_x) {
+    set_error("fr_capsule_restore: x requested but the capsule holds none");
+    return FR_ERR_STATE;
+  }
+  FR_CUDA(cudaSetDevice(h->device));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* cap = const_cast<char*>(static_cast<const char*>(cap_dev));   // read only
+  int rc = copy_prefix(h, cap, desc->B, desc->P, m.data(), B, false, s);
+  if (rc) return rc;
+  if (x_dev) {
+    const CapsuleLayout lay = capsule_layout(c, desc->B, desc->P, 1);
+    rc = copy_x(c, reinterpret_cast<const float*>(cap + lay.x_off), x_dev, m.data(), B, s);
+    if (rc) return rc;
+  }
+  h->prefix_B = B;
+  h->prefix_P = desc->P;
+  return FR_OK;
+}
+
+int fr_set_graph_capacity(fr_handle* h, int capacity) {
+  if (!h || capacity < 1) {
+    set_error("fr_set_graph_capacity: NULL handle or capacity < 1");
+    return FR_ERR_ARG;
+  }
+  if (h->tp) return tensor_path_set_graph_capacity(h->tp, capacity);
+  return FR_OK;
+}
+
+int fr_graph_count(const fr_handle* h) {
+  if (!h) {
+    set_error("fr_graph_count: NULL handle");
+    return FR_ERR_ARG;
+  }
+  return h->tp ? tensor_path_graph_count(h->tp) : 0;
 }
 
 int fr_denoise(fr_handle* h, const float* x0_dev, float* x_out_dev, int B, fr_stream_t stream) {

@@ -256,18 +256,21 @@ __global__ void k_rope_qkv(const float* __restrict__ qkv, float* __restrict__ q,
 }
 
 // ------------------------------------------------------------------ prefix ingest
-// in [L][B][P][Hkv][dh] -> cache [L][B_max][Hkv][S_max][dh], K rotated at position p.
+// in [L][B_src][P][Hkv][dh] (samples b0 .. b0+nb-1) -> cache [L][B_max][Hkv][S_max][dh] at the
+// slots of `map`, K rotated at position p.
 __global__ void k_prefix_ingest(const void* k_in, const void* v_in, void* kv_k, void* kv_v,
                                 int kv_bf, const float* __restrict__ cos_t,
-                                const float* __restrict__ sin_t, int B, int B_max, int P,
+                                const float* __restrict__ sin_t, int B_src, int b0, int nb,
+                                const __grid_constant__ SlotMap map, int B_max, int P,
                                 int S_max, int Hkv, int dh, int rotate) {
-  const int row = blockIdx.x;      // over L*B*P*Hkv
-  const int g = row % Hkv;
-  const int p = (row / Hkv) % P;
-  const int b = (row / (Hkv * P)) % B;
-  const int l = row / (Hkv * P * B);
-  const size_t src = static_cast<size_t>(row) * dh;
-  const size_t dst = ((((static_cast<size_t>(l) * B_max + b) * Hkv + g) * S_max) + p) * dh;
+  const long row = blockIdx.x;     // over L*nb*P*Hkv
+  const int g = static_cast<int>(row % Hkv);
+  const int p = static_cast<int>((row / Hkv) % P);
+  const int bl = static_cast<int>((row / (static_cast<long>(Hkv) * P)) % nb);
+  const int l = static_cast<int>(row / (static_cast<long>(Hkv) * P * nb));
+  const int slot = map.n ? map.slot[bl] : b0 + bl;
+  const size_t src = ((((static_cast<size_t>(l) * B_src + b0 + bl) * P + p) * Hkv) + g) * dh;
+  const size_t dst = ((((static_cast<size_t>(l) * B_max + slot) * Hkv + g) * S_max) + p) * dh;
   const int half = dh / 2;
   for (int d = threadIdx.x; d < half; d += blockDim.x) {
     const float lo = kv_get(k_in, src + d, kv_bf), hi = kv_get(k_in, src + d + half, kv_bf);
@@ -414,11 +417,13 @@ void launch_rope_qkv(const float* qkv, float* q, void* kv_k, void* kv_v, int kv_
 }
 
 void launch_prefix_ingest(const void* k_in, const void* v_in, void* kv_k, void* kv_v, int kv_bf,
-                          const float* cos_t, const float* sin_t, int L, int B, int B_max, int P,
-                          int S_max, int Hkv, int dh, int rotate, cudaStream_t s) {
-  const long rows = static_cast<long>(L) * B * P * Hkv;
+                          const float* cos_t, const float* sin_t, int L, int B_src, int b0, int nb,
+                          const SlotMap& map, int B_max, int P, int S_max, int Hkv, int dh, int rotate,
+                          cudaStream_t s) {
+  const long rows = static_cast<long>(L) * nb * P * Hkv;
   k_prefix_ingest<<<static_cast<unsigned>(rows), 64, 0, s>>>(k_in, v_in, kv_k, kv_v, kv_bf, cos_t, sin_t,
-                                                             B, B_max, P, S_max, Hkv, dh, rotate);
+                                                             B_src, b0, nb, map, B_max, P, S_max, Hkv, dh,
+                                                             rotate);
 }
 
 void launch_attention(const float* q, const void* kv_k, const void* kv_v, int kv_bf, float* act,

@@ -78,6 +78,7 @@ struct GraphEntry {
   const float* x0 = nullptr;
   float* x_out = nullptr;
   StepPlan plan;
+  unsigned long long last_use = 0;  // graph-variant table: least recently used goes first
 };
 
 }  // namespace
@@ -110,7 +111,9 @@ struct TensorPath {
   __nv_bfloat16* w_in_bf = nullptr;   // [A][D]
   __nv_bfloat16* w_out_bf = nullptr;  // [A][D]
   cudaStream_t cap = nullptr;
-  std::map<std::pair<int, int>, GraphEntry> graphs;
+  std::map<std::pair<int, int>, GraphEntry> graphs;   // graph-variant table keyed by (B, P)
+  size_t graph_capacity = 8;
+  unsigned long long use_clock = 0;
   std::vector<float> gains_host;
 };
 
@@ -681,10 +684,42 @@ int tensor_path_set_scales(TensorPath*, const float*, const float*) {
   return FR_OK;   // kernels read the handle's device scale arrays directly
 }
 
+namespace {
+
+void destroy_entry(GraphEntry& ge) {
+  // an exec still running on a stream is freed by CUDA once it completes
+  if (ge.exec) cudaGraphExecDestroy(ge.exec);
+  if (ge.graph) cudaGraphDestroy(ge.graph);
+  ge.exec = nullptr;
+  ge.graph = nullptr;
+}
+
+// Drop least recently used variants until at most `keep` remain.
+void evict_to(TensorPath* tp, size_t keep) {
+  while (tp->graphs.size() > keep) {
+    auto victim = tp->graphs.begin();
+    for (auto it = tp->graphs.begin(); it != tp->graphs.end(); ++it)
+      if (it->second.last_use < victim->second.last_use) victim = it;
+    destroy_entry(victim->second);
+    tp->graphs.erase(victim);
+  }
+}
+
+}  // namespace
+
+int tensor_path_set_graph_capacity(TensorPath* tp, int capacity) {
+  tp->graph_capacity = static_cast<size_t>(capacity);
+  evict_to(tp, tp->graph_capacity);
+  return FR_OK;
+}
+
+int tensor_path_graph_count(const TensorPath* tp) { return static_cast<int>(tp->graphs.size()); }
+
 int tensor_path_denoise(TensorPath* tp, const float* x0, float* x_out, int B, int P, cudaStream_t s) {
   auto key = std::make_pair(B, P);
   auto it = tp->graphs.find(key);
   if (it == tp->graphs.end()) {
+    evict_to(tp, tp->graph_capacity - 1);
     GraphEntry ge;
     int rc = build_graph(tp, B, P, x0, x_out, ge);
     if (rc) {
@@ -694,6 +729,7 @@ int tensor_path_denoise(TensorPath* tp, const float* x0, float* x_out, int B, in
     }
     it = tp->graphs.emplace(key, ge).first;
   }
+  it->second.last_use = ++tp->use_clock;
   int rc = retarget(it->second, x0, x_out);
   if (rc) return rc;
   FR_CUDA(cudaGraphLaunch(it->second.exec, s));
@@ -704,10 +740,7 @@ int tensor_path_launches(const TensorPath* tp, int) { return tp->c.K * (2 + 5 * 
 
 void tensor_path_destroy(TensorPath* tp) {
   if (!tp) return;
-  for (auto& kv : tp->graphs) {
-    if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
-    if (kv.second.graph) cudaGraphDestroy(kv.second.graph);
-  }
+  for (auto& kv : tp->graphs) destroy_entry(kv.second);
   if (tp->cap) cudaStreamDestroy(tp->cap);
   delete tp;
 }

@@ -217,6 +217,102 @@ const char* fr_path_name(const fr_handle* h);
 /* Number of kernel launches one fr_denoise call issues for batch B. */
 int fr_launches_per_call(const fr_handle* h, int B);
 
+/* ---- execution contract across chunks: selective refresh, named buffers, capsules ---- */
+
+/*
+ * fr_refresh_prefix_kv -- selective refresh of the prefix state (FlashRT-PAI overview,
+ * mechanism 2 "execution contract": state reused across decision cycles and refreshed
+ * only where it changed): replace the prefix KV of n batch slots and leave every other
+ * slot as it is, e.g. when one camera's observation of a batch of robots changed.
+ * k_dev, v_dev: device [L][n][P][Hkv][dh] in the type of fr_set_prefix_kv; source sample
+ * i goes to slot slots[i] (host array of n distinct slots, each below the B of the last
+ * fr_set_prefix_kv or fr_capsule_restore).  P must equal that call's P: the cache holds
+ * one prefix length.  K is rotated at 0..P-1 unless FR_PREFIX_K_ROTATED.  Asynchronous.
+ * Errors: FR_ERR_ARG (NULL, n < 1, a slot given twice, unknown flags), FR_ERR_STATE (no
+ * prefix yet), FR_ERR_SHAPE (P differs, slot out of range), FR_ERR_CUDA.
+ */
+int fr_refresh_prefix_kv(fr_handle* h, const void* k_dev, const void* v_dev, const int* slots, int n, int P,
+                         unsigned flags, fr_stream_t stream);
+
+/*
+ * fr_get_buffer -- a named device buffer of the handle (FlashRT walkthrough, "exec/: C
+ * ABI execution contract": named device buffers are the only state and are shared by
+ * pointer between graphs, without copies).  Names and contents:
+ *   "kv_k", "kv_v"          KV cache [L][B_max][Hkv][P_max+H][dh], each layer starting on
+ *                           a 256-byte boundary; float32 for f32 handles, bf16 otherwise
+ *   "rope_cos", "rope_sin"  RoPE tables [P_max+H][dh/2] float32
+ *   "temb"                  time embeddings of the K steps [K][D] float32
+ *   "s_act"                 fp8 activation scales [L][4] float32 (see fr_get_scales)
+ *   "status"                the device status word (uint32)
+ * *dev receives the device address and *bytes the size; the handle owns both until
+ * fr_destroy.  Writing into them is the caller's responsibility.  No device work.
+ * Errors: FR_ERR_ARG (NULL argument, unknown name).
+ */
+int fr_get_buffer(const fr_handle* h, const char* name, void** dev, size_t* bytes);
+
+/*
+ * Execution-state capsules (FlashRT-PAI overview, mechanism 3: snapshot, restore and
+ * fork of the resident pipeline state; FlashRT walkthrough, "serving/": snapshot,
+ * restore, fork and time travel).  Between chunks the state of a handle is the prefix
+ * KV of its batch slots; a capsule holds it for B samples, plus the caller's action
+ * chunk x [B][H][A] float32 when saved with one.  The capsule's bytes live in a device
+ * buffer the caller owns; the fr_capsule description stays on the host.
+ * Device layout: K [L][B][Hkv][P][dh], then V in the same layout, then x; each part
+ * starts on a 256-byte boundary; K/V in the KV cache's type (K already rotated).
+ */
+#define FR_CAPSULE_MAGIC 0x46524350u
+typedef struct fr_capsule {
+  uint32_t magic;          /* FR_CAPSULE_MAGIC once written by fr_capsule_save */
+  int L, Hkv, dh;          /* shape of the handle that wrote it */
+  int kv_bytes_per_elem;   /* 2 (bf16) or 4 (float32) */
+  int H, A;
+  int B, P;                /* samples and prefix length held */
+  int has_x;               /* 1: x [B][H][A] follows the KV */
+  size_t bytes;            /* device bytes in use */
+} fr_capsule;
+
+/* Device bytes of a capsule of B samples and prefix length P (with x when with_x != 0)
+ * for handles created from *cfg; 0 if cfg is invalid, B outside [1, B_max] or P outside
+ * [1, P_max].  Host arithmetic only. */
+size_t fr_capsule_bytes(const fr_config* cfg, int B, int P, int with_x);
+
+/*
+ * fr_capsule_save -- snapshot the prefix KV of slots 0..B-1 (B at most the cached batch)
+ * and, when x_dev is not NULL, the chunk x_dev [B][H][A] into cap_dev, a device buffer of
+ * cap_bytes >= fr_capsule_bytes(cfg, B, P, x_dev != NULL) bytes.  *desc receives the
+ * description.  Asynchronous: the snapshot is the state at this point of `stream`.
+ * Errors: FR_ERR_ARG (NULL), FR_ERR_STATE (no prefix yet), FR_ERR_SHAPE (B, cap_bytes),
+ * FR_ERR_CUDA.
+ */
+int fr_capsule_save(const fr_handle* h, void* cap_dev, size_t cap_bytes, int B, const float* x_dev,
+                    fr_capsule* desc, fr_stream_t stream);
+
+/*
+ * fr_capsule_restore -- make a capsule the handle's prefix state: slot b (b < B) receives
+ * capsule sample map[b] (map NULL: sample b, then B <= desc->B).  A map that repeats a
+ * sample forks it into several slots (several noise draws against one observation).  A
+ * capsule saved earlier brings back an earlier state.  Afterwards the cached prefix covers
+ * slots 0..B-1 with length desc->P, as after fr_set_prefix_kv.  When x_dev is not NULL,
+ * x_dev [B][H][A] receives the capsule's x of the same samples.  Asynchronous.
+ * Errors: FR_ERR_ARG (NULL, not a capsule description, map entry out of range),
+ * FR_ERR_SHAPE (capsule of a handle of another shape, B outside [1, B_max], desc->P >
+ * P_max, B > desc->B without a map), FR_ERR_STATE (x_dev given, capsule without x),
+ * FR_ERR_CUDA.
+ */
+int fr_capsule_restore(fr_handle* h, const void* cap_dev, const fr_capsule* desc, const int* map, int B,
+                       float* x_dev, fr_stream_t stream);
+
+/*
+ * fr_set_graph_capacity / fr_graph_count -- the tensor path keeps one instantiated CUDA
+ * graph per (B, P) it has run (FlashRT walkthrough, "exec/": shape key -> graph variant,
+ * exact key, least recently used evicted).  At most `capacity` (>= 1; 8 at fr_create)
+ * stay; the least recently used goes first, a graph still running being freed once it
+ * completes.  fr_graph_count returns how many are cached (0 on the stepwise path).
+ * Errors: FR_ERR_ARG (NULL, capacity < 1).
+ */
+int fr_set_graph_capacity(fr_handle* h, int capacity);
+int fr_graph_count(const fr_handle* h);
+
 /* ---- kernel library: one op on caller buffers (no handle) ---- */
 
 /*

@@ -117,3 +117,32 @@ def test_packer_w4_matches_oracle_quantiser(abi):
     sv = (sb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     assert np.array_equal(sv, os_)
     assert abi.load_library().fr_quantize_w4(None, 1, 1, None, None) == abi.FR_ERR_ARG
+
+
+def test_capsule_sizes_and_contract_calls_reject_before_device_work(abi):
+    import synthetic
+    cfg = synthetic.CONFIGS["pi05_bf16_b1"]
+    fc = abi.make_config(cfg, B_max=4, P_max=cfg.P)
+    # K then V [L][B][Hkv][P][dh] bf16, then x [B][H][A] float32, each part on a 256-byte boundary
+    kv = cfg.L * 2 * cfg.Hkv * cfg.P * cfg.dh * 2
+    up = lambda n: -(-n // 256) * 256   # noqa: E731
+    assert abi.fr_capsule_bytes(fc, 2, cfg.P, False) == 2 * up(kv)
+    assert abi.fr_capsule_bytes(fc, 2, cfg.P, True) == 2 * up(kv) + up(2 * cfg.H * cfg.A * 4)
+    f32 = abi.make_config(synthetic.CONFIGS["tiny_f32"], B_max=3)
+    t = synthetic.CONFIGS["tiny_f32"]
+    assert abi.fr_capsule_bytes(f32, 3, t.P, False) == 2 * up(t.L * 3 * t.Hkv * t.P * t.dh * 4)
+    for B, P in ((0, cfg.P), (5, cfg.P), (1, 0), (1, cfg.P + 1)):
+        assert abi.fr_capsule_bytes(fc, B, P, True) == 0
+    assert abi.fr_capsule_bytes(abi.make_config(cfg.replace(L=0)), 1, 1, False) == 0
+    lib = abi.load_library()
+    assert lib.fr_capsule_bytes(None, 1, 1, 0) == 0
+    p = ctypes.c_void_p(1)
+    sl = (ctypes.c_int * 1)(0)
+    assert lib.fr_refresh_prefix_kv(None, p, p, sl, 1, 1, 0, None) == abi.FR_ERR_ARG
+    out, n = ctypes.c_void_p(), ctypes.c_size_t()
+    assert lib.fr_get_buffer(None, b"kv_k", ctypes.byref(out), ctypes.byref(n)) == abi.FR_ERR_ARG
+    d = abi.FrCapsule()
+    assert lib.fr_capsule_save(None, p, 1, 1, None, ctypes.byref(d), None) == abi.FR_ERR_ARG
+    assert lib.fr_capsule_restore(None, p, ctypes.byref(d), None, 1, None, None) == abi.FR_ERR_ARG
+    assert lib.fr_set_graph_capacity(None, 1) == abi.FR_ERR_ARG
+    assert lib.fr_graph_count(None) == abi.FR_ERR_ARG
