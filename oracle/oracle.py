@@ -55,6 +55,19 @@ Readings where the pages are silent (each listed in the design notes):
       scale per group, s = bf16(max|w| / 7), q = clamp(round-half-even(w / s));
       the tensor-core operand is the dequantised weight bf16(q * s).
       Projection inputs are bf16 as in R10; everything else is as bf16.
+  R17 adaRMS workloads (pi0.5-style time conditioning; the pages describe the
+      pi0.5 action expert but not its conditioning, so the variant follows the
+      "Pi0.5-style" workload description): the time embedding is not added to
+      the tokens (R4 does not apply); it is the condition c = temb(t), rounded
+      like any projection input, of every RMSNorm.  Each of the two norms of a
+      layer has (s, b, g) = W_mod c + b_mod (three D-vectors: scale, shift,
+      gate); the final norm has (s, b).  The normalised tensor is
+      RMS(h) * (1 + s) + b, and each residual update is scaled by the gate:
+      h <- h + g * update.  Where the normalised tensor feeds a projection W,
+      the projection input (rounded or quantised as in R10/R11/R16) is
+      RMS(h) * (1 + s) and W b is added to the projection's output in full
+      precision: W (a + b) = W a + W b, with the rounding point placed before
+      the shift, as R10 places it before the rstd factor.
 """
 from __future__ import annotations
 
@@ -304,6 +317,14 @@ class PreparedModel:
                 for p in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
                     d[p] = rnd(lw[p])
             self.layers.append(d)
+        self.adarms = bool(getattr(cfg, "adarms", False))
+        if self.adarms:   # R17: modulation projections of the condition, stored like the time MLP
+            for d, lw in zip(self.layers, weights["layers"]):
+                for n in ("1", "2"):
+                    d["w_mod" + n] = rnd(lw["w_mod" + n])
+                    d["b_mod" + n] = np.asarray(lw["b_mod" + n], np.float64)
+            self.w_modf = rnd(weights["w_modf"])
+            self.b_modf = np.asarray(weights["b_modf"], np.float64)
         self.cos, self.sin = rope_tables(cfg.P + cfg.H, cfg.dh, cfg.rope_theta)
 
     def temb(self, t: float) -> np.ndarray:
@@ -347,6 +368,19 @@ def _project(model: PreparedModel, l: int, which: str, a, ws, scales, record):
     return [ar @ w.T for w in ws]
 
 
+def _dequantised(model: PreparedModel, l: int, which: str, w):
+    """The weight values a projection multiplies by (s_w * codes for fp8)."""
+    return w * model.layers[l]["sw_" + which] if model.dtype == "fp8" else w
+
+
+def _modulation(model: PreparedModel, c, l: int, n: str):
+    """R17: (scale, shift, gate) of norm n ("1" pre-attention, "2" pre-MLP) of layer l."""
+    lay = model.layers[l]
+    m = lay["w_mod" + n] @ c + lay["b_mod" + n]
+    D = model.cfg.D
+    return m[:D], m[D:2 * D], m[2 * D:]
+
+
 def velocity(model: PreparedModel, x, k_step: int, t: float, kv_k, kv_v,
              scales: Optional[Dict] = None, record: Optional[Dict] = None) -> np.ndarray:
     """v(x, t) for one chunk x [H][A] (the action expert; configs' architecture).
@@ -356,13 +390,28 @@ def velocity(model: PreparedModel, x, k_step: int, t: float, kv_k, kv_v,
     cfg = model.cfg
     rnd = model.rnd
     P, H, dh, Hq, Hkv = cfg.P, cfg.H, cfg.dh, cfg.Hq, cfg.Hkv
-    # in-proj + time (R3, R4)
-    h = rnd(x) @ model.w_in.T + model.b_in + model.temb(t)
+    ones = np.ones(cfg.D)
+    if model.adarms:
+        # R17: in-proj only; the time embedding conditions the norms
+        h = rnd(x) @ model.w_in.T + model.b_in
+        cond = rnd(model.temb(t))
+    else:
+        # in-proj + time (R3, R4)
+        h = rnd(x) @ model.w_in.T + model.b_in + model.temb(t)
     cos_a, sin_a = model.cos[P:P + H], model.sin[P:P + H]
     for l, lay in enumerate(model.layers):
+        if model.adarms:
+            s1, b1, g1 = _modulation(model, cond, l, "1")
+            s2, b2, g2 = _modulation(model, cond, l, "2")
+            gain1, gain2 = 1.0 + s1, 1.0 + s2
+        else:
+            gain1, gain2, g1, g2 = lay["g1"], lay["g2"], ones, ones
         # pre-attention RMSNorm, fused QKV projection (PhyAI page: Q/K/V in one GEMM)
-        a = rms_norm(h, lay["g1"], cfg.eps)
+        a = rms_norm(h, gain1, cfg.eps)
         q, k, v = _project(model, l, "qkv", a, (lay["wq"], lay["wk"], lay["wv"]), scales, record)
+        if model.adarms:   # R17: the shift enters as W b
+            q, k, v = (y + _dequantised(model, l, "qkv", w) @ b1
+                       for y, w in ((q, lay["wq"]), (k, lay["wk"]), (v, lay["wv"])))
         q = q.reshape(H, Hq, dh).transpose(1, 0, 2)           # [Hq][H][dh]
         k = k.reshape(H, Hkv, dh).transpose(1, 0, 2)          # [Hkv][H][dh]
         v = v.reshape(H, Hkv, dh).transpose(1, 0, 2)
@@ -375,14 +424,21 @@ def velocity(model: PreparedModel, x, k_step: int, t: float, kv_k, kv_v,
         o = attention(q, keys, vals)                           # [Hq][H][dh]
         o = o.transpose(1, 0, 2).reshape(H, Hq * dh)
         (dh_o,) = _project(model, l, "o", o, (lay["wo"],), scales, record)
-        h = h + dh_o
+        h = h + g1 * dh_o
         # pre-MLP RMSNorm, merged gate|up projection, GeLU(gate) * up, down (R9)
-        a = rms_norm(h, lay["g2"], cfg.eps)
+        a = rms_norm(h, gain2, cfg.eps)
         g, u = _project(model, l, "gu", a, (lay["wg"], lay["wu"]), scales, record)
+        if model.adarms:
+            g = g + _dequantised(model, l, "gu", lay["wg"]) @ b2
+            u = u + _dequantised(model, l, "gu", lay["wu"]) @ b2
         m = gelu_tanh(g) * u
         (dh_d,) = _project(model, l, "down", m, (lay["wd"],), scales, record)
-        h = h + dh_d
-    # final RMSNorm + out-proj (R5)
+        h = h + g2 * dh_d
+    # final RMSNorm + out-proj (R5; R17 modulates it)
+    if model.adarms:
+        mf = model.w_modf @ cond + model.b_modf
+        s_f, b_f = mf[:cfg.D], mf[cfg.D:]
+        return rnd(rms_norm(h, 1.0 + s_f, cfg.eps)) @ model.w_out.T + model.w_out @ b_f + model.b_out
     return rnd(rms_norm(h, model.g_f, cfg.eps)) @ model.w_out.T + model.b_out
 
 

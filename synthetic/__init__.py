@@ -19,6 +19,8 @@ scaled, then stored as float32):
   2. W_in, W_out, W_t1, W_t2, each / sqrt(fan_in)
   3. prefix K then prefix V, shape [L][B][P][Hkv][dh], N(0, 1)
   4. noise x0, shape [B][H][A], N(0, 1)
+  5. adaRMS workloads only: for each layer W_mod1 then W_mod2 [3D][D], then W_modf [2D][D],
+     each / sqrt(D) (drawn last, so the other tensors equal those of the plain workload)
 RMSNorm gains are ones and biases are zeros (explicit arrays, not drawn).
 """
 from __future__ import annotations
@@ -28,7 +30,7 @@ from typing import Dict, List
 
 import numpy as np
 
-__all__ = ["ActionExpertConfig", "CONFIGS", "make_inputs", "make_noise", "make_prefix"]
+__all__ = ["ActionExpertConfig", "CONFIGS", "make_inputs", "make_modulation", "make_noise", "make_prefix"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -57,6 +59,7 @@ class ActionExpertConfig:
     eps: float = 1e-6
     time_dim: int = 256
     time_base: float = 10000.0
+    adarms: bool = False   # time conditioning by adaptive RMSNorm instead of an added embedding
 
     @property
     def T(self) -> int:
@@ -86,6 +89,10 @@ CONFIGS: Dict[str, ActionExpertConfig] = {
     # same with 4-bit weights (group scales) and bf16 projection inputs
     "pi05_w4a16_b1": ActionExpertConfig("pi05_w4a16_b1", L=18, D=1024, Hq=8, Hkv=1, dh=256,
                                         F=4096, H=50, A=32, B=1, P=816, K=10, dtype="w4a16"),
+    # π0.5-style adaptive-RMSNorm time conditioning, batch 1, bf16
+    "pi05_adarms_bf16_b1": ActionExpertConfig("pi05_adarms_bf16_b1", L=18, D=1024, Hq=8, Hkv=1, dh=256,
+                                              F=4096, H=50, A=32, B=1, P=816, K=10, dtype="bf16",
+                                              adarms=True),
     # larger stress variant
     "stress_bf16_b4": ActionExpertConfig("stress_bf16_b4", L=18, D=2048, Hq=16, Hkv=2, dh=128,
                                          F=8192, H=100, A=32, B=4, P=2048, K=10, dtype="bf16"),
@@ -141,12 +148,28 @@ def make_noise(cfg: ActionExpertConfig, rng: np.random.Generator) -> np.ndarray:
     return rng.standard_normal(size=(cfg.B, cfg.H, cfg.A), dtype=np.float64).astype(np.float32)
 
 
+def make_modulation(cfg: ActionExpertConfig, rng: np.random.Generator, w: dict) -> None:
+    """adaRMS modulation weights (draw step 5) into w: per layer w_mod1/b_mod1 (pre-attention norm)
+    and w_mod2/b_mod2 (pre-MLP norm) [3D][D], [3D] as (scale | shift | gate) rows; w_modf/b_modf
+    [2D][D], [2D] as (scale | shift) rows for the final norm.  Biases are zeros."""
+    D = cfg.D
+    for lw in w["layers"]:
+        lw["w_mod1"] = _scaled_normal(rng, (3 * D, D), D)
+        lw["w_mod2"] = _scaled_normal(rng, (3 * D, D), D)
+        lw["b_mod1"] = np.zeros(3 * D, np.float32)
+        lw["b_mod2"] = np.zeros(3 * D, np.float32)
+    w["w_modf"] = _scaled_normal(rng, (2 * D, D), D)
+    w["b_modf"] = np.zeros(2 * D, np.float32)
+
+
 def make_inputs(cfg: ActionExpertConfig, seed: int = 0) -> dict:
     """All inputs of one workload from one seed, in the documented draw order."""
     rng = np.random.default_rng(seed)
     w = make_weights(cfg, rng)
     pk, pv = make_prefix(cfg, rng)
     x0 = make_noise(cfg, rng)
+    if cfg.adarms:
+        make_modulation(cfg, rng, w)
     return {"weights": w, "prefix_k": pk, "prefix_v": pv, "x0": x0}
 
 
