@@ -49,6 +49,8 @@ def workload_bytes(cfg) -> dict:
         layer_bytes = layer_w * {"f32": 4, "bf16": 2, "fp8": 1}[cfg.dtype]
     small = 2 * (cfg.D * cfg.A * 2 + 3 * cfg.D * 4) + cfg.A * 4   # in/out-proj (bf16) + gains/biases
     w_step = cfg.L * (layer_bytes + 2 * D * 4) + small
+    if getattr(cfg, "adarms", False):   # per-step gates and folded shifts (W b) read by the epilogues
+        w_step += cfg.L * (2 * D * 4 + ((dq + 2 * nkv) + 2 * F) * 4)
     kv_step = cfg.L * cfg.B * cfg.Hkv * (cfg.P + cfg.H) * cfg.dh * 2 * (4 if cfg.dtype == "f32" else 2)
     return {"weights_per_step": w_step, "kv_per_step": kv_step, "per_chunk": cfg.K * (w_step + kv_step),
             "weights_per_chunk": cfg.K * w_step}

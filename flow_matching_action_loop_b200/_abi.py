@@ -40,19 +40,23 @@ class FrConfig(ctypes.Structure):
                 ("dh", ctypes.c_int), ("F", ctypes.c_int), ("H", ctypes.c_int), ("A", ctypes.c_int),
                 ("B_max", ctypes.c_int), ("P_max", ctypes.c_int), ("K", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("path", ctypes.c_int), ("rope_theta", ctypes.c_float),
-                ("eps", ctypes.c_float), ("time_dim", ctypes.c_int), ("time_base", ctypes.c_float)]
+                ("eps", ctypes.c_float), ("time_dim", ctypes.c_int), ("time_base", ctypes.c_float),
+                ("adarms", ctypes.c_int)]
 
 
 _FP = ctypes.POINTER(ctypes.c_float)
 
 
+LAYER_TENSORS = ("wq", "wk", "wv", "wo", "wg", "wu", "wd", "g1", "g2", "w_mod1", "b_mod1", "w_mod2", "b_mod2")
+MODEL_TENSORS = ("w_in", "b_in", "w_out", "b_out", "w_t1", "b_t1", "w_t2", "b_t2", "g_f", "w_modf", "b_modf")
+
+
 class FrLayerWeights(ctypes.Structure):
-    _fields_ = [(n, _FP) for n in ("wq", "wk", "wv", "wo", "wg", "wu", "wd", "g1", "g2")]
+    _fields_ = [(n, _FP) for n in LAYER_TENSORS]
 
 
 class FrWeights(ctypes.Structure):
-    _fields_ = [("layers", ctypes.POINTER(FrLayerWeights))] + \
-               [(n, _FP) for n in ("w_in", "b_in", "w_out", "b_out", "w_t1", "b_t1", "w_t2", "b_t2", "g_f")]
+    _fields_ = [("layers", ctypes.POINTER(FrLayerWeights))] + [(n, _FP) for n in MODEL_TENSORS]
 
 
 FR_CAPSULE_MAGIC = 0x46524350
@@ -146,7 +150,8 @@ def make_config(cfg, B_max: Optional[int] = None, P_max: Optional[int] = None, p
     dtype = cfg.dtype if isinstance(cfg.dtype, int) else DTYPES[cfg.dtype]
     return FrConfig(L=cfg.L, D=cfg.D, Hq=cfg.Hq, Hkv=cfg.Hkv, dh=cfg.dh, F=cfg.F, H=cfg.H, A=cfg.A,
                     B_max=B_max or cfg.B, P_max=P_max or cfg.P, K=cfg.K, dtype=dtype, path=path,
-                    rope_theta=cfg.rope_theta, eps=cfg.eps, time_dim=cfg.time_dim, time_base=cfg.time_base)
+                    rope_theta=cfg.rope_theta, eps=cfg.eps, time_dim=cfg.time_dim, time_base=cfg.time_base,
+                    adarms=1 if getattr(cfg, "adarms", False) else 0)
 
 
 # ------------------------------------------------------------------ same-name wrappers
@@ -158,20 +163,22 @@ def fr_create(cfg: FrConfig, device: int = 0) -> ctypes.c_void_p:
 
 
 def fr_load_weights(h, weights: dict, stream: int = 0) -> None:
-    """weights: the dict layout of host float32 arrays ({'layers': [...], 'w_in': ..., ...})."""
+    """weights: the dict layout of host float32 arrays ({'layers': [...], 'w_in': ..., ...}); a tensor
+    the dict does not hold (the adaRMS ones of a plain model) is passed as NULL."""
     keep = []
 
     def p(a):
+        if a is None:
+            return _FP()
         a = _f32(a)
         keep.append(a)
         return _fptr(a)
 
     layers = (FrLayerWeights * len(weights["layers"]))()
     for i, lw in enumerate(weights["layers"]):
-        for n in ("wq", "wk", "wv", "wo", "wg", "wu", "wd", "g1", "g2"):
-            setattr(layers[i], n, p(lw[n]))
-    w = FrWeights(layers=layers, **{n: p(weights[n]) for n in
-                                    ("w_in", "b_in", "w_out", "b_out", "w_t1", "b_t1", "w_t2", "b_t2", "g_f")})
+        for n in LAYER_TENSORS:
+            setattr(layers[i], n, p(lw.get(n)))
+    w = FrWeights(layers=layers, **{n: p(weights.get(n)) for n in MODEL_TENSORS})
     _check(load_library().fr_load_weights(h, ctypes.byref(w), stream), "fr_load_weights")
 
 

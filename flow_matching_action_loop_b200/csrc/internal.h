@@ -56,8 +56,12 @@ void launch_inproj(const float* x, const float* w_in, const float* b_in, const f
                    float* h, int T, int D, int A, int round_bf16, cudaStream_t s);
 void launch_rmsnorm_q(const float* h, const float* gamma, float* out, int T, int D, float eps,
                       int qmode, const float* s_a, unsigned* amax, cudaStream_t s);
+// C[t][n] (+)= gate[n] * alpha * (A W^T)[t][n] + bias[n]  (gate, bias: NULL = 1, 0)
 void launch_gemm(const float* A, int lda, const void* W, int wtype, const float* alpha,
-                 float* C, int ldc, int T, int N, int Kd, int accumulate, cudaStream_t s);
+                 float* C, int ldc, int T, int N, int Kd, int accumulate, cudaStream_t s,
+                 const float* bias = nullptr, const float* gate = nullptr);
+void launch_round_rows(const float* in, int in_ld, float* out, int rows, int n, int round_bf16, cudaStream_t s);
+void launch_one_plus(const float* in, int in_ld, float* out, int rows, int n, cudaStream_t s);
 void launch_rope_qkv(const float* qkv, float* q, void* kv_k, void* kv_v, int kv_bf16,
                      const float* cos_t, const float* sin_t, int B, int H, int P, int S_max,
                      int Hq, int Hkv, int dh, int round_bf16, cudaStream_t s);

@@ -69,6 +69,17 @@ struct fr_handle {
   std::vector<float> h_sw, h_sa;
 
   TensorPath* tp = nullptr;                 // tensor-core kernel set (bf16/fp8)
+
+  // adaptive RMSNorm (cfg.adarms): every step's norm modulation, precomputed by fr_load_weights
+  float* ada_stage = nullptr;   // one modulation weight [3D][D] and its bias [3D], staged for the GEMM
+  float* ada_c = nullptr;       // [K][D] condition of each step: the time embedding, rounded like an input
+  float* ada_mod = nullptr;     // [K][L][2][3D] (scale | shift | gate) of the pre-attention / pre-MLP norm
+  float* ada_gain = nullptr;    // [K][L][2][D] 1 + scale
+  float* ada_modf = nullptr;    // [K][2D] final norm (scale | shift)
+  float* ada_gainf = nullptr;   // [K][D]
+  float* ada_bout = nullptr;    // [K][A] b_out + W_out shift_f
+  float* ada_cq = nullptr;      // [K][L][(Hq+2Hkv)dh] W_qkv shift_1
+  float* ada_cg = nullptr;      // [K][L][2F] W_gu shift_2
 };
 
 namespace {
@@ -125,10 +136,20 @@ void run_stepwise(fr_handle* h, int B, bool measure, cudaStream_t s) {
   const int qm = qmode_of(h, measure);
   const float dt = static_cast<float>(-1.0 / c.K);
   const int P = h->prefix_P;
+  const bool ada = c.adarms != 0;
   for (int k = 0; k < c.K; ++k) {
-    launch_inproj(h->x, h->w_in, h->b_in, h->temb + static_cast<size_t>(k) * c.D, h->h, T, c.D, c.A, rb, s);
+    // adaptive RMSNorm: the time embedding conditions the norms instead of being added
+    launch_inproj(h->x, h->w_in, h->b_in, ada ? nullptr : h->temb + static_cast<size_t>(k) * c.D, h->h, T, c.D,
+                  c.A, rb, s);
     for (int l = 0; l < c.L; ++l) {
       const StepwiseWeights& w = h->lw[l];
+      const size_t kl = static_cast<size_t>(k) * c.L + l;
+      const float* gain1 = ada ? h->ada_gain + kl * 2 * c.D : w.g1;
+      const float* gain2 = ada ? gain1 + c.D : w.g2;
+      const float* gate1 = ada ? h->ada_mod + kl * 6 * c.D + 2 * c.D : nullptr;
+      const float* gate2 = ada ? gate1 + 3 * c.D : nullptr;
+      const float* bias_qkv = ada ? h->ada_cq + kl * h->n_qkv : nullptr;
+      const float* bias_gu = ada ? h->ada_cg + kl * 2 * c.F : nullptr;
       void* kk = h->kv_k + l * h->kv_layer_bytes;
       void* vv = h->kv_v + l * h->kv_layer_bytes;
       const float* sa = h->s_a + l * PI_COUNT;
@@ -137,19 +158,21 @@ void run_stepwise(fr_handle* h, int B, bool measure, cudaStream_t s) {
         if (c.dtype != FR_DTYPE_FP8) return nullptr;
         return (measure ? h->s_w : h->alpha) + l * PI_COUNT + i;
       };
-      launch_rmsnorm_q(h->h, w.g1, h->act, T, c.D, c.eps, qm, sa + PI_QKV, am + PI_QKV, s);
-      launch_gemm(h->act, c.D, w.wqkv, h->wtype, alpha(PI_QKV), h->qkv, h->n_qkv, T, h->n_qkv, c.D, 0, s);
+      launch_rmsnorm_q(h->h, gain1, h->act, T, c.D, c.eps, qm, sa + PI_QKV, am + PI_QKV, s);
+      launch_gemm(h->act, c.D, w.wqkv, h->wtype, alpha(PI_QKV), h->qkv, h->n_qkv, T, h->n_qkv, c.D, 0, s,
+                  bias_qkv);
       launch_rope_qkv(h->qkv, h->q, kk, vv, h->kv_bf, h->rope_cos, h->rope_sin, B, c.H, P, h->S_max,
                       c.Hq, c.Hkv, c.dh, rb, s);
       launch_attention(h->q, kk, vv, h->kv_bf, h->act, h->dq, B, c.H, P, h->S_max, c.Hq, c.Hkv, c.dh,
                        qm, sa + PI_O, am + PI_O, s);
-      launch_gemm(h->act, h->dq, w.wo, h->wtype, alpha(PI_O), h->h, c.D, T, c.D, h->dq, 1, s);
-      launch_rmsnorm_q(h->h, w.g2, h->act, T, c.D, c.eps, qm, sa + PI_GU, am + PI_GU, s);
-      launch_gemm(h->act, c.D, w.wgu, h->wtype, alpha(PI_GU), h->gu, 2 * c.F, T, 2 * c.F, c.D, 0, s);
+      launch_gemm(h->act, h->dq, w.wo, h->wtype, alpha(PI_O), h->h, c.D, T, c.D, h->dq, 1, s, nullptr, gate1);
+      launch_rmsnorm_q(h->h, gain2, h->act, T, c.D, c.eps, qm, sa + PI_GU, am + PI_GU, s);
+      launch_gemm(h->act, c.D, w.wgu, h->wtype, alpha(PI_GU), h->gu, 2 * c.F, T, 2 * c.F, c.D, 0, s, bias_gu);
       launch_gelu_mul(h->gu, h->act, T, c.F, qm, sa + PI_DOWN, am + PI_DOWN, s);
-      launch_gemm(h->act, c.F, w.wd, h->wtype, alpha(PI_DOWN), h->h, c.D, T, c.D, c.F, 1, s);
+      launch_gemm(h->act, c.F, w.wd, h->wtype, alpha(PI_DOWN), h->h, c.D, T, c.D, c.F, 1, s, nullptr, gate2);
     }
-    launch_final(h->h, h->g_f, h->w_out, h->b_out, h->x, T, c.D, c.A, c.eps, dt, rb, s);
+    launch_final(h->h, ada ? h->ada_gainf + static_cast<size_t>(k) * c.D : h->g_f, h->w_out,
+                 ada ? h->ada_bout + static_cast<size_t>(k) * c.A : h->b_out, h->x, T, c.D, c.A, c.eps, dt, rb, s);
   }
 }
 
@@ -271,6 +294,17 @@ int fr_create(const fr_config* cfg, int device, fr_handle** out) {
   const size_t o_sa = cv.take<float>(c.L * PI_COUNT), o_sw = cv.take<float>(c.L * PI_COUNT);
   const size_t o_alpha = cv.take<float>(c.L * PI_COUNT), o_amax = cv.take<unsigned>(c.L * PI_COUNT);
   const size_t o_status = cv.take<unsigned>(4);
+  const bool ada = c.adarms != 0;
+  const size_t KL = static_cast<size_t>(c.K) * c.L;
+  const size_t o_ada_stage = cv.take<float>(ada ? 3 * D * (D + 1) : 0);
+  const size_t o_ada_c = cv.take<float>(ada ? c.K * D : 0);
+  const size_t o_ada_mod = cv.take<float>(ada ? KL * 6 * D : 0);
+  const size_t o_ada_gain = cv.take<float>(ada ? KL * 2 * D : 0);
+  const size_t o_ada_modf = cv.take<float>(ada ? c.K * 2 * D : 0);
+  const size_t o_ada_gainf = cv.take<float>(ada ? c.K * D : 0);
+  const size_t o_ada_bout = cv.take<float>(ada ? static_cast<size_t>(c.K) * c.A : 0);
+  const size_t o_ada_cq = cv.take<float>(ada ? KL * h->n_qkv : 0);
+  const size_t o_ada_cg = cv.take<float>(ada ? KL * 2 * F : 0);
   size_t tp_bytes = 0;
   if (h->path == FR_PATH_TENSOR) tp_bytes = tensor_path_bytes(c);
   const size_t o_tp = cv.take<uint8_t>(tp_bytes, 1024);
@@ -324,6 +358,17 @@ int fr_create(const fr_config* cfg, int device, fr_handle** out) {
   h->alpha = reinterpret_cast<float*>(p + o_alpha);
   h->amax = reinterpret_cast<unsigned*>(p + o_amax);
   h->status = reinterpret_cast<unsigned*>(p + o_status);
+  if (ada) {
+    h->ada_stage = reinterpret_cast<float*>(p + o_ada_stage);
+    h->ada_c = reinterpret_cast<float*>(p + o_ada_c);
+    h->ada_mod = reinterpret_cast<float*>(p + o_ada_mod);
+    h->ada_gain = reinterpret_cast<float*>(p + o_ada_gain);
+    h->ada_modf = reinterpret_cast<float*>(p + o_ada_modf);
+    h->ada_gainf = reinterpret_cast<float*>(p + o_ada_gainf);
+    h->ada_bout = reinterpret_cast<float*>(p + o_ada_bout);
+    h->ada_cq = reinterpret_cast<float*>(p + o_ada_cq);
+    h->ada_cg = reinterpret_cast<float*>(p + o_ada_cg);
+  }
 
   // RoPE tables (R6): float64 math on the host, rounded once to float32.
   std::vector<float> ct(h->S_max * half), st(h->S_max * half);
@@ -353,6 +398,12 @@ int fr_create(const fr_config* cfg, int device, fr_handle** out) {
     tb.alpha = h->alpha;
     tb.s_a = h->s_a;
     tb.status = h->status;
+    tb.ada_gain = h->ada_gain;
+    tb.ada_mod = h->ada_mod;
+    tb.ada_gainf = h->ada_gainf;
+    tb.ada_bout = h->ada_bout;
+    tb.ada_cq = h->ada_cq;
+    tb.ada_cg = h->ada_cg;
     rc = tensor_path_create(c, tb, &h->tp);
     if (rc) {
       fr_destroy(h);
@@ -363,20 +414,79 @@ int fr_create(const fr_config* cfg, int device, fr_handle** out) {
   return FR_OK;
 }
 
-int fr_load_weights(fr_handle* h, const fr_weights* w, fr_stream_t stream) {
-  if (!h || !w || !w->layers || !w->w_in || !w->b_in || !w->w_out || !w->b_out || !w->w_t1 || !w->b_t1 ||
-      !w->w_t2 || !w->b_t2 || !w->g_f) {
+// Adaptive RMSNorm, once per weight load: the condition of every Euler step (its time embedding,
+// rounded like a projection input), each norm's (scale | shift | gate) = W_mod c + b_mod, the gains
+// 1 + scale, and the shifts folded into the projections they feed: W_qkv shift_1, W_gu shift_2 and
+// b_out + W_out shift_f.  Runs the stepwise GEMM kernel on the stored (rounded / quantised) weights.
+int prepare_adarms(fr_handle* h, const fr_weights& w, bool rb, cudaStream_t s) {
+  const fr_config& c = h->cfg;
+  const int D = c.D, K = c.K, L = c.L;
+  const int ld_mod = L * 6 * D;   // row stride of ada_mod between steps
+  launch_round_rows(h->temb, D, h->ada_c, K, D, rb ? 1 : 0, s);
+  auto modulate = [&](const float* W, const float* b, int rows, float* out, int ldo) -> int {
+    std::vector<float> v = rounded_f32(W, static_cast<size_t>(rows) * D, rb);
+    FR_CUDA(cudaMemcpyAsync(h->ada_stage, v.data(), v.size() * 4, cudaMemcpyHostToDevice, s));
+    FR_CUDA(cudaMemcpyAsync(h->ada_stage + v.size(), b, static_cast<size_t>(rows) * 4, cudaMemcpyHostToDevice, s));
+    launch_gemm(h->ada_c, D, h->ada_stage, W_F32, nullptr, out, ldo, K, rows, D, 0, s, h->ada_stage + v.size());
+    int rc = check_launch("adaRMS modulation GEMM");
+    if (rc) return rc;
+    FR_CUDA(cudaStreamSynchronize(s));   // the stage is rewritten by the next call
+    return FR_OK;
+  };
+  int rc;
+  for (int l = 0; l < L; ++l) {
+    const fr_layer_weights& lw = w.layers[l];
+    if ((rc = modulate(lw.w_mod1, lw.b_mod1, 3 * D, h->ada_mod + static_cast<size_t>(l) * 6 * D, ld_mod))) return rc;
+    if ((rc = modulate(lw.w_mod2, lw.b_mod2, 3 * D, h->ada_mod + static_cast<size_t>(l) * 6 * D + 3 * D, ld_mod)))
+      return rc;
+  }
+  if ((rc = modulate(w.w_modf, w.b_modf, 2 * D, h->ada_modf, 2 * D))) return rc;
+  launch_one_plus(h->ada_mod, 3 * D, h->ada_gain, K * L * 2, D, s);
+  launch_one_plus(h->ada_modf, 2 * D, h->ada_gainf, K, D, s);
+  const bool fp8 = c.dtype == FR_DTYPE_FP8;
+  for (int l = 0; l < L; ++l) {   // shifts folded into the projections (fp8: dequantised by s_w)
+    const StepwiseWeights& lw = h->lw[l];
+    const float* shift1 = h->ada_mod + static_cast<size_t>(l) * 6 * D + D;
+    const float* shift2 = shift1 + 3 * D;
+    launch_gemm(shift1, ld_mod, lw.wqkv, h->wtype, fp8 ? h->s_w + l * PI_COUNT + PI_QKV : nullptr,
+                h->ada_cq + static_cast<size_t>(l) * h->n_qkv, L * h->n_qkv, K, h->n_qkv, D, 0, s);
+    launch_gemm(shift2, ld_mod, lw.wgu, h->wtype, fp8 ? h->s_w + l * PI_COUNT + PI_GU : nullptr,
+                h->ada_cg + static_cast<size_t>(l) * 2 * c.F, L * 2 * c.F, K, 2 * c.F, D, 0, s);
+  }
+  launch_gemm(h->ada_modf + D, 2 * D, h->w_out, W_F32, nullptr, h->ada_bout, c.A, K, c.A, D, 0, s, h->b_out);
+  return check_launch("adaRMS preparation kernels");
+}
+
+int fr_load_weights(fr_handle* h, const fr_weights* w_in, fr_stream_t stream) {
+  if (!h || !w_in || !w_in->layers || !w_in->w_in || !w_in->b_in || !w_in->w_out || !w_in->b_out ||
+      !w_in->w_t1 || !w_in->b_t1 || !w_in->w_t2 || !w_in->b_t2) {
     set_error("fr_load_weights: NULL argument");
     return FR_ERR_ARG;
   }
   const fr_config& c = h->cfg;
+  const bool ada = c.adarms != 0;
+  if (ada ? (!w_in->w_modf || !w_in->b_modf) : !w_in->g_f) {
+    set_error(ada ? "fr_load_weights: adarms handle without w_modf / b_modf" : "fr_load_weights: NULL g_f");
+    return FR_ERR_ARG;
+  }
   for (int l = 0; l < c.L; ++l) {
-    const fr_layer_weights& L = w->layers[l];
-    if (!L.wq || !L.wk || !L.wv || !L.wo || !L.wg || !L.wu || !L.wd || !L.g1 || !L.g2) {
+    const fr_layer_weights& L = w_in->layers[l];
+    if (!L.wq || !L.wk || !L.wv || !L.wo || !L.wg || !L.wu || !L.wd ||
+        (ada ? (!L.w_mod1 || !L.b_mod1 || !L.w_mod2 || !L.b_mod2) : (!L.g1 || !L.g2))) {
       set_error("fr_load_weights: NULL tensor in layer %d", l);
       return FR_ERR_ARG;
     }
   }
+  // adaptive RMSNorm replaces the static gains: they are unused, read as ones
+  const std::vector<float> ones(ada ? static_cast<size_t>(c.D) : 0, 1.f);
+  std::vector<fr_layer_weights> layers(w_in->layers, w_in->layers + c.L);
+  fr_weights wcopy = *w_in;
+  if (ada) {
+    for (fr_layer_weights& L : layers) L.g1 = L.g2 = ones.data();
+    wcopy.g_f = ones.data();
+  }
+  wcopy.layers = layers.data();
+  const fr_weights* w = &wcopy;
   FR_CUDA(cudaSetDevice(h->device));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t D = c.D, F = c.F, dq = h->dq, nkv = static_cast<size_t>(c.Hkv) * c.dh;
@@ -445,6 +555,7 @@ int fr_load_weights(fr_handle* h, const fr_weights* w, fr_stream_t stream) {
   FR_CUDA(cudaMemcpy(h->s_w, h->h_sw.data(), h->h_sw.size() * 4, cudaMemcpyHostToDevice));
   launch_temb(h->w_t1, h->b_t1, h->w_t2, h->b_t2, h->temb, c.D, c.time_dim, c.K, c.time_base, rb, s);
   if ((rc = check_launch("time MLP kernel"))) return rc;
+  if (ada && (rc = prepare_adarms(h, *w, rb, s))) return rc;
   FR_CUDA(cudaStreamSynchronize(s));
   if (h->tp) {
     rc = tensor_path_finish_load(h->tp, s);

@@ -122,7 +122,7 @@ __global__ void k_inproj(const float* __restrict__ x, const float* __restrict__ 
     const float* row = w_in + static_cast<size_t>(n) * A;
     float acc = 0.f;
     for (int a = 0; a < A; ++a) acc = fmaf(row[a], xs[a], acc);
-    h[static_cast<size_t>(t) * D + n] = acc + b_in[n] + temb_k[n];
+    h[static_cast<size_t>(t) * D + n] = acc + b_in[n] + (temb_k ? temb_k[n] : 0.f);   // no temb: adaRMS
   }
 }
 
@@ -161,7 +161,8 @@ template <typename WT>
 __global__ void __launch_bounds__(256) k_gemm(const float* __restrict__ A, int lda,
                                               const WT* __restrict__ W, const float* __restrict__ alpha,
                                               float* __restrict__ C, int ldc, int T, int N, int Kd,
-                                              int accumulate) {
+                                              int accumulate, const float* __restrict__ bias,
+                                              const float* __restrict__ gate) {
   __shared__ float As[GK][GT + 4];
   __shared__ float Ws[GK][GN + 4];
   const int t0 = blockIdx.y * GT, n0 = blockIdx.x * GN;
@@ -200,7 +201,9 @@ __global__ void __launch_bounds__(256) k_gemm(const float* __restrict__ A, int l
       const int n = n0 + tx * 4 + j;
       if (n >= N) continue;
       float* c = C + static_cast<size_t>(t) * ldc + n;
-      const float v = al * acc[i][j];
+      float v = al * acc[i][j];
+      if (gate) v *= gate[n];   // adaRMS gated residual update
+      if (bias) v += bias[n];   // adaRMS shift folded into the projection (W b)
       *c = accumulate ? *c + v : v;
     }
   }
@@ -395,19 +398,49 @@ void launch_rmsnorm_q(const float* h, const float* gamma, float* out, int T, int
 }
 
 void launch_gemm(const float* A, int lda, const void* W, int wtype, const float* alpha, float* C,
-                 int ldc, int T, int N, int Kd, int accumulate, cudaStream_t s) {
+                 int ldc, int T, int N, int Kd, int accumulate, cudaStream_t s, const float* bias,
+                 const float* gate) {
   dim3 grid((N + GN - 1) / GN, (T + GT - 1) / GT);
   switch (wtype) {
     case W_F32:
-      k_gemm<float><<<grid, 256, 0, s>>>(A, lda, static_cast<const float*>(W), alpha, C, ldc, T, N, Kd, accumulate);
+      k_gemm<float><<<grid, 256, 0, s>>>(A, lda, static_cast<const float*>(W), alpha, C, ldc, T, N, Kd, accumulate,
+                                         bias, gate);
       break;
     case W_BF16:
-      k_gemm<__nv_bfloat16><<<grid, 256, 0, s>>>(A, lda, static_cast<const __nv_bfloat16*>(W), alpha, C, ldc, T, N, Kd, accumulate);
+      k_gemm<__nv_bfloat16><<<grid, 256, 0, s>>>(A, lda, static_cast<const __nv_bfloat16*>(W), alpha, C, ldc, T, N,
+                                                 Kd, accumulate, bias, gate);
       break;
     default:
-      k_gemm<uint8_t><<<grid, 256, 0, s>>>(A, lda, static_cast<const uint8_t*>(W), alpha, C, ldc, T, N, Kd, accumulate);
+      k_gemm<uint8_t><<<grid, 256, 0, s>>>(A, lda, static_cast<const uint8_t*>(W), alpha, C, ldc, T, N, Kd,
+                                           accumulate, bias, gate);
       break;
   }
+}
+
+// ------------------------------------------------------------------ adaRMS preparation (load time)
+// out[r][j] = in[r * in_ld + j], rounded to bf16 when rb
+__global__ void k_round_rows(const float* __restrict__ in, int in_ld, float* __restrict__ out, int rows, int n,
+                             int rb) {
+  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < static_cast<long>(rows) * n;
+       i += static_cast<long>(gridDim.x) * blockDim.x) {
+    const float v = in[(i / n) * in_ld + i % n];
+    out[i] = rb ? round_bf16(v) : v;
+  }
+}
+
+// out[r][j] = 1 + in[r * in_ld + j]: the norm gain 1 + s of each modulation row
+__global__ void k_one_plus(const float* __restrict__ in, int in_ld, float* __restrict__ out, int rows, int n) {
+  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < static_cast<long>(rows) * n;
+       i += static_cast<long>(gridDim.x) * blockDim.x)
+    out[i] = 1.0f + in[(i / n) * in_ld + i % n];
+}
+
+void launch_round_rows(const float* in, int in_ld, float* out, int rows, int n, int rb, cudaStream_t s) {
+  k_round_rows<<<148, 256, 0, s>>>(in, in_ld, out, rows, n, rb);
+}
+
+void launch_one_plus(const float* in, int in_ld, float* out, int rows, int n, cudaStream_t s) {
+  k_one_plus<<<148, 256, 0, s>>>(in, in_ld, out, rows, n);
 }
 
 void launch_rope_qkv(const float* qkv, float* q, void* kv_k, void* kv_v, int kv_bf,

@@ -575,6 +575,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
     if (S > 1 && !mbar_wait(&sh.hbar, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0x600);
     float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f);
     if (a.xb_out && fok) g4 = *reinterpret_cast<const float4*>(a.xb_gamma + f);
+    float4 gt = make_float4(1.f, 1.f, 1.f, 1.f);   // adaptive RMSNorm: gated residual update
+    if (a.gate && fok) gt = *reinterpret_cast<const float4*>(a.gate + f);
     for (int tb = tok0 + warp; tb < tok1; tb += 8 * EPU) {
       float4 hold[EPU];
       float acc[EPU][4];
@@ -593,8 +595,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         if (tok >= tok1 || t >= a.T) break;   // warp-uniform
         float sq = 0.f;
         if (fok) {
-          const float4 hv = make_float4(hold[u].x + acc[u][0], hold[u].y + acc[u][1], hold[u].z + acc[u][2],
-                                        hold[u].w + acc[u][3]);
+          const float4 hv = make_float4(hold[u].x + gt.x * acc[u][0], hold[u].y + gt.y * acc[u][1],
+                                        hold[u].z + gt.z * acc[u][2], hold[u].w + gt.w * acc[u][3]);
           sq = ((hv.x * hv.x + hv.y * hv.y) + hv.z * hv.z) + hv.w * hv.w;
           *reinterpret_cast<float4*>(a.h_out + htile_offset(t, f, Nt, a.KB)) = hv;
           if (a.xb_out)
@@ -609,12 +611,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
     const int p = lane * 2;
     const int f = mb * 64 + p;   // F is a multiple of 64
     const float inv = (FP8 && a.s_a_out) ? 1.0f / *a.s_a_out : 1.0f;
+    float2 bg = make_float2(0.f, 0.f), bu = make_float2(0.f, 0.f);   // adaptive RMSNorm shift, W b
+    if (a.bias && f < a.F) {
+      bg = *reinterpret_cast<const float2*>(a.bias + f);
+      bu = *reinterpret_cast<const float2*>(a.bias + a.F + f);
+    }
     for (int tok = tok0 + warp; tok < tok1; tok += 8) {
       const int t = n0 + tok;
       if (t >= a.T || f >= a.F) break;
       float g[2], up[2];
       vals(tok, p, g, Two{});
       vals(tok, p + 64, up, Two{});
+      g[0] += bg.x;
+      g[1] += bg.y;
+      up[0] += bu.x;
+      up[1] += bu.y;
       const float u0 = gelu_tanh(g[0]) * up[0], u1 = gelu_tanh(g[1]) * up[1];
       if (FP8) {
         *reinterpret_cast<uint16_t*>(a.u_out + btile_offset(t, f, Nt, a.NKC_u)) =
@@ -629,6 +640,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       const int p = lane * 2;                 // rotate-half pairs p, p+1 (same head: half is even)
       const int pi = mb * 64 + p;
       const int head = pi / half, j = pi % half;
+      float2 blo = make_float2(0.f, 0.f), bhi = make_float2(0.f, 0.f);   // adaptive RMSNorm shift, W b
+      if (a.bias) {
+        blo = *reinterpret_cast<const float2*>(a.bias + head * a.dh + j);
+        bhi = *reinterpret_cast<const float2*>(a.bias + head * a.dh + j + half);
+      }
       for (int tb = tok0 + warp; tb < tok1; tb += 8 * EPU) {
         float2 cs[EPU], sn[EPU];
 #pragma unroll
@@ -648,6 +664,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
           float lo[2], hi[2];
           vals(tok, p, lo, Two{});
           vals(tok, p + 64, hi, Two{});
+          lo[0] += blo.x;
+          lo[1] += blo.y;
+          hi[0] += bhi.x;
+          hi[1] += bhi.y;
           const float r00 = lo[0] * cs[u].x - hi[0] * sn[u].x, r10 = lo[0] * sn[u].x + hi[0] * cs[u].x;
           const float r01 = lo[1] * cs[u].y - hi[1] * sn[u].y, r11 = lo[1] * sn[u].y + hi[1] * cs[u].y;
           __nv_bfloat16* dst;
@@ -661,12 +681,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       const int row = lane * 4;
       const int idx = (mb - a.MB_rot) * BM + row;
       const int g = idx / a.dh, d = idx % a.dh;
+      float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);   // adaptive RMSNorm shift, W b
+      if (a.bias) bv = *reinterpret_cast<const float4*>(a.bias + (a.Hq + a.Hkv) * a.dh + idx);
       for (int tok = tok0 + warp; tok < tok1; tok += 8) {
         const int t = n0 + tok;
         if (t >= a.T) break;
         const int b = t / a.H, i = t % a.H, pos = a.P + i;
         float v4[4];
         vals(tok, row, v4, Four{});
+        v4[0] += bv.x;
+        v4[1] += bv.y;
+        v4[2] += bv.z;
+        v4[3] += bv.w;
         *reinterpret_cast<uint2*>(a.kv_v + ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max + pos) * a.dh + d) =
             make_uint2(pack_bf16x2(v4[0], v4[1]), pack_bf16x2(v4[2], v4[3]));
       }
@@ -1448,7 +1474,7 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
 #pragma unroll
   for (int q = 0; q < QMAX; ++q) {
     const int n = tid + q * 256;
-    base[q] = n < a.D ? a.b_in[n] + a.temb[n] : 0.f;
+    base[q] = n < a.D ? a.b_in[n] + (a.temb ? a.temb[n] : 0.f) : 0.f;   // no temb: adaptive RMSNorm
   }
   grid_dep_wait();
   if (tid == 0) TL(1);

@@ -82,6 +82,8 @@ struct GemmArgs {
   // epilogue
   int epi;
   const float* alpha;      // fp8: dequantisation scale s_a * s_w (device scalar), else nullptr
+  const float* bias;       // EPI_QKV / EPI_GELU: added per output feature (natural row order), or nullptr
+  const float* gate;       // EPI_RESID: the update is scaled per feature before h +=, or nullptr
   // EPI_QKV
   __nv_bfloat16* q_out;    // [B][Hq][H][dh]
   __nv_bfloat16* kv_k;     // layer slice of the KV cache [B_max][Hkv][S_max][dh]

@@ -312,15 +312,20 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
   const float dt = static_cast<float>(-1.0 / c.K);
   const size_t o_off = tp->qkv.bytes, gu_off = o_off + tp->o.bytes, dn_off = gu_off + tp->gu.bytes;
   cudaError_t e;
+  const bool ada = c.adarms != 0;
   for (int k = 0; k < c.K; ++k) {
     const float* x_in = (k == 0) ? x0 : tp->xs;
     float* x_nx = (k == c.K - 1) ? x_out : tp->xs;
+    // adaptive RMSNorm: this step's gain of norm n (0 pre-attention, 1 pre-MLP) of layer l, and its
+    // (scale | shift | gate) row
+    auto ada_gain = [&](int l, int n) { return tp->tb.ada_gain + ((static_cast<size_t>(k) * c.L + l) * 2 + n) * c.D; };
+    auto ada_mod = [&](int l, int n) { return tp->tb.ada_mod + ((static_cast<size_t>(k) * c.L + l) * 2 + n) * 3 * c.D; };
     InprojArgs ia{};
     ia.max_ctas = 2 * tp->nsm;
     ia.x = x_in;
     ia.w_in = tp->w_in_bf;
     ia.b_in = tp->tb.b_in;
-    ia.temb = tp->tb.temb + static_cast<size_t>(k) * c.D;
+    ia.temb = ada ? nullptr : tp->tb.temb + static_cast<size_t>(k) * c.D;
     ia.h = tp->h;
     ia.ssq = tp->ssq_a;
     ia.T = p.T;
@@ -330,7 +335,7 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
     ia.KB = tp->KB;
     ia.ssq_ld = tp->ssq_ld;
     ia.xb = tp->fp8 ? nullptr : tp->xbuf;
-    ia.xb_gamma = tp->gains;   // gamma1 of layer 0
+    ia.xb_gamma = ada ? ada_gain(0, 0) : tp->gains;   // gamma1 of layer 0
     ia.NKC_x = tp->qkv.NKC;
     ia.first = (k == 0);
     if ((e = launch_inproj_tc(ia, s, true)) != cudaSuccess) return cuda_fail(e, "in-proj kernel launch");
@@ -339,8 +344,8 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       const float* al = tp->tb.alpha ? tp->tb.alpha + l * PI_COUNT : nullptr;
       __nv_bfloat16* kvk = reinterpret_cast<__nv_bfloat16*>(tp->tb.kv_k + l * tp->tb.kv_layer_bytes);
       __nv_bfloat16* kvv = reinterpret_cast<__nv_bfloat16*>(tp->tb.kv_v + l * tp->tb.kv_layer_bytes);
-      const float* g1 = tp->gains + static_cast<size_t>(l) * 2 * c.D;
-      const float* g2 = g1 + c.D;
+      const float* g1 = ada ? ada_gain(l, 0) : tp->gains + static_cast<size_t>(l) * 2 * c.D;
+      const float* g2 = ada ? ada_gain(l, 1) : g1 + c.D;
       // QKV: RMSNorm fused into the B staging, split + RoPE fused into the epilogue
       GemmArgs q = base_args(tp, p, tp->qkv, p.qkv, l, 0);
       if (tp->fp8) {
@@ -368,6 +373,7 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       q.Hkv = c.Hkv;
       q.dh = c.dh;
       q.MB_rot = tp->MB_rot;
+      q.bias = ada ? tp->tb.ada_cq + (static_cast<size_t>(k) * c.L + l) * (c.Hq + 2 * c.Hkv) * c.dh : nullptr;
       if ((e = launch_gemm_tc(q, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "qkv GEMM launch");
       // attention over [prefix; actions]
       AttnArgs at{};
@@ -403,6 +409,7 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       og.xb_out = tp->fp8 ? nullptr : tp->xbuf;
       og.xb_gamma = g2;
       og.NKC_x = tp->qkv.NKC;
+      og.gate = ada ? ada_mod(l, 0) + 2 * c.D : nullptr;
       if ((e = launch_gemm_tc(og, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "o GEMM launch");
       // gate|up with RMSNorm fused, GeLU(gate)*up epilogue
       GemmArgs gg = base_args(tp, p, tp->gu, p.gu, l, gu_off);
@@ -423,6 +430,7 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       gg.NKC_u = tp->dn.NKC;
       gg.s_a_out = tp->fp8 ? sa + PI_DOWN : nullptr;
       gg.F = c.F;
+      gg.bias = ada ? tp->tb.ada_cg + (static_cast<size_t>(k) * c.L + l) * 2 * c.F : nullptr;
       if ((e = launch_gemm_tc(gg, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "gate|up GEMM launch");
       // down projection + residual (+ sum of squares for the next norm)
       GemmArgs dg = base_args(tp, p, tp->dn, p.dn, l, dn_off);
@@ -433,8 +441,9 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
       dg.h_out = tp->h;
       dg.ssq_out = tp->ssq_a;
       dg.xb_out = (tp->fp8 || l == c.L - 1) ? nullptr : tp->xbuf;
-      dg.xb_gamma = g1 + 2 * c.D;   // gamma1 of layer l+1
+      dg.xb_gamma = (l == c.L - 1) ? nullptr : (ada ? ada_gain(l + 1, 0) : g1 + 2 * c.D);   // gamma1 of layer l+1
       dg.NKC_x = tp->qkv.NKC;
+      dg.gate = ada ? ada_mod(l, 1) + 2 * c.D : nullptr;
       if ((e = launch_gemm_tc(dg, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "down GEMM launch");
     }
     FinalArgs fa{};
@@ -443,9 +452,9 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
     fa.ssq = tp->ssq_a;
     fa.ssq_ld = tp->ssq_ld;
     fa.ssq_parts = tp->MBd;
-    fa.g_f = tp->tb.g_f;
+    fa.g_f = ada ? tp->tb.ada_gainf + static_cast<size_t>(k) * c.D : tp->tb.g_f;
     fa.w_out = tp->w_out_bf;
-    fa.b_out = tp->tb.b_out;
+    fa.b_out = ada ? tp->tb.ada_bout + static_cast<size_t>(k) * c.A : tp->tb.b_out;
     fa.x_in = x_in;
     fa.x_out = x_nx;
     fa.T = p.T;

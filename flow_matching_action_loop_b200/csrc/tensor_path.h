@@ -27,6 +27,13 @@ struct TensorPathBuffers {
   const float* alpha;         // [L][4] fp8 GEMM epilogue scales
   const float* s_a;           // [L][4] fp8 activation scales
   unsigned* status;           // device status word
+  // adaptive RMSNorm (cfg.adarms), per Euler step k and layer l (see AdaRmsBuffers in runtime.cu)
+  const float* ada_gain;      // [K][L][2][D] 1 + scale of the pre-attention / pre-MLP norm
+  const float* ada_mod;       // [K][L][2][3D] (scale | shift | gate)
+  const float* ada_gainf;     // [K][D] final norm gain
+  const float* ada_bout;      // [K][A] b_out + W_out shift_f
+  const float* ada_cq;        // [K][L][(Hq+2Hkv)dh] W_qkv shift_1
+  const float* ada_cg;        // [K][L][2F] W_gu shift_2
 };
 
 struct TensorPath;

@@ -90,6 +90,8 @@ typedef struct fr_config {
   float eps;
   int time_dim;
   float time_base;
+  int adarms;     /* 0: the time embedding is added to the action tokens; 1: it conditions every
+                     RMSNorm (adaptive RMSNorm, see fr_layer_weights.w_mod1) */
 } fr_config;
 
 /* Host float32 weights of one layer, row-major [out][in] (the nn.Linear convention). */
@@ -101,8 +103,16 @@ typedef struct fr_layer_weights {
   const float* wg;   /* [F][D] gate */
   const float* wu;   /* [F][D] up   */
   const float* wd;   /* [D][F] down */
-  const float* g1;   /* [D] pre-attention RMSNorm gain */
-  const float* g2;   /* [D] pre-MLP RMSNorm gain */
+  const float* g1;   /* [D] pre-attention RMSNorm gain (ignored and may be NULL when adarms) */
+  const float* g2;   /* [D] pre-MLP RMSNorm gain (ignored and may be NULL when adarms) */
+  /* adarms handles only (NULL otherwise).  The time embedding c of the step (the time MLP's
+   * output) gives each norm (scale s, shift b, gate g) = w_mod c + b_mod, rows [s | b | g];
+   * the norm's output is RMS(h) * (1 + s) + b and the residual update it feeds is scaled by g
+   * (pi0.5-style adaptive RMSNorm; the pages do not describe the conditioning). */
+  const float* w_mod1;   /* [3D][D] pre-attention norm */
+  const float* b_mod1;   /* [3D] */
+  const float* w_mod2;   /* [3D][D] pre-MLP norm */
+  const float* b_mod2;   /* [3D] */
 } fr_layer_weights;
 
 /* Host float32 weights of the action expert, by name. */
@@ -116,7 +126,9 @@ typedef struct fr_weights {
   const float* b_t1;   /* [D] */
   const float* w_t2;   /* [D][D] */
   const float* b_t2;   /* [D] */
-  const float* g_f;    /* [D] final RMSNorm gain */
+  const float* g_f;    /* [D] final RMSNorm gain (ignored and may be NULL when adarms) */
+  const float* w_modf; /* adarms only: [2D][D] final norm modulation, rows [scale | shift] */
+  const float* b_modf; /* adarms only: [2D] */
 } fr_weights;
 
 /*
@@ -137,7 +149,10 @@ int fr_create(const fr_config* cfg, int device, fr_handle** out);
  * for FR_DTYPE_FP8, quantises each fused projection to e4m3 with
  * s_w = max|w| / 448, or, for FR_DTYPE_W4A16, quantises every layer projection
  * to 4-bit codes with a bf16 scale per FR_W4_GROUP inputs (fr_quantize_w4), and
- * precomputes the K time embeddings and the RoPE tables.  Synchronous with respect to the host pointers; the caller keeps
+ * precomputes the K time embeddings and the RoPE tables.  For adarms handles it also
+ * precomputes every step's norm modulation and folds each shift b into the projection it
+ * feeds (W b added to that projection's output; the projection input is RMS(h) * (1 + s)).
+ * Synchronous with respect to the host pointers; the caller keeps
  * ownership of `w`.  Errors: FR_ERR_ARG, FR_ERR_CUDA.
  */
 int fr_load_weights(fr_handle* h, const fr_weights* w, fr_stream_t stream);

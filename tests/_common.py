@@ -31,6 +31,10 @@ RAGGED = {
     "minimal_bf16": synthetic.ActionExpertConfig("minimal_bf16", L=1, D=128, Hq=1, Hkv=1, dh=128, F=128, H=1,
                                                  A=1, B=1, P=1, K=1, dtype="bf16"),
 }
+# the same ragged shapes with adaptive-RMSNorm time conditioning
+for _n in ("bf16", "fp8", "w4a16", "f32"):
+    _c = RAGGED["ragged_" + _n]
+    RAGGED["ragged_adarms_" + _n] = _c.replace(name="ragged_adarms_" + _n, adarms=True)
 
 
 def get_config(name):
