@@ -68,6 +68,15 @@ Readings where the pages are silent (each listed in the design notes):
       RMS(h) * (1 + s) and W b is added to the projection's output in full
       precision: W (a + b) = W a + W b, with the rounding point placed before
       the shift, as R10 places it before the rstd factor.
+  R18 prefix pass (the step before the loop; FlashRT walkthrough, component 5:
+      the Pi0.5 attention sites; the KV cache the loop reads is the backbone's
+      per-layer keys and values): the backbone is the action expert's layer
+      block at its own sizes, run once over the P embedded prefix tokens of a
+      sample (inputs: the vision encoder's and text embedding's outputs, bf16)
+      with full attention among them (no mask inside the prefix), RoPE at
+      positions 0..P-1, no time input; layer l's rotated K and its V are the
+      action expert's prefix K/V of layer l.  The last layer stops after its
+      QKV projection.
 """
 from __future__ import annotations
 
@@ -275,6 +284,26 @@ def attention(q, k, v):
 # Model preparation: the stored (rounded / quantised) weights the method computes with
 # --------------------------------------------------------------------------------------
 
+def _prepare_layer(dtype: str, lw: dict, rnd) -> dict:
+    """One layer's weights as the method stores them (R10, R11, R16)."""
+    d = {"g1": np.asarray(lw["g1"], np.float64), "g2": np.asarray(lw["g2"], np.float64)}
+    if dtype == "fp8":
+        for name, parts in (("qkv", ("wq", "wk", "wv")), ("o", ("wo",)),
+                            ("gu", ("wg", "wu")), ("down", ("wd",))):
+            amax = max(float(np.max(np.abs(np.asarray(lw[p], np.float64)))) for p in parts)
+            s_w = amax / E4M3_MAX
+            d["sw_" + name] = s_w
+            for p in parts:
+                d[p] = round_e4m3(np.asarray(lw[p], np.float64) / s_w)   # codes' values
+    elif dtype == "w4a16":
+        for p in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
+            d[p] = dequantize_w4(*quantize_w4(lw[p]))
+    else:
+        for p in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
+            d[p] = rnd(lw[p])
+    return d
+
+
 class PreparedModel:
     """Weights as the method stores them for one workload (R10, R11, R12).
 
@@ -299,24 +328,7 @@ class PreparedModel:
         self.b_t1 = np.asarray(weights["b_t1"], np.float64)
         self.b_t2 = np.asarray(weights["b_t2"], np.float64)
         self.g_f = np.asarray(weights["g_f"], np.float64)
-        self.layers: List[dict] = []
-        for lw in weights["layers"]:
-            d = {"g1": np.asarray(lw["g1"], np.float64), "g2": np.asarray(lw["g2"], np.float64)}
-            if cfg.dtype == "fp8":
-                for name, parts in (("qkv", ("wq", "wk", "wv")), ("o", ("wo",)),
-                                    ("gu", ("wg", "wu")), ("down", ("wd",))):
-                    amax = max(float(np.max(np.abs(np.asarray(lw[p], np.float64)))) for p in parts)
-                    s_w = amax / E4M3_MAX
-                    d["sw_" + name] = s_w
-                    for p in parts:
-                        d[p] = round_e4m3(np.asarray(lw[p], np.float64) / s_w)   # codes' values
-            elif cfg.dtype == "w4a16":
-                for p in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
-                    d[p] = dequantize_w4(*quantize_w4(lw[p]))
-            else:
-                for p in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
-                    d[p] = rnd(lw[p])
-            self.layers.append(d)
+        self.layers: List[dict] = [_prepare_layer(cfg.dtype, lw, rnd) for lw in weights["layers"]]
         self.adarms = bool(getattr(cfg, "adarms", False))
         if self.adarms:   # R17: modulation projections of the condition, stored like the time MLP
             for d, lw in zip(self.layers, weights["layers"]):
@@ -442,20 +454,24 @@ def velocity(model: PreparedModel, x, k_step: int, t: float, kv_k, kv_v,
     return rnd(rms_norm(h, model.g_f, cfg.eps)) @ model.w_out.T + model.b_out
 
 
-def _sample_kv(model: PreparedModel, prefix_k, prefix_v, b: int):
-    kv_k = model.rotate_prefix_k(np.asarray(prefix_k)[:, b])          # [L][Hkv][P][dh]
+def _sample_kv(model: PreparedModel, prefix_k, prefix_v, b: int, k_rotated: bool = False):
+    if k_rotated:   # already carries RoPE at 0..P-1 (the prefix pass's output)
+        kv_k = model.rnd(np.asarray(prefix_k)[:, b]).transpose(0, 2, 1, 3)
+    else:
+        kv_k = model.rotate_prefix_k(np.asarray(prefix_k)[:, b])          # [L][Hkv][P][dh]
     kv_v = model.rnd(np.asarray(prefix_v)[:, b]).transpose(0, 2, 1, 3)
     return kv_k, kv_v
 
 
 def denoise(cfg, weights: dict, prefix_k, prefix_v, x0, scales: Optional[Dict] = None,
             samples: Optional[List[int]] = None, K: Optional[int] = None,
-            model: Optional[PreparedModel] = None) -> np.ndarray:
+            model: Optional[PreparedModel] = None, prefix_k_rotated: bool = False) -> np.ndarray:
     """Run the K-step Euler loop for the chosen samples of the batch; returns [len(samples)][H][A].
 
     Samples are independent (each has its own prefix and noise), so a subset of
     the batch can be checked without the rest.  K defaults to cfg.K; a smaller K
     runs only the first K steps of the same grid (a bounded sample of the work).
+    prefix_k_rotated: the prefix K already carries RoPE (R8 does not rotate it again).
     """
     model = model or PreparedModel(cfg, weights)
     samples = list(range(cfg.B)) if samples is None else list(samples)
@@ -466,7 +482,7 @@ def denoise(cfg, weights: dict, prefix_k, prefix_v, x0, scales: Optional[Dict] =
     nsteps = Kfull if K is None else K
     out = []
     for b in samples:
-        kv_k, kv_v = _sample_kv(model, prefix_k, prefix_v, b)
+        kv_k, kv_v = _sample_kv(model, prefix_k, prefix_v, b, prefix_k_rotated)
         x = np.asarray(x0[b], dtype=np.float64).copy()
         for k in range(nsteps):
             x = x + dt * velocity(model, x, k, ts[k], kv_k, kv_v, scales=scales)
@@ -510,3 +526,57 @@ def array_to_scales(arr) -> Dict:
 def weight_scales(model: PreparedModel) -> np.ndarray:
     """[L][4] e4m3 weight scales s_w of the fused projections (fp8 workloads)."""
     return np.array([[lay["sw_" + w] for w in PROJ_INPUTS] for lay in model.layers], np.float64)
+
+
+# --------------------------------------------------------------------------------------
+# The prefix pass (R18): the backbone over the observation's tokens, producing the KV cache
+# --------------------------------------------------------------------------------------
+
+class PrefixModel:
+    """Backbone weights of the prefix pass as the method stores them (R10, R16): the same layer
+    block as the action expert (pi0.5's action expert attends to the backbone's per-layer keys and
+    values; FlashRT walkthrough, component 5, attention sites of the Pi0.5 model)."""
+
+    def __init__(self, cfg, weights: dict):
+        self.cfg = cfg
+        self.dtype = cfg.dtype
+        self.rnd = round_bf16
+        self.layers: List[dict] = [_prepare_layer(cfg.dtype, lw, self.rnd) for lw in weights["layers"]]
+        self.cos, self.sin = rope_tables(cfg.P, cfg.dh, cfg.rope_theta)
+
+
+def prefill(cfg, weights: dict, emb, model: Optional[PrefixModel] = None, samples: Optional[List[int]] = None):
+    """Keys and values of every layer for the P prefix tokens of each sample (R18).
+
+    emb [B][P][D]: the embedded tokens.  Per layer: a = RMS(h) gamma1, fused QKV, RoPE at
+    positions 0..P-1, K and V stored (bf16, K rotated); then, except after the last layer (whose
+    keys and values are all the action expert needs), full attention among the P tokens, the
+    O projection and residual, RMS(h) gamma2, gated-GeLU MLP and residual.
+    Returns (K, V), each [L][len(samples)][P][Hkv][dh]: the rotated prefix K and V.
+    """
+    model = model or PrefixModel(cfg, weights)
+    rnd = model.rnd
+    samples = list(range(cfg.B)) if samples is None else list(samples)
+    P, dh, Hq, Hkv = cfg.P, cfg.dh, cfg.Hq, cfg.Hkv
+    K_out = np.zeros((cfg.L, len(samples), P, Hkv, dh))
+    V_out = np.zeros_like(K_out)
+    for si, b in enumerate(samples):
+        h = rnd(np.asarray(emb[b], np.float64))         # the caller hands bf16 embeddings
+        for l, lay in enumerate(model.layers):
+            a = rms_norm(h, lay["g1"], cfg.eps)
+            q, k, v = _project(model, l, "qkv", a, (lay["wq"], lay["wk"], lay["wv"]), None, None)
+            q = rnd(rope_rotate(q.reshape(P, Hq, dh).transpose(1, 0, 2), model.cos, model.sin))
+            k = rnd(rope_rotate(k.reshape(P, Hkv, dh).transpose(1, 0, 2), model.cos, model.sin))
+            v = rnd(v.reshape(P, Hkv, dh).transpose(1, 0, 2))
+            K_out[l, si] = k.transpose(1, 0, 2)
+            V_out[l, si] = v.transpose(1, 0, 2)
+            if l == cfg.L - 1:
+                break
+            o = attention(q, k, v).transpose(1, 0, 2).reshape(P, Hq * dh)
+            (dh_o,) = _project(model, l, "o", o, (lay["wo"],), None, None)
+            h = h + dh_o
+            a = rms_norm(h, lay["g2"], cfg.eps)
+            g, u = _project(model, l, "gu", a, (lay["wg"], lay["wu"]), None, None)
+            (dh_d,) = _project(model, l, "down", gelu_tanh(g) * u, (lay["wd"],), None, None)
+            h = h + dh_d
+    return K_out, V_out

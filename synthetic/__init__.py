@@ -30,7 +30,8 @@ from typing import Dict, List
 
 import numpy as np
 
-__all__ = ["ActionExpertConfig", "CONFIGS", "make_inputs", "make_modulation", "make_noise", "make_prefix"]
+__all__ = ["ActionExpertConfig", "CONFIGS", "PREFIX_CONFIGS", "PrefixConfig", "make_inputs", "make_modulation",
+           "make_noise", "make_prefix", "make_prefix_pass_inputs"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -190,3 +191,69 @@ def zero_weights(cfg: ActionExpertConfig) -> dict:
     for k in ("w_in", "w_out", "w_t1", "w_t2", "b_in", "b_out", "b_t1", "b_t2"):
         w[k][...] = 0.0
     return w
+
+
+# --------------------------------------------------------------------------------------
+# The prefix pass: the vision-language backbone run once over the observation's tokens to
+# produce the per-layer keys and values the action expert attends to.
+# --------------------------------------------------------------------------------------
+
+@dataclasses.dataclass(frozen=True)
+class PrefixConfig:
+    """Sizes of one prefix-pass workload: an L-layer transformer of the action expert's block
+    (RMSNorm, fused QKV with RoPE, grouped-query attention, gated-GeLU MLP) over P prefix tokens
+    per sample with full attention among them; its KV shape (L, Hkv, dh) matches the expert's."""
+
+    name: str
+    L: int
+    D: int
+    Hq: int
+    Hkv: int
+    dh: int
+    F: int
+    B: int
+    P: int          # prefix tokens per sample
+    dtype: str
+    rope_theta: float = 10000.0
+    eps: float = 1e-6
+
+    @property
+    def n_qkv(self) -> int:
+        return (self.Hq + 2 * self.Hkv) * self.dh
+
+    def replace(self, **kw) -> "PrefixConfig":
+        return dataclasses.replace(self, **kw)
+
+
+PREFIX_CONFIGS: Dict[str, PrefixConfig] = {
+    # the 2B-parameter backbone of a pi0.5-style policy (width 2048, 18 layers, 8 query heads
+    # sharing one 256-wide KV head, MLP 16384) over the 816-token three-view observation
+    "vlm_bf16_p816": PrefixConfig("vlm_bf16_p816", L=18, D=2048, Hq=8, Hkv=1, dh=256, F=16384, B=1, P=816,
+                                  dtype="bf16"),
+}
+
+
+def make_prefix_pass_inputs(cfg: PrefixConfig, seed: int = 0) -> dict:
+    """Weights and token embeddings of one prefix-pass workload.
+
+    Draw order (PCG64 ``default_rng(seed)``, standard normal drawn in float32 to keep the
+    2B-parameter case affordable, scaled by 1/sqrt(fan_in) in float32): for each layer W_q, W_k,
+    W_v, W_o, W_gate, W_up, W_down; then the embedded prefix tokens [B][P][D] ~ N(0, 1) (the
+    vision encoder's and the text embedding's outputs, synthetic).  Gains are ones."""
+    rng = np.random.default_rng(seed)
+    D, F, dh = cfg.D, cfg.F, cfg.dh
+
+    def w(shape, fan_in):
+        a = rng.standard_normal(size=shape, dtype=np.float32)
+        a *= np.float32(1.0 / np.sqrt(float(fan_in)))
+        return a
+
+    layers = []
+    for _ in range(cfg.L):
+        layers.append({
+            "wq": w((cfg.Hq * dh, D), D), "wk": w((cfg.Hkv * dh, D), D), "wv": w((cfg.Hkv * dh, D), D),
+            "wo": w((D, cfg.Hq * dh), cfg.Hq * dh), "wg": w((F, D), D), "wu": w((F, D), D), "wd": w((D, F), F),
+            "g1": np.ones(D, np.float32), "g2": np.ones(D, np.float32),
+        })
+    emb = rng.standard_normal(size=(cfg.B, cfg.P, D), dtype=np.float32)
+    return {"weights": {"layers": layers}, "emb": emb}
