@@ -25,12 +25,12 @@ from ._abi import (  # noqa: F401
     fr_get_scales, fr_graph_count, fr_last_error, fr_launches_per_call, fr_load_weights, fr_path_name,
     fr_quantize_e4m3, fr_quantize_w4, fr_read_kv, fr_refresh_prefix_kv, fr_rope_tables, fr_round_bf16,
     fr_set_graph_capacity, fr_set_prefix_kv, fr_set_scales, fr_sync_status, header_functions, load_library,
-    make_config,
+    make_config, make_prefix_config, fr_prefill, FR_ROLE_EXPERT, FR_ROLE_PREFIX,
 )
 
 load_library()
 
-__all__ = ["ActionExpertLoop", "FrError", "load_library", "make_config"]
+__all__ = ["ActionExpertLoop", "FrError", "PrefixPass", "load_library", "make_config"]
 
 
 class ActionExpertLoop:
@@ -160,6 +160,58 @@ class ActionExpertLoop:
 
     def rope_tables(self, n_pos: int):
         return fr_get_rope_tables(self.h, n_pos, self.cfg.dh)
+
+    def close(self) -> None:
+        if self.h:
+            fr_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class PrefixPass:
+    """One prefix-pass (backbone) handle: the step before the loop, producing the expert's prefix KV."""
+
+    def __init__(self, cfg, device: int = 0, B_max: Optional[int] = None, P_max: Optional[int] = None):
+        import torch
+        self._torch = torch
+        self.cfg = cfg
+        self.device = device
+        self.h = fr_create(make_prefix_config(cfg, B_max, P_max), device)
+
+    def _stream(self) -> int:
+        return self._torch.cuda.current_stream(self.device).cuda_stream
+
+    def load_weights(self, weights: dict) -> None:
+        """weights: {'layers': [...]} with the layer tensors of the backbone (host float32)."""
+        fr_load_weights(self.h, weights, self._stream())
+
+    def run(self, emb, expert: Optional["ActionExpertLoop"] = None) -> None:
+        """emb: bf16 CUDA tensor [B][P][D].  Fills this handle's KV cache and, if given, the expert's prefix."""
+        torch = self._torch
+        if not isinstance(emb, torch.Tensor) or emb.device.type != "cuda" or emb.dtype != torch.bfloat16 \
+                or not emb.is_contiguous() or emb.dim() != 3 or emb.shape[2] != self.cfg.D:
+            raise FrError(FR_ERR_ARG, "fr_prefill", "expected a contiguous bf16 CUDA tensor [B][P][D]")
+        B, P = emb.shape[0], emb.shape[1]
+        fr_prefill(self.h, emb.data_ptr(), B, P, expert.h if expert is not None else None, self._stream())
+        if expert is not None:
+            expert._P = P
+
+    def buffer(self, name: str):
+        return fr_get_buffer(self.h, name)
+
+    def read_kv(self, layer: int, b: int, n_slots: int):
+        return fr_read_kv(self.h, layer, b, n_slots, self.cfg.Hkv, self.cfg.dh, True)
+
+    def sync_status(self) -> int:
+        return fr_sync_status(self.h, self._stream())
+
+    def launches_per_call(self) -> int:
+        return fr_launches_per_call(self.h, 1)
 
     def close(self) -> None:
         if self.h:

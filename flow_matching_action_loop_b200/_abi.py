@@ -23,6 +23,7 @@ FR_DTYPE_F32, FR_DTYPE_BF16, FR_DTYPE_FP8, FR_DTYPE_W4A16 = 0, 1, 2, 3
 FR_W4_GROUP = 128
 FR_PATH_AUTO, FR_PATH_STEPWISE, FR_PATH_TENSOR = 0, 1, 2
 FR_PREFIX_K_ROTATED = 1
+FR_ROLE_EXPERT, FR_ROLE_PREFIX = 0, 1
 DTYPES = {"f32": FR_DTYPE_F32, "bf16": FR_DTYPE_BF16, "fp8": FR_DTYPE_FP8, "w4a16": FR_DTYPE_W4A16}
 ERR_NAMES = {FR_ERR_ARG: "FR_ERR_ARG", FR_ERR_SHAPE: "FR_ERR_SHAPE", FR_ERR_STATE: "FR_ERR_STATE",
              FR_ERR_CUDA: "FR_ERR_CUDA", FR_ERR_TIMEOUT: "FR_ERR_TIMEOUT", FR_ERR_DEVICE: "FR_ERR_DEVICE",
@@ -41,7 +42,7 @@ class FrConfig(ctypes.Structure):
                 ("B_max", ctypes.c_int), ("P_max", ctypes.c_int), ("K", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("path", ctypes.c_int), ("rope_theta", ctypes.c_float),
                 ("eps", ctypes.c_float), ("time_dim", ctypes.c_int), ("time_base", ctypes.c_float),
-                ("adarms", ctypes.c_int)]
+                ("adarms", ctypes.c_int), ("role", ctypes.c_int)]
 
 
 _FP = ctypes.POINTER(ctypes.c_float)
@@ -109,6 +110,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fr_attention_scratch_bytes": (ctypes.c_size_t, [c_int, c_int, c_int, c_int, c_int]),
         "fr_attention_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
                                          c_int, c_void_p]),
+        "fr_prefill": (c_int, [H, c_void_p, c_int, c_int, H, c_void_p]),
         "fr_refresh_prefix_kv": (c_int, [H, c_void_p, c_void_p, ctypes.POINTER(c_int), c_int, c_int, c_uint,
                                          c_void_p]),
         "fr_get_buffer": (c_int, [H, c_char_p, ctypes.POINTER(c_void_p), ctypes.POINTER(ctypes.c_size_t)]),
@@ -152,6 +154,16 @@ def make_config(cfg, B_max: Optional[int] = None, P_max: Optional[int] = None, p
                     B_max=B_max or cfg.B, P_max=P_max or cfg.P, K=cfg.K, dtype=dtype, path=path,
                     rope_theta=cfg.rope_theta, eps=cfg.eps, time_dim=cfg.time_dim, time_base=cfg.time_base,
                     adarms=1 if getattr(cfg, "adarms", False) else 0)
+
+
+def make_prefix_config(cfg, B_max: Optional[int] = None, P_max: Optional[int] = None) -> FrConfig:
+    """fr_config of a prefix-pass (backbone) handle from a PrefixConfig-like object: H is the
+    largest number of prefix tokens per sample; the loop-only fields get neutral values."""
+    dtype = cfg.dtype if isinstance(cfg.dtype, int) else DTYPES[cfg.dtype]
+    return FrConfig(L=cfg.L, D=cfg.D, Hq=cfg.Hq, Hkv=cfg.Hkv, dh=cfg.dh, F=cfg.F, H=P_max or cfg.P, A=1,
+                    B_max=B_max or cfg.B, P_max=1, K=1, dtype=dtype, path=FR_PATH_TENSOR,
+                    rope_theta=cfg.rope_theta, eps=cfg.eps, time_dim=2, time_base=10000.0, adarms=0,
+                    role=FR_ROLE_PREFIX)
 
 
 # ------------------------------------------------------------------ same-name wrappers
@@ -245,6 +257,10 @@ def fr_launches_per_call(h, B: int) -> int:
 def _ints(values):
     a = (ctypes.c_int * len(values))(*[int(v) for v in values])
     return a
+
+
+def fr_prefill(h, emb_dev: int, B: int, P: int, expert=None, stream: int = 0) -> None:
+    _check(load_library().fr_prefill(h, emb_dev, B, P, expert, stream), "fr_prefill")
 
 
 def fr_refresh_prefix_kv(h, k_dev: int, v_dev: int, slots, P: int, flags: int = 0, stream: int = 0) -> None:

@@ -119,6 +119,15 @@ int validate(const fr_config& c) {
     set_error("fr_create: the tensor-core path needs a bf16, fp8 or w4a16 handle");
     return FR_ERR_UNSUPPORTED;
   }
+  if (c.role != FR_ROLE_EXPERT && c.role != FR_ROLE_PREFIX) {
+    set_error("fr_create: bad role enum");
+    return FR_ERR_ARG;
+  }
+  if (c.role == FR_ROLE_PREFIX &&
+      ((c.dtype != FR_DTYPE_BF16 && c.dtype != FR_DTYPE_W4A16) || c.path == FR_PATH_STEPWISE || c.adarms)) {
+    set_error("fr_create: the prefix pass runs bf16 or w4a16 on the tensor-core path, without adarms");
+    return FR_ERR_UNSUPPORTED;
+  }
   return FR_OK;
 }
 
@@ -263,7 +272,7 @@ int fr_create(const fr_config* cfg, int device, fr_handle** out) {
   h->path = c.path;
   if (h->path == FR_PATH_AUTO) h->path = (c.dtype == FR_DTYPE_F32) ? FR_PATH_STEPWISE : FR_PATH_TENSOR;
   if (h->path == FR_PATH_TENSOR && !tensor_path_supports(c)) {
-    if (c.path == FR_PATH_TENSOR) {
+    if (c.path == FR_PATH_TENSOR || c.role == FR_ROLE_PREFIX) {
       set_error("fr_create: sizes outside the tensor-core path (%s)", tensor_path_limits());
       delete h;
       return FR_ERR_UNSUPPORTED;
@@ -458,14 +467,19 @@ int prepare_adarms(fr_handle* h, const fr_weights& w, bool rb, cudaStream_t s) {
 }
 
 int fr_load_weights(fr_handle* h, const fr_weights* w_in, fr_stream_t stream) {
-  if (!h || !w_in || !w_in->layers || !w_in->w_in || !w_in->b_in || !w_in->w_out || !w_in->b_out ||
-      !w_in->w_t1 || !w_in->b_t1 || !w_in->w_t2 || !w_in->b_t2) {
+  if (!h || !w_in || !w_in->layers) {
     set_error("fr_load_weights: NULL argument");
     return FR_ERR_ARG;
   }
   const fr_config& c = h->cfg;
+  if (c.role != FR_ROLE_PREFIX && (!w_in->w_in || !w_in->b_in || !w_in->w_out || !w_in->b_out || !w_in->w_t1 ||
+                                   !w_in->b_t1 || !w_in->w_t2 || !w_in->b_t2)) {
+    set_error("fr_load_weights: NULL argument");
+    return FR_ERR_ARG;
+  }
   const bool ada = c.adarms != 0;
-  if (ada ? (!w_in->w_modf || !w_in->b_modf) : !w_in->g_f) {
+  const bool pre = c.role == FR_ROLE_PREFIX;   // the backbone: only the layer tensors are read
+  if (!pre && (ada ? (!w_in->w_modf || !w_in->b_modf) : !w_in->g_f)) {
     set_error(ada ? "fr_load_weights: adarms handle without w_modf / b_modf" : "fr_load_weights: NULL g_f");
     return FR_ERR_ARG;
   }
@@ -543,19 +557,21 @@ int fr_load_weights(fr_handle* h, const fr_weights* w_in, fr_stream_t stream) {
     return FR_OK;
   };
   int rc = FR_OK;
-  if ((rc = up(h->w_in, w->w_in, D * c.A, rb))) return rc;
-  if ((rc = up(h->b_in, w->b_in, D, false))) return rc;
-  if ((rc = up(h->w_out, w->w_out, c.A * D, rb))) return rc;
-  if ((rc = up(h->b_out, w->b_out, c.A, false))) return rc;
-  if ((rc = up(h->w_t1, w->w_t1, D * c.time_dim, rb))) return rc;
-  if ((rc = up(h->b_t1, w->b_t1, D, false))) return rc;
-  if ((rc = up(h->w_t2, w->w_t2, D * D, rb))) return rc;
-  if ((rc = up(h->b_t2, w->b_t2, D, false))) return rc;
-  if ((rc = up(h->g_f, w->g_f, D, false))) return rc;
   FR_CUDA(cudaMemcpy(h->s_w, h->h_sw.data(), h->h_sw.size() * 4, cudaMemcpyHostToDevice));
-  launch_temb(h->w_t1, h->b_t1, h->w_t2, h->b_t2, h->temb, c.D, c.time_dim, c.K, c.time_base, rb, s);
-  if ((rc = check_launch("time MLP kernel"))) return rc;
-  if (ada && (rc = prepare_adarms(h, *w, rb, s))) return rc;
+  if (!pre) {   // in/out-proj, time MLP and final norm of the expert
+    if ((rc = up(h->w_in, w->w_in, D * c.A, rb))) return rc;
+    if ((rc = up(h->b_in, w->b_in, D, false))) return rc;
+    if ((rc = up(h->w_out, w->w_out, c.A * D, rb))) return rc;
+    if ((rc = up(h->b_out, w->b_out, c.A, false))) return rc;
+    if ((rc = up(h->w_t1, w->w_t1, D * c.time_dim, rb))) return rc;
+    if ((rc = up(h->b_t1, w->b_t1, D, false))) return rc;
+    if ((rc = up(h->w_t2, w->w_t2, D * D, rb))) return rc;
+    if ((rc = up(h->b_t2, w->b_t2, D, false))) return rc;
+    if ((rc = up(h->g_f, w->g_f, D, false))) return rc;
+    launch_temb(h->w_t1, h->b_t1, h->w_t2, h->b_t2, h->temb, c.D, c.time_dim, c.K, c.time_base, rb, s);
+    if ((rc = check_launch("time MLP kernel"))) return rc;
+    if (ada && (rc = prepare_adarms(h, *w, rb, s))) return rc;
+  }
   FR_CUDA(cudaStreamSynchronize(s));
   if (h->tp) {
     rc = tensor_path_finish_load(h->tp, s);
@@ -580,6 +596,10 @@ int fr_set_prefix_kv(fr_handle* h, const void* k_dev, const void* v_dev, int B, 
   if (flags & ~FR_PREFIX_K_ROTATED) {
     set_error("fr_set_prefix_kv: unknown flag bits 0x%x", flags);
     return FR_ERR_ARG;
+  }
+  if (c.role != FR_ROLE_EXPERT) {
+    set_error("fr_set_prefix_kv: a prefix-pass handle writes its KV with fr_prefill");
+    return FR_ERR_STATE;
   }
   FR_CUDA(cudaSetDevice(h->device));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -804,6 +824,10 @@ int fr_capsule_restore(fr_handle* h, const void* cap_dev, const fr_capsule* desc
     return FR_ERR_ARG;
   }
   const fr_config& c = h->cfg;
+  if (c.role != FR_ROLE_EXPERT) {
+    set_error("fr_capsule_restore: not an expert handle");
+    return FR_ERR_STATE;
+  }
   if (desc->magic != FR_CAPSULE_MAGIC || desc->B < 1 || desc->P < 1) {
     set_error("fr_capsule_restore: not a capsule description (magic 0x%x, B=%d, P=%d)", desc->magic, desc->B,
               desc->P);
@@ -867,12 +891,84 @@ int fr_graph_count(const fr_handle* h) {
   return h->tp ? tensor_path_graph_count(h->tp) : 0;
 }
 
+int fr_prefill(fr_handle* bb, const void* emb_dev, int B, int P, fr_handle* ex, fr_stream_t stream) {
+  if (!bb || !emb_dev) {
+    set_error("fr_prefill: NULL argument");
+    return FR_ERR_ARG;
+  }
+  const fr_config& c = bb->cfg;
+  if (c.role != FR_ROLE_PREFIX || !bb->tp) {
+    set_error("fr_prefill: not a prefix-pass handle (create it with role FR_ROLE_PREFIX)");
+    return FR_ERR_STATE;
+  }
+  if (!bb->weights_loaded) {
+    set_error("fr_prefill: no weights loaded");
+    return FR_ERR_STATE;
+  }
+  if (B < 1 || B > c.B_max || P < 1 || P > c.H) {
+    set_error("fr_prefill: need 1 <= B <= %d and 1 <= P <= %d (got B=%d P=%d)", c.B_max, c.H, B, P);
+    return FR_ERR_SHAPE;
+  }
+  if (ex) {
+    const fr_config& e = ex->cfg;
+    if (e.role != FR_ROLE_EXPERT) {
+      set_error("fr_prefill: the destination is not an expert handle");
+      return FR_ERR_STATE;
+    }
+    if (e.L != c.L || e.Hkv != c.Hkv || e.dh != c.dh || !ex->kv_bf || B > e.B_max || P > e.P_max) {
+      set_error("fr_prefill: expert KV [L=%d Hkv=%d dh=%d, B_max=%d P_max=%d, %s] cannot take the pass's "
+                "[L=%d Hkv=%d dh=%d] for B=%d P=%d",
+                e.L, e.Hkv, e.dh, e.B_max, e.P_max, ex->kv_bf ? "bf16" : "f32", c.L, c.Hkv, c.dh, B, P);
+      return FR_ERR_SHAPE;
+    }
+  }
+  FR_CUDA(cudaSetDevice(bb->device));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int rc = tensor_path_prefill(bb->tp, emb_dev, B, P, s);
+  if (rc) return rc;
+  if ((rc = check_launch("prefix pass"))) return rc;
+  if (ex) {   // rows 0..P-1 of slots 0..B-1, every layer and KV head, into the expert's cache
+    const long long rowb = static_cast<long long>(c.dh) * 2;
+    for (int b0 = 0; b0 < B; b0 += SLOT_MAP_MAX) {
+      RowCopy rcp{};
+      rcp.parts = 2;
+      rcp.n_outer = c.L;
+      rcp.n_sample = std::min(SLOT_MAP_MAX, B - b0);
+      rcp.n_mid = c.Hkv;
+      rcp.n_row = P;
+      rcp.s_outer = static_cast<long long>(bb->kv_layer_bytes);
+      rcp.s_sample = c.Hkv * bb->S_max * rowb;
+      rcp.s_mid = bb->S_max * rowb;
+      rcp.s_row = rowb;
+      rcp.d_outer = static_cast<long long>(ex->kv_layer_bytes);
+      rcp.d_sample = ex->cfg.Hkv * ex->S_max * rowb;
+      rcp.d_mid = ex->S_max * rowb;
+      rcp.d_row = rowb;
+      rcp.src[0] = bb->kv_k;
+      rcp.src[1] = bb->kv_v;
+      rcp.dst[0] = ex->kv_k + b0 * rcp.d_sample;
+      rcp.dst[1] = ex->kv_v + b0 * rcp.d_sample;
+      rcp.row_bytes = rowb;
+      for (int i = 0; i < rcp.n_sample; ++i) rcp.map[i] = b0 + i;
+      launch_state_copy(rcp, s);
+      if ((rc = check_launch("state copy kernel"))) return rc;
+    }
+    ex->prefix_B = B;
+    ex->prefix_P = P;
+  }
+  return FR_OK;
+}
+
 int fr_denoise(fr_handle* h, const float* x0_dev, float* x_out_dev, int B, fr_stream_t stream) {
   if (!h || !x0_dev || !x_out_dev) {
     set_error("fr_denoise: NULL argument");
     return FR_ERR_ARG;
   }
   const fr_config& c = h->cfg;
+  if (c.role != FR_ROLE_EXPERT) {
+    set_error("fr_denoise: a prefix-pass handle runs fr_prefill, not the loop");
+    return FR_ERR_STATE;
+  }
   if (B < 1 || B > c.B_max) {
     set_error("fr_denoise: need 1 <= B <= %d (got %d)", c.B_max, B);
     return FR_ERR_SHAPE;

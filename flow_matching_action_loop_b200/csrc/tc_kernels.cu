@@ -156,15 +156,18 @@ __host__ __device__ __forceinline__ GemmGeom gemm_geom(int Nt, int stages, int b
   return g;
 }
 
+// RoPE (cos, sin) rows the QKV epilogue stages: one per action position when the H positions are
+// fewer than the tile's tokens, else one per token of the tile (long sequences, e.g. the prefix pass).
+__host__ __device__ __forceinline__ bool rope_by_token(int H, int Nt) { return H > Nt; }
+
 // Bytes of the epilogue stage that follows the main-loop and exchange regions: the QKV epilogue's
 // RoPE (cos, sin) pairs.  (Staging the other epilogues' outputs for bulk stores was measured slower
 // than direct stores: the kernel would have to wait for its stores before exiting.)
 __host__ __device__ __forceinline__ uint32_t gemm_stage_bytes(int epi, int fp8, int Nt, int S, int H, int xb) {
   (void)fp8;
-  (void)Nt;
   (void)S;
   (void)xb;
-  return epi == EPI_QKV ? static_cast<uint32_t>(H) * 64u * 8u : 0u;
+  return epi == EPI_QKV ? static_cast<uint32_t>(rope_by_token(H, Nt) ? Nt : H) * 64u * 8u : 0u;
 }
 
 // Largest chunk count of any split-K rank: the shared-memory layout is the same in every CTA.
@@ -243,9 +246,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   float2* rope_sh = reinterpret_cast<float2*>(dsm + gemm_rope_off(Nt, stages, NORM ? B_NORM : B_ROWS, FP8, S, nk_max_of(a), W4, EPI));
   if (EPI == EPI_QKV && mb < a.MB_rot && warp >= 2) {   // warps 2-7: the producer and MMA warps go on
     const int half = a.dh >> 1;
-    for (int idx = tid - 64; idx < a.H * 64; idx += GEMM_THREADS - 64) {
+    const bool by_tok = rope_by_token(a.H, Nt);
+    for (int idx = tid - 64; idx < (by_tok ? Nt : a.H) * 64; idx += GEMM_THREADS - 64) {
       const int i = idx >> 6, p = idx & 63;
-      const int j = (mb * 64 + p) % half, pos = a.P + i;
+      const int j = (mb * 64 + p) % half, pos = a.P + (by_tok ? (n0 + i) % a.H : i);
       rope_sh[idx] = make_float2(a.rope_cos[pos * half + j], a.rope_sin[pos * half + j]);
     }
   }
@@ -651,7 +655,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         for (int u = 0; u < EPU; ++u) {
           const int tok = tb + 8 * u, t = n0 + tok;
           if (tok < tok1 && t < a.T) {
-            const float4 r4 = *reinterpret_cast<const float4*>(rope_sh + (t % a.H) * 64 + p);   // pairs p, p+1
+            const float4 r4 = *reinterpret_cast<const float4*>(rope_sh + (rope_by_token(a.H, Nt) ? tok : t % a.H) * 64 + p);   // pairs p, p+1
             cs[u] = make_float2(r4.x, r4.z);
             sn[u] = make_float2(r4.y, r4.w);
           }
@@ -1462,11 +1466,14 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
   __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(dsm);   // [A][D]: consecutive threads read consecutive n
   const int tid = threadIdx.x;
   const uint32_t wbytes = static_cast<uint32_t>(a.D) * a.A * 2;
+  const bool emb = a.emb != nullptr;   // prefix pass: h is the embedded token itself
   if (tid == 0) {
     mbar_init(&wbar, 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(&wbar, wbytes);
-    bulk_g2s(wsm, a.w_in, wbytes, &wbar);   // static weights: before the dependency wait
+    if (!emb) {
+      mbar_arrive_expect_tx(&wbar, wbytes);
+      bulk_g2s(wsm, a.w_in, wbytes, &wbar);   // static weights: before the dependency wait
+    }
   }
   grid_dep_launch();
   constexpr int QMAX = 16;                 // D <= 4096
@@ -1474,14 +1481,14 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
 #pragma unroll
   for (int q = 0; q < QMAX; ++q) {
     const int n = tid + q * 256;
-    base[q] = n < a.D ? a.b_in[n] + (a.temb ? a.temb[n] : 0.f) : 0.f;   // no temb: adaptive RMSNorm
+    base[q] = (n < a.D && !emb) ? a.b_in[n] + (a.temb ? a.temb[n] : 0.f) : 0.f;   // no temb: adaptive RMSNorm
   }
   grid_dep_wait();
   if (tid == 0) TL(1);
-  mbar_wait(&wbar, 0, WAIT_LIMIT_NS);
+  if (!emb) mbar_wait(&wbar, 0, WAIT_LIMIT_NS);
   const int warp = tid >> 5, lane = tid & 31;
   for (int t = blockIdx.x; t < a.T; t += gridDim.x) {   // the weights are staged once per CTA
-  if (tid < a.A) xs[tid] = __bfloat162float(__float2bfloat16_rn(a.x[static_cast<size_t>(t) * a.A + tid]));
+  if (!emb && tid < a.A) xs[tid] = __bfloat162float(__float2bfloat16_rn(a.x[static_cast<size_t>(t) * a.A + tid]));
   __syncthreads();
 #pragma unroll
   for (int q = 0; q < QMAX; ++q) {
@@ -1489,9 +1496,13 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
     if (q * 256 >= a.D) continue;   // uniform across the block
     float hv = 0.f;
     if (n < a.D) {
-      float acc = 0.f;
-      for (int i = 0; i < a.A; ++i) acc = fmaf(__bfloat162float(wsm[static_cast<size_t>(i) * a.D + n]), xs[i], acc);
-      hv = acc + base[q];
+      if (emb) {
+        hv = __bfloat162float(a.emb[static_cast<size_t>(t) * a.D + n]);
+      } else {
+        float acc = 0.f;
+        for (int i = 0; i < a.A; ++i) acc = fmaf(__bfloat162float(wsm[static_cast<size_t>(i) * a.D + n]), xs[i], acc);
+        hv = acc + base[q];
+      }
       a.h[htile_offset(t, n, a.Nt, a.KB)] = hv;
       if (a.xb)
         *reinterpret_cast<__nv_bfloat16*>(a.xb + btile_offset(t, 2 * n, a.Nt, a.NKC_x)) =

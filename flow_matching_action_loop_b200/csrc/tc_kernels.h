@@ -141,10 +141,10 @@ inline int attn_tiles(int B, int Hq, int Hkv, int H) { return B * Hkv * ((Hq / H
 // the warp-MMA kernel runs, one CTA per (key chunk, query head), with attn_chunks' split;
 // otherwise the tcgen05 kernel runs with enough chunks to give every SM a CTA.  Either way
 // C <= attn_chunks' C, so the scratch bound holds.  Returns 1 for the tcgen05 kernel.
-inline int attn_plan(int S, int tiles, int nsm, int& C, int& KC) {
+inline int attn_plan(int S, int tiles, int nsm, int& C, int& KC, bool force_umma = false) {
   int cmax = 1, kc = 64;
   attn_chunks(S, cmax, kc);
-  if (tiles * cmax < nsm) {
+  if (tiles * cmax < nsm && !force_umma) {
     C = cmax;
     KC = kc;
     return 0;
@@ -162,7 +162,8 @@ struct InprojArgs {
   const float* x;              // [T][A] state at the start of the step
   const __nv_bfloat16* w_in;   // [A][D] (transposed by the loader)
   const float* b_in;
-  const float* temb;           // [D] of this step
+  const float* temb;           // [D] of this step, or nullptr
+  const __nv_bfloat16* emb;    // prefix pass: h = emb [T][D] (no in-proj, no time), or nullptr
   float* h;                    // tiled h
   float* ssq;                  // [T_pad][ssq_ld]
   uint8_t* xb;                 // bf16(h * gamma1 of layer 0), tiled operand layout, or nullptr

@@ -58,7 +58,7 @@ struct GemmPlan {
 };
 
 struct StepPlan {
-  int B = 0, P = 0, T = 0, NT = 0, Nt = 0;
+  int B = 0, P = 0, H = 0, T = 0, NT = 0, Nt = 0;   // H: query tokens per sample (action rows or prefix tokens)
   GemmPlan qkv, o, gu, dn;
   int attn_C = 1, attn_KC = 64, attn_umma = 0;
 };
@@ -110,6 +110,7 @@ struct TensorPath {
   float* xs = nullptr;           // [T_max][A] state between steps
   __nv_bfloat16* w_in_bf = nullptr;   // [A][D]
   __nv_bfloat16* w_out_bf = nullptr;  // [A][D]
+  __nv_bfloat16* emb = nullptr;       // prefix pass: the embedded tokens of the call [B_max][H][D]
   cudaStream_t cap = nullptr;
   std::map<std::pair<int, int>, GraphEntry> graphs;   // graph-variant table keyed by (B, P)
   size_t graph_capacity = 8;
@@ -154,6 +155,7 @@ size_t carve_all(TensorPath* tp, char* base) {
   tp->xscratch = cv.take<float>(tp->xscratch_bytes / sizeof(float) + 64);
   tp->w_in_bf = cv.take<__nv_bfloat16>(static_cast<size_t>(c.D) * c.A);
   tp->w_out_bf = cv.take<__nv_bfloat16>(static_cast<size_t>(c.A) * c.D);
+  tp->emb = cv.take<__nv_bfloat16>(c.role == FR_ROLE_PREFIX ? static_cast<size_t>(tp->T_max) * c.D : 0);
   return align_up(cv.off, 1024);
 }
 
@@ -216,26 +218,32 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, in
   return best;
 }
 
-StepPlan make_plan(const TensorPath* tp, int B, int P) {
+// Plan of one call: B samples of H query tokens (the action rows, or the prefix pass's tokens)
+// attending to P cached keys plus themselves.
+StepPlan make_plan(const TensorPath* tp, int B, int P, int H) {
   const fr_config& c = tp->c;
   StepPlan p;
   p.B = B;
   p.P = P;
-  p.T = B * c.H;
+  p.H = H;
+  p.T = B * H;
   p.NT = ceil_div(p.T, NT_MAX);
   p.Nt = static_cast<int>(align_up(ceil_div(p.T, p.NT), 16));
   const int norm_kind = tp->fp8 ? B_NORM : B_ROWS;   // bf16: the producer wrote bf16(h*gamma) already
-  p.qkv = choose_plan(tp->qkv.MB * p.NT, tp->qkv.NKC, p.Nt, norm_kind, tp->fp8, tp->w4, EPI_QKV, c.H, 0, tp->nsm,
+  p.qkv = choose_plan(tp->qkv.MB * p.NT, tp->qkv.NKC, p.Nt, norm_kind, tp->fp8, tp->w4, EPI_QKV, H, 0, tp->nsm,
                       tp->max_dyn);
-  p.o = choose_plan(tp->o.MB * p.NT, tp->o.NKC, p.Nt, B_ROWS, tp->fp8, tp->w4, EPI_RESID, c.H, !tp->fp8, tp->nsm,
+  p.o = choose_plan(tp->o.MB * p.NT, tp->o.NKC, p.Nt, B_ROWS, tp->fp8, tp->w4, EPI_RESID, H, !tp->fp8, tp->nsm,
                     tp->max_dyn);
-  p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, norm_kind, tp->fp8, tp->w4, EPI_GELU, c.H, 0, tp->nsm,
+  p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, norm_kind, tp->fp8, tp->w4, EPI_GELU, H, 0, tp->nsm,
                      tp->max_dyn);
-  p.dn = choose_plan(tp->dn.MB * p.NT, tp->dn.NKC, p.Nt, B_ROWS, tp->fp8, tp->w4, EPI_RESID, c.H, !tp->fp8, tp->nsm,
+  p.dn = choose_plan(tp->dn.MB * p.NT, tp->dn.NKC, p.Nt, B_ROWS, tp->fp8, tp->w4, EPI_RESID, H, !tp->fp8, tp->nsm,
                      tp->max_dyn);
-  p.attn_umma = attn_plan(P + c.H, attn_tiles(B, c.Hq, c.Hkv, c.H), tp->nsm, p.attn_C, p.attn_KC);
+  // the warp-MMA attention kernel holds at most 128 query rows per head: longer sequences take tcgen05
+  p.attn_umma = attn_plan(P + H, attn_tiles(B, c.Hq, c.Hkv, H), tp->nsm, p.attn_C, p.attn_KC, H > 128);
   return p;
 }
+
+StepPlan make_plan(const TensorPath* tp, int B, int P) { return make_plan(tp, B, P, tp->c.H); }
 
 // Pre-tile rows of one projection: rowsrc(r) gives the float32 row r (length K) or nullptr (zero row).
 template <typename RowFn>
@@ -307,12 +315,159 @@ GemmArgs base_args(const TensorPath* tp, const StepPlan& p, const ProjLayout& L,
   return a;
 }
 
+// Per-layer vectors of one recorded layer: the two norms' gains, the gain of the next layer's first
+// norm (nullptr after the last layer), and the adaptive-RMSNorm gates and folded shifts (nullptr
+// without it).
+struct LayerVectors {
+  const float *g1, *g2, *g1_next;
+  const float *gate1, *gate2, *bias_qkv, *bias_gu;
+};
+
+// One layer: QKV GEMM (+RoPE, K/V into the cache), attention, O GEMM + residual, gate|up GEMM,
+// down GEMM + residual.  qkv_only: stop after the QKV GEMM (the prefix pass's last layer, whose
+// keys and values are all that is needed).
+int record_layer(TensorPath* tp, const StepPlan& p, int l, const LayerVectors& v, bool qkv_only, cudaStream_t s) {
+  const fr_config& c = tp->c;
+  const size_t o_off = tp->qkv.bytes, gu_off = o_off + tp->o.bytes, dn_off = gu_off + tp->gu.bytes;
+  cudaError_t e;
+  const float* sa = tp->tb.s_a ? tp->tb.s_a + l * PI_COUNT : nullptr;
+  const float* al = tp->tb.alpha ? tp->tb.alpha + l * PI_COUNT : nullptr;
+  __nv_bfloat16* kvk = reinterpret_cast<__nv_bfloat16*>(tp->tb.kv_k + l * tp->tb.kv_layer_bytes);
+  __nv_bfloat16* kvv = reinterpret_cast<__nv_bfloat16*>(tp->tb.kv_v + l * tp->tb.kv_layer_bytes);
+  // QKV: RMSNorm fused into the B staging, split + RoPE fused into the epilogue
+  GemmArgs q = base_args(tp, p, tp->qkv, p.qkv, l, 0);
+  if (tp->fp8) {
+    q.b_kind = B_NORM;
+  } else {
+    q.b_kind = B_ROWS;
+    q.act = tp->xbuf;
+    q.rscale = 1;
+  }
+  q.h = tp->h;
+  q.gamma = v.g1;
+  q.ssq = tp->ssq_a;
+  q.s_a = tp->fp8 ? sa + PI_QKV : nullptr;
+  q.alpha = tp->fp8 ? al + PI_QKV : nullptr;
+  q.epi = EPI_QKV;
+  q.q_out = tp->qbuf;
+  q.kv_k = kvk;
+  q.kv_v = kvv;
+  q.rope_cos = tp->tb.rope_cos;
+  q.rope_sin = tp->tb.rope_sin;
+  q.H = p.H;
+  q.P = p.P;
+  q.S_max = c.P_max + c.H;
+  q.Hq = c.Hq;
+  q.Hkv = c.Hkv;
+  q.dh = c.dh;
+  q.MB_rot = tp->MB_rot;
+  q.bias = v.bias_qkv;
+  if ((e = launch_gemm_tc(q, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "qkv GEMM launch");
+  if (qkv_only) return FR_OK;
+  // attention over [cached keys; the tokens themselves]
+  AttnArgs at{};
+  at.q = tp->qbuf;
+  at.kv_k = kvk;
+  at.kv_v = kvv;
+  at.o = tp->obuf;
+  at.Nt = p.Nt;
+  at.NKC_o = tp->o.NKC;
+  at.s_a = tp->fp8 ? sa + PI_O : nullptr;
+  at.fp8 = tp->fp8;
+  at.H = p.H;
+  at.P = p.P;
+  at.S_max = c.P_max + c.H;
+  at.Hq = c.Hq;
+  at.Hkv = c.Hkv;
+  at.dh = c.dh;
+  at.C = p.attn_C;
+  at.KC = p.attn_KC;
+  at.scale = 1.0f / std::sqrt(static_cast<float>(c.dh));
+  at.xscratch = tp->xscratch;
+  at.status = tp->tb.status;
+  at.umma = p.attn_umma;
+  if ((e = launch_attention_tc(at, p.B, s, true)) != cudaSuccess) return cuda_fail(e, "attention launch");
+  // O projection + residual (+ sum of squares for the pre-MLP norm)
+  GemmArgs og = base_args(tp, p, tp->o, p.o, l, o_off);
+  og.b_kind = B_ROWS;
+  og.act = tp->obuf;
+  og.alpha = tp->fp8 ? al + PI_O : nullptr;
+  og.epi = EPI_RESID;
+  og.h_out = tp->h;
+  og.ssq_out = tp->ssq_b;
+  og.xb_out = tp->fp8 ? nullptr : tp->xbuf;
+  og.xb_gamma = v.g2;
+  og.NKC_x = tp->qkv.NKC;
+  og.gate = v.gate1;
+  if ((e = launch_gemm_tc(og, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "o GEMM launch");
+  // gate|up with RMSNorm fused, GeLU(gate)*up epilogue
+  GemmArgs gg = base_args(tp, p, tp->gu, p.gu, l, gu_off);
+  if (tp->fp8) {
+    gg.b_kind = B_NORM;
+  } else {
+    gg.b_kind = B_ROWS;
+    gg.act = tp->xbuf;
+    gg.rscale = 1;
+  }
+  gg.h = tp->h;
+  gg.gamma = v.g2;
+  gg.ssq = tp->ssq_b;
+  gg.s_a = tp->fp8 ? sa + PI_GU : nullptr;
+  gg.alpha = tp->fp8 ? al + PI_GU : nullptr;
+  gg.epi = EPI_GELU;
+  gg.u_out = tp->ubuf;
+  gg.NKC_u = tp->dn.NKC;
+  gg.s_a_out = tp->fp8 ? sa + PI_DOWN : nullptr;
+  gg.F = c.F;
+  gg.bias = v.bias_gu;
+  if ((e = launch_gemm_tc(gg, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "gate|up GEMM launch");
+  // down projection + residual (+ sum of squares for the next norm)
+  GemmArgs dg = base_args(tp, p, tp->dn, p.dn, l, dn_off);
+  dg.b_kind = B_ROWS;
+  dg.act = tp->ubuf;
+  dg.alpha = tp->fp8 ? al + PI_DOWN : nullptr;
+  dg.epi = EPI_RESID;
+  dg.h_out = tp->h;
+  dg.ssq_out = tp->ssq_a;
+  dg.xb_out = (tp->fp8 || !v.g1_next) ? nullptr : tp->xbuf;
+  dg.xb_gamma = v.g1_next;   // gamma1 of layer l+1
+  dg.NKC_x = tp->qkv.NKC;
+  dg.gate = v.gate2;
+  if ((e = launch_gemm_tc(dg, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "down GEMM launch");
+  return FR_OK;
+}
+
+// The first kernel of a call: h, its Σh² partials and bf16(h * gamma1) of layer 0, from the
+// in-projected actions plus the step's time embedding, or from the prefix pass's embeddings.
+InprojArgs inproj_args(const TensorPath* tp, const StepPlan& p, const float* x_in, const float* temb,
+                       const float* gamma1, bool first) {
+  const fr_config& c = tp->c;
+  InprojArgs ia{};
+  ia.max_ctas = 2 * tp->nsm;
+  ia.x = x_in;
+  ia.w_in = tp->w_in_bf;
+  ia.b_in = tp->tb.b_in;
+  ia.temb = temb;
+  ia.h = tp->h;
+  ia.ssq = tp->ssq_a;
+  ia.T = p.T;
+  ia.D = c.D;
+  ia.A = c.A;
+  ia.Nt = p.Nt;
+  ia.KB = tp->KB;
+  ia.ssq_ld = tp->ssq_ld;
+  ia.xb = tp->fp8 ? nullptr : tp->xbuf;
+  ia.xb_gamma = gamma1;
+  ia.NKC_x = tp->qkv.NKC;
+  ia.first = first;
+  return ia;
+}
+
 int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out, cudaStream_t s) {
   const fr_config& c = tp->c;
   const float dt = static_cast<float>(-1.0 / c.K);
-  const size_t o_off = tp->qkv.bytes, gu_off = o_off + tp->o.bytes, dn_off = gu_off + tp->gu.bytes;
-  cudaError_t e;
   const bool ada = c.adarms != 0;
+  cudaError_t e;
   for (int k = 0; k < c.K; ++k) {
     const float* x_in = (k == 0) ? x0 : tp->xs;
     float* x_nx = (k == c.K - 1) ? x_out : tp->xs;
@@ -320,131 +475,25 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
     // (scale | shift | gate) row
     auto ada_gain = [&](int l, int n) { return tp->tb.ada_gain + ((static_cast<size_t>(k) * c.L + l) * 2 + n) * c.D; };
     auto ada_mod = [&](int l, int n) { return tp->tb.ada_mod + ((static_cast<size_t>(k) * c.L + l) * 2 + n) * 3 * c.D; };
-    InprojArgs ia{};
-    ia.max_ctas = 2 * tp->nsm;
-    ia.x = x_in;
-    ia.w_in = tp->w_in_bf;
-    ia.b_in = tp->tb.b_in;
-    ia.temb = ada ? nullptr : tp->tb.temb + static_cast<size_t>(k) * c.D;
-    ia.h = tp->h;
-    ia.ssq = tp->ssq_a;
-    ia.T = p.T;
-    ia.D = c.D;
-    ia.A = c.A;
-    ia.Nt = p.Nt;
-    ia.KB = tp->KB;
-    ia.ssq_ld = tp->ssq_ld;
-    ia.xb = tp->fp8 ? nullptr : tp->xbuf;
-    ia.xb_gamma = ada ? ada_gain(0, 0) : tp->gains;   // gamma1 of layer 0
-    ia.NKC_x = tp->qkv.NKC;
-    ia.first = (k == 0);
+    auto gain = [&](int l, int n) -> const float* {
+      return ada ? ada_gain(l, n) : tp->gains + (static_cast<size_t>(l) * 2 + n) * c.D;
+    };
+    InprojArgs ia = inproj_args(tp, p, x_in, ada ? nullptr : tp->tb.temb + static_cast<size_t>(k) * c.D, gain(0, 0),
+                                k == 0);
     if ((e = launch_inproj_tc(ia, s, true)) != cudaSuccess) return cuda_fail(e, "in-proj kernel launch");
     for (int l = 0; l < c.L; ++l) {
-      const float* sa = tp->tb.s_a ? tp->tb.s_a + l * PI_COUNT : nullptr;
-      const float* al = tp->tb.alpha ? tp->tb.alpha + l * PI_COUNT : nullptr;
-      __nv_bfloat16* kvk = reinterpret_cast<__nv_bfloat16*>(tp->tb.kv_k + l * tp->tb.kv_layer_bytes);
-      __nv_bfloat16* kvv = reinterpret_cast<__nv_bfloat16*>(tp->tb.kv_v + l * tp->tb.kv_layer_bytes);
-      const float* g1 = ada ? ada_gain(l, 0) : tp->gains + static_cast<size_t>(l) * 2 * c.D;
-      const float* g2 = ada ? ada_gain(l, 1) : g1 + c.D;
-      // QKV: RMSNorm fused into the B staging, split + RoPE fused into the epilogue
-      GemmArgs q = base_args(tp, p, tp->qkv, p.qkv, l, 0);
-      if (tp->fp8) {
-        q.b_kind = B_NORM;
-      } else {
-        q.b_kind = B_ROWS;
-        q.act = tp->xbuf;
-        q.rscale = 1;
+      LayerVectors v{};
+      v.g1 = gain(l, 0);
+      v.g2 = gain(l, 1);
+      v.g1_next = (l + 1 < c.L) ? gain(l + 1, 0) : nullptr;
+      if (ada) {
+        v.gate1 = ada_mod(l, 0) + 2 * c.D;
+        v.gate2 = ada_mod(l, 1) + 2 * c.D;
+        v.bias_qkv = tp->tb.ada_cq + (static_cast<size_t>(k) * c.L + l) * (c.Hq + 2 * c.Hkv) * c.dh;
+        v.bias_gu = tp->tb.ada_cg + (static_cast<size_t>(k) * c.L + l) * 2 * c.F;
       }
-      q.h = tp->h;
-      q.gamma = g1;
-      q.ssq = tp->ssq_a;
-      q.s_a = tp->fp8 ? sa + PI_QKV : nullptr;
-      q.alpha = tp->fp8 ? al + PI_QKV : nullptr;
-      q.epi = EPI_QKV;
-      q.q_out = tp->qbuf;
-      q.kv_k = kvk;
-      q.kv_v = kvv;
-      q.rope_cos = tp->tb.rope_cos;
-      q.rope_sin = tp->tb.rope_sin;
-      q.H = c.H;
-      q.P = p.P;
-      q.S_max = c.P_max + c.H;
-      q.Hq = c.Hq;
-      q.Hkv = c.Hkv;
-      q.dh = c.dh;
-      q.MB_rot = tp->MB_rot;
-      q.bias = ada ? tp->tb.ada_cq + (static_cast<size_t>(k) * c.L + l) * (c.Hq + 2 * c.Hkv) * c.dh : nullptr;
-      if ((e = launch_gemm_tc(q, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "qkv GEMM launch");
-      // attention over [prefix; actions]
-      AttnArgs at{};
-      at.q = tp->qbuf;
-      at.kv_k = kvk;
-      at.kv_v = kvv;
-      at.o = tp->obuf;
-      at.Nt = p.Nt;
-      at.NKC_o = tp->o.NKC;
-      at.s_a = tp->fp8 ? sa + PI_O : nullptr;
-      at.fp8 = tp->fp8;
-      at.H = c.H;
-      at.P = p.P;
-      at.S_max = c.P_max + c.H;
-      at.Hq = c.Hq;
-      at.Hkv = c.Hkv;
-      at.dh = c.dh;
-      at.C = p.attn_C;
-      at.KC = p.attn_KC;
-      at.scale = 1.0f / std::sqrt(static_cast<float>(c.dh));
-      at.xscratch = tp->xscratch;
-      at.status = tp->tb.status;
-      at.umma = p.attn_umma;
-      if ((e = launch_attention_tc(at, p.B, s, true)) != cudaSuccess) return cuda_fail(e, "attention launch");
-      // O projection + residual (+ sum of squares for the pre-MLP norm)
-      GemmArgs og = base_args(tp, p, tp->o, p.o, l, o_off);
-      og.b_kind = B_ROWS;
-      og.act = tp->obuf;
-      og.alpha = tp->fp8 ? al + PI_O : nullptr;
-      og.epi = EPI_RESID;
-      og.h_out = tp->h;
-      og.ssq_out = tp->ssq_b;
-      og.xb_out = tp->fp8 ? nullptr : tp->xbuf;
-      og.xb_gamma = g2;
-      og.NKC_x = tp->qkv.NKC;
-      og.gate = ada ? ada_mod(l, 0) + 2 * c.D : nullptr;
-      if ((e = launch_gemm_tc(og, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "o GEMM launch");
-      // gate|up with RMSNorm fused, GeLU(gate)*up epilogue
-      GemmArgs gg = base_args(tp, p, tp->gu, p.gu, l, gu_off);
-      if (tp->fp8) {
-        gg.b_kind = B_NORM;
-      } else {
-        gg.b_kind = B_ROWS;
-        gg.act = tp->xbuf;
-        gg.rscale = 1;
-      }
-      gg.h = tp->h;
-      gg.gamma = g2;
-      gg.ssq = tp->ssq_b;
-      gg.s_a = tp->fp8 ? sa + PI_GU : nullptr;
-      gg.alpha = tp->fp8 ? al + PI_GU : nullptr;
-      gg.epi = EPI_GELU;
-      gg.u_out = tp->ubuf;
-      gg.NKC_u = tp->dn.NKC;
-      gg.s_a_out = tp->fp8 ? sa + PI_DOWN : nullptr;
-      gg.F = c.F;
-      gg.bias = ada ? tp->tb.ada_cg + (static_cast<size_t>(k) * c.L + l) * 2 * c.F : nullptr;
-      if ((e = launch_gemm_tc(gg, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "gate|up GEMM launch");
-      // down projection + residual (+ sum of squares for the next norm)
-      GemmArgs dg = base_args(tp, p, tp->dn, p.dn, l, dn_off);
-      dg.b_kind = B_ROWS;
-      dg.act = tp->ubuf;
-      dg.alpha = tp->fp8 ? al + PI_DOWN : nullptr;
-      dg.epi = EPI_RESID;
-      dg.h_out = tp->h;
-      dg.ssq_out = tp->ssq_a;
-      dg.xb_out = (tp->fp8 || l == c.L - 1) ? nullptr : tp->xbuf;
-      dg.xb_gamma = (l == c.L - 1) ? nullptr : (ada ? ada_gain(l + 1, 0) : g1 + 2 * c.D);   // gamma1 of layer l+1
-      dg.NKC_x = tp->qkv.NKC;
-      dg.gate = ada ? ada_mod(l, 1) + 2 * c.D : nullptr;
-      if ((e = launch_gemm_tc(dg, p.NT, s, true)) != cudaSuccess) return cuda_fail(e, "down GEMM launch");
+      int rc = record_layer(tp, p, l, v, false, s);
+      if (rc) return rc;
     }
     FinalArgs fa{};
     fa.max_ctas = 2 * tp->nsm;
@@ -471,11 +520,31 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
   return FR_OK;
 }
 
+// The prefix pass (one forward over the P = p.H embedded tokens of each sample, no cached keys):
+// every layer's rotated K and its V land in this handle's KV cache, slots 0..P-1.
+int record_prefill(TensorPath* tp, const StepPlan& p, cudaStream_t s) {
+  const fr_config& c = tp->c;
+  InprojArgs ia = inproj_args(tp, p, nullptr, nullptr, tp->gains, false);
+  ia.emb = tp->emb;
+  cudaError_t e;
+  if ((e = launch_inproj_tc(ia, s, true)) != cudaSuccess) return cuda_fail(e, "embedding kernel launch");
+  for (int l = 0; l < c.L; ++l) {
+    LayerVectors v{};
+    v.g1 = tp->gains + static_cast<size_t>(l) * 2 * c.D;
+    v.g2 = v.g1 + c.D;
+    v.g1_next = (l + 1 < c.L) ? v.g1 + 2 * c.D : nullptr;
+    int rc = record_layer(tp, p, l, v, l == c.L - 1, s);
+    if (rc) return rc;
+  }
+  return FR_OK;
+}
+
 int build_graph(TensorPath* tp, int B, int P, const float* x0, float* x_out, GraphEntry& ge) {
-  ge.plan = make_plan(tp, B, P);
+  const bool prefix = tp->c.role == FR_ROLE_PREFIX;   // (B, P): P prefix tokens per sample, no cached keys
+  ge.plan = prefix ? make_plan(tp, B, 0, P) : make_plan(tp, B, P);
   cudaGraph_t g = nullptr;
   FR_CUDA(cudaStreamBeginCapture(tp->cap, cudaStreamCaptureModeThreadLocal));
-  int rc = record_call(tp, ge.plan, x0, x_out, tp->cap);
+  int rc = prefix ? record_prefill(tp, ge.plan, tp->cap) : record_call(tp, ge.plan, x0, x_out, tp->cap);
   cudaError_t e = cudaStreamEndCapture(tp->cap, &g);
   if (rc) {
     if (g) cudaGraphDestroy(g);
@@ -547,11 +616,13 @@ bool tensor_path_supports(const fr_config& c) {
   if (((c.Hq + c.Hkv) * c.dh / 2) % 64 != 0) return false;   // RoPE pairs fill whole m-blocks
   if ((c.Hkv * c.dh) % BM != 0) return false;                // V rows fill whole m-blocks
   if (c.F % 64 != 0) return false;                            // gate/up pairs fill whole m-blocks
-  if (c.H > 128) return false;                                // one attention row-group pass per warp
   if (c.D % 16 != 0 || (c.Hq * c.dh) % 16 != 0) return false; // 16-byte operand rows
-  if (c.D > 2048 || c.A > 64) return false;                     // per-token kernels keep a row in registers
-  if (static_cast<size_t>(c.D) * c.A * 2 > 160 * 1024) return false;   // in/out-proj weights fit shared memory
+  if (c.D > 2048) return false;                               // per-token kernels keep a row in registers
   if (attn_smem_bytes(c.H, c.dh, 64, 1, 1) > 218 * 1024) return false;   // B200: 227 KB less the static part
+  if (c.role == FR_ROLE_PREFIX) return c.dtype != FR_DTYPE_FP8;   // longer sequences: tcgen05 attention
+  if (c.H > 128) return false;                                // one attention row-group pass per warp
+  if (c.A > 64) return false;
+  if (static_cast<size_t>(c.D) * c.A * 2 > 160 * 1024) return false;   // in/out-proj weights fit shared memory
   int C = 1, KC = 64;
   attn_chunks(c.P_max + c.H, C, KC);
   if (attn_smem_bytes(c.H, c.dh, KC, C, 0) > 200 * 1024) return false;
@@ -567,6 +638,17 @@ const char* tensor_path_limits() {
 size_t exchange_scratch_bytes(TensorPath* tp) {
   const fr_config& c = tp->c;
   size_t mx = 0;
+  if (c.role == FR_ROLE_PREFIX) {   // every batch and prefix length the pass accepts (no cached keys)
+    const ProjLayout* L[4] = {&tp->qkv, &tp->o, &tp->gu, &tp->dn};
+    for (int B = 1; B <= c.B_max; ++B)
+      for (int H = 1; H <= c.H; ++H) {
+        const StepPlan p = make_plan(tp, B, 0, H);
+        const GemmPlan* G[4] = {&p.qkv, &p.o, &p.gu, &p.dn};
+        for (int i = 0; i < 4; ++i) mx = std::max(mx, gemm_scratch_bytes(p.NT, L[i]->MB, G[i]->S, p.Nt));
+        if (p.attn_C > 1) mx = std::max(mx, attn_scratch_bytes(B, c.Hq, p.attn_C, H, c.dh));
+      }
+    return mx;
+  }
   for (int B = 1; B <= c.B_max; ++B) {
     const StepPlan p = make_plan(tp, B, c.P_max);
     const ProjLayout* L[4] = {&tp->qkv, &tp->o, &tp->gu, &tp->dn};
@@ -745,7 +827,16 @@ int tensor_path_denoise(TensorPath* tp, const float* x0, float* x_out, int B, in
   return FR_OK;
 }
 
-int tensor_path_launches(const TensorPath* tp, int) { return tp->c.K * (2 + 5 * tp->c.L); }
+int tensor_path_launches(const TensorPath* tp, int) {
+  if (tp->c.role == FR_ROLE_PREFIX) return 1 + 5 * (tp->c.L - 1) + 1;
+  return tp->c.K * (2 + 5 * tp->c.L);
+}
+
+int tensor_path_prefill(TensorPath* tp, const void* emb, int B, int P, cudaStream_t s) {
+  FR_CUDA(cudaMemcpyAsync(tp->emb, emb, static_cast<size_t>(B) * P * tp->c.D * sizeof(__nv_bfloat16),
+                          cudaMemcpyDeviceToDevice, s));
+  return tensor_path_denoise(tp, nullptr, nullptr, B, P, s);   // the (B, P) graph of the pass
+}
 
 void tensor_path_destroy(TensorPath* tp) {
   if (!tp) return;

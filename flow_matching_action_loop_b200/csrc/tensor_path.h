@@ -47,6 +47,8 @@ int tensor_path_finish_load(TensorPath* tp, cudaStream_t s);
 int tensor_path_set_scales(TensorPath* tp, const float* s_a, const float* alpha);
 int tensor_path_denoise(TensorPath* tp, const float* x0, float* x_out, int B, int P, cudaStream_t s);
 int tensor_path_launches(const TensorPath* tp, int B);
+// prefix-role paths: the pass over B x P embedded tokens (device bf16 [B][P][D]) into the KV cache
+int tensor_path_prefill(TensorPath* tp, const void* emb, int B, int P, cudaStream_t s);
 int tensor_path_set_graph_capacity(TensorPath* tp, int capacity);   // capacity >= 1
 int tensor_path_graph_count(const TensorPath* tp);
 void tensor_path_destroy(TensorPath* tp);

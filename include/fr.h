@@ -63,6 +63,12 @@ enum { FR_DTYPE_F32 = 0, FR_DTYPE_BF16 = 1, FR_DTYPE_FP8 = 2, FR_DTYPE_W4A16 = 3
  * one-kernel-per-operation CUDA-core path (used by fp8 calibration as well). */
 enum { FR_PATH_AUTO = 0, FR_PATH_STEPWISE = 1, FR_PATH_TENSOR = 2 };
 
+/* What a handle runs (fr_config.role).  FR_ROLE_EXPERT: the denoising loop (fr_denoise).
+ * FR_ROLE_PREFIX: the prefix pass (fr_prefill), the backbone whose per-layer keys and values
+ * are the expert's prefix KV cache; there H is the largest number of prefix tokens per sample,
+ * A, K and the time fields are unused (any valid value), dtype is bf16 or w4a16. */
+enum { FR_ROLE_EXPERT = 0, FR_ROLE_PREFIX = 1 };
+
 /* Flags of fr_set_prefix_kv. */
 #define FR_PREFIX_K_ROTATED 1u   /* prefix K already carries RoPE at positions 0..P-1 */
 
@@ -92,6 +98,7 @@ typedef struct fr_config {
   float time_base;
   int adarms;     /* 0: the time embedding is added to the action tokens; 1: it conditions every
                      RMSNorm (adaptive RMSNorm, see fr_layer_weights.w_mod1) */
+  int role;       /* FR_ROLE_* (0: the denoising loop) */
 } fr_config;
 
 /* Host float32 weights of one layer, row-major [out][in] (the nn.Linear convention). */
@@ -231,6 +238,25 @@ const char* fr_path_name(const fr_handle* h);
 
 /* Number of kernel launches one fr_denoise call issues for batch B. */
 int fr_launches_per_call(const fr_handle* h, int B);
+
+/*
+ * fr_prefill -- the prefix pass, the step before the loop (FlashRT walkthrough, component 5:
+ * the attention sites of the Pi0.5 model; the loop's per-layer KV cache is the backbone's keys and
+ * values of the observation's tokens).  `backbone` is an FR_ROLE_PREFIX handle with weights (only
+ * the layer tensors of fr_weights are read; the others may be NULL).  emb_dev: device bf16
+ * [B][P][D] embedded prefix tokens (vision encoder and text embedding outputs).  Runs the
+ * backbone's layers over the P tokens of each sample with full attention among them and RoPE
+ * at positions 0..P-1 (one CUDA graph per (B, P); the last layer stops after its QKV
+ * projection); every layer's rotated K and its V land in the backbone's KV cache (named buffers
+ * "kv_k"/"kv_v", slots 0..P-1).  When `expert` is not NULL they are also copied into its prefix
+ * KV for slots 0..B-1, which then holds (B, P) as after fr_set_prefix_kv with
+ * FR_PREFIX_K_ROTATED; the expert needs the backbone's L, Hkv and dh and a bf16 KV cache.
+ * Asynchronous on `stream`; allocates nothing.
+ * Errors: FR_ERR_ARG (NULL), FR_ERR_STATE (not a prefix handle, no weights, expert not an
+ * expert handle), FR_ERR_SHAPE (B > B_max, P > H of the backbone or P_max of the expert, KV
+ * shapes differ), FR_ERR_CUDA.
+ */
+int fr_prefill(fr_handle* backbone, const void* emb_dev, int B, int P, fr_handle* expert, fr_stream_t stream);
 
 /* ---- execution contract across chunks: selective refresh, named buffers, capsules ---- */
 
