@@ -196,8 +196,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   TL_BEGIN(10 + EPI);
   const int ks = blockIdx.x;            // split-K rank (= cluster rank)
-  const int mb = blockIdx.y;            // m-block
-  const int nt = blockIdx.z;            // n-tile
+  const int nt = blockIdx.y;            // n-tile (varies fastest after the split: CTAs that share a
+  const int mb = blockIdx.z;            // weight m-block run together and read it once from HBM)
   const int Nt = a.Nt;
   const int n0 = nt * Nt;
   const int S = a.S;
@@ -1711,7 +1711,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int n_tiles, cudaStream_t s, bool 
   const int nk_max = (a.NKC + a.S - 1) / a.S;
   const void* f = gemm_kernel(a.epi, a.fp8, a.b_kind == B_NORM, a.w4);
   if (!f) return cudaErrorInvalidValue;
-  return launch_ex(f, dim3(a.S, a.MB, n_tiles), dim3(GEMM_THREADS),
+  return launch_ex(f, dim3(a.S, n_tiles, a.MB), dim3(GEMM_THREADS),
                    gemm_smem_bytes(a.Nt, a.stages, a.b_kind, a.fp8, a.S, nk_max, a.w4, a.epi, a.H, a.xb_out != nullptr), s,
                    pdl, a.S, args);
 }
