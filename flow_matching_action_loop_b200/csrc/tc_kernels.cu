@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         const uint32_t tb = static_cast<uint32_t>(Nt) * KCB;
         mbar_arrive_expect_tx(&sh.full_b[0], pre * tb);
         bulk_g2s(b_slot(0), a.act + (static_cast<size_t>(nt) * a.NKC + kc0) * tb, pre * tb, &sh.full_b[0]);
-        for (int i = 1; i < pre; ++i) mbar_arrive(&sh.full_b[i]);   // round 0 of these slots is covered by slot 0
+        for (int i = 1; i < pre; ++i) mbar_arrive(&sh.full_b[i]);   // their first fill is covered by slot 0's copy
       } else {
         for (int i = 0; i < pre; ++i) issue_b(i);
       }
@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       for (int i = 0; i < nk; ++i) {
         const int s = i % stages;
         const uint32_t par = (i / stages) & 1;
-        // round 0 of batch-1 tiles without B_NORM: one copy brought every resident B chunk and completes
+        // first pass over the ring, batch-1 tiles without B_NORM: one copy brought every resident B chunk and completes
         // slot 0; the chunks after it need no wait of their own
         const bool wait_b = NORM || Nt > 64 || i >= stages || i == 0;
         if (!mbar_wait(&sh.full_a[s], par, WAIT_LIMIT_NS) || (wait_b && !mbar_wait(&sh.full_b[s], par, WAIT_LIMIT_NS))) {

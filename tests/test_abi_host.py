@@ -146,3 +146,15 @@ def test_capsule_sizes_and_contract_calls_reject_before_device_work(abi):
     assert lib.fr_capsule_restore(None, p, ctypes.byref(d), None, 1, None, None) == abi.FR_ERR_ARG
     assert lib.fr_set_graph_capacity(None, 1) == abi.FR_ERR_ARG
     assert lib.fr_graph_count(None) == abi.FR_ERR_ARG
+
+
+def test_plain_c_client_of_the_header(abi, tmp_path):
+    """A C program built against include/fr.h alone links the library and uses its host calls."""
+    import os
+    src = os.path.join(os.path.dirname(__file__), "c", "abi_host.c")
+    exe = str(tmp_path / "abi_host")
+    lib_dir = os.path.dirname(abi.LIB_PATH)
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.dirname(abi.HEADER), src, "-o", exe,
+                    "-L", lib_dir, "-lflowloop", "-lm", f"-Wl,-rpath,{lib_dir}"], check=True)
+    out = subprocess.run([exe], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.stderr
