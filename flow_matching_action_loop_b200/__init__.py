@@ -25,7 +25,7 @@ from ._abi import (  # noqa: F401
     fr_get_scales, fr_graph_count, fr_last_error, fr_launches_per_call, fr_load_weights, fr_path_name,
     fr_quantize_e4m3, fr_quantize_w4, fr_read_kv, fr_refresh_prefix_kv, fr_rope_tables, fr_round_bf16,
     fr_set_graph_capacity, fr_set_prefix_kv, fr_set_scales, fr_sync_status, header_functions, load_library,
-    make_config, make_prefix_config, fr_prefill, FR_ROLE_EXPERT, FR_ROLE_PREFIX,
+    make_config, make_prefix_config, fr_prefill, fr_selftest_wait, FR_ROLE_EXPERT, FR_ROLE_PREFIX,
 )
 
 load_library()

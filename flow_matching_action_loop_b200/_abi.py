@@ -98,6 +98,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fr_get_scales": (c_int, [H, _FP, _FP, c_int]),
         "fr_set_scales": (c_int, [H, _FP, c_int]),
         "fr_sync_status": (c_int, [H, c_void_p]),
+        "fr_selftest_wait": (c_int, [H, ctypes.c_uint64, c_void_p]),
         "fr_last_error": (c_char_p, []),
         "fr_destroy": (None, [H]),
         "fr_read_kv": (c_int, [H, c_int, c_int, c_void_p, c_void_p, c_int]),
@@ -220,6 +221,10 @@ def fr_set_scales(h, s_act) -> None:
 
 def fr_sync_status(h, stream: int = 0) -> int:
     return _check(load_library().fr_sync_status(h, stream), "fr_sync_status")
+
+
+def fr_selftest_wait(h, limit_ns: int, stream: int = 0) -> None:
+    _check(load_library().fr_selftest_wait(h, limit_ns, stream), "fr_selftest_wait")
 
 
 def fr_last_error() -> str:

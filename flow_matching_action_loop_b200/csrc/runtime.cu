@@ -17,6 +17,7 @@
 #include <vector>
 
 #include "internal.h"
+#include "tc_kernels.h"
 #include "tensor_path.h"
 
 namespace fr {
@@ -1081,6 +1082,17 @@ int fr_set_scales(fr_handle* h, const float* s_act, int n) {
     if (rc) return rc;
   }
   h->scales_set = true;
+  return FR_OK;
+}
+
+int fr_selftest_wait(fr_handle* h, uint64_t limit_ns, fr_stream_t stream) {
+  if (!h || limit_ns < 1000 || limit_ns > 100000000ull) {
+    set_error("fr_selftest_wait: NULL handle or limit outside [1 us, 100 ms]");
+    return FR_ERR_ARG;
+  }
+  FR_CUDA(cudaSetDevice(h->device));
+  FR_CUDA(tc::launch_wait_selftest(h->status, static_cast<unsigned long long>(limit_ns),
+                                   reinterpret_cast<cudaStream_t>(stream)));
   return FR_OK;
 }
 

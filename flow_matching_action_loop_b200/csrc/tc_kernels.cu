@@ -1625,6 +1625,18 @@ cudaError_t launch_ex(const void* func, dim3 grid, dim3 block, size_t smem, cuda
   return cudaLaunchKernelExC(&cfg, func, args);
 }
 
+// Failure-detection self-test: one device wait on a barrier that nothing completes.  It gives
+// up after limit_ns, latches the timeout bit with where-code 0x7F0, and the kernel returns.
+__global__ void k_wait_selftest(unsigned* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, limit_ns)) report_timeout(status, 0x7F0);
+}
+
 }  // namespace
 
 size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4, int epi, int H, int xb) {
@@ -1752,6 +1764,11 @@ cudaError_t launch_final_tc(const FinalArgs& a, cudaStream_t s, bool pdl) {
 
 cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s) {
   k_to_bf16<<<static_cast<unsigned>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0, s>>>(src, dst, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_selftest(unsigned* status, unsigned long long limit_ns, cudaStream_t s) {
+  k_wait_selftest<<<1, 32, 0, s>>>(status, limit_ns);
   return cudaGetLastError();
 }
 

@@ -214,6 +214,17 @@ int fr_set_scales(fr_handle* h, const float* s_act, int n);
  */
 int fr_sync_status(fr_handle* h, fr_stream_t stream);
 
+/*
+ * fr_selftest_wait -- failure-detection self-test: launches one kernel whose single device wait
+ * (an mbarrier that nothing completes) gives up after limit_ns, exactly as a wait of the loop's
+ * kernels does: it latches the timeout bit and the where-code 0x7F0 in the status word and the
+ * kernel returns, leaving the context usable.  The next fr_sync_status returns FR_ERR_TIMEOUT
+ * and clears the word.  No counterpart in the pages: it exists to test that path without
+ * faulting or hanging the GPU.  limit_ns in [1 us, 100 ms].  Asynchronous.
+ * Errors: FR_ERR_ARG (NULL, limit out of range), FR_ERR_CUDA.
+ */
+int fr_selftest_wait(fr_handle* h, uint64_t limit_ns, fr_stream_t stream);
+
 /* Text of the last error on the calling thread ("" if none).  Never NULL. */
 const char* fr_last_error(void);
 

@@ -146,6 +146,8 @@ def test_capsule_sizes_and_contract_calls_reject_before_device_work(abi):
     assert lib.fr_capsule_restore(None, p, ctypes.byref(d), None, 1, None, None) == abi.FR_ERR_ARG
     assert lib.fr_set_graph_capacity(None, 1) == abi.FR_ERR_ARG
     assert lib.fr_graph_count(None) == abi.FR_ERR_ARG
+    assert lib.fr_selftest_wait(None, 1000000, None) == abi.FR_ERR_ARG
+    assert lib.fr_prefill(None, p, 1, 1, None, None) == abi.FR_ERR_ARG
 
 
 def test_plain_c_client_of_the_header(abi, tmp_path):
