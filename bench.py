@@ -229,6 +229,26 @@ class _DeviceView:
                                          "version": 3}
 
 
+def cpu_prefix_time(cfg, inp):
+    """Oracle wall time of the prefix pass, sampled as its first layer over every token and scaled by the
+    layer count; returns (us per pass, threads, sample description)."""
+    from oracle import oracle as O
+    one = cfg.replace(L=1)
+    w = {"layers": inp["weights"]["layers"][:1]}
+    model = O.PrefixModel(one, w)
+    t0 = time.perf_counter()
+    O.prefill(one, w, inp["emb"], model=model, samples=[0])
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    sample = (f"layer 0 of {cfg.name} over all {cfg.P} tokens of sample 0 (float64 numpy), "
+              f"scaled x{cfg.L} layers x{cfg.B} samples")
+    return dt * cfg.L * cfg.B * 1e6, threads, sample
+
+
 def run_prefix(args, cfg):
     """The prefix pass (the step before the loop): us per pass over B x P embedded tokens."""
     import synthetic
@@ -299,6 +319,10 @@ def run_prefix(args, cfg):
         "device_status": pp.sync_status(),
         "clocks": clk.summary(),
     }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        us_cpu, threads, sample = cpu_prefix_time(cfg, inp)
+        line["cpu_baseline"] = {"value": round(us_cpu, 1), "unit": "us/pass", "cores": threads, "kind": "oracle",
+                                "sample": sample}
     if rank == 0:
         print(json.dumps(line), flush=True)
     pp.close()

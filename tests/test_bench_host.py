@@ -50,3 +50,17 @@ def test_whole_job_time_per_chunk_counts_every_rank():
     # 2 ranks x 50 calls x 32 chunks in 1000 ms -> 1e6 us / 3200 chunks
     assert bench.job_us_per_chunk(1000.0, 2, 50, 32) == pytest.approx(312.5)
     assert bench.job_us_per_chunk(9.0, 1, 1, 1) == pytest.approx(9000.0)
+
+
+def test_prefix_cpu_baseline_samples_one_layer():
+    import synthetic
+    import bench
+    cfg = synthetic.PrefixConfig("tiny_prefix", L=4, D=64, Hq=2, Hkv=1, dh=32, F=96, B=2, P=20, dtype="bf16")
+    inp = synthetic.make_prefix_pass_inputs(cfg, 0)
+    us, threads, sample = bench.cpu_prefix_time(cfg, inp)
+    assert us > 0 and threads >= 1 and "layer 0" in sample
+    # algorithmic FLOPs: (L-1) full layers and the last layer's QKV per token
+    D, F, dq, nkv, P = cfg.D, cfg.F, cfg.Hq * cfg.dh, cfg.Hkv * cfg.dh, cfg.P
+    full = 2 * ((dq + 2 * nkv) * D + D * dq + 2 * F * D + D * F) + 4 * P * cfg.dh * cfg.Hq
+    want = cfg.B * P * ((cfg.L - 1) * full + 2 * (dq + 2 * nkv) * D)
+    assert bench.prefix_flops(cfg) == want
