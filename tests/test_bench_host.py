@@ -64,3 +64,28 @@ def test_prefix_cpu_baseline_samples_one_layer():
     full = 2 * ((dq + 2 * nkv) * D + D * dq + 2 * F * D + D * F) + 4 * P * cfg.dh * cfg.Hq
     want = cfg.B * P * ((cfg.L - 1) * full + 2 * (dq + 2 * nkv) * D)
     assert bench.prefix_flops(cfg) == want
+
+
+def test_reference_arm_prints_the_contract_line(capsys, monkeypatch):
+    """`bench.py --impl reference` (the oracle on the host cores) prints one JSON line with the keys the
+    native arm prints, on the same metric and workload."""
+    import json
+    monkeypatch.delenv("RANK", raising=False)
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["higher_is_better"] is False and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert "pi05_bf16_b1" in line["config"]["workload"]
+
+
+def test_reference_arm_is_silent_on_other_ranks(capsys, monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"]) == 0
+    assert capsys.readouterr().out.strip() == ""
