@@ -59,7 +59,7 @@ enum { FR_DTYPE_F32 = 0, FR_DTYPE_BF16 = 1, FR_DTYPE_FP8 = 2, FR_DTYPE_W4A16 = 3
 #define FR_W4_GROUP 128
 
 /* Kernel set used by fr_denoise.  FR_PATH_AUTO picks the tensor-core path for
- * bf16/fp8 and the CUDA-core path for f32.  FR_PATH_STEPWISE forces the simple
+ * bf16/fp8/w4a16 and the CUDA-core path for f32.  FR_PATH_STEPWISE forces the simple
  * one-kernel-per-operation CUDA-core path (used by fp8 calibration as well). */
 enum { FR_PATH_AUTO = 0, FR_PATH_STEPWISE = 1, FR_PATH_TENSOR = 2 };
 
@@ -247,7 +247,7 @@ int fr_get_rope_tables(const fr_handle* h, float* cos_host, float* sin_host, int
 /* Name of the kernel set fr_denoise runs ("stepwise" or "tensor"). */
 const char* fr_path_name(const fr_handle* h);
 
-/* Number of kernel launches one fr_denoise call issues for batch B. */
+/* Number of kernel launches one fr_denoise call (fr_prefill for a prefix handle) issues for batch B. */
 int fr_launches_per_call(const fr_handle* h, int B);
 
 /*
