@@ -11,6 +11,7 @@ import pytest
 
 import synthetic
 from oracle import oracle as O
+from tests import _loops as L_
 
 MICRO = synthetic.ActionExpertConfig("micro", L=2, D=8, Hq=4, Hkv=2, dh=4, F=6, H=3, A=2, B=2,
                                      P=2, K=3, dtype="f32", time_dim=8)
@@ -299,3 +300,106 @@ def test_calibration_scales_cover_every_projection_input():
     ref = O.denoise(cfg.replace(dtype="bf16"), inp["weights"], inp["prefix_k"], inp["prefix_v"], inp["x0"])
     cos = np.sum(out * ref) / np.linalg.norm(out) / np.linalg.norm(ref)
     assert cos > 0.99
+
+
+# ---------------------------------------------------------------- calibration, second formulation
+
+def _measure_velocity_loops(cfg, model, w, x, t, kv_k, kv_v, amax):
+    """The fp8 measure pass (reading R11a) for one sample as scalar loops: e4m3 weights dequantised
+    (w_q * s_w, taken from the prepared model: weight quantisation is pinned by the e4m3 tests),
+    projection inputs unquantised, every other rounding point as the bf16 workload (R10).
+    amax[(layer, input)] is raised to the largest |a| over this call's tokens and features."""
+    D, Hq, Hkv, dh, H, P = cfg.D, cfg.Hq, cfg.Hkv, cfg.dh, cfg.H, cfg.P
+    rb = L_.bf16
+    W2 = lambda m: [[rb(float(v)) for v in row] for row in m]   # bf16-stored matrices (R10)
+    vec = lambda a: [float(v) for v in a]                          # float64 scalars throughout
+    half_t = cfg.time_dim // 2
+    e = [rb(math.sin(t * cfg.time_base ** (-i / half_t))) for i in range(half_t)] + \
+        [rb(math.cos(t * cfg.time_base ** (-i / half_t))) for i in range(half_t)]
+    z = [a + b for a, b in zip(L_.matvec(W2(w["w_t1"]), e), vec(w["b_t1"]))]
+    z = [rb(a / (1 + math.exp(-a))) for a in z]
+    temb = [a + b for a, b in zip(L_.matvec(W2(w["w_t2"]), z), vec(w["b_t2"]))]
+    w_in = W2(w["w_in"])
+    hs = [[a + b + c for a, b, c in zip(L_.matvec(w_in, [rb(float(v)) for v in x[i]]), vec(w["b_in"]), temb)]
+          for i in range(H)]
+
+    def note(l, which, rows):
+        m = 0.0
+        for r in rows:
+            for v in r:
+                m = max(m, abs(v))
+        amax[(l, which)] = max(amax.get((l, which), 0.0), m)
+
+    for l, lay in enumerate(model.layers):
+        deq = {n: (lay[n] * lay["sw_" + key]).tolist() for n, key in
+               (("wq", "qkv"), ("wk", "qkv"), ("wv", "qkv"), ("wo", "o"), ("wg", "gu"), ("wu", "gu"), ("wd", "down"))}
+        a = [L_.rms(hs[i], vec(lay["g1"]), cfg.eps) for i in range(H)]
+        note(l, "qkv", a)
+        q = [L_.matvec(deq["wq"], a[i]) for i in range(H)]
+        k = [L_.matvec(deq["wk"], a[i]) for i in range(H)]
+        v = [L_.matvec(deq["wv"], a[i]) for i in range(H)]
+        os_ = []
+        for i in range(H):
+            o = []
+            for j in range(Hq):
+                g = j * Hkv // Hq
+                qi = [rb(u) for u in L_.rotate_half(q[i][j * dh:(j + 1) * dh], P + i, cfg.rope_theta)]
+                keys = [list(kv_k[l][g][p]) for p in range(P)] + \
+                       [[rb(u) for u in L_.rotate_half(k[r][g * dh:(g + 1) * dh], P + r, cfg.rope_theta)] for r in range(H)]
+                vals = [list(kv_v[l][g][p]) for p in range(P)] + [[rb(u) for u in v[r][g * dh:(g + 1) * dh]] for r in range(H)]
+                sc = [sum(qi[d] * kk[d] for d in range(dh)) / math.sqrt(dh) for kk in keys]
+                mx = max(sc)
+                ex = [math.exp(s - mx) for s in sc]
+                tot = sum(ex)
+                o += [sum(ex[s] * vals[s][d] for s in range(len(vals))) / tot for d in range(dh)]
+            os_.append(o)
+        note(l, "o", os_)
+        hs = [[hh + dd for hh, dd in zip(hs[i], L_.matvec(deq["wo"], os_[i]))] for i in range(H)]
+        a2 = [L_.rms(hs[i], vec(lay["g2"]), cfg.eps) for i in range(H)]
+        note(l, "gu", a2)
+        ms = []
+        for i in range(H):
+            gate, up = L_.matvec(deq["wg"], a2[i]), L_.matvec(deq["wu"], a2[i])
+            ms.append([L_.gelu(gg) * uu for gg, uu in zip(gate, up)])
+        note(l, "down", ms)
+        hs = [[hh + dd for hh, dd in zip(hs[i], L_.matvec(deq["wd"], ms[i]))] for i in range(H)]
+    w_out = W2(w["w_out"])
+    return np.array([[a + b for a, b in zip(L_.matvec(w_out, [rb(u) for u in L_.rms(hs[i], vec(w["g_f"]), cfg.eps)]),
+                                            vec(w["b_out"]))] for i in range(H)])
+
+
+def test_calibration_amax_over_every_step_token_and_sample():
+    """fr_calibrate's reference: s_a = amax / 448 with amax over all K steps, all tokens and all
+    samples of the calibration run (reading R11; FlashRT walkthrough, component 6, the measure
+    pass).  Checked against the measure pass written as loops, run sample by sample and step by
+    step with the maxima taken by hand; the case is built so that a maximum taken over one step,
+    the last step or one sample only would differ."""
+    cfg = MICRO.replace(dtype="fp8", B=3, K=4)
+    inp = synthetic.make_inputs(cfg, seed=1)
+    w = inp["weights"]
+    pk, pv = inp["prefix_k"].copy(), inp["prefix_v"].copy()
+    pv[:, 2] *= 4.0            # sample 2's attention outputs dominate the O-projection input
+    x0 = inp["x0"].copy()
+    x0[1] *= 3.0               # sample 1's in-projection is larger
+    model = O.PreparedModel(cfg, w)
+    ts, dt = O.time_grid(cfg.K)
+    per = {}
+    for b in range(cfg.B):
+        kv_k, kv_v = O._sample_kv(model, pk, pv, b)      # R8 rotation is pinned by the RoPE tests
+        x = np.asarray(x0[b], np.float64)
+        for k, t in enumerate(ts):
+            per[(b, k)] = {}
+            x = x + dt * _measure_velocity_loops(cfg, model, w, x, t, kv_k, kv_v, per[(b, k)])
+    keys = {(l, n) for l in range(cfg.L) for n in O.PROJ_INPUTS}
+    total = {key: max(per[bk][key] for bk in per) for key in keys}
+    got = O.calibrate(cfg, w, pk, pv, x0)
+    assert set(got) == keys
+    for key in keys:
+        assert math.isclose(got[key] * 448.0, total[key], rel_tol=1e-9), key
+    # the case discriminates: for some input the maximum is reached neither in step 0, nor in the
+    # last step, nor in sample 0
+    def partial(sel):
+        return {key: max(per[bk][key] for bk in per if sel(bk)) for key in keys}
+    for sel in (lambda bk: bk[1] == 0, lambda bk: bk[1] == cfg.K - 1, lambda bk: bk[0] == 0):
+        part = partial(sel)
+        assert any(part[key] < total[key] * (1 - 1e-3) for key in keys)

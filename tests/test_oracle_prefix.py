@@ -4,12 +4,17 @@ Structural facts the pass must have whatever its weights: layer 0's keys and val
 token come from that token alone; attention inside the prefix is unmasked, so a later
 token reaches an earlier one from layer 1 on; identical tokens give identical values and
 keys that differ only by their RoPE position; and the pass's output, handed to the action
-expert as an already-rotated prefix, is what the loop consumes.
+expert as an already-rotated prefix, is what the loop consumes.  On top of these, the whole
+pass is compared with a second, loop-by-loop formulation that has its own bf16 rounding
+(written on the IEEE bit pattern), on a micro backbone with non-unit gains.
 """
+import math
+
 import numpy as np
 
 import synthetic
 from oracle import oracle as O
+from tests._loops import bf16 as _bf16, gelu, matvec as _matvec, rms as _rms, rotate_half
 
 MICRO = synthetic.PrefixConfig("micro_prefix", L=3, D=32, Hq=4, Hkv=2, dh=8, F=48, B=2, P=7, dtype="bf16")
 
@@ -86,3 +91,112 @@ def test_the_loop_consumes_the_rotated_prefix():
     # and the prefix matters
     other = O.denoise(ecfg, ein["weights"], K[:, ::-1].copy(), V[:, ::-1].copy(), ein["x0"], prefix_k_rotated=True)
     assert np.linalg.norm(other - rot) / np.linalg.norm(rot) > 1e-3
+
+
+# ---------------------------------------------------------------- second formulation (loops)
+
+def _prefill_loops(cfg, w, emb_b):
+    """K and V of every layer for one sample, as explicit scalar loops (reading R18, bf16 rounding
+    points as R10): h = emb; per layer a = bf16(RMS(h) g1), q/k/v = W a, RoPE at the token's
+    position then bf16; after the last layer's QKV nothing more is needed; otherwise softmax
+    attention over all P tokens, h += W_o bf16(o), a = bf16(RMS(h) g2), h += W_d bf16(gelu(W_g a) W_u a)."""
+    L, Hq, Hkv, dh, P = cfg.L, cfg.Hq, cfg.Hkv, cfg.dh, cfg.P
+
+    def rms(vec, g):
+        return _rms(vec, g, cfg.eps)
+
+    def rot(vec, pos):
+        return rotate_half(vec, pos, cfg.rope_theta)
+
+    Kl = np.zeros((L, P, Hkv, dh))
+    Vl = np.zeros((L, P, Hkv, dh))
+    hs = [[_bf16(float(x)) for x in emb_b[p]] for p in range(P)]
+    for l, lw in enumerate(w["layers"]):
+        W = {n: [[_bf16(float(x)) for x in row] for row in lw[n]] for n in ("wq", "wk", "wv", "wo", "wg", "wu", "wd")}
+        g1 = [float(x) for x in lw["g1"]]
+        g2 = [float(x) for x in lw["g2"]]
+        qs, ks, vs = [], [], []
+        for p in range(P):
+            a = [_bf16(x) for x in rms(hs[p], g1)]
+            q, k, v = _matvec(W["wq"], a), _matvec(W["wk"], a), _matvec(W["wv"], a)
+            qs.append([[_bf16(x) for x in rot(q[j * dh:(j + 1) * dh], p)] for j in range(Hq)])
+            ks.append([[_bf16(x) for x in rot(k[g * dh:(g + 1) * dh], p)] for g in range(Hkv)])
+            vs.append([[_bf16(x) for x in v[g * dh:(g + 1) * dh]] for g in range(Hkv)])
+            Kl[l, p] = ks[p]
+            Vl[l, p] = vs[p]
+        if l == L - 1:
+            break
+        for p in range(P):
+            o = []
+            for j in range(Hq):
+                g = j * Hkv // Hq
+                sc = [sum(qs[p][j][d] * ks[s][g][d] for d in range(dh)) / math.sqrt(dh) for s in range(P)]
+                mx = max(sc)
+                ex = [math.exp(x - mx) for x in sc]
+                tot = sum(ex)
+                o += [sum(ex[s] * vs[s][g][d] for s in range(P)) / tot for d in range(dh)]
+            hs[p] = [hh + dd for hh, dd in zip(hs[p], _matvec(W["wo"], [_bf16(x) for x in o]))]
+            a2 = [_bf16(x) for x in rms(hs[p], g2)]
+            gate, up = _matvec(W["wg"], a2), _matvec(W["wu"], a2)
+            m = [_bf16(gelu(gg) * uu) for gg, uu in zip(gate, up)]
+            hs[p] = [hh + dd for hh, dd in zip(hs[p], _matvec(W["wd"], m))]
+    return Kl, Vl
+
+
+LOOPS = synthetic.PrefixConfig("loops_prefix", L=3, D=16, Hq=4, Hkv=2, dh=4, F=24, B=2, P=5, dtype="bf16")
+
+
+def _loops_inputs(seed=21):
+    """Micro prefix-pass inputs with non-unit gains, so that g1 and g2 are told apart."""
+    inp = synthetic.make_prefix_pass_inputs(LOOPS, seed)
+    rng = np.random.default_rng(seed + 1)
+    for lw in inp["weights"]["layers"]:
+        lw["g1"] = (1 + 0.3 * rng.standard_normal(LOOPS.D)).astype(np.float32)
+        lw["g2"] = (1 + 0.3 * rng.standard_normal(LOOPS.D)).astype(np.float32)
+    return inp
+
+
+def _rel(a, b):
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+def _worst_layer_rel(K, V, want):
+    return max(max(_rel(K[l, si], want[si][0][l]), _rel(V[l, si], want[si][1][l]))
+               for si in range(K.shape[1]) for l in range(K.shape[0]))
+
+
+def test_prefill_matches_loop_formulation():
+    """Every layer's K and V of every sample equal the loop formulation's: residuals after the
+    O projection and after the MLP, g1 before QKV and g2 before the MLP in every layer, gate
+    through GeLU times up, and the last layer's QKV.  The two sides round at the same points;
+    only their float64 summation orders differ."""
+    inp = _loops_inputs()
+    K, V = O.prefill(LOOPS, inp["weights"], inp["emb"])
+    want = [_prefill_loops(LOOPS, inp["weights"], inp["emb"][b]) for b in range(LOOPS.B)]
+    assert _worst_layer_rel(K, V, want) < 1e-12
+
+
+def test_prefill_loop_pin_catches_planted_mistakes(monkeypatch):
+    """Mistakes planted in the oracle (CPU only) make the loop comparison fail: the pin above is
+    not blind to them."""
+    inp = _loops_inputs()
+    want = [_prefill_loops(LOOPS, inp["weights"], inp["emb"][b]) for b in range(LOOPS.B)]
+    # g1 applied where g2 belongs
+    w_bad = {"layers": [dict(lw, g2=lw["g1"]) for lw in inp["weights"]["layers"]]}
+    K, V = O.prefill(LOOPS, w_bad, inp["emb"])
+    assert _worst_layer_rel(K, V, want) > 1e-2
+    # gate and up swapped
+    real_project = O._project
+
+    def swapped(model, l, which, a, ws, scales, record):
+        out = real_project(model, l, which, a, ws, scales, record)
+        return out[::-1] if which == "gu" else out
+
+    monkeypatch.setattr(O, "_project", swapped)
+    K, V = O.prefill(LOOPS, inp["weights"], inp["emb"])
+    assert _worst_layer_rel(K, V, want) > 1e-2
+    monkeypatch.setattr(O, "_project", real_project)
+    # the MLP's residual update dropped
+    monkeypatch.setattr(O, "gelu_tanh", lambda z: np.zeros_like(np.asarray(z, np.float64)))
+    K, V = O.prefill(LOOPS, inp["weights"], inp["emb"])
+    assert _worst_layer_rel(K, V, want) > 1e-2
