@@ -32,10 +32,27 @@ METRIC = "µs per 10-step action chunk (batch 1); achieved HBM GB/s vs 8 TB/s"
 UNIT = "us/chunk"
 
 
-# DRAM bytes (read + written) of one whole chunk, summed over the launch list of one ncu capture of
-# this build's kernels (profiles/launches_pi05_bf16_b1.md gives the command).  Reported as the roofline
-# traffic for the workload it was taken on; other workloads report null.
-MEASURED_TRAFFIC = {"pi05_bf16_b1": 6.384e9 + 0.1956e9}
+# DRAM bytes (read + written) of one whole chunk from an ncu capture, keyed by workload and by the
+# digest of the kernel sources it was taken on (kernel_digest()): a figure is reported as the
+# roofline traffic only while those sources are unchanged, otherwise traffic is null.
+MEASURED_TRAFFIC = {}
+
+# Workloads measured besides the headline one in a default single-GPU run (their results go into
+# the line's "workloads" object); each is timed for EXTRA_STEPS calls after EXTRA_WARMUP.
+EXTRA_WORKLOADS = ("tiny_f32", "pi05_fp8_b1", "pi05_bf16_b32", "stress_bf16_b4", "pi05_w4a16_b1")
+EXTRA_STEPS, EXTRA_WARMUP = 20, 3
+
+
+def kernel_digest() -> str:
+    """First 16 hex digits of the SHA-256 of the library's kernel sources (csrc/*.cu, *.h)."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "flow_matching_action_loop_b200", "csrc", "*"))):
+        if f.endswith((".cu", ".h", ".cpp")):
+            with open(f, "rb") as fh:
+                h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
 
 
 def workload_bytes(cfg) -> dict:
@@ -54,6 +71,16 @@ def workload_bytes(cfg) -> dict:
     kv_step = cfg.L * cfg.B * cfg.Hkv * (cfg.P + cfg.H) * cfg.dh * 2 * (4 if cfg.dtype == "f32" else 2)
     return {"weights_per_step": w_step, "kv_per_step": kv_step, "per_chunk": cfg.K * (w_step + kv_step),
             "weights_per_chunk": cfg.K * w_step}
+
+
+def workload_flops(cfg) -> float:
+    """Algorithmic FLOPs of one call (B chunks of K steps): every projection of every token and layer,
+    attention of every query row over its P + H keys, the in/out projections; unpadded."""
+    D, F, dq, nkv = cfg.D, cfg.F, cfg.Hq * cfg.dh, cfg.Hkv * cfg.dh
+    proj = (dq + 2 * nkv) * D + D * dq + 2 * F * D + D * F
+    attn = 2 * (cfg.P + cfg.H) * cfg.dh * cfg.Hq * 2          # QK^T and PV per query token
+    per_tok = cfg.L * (2 * proj + attn) + 2 * 2 * cfg.A * D
+    return float(per_tok) * cfg.B * cfg.H * cfg.K
 
 
 def workload_desc(cfg) -> str:
@@ -163,8 +190,11 @@ def cpu_oracle_time(cfg, inp, n_steps: int):
     """Oracle wall time for n_steps Euler steps (model preparation outside); returns (us per chunk, threads)."""
     from oracle import oracle as O
     model = O.PreparedModel(cfg, inp["weights"])
+    # fp8: fixed activation scales for the timing sample (the arithmetic does not depend on them)
+    scales = {(l, n): 0.01 for l in range(cfg.L) for n in O.PROJ_INPUTS} if cfg.dtype == "fp8" else None
     t0 = time.perf_counter()
-    O.denoise(cfg, inp["weights"], inp["prefix_k"], inp["prefix_v"], inp["x0"], samples=[0], K=n_steps, model=model)
+    O.denoise(cfg, inp["weights"], inp["prefix_k"], inp["prefix_v"], inp["x0"], samples=[0], K=n_steps, model=model,
+              scales=scales)
     dt = time.perf_counter() - t0
     try:
         from threadpoolctl import threadpool_info
@@ -338,7 +368,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", default="pi05_bf16_b1")
+    ap.add_argument("--workload", default="pi05_bf16_b1", help="a workload name, or 'all' (one line each)")
+    ap.add_argument("--no-extra", action="store_true", help="headline workload only (no 'workloads' object)")
     ap.add_argument("--path", type=int, default=0, help="FR_PATH_* (0 auto, 1 stepwise, 2 tensor)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-steps", type=int, default=10, help="oracle Euler steps timed for cpu_baseline")
@@ -351,13 +382,41 @@ def main(argv=None):
             print(json.dumps({"impl": "reference", "unavailable": "the prefix-pass workload has no oracle timing arm"}))
             return 0
         return run_prefix(args, synthetic.PREFIX_CONFIGS[args.workload])
-    cfg = synthetic.CONFIGS[args.workload]
+    cfg = synthetic.CONFIGS["pi05_bf16_b1" if args.workload == "all" else args.workload]
     if args.impl == "reference":
         return run_reference(args, cfg)
 
+    world, rank, local = dist_setup(args.gpus)
+    if args.workload == "all":
+        names = ("pi05_bf16_b1",) + EXTRA_WORKLOADS
+        for name in names:
+            line = run_loop(synthetic.CONFIGS[name], args, world, rank, local, args.steps, args.warmup,
+                            cpu_steps=1 if name != "pi05_bf16_b1" else args.cpu_steps)
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+    else:
+        line = run_loop(cfg, args, world, rank, local, args.steps, args.warmup, cpu_steps=args.cpu_steps)
+        if world == 1 and not args.no_extra and args.workload == "pi05_bf16_b1":
+            line["workloads"] = {}
+            for name in EXTRA_WORKLOADS:
+                sub = run_loop(synthetic.CONFIGS[name], args, world, rank, local, EXTRA_STEPS, EXTRA_WARMUP,
+                               cpu_steps=1)
+                line["workloads"][name] = {k: sub[k] for k in (
+                    "value", "unit", "ms_per_step", "chunks_per_s", "dtype", "config", "roofline", "e2e",
+                    "gpu_launches", "device_status", "clocks", "cpu_baseline", "steps", "warmup") if k in sub}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def run_loop(cfg, args, world, rank, local, steps, warmup, cpu_steps):
+    """Time fr_denoise on one workload; returns the bench line (without printing it)."""
+    import synthetic
     import torch
     from flow_matching_action_loop_b200 import ActionExpertLoop, fr_launches_per_call
-    world, rank, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
 
@@ -377,12 +436,17 @@ def main(argv=None):
     pk = torch.from_numpy(inp["prefix_k"]).to(dev).to(kv_dtype)
     pv = torch.from_numpy(inp["prefix_v"]).to(dev).to(kv_dtype)
     loop.set_prefix_kv(pk, pv)
+    del pk, pv
     x0 = torch.from_numpy(inp["x0"]).to(dev)
     out = torch.empty_like(x0)
     stream = torch.cuda.current_stream(dev)
+    wb = workload_bytes(cfg)
+    l2_note = (f"weights stream {wb['weights_per_step'] / 1e6:.0f} MB/step > 126 MB L2; no flush needed"
+               if wb["weights_per_step"] > 126e6 else
+               f"weights {wb['weights_per_step'] / 1e6:.1f} MB/step fit L2: timed L2-warm, latency-bound parity case")
 
     # ---- device-resident timing
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         loop.denoise(x0, out)
     torch.cuda.synchronize(dev)
     assert loop.sync_status() == 0, "device status after warm-up"
@@ -390,28 +454,28 @@ def main(argv=None):
     torch.cuda.synchronize(dev)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     with ClockSampler(local) as clk:
         ev0.record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             loop.denoise(x0, out)
             marks[i].record(stream)
         ev1.record(stream)
         torch.cuda.synchronize(dev)
-    per_call = sorted([ev0.elapsed_time(marks[0])] + [marks[i - 1].elapsed_time(marks[i]) for i in range(1, args.steps)])
+    per_call = sorted([ev0.elapsed_time(marks[0])] + [marks[i - 1].elapsed_time(marks[i]) for i in range(1, steps)])
     barrier(world)
-    ms = ev0.elapsed_time(ev1)
-    ms = max_over_ranks(ms, world)
+    ms_local = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms_local, world)
     status = loop.sync_status()
-    ms_per_step = ms / args.steps
-    chunks = world * args.steps * cfg.B
-    us_per_chunk = job_us_per_chunk(ms, world, args.steps, cfg.B)
+    ms_per_step = ms / steps
+    chunks = world * steps * cfg.B
+    us_per_chunk = job_us_per_chunk(ms, world, steps, cfg.B)
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
     hx0 = torch.from_numpy(inp["x0"]).pin_memory()
     hout = torch.empty_like(hx0).pin_memory()
     dx = torch.empty_like(x0)
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         dx.copy_(hx0, non_blocking=True)
         loop.denoise(dx, dx)
         hout.copy_(dx, non_blocking=True)
@@ -420,7 +484,7 @@ def main(argv=None):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         dx.copy_(hx0, non_blocking=True)
         loop.denoise(dx, dx)
         hout.copy_(dx, non_blocking=True)
@@ -432,44 +496,57 @@ def main(argv=None):
     xbytes = cfg.B * cfg.H * cfg.A * 4
 
     hbm, tf, tf_sus, peak_kind = load_peaks()
-    wb = workload_bytes(cfg)
+    flops = workload_flops(cfg)
     launches = fr_launches_per_call(loop.h, cfg.B)
-    # dominant kernel: the path's kernel set per chunk; per-launch algorithmic bytes over its device time
-    achieved_gbs = wb["per_chunk"] / (ms_per_step * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved_gbs / hbm, 4), "traffic": MEASURED_TRAFFIC.get(cfg.name),
-                "peak_kind": f"{peak_kind} HBM copy", "kernel": f"{loop.path} path, whole chunk",
-                "bytes_per_launch": wb["per_chunk"]}
+    # dominant kernel: the path's kernel set of one call; its algorithmic work over its device time.
+    # Bound by arithmetic intensity against the ridge of the measured peaks (sustained bf16: the call
+    # is a long step); fp8 contractions take the bf16 peak x 2 (nominal ratio).
+    tf_dtype = tf_sus * (2.0 if cfg.dtype == "fp8" else 1.0)
+    # (the tensor roofline only when it binds clearly: its time at least 1.1x the HBM roofline's)
+    tensor_bound = flops / (tf_dtype * 1e12) > 1.1 * wb["per_chunk"] / (hbm * 1e9) and cfg.dtype != "f32"
+    digest = kernel_digest()
+    traffic = MEASURED_TRAFFIC.get((cfg.name, digest))
+    if tensor_bound:
+        achieved = flops / (ms_per_step * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(tf_dtype, 1), "unit": "TFLOP/s",
+                    "frac": round(achieved / tf_dtype, 4), "traffic": traffic,
+                    "peak_kind": f"{peak_kind} cuBLAS bf16, sustained" + (" x2 (fp8 nominal ratio)" if cfg.dtype == "fp8" else ""),
+                    "kernel": f"{loop.path} path, whole call", "flops_per_launch": flops,
+                    "frac_of_burst": round(achieved / (tf * (2.0 if cfg.dtype == "fp8" else 1.0)), 4)}
+    else:
+        achieved_gbs = wb["per_chunk"] / (ms_per_step * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(achieved_gbs / hbm, 4), "traffic": traffic,
+                    "peak_kind": f"{peak_kind} HBM copy", "kernel": f"{loop.path} path, whole call",
+                    "bytes_per_launch": wb["per_chunk"]}
     line = {
-        "metric": METRIC, "value": round(us_per_chunk, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "metric": METRIC, "value": round(us_per_chunk, 2), "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": round(ms_per_step, 4),
         "ms_per_step_p50": round(per_call[len(per_call) // 2], 4),
         "ms_per_step_p99": round(per_call[min(len(per_call) - 1, (len(per_call) * 99) // 100)], 4),
         "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded, random-init)",
         "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * world, "parallelism": f"replicas x{world}",
-                   "l2": "weights stream 623 MB/step > 126 MB L2; no flush needed",
-                   "path": loop.path},
-        "achieved_hbm_gbs": round(achieved_gbs, 1),
+                   "l2": l2_note, "path": loop.path, "kernel_digest": digest},
+        "per_replica_us_per_chunk": round(ms_local * 1e3 / (steps * cfg.B), 2),
+        "chunks_per_s": round(chunks / (ms * 1e-3), 1),
+        "achieved_hbm_gbs": round(wb["per_chunk"] / (ms_per_step * 1e-3) / 1e9, 1),
         "frac_of_8tbs_weights_only": round(wb["weights_per_chunk"] / (ms_per_step * 1e-3) / 8e12, 4),
         "roofline": roofline,
         "e2e": {"value": round(e2e_us, 2), "unit": UNIT, "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": xbytes},
-        "gpu_launches": launches * args.steps,
+        "gpu_launches": launches * steps,
         "device_status": status,
     }
     line["clocks"] = clk.summary()
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        us_cpu, threads = cpu_oracle_time(cfg, inp, args.cpu_steps)
-        line["cpu_baseline"] = {"value": round(us_cpu, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
-                                "sample": f"{args.cpu_steps} Euler steps of sample 0 of {cfg.name} "
-                                          f"(float64 numpy), scaled to a {cfg.K}-step chunk"}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
     loop.close()
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
-    return 0
+    del x0, out, dx, hx0, hout
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        us_cpu, threads = cpu_oracle_time(cfg, inp, cpu_steps)
+        line["cpu_baseline"] = {"value": round(us_cpu, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": f"{cpu_steps} Euler step(s) of sample 0 of {cfg.name} "
+                                          f"(float64 numpy), scaled to {cfg.B} chunk(s) of {cfg.K} steps"}
+    return line
 
 
 if __name__ == "__main__":

@@ -20,7 +20,7 @@ from ._abi import (  # noqa: F401
     DTYPES, FR_DTYPE_BF16, FR_DTYPE_F32, FR_DTYPE_FP8, FR_DTYPE_W4A16, FR_ERR_ARG, FR_ERR_CUDA, FR_ERR_DEVICE, FR_ERR_SHAPE,
     FR_ERR_STATE, FR_ERR_TIMEOUT, FR_ERR_UNSUPPORTED, FR_OK, FR_PATH_AUTO, FR_PATH_STEPWISE, FR_PATH_TENSOR,
     FR_ATTENTION_NOALLOC_SCRATCH_BYTES, FR_CAPSULE_MAGIC, FR_PREFIX_K_ROTATED, FrCapsule, FrConfig, FrError,
-    fr_attention, fr_attention_noalloc, fr_attention_scratch_bytes, fr_calibrate, fr_capsule_bytes,
+    fr_attention, fr_attention_noalloc, fr_attention_scratch_bytes, fr_ops_sync_status, fr_calibrate, fr_capsule_bytes,
     fr_capsule_restore, fr_capsule_save, fr_create, fr_denoise, fr_destroy, fr_get_buffer, fr_get_rope_tables,
     fr_get_scales, fr_graph_count, fr_last_error, fr_launches_per_call, fr_load_weights, fr_path_name,
     fr_quantize_e4m3, fr_quantize_w4, fr_read_kv, fr_refresh_prefix_kv, fr_rope_tables, fr_round_bf16,

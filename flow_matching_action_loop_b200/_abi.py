@@ -109,6 +109,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fr_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                  c_void_p, ctypes.c_size_t, c_void_p]),
         "fr_attention_scratch_bytes": (ctypes.c_size_t, [c_int, c_int, c_int, c_int, c_int]),
+        "fr_ops_sync_status": (c_int, [c_void_p]),
         "fr_attention_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
                                          c_int, c_void_p]),
         "fr_prefill": (c_int, [H, c_void_p, c_int, c_int, H, c_void_p]),
@@ -312,6 +313,10 @@ def fr_attention(q: int, k: int, v: int, o: int, B: int, Hq: int, Hkv: int, H: i
                  scratch: int = 0, scratch_bytes: int = 0, stream: int = 0) -> None:
     _check(load_library().fr_attention(q, k, v, o, B, Hq, Hkv, H, S_keys, dh, scratch, scratch_bytes, stream),
            "fr_attention")
+
+
+def fr_ops_sync_status(stream: int = 0) -> int:
+    return _check(load_library().fr_ops_sync_status(stream), "fr_ops_sync_status")
 
 
 def fr_attention_scratch_bytes(B: int, Hq: int, H: int, S_keys: int, dh: int) -> int:

@@ -32,7 +32,30 @@ cudaError_t ensure_tc_kernels(int* dev_out) {
 
 namespace {
 
+// Status word of the stand-alone ops ([0] flags, [1] where, [2] block, as a handle's): one per
+// device (module globals are per context), its address looked up once per device.
+static __device__ __align__(16) unsigned g_ops_status[4];
+
+std::once_flag g_status_once[MAX_DEVICES];
+unsigned* g_status_ptr[MAX_DEVICES];
+cudaError_t g_status_err[MAX_DEVICES];
+
 }  // namespace
+
+// Device address of the ops' status word on the current device (kernel attributes set too).
+cudaError_t ops_status_word(unsigned** out, int* dev_out) {
+  int dev = 0;
+  cudaError_t e = ensure_tc_kernels(&dev);
+  if (e != cudaSuccess) return e;
+  std::call_once(g_status_once[dev], [dev] {
+    void* p = nullptr;
+    g_status_err[dev] = cudaGetSymbolAddress(&p, g_ops_status);
+    g_status_ptr[dev] = static_cast<unsigned*>(p);
+  });
+  *out = g_status_ptr[dev];
+  if (dev_out) *dev_out = dev;
+  return g_status_err[dev];
+}
 
 int check_attention(const void* q, const void* k, const void* v, const void* o, int B, int Hq, int Hkv, int H,
                     int S_keys, int dh) {
@@ -58,7 +81,7 @@ int check_attention(const void* q, const void* k, const void* v, const void* o, 
 }
 
 tc::AttnArgs attention_args(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int H,
-                            int S_keys, int dh, float* scratch) {
+                            int S_keys, int dh, float* scratch, unsigned* status) {
   tc::AttnArgs a{};
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.kv_k = static_cast<const __nv_bfloat16*>(k);
@@ -77,6 +100,7 @@ tc::AttnArgs attention_args(const void* q, const void* k, const void* v, void* o
   a.umma = tc::attn_plan(S_keys, tc::attn_tiles(B, Hq, Hkv, H), nsm, a.C, a.KC);
   a.scale = 1.0f / std::sqrt(static_cast<float>(dh));
   a.xscratch = scratch;
+  a.status = status;
   return a;
 }
 
@@ -102,9 +126,26 @@ int fr_attention(const void* q, const void* k, const void* v, void* o, int B, in
     set_error("fr_attention: scratch of %zu bytes needed, %zu given", need, scratch ? scratch_bytes : size_t(0));
     return FR_ERR_SHAPE;
   }
-  FR_CUDA(ensure_tc_kernels(nullptr));
-  const tc::AttnArgs a = attention_args(q, k, v, o, B, Hq, Hkv, H, S_keys, dh, static_cast<float*>(scratch));
+  unsigned* status = nullptr;
+  FR_CUDA(ops_status_word(&status, nullptr));
+  const tc::AttnArgs a = attention_args(q, k, v, o, B, Hq, Hkv, H, S_keys, dh, static_cast<float*>(scratch), status);
   FR_CUDA(tc::launch_attention_tc(a, B, reinterpret_cast<cudaStream_t>(stream), false));
+  return FR_OK;
+}
+
+int fr_ops_sync_status(fr_stream_t stream) {
+  unsigned* status = nullptr;
+  FR_CUDA(ops_status_word(&status, nullptr));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned st[4] = {0, 0, 0, 0};
+  FR_CUDA(cudaMemcpyAsync(st, status, sizeof(st), cudaMemcpyDeviceToHost, s));
+  FR_CUDA(cudaStreamSynchronize(s));
+  FR_CUDA(cudaMemsetAsync(status, 0, sizeof(st), s));
+  FR_CUDA(cudaStreamSynchronize(s));
+  if (st[0] & ST_TIMEOUT) {
+    set_error("device wait gave up in an op (phase word 0x%08x, block %u)", st[1], st[2]);
+    return FR_ERR_TIMEOUT;
+  }
   return FR_OK;
 }
 
@@ -138,7 +179,8 @@ extern "C" int fr_attention_noalloc(const void* q, const void* k, const void* v,
     return FR_ERR_UNSUPPORTED;
   }
   int dev = 0;
-  FR_CUDA(ensure_tc_kernels(&dev));
+  unsigned* status = nullptr;
+  FR_CUDA(ops_status_word(&status, &dev));
   // once per device, with that device current: the array's device address
   std::call_once(g_noalloc_once[dev], [dev] {
     g_noalloc_err[dev] = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
@@ -146,7 +188,7 @@ extern "C" int fr_attention_noalloc(const void* q, const void* k, const void* v,
   if (g_noalloc_err[dev] != cudaSuccess) return cuda_fail(g_noalloc_err[dev], "cudaGetSymbolAddress(scratch)");
   // every scratch word the kernel reads is written earlier in the same launch: nothing to clear
   const tc::AttnArgs a =
-      attention_args(q, k, v, o, B, Hq, Hkv, H, S_keys, dh, static_cast<float*>(g_noalloc_ptr[dev]));
+      attention_args(q, k, v, o, B, Hq, Hkv, H, S_keys, dh, static_cast<float*>(g_noalloc_ptr[dev]), status);
   FR_CUDA(tc::launch_attention_tc(a, B, reinterpret_cast<cudaStream_t>(stream), false));
   return FR_OK;
 }

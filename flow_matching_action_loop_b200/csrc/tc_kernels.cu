@@ -323,8 +323,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       for (int i = (issued > stages ? issued - stages : 0); i < issued; ++i) {
         const int s = i % stages;
         const uint32_t par = (i / stages) & 1;
-        mbar_wait(W4 ? &sh.raw_a[s] : &sh.full_a[s], par, WAIT_LIMIT_NS);
-        mbar_wait(norm ? &sh.raw_b[s] : &sh.full_b[s], par, WAIT_LIMIT_NS);
+        if (!mbar_wait(W4 ? &sh.raw_a[s] : &sh.full_a[s], par, WAIT_LIMIT_NS) ||
+            !mbar_wait(norm ? &sh.raw_b[s] : &sh.full_b[s], par, WAIT_LIMIT_NS))
+          report_timeout(a.status, 0x101);
       }
     }
   } else if (warp == 1) {
@@ -975,7 +976,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
           bulk_g2s(stage + static_cast<size_t>(s2) * gm.R * OLD, xs + (static_cast<size_t>(s2) * H + r_lo) * OLD, sb,
                    &stage_bar);
     }
-    mbar_wait(&stage_bar, 0, WAIT_LIMIT_NS);
+    if (!mbar_wait(&stage_bar, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0x704);
   }
   // row rr of chunk s: src + (s * sstride + roff + rr) * OLD
   const float* src = (C > 1) ? stage : Obuf;
@@ -1361,6 +1362,9 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
                                                                   __uint_as_float(ov[e + 2]), __uint_as_float(ov[e + 3]));
     }
     if (rv) *reinterpret_cast<float4*>(xrow + DH) = make_float4(m_run, l_run, 0.f, 0.f);
+    // the peers fetch these rows with bulk copies (async proxy): order this thread's generic-proxy
+    // stores before them, ahead of the cluster barrier's release
+    fence_proxy_async_global();
   }
   tc_fence_before();
   fence_proxy_async_smem();   // the staging below overwrites Q/K/V/P by bulk copy
@@ -1485,7 +1489,7 @@ __global__ void __launch_bounds__(256) k_inproj_tc(const __grid_constant__ Inpro
   }
   grid_dep_wait();
   if (tid == 0) TL(1);
-  if (!emb) mbar_wait(&wbar, 0, WAIT_LIMIT_NS);
+  if (!emb && !mbar_wait(&wbar, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0x800);
   const int warp = tid >> 5, lane = tid & 31;
   for (int t = blockIdx.x; t < a.T; t += gridDim.x) {   // the weights are staged once per CTA
   if (!emb && tid < a.A) xs[tid] = __bfloat162float(__float2bfloat16_rn(a.x[static_cast<size_t>(t) * a.A + tid]));
@@ -1564,7 +1568,7 @@ __global__ void __launch_bounds__(256) k_final_tc(const __grid_constant__ FinalA
     if (k < a.D) hn[k] = __bfloat162float(__float2bfloat16_rn(hv[q] * r * gf[q]));
   }
   __syncthreads();
-  mbar_wait(&wbar, 0, WAIT_LIMIT_NS);
+  if (!mbar_wait(&wbar, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0x801);
   const int warp = tid >> 5, lane = tid & 31;
   for (int i = warp; i < a.A; i += 8) {
     const __nv_bfloat16* wr = wsm + static_cast<size_t>(i) * a.D;

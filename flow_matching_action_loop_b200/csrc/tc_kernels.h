@@ -171,6 +171,7 @@ struct InprojArgs {
   int NKC_x;
   int T, D, A, Nt, KB, ssq_ld;
   int first;                   // x is the caller's x0 (graph node lookup)
+  unsigned* status;            // device status word (timeouts), or nullptr
 };
 
 struct FinalArgs {
@@ -187,6 +188,7 @@ struct FinalArgs {
   float eps, dt;
   int first;                   // x_in is the caller's x0 (graph node lookup)
   int last;                    // x_out is the caller's output (graph node lookup)
+  unsigned* status;            // device status word (timeouts), or nullptr
 };
 
 // Launchers (tc_kernels.cu).  `pdl` adds the programmatic-stream-serialisation attribute.

@@ -460,6 +460,7 @@ InprojArgs inproj_args(const TensorPath* tp, const StepPlan& p, const float* x_i
   ia.xb_gamma = gamma1;
   ia.NKC_x = tp->qkv.NKC;
   ia.first = first;
+  ia.status = tp->tb.status;
   return ia;
 }
 
@@ -515,6 +516,7 @@ int record_call(TensorPath* tp, const StepPlan& p, const float* x0, float* x_out
     fa.dt = dt;
     fa.first = (k == 0);
     fa.last = (k == c.K - 1);
+    fa.status = tp->tb.status;
     if ((e = launch_final_tc(fa, s, true)) != cudaSuccess) return cuda_fail(e, "final kernel launch");
   }
   return FR_OK;

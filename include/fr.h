@@ -380,10 +380,21 @@ int fr_graph_count(const fr_handle* h);
  * owned by the caller (NULL when that size is 0).  Asynchronous on `stream`.
  * Limits: dh in {64, 128, 256}, Hq % Hkv == 0, 1 <= H <= 128, H <= S_keys <= 32768.
  * Errors: FR_ERR_ARG (NULL pointer, bad size), FR_ERR_UNSUPPORTED (limits),
- * FR_ERR_SHAPE (scratch smaller than needed), FR_ERR_CUDA.
+ * FR_ERR_SHAPE (scratch smaller than needed), FR_ERR_CUDA.  A device wait of the op that
+ * gives up (see fr_sync_status) is latched in the ops' status word of the device: read it
+ * with fr_ops_sync_status.
  */
 int fr_attention(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int H, int S_keys,
                  int dh, void* scratch, size_t scratch_bytes, fr_stream_t stream);
+
+/*
+ * fr_ops_sync_status -- synchronise `stream`, then read and clear the status word that the
+ * stand-alone ops (fr_attention, fr_attention_noalloc) of the current device latch their
+ * device-side failures in.  Returns FR_OK or FR_ERR_TIMEOUT (the message gives the wait's
+ * where-code and block).  The word is one per device, shared by every op call on it.
+ * Errors: FR_ERR_CUDA.
+ */
+int fr_ops_sync_status(fr_stream_t stream);
 
 /* Bytes of scratch fr_attention needs for these sizes (0 if the keys fit one chunk). */
 size_t fr_attention_scratch_bytes(int B, int Hq, int H, int S_keys, int dh);
@@ -408,7 +419,8 @@ size_t fr_attention_scratch_bytes(int B, int Hq, int H, int S_keys, int dh);
  * later calls.  All calls on one device share the one array: two calls whose kernels can
  * overlap in time (different streams, or different host threads without ordering) race
  * on it and may return wrong results; calls ordered on one stream are safe.  The array
- * needs no clearing: each launch writes every word it reads before reading it.
+ * needs no clearing: each launch writes every word it reads before reading it.  Device-side
+ * failures go to the ops' status word (fr_ops_sync_status).
  */
 int fr_attention_noalloc(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int H,
                          int S_keys, int dh, fr_stream_t stream);

@@ -17,7 +17,7 @@ if not torch.cuda.is_available():
 
 from flow_matching_action_loop_b200 import (  # noqa: E402
     FR_ATTENTION_NOALLOC_SCRATCH_BYTES, FR_ERR_UNSUPPORTED, FrError, fr_attention, fr_attention_noalloc,
-    fr_attention_scratch_bytes,
+    fr_attention_scratch_bytes, fr_ops_sync_status,
 )
 
 CASES = [
@@ -25,6 +25,7 @@ CASES = [
     (1, 8, 1, 50, 866, 256),    # the π0.5 layer shape: 14 key chunks, 5.8 MB of scratch
     (2, 4, 2, 37, 112, 64),     # ragged: 2 chunks
     (1, 1, 1, 1, 2, 128),       # one chunk: no scratch used
+    (4, 8, 1, 128, 320, 64),    # enough query tiles for the tcgen05 kernel: its merge reads the array, 5.6 MB
 ]
 
 
@@ -65,6 +66,7 @@ def test_noalloc_matches_caller_scratch_on_two_calls(B, Hq, Hkv, H, S, dh):
                      scratch.data_ptr(), nbytes, stream)
         torch.cuda.synchronize()
         _close(o, ref, B, H, Hq, dh)
+    assert fr_ops_sync_status(stream) == 0          # no device wait gave up
 
 
 def test_noalloc_rejects_sizes_beyond_its_array():
