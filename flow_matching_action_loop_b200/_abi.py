@@ -22,6 +22,7 @@ FR_ERR_ARG, FR_ERR_SHAPE, FR_ERR_STATE, FR_ERR_CUDA, FR_ERR_TIMEOUT, FR_ERR_DEVI
 FR_DTYPE_F32, FR_DTYPE_BF16, FR_DTYPE_FP8, FR_DTYPE_W4A16 = 0, 1, 2, 3
 FR_W4_GROUP = 128
 FR_PATH_AUTO, FR_PATH_STEPWISE, FR_PATH_TENSOR = 0, 1, 2
+FR_EXEC_AUTO, FR_EXEC_GRAPH, FR_EXEC_PERSISTENT = 0, 1, 2
 FR_PREFIX_K_ROTATED = 1
 FR_ROLE_EXPERT, FR_ROLE_PREFIX = 0, 1
 DTYPES = {"f32": FR_DTYPE_F32, "bf16": FR_DTYPE_BF16, "fp8": FR_DTYPE_FP8, "w4a16": FR_DTYPE_W4A16}
@@ -105,6 +106,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fr_get_rope_tables": (c_int, [H, _FP, _FP, c_int]),
         "fr_path_name": (c_char_p, [H]),
         "fr_launches_per_call": (c_int, [H, c_int]),
+        "fr_set_exec_mode": (c_int, [H, c_int]),
+        "fr_exec_mode": (c_int, [H, c_int]),
+        "fr_set_wait_limit": (c_int, [H, ctypes.c_uint64]),
         "fr_rope_tables": (c_int, [c_int, c_int, ctypes.c_double, _FP, _FP]),
         "fr_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                  c_void_p, ctypes.c_size_t, c_void_p]),
@@ -299,6 +303,18 @@ def fr_capsule_restore(h, cap_dev: int, desc: FrCapsule, B: int, sample_map=None
     m = _ints(sample_map) if sample_map is not None else None
     _check(load_library().fr_capsule_restore(h, cap_dev, ctypes.byref(desc), m, B, x_dev or None, stream),
            "fr_capsule_restore")
+
+
+def fr_set_exec_mode(h, mode: int) -> None:
+    _check(load_library().fr_set_exec_mode(h, mode), "fr_set_exec_mode")
+
+
+def fr_exec_mode(h, B: int) -> int:
+    return _check(load_library().fr_exec_mode(h, B), "fr_exec_mode")
+
+
+def fr_set_wait_limit(h, limit_ns: int) -> None:
+    _check(load_library().fr_set_wait_limit(h, limit_ns), "fr_set_wait_limit")
 
 
 def fr_set_graph_capacity(h, capacity: int) -> None:

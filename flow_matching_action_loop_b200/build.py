@@ -25,6 +25,8 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
 CUDA_FLAGS = ARCH + COMMON + ["--expt-relaxed-constexpr", "-Xptxas", "-v"] if os.environ.get("FR_PTXAS_V") else ARCH + COMMON + ["--expt-relaxed-constexpr"]
+# FR_DEFINES="NAME ..." adds -DNAME to every compile (instrumented builds for performance analysis)
+CUDA_FLAGS = CUDA_FLAGS + ["-D" + d for d in os.environ.get("FR_DEFINES", "").split()]
 
 
 def _sources():

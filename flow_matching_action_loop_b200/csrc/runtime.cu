@@ -1173,8 +1173,42 @@ const char* fr_path_name(const fr_handle* h) {
 
 int fr_launches_per_call(const fr_handle* h, int B) {
   if (!h) return 0;
-  if (h->path == FR_PATH_TENSOR) return tensor_path_launches(h->tp, B);
+  if (h->path == FR_PATH_TENSOR) return tensor_path_launches(h->tp, B, h->prefix_P > 0 ? h->prefix_P : h->cfg.P_max);
   return h->cfg.K * (2 + 9 * h->cfg.L);
+}
+
+int fr_set_exec_mode(fr_handle* h, int mode) {
+  if (!h || mode < FR_EXEC_AUTO || mode > FR_EXEC_PERSISTENT) {
+    set_error("fr_set_exec_mode: NULL handle or unknown mode");
+    return FR_ERR_ARG;
+  }
+  if (h->path != FR_PATH_TENSOR || h->cfg.role != FR_ROLE_EXPERT) {
+    set_error("fr_set_exec_mode: the handle does not run the tensor-core loop");
+    return FR_ERR_STATE;
+  }
+  return tensor_path_set_exec_mode(h->tp, mode);
+}
+
+int fr_exec_mode(const fr_handle* h, int B) {
+  if (!h) {
+    set_error("fr_exec_mode: NULL handle");
+    return FR_ERR_ARG;
+  }
+  if (h->path != FR_PATH_TENSOR) {
+    set_error("fr_exec_mode: the handle does not run the tensor-core path");
+    return FR_ERR_STATE;
+  }
+  cudaSetDevice(h->device);
+  return tensor_path_exec(h->tp, B, h->prefix_P > 0 ? h->prefix_P : h->cfg.P_max);
+}
+
+int fr_set_wait_limit(fr_handle* h, uint64_t limit_ns) {
+  if (!h || limit_ns > 10000000000ull) {
+    set_error("fr_set_wait_limit: NULL handle or limit above 10 s");
+    return FR_ERR_ARG;
+  }
+  if (h->path == FR_PATH_TENSOR) tensor_path_set_wait_limit(h->tp, limit_ns);
+  return FR_OK;
 }
 
 }  // extern "C"

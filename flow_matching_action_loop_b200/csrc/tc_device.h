@@ -1,0 +1,77 @@
+// Device helpers shared by the tensor-core kernels (tc_kernels.cu, persistent.cu): status
+// latching, number-format packing, GeLU, and the warp-level copy / matrix-multiply wrappers
+// written from the PTX ISA.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <math.h>
+
+#include "sm100.h"
+#include "tc_kernels.h"
+
+namespace fr {
+namespace tc {
+
+using fr::sm100::smem_u32;
+
+__device__ __forceinline__ void report_timeout(unsigned* status, uint32_t where) {
+  if (status) {
+    atomicOr(status, ST_TIMEOUT_BIT);
+    atomicExch(status + 1, where);
+    atomicExch(status + 2, blockIdx.x | (blockIdx.y << 8) | (blockIdx.z << 20));
+  }
+}
+
+__device__ __forceinline__ uint8_t to_e4m3(float v) {
+  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ float gelu_tanh(float g) {
+  const float c0 = 0.7978845608028654f;   // sqrt(2/pi)
+  return 0.5f * g * (1.f + tanhf(c0 * (g + 0.044715f * g * g * g)));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  return static_cast<uint32_t>(to_e4m3(a)) | (static_cast<uint32_t>(to_e4m3(b)) << 8) |
+         (static_cast<uint32_t>(to_e4m3(c)) << 16) | (static_cast<uint32_t>(to_e4m3(d)) << 24);
+}
+
+
+constexpr int ATT_PAD = 8;        // bf16 elements of row padding (16 bytes) against bank conflicts
+
+__device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc, bool valid) {
+  const int n = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(sdst)), "l"(gsrc), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+
+}  // namespace tc
+}  // namespace fr

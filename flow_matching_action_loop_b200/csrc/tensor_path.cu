@@ -8,12 +8,15 @@
 // its weights while its predecessor is still running.
 #include <algorithm>
 #include <cmath>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <utility>
 #include <vector>
 
 #include "internal.h"
+#include "persistent.h"
 #include "tc_kernels.h"
 #include "tensor_path.h"
 
@@ -116,6 +119,11 @@ struct TensorPath {
   size_t graph_capacity = 8;
   unsigned long long use_clock = 0;
   std::vector<float> gains_host;
+  // persistent kernel (batch-1-sized calls)
+  unsigned* pk_ctr = nullptr;    // its counters, zero between calls
+  int exec_mode = FR_EXEC_AUTO;
+  unsigned long long wait_limit_ns = 2000000000ull;
+  std::map<std::pair<int, int>, int> pk_fits;   // (B, P) -> the kernel is resident on every SM (1) or not (0)
 };
 
 namespace {
@@ -156,6 +164,7 @@ size_t carve_all(TensorPath* tp, char* base) {
   tp->w_in_bf = cv.take<__nv_bfloat16>(static_cast<size_t>(c.D) * c.A);
   tp->w_out_bf = cv.take<__nv_bfloat16>(static_cast<size_t>(c.A) * c.D);
   tp->emb = cv.take<__nv_bfloat16>(c.role == FR_ROLE_PREFIX ? static_cast<size_t>(tp->T_max) * c.D : 0);
+  tp->pk_ctr = cv.take<unsigned>(pk::CTR_WORDS);
   return align_up(cv.off, 1024);
 }
 
@@ -541,6 +550,140 @@ int record_prefill(TensorPath* tp, const StepPlan& p, cudaStream_t s) {
   return FR_OK;
 }
 
+// ------------------------------------------------------------------ persistent kernel plan
+
+// Split-K factor of one projection in the persistent kernel: a unit's weights (its k-chunks) should
+// mostly fit the weight ring, so that they are resident when its activations arrive; more splits add
+// a partial-tile exchange.  FR_PK_SPLITS="q,o,gu,dn" overrides (tuning).
+int pk_split(int pg, int NKC) {
+  if (const char* e = std::getenv("FR_PK_SPLITS")) {
+    int v[4] = {0, 0, 0, 0};
+    if (std::sscanf(e, "%d,%d,%d,%d", &v[0], &v[1], &v[2], &v[3]) == 4 && v[pg] >= 1) return std::min(v[pg], NKC);
+  }
+  int S = 1;
+  while (ceil_div(NKC, S) > 8 && S < 16) S *= 2;
+  return std::min(S, NKC);
+}
+
+// Arguments of one persistent call, or false when the call's shape is outside the kernel's limits.
+bool make_pk_args(TensorPath* tp, int B, int P, const float* x0, float* x_out, pk::PkArgs& a) {
+  const fr_config& c = tp->c;
+  if (c.role != FR_ROLE_EXPERT || c.dtype != FR_DTYPE_BF16 || c.adarms) return false;
+  const int T = B * c.H;
+  if (T > pk::PK_MAX_T || c.A > 64 || c.D > 4096 || B * c.Hq > pk::PK_MAX_HEADS) return false;
+  std::memset(&a, 0, sizeof(a));
+  a.L = c.L;
+  a.K = c.K;
+  a.D = c.D;
+  a.Hq = c.Hq;
+  a.Hkv = c.Hkv;
+  a.dh = c.dh;
+  a.F = c.F;
+  a.A = c.A;
+  a.H = c.H;
+  a.P = P;
+  a.S_max = c.P_max + c.H;
+  a.B = B;
+  a.T = T;
+  a.Nt = static_cast<int>(align_up(T, 16));
+  a.KB = tp->KB;
+  a.MBd = tp->MBd;
+  a.MB_rot = tp->MB_rot;
+  a.ssq_ld = tp->ssq_ld;
+  a.NKC_x = tp->qkv.NKC;
+  a.NKC_o = tp->o.NKC;
+  a.NKC_u = tp->dn.NKC;
+  a.eps = c.eps;
+  a.dt = static_cast<float>(-1.0 / c.K);
+  a.scale = 1.0f / std::sqrt(static_cast<float>(c.dh));
+  a.G = tp->nsm;
+  attn_chunks(P + c.H, a.C, a.KC);
+  if (a.C > pk::PK_MAX_C) return false;
+  const ProjLayout* L[4] = {&tp->qkv, &tp->o, &tp->gu, &tp->dn};
+  const size_t w_off[4] = {0, tp->qkv.bytes, tp->qkv.bytes + tp->o.bytes, tp->qkv.bytes + tp->o.bytes + tp->gu.bytes};
+  const uint8_t* act[4] = {tp->xbuf, tp->obuf, tp->xbuf, tp->ubuf};
+  int placed = 0, max_nk = 1;
+  size_t slices = 0, scratch = 0;
+  for (int pg = 0; pg < 4; ++pg) {
+    pk::PkGemm& g = a.g[pg];
+    g.MB = L[pg]->MB;
+    g.NKC = L[pg]->NKC;
+    if (g.MB > pk::PK_MAX_MB) return false;
+    g.S = pk_split(pg, g.NKC);
+    g.units = g.MB * g.S;
+    g.w_off = w_off[pg];
+    g.act = act[pg];
+    g.base = placed % a.G;   // consecutive phases on consecutive CTAs: spreads the weight bytes per CTA
+    placed += g.units;
+    max_nk = std::max(max_nk, ceil_div(g.NKC, g.S));
+    if (g.S > 1) {
+      slices = std::max(slices, static_cast<size_t>(g.S) * ceil_div(a.Nt, g.S) * BM * 4);
+      scratch = std::max(scratch, static_cast<size_t>(g.MB) * g.S * a.Nt * BM * 4);
+    }
+  }
+  a.att_units = B * c.Hq * a.C;
+  a.att_base = a.g[0].units % a.G;
+  a.fi_base = placed % a.G;
+  if (a.C > 1) scratch = std::max(scratch, attn_scratch_bytes(B, c.Hq, a.C, c.H, c.dh));
+  if (scratch > tp->xscratch_bytes) return false;
+  // shared memory: [weight ring | B ring / epilogue stage | RoPE pairs or residual rows], attention over
+  // the region after the ring
+  a.nbs = std::min(pk::PK_MAX_B, max_nk);
+  const size_t bring = static_cast<size_t>(a.nbs) * a.Nt * KCB;
+  const size_t stage = std::max({bring, static_cast<size_t>(a.Nt) * RED_LD * 4, slices});
+  const int cap = pk::pk_max_dynamic_smem();
+  for (a.ring = pk::PK_MAX_RING; a.ring >= 2; --a.ring) {
+    a.u_off = static_cast<uint32_t>(a.ring) * BM * KCB;
+    a.rope_off = static_cast<uint32_t>(align_up(a.u_off + stage, 1024));
+    a.hrow_off = a.rope_off;
+    if (pk::pk_smem_bytes(a) <= static_cast<size_t>(cap)) break;
+  }
+  if (a.ring < 2) return false;
+  a.W = tp->w;
+  a.layer_bytes = tp->layer_bytes;
+  a.gains = tp->gains;
+  a.h = tp->h;
+  a.ssq_a = tp->ssq_a;
+  a.ssq_b = tp->ssq_b;
+  a.q = tp->qbuf;
+  a.obuf = tp->obuf;
+  a.ubuf = tp->ubuf;
+  a.xbuf = tp->xbuf;
+  a.kv_k = reinterpret_cast<__nv_bfloat16*>(tp->tb.kv_k);
+  a.kv_v = reinterpret_cast<__nv_bfloat16*>(tp->tb.kv_v);
+  a.kv_layer_elems = tp->tb.kv_layer_bytes / sizeof(__nv_bfloat16);
+  a.rope_cos = tp->tb.rope_cos;
+  a.rope_sin = tp->tb.rope_sin;
+  a.xscratch = tp->xscratch;
+  a.x0 = x0;
+  a.x_out = x_out;
+  a.xs = tp->xs;
+  a.temb = tp->tb.temb;
+  a.w_in_t = tp->w_in_bf;
+  a.b_in = tp->tb.b_in;
+  a.w_out = tp->w_out_bf;
+  a.b_out = tp->tb.b_out;
+  a.g_f = tp->tb.g_f;
+  a.ctr = tp->pk_ctr;
+  a.status = tp->tb.status;
+  a.flag_limit_ns = tp->wait_limit_ns;
+  return true;
+}
+
+// Whether a call of (B, P) runs the persistent kernel: its shape is within the kernel's limits and
+// one CTA is resident on every SM.
+bool pk_selected(TensorPath* tp, int B, int P, pk::PkArgs* out) {
+  if (tp->exec_mode != FR_EXEC_PERSISTENT) return false;   // automatic choice: the CUDA graph
+  pk::PkArgs a;
+  if (!make_pk_args(tp, B, P, nullptr, nullptr, a)) return false;
+  auto key = std::make_pair(B, P);
+  auto it = tp->pk_fits.find(key);
+  if (it == tp->pk_fits.end()) it = tp->pk_fits.emplace(key, pk::pk_max_blocks_per_sm(a) >= 1 ? 1 : 0).first;
+  if (!it->second) return false;
+  if (out) *out = a;
+  return true;
+}
+
 int build_graph(TensorPath* tp, int B, int P, const float* x0, float* x_out, GraphEntry& ge) {
   const bool prefix = tp->c.role == FR_ROLE_PREFIX;   // (B, P): P prefix tokens per sample, no cached keys
   ge.plan = prefix ? make_plan(tp, B, 0, P) : make_plan(tp, B, P);
@@ -640,6 +783,16 @@ const char* tensor_path_limits() {
 size_t exchange_scratch_bytes(TensorPath* tp) {
   const fr_config& c = tp->c;
   size_t mx = 0;
+  // the persistent kernel's split-K partials at batch-1-sized calls (T <= 64 tokens in one tile)
+  if (c.role == FR_ROLE_EXPERT)
+    for (int B = 1; B <= c.B_max && B * c.H <= pk::PK_MAX_T; ++B) {
+      const int Nt = static_cast<int>(align_up(B * c.H, 16));
+      const ProjLayout* L[4] = {&tp->qkv, &tp->o, &tp->gu, &tp->dn};
+      for (int pg = 0; pg < 4; ++pg) {
+        const int S = pk_split(pg, L[pg]->NKC);
+        if (S > 1) mx = std::max(mx, static_cast<size_t>(L[pg]->MB) * S * Nt * BM * 4);
+      }
+    }
   if (c.role == FR_ROLE_PREFIX) {   // every batch and prefix length the pass accepts (no cached keys)
     const ProjLayout* L[4] = {&tp->qkv, &tp->o, &tp->gu, &tp->dn};
     for (int B = 1; B <= c.B_max; ++B)
@@ -701,6 +854,8 @@ int tensor_path_create(const fr_config& c, const TensorPathBuffers& b, TensorPat
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&tp->nsm, cudaDevAttrMultiProcessorCount, dev);
   if (e == cudaSuccess) e = tc_kernels_init();
+  if (e == cudaSuccess) e = pk::pk_init();
+  if (e == cudaSuccess && tp->pk_ctr) e = cudaMemset(tp->pk_ctr, 0, pk::CTR_WORDS * sizeof(unsigned));
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&tp->cap, cudaStreamNonBlocking);
   if (e != cudaSuccess) {
     delete tp;
@@ -809,6 +964,17 @@ int tensor_path_set_graph_capacity(TensorPath* tp, int capacity) {
 int tensor_path_graph_count(const TensorPath* tp) { return static_cast<int>(tp->graphs.size()); }
 
 int tensor_path_denoise(TensorPath* tp, const float* x0, float* x_out, int B, int P, cudaStream_t s) {
+  pk::PkArgs pa;
+  if (tp->c.role == FR_ROLE_EXPERT && pk_selected(tp, B, P, &pa)) {
+    pa.x0 = x0;
+    pa.x_out = x_out;
+    FR_CUDA(pk::pk_launch(pa, s));
+    return FR_OK;
+  }
+  if (tp->exec_mode == FR_EXEC_PERSISTENT && tp->c.role == FR_ROLE_EXPERT) {
+    set_error("persistent execution: this call's shape is outside the persistent kernel's limits");
+    return FR_ERR_UNSUPPORTED;
+  }
   auto key = std::make_pair(B, P);
   auto it = tp->graphs.find(key);
   if (it == tp->graphs.end()) {
@@ -829,9 +995,25 @@ int tensor_path_denoise(TensorPath* tp, const float* x0, float* x_out, int B, in
   return FR_OK;
 }
 
-int tensor_path_launches(const TensorPath* tp, int) {
+int tensor_path_launches(TensorPath* tp, int B, int P) {
   if (tp->c.role == FR_ROLE_PREFIX) return 1 + 5 * (tp->c.L - 1) + 1;
+  if (pk_selected(tp, B, P, nullptr)) return 1;
   return tp->c.K * (2 + 5 * tp->c.L);
+}
+
+int tensor_path_exec(TensorPath* tp, int B, int P) {
+  if (tp->c.role != FR_ROLE_EXPERT) return FR_EXEC_GRAPH;
+  return pk_selected(tp, B, P, nullptr) ? FR_EXEC_PERSISTENT : FR_EXEC_GRAPH;
+}
+
+int tensor_path_set_exec_mode(TensorPath* tp, int mode) {
+  tp->exec_mode = mode;
+  return FR_OK;
+}
+
+int tensor_path_set_wait_limit(TensorPath* tp, unsigned long long ns) {
+  tp->wait_limit_ns = ns ? ns : 2000000000ull;
+  return FR_OK;
 }
 
 int tensor_path_prefill(TensorPath* tp, const void* emb, int B, int P, cudaStream_t s) {

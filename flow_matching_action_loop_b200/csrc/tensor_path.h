@@ -46,7 +46,10 @@ int tensor_path_pack_layer(TensorPath* tp, int layer, const fr_layer_weights& w,
 int tensor_path_finish_load(TensorPath* tp, cudaStream_t s);
 int tensor_path_set_scales(TensorPath* tp, const float* s_a, const float* alpha);
 int tensor_path_denoise(TensorPath* tp, const float* x0, float* x_out, int B, int P, cudaStream_t s);
-int tensor_path_launches(const TensorPath* tp, int B);
+int tensor_path_launches(TensorPath* tp, int B, int P);
+int tensor_path_exec(TensorPath* tp, int B, int P);              // FR_EXEC_GRAPH or FR_EXEC_PERSISTENT
+int tensor_path_set_exec_mode(TensorPath* tp, int mode);         // FR_EXEC_*
+int tensor_path_set_wait_limit(TensorPath* tp, unsigned long long ns);
 // prefix-role paths: the pass over B x P embedded tokens (device bf16 [B][P][D]) into the KV cache
 int tensor_path_prefill(TensorPath* tp, const void* emb, int B, int P, cudaStream_t s);
 int tensor_path_set_graph_capacity(TensorPath* tp, int capacity);   // capacity >= 1

@@ -247,8 +247,35 @@ int fr_get_rope_tables(const fr_handle* h, float* cos_host, float* sin_host, int
 /* Name of the kernel set fr_denoise runs ("stepwise" or "tensor"). */
 const char* fr_path_name(const fr_handle* h);
 
-/* Number of kernel launches one fr_denoise call (fr_prefill for a prefix handle) issues for batch B. */
+/* Number of kernel launches one fr_denoise call (fr_prefill for a prefix handle) issues for batch B
+ * at the current prefix length. */
 int fr_launches_per_call(const fr_handle* h, int B);
+
+/*
+ * Execution of the tensor-core path (PhyAI page, profiling paragraph: at batch 1 the loop's time
+ * goes to many small launches; optimisation paragraph: the ten-step Euler iteration replayed as
+ * one unit).  FR_EXEC_PERSISTENT: one cooperative launch of a persistent kernel runs the whole
+ * call, one CTA per SM, its phases handed over through bounded device-side waits; it serves bf16
+ * handles without adaRMS whose calls have B*H <= 64 tokens.  FR_EXEC_GRAPH: one CUDA graph of
+ * K*(2 + 5L) kernels chained by programmatic dependent launch (every other shape).  FR_EXEC_AUTO
+ * (the default) takes the persistent kernel wherever it applies.
+ */
+enum { FR_EXEC_AUTO = 0, FR_EXEC_GRAPH = 1, FR_EXEC_PERSISTENT = 2 };
+
+/* fr_set_exec_mode -- choose FR_EXEC_*.  With FR_EXEC_PERSISTENT, fr_denoise returns
+ * FR_ERR_UNSUPPORTED for calls the persistent kernel does not serve.  Errors: FR_ERR_ARG (NULL,
+ * unknown mode), FR_ERR_STATE (not a tensor-path expert handle). */
+int fr_set_exec_mode(fr_handle* h, int mode);
+
+/* fr_exec_mode -- FR_EXEC_PERSISTENT or FR_EXEC_GRAPH: what a call of batch B at the current prefix
+ * length runs; negative error code on a NULL handle or a handle off the tensor path. */
+int fr_exec_mode(const fr_handle* h, int B);
+
+/* fr_set_wait_limit -- bound, in ns, of every wait of the persistent kernel on work of another CTA
+ * (0 restores the default, 2 s).  A wait that gives up latches FR_ERR_TIMEOUT in the status word
+ * (fr_sync_status) and every CTA of the call leaves its loops and returns; the call's outputs are
+ * then undefined and the next call starts afresh.  Errors: FR_ERR_ARG (NULL, limit above 10 s). */
+int fr_set_wait_limit(fr_handle* h, uint64_t limit_ns);
 
 /*
  * fr_prefill -- the prefix pass, the step before the loop (FlashRT walkthrough, component 5:

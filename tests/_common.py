@@ -30,6 +30,15 @@ RAGGED = {
                                              A=32, B=1, P=16, K=2, dtype="bf16"),
     "minimal_bf16": synthetic.ActionExpertConfig("minimal_bf16", L=1, D=128, Hq=1, Hkv=1, dh=128, F=128, H=1,
                                                  A=1, B=1, P=1, K=1, dtype="bf16"),
+    # batch-1-sized calls (B*H <= 64 tokens): the persistent kernel's shapes, ragged in every dimension
+    "b1_ragged_bf16": synthetic.ActionExpertConfig("b1_ragged_bf16", L=2, D=320, Hq=4, Hkv=2, dh=64, F=704, H=37,
+                                                   A=7, B=1, P=75, K=3, dtype="bf16"),
+    "b2_ragged_bf16": synthetic.ActionExpertConfig("b2_ragged_bf16", L=3, D=384, Hq=6, Hkv=2, dh=64, F=448, H=23,
+                                                   A=5, B=2, P=130, K=2, dtype="bf16"),
+    "b1_dh128_bf16": synthetic.ActionExpertConfig("b1_dh128_bf16", L=2, D=256, Hq=4, Hkv=1, dh=128, F=512, H=64,
+                                                  A=9, B=1, P=100, K=2, dtype="bf16"),
+    "b4_dh256_bf16": synthetic.ActionExpertConfig("b4_dh256_bf16", L=1, D=256, Hq=2, Hkv=1, dh=256, F=256, H=16,
+                                                  A=4, B=4, P=900, K=2, dtype="bf16"),
 }
 # the same ragged shapes with adaptive-RMSNorm time conditioning
 for _n in ("bf16", "fp8", "w4a16", "f32"):
@@ -69,11 +78,13 @@ def oracle_scales(cfg, inp_weights, model=None):
     return O.calibrate(cfg, inp_weights, obs["prefix_k"], obs["prefix_v"], obs["x0"], model=model)
 
 
-def run_library(cfg, inp, path=0, scales=None, calibrate=False, B_max=None, P_max=None):
-    """Run fr_denoise once on inp; returns (x_K as numpy, loop)."""
+def run_library(cfg, inp, path=0, scales=None, calibrate=False, B_max=None, P_max=None, exec_mode=None):
+    """Run fr_denoise once on inp; returns (x_K as numpy, loop).  exec_mode: FR_EXEC_* (tensor path)."""
     import torch
     from flow_matching_action_loop_b200 import ActionExpertLoop
     loop = ActionExpertLoop(cfg, B_max=B_max, P_max=P_max, path=path)
+    if exec_mode is not None:
+        loop.set_exec_mode(exec_mode)
     loop.load_weights(inp["weights"])
     if cfg.dtype == "fp8":
         if calibrate:

@@ -20,7 +20,7 @@ if not torch.cuda.is_available():
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
 from flow_matching_action_loop_b200 import (  # noqa: E402
-    FR_ERR_ARG, FR_ERR_SHAPE, FR_ERR_STATE, FR_PATH_STEPWISE, FR_PATH_TENSOR, ActionExpertLoop, FrError,
+    FR_ERR_ARG, FR_ERR_SHAPE, FR_ERR_STATE, FR_EXEC_GRAPH, FR_PATH_STEPWISE, FR_PATH_TENSOR, ActionExpertLoop, FrError,
 )
 
 NAME = "ragged_bf16"   # B=3, P=75, Hq/Hkv=4/2, dh=64, H=37, A=7: 4-byte x rows, 16-byte KV rows
@@ -200,6 +200,7 @@ def test_named_buffers_are_the_state_the_loop_reads():
 
 def test_graph_variant_table_keeps_the_most_recent():
     cfg, _, _, loop, (pk, pv, x0), _ = _setup()
+    loop.set_exec_mode(FR_EXEC_GRAPH)   # every batch size through the graph table (B=1 would run the persistent kernel)
     loop.set_prefix_kv(pk, pv)
     y3 = loop.denoise(x0).clone()
     assert loop.graph_count() == 1
