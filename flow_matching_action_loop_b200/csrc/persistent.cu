@@ -32,28 +32,46 @@ constexpr int WK0 = 4;                   // first worker warp
 constexpr int ATT_LD_PAD = 8;
 
 // Optional per-unit timestamps (globaltimer), compiled in only with -DFR_PK_TIMELINE for
-// performance analysis: per CTA, 6 words per unit (tag, start, inputs ready, accumulator or
-// attention done, exchange done, end); the product build has none of this code.
+// performance analysis: per CTA, a 12-word record per worker unit (tag, then the times of its
+// steps, the last word its end) and a 4-word record per GEMM unit of the MMA warp; the product
+// build has none of this code.
 #ifdef FR_PK_TIMELINE
+constexpr int PKT_W = 12;                // words per record: tag, then up to 11 timestamps
 __device__ unsigned long long* g_pk_tl = nullptr;
-__device__ unsigned g_pk_tl_words = 0;   // words per CTA
-#define PKT_DECL unsigned pkt_n_ = 0; unsigned long long pkt_[6] = {0, 0, 0, 0, 0, 0};
+__device__ unsigned g_pk_tl_words = 0;   // words per CTA (worker records, then MMA records from the middle)
+#define PKT_DECL unsigned long long pkt_[PKT_W] = {0};
 #define PKT(i) do { if (c.wt == 0) pkt_[i] = globaltimer(); } while (0)
 #define PKT_TAG(v) do { pkt_[0] = (v); } while (0)
-#define PKT_FLUSH() do { if (c.wt == 0 && g_pk_tl) { pkt_[5] = globaltimer(); \
-    const unsigned o_ = c.tl_n * 6; if (o_ + 6 <= g_pk_tl_words) \
-      for (int q_ = 0; q_ < 6; ++q_) g_pk_tl[static_cast<size_t>(c.cta) * g_pk_tl_words + o_ + q_] = pkt_[q_]; \
+#define PKT_FLUSH() do { if (c.wt == 0 && g_pk_tl) { pkt_[PKT_W - 1] = globaltimer(); \
+    const unsigned o_ = c.tl_n * PKT_W; if (o_ + PKT_W <= g_pk_tl_words / 2) \
+      for (int q_ = 0; q_ < PKT_W; ++q_) g_pk_tl[static_cast<size_t>(c.cta) * g_pk_tl_words + o_ + q_] = pkt_[q_]; \
     ++c.tl_n; } } while (0)
+#define PKX_DECL unsigned long long pkx_[PKT_W] = {0};
+#define PKX(i) do { if (c.wt == 0) pkx_[i] = globaltimer(); } while (0)
+#define PKX_FLUSH(tagv) do { if (c.wt == 0 && g_pk_tl) { pkx_[0] = (tagv); \
+    const unsigned o_ = c.tl_n * PKT_W; if (o_ + PKT_W <= g_pk_tl_words / 2) \
+      for (int q_ = 0; q_ < PKT_W; ++q_) g_pk_tl[static_cast<size_t>(c.cta) * g_pk_tl_words + o_ + q_] = pkx_[q_]; \
+    ++c.tl_n; } } while (0)
+// MMA warp: per GEMM unit, (tag, first weight chunk ready, first activation chunk ready, last MMA issued)
+#define PKM_REC(tag, t1, t2, t3) do { if (g_pk_tl) { const unsigned o_ = g_pk_tl_words / 2 + mrec * 4; \
+    if (o_ + 4 <= g_pk_tl_words) { unsigned long long* r_ = g_pk_tl + static_cast<size_t>(cta) * g_pk_tl_words + o_; \
+      r_[0] = (tag); r_[1] = (t1); r_[2] = (t2); r_[3] = (t3); } ++mrec; } } while (0)
 #else
 #define PKT_DECL
 #define PKT(i) do {} while (0)
 #define PKT_TAG(v) do {} while (0)
 #define PKT_FLUSH() do {} while (0)
+#define PKM_REC(tag, t1, t2, t3) do {} while (0)
+#define PKX_DECL
+#define PKX(i) do {} while (0)
+#define PKX_FLUSH(tagv) do {} while (0)
 #endif
+
+static_assert(sizeof(PkArgs) % 4 == 0, "argument block copied by words");
 
 struct PkSmem {
   uint64_t wfull[PK_MAX_RING], wempty[PK_MAX_RING];
-  uint64_t bfull[PK_MAX_B], bempty[PK_MAX_B];
+  uint64_t bfull;                   // the unit's activation chunks landed (one copy per unit)
   uint64_t accfull, accempty, fin, stage;
   uint32_t tmem_base;
   int abort;
@@ -124,7 +142,7 @@ struct Ctx {
   PkSmem& sh;
   uint8_t* dsm;
   int cta, wt, ww, lane;
-  uint32_t nb;      // activation chunks issued (B ring position)
+  uint32_t nb;      // activation copies issued (one per GEMM unit)
   uint32_t acc;     // accumulators consumed
   uint32_t stage;   // uses of the stage barrier
   uint32_t tl_n;    // timeline records written (instrumented builds)
@@ -181,23 +199,20 @@ __device__ __noinline__ bool gemm_unit(Ctx& c, int pg, int k, int l, int u) {
       rope_sh[idx] = make_float2(a.rope_cos[pos * half + j], a.rope_sin[pos * half + j]);
     }
   }
-  // inputs of the phase ready: the activation chunks of this unit into the B ring
+  // inputs of the phase ready: the unit's activation chunks, one copy into the B region
   if (c.wt == 0) {
     bool ok = wait_counter(a.ctr + CTR_DONE, before(a, k, l, stage), a.flag_limit_ns, a.ctr + CTR_ABORT, &c.sh.abort);
     if (!ok) fail(c, 0x1100 + pg);
     PKT(2);
     if (ok) {
+      // the unit's chunks are contiguous in global memory and in the B region: one copy.  The region
+      // is free: the previous unit's MMAs completed before its epilogue reused it.
       fence_proxy_async_global();
-      for (int i = 0; i < nk; ++i, ++c.nb) {
-        const int bs = c.nb % a.nbs;
-        if (c.nb >= static_cast<uint32_t>(a.nbs) && !pk_wait(&c.sh.bempty[bs], ((c.nb / a.nbs) - 1) & 1, &c.sh.abort)) {
-          fail(c, 0x1110 + pg);
-          break;
-        }
-        mbar_arrive_expect_tx(&c.sh.bfull[bs], btile);
-        bulk_g2s(ureg + bs * btile, gp.act + static_cast<size_t>(kc0 + i) * btile, btile, &c.sh.bfull[bs]);
-      }
+      mbar_arrive_expect_tx(&c.sh.bfull, nk * btile);
+      bulk_g2s(ureg, gp.act + static_cast<size_t>(kc0) * btile, nk * btile, &c.sh.bfull);
+      ++c.nb;
     }
+    PKT(3);
   }
   wk_sync();
   if (c.sh.abort) return false;
@@ -215,13 +230,14 @@ __device__ __noinline__ bool gemm_unit(Ctx& c, int pg, int k, int l, int u) {
       c.sh.rstd[r] = rs;
     }
   }
+  PKT(4);
   // accumulator of this unit
   if (!pk_wait(&c.sh.accfull, c.acc & 1, &c.sh.abort)) {
     if (c.wt == 0) fail(c, 0x1120 + pg);
     return false;
   }
   tc_fence_after();
-  PKT(3);
+  PKT(5);
   const uint32_t tacc = c.sh.tmem_base;
   float* red = reinterpret_cast<float*>(ureg);   // S == 1: [Nt][RED_LD]; S > 1: [T][BM] (the partial tile)
   {
@@ -256,17 +272,20 @@ __device__ __noinline__ bool gemm_unit(Ctx& c, int pg, int k, int l, int u) {
     float* xs = a.xscratch + static_cast<size_t>(mb) * S * Nt * BM;
     fence_proxy_async_smem();
     wk_sync();
+    PKT(6);
     if (c.wt == 0) {
       c.sh.staged = 0;
       bulk_s2g(xs + static_cast<size_t>(ks) * Nt * BM, red, static_cast<uint32_t>(T) * BM * 4u);
       bulk_commit();
       bulk_wait_all();
       fence_proxy_async_global();
+      PKT(7);
       unsigned* rc = a.ctr + CTR_RED + pg * PK_MAX_MB + mb;
       red_release_gpu_add(rc, 1u);
       if (!wait_counter(rc, static_cast<uint32_t>(S) * (it + 1), a.flag_limit_ns, a.ctr + CTR_ABORT, &c.sh.abort)) {
         fail(c, 0x1130 + pg);
       } else {
+        PKT(8);
         fence_proxy_async_global();
         const uint32_t sb = static_cast<uint32_t>(tok1 - tok0) * BM * 4u;
         const uint32_t hb = resid ? static_cast<uint32_t>(tok1 - tok0) * 256u : 0u;
@@ -292,7 +311,7 @@ __device__ __noinline__ bool gemm_unit(Ctx& c, int pg, int k, int l, int u) {
   } else {
     wk_sync();
   }
-  PKT(4);
+  PKT(9);
   // split-K sum of N consecutive rows of token tok in rank order, times the deferred rstd
   auto vals = [&](int tok, int row, float* out, int N) {
     const float sc = rscale ? c.sh.rstd[tok] : 1.0f;
@@ -381,6 +400,7 @@ __device__ __noinline__ bool gemm_unit(Ctx& c, int pg, int k, int l, int u) {
       if (c.lane == 0) ssq_out[static_cast<size_t>(tok) * a.ssq_ld + mb] = sq;
     }
   }
+  PKT(10);
   unit_done(c);
   PKT_FLUSH();
   return true;
@@ -643,6 +663,7 @@ __device__ __noinline__ bool attn_unit(Ctx& c, int k, int l, int u) {
         make_uint4(pack_bf16x2(acc8[0] * id, acc8[1] * id), pack_bf16x2(acc8[2] * id, acc8[3] * id),
                    pack_bf16x2(acc8[4] * id, acc8[5] * id), pack_bf16x2(acc8[6] * id, acc8[7] * id));
   }
+  PKT(10);
   unit_done(c);
   PKT_FLUSH();
   return true;
@@ -718,20 +739,24 @@ __device__ __noinline__ bool fi_unit(Ctx& c, int kf, int t) {
 // ---------------------------------------------------------------------------------------------- the kernel
 
 template <int DH>
-__global__ void __launch_bounds__(PK_THREADS, 1) k_loop_persistent(const __grid_constant__ PkArgs a) {
+__global__ void __launch_bounds__(PK_THREADS, 1) k_loop_persistent(const __grid_constant__ PkArgs args) {
   extern __shared__ __align__(1024) uint8_t dsm[];
   __shared__ PkSmem sh;
+  // The unit functions are not inlined and reach the arguments through a reference: a copy in shared
+  // memory keeps those reads on-chip (a generic pointer into the parameter space is not known to be
+  // read-only, so every use inside a loop would be a reload).
+  __shared__ __align__(16) PkArgs a;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < static_cast<int>(sizeof(PkArgs) / 4); i += PK_THREADS)
+    reinterpret_cast<uint32_t*>(&a)[i] = reinterpret_cast<const uint32_t*>(&args)[i];
+  __syncthreads();
   const int cta = blockIdx.x, G = a.G;
   if (tid == 0) {
     for (int s = 0; s < a.ring; ++s) {
       mbar_init(&sh.wfull[s], 1);
       mbar_init(&sh.wempty[s], 1);
     }
-    for (int s = 0; s < a.nbs; ++s) {
-      mbar_init(&sh.bfull[s], 1);
-      mbar_init(&sh.bempty[s], 1);
-    }
+    mbar_init(&sh.bfull, 1);
     mbar_init(&sh.accfull, 1);
     mbar_init(&sh.accempty, PK_WORKERS);
     mbar_init(&sh.fin, 1);
@@ -792,6 +817,9 @@ __global__ void __launch_bounds__(PK_THREADS, 1) k_loop_persistent(const __grid_
       const uint32_t idesc = idesc_f32acc(FMT_BF16, BM, a.Nt);
       const uint32_t tacc = sh.tmem_base;
       uint32_t n = 0, nb = 0, acc = 0;
+#ifdef FR_PK_TIMELINE
+      unsigned mrec = 0;
+#endif
       bool ok = true;
       for (int k = 0; k < a.K && ok; ++k)
         for (int l = 0; l < a.L && ok; ++l)
@@ -804,25 +832,40 @@ __global__ void __launch_bounds__(PK_THREADS, 1) k_loop_persistent(const __grid_
                 ok = false;
                 break;
               }
-              for (int i = 0; i < nk; ++i, ++n, ++nb) {
-                const int s = n % a.ring, bs = nb % a.nbs;
-                if (!pk_wait(&sh.wfull[s], (n / a.ring) & 1, &sh.abort) ||
-                    !pk_wait(&sh.bfull[bs], (nb / a.nbs) & 1, &sh.abort)) {
+#ifdef FR_PK_TIMELINE
+              unsigned long long tw = 0, tb = 0;
+#endif
+              for (int i = 0; i < nk; ++i, ++n) {
+                const int s = n % a.ring;
+                if (!pk_wait(&sh.wfull[s], (n / a.ring) & 1, &sh.abort)) {
                   ok = false;
                   break;
                 }
+#ifdef FR_PK_TIMELINE
+                if (i == 0) tw = globaltimer();
+#endif
+                if (i == 0 && !pk_wait(&sh.bfull, nb & 1, &sh.abort)) {   // the unit's activation chunks
+                  ok = false;
+                  break;
+                }
+#ifdef FR_PK_TIMELINE
+                if (i == 0) tb = globaltimer();
+#endif
                 tc_fence_after();
                 const uint32_t a0 = smem_u32(dsm + s * CHUNK);
-                const uint32_t b0 = smem_u32(dsm + a.u_off + bs * a.Nt * KCB);
+                const uint32_t b0 = smem_u32(dsm + a.u_off + i * a.Nt * KCB);
 #pragma unroll
                 for (int kk = 0; kk < KCB / 32; ++kk)
                   mma_bf16(tacc, smem_desc(a0 + kk * 2 * BM * 16, BM * 16, 128),
                            smem_desc(b0 + kk * 2 * a.Nt * 16, a.Nt * 16, 128), idesc, (i | kk) != 0);
                 mma_commit(&sh.wempty[s]);
-                mma_commit(&sh.bempty[bs]);
               }
+              ++nb;
               if (!ok) break;
               mma_commit(&sh.accfull);
+              PKM_REC(static_cast<unsigned long long>(pg) | (static_cast<unsigned long long>(k) << 8) |
+                          (static_cast<unsigned long long>(l) << 16) | (static_cast<unsigned long long>(u) << 32),
+                      tw, tb, globaltimer());
               ++acc;
             }
           }
@@ -850,12 +893,11 @@ __global__ void __launch_bounds__(PK_THREADS, 1) k_loop_persistent(const __grid_
       }
       for (int t = first_unit(cta, a.fi_base, G); t < a.T && ok; t += G) ok = fi_unit(c, k, t);
     }
-    // leave nothing in flight: cp.async groups, bulk stores, the activation copies of the B ring
+    // leave nothing in flight: cp.async groups, bulk stores, the last activation copy
     cp_async_wait_all();
     if (c.wt == 0) {
       bulk_wait_all();
-      for (uint32_t i = c.nb > static_cast<uint32_t>(a.nbs) ? c.nb - a.nbs : 0; i < c.nb; ++i)
-        mbar_wait(&sh.bfull[i % a.nbs], (i / a.nbs) & 1, WAIT_LIMIT_NS);
+      if (c.nb > 0) mbar_wait(&sh.bfull, (c.nb - 1) & 1, WAIT_LIMIT_NS);
     }
     __syncwarp();
   }
@@ -891,6 +933,7 @@ size_t pk_smem_bytes(const PkArgs& a) {
   const size_t att = static_cast<size_t>(Hp) * (a.dh + ATT_LD_PAD) * 2 + 2ull * a.KC * (a.dh + ATT_LD_PAD) * 2;
   const int R = (a.H + a.C - 1) / a.C;
   const size_t merge = std::max(static_cast<size_t>(Hp) * (a.dh + 4) * 4, static_cast<size_t>(a.C) * R * (a.dh + 4) * 4);
+  // GEMM units: the B region / epilogue stage, then the RoPE pairs or the residual rows after it
   const size_t rope_end = a.rope_off + static_cast<size_t>(a.H) * 64 * 8;
   const size_t hrow_end = a.hrow_off + 2ull * a.Nt * 64 * 4;   // [2][TS][64], TS <= Nt
   size_t end = std::max(rope_end, hrow_end);

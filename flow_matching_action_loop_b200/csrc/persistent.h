@@ -30,7 +30,7 @@ namespace pk {
 constexpr int PK_THREADS = 256;     // warp 0: weight producer, warp 1: MMA issuer, warps 4-7: workers
 constexpr int PK_WORKERS = 128;
 constexpr int PK_MAX_RING = 16;     // weight ring slots (16 KB each)
-constexpr int PK_MAX_B = 8;         // activation (B operand) ring slots
+constexpr int PK_MAX_B = 8;         // activation (B operand) chunks of one unit (8 KB each at 64 tokens)
 constexpr int PK_MAX_T = 64;        // tokens per call (one n-tile)
 constexpr int PK_MAX_C = 16;        // attention key chunks per head
 
@@ -58,7 +58,7 @@ struct PkArgs {
   int L, K, D, Hq, Hkv, dh, F, A, H, P, S_max, B, T, Nt, KB, MBd, MB_rot, ssq_ld, NKC_x, NKC_o, NKC_u;
   float eps, dt, scale;
   int G;                   // CTAs (one per SM, co-resident)
-  int ring, nbs;           // weight ring slots, B ring slots
+  int ring, nbs;           // weight ring slots, largest activation chunk count of a unit
   uint32_t u_off;          // shared memory: start of the region the workers' jobs share
   uint32_t rope_off;       // QKV units: (cos, sin) pairs of the m-block [H][64]
   uint32_t hrow_off;       // residual units: the owned tokens' h rows [2][TS][64]

@@ -552,21 +552,30 @@ int record_prefill(TensorPath* tp, const StepPlan& p, cudaStream_t s) {
 
 // ------------------------------------------------------------------ persistent kernel plan
 
-// Split-K factor of one projection in the persistent kernel: a unit's weights (its k-chunks) should
-// mostly fit the weight ring, so that they are resident when its activations arrive; more splits add
-// a partial-tile exchange.  FR_PK_SPLITS="q,o,gu,dn" overrides (tuning).
-int pk_split(int pg, int NKC) {
+// Split-K factor of one projection in the persistent kernel: at most PK_MAX_B chunks (128 KB of weights)
+// per unit, so that its activation chunks fit the B region in one copy and most of its weights are
+// resident before they are needed; and more splits while they leave at least half the SMs to the
+// other phases (measured at pi0.5 batch 1: splits 2, 8, 2, 8 for QKV, O, gate|up, down).
+// FR_PK_SPLITS="q,o,gu,dn" overrides (tuning).
+int pk_split(int pg, int MB, int NKC, int nsm) {
   if (const char* e = std::getenv("FR_PK_SPLITS")) {
     int v[4] = {0, 0, 0, 0};
-    if (std::sscanf(e, "%d,%d,%d,%d", &v[0], &v[1], &v[2], &v[3]) == 4 && v[pg] >= 1) return std::min(v[pg], NKC);
+    if (std::sscanf(e, "%d,%d,%d,%d", &v[0], &v[1], &v[2], &v[3]) == 4 && v[pg] >= 1) {
+      int S = std::min(v[pg], NKC);
+      while (ceil_div(NKC, S) > pk::PK_MAX_B) ++S;   // a unit's activation chunks fit its B region
+      return S;
+    }
   }
   int S = 1;
-  while (ceil_div(NKC, S) > 8 && S < 16) S *= 2;
+  while (ceil_div(NKC, S) > pk::PK_MAX_B) S *= 2;
+  while (S * 2 <= NKC && MB * S * 2 <= nsm / 2) S *= 2;
   return std::min(S, NKC);
 }
 
 // Arguments of one persistent call, or false when the call's shape is outside the kernel's limits.
-bool make_pk_args(TensorPath* tp, int B, int P, const float* x0, float* x_out, pk::PkArgs& a) {
+// scratch_needed: report the exchange scratch the call needs instead of checking the handle's.
+bool make_pk_args(TensorPath* tp, int B, int P, const float* x0, float* x_out, pk::PkArgs& a,
+                  size_t* scratch_needed = nullptr) {
   const fr_config& c = tp->c;
   if (c.role != FR_ROLE_EXPERT || c.dtype != FR_DTYPE_BF16 || c.adarms) return false;
   const int T = B * c.H;
@@ -609,7 +618,7 @@ bool make_pk_args(TensorPath* tp, int B, int P, const float* x0, float* x_out, p
     g.MB = L[pg]->MB;
     g.NKC = L[pg]->NKC;
     if (g.MB > pk::PK_MAX_MB) return false;
-    g.S = pk_split(pg, g.NKC);
+    g.S = pk_split(pg, g.MB, g.NKC, a.G);
     g.units = g.MB * g.S;
     g.w_off = w_off[pg];
     g.act = act[pg];
@@ -625,8 +634,9 @@ bool make_pk_args(TensorPath* tp, int B, int P, const float* x0, float* x_out, p
   a.att_base = a.g[0].units % a.G;
   a.fi_base = placed % a.G;
   if (a.C > 1) scratch = std::max(scratch, attn_scratch_bytes(B, c.Hq, a.C, c.H, c.dh));
-  if (scratch > tp->xscratch_bytes) return false;
-  // shared memory: [weight ring | B ring / epilogue stage | RoPE pairs or residual rows], attention over
+  if (scratch_needed) *scratch_needed = scratch;
+  else if (scratch > tp->xscratch_bytes) return false;
+  // shared memory: [weight ring | B region / epilogue stage | RoPE pairs or residual rows], attention over
   // the region after the ring
   a.nbs = std::min(pk::PK_MAX_B, max_nk);
   const size_t bring = static_cast<size_t>(a.nbs) * a.Nt * KCB;
@@ -783,15 +793,13 @@ const char* tensor_path_limits() {
 size_t exchange_scratch_bytes(TensorPath* tp) {
   const fr_config& c = tp->c;
   size_t mx = 0;
-  // the persistent kernel's split-K partials at batch-1-sized calls (T <= 64 tokens in one tile)
+  // the persistent kernel's split-K partials at batch-1-sized calls (T <= 64 tokens in one tile); its
+  // splits grow as its weight ring shrinks, and the ring is smallest at the longest prefix
   if (c.role == FR_ROLE_EXPERT)
     for (int B = 1; B <= c.B_max && B * c.H <= pk::PK_MAX_T; ++B) {
-      const int Nt = static_cast<int>(align_up(B * c.H, 16));
-      const ProjLayout* L[4] = {&tp->qkv, &tp->o, &tp->gu, &tp->dn};
-      for (int pg = 0; pg < 4; ++pg) {
-        const int S = pk_split(pg, L[pg]->NKC);
-        if (S > 1) mx = std::max(mx, static_cast<size_t>(L[pg]->MB) * S * Nt * BM * 4);
-      }
+      pk::PkArgs a;
+      size_t need = 0;
+      if (make_pk_args(tp, B, c.P_max, nullptr, nullptr, a, &need)) mx = std::max(mx, need);
     }
   if (c.role == FR_ROLE_PREFIX) {   // every batch and prefix length the pass accepts (no cached keys)
     const ProjLayout* L[4] = {&tp->qkv, &tp->o, &tp->gu, &tp->dn};
