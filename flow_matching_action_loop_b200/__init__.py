@@ -20,6 +20,7 @@ from ._abi import (  # noqa: F401
     DTYPES, FR_DTYPE_BF16, FR_DTYPE_F32, FR_DTYPE_FP8, FR_DTYPE_W4A16, FR_ERR_ARG, FR_ERR_CUDA, FR_ERR_DEVICE, FR_ERR_SHAPE,
     FR_ERR_STATE, FR_ERR_TIMEOUT, FR_ERR_UNSUPPORTED, FR_OK, FR_PATH_AUTO, FR_PATH_STEPWISE, FR_PATH_TENSOR,
     FR_EXEC_AUTO, FR_EXEC_GRAPH, FR_EXEC_PERSISTENT, fr_set_exec_mode, fr_exec_mode, fr_set_wait_limit,
+    fr_device_checks, fr_debug_limit_extent,
     FR_ATTENTION_NOALLOC_SCRATCH_BYTES, FR_CAPSULE_MAGIC, FR_PREFIX_K_ROTATED, FrCapsule, FrConfig, FrError,
     fr_attention, fr_attention_noalloc, fr_attention_scratch_bytes, fr_ops_sync_status, fr_calibrate, fr_capsule_bytes,
     fr_capsule_restore, fr_capsule_save, fr_create, fr_denoise, fr_destroy, fr_get_buffer, fr_get_rope_tables,
@@ -144,6 +145,10 @@ class ActionExpertLoop:
     def exec_mode(self, B: Optional[int] = None) -> int:
         """FR_EXEC_PERSISTENT or FR_EXEC_GRAPH: what a call of batch B runs."""
         return fr_exec_mode(self.h, B or self.B_max)
+
+    def limit_extent(self, buffer: str, elems: int) -> None:
+        """Checked builds: declare a smaller extent for one of the handle's buffers (0: the real one)."""
+        fr_debug_limit_extent(self.h, buffer, elems)
 
     def set_wait_limit(self, limit_ns: int) -> None:
         """Bound of the persistent kernel's waits on other CTAs (0: the default)."""

@@ -14,7 +14,8 @@ from typing import Optional
 import numpy as np
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libflowloop.so")
+# FR_LIBRARY selects another build of the library (e.g. the checked build, libflowloop_checked.so)
+LIB_PATH = os.environ.get("FR_LIBRARY") or os.path.join(PKG, "libflowloop.so")
 HEADER = os.path.join(os.path.dirname(PKG), "include", "fr.h")
 
 FR_OK = 0
@@ -109,6 +110,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fr_set_exec_mode": (c_int, [H, c_int]),
         "fr_exec_mode": (c_int, [H, c_int]),
         "fr_set_wait_limit": (c_int, [H, ctypes.c_uint64]),
+        "fr_device_checks": (c_int, []),
+        "fr_debug_limit_extent": (c_int, [H, c_char_p, ctypes.c_uint64]),
         "fr_rope_tables": (c_int, [c_int, c_int, ctypes.c_double, _FP, _FP]),
         "fr_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                  c_void_p, ctypes.c_size_t, c_void_p]),
@@ -311,6 +314,14 @@ def fr_set_exec_mode(h, mode: int) -> None:
 
 def fr_exec_mode(h, B: int) -> int:
     return _check(load_library().fr_exec_mode(h, B), "fr_exec_mode")
+
+
+def fr_device_checks() -> bool:
+    return load_library().fr_device_checks() == 1
+
+
+def fr_debug_limit_extent(h, buffer: str, elems: int) -> None:
+    _check(load_library().fr_debug_limit_extent(h, buffer.encode(), elems), "fr_debug_limit_extent")
 
 
 def fr_set_wait_limit(h, limit_ns: int) -> None:

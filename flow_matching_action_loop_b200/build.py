@@ -58,7 +58,19 @@ def _compile(src, verbose):
     return obj
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    """Build libflowloop.so, or with checked=True libflowloop_checked.so (device bounds checks,
+    -DFR_DEVICE_CHECKS) in its own object directory."""
+    global CUDA_FLAGS, BUILD, LIB
+    if checked:
+        saved = (CUDA_FLAGS, BUILD, LIB)
+        CUDA_FLAGS = CUDA_FLAGS + ["-DFR_DEVICE_CHECKS"]
+        BUILD = os.path.join(ROOT, "_build_checked")
+        LIB = os.path.join(PKG, "libflowloop_checked.so")
+        try:
+            return build(force, verbose)
+        finally:
+            CUDA_FLAGS, BUILD, LIB = saved
     os.makedirs(BUILD, exist_ok=True)
     srcs = _sources()
     hdrs = _headers()
@@ -81,8 +93,9 @@ def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
+    ap.add_argument("--checked", action="store_true", help="the build with device bounds checks")
     a = ap.parse_args(argv)
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose, checked=a.checked))
 
 
 if __name__ == "__main__":

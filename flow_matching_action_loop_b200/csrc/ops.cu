@@ -101,6 +101,7 @@ tc::AttnArgs attention_args(const void* q, const void* k, const void* v, void* o
   a.scale = 1.0f / std::sqrt(static_cast<float>(dh));
   a.xscratch = scratch;
   a.status = status;
+  a.o_extent = static_cast<uint64_t>(B) * H * Hq * dh * 2;
   return a;
 }
 

@@ -341,11 +341,14 @@ __device__ __noinline__ bool gemm_unit(Ctx& c, int pg, int k, int l, int u) {
         vals(tok, p + 64, hi, 2);
         const float r00 = lo[0] * r4.x - hi[0] * r4.y, r10 = lo[0] * r4.y + hi[0] * r4.x;
         const float r01 = lo[1] * r4.z - hi[1] * r4.w, r11 = lo[1] * r4.w + hi[1] * r4.z;
-        __nv_bfloat16* dst;
-        if (head < a.Hq) dst = a.q + ((static_cast<size_t>(b) * a.Hq + head) * a.H + i) * a.dh;
-        else dst = kvk + ((static_cast<size_t>(b) * a.Hkv + (head - a.Hq)) * a.S_max + pos) * a.dh;
-        *reinterpret_cast<uint32_t*>(dst + j) = pack_bf16x2(r00, r01);
-        *reinterpret_cast<uint32_t*>(dst + j + half) = pack_bf16x2(r10, r11);
+        const bool isq = head < a.Hq;
+        const size_t o = isq ? ((static_cast<size_t>(b) * a.Hq + head) * a.H + i) * a.dh
+                             : ((static_cast<size_t>(b) * a.Hkv + (head - a.Hq)) * a.S_max + pos) * a.dh;
+        __nv_bfloat16* dst = (isq ? a.q : kvk) + o;
+        if (in_bounds(a.status, o + j + half + 1, isq ? a.ext.q : a.ext.kv, isq ? 0xA005 : 0xA006)) {
+          *reinterpret_cast<uint32_t*>(dst + j) = pack_bf16x2(r00, r01);
+          *reinterpret_cast<uint32_t*>(dst + j + half) = pack_bf16x2(r10, r11);
+        }
       }
     } else {
       const int row = c.lane * 4;
@@ -355,8 +358,9 @@ __device__ __noinline__ bool gemm_unit(Ctx& c, int pg, int k, int l, int u) {
         const int b = tok / a.H, i = tok % a.H, pos = a.P + i;
         float v4[4];
         vals(tok, row, v4, 4);
-        *reinterpret_cast<uint2*>(kvv + ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max + pos) * a.dh + d) =
-            make_uint2(pack_bf16x2(v4[0], v4[1]), pack_bf16x2(v4[2], v4[3]));
+        const size_t vo = ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max + pos) * a.dh + d;
+        if (in_bounds(a.status, vo + 3, a.ext.kv, 0xA007))
+          *reinterpret_cast<uint2*>(kvv + vo) = make_uint2(pack_bf16x2(v4[0], v4[1]), pack_bf16x2(v4[2], v4[3]));
       }
     }
   } else if (pg == PG_GU) {
@@ -367,8 +371,9 @@ __device__ __noinline__ bool gemm_unit(Ctx& c, int pg, int k, int l, int u) {
         float g[2], up[2];
         vals(tok, p, g, 2);
         vals(tok, p + 64, up, 2);
-        *reinterpret_cast<uint32_t*>(a.ubuf + btile_offset(tok, 2 * f, Nt, a.NKC_u)) =
-            pack_bf16x2(gelu_tanh(g[0]) * up[0], gelu_tanh(g[1]) * up[1]);
+        const size_t uo = btile_offset(tok, 2 * f, Nt, a.NKC_u);
+        if (in_bounds(a.status, uo + 3, a.ext.ubuf, 0xA004))
+          *reinterpret_cast<uint32_t*>(a.ubuf + uo) = pack_bf16x2(gelu_tanh(g[0]) * up[0], gelu_tanh(g[1]) * up[1]);
       }
   } else {   // residual: h += update; sum of squares for the next norm; bf16(h * gamma_next)
     const int row = c.lane * 4;
@@ -391,13 +396,16 @@ __device__ __noinline__ bool gemm_unit(Ctx& c, int pg, int k, int l, int u) {
         hv.z += d4[2];
         hv.w += d4[3];
         sq = ((hv.x * hv.x + hv.y * hv.y) + hv.z * hv.z) + hv.w * hv.w;
-        *reinterpret_cast<float4*>(a.h + htile_offset(tok, f, Nt, a.KB)) = hv;
-        if (g_next)
-          *reinterpret_cast<uint2*>(a.xbuf + btile_offset(tok, 2 * f, Nt, a.NKC_x)) =
+        const size_t ho = htile_offset(tok, f, Nt, a.KB);
+        if (in_bounds(a.status, ho + 3, a.ext.h, 0xA001)) *reinterpret_cast<float4*>(a.h + ho) = hv;
+        const size_t xo = btile_offset(tok, 2 * f, Nt, a.NKC_x);
+        if (g_next && in_bounds(a.status, xo + 7, a.ext.xbuf, 0xA002))
+          *reinterpret_cast<uint2*>(a.xbuf + xo) =
               make_uint2(pack_bf16x2(hv.x * g4.x, hv.y * g4.y), pack_bf16x2(hv.z * g4.z, hv.w * g4.w));
       }
       for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-      if (c.lane == 0) ssq_out[static_cast<size_t>(tok) * a.ssq_ld + mb] = sq;
+      const size_t so = static_cast<size_t>(tok) * a.ssq_ld + mb;
+      if (c.lane == 0 && in_bounds(a.status, so, a.ext.ssq, 0xA003)) ssq_out[so] = sq;
     }
   }
   PKT(10);
@@ -659,9 +667,11 @@ __device__ __noinline__ bool attn_unit(Ctx& c, int k, int l, int u) {
     const float id = c.sh.inv_den[rr];
     const int t = b * H + r_lo + rr;
     const int kidx = j * DH + d0;
-    *reinterpret_cast<uint4*>(a.obuf + btile_offset(t, 2 * kidx, a.Nt, a.NKC_o)) =
-        make_uint4(pack_bf16x2(acc8[0] * id, acc8[1] * id), pack_bf16x2(acc8[2] * id, acc8[3] * id),
-                   pack_bf16x2(acc8[4] * id, acc8[5] * id), pack_bf16x2(acc8[6] * id, acc8[7] * id));
+    const size_t ob = btile_offset(t, 2 * kidx, a.Nt, a.NKC_o);
+    if (in_bounds(a.status, ob + 15, a.ext.obuf, 0xA010))
+      *reinterpret_cast<uint4*>(a.obuf + ob) =
+          make_uint4(pack_bf16x2(acc8[0] * id, acc8[1] * id), pack_bf16x2(acc8[2] * id, acc8[3] * id),
+                     pack_bf16x2(acc8[4] * id, acc8[5] * id), pack_bf16x2(acc8[6] * id, acc8[7] * id));
   }
   PKT(10);
   unit_done(c);
@@ -698,7 +708,7 @@ __device__ __noinline__ bool fi_unit(Ctx& c, int kf, int t) {
       if (c.lane == 0) {
         const size_t xi = static_cast<size_t>(t) * A + i;
         const float xn = x_in[xi] + a.dt * (acc + a.b_out[i]);
-        x_nx[xi] = xn;
+        if (in_bounds(a.status, xi, a.ext.x, 0xA020)) x_nx[xi] = xn;
         c.sh.xrow[i] = xn;
       }
     }
@@ -719,15 +729,17 @@ __device__ __noinline__ bool fi_unit(Ctx& c, int kf, int t) {
         float acc = 0.f;
         for (int i = 0; i < A; ++i) acc = fmaf(__bfloat162float(a.w_in_t[static_cast<size_t>(i) * D + n]), bf16r(c.sh.xrow[i]), acc);
         hv = acc + a.b_in[n] + temb[n];
-        a.h[htile_offset(t, n, a.Nt, a.KB)] = hv;
-        *reinterpret_cast<__nv_bfloat16*>(a.xbuf + btile_offset(t, 2 * n, a.Nt, a.NKC_x)) = __float2bfloat16_rn(hv * g1[n]);
+        const size_t ho = htile_offset(t, n, a.Nt, a.KB), xo = btile_offset(t, 2 * n, a.Nt, a.NKC_x);
+        if (in_bounds(a.status, ho, a.ext.h, 0xA021)) a.h[ho] = hv;
+        if (in_bounds(a.status, xo + 1, a.ext.xbuf, 0xA022))
+          *reinterpret_cast<__nv_bfloat16*>(a.xbuf + xo) = __float2bfloat16_rn(hv * g1[n]);
       }
       float sq = hv * hv;
       for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
       if (c.lane == 0) c.sh.part[c.ww][qb] = sq;
     }
     wk_sync();
-    if (c.wt < nq)
+    if (c.wt < nq && in_bounds(a.status, static_cast<size_t>(t) * a.ssq_ld + c.wt, a.ext.ssq, 0xA023))
       a.ssq_a[static_cast<size_t>(t) * a.ssq_ld + c.wt] =
           ((c.sh.part[0][c.wt] + c.sh.part[1][c.wt]) + c.sh.part[2][c.wt]) + c.sh.part[3][c.wt];
   }

@@ -24,6 +24,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "tc_kernels.h"
+
 namespace fr {
 namespace pk {
 
@@ -92,6 +94,7 @@ struct PkArgs {
   unsigned* ctr;           // CTR_WORDS counters
   unsigned* status;        // device status word
   unsigned long long flag_limit_ns;   // bound of every wait on another CTA
+  tc::DevExtents ext;      // extents of the stored-to buffers (checked builds)
 };
 
 size_t pk_smem_bytes(const PkArgs& a);

@@ -1202,6 +1202,31 @@ int fr_exec_mode(const fr_handle* h, int B) {
   return tensor_path_exec(h->tp, B, h->prefix_P > 0 ? h->prefix_P : h->cfg.P_max);
 }
 
+int fr_device_checks(void) {
+#ifdef FR_DEVICE_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int fr_debug_limit_extent(fr_handle* h, const char* buffer, uint64_t elems) {
+  if (!h || !buffer) {
+    set_error("fr_debug_limit_extent: NULL argument");
+    return FR_ERR_ARG;
+  }
+  if (!fr_device_checks()) {
+    set_error("fr_debug_limit_extent: this library was built without device bounds checks");
+    return FR_ERR_UNSUPPORTED;
+  }
+  if (h->path != FR_PATH_TENSOR) {
+    set_error("fr_debug_limit_extent: the handle does not run the tensor-core path");
+    return FR_ERR_STATE;
+  }
+  FR_CUDA(cudaSetDevice(h->device));
+  return tensor_path_limit_extent(h->tp, buffer, elems);
+}
+
 int fr_set_wait_limit(fr_handle* h, uint64_t limit_ns) {
   if (!h || limit_ns > 10000000000ull) {
     set_error("fr_set_wait_limit: NULL handle or limit above 10 s");

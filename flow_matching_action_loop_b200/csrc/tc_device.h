@@ -16,6 +16,27 @@ namespace tc {
 
 using fr::sm100::smem_u32;
 
+// Checked builds: an index at or past its buffer's extent latches the bounds bit and, for the first
+// such index, the site's where-code and the index (low 32 bits) in the status word; the access is
+// skipped.  The
+// product build compiles every check to true.
+__device__ __forceinline__ bool in_bounds(unsigned* status, uint64_t idx, uint64_t extent, uint32_t where) {
+#ifdef FR_DEVICE_CHECKS
+  if (idx < extent) return true;
+  if (status && !(atomicOr(status, ST_BOUNDS_BIT) & ST_BOUNDS_BIT)) {   // the first failing check reports
+    atomicExch(status + 1, where);
+    atomicExch(status + 2, static_cast<unsigned>(idx));
+  }
+  return false;
+#else
+  (void)status;
+  (void)idx;
+  (void)extent;
+  (void)where;
+  return true;
+#endif
+}
+
 __device__ __forceinline__ void report_timeout(unsigned* status, uint32_t where) {
   if (status) {
     atomicOr(status, ST_TIMEOUT_BIT);

@@ -519,9 +519,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
     float acc[N];
 #pragma unroll
     for (int e = 0; e < N; ++e) acc[e] = 0.f;
-    const float* p = (S == 1) ? red + tok * RED_LD + row : xst + static_cast<size_t>(tok - tok0) * BM + row;
+    if (S == 1) {   // no split: the accumulator rows as staged (wide tiles: no per-rank predication)
+      const float* p = red + tok * RED_LD + row;
+#pragma unroll
+      for (int e = 0; e < N; ++e) out[e] = p[e] * sc;
+      return;
+    }
+    const float* p = xst + static_cast<size_t>(tok - tok0) * BM + row;
     const size_t stride = static_cast<size_t>(gm.TS) * BM;
-    const int ns = (S == 1) ? 1 : S;
+    if (S == 2) {
+#pragma unroll
+      for (int e = 0; e < N; ++e) out[e] = (p[e] + p[stride + e]) * sc;   // rank order
+      return;
+    }
+    const int ns = S;
 #pragma unroll
     for (int s2 = 0; s2 < 16; ++s2)
       if (s2 < ns) {
@@ -564,7 +575,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         const int tok = tb + 8 * u, t = n0 + tok;
         if (tok < tok1 && t < a.T && fok) {
           hold[u] = (S > 1) ? *reinterpret_cast<const float4*>(hst + ((row >> 6) * gm.TS + (tok - tok0)) * 64 + (row & 63))
-                            : *reinterpret_cast<const float4*>(a.h_out + htile_offset(t, f, Nt, a.KB));
+                            : *reinterpret_cast<const float4*>(a.h_out + htile_offset_nt(nt, tok, f, Nt, a.KB));
           vals(tok, row, acc[u], Four{});
         }
       }
@@ -577,13 +588,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
           const float4 hv = make_float4(hold[u].x + gt.x * acc[u][0], hold[u].y + gt.y * acc[u][1],
                                         hold[u].z + gt.z * acc[u][2], hold[u].w + gt.w * acc[u][3]);
           sq = ((hv.x * hv.x + hv.y * hv.y) + hv.z * hv.z) + hv.w * hv.w;
-          *reinterpret_cast<float4*>(a.h_out + htile_offset(t, f, Nt, a.KB)) = hv;
-          if (a.xb_out)
-            *reinterpret_cast<uint2*>(a.xb_out + btile_offset(t, 2 * f, Nt, a.NKC_x)) =
+          const size_t ho = htile_offset_nt(nt, tok, f, Nt, a.KB);
+          if (in_bounds(a.status, ho + 3, a.ext.h, 0x9001)) *reinterpret_cast<float4*>(a.h_out + ho) = hv;
+          const size_t xo = btile_offset_nt(nt, tok, 2 * f, Nt, a.NKC_x);
+          if (a.xb_out && in_bounds(a.status, xo + 7, a.ext.xbuf, 0x9002))
+            *reinterpret_cast<uint2*>(a.xb_out + xo) =
                 make_uint2(pack_bf16x2(hv.x * g4.x, hv.y * g4.y), pack_bf16x2(hv.z * g4.z, hv.w * g4.w));
         }
         for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-        if (lane == 0) a.ssq_out[static_cast<size_t>(t) * a.ssq_ld + mb] = sq;
+        const size_t so = static_cast<size_t>(t) * a.ssq_ld + mb;
+        if (lane == 0 && in_bounds(a.status, so, a.ext.ssq, 0x9003)) a.ssq_out[so] = sq;
       }
     }
   } else if (EPI == EPI_GELU) {
@@ -607,10 +621,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       up[1] += bu.y;
       const float u0 = gelu_tanh(g[0]) * up[0], u1 = gelu_tanh(g[1]) * up[1];
       if (FP8) {
-        *reinterpret_cast<uint16_t*>(a.u_out + btile_offset(t, f, Nt, a.NKC_u)) =
-            static_cast<uint16_t>(to_e4m3(u0 * inv) | (static_cast<uint32_t>(to_e4m3(u1 * inv)) << 8));
+        const size_t uo = btile_offset_nt(nt, tok, f, Nt, a.NKC_u);
+        if (in_bounds(a.status, uo + 1, a.ext.ubuf, 0x9004))
+          *reinterpret_cast<uint16_t*>(a.u_out + uo) =
+              static_cast<uint16_t>(to_e4m3(u0 * inv) | (static_cast<uint32_t>(to_e4m3(u1 * inv)) << 8));
       } else {
-        *reinterpret_cast<uint32_t*>(a.u_out + btile_offset(t, 2 * f, Nt, a.NKC_u)) = pack_bf16x2(u0, u1);
+        const size_t uo = btile_offset_nt(nt, tok, 2 * f, Nt, a.NKC_u);
+        if (in_bounds(a.status, uo + 3, a.ext.ubuf, 0x9004))
+          *reinterpret_cast<uint32_t*>(a.u_out + uo) = pack_bf16x2(u0, u1);
       }
     }
   } else {   // EPI_QKV
@@ -649,11 +667,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
           hi[1] += bhi.y;
           const float r00 = lo[0] * cs[u].x - hi[0] * sn[u].x, r10 = lo[0] * sn[u].x + hi[0] * cs[u].x;
           const float r01 = lo[1] * cs[u].y - hi[1] * sn[u].y, r11 = lo[1] * sn[u].y + hi[1] * cs[u].y;
-          __nv_bfloat16* dst;
-          if (head < a.Hq) dst = a.q_out + ((static_cast<size_t>(b) * a.Hq + head) * a.H + i) * a.dh;
-          else dst = a.kv_k + ((static_cast<size_t>(b) * a.Hkv + (head - a.Hq)) * a.S_max + pos) * a.dh;
-          *reinterpret_cast<uint32_t*>(dst + j) = pack_bf16x2(r00, r01);
-          *reinterpret_cast<uint32_t*>(dst + j + half) = pack_bf16x2(r10, r11);
+          const bool isq = head < a.Hq;
+          const size_t o = isq ? ((static_cast<size_t>(b) * a.Hq + head) * a.H + i) * a.dh
+                               : ((static_cast<size_t>(b) * a.Hkv + (head - a.Hq)) * a.S_max + pos) * a.dh;
+          __nv_bfloat16* dst = (isq ? a.q_out : a.kv_k) + o;
+          if (in_bounds(a.status, o + j + half + 1, isq ? a.ext.q : a.ext.kv, isq ? 0x9005 : 0x9006)) {
+            *reinterpret_cast<uint32_t*>(dst + j) = pack_bf16x2(r00, r01);
+            *reinterpret_cast<uint32_t*>(dst + j + half) = pack_bf16x2(r10, r11);
+          }
         }
       }
     } else {
@@ -672,8 +693,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         v4[1] += bv.y;
         v4[2] += bv.z;
         v4[3] += bv.w;
-        *reinterpret_cast<uint2*>(a.kv_v + ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max + pos) * a.dh + d) =
-            make_uint2(pack_bf16x2(v4[0], v4[1]), pack_bf16x2(v4[2], v4[3]));
+        const size_t vo = ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max + pos) * a.dh + d;
+        if (in_bounds(a.status, vo + 3, a.ext.kv, 0x9007))
+          *reinterpret_cast<uint2*>(a.kv_v + vo) = make_uint2(pack_bf16x2(v4[0], v4[1]), pack_bf16x2(v4[2], v4[3]));
       }
     }
   }
@@ -987,6 +1009,9 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
     for (int e = 0; e < 8; ++e) acc[e] *= id;
     const int t = b * H + r_lo + rr;
     const int kidx = j * DH + d0;
+    const size_t ob = a.o_rowmajor ? (static_cast<size_t>(t) * a.Hq * DH + kidx) * 2
+                    : a.fp8 ? btile_offset(t, kidx, a.Nt, a.NKC_o) : btile_offset(t, 2 * kidx, a.Nt, a.NKC_o);
+    if (!in_bounds(a.status, ob + (a.fp8 && !a.o_rowmajor ? 7 : 15), a.o_extent, 0x9010)) continue;
     if (a.o_rowmajor) {
       *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + static_cast<size_t>(t) * a.Hq * DH + kidx) =
           make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
@@ -1261,6 +1286,9 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   // writes 16 consecutive output features d0.. of row (token t, head jq)
   auto store16 = [&](int t, int jh, int d0, const float* v) {
     const int kidx = jh * DH + d0;
+    const size_t ob = a.o_rowmajor ? (static_cast<size_t>(t) * a.Hq * DH + kidx) * 2
+                    : a.fp8 ? btile_offset(t, kidx, a.Nt, a.NKC_o) : btile_offset(t, 2 * kidx + 16, a.Nt, a.NKC_o);
+    if (!in_bounds(a.status, ob + (a.o_rowmajor ? 31 : 15), a.o_extent, 0x9011)) return;
     if (a.o_rowmajor) {
       uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + static_cast<size_t>(t) * a.Hq * DH + kidx);
       dst[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));

@@ -40,19 +40,41 @@ enum BKind : int { B_NORM = 0, B_ROWS = 1 };
 enum EpiKind : int { EPI_QKV = 0, EPI_RESID = 1, EPI_GELU = 2 };
 
 // Status word layout: [0] flags, [1] where, [2] block (see fr_sync_status).
-enum : uint32_t { ST_TIMEOUT_BIT = 1u };
+enum : uint32_t { ST_TIMEOUT_BIT = 1u, ST_BOUNDS_BIT = 2u };
 
-// Byte offset of element (token t, K byte kb) in a tiled GEMM B input.
-__host__ __device__ __forceinline__ size_t btile_offset(int t, int kb, int Nt, int NKC) {
-  const int nt = t / Nt, r = t - nt * Nt;
+// Extents of the buffers the kernels store into (elements of the buffer's type; bytes for the
+// tiled operand buffers).  Checked builds (-DFR_DEVICE_CHECKS) verify every epilogue store index
+// against them; the product build carries them unused.
+struct DevExtents {
+  uint64_t h;      // tiled residual, floats
+  uint64_t q;      // q buffer, bf16 elements
+  uint64_t kv;     // one layer's K (or V) cache slice, bf16 elements
+  uint64_t xbuf;   // bf16(h * gamma) operand, bytes
+  uint64_t obuf;   // attention output operand, bytes
+  uint64_t ubuf;   // GeLU(gate) * up operand, bytes
+  uint64_t ssq;    // sums of squares, floats
+  uint64_t x;      // action state of the call, floats
+};
+
+// Byte offset of element (row r of n-tile nt, K byte kb) in a tiled GEMM B input.
+__host__ __device__ __forceinline__ size_t btile_offset_nt(int nt, int r, int kb, int Nt, int NKC) {
   const int kc = kb >> 7, w = kb & 127;
   return (static_cast<size_t>(nt) * NKC + kc) * Nt * 128 + (w >> 4) * Nt * 16 + (r >> 3) * 128 + (r & 7) * 16 +
          (w & 15);
 }
+// Byte offset of element (token t, K byte kb) in a tiled GEMM B input.
+__host__ __device__ __forceinline__ size_t btile_offset(int t, int kb, int Nt, int NKC) {
+  const int nt = t / Nt;
+  return btile_offset_nt(nt, t - nt * Nt, kb, Nt, NKC);
+}
+// Float offset of element (row r of n-tile nt, feature f) in the tiled residual h.
+__host__ __device__ __forceinline__ size_t htile_offset_nt(int nt, int r, int f, int Nt, int KB) {
+  return ((static_cast<size_t>(nt) * KB + (f >> 6)) * Nt + r) * 64 + (f & 63);
+}
 // Float offset of element (token t, feature f) in the tiled residual h.
 __host__ __device__ __forceinline__ size_t htile_offset(int t, int f, int Nt, int KB) {
-  const int nt = t / Nt, r = t - nt * Nt;
-  return ((static_cast<size_t>(nt) * KB + (f >> 6)) * Nt + r) * 64 + (f & 63);
+  const int nt = t / Nt;
+  return htile_offset_nt(nt, t - nt * Nt, f, Nt, KB);
 }
 
 struct GemmArgs {
@@ -105,6 +127,7 @@ struct GemmArgs {
   // split-K exchange (S > 1): fp32 partial tiles [NT][MB][S][Nt][128], L2-resident scratch
   float* xscratch;
   unsigned* status;
+  DevExtents ext;
 };
 
 struct AttnArgs {
@@ -123,6 +146,7 @@ struct AttnArgs {
   int o_rowmajor;              // 1: o is bf16 [B][H][Hq*dh] row-major instead of the tiled operand layout
   unsigned* status;            // device status word (timeouts), or nullptr
   int umma;                    // 1: tcgen05 kernel over GQA-group tiles; 0: warp-MMA kernel per query head
+  uint64_t o_extent;           // bytes of o (checked builds)
 };
 
 // Key chunks of the split-KV attention over S keys: at most 16 (one cluster), each a multiple

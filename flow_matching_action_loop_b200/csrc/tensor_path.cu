@@ -124,6 +124,7 @@ struct TensorPath {
   int exec_mode = FR_EXEC_AUTO;
   unsigned long long wait_limit_ns = 2000000000ull;
   std::map<std::pair<int, int>, int> pk_fits;   // (B, P) -> the kernel is resident on every SM (1) or not (0)
+  DevExtents ext_limit{};        // checked builds: smaller extents declared by fr_debug_limit_extent (0: none)
 };
 
 namespace {
@@ -298,6 +299,31 @@ void tile_projection_w4(const ProjLayout& L, RowFn rowsrc, std::vector<uint8_t>&
   }
 }
 
+// Extents of the buffers the kernels store into (checked builds verify every store against them).
+DevExtents extents(const TensorPath* tp, int B) {
+  const fr_config& c = tp->c;
+  DevExtents e;
+  e.h = static_cast<uint64_t>(tp->tok_alloc) * tp->KB * 64;
+  e.q = static_cast<uint64_t>(c.B_max) * c.Hq * c.H * c.dh;
+  e.kv = tp->tb.kv_layer_bytes / 2;
+  e.xbuf = tp->fp8 ? 0 : static_cast<uint64_t>(tp->tok_alloc) * tp->qkv.NKC * KCB;
+  e.obuf = static_cast<uint64_t>(tp->tok_alloc) * tp->o.NKC * KCB;
+  e.ubuf = static_cast<uint64_t>(tp->tok_alloc) * tp->dn.NKC * KCB;
+  e.ssq = static_cast<uint64_t>(tp->T_pad) * tp->ssq_ld;
+  e.x = static_cast<uint64_t>(B) * c.H * c.A;
+  const DevExtents& m = tp->ext_limit;
+  auto lim = [](uint64_t& v, uint64_t l) { if (l && l < v) v = l; };
+  lim(e.h, m.h);
+  lim(e.q, m.q);
+  lim(e.kv, m.kv);
+  lim(e.xbuf, m.xbuf);
+  lim(e.obuf, m.obuf);
+  lim(e.ubuf, m.ubuf);
+  lim(e.ssq, m.ssq);
+  lim(e.x, m.x);
+  return e;
+}
+
 GemmArgs base_args(const TensorPath* tp, const StepPlan& p, const ProjLayout& L, const GemmPlan& g, int layer,
                    size_t w_off) {
   const fr_config& c = tp->c;
@@ -321,6 +347,7 @@ GemmArgs base_args(const TensorPath* tp, const StepPlan& p, const ProjLayout& L,
   a.ssq_parts = tp->MBd;
   a.xscratch = tp->xscratch;
   a.status = tp->tb.status;
+  a.ext = extents(tp, p.B);
   return a;
 }
 
@@ -395,6 +422,7 @@ int record_layer(TensorPath* tp, const StepPlan& p, int l, const LayerVectors& v
   at.xscratch = tp->xscratch;
   at.status = tp->tb.status;
   at.umma = p.attn_umma;
+  at.o_extent = extents(tp, p.B).obuf;
   if ((e = launch_attention_tc(at, p.B, s, true)) != cudaSuccess) return cuda_fail(e, "attention launch");
   // O projection + residual (+ sum of squares for the pre-MLP norm)
   GemmArgs og = base_args(tp, p, tp->o, p.o, l, o_off);
@@ -677,6 +705,7 @@ bool make_pk_args(TensorPath* tp, int B, int P, const float* x0, float* x_out, p
   a.ctr = tp->pk_ctr;
   a.status = tp->tb.status;
   a.flag_limit_ns = tp->wait_limit_ns;
+  a.ext = extents(tp, B);
   return true;
 }
 
@@ -1017,6 +1046,21 @@ int tensor_path_exec(TensorPath* tp, int B, int P) {
 int tensor_path_set_exec_mode(TensorPath* tp, int mode) {
   tp->exec_mode = mode;
   return FR_OK;
+}
+
+int tensor_path_limit_extent(TensorPath* tp, const char* name, unsigned long long elems) {
+  DevExtents& m = tp->ext_limit;
+  const struct { const char* n; uint64_t* v; } f[] = {{"h", &m.h},       {"q", &m.q},       {"kv", &m.kv},
+                                                       {"xbuf", &m.xbuf}, {"obuf", &m.obuf}, {"ubuf", &m.ubuf},
+                                                       {"ssq", &m.ssq},   {"x", &m.x}};
+  for (const auto& e : f)
+    if (std::strcmp(name, e.n) == 0) {
+      *e.v = elems;
+      evict_to(tp, 0);   // captured graphs carry the extents they were recorded with
+      return FR_OK;
+    }
+  set_error("fr_debug_limit_extent: unknown buffer '%s' (h, q, kv, xbuf, obuf, ubuf, ssq, x)", name);
+  return FR_ERR_ARG;
 }
 
 int tensor_path_set_wait_limit(TensorPath* tp, unsigned long long ns) {

@@ -50,6 +50,7 @@ int tensor_path_launches(TensorPath* tp, int B, int P);
 int tensor_path_exec(TensorPath* tp, int B, int P);              // FR_EXEC_GRAPH or FR_EXEC_PERSISTENT
 int tensor_path_set_exec_mode(TensorPath* tp, int mode);         // FR_EXEC_*
 int tensor_path_set_wait_limit(TensorPath* tp, unsigned long long ns);
+int tensor_path_limit_extent(TensorPath* tp, const char* name, unsigned long long elems);   // checked builds
 // prefix-role paths: the pass over B x P embedded tokens (device bf16 [B][P][D]) into the KV cache
 int tensor_path_prefill(TensorPath* tp, const void* emb, int B, int P, cudaStream_t s);
 int tensor_path_set_graph_capacity(TensorPath* tp, int capacity);   // capacity >= 1

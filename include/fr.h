@@ -277,6 +277,22 @@ int fr_exec_mode(const fr_handle* h, int B);
  * then undefined and the next call starts afresh.  Errors: FR_ERR_ARG (NULL, limit above 10 s). */
 int fr_set_wait_limit(fr_handle* h, uint64_t limit_ns);
 
+/* ---- device bounds checks (checked builds) ---- */
+
+/* 1 if this library was built with device bounds checks (-DFR_DEVICE_CHECKS), else 0.  In a checked
+ * build every store of the GEMM epilogues, of the attention kernels and of the persistent kernel
+ * verifies its index against its buffer's extent; an index at or past it latches FR_ERR_DEVICE in the
+ * status word (fr_sync_status / fr_ops_sync_status: where-code and index) and the store is skipped.
+ * No counterpart in the pages: it stands in for a memory checker in debugging. */
+int fr_device_checks(void);
+
+/* fr_debug_limit_extent -- checked builds: declare a smaller extent (elements of the buffer's type;
+ * bytes for the tiled operands) for one of the handle's buffers "h", "q", "kv", "xbuf", "obuf",
+ * "ubuf", "ssq" or "x" (0 restores the real one), so that the bounds checks can be exercised without
+ * any access leaving the real allocation.  Cached graphs are dropped.  Errors: FR_ERR_ARG (NULL,
+ * unknown name), FR_ERR_STATE (not a tensor-path handle), FR_ERR_UNSUPPORTED (not a checked build). */
+int fr_debug_limit_extent(fr_handle* h, const char* buffer, uint64_t elems);
+
 /*
  * fr_prefill -- the prefix pass, the step before the loop (FlashRT walkthrough, component 5:
  * the attention sites of the Pi0.5 model; the loop's per-layer KV cache is the backbone's keys and
