@@ -1043,6 +1043,7 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
 // same rank-order log-sum-exp weights as the flash-decoding merge.
 
 constexpr int UA_SUB = 64;        // keys per sub-chunk
+constexpr float UA_RESCALE = 8.f; // the softmax reference moves when the row maximum grows by more (log2 units)
 constexpr int UA_THREADS = 128;   // one thread per query row of the tile
 
 struct UAttnGeom {
@@ -1176,8 +1177,10 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   bool failed = false;
   for (int sc = 0; sc < nsub; ++sc) {
     const int bf = sc & 1;
-    if (sc >= 2) {   // K(sc) and V(sc) were issued in the two previous sub-chunks
-      cp_async_wait_all();
+    if (sc >= 2) {   // K(sc) and V(sc) were issued in the two previous sub-chunks; K(sc+1), committed
+                     // last, may stay in flight
+      if (sc + 1 < nsub) cp_async_wait_one_pending();
+      else cp_async_wait_all();
       fence_proxy_async_smem();
       __syncthreads();
     }
@@ -1197,10 +1200,6 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
       break;
     }
     tc_fence_after();
-    if (sc + 2 < nsub) {   // K buffer bf is free once S(sc) is done
-      load_k(sc + 2, Kbuf(bf), 2);
-      cp_async_commit();
-    }
     uint32_t sv[UA_SUB];
 #pragma unroll
     for (int u = 0; u < UA_SUB / 16; ++u) tmem_ld16_nowait(tS + lane_base + 16 * u, sv + 16 * u);
@@ -1227,7 +1226,16 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
         cp_async_commit();
       }
     }
-    const float corr = exp2f(m_run - mx);
+    if (sc + 2 < nsub) {   // K buffer bf is free once S(sc) is done; committed after V(sc+1)
+      load_k(sc + 2, Kbuf(bf), 2);
+      cp_async_commit();
+    }
+    // The reference of the exponentials moves only when the row maximum has grown by more than
+    // UA_RESCALE (log2 units): P stays below 2^UA_RESCALE, the sum and O are relative to the same
+    // reference, and O / l is unchanged; O in tensor memory is rescaled only when a row's reference
+    // moves, which after the first sub-chunks is rare.
+    const float ref = (mx > m_run + UA_RESCALE) ? mx : m_run;
+    const float corr = exp2f(m_run - ref);
     float psum = 0.f;
     uint8_t* prow = dsm + gm.p_off + (tid >> 3) * 128 + (tid & 7) * 16;   // P row, K-major [128 x 64]
 #pragma unroll
@@ -1235,14 +1243,14 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
       float p[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        p[e] = exp2f(__uint_as_float(sv[kk * 8 + e]) - mx);
+        p[e] = exp2f(__uint_as_float(sv[kk * 8 + e]) - ref);
         psum += p[e];
       }
       *reinterpret_cast<uint4*>(prow + kk * 2048) =
           make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
     }
     l_run = l_run * corr + psum;
-    m_run = mx;
+    m_run = ref;
     if (sc > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
 #pragma unroll 1
       for (int c0 = 0; c0 < DH; c0 += 16) {
