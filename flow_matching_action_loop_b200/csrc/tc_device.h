@@ -49,9 +49,15 @@ __device__ __forceinline__ uint8_t to_e4m3(float v) {
   return static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
 }
 
+// GeLU in its tanh form, 0.5·g·(1 + tanh z) with z = sqrt(2/pi)·(g + 0.044715·g³), evaluated as
+// g·σ(2z) = g / (1 + e^{-2z}) (the identity 1 + tanh z = 2 / (1 + e^{-2z})): one exponential and one
+// fast division instead of a full tanh. The exponent is capped at 80 so the denominator stays far
+// below the range where the fast division returns 0 for a finite quotient; there the result is
+// already below 1e-33·|g|.
 __device__ __forceinline__ float gelu_tanh(float g) {
   const float c0 = 0.7978845608028654f;   // sqrt(2/pi)
-  return 0.5f * g * (1.f + tanhf(c0 * (g + 0.044715f * g * g * g)));
+  const float t = fminf(-2.f * c0 * (g + 0.044715f * g * g * g), 80.f);
+  return __fdividef(g, 1.f + __expf(t));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
