@@ -150,14 +150,14 @@ __host__ __device__ __forceinline__ int nk_max_of(const GemmArgs& a) { return (a
 // Bytes of the main loop and epilogue regions; the QKV epilogue's RoPE stage ([H][64] (cos, sin)
 // pairs of the m-block) follows them.
 __host__ __device__ __forceinline__ uint32_t gemm_rope_off(int Nt, int stages, int b_kind, int fp8, int S, int nk,
-                                                          int w4, int epi_kind) {
+                                                          int w4, int epi_kind, int red_tok) {
   const GemmGeom g = gemm_geom(Nt, stages, b_kind, fp8, S, nk, w4, 1);   // kc0 odd: the larger group count
   const uint32_t kel = fp8 ? KCB : KCB / 2;
   const uint32_t main = g.gamma_off + (b_kind == B_NORM ? static_cast<uint32_t>(nk) * kel * 4u : 0u);
   const uint32_t TS = (Nt + S - 1) / S;
-  // split-K slices (S > 1) or the S == 1 accumulator rows overlay the ring; the residual epilogue's
-  // prefetched h rows (S > 1) follow at recv_off
-  uint32_t epi = S > 1 ? static_cast<uint32_t>(S) * TS * BM * 4u : static_cast<uint32_t>(Nt) * RED_LD * 4u;
+  // split-K slices (S > 1) or one pass of the S == 1 accumulator rows overlay the ring; the residual
+  // epilogue's prefetched h rows (S > 1) follow at recv_off
+  uint32_t epi = S > 1 ? static_cast<uint32_t>(S) * TS * BM * 4u : static_cast<uint32_t>(red_tok) * RED_LD * 4u;
   if (S > 1 && epi_kind == EPI_RESID && g.recv_off + 2u * TS * 64u * 4u > epi) epi = g.recv_off + 2u * TS * 64u * 4u;
   return ((main > epi ? main : epi) + 15u) & ~15u;
 }
@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   const uint32_t tacc = sh.tmem_base;
   // QKV: (cos, sin) of this m-block's 64 rotate-half pairs at every action position, staged while
   // the previous kernel runs (the tables are static); read by the epilogue after the main loop
-  float2* rope_sh = reinterpret_cast<float2*>(dsm + gemm_rope_off(Nt, stages, NORM ? B_NORM : B_ROWS, FP8, S, nk_max_of(a), W4, EPI));
+  float2* rope_sh = reinterpret_cast<float2*>(dsm + gemm_rope_off(Nt, stages, NORM ? B_NORM : B_ROWS, FP8, S, nk_max_of(a), W4, EPI, a.red_tok));
   if (EPI == EPI_QKV && mb < a.MB_rot && warp >= 2) {   // warps 2-7: the producer and MMA warps go on
     const int half = a.dh >> 1;
     const bool by_tok = rope_by_token(a.H, Nt);
@@ -452,34 +452,36 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   tc_fence_after();
   __syncthreads();
   if (tid == 0) TL(3);
-  float* red = reinterpret_cast<float*>(dsm);   // S == 1: [Nt][RED_LD], aliases the drained ring
+  float* red = reinterpret_cast<float*>(dsm);   // S == 1: [red_tok][RED_LD], aliases the drained ring
   float* xs = (S > 1) ? a.xscratch + (static_cast<size_t>(nt) * a.MB + mb) * S * Nt * BM : nullptr;
   const int t_hi = min(Nt, a.T - n0);           // valid tokens of this n-tile
-  {
-    // TMEM -> red (S == 1) or the scratch (S > 1) by all eight warps: warp w reads the lane
-    // quadrant w % 4; warps 0-3 take the first half of the token columns, warps 4-7 the rest
+  // TMEM columns [cb, ce) -> red (S == 1: row stride RED_LD, from token cb) or the split-K staging
+  // (S > 1: valid tokens, row stride BM) by all eight warps: warp w reads the lane quadrant w % 4;
+  // warps 0-3 take the first half of the columns, warps 4-7 the rest
+  auto stage_tmem = [&](int cb, int ce) {
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    const int hc = ((Nt >> 4) + 1) / 2 * 16;
-    const int cbeg = warp < 4 ? 0 : hc, cend = warp < 4 ? min(hc, Nt) : Nt;
-    for (int c0 = cbeg; c0 < cend; c0 += 64) {   // up to 4 loads in flight, one wait
-      uint32_t v[4][16];
+    const int hc = (((ce - cb) >> 4) + 1) / 2 * 16;
+    const int cbeg = cb + (warp < 4 ? 0 : hc), cend = warp < 4 ? min(cb + hc, ce) : ce;
+    for (int c0 = cbeg; c0 < cend; c0 += 32) {   // up to 2 loads in flight, one wait
+      uint32_t v[2][16];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < 2; ++u)
         if (c0 + 16 * u < cend) tmem_ld16_nowait(tacc + (static_cast<uint32_t>(q * 32) << 16) + c0 + 16 * u, v[u]);
       tmem_wait_ld();
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < 2; ++u)
         if (c0 + 16 * u < cend)
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int tok = c0 + 16 * u + j;
-            if (S == 1) red[tok * RED_LD + row] = __uint_as_float(v[u][j]);
+            if (S == 1) red[(tok - cb) * RED_LD + row] = __uint_as_float(v[u][j]);
             else if (tok < t_hi) red[tok * BM + row] = __uint_as_float(v[u][j]);   // staged for one bulk store
           }
     }
-  }
+  };
   if (S > 1) {   // the partial tile (valid tokens) into the scratch with one bulk store
+    stage_tmem(0, Nt);
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
@@ -505,12 +507,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
                  &sh.xbar);
     }
     if (!mbar_wait(&sh.xbar, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0x500);
-  } else {
-    __syncthreads();
   }
   if (tid == 0) TL(4);
 
   const float al = a.alpha ? *a.alpha : 1.0f;
+  int rbase = 0;   // S == 1: first token of the staged pass
   // Split-K sums of N (2 or 4) consecutive accumulator rows of one token over the cluster, in
   // rank order (deterministic), times the dequantisation / deferred-rstd scale.
   auto vals = [&](int tok, int row, float* out, auto n_tag) {
@@ -520,7 +521,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
 #pragma unroll
     for (int e = 0; e < N; ++e) acc[e] = 0.f;
     if (S == 1) {   // no split: the accumulator rows as staged (wide tiles: no per-rank predication)
-      const float* p = red + tok * RED_LD + row;
+      const float* p = red + (tok - rbase) * RED_LD + row;
 #pragma unroll
       for (int e = 0; e < N; ++e) out[e] = p[e] * sc;
       return;
@@ -557,6 +558,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   // features; EPU tokens per warp have their independent loads issued before any is used.
   constexpr int EPU = 4;
 
+  // S == 1: the accumulator is staged and written in passes of red_tok tokens (a wide tile's
+  // staging then fits half of an SM's shared memory and two CTAs share the SM)
+  const int npass = S == 1 ? (Nt + a.red_tok - 1) / a.red_tok : 1;
+  for (int pass = 0; pass < npass; ++pass) {
+  const int ebeg = S == 1 ? pass * a.red_tok : tok0;
+  const int eend = S == 1 ? min(Nt, ebeg + a.red_tok) : tok1;
+  if (S == 1) {
+    if (pass > 0) __syncthreads();   // every warp is done with the previous pass's rows
+    stage_tmem(ebeg, eend);
+    tc_fence_before();
+    __syncthreads();
+    rbase = ebeg;
+  }
   if (EPI == EPI_RESID) {
     const int row = lane * 4;
     const int f = mb * BM + row;
@@ -567,13 +581,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
     if (a.xb_out && fok) g4 = *reinterpret_cast<const float4*>(a.xb_gamma + f);
     float4 gt = make_float4(1.f, 1.f, 1.f, 1.f);   // adaptive RMSNorm: gated residual update
     if (a.gate && fok) gt = *reinterpret_cast<const float4*>(a.gate + f);
-    for (int tb = tok0 + warp; tb < tok1; tb += 8 * EPU) {
+    for (int tb = ebeg + warp; tb < eend; tb += 8 * EPU) {
       float4 hold[EPU];
       float acc[EPU][4];
 #pragma unroll
       for (int u = 0; u < EPU; ++u) {
         const int tok = tb + 8 * u, t = n0 + tok;
-        if (tok < tok1 && t < a.T && fok) {
+        if (tok < eend && t < a.T && fok) {
           hold[u] = (S > 1) ? *reinterpret_cast<const float4*>(hst + ((row >> 6) * gm.TS + (tok - tok0)) * 64 + (row & 63))
                             : *reinterpret_cast<const float4*>(a.h_out + htile_offset_nt(nt, tok, f, Nt, a.KB));
           vals(tok, row, acc[u], Four{});
@@ -582,7 +596,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
 #pragma unroll
       for (int u = 0; u < EPU; ++u) {
         const int tok = tb + 8 * u, t = n0 + tok;
-        if (tok >= tok1 || t >= a.T) break;   // warp-uniform
+        if (tok >= eend || t >= a.T) break;   // warp-uniform
         float sq = 0.f;
         if (fok) {
           const float4 hv = make_float4(hold[u].x + gt.x * acc[u][0], hold[u].y + gt.y * acc[u][1],
@@ -609,7 +623,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       bg = *reinterpret_cast<const float2*>(a.bias + f);
       bu = *reinterpret_cast<const float2*>(a.bias + a.F + f);
     }
-    for (int tok = tok0 + warp; tok < tok1; tok += 8) {
+    for (int tok = ebeg + warp; tok < eend; tok += 8) {
       const int t = n0 + tok;
       if (t >= a.T || f >= a.F) break;
       float g[2], up[2];
@@ -642,12 +656,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         blo = *reinterpret_cast<const float2*>(a.bias + head * a.dh + j);
         bhi = *reinterpret_cast<const float2*>(a.bias + head * a.dh + j + half);
       }
-      for (int tb = tok0 + warp; tb < tok1; tb += 8 * EPU) {
+      for (int tb = ebeg + warp; tb < eend; tb += 8 * EPU) {
         float2 cs[EPU], sn[EPU];
 #pragma unroll
         for (int u = 0; u < EPU; ++u) {
           const int tok = tb + 8 * u, t = n0 + tok;
-          if (tok < tok1 && t < a.T) {
+          if (tok < eend && t < a.T) {
             const float4 r4 = *reinterpret_cast<const float4*>(rope_sh + (rope_by_token(a.H, Nt) ? tok : t % a.H) * 64 + p);   // pairs p, p+1
             cs[u] = make_float2(r4.x, r4.z);
             sn[u] = make_float2(r4.y, r4.w);
@@ -656,7 +670,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
 #pragma unroll
         for (int u = 0; u < EPU; ++u) {
           const int tok = tb + 8 * u, t = n0 + tok;
-          if (tok >= tok1 || t >= a.T) break;
+          if (tok >= eend || t >= a.T) break;
           const int b = t / a.H, i = t % a.H, pos = a.P + i;
           float lo[2], hi[2];
           vals(tok, p, lo, Two{});
@@ -683,7 +697,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       const int g = idx / a.dh, d = idx % a.dh;
       float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);   // adaptive RMSNorm shift, W b
       if (a.bias) bv = *reinterpret_cast<const float4*>(a.bias + (a.Hq + a.Hkv) * a.dh + idx);
-      for (int tok = tok0 + warp; tok < tok1; tok += 8) {
+      for (int tok = ebeg + warp; tok < eend; tok += 8) {
         const int t = n0 + tok;
         if (t >= a.T) break;
         const int b = t / a.H, i = t % a.H, pos = a.P + i;
@@ -699,6 +713,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       }
     }
   }
+  }   // passes
   if (tid == 0) TL(9);
   __syncthreads();
   if (tid == 0) TL(5);
@@ -1047,30 +1062,34 @@ constexpr float UA_RESCALE = 8.f; // the softmax reference moves when the row ma
 constexpr int UA_THREADS = 128;   // one thread per query row of the tile
 
 struct UAttnGeom {
-  uint32_t q_off, k_off0, k_off1, v_off0, v_off1, p_off, total, tcols, o_col;
+  uint32_t q_off, k_off0, k_off1, v_off0, v_off1, p_off0, p_off1, w_off, total, tcols, o_col;
 };
 
+// Shared memory: Q tile, two K and two V sub-chunk buffers, two P tiles.  Tensor memory: the
+// scores of two sub-chunks at columns 0 and UA_SUB, O at o_col.  The merge stage of the split-KV
+// case (at most 144 rows of dh + 4 floats) and the merge weights after it overlay the buffers.
 __host__ __device__ __forceinline__ UAttnGeom uattn_geom(int dh) {
   UAttnGeom g;
-  const uint32_t q = 128u * dh * 2u, kv = static_cast<uint32_t>(UA_SUB) * dh * 2u;
+  const uint32_t q = 128u * dh * 2u, kv = static_cast<uint32_t>(UA_SUB) * dh * 2u, pt = 128u * UA_SUB * 2u;
   g.q_off = 0;
   g.k_off0 = q;
   g.v_off0 = q + kv;
   g.k_off1 = q + 2 * kv;
   g.v_off1 = q + 3 * kv;
-  g.p_off = q + 4 * kv;
-  g.total = g.p_off + 128u * UA_SUB * 2u;
-  g.tcols = dh == 256 ? 512u : (dh == 128 ? 256u : 128u);   // S at column 0, O at o_col
-  g.o_col = dh == 256 ? 256u : (dh == 128 ? 128u : 64u);
+  g.p_off0 = q + 4 * kv;
+  g.p_off1 = g.p_off0 + pt;
+  g.total = g.p_off1 + pt;
+  g.w_off = 144u * (dh + 4) * 4u;
+  g.tcols = dh == 256 ? 512u : 256u;
+  g.o_col = dh == 256 ? 256u : 128u;
   return g;
 }
 
 template <int DH>
 __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_constant__ AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t dsm[];
-  __shared__ uint64_t bar_s, bar_o, stage_bar;
+  __shared__ uint64_t bar_s[2], bar_o[2], stage_bar;
   __shared__ uint32_t tmem_base;
-  __shared__ float w_sh[16][128];   // merge weight of chunk s for owned row rr (C <= 16)
   __shared__ float inv_den[128];
   TL_DECL
   TL_BEGIN(20);
@@ -1097,8 +1116,10 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   const __nv_bfloat16* qg = a.q + ((static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G) * a.H + row0) * DH;
 
   if (tid == 0) {
-    mbar_init(&bar_s, 1);
-    mbar_init(&bar_o, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_s[i], 1);
+      mbar_init(&bar_o[i], 1);
+    }
     mbar_init(&stage_bar, 1);
     fence_mbar_init();
   }
@@ -1173,36 +1194,43 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   if (tid == 0) TL(2);
 
   const float sl2 = a.scale * 1.4426950408889634f;   // scores in log2 units
+  // S(j) = Q K(j)^T into score buffer j & 1 (thread 0; K(j) resident and made visible)
+  auto issue_s = [&](int j) {
+    tc_fence_after();
+    const uint32_t qa = smem_u32(dsm + gm.q_off), ka = smem_u32(Kbuf(j & 1));
+#pragma unroll
+    for (int k = 0; k < DH / 16; ++k)
+      mma_bf16(tS + (j & 1) * UA_SUB, smem_desc(qa + k * 2 * 2048, 2048, 128),
+               smem_desc(ka + k * 2 * (UA_SUB * 16), UA_SUB * 16, 128), IDESC_S, k > 0);
+    mma_commit(&bar_s[j & 1]);
+  };
+  if (tid == 0) {
+    issue_s(0);
+    if (nsub > 1) issue_s(1);
+  }
+  // Sub-chunk sc: the scores of sc + 1 are computed by the tensor core while the threads run the
+  // softmax of sc, and O += P(sc) V(sc) runs while they start on sc + 1 (P has two buffers).
+  // Copy groups in issue order: sub-chunk sc commits K(sc + 2), then V(sc + 1).
   float m_run = -INFINITY, l_run = 0.f;
-  bool failed = false;
+  bool ok = true, failed = false;
   for (int sc = 0; sc < nsub; ++sc) {
     const int bf = sc & 1;
-    if (sc >= 2) {   // K(sc) and V(sc) were issued in the two previous sub-chunks; K(sc+1), committed
-                     // last, may stay in flight
-      if (sc + 1 < nsub) cp_async_wait_one_pending();
+    if (sc >= 1 && sc + 1 < nsub) {   // K(sc+1) landed (V(sc), committed after it, may stay in flight)
+      if (sc >= 2) cp_async_wait_one_pending();
       else cp_async_wait_all();
       fence_proxy_async_smem();
       __syncthreads();
+      if (tid == 0) issue_s(sc + 1);
     }
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t qa = smem_u32(dsm + gm.q_off), ka = smem_u32(Kbuf(bf));
-#pragma unroll
-      for (int k = 0; k < DH / 16; ++k)
-        mma_bf16(tS, smem_desc(qa + k * 2 * 2048, 2048, 128), smem_desc(ka + k * 2 * (UA_SUB * 16), UA_SUB * 16, 128),
-                 IDESC_S, k > 0);
-      mma_commit(&bar_s);
-    }
-    const bool got_s = mbar_wait(&bar_s, sc & 1, WAIT_LIMIT_NS);
-    if (__syncthreads_or(!got_s)) {
-      if (tid == 0) report_timeout(a.status, 0x700);
-      failed = true;
-      break;
-    }
+    ok &= mbar_wait(&bar_s[bf], (sc >> 1) & 1, WAIT_LIMIT_NS);
     tc_fence_after();
+    if (sc + 2 < nsub) {   // S(sc) has read K buffer bf
+      load_k(sc + 2, Kbuf(bf), 2);
+      cp_async_commit();
+    }
     uint32_t sv[UA_SUB];
 #pragma unroll
-    for (int u = 0; u < UA_SUB / 16; ++u) tmem_ld16_nowait(tS + lane_base + 16 * u, sv + 16 * u);
+    for (int u = 0; u < UA_SUB / 16; ++u) tmem_ld16_nowait(tS + bf * UA_SUB + lane_base + 16 * u, sv + 16 * u);
     tmem_wait_ld();
     const int kb = sc * UA_SUB;
     float mx = m_run;
@@ -1213,31 +1241,16 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
       sv[jj] = __float_as_uint(v);
       mx = fmaxf(mx, v);
     }
-    if (sc > 0) {   // O(sc-1) complete: P may be overwritten and O rescaled
-      const bool got_o = mbar_wait(&bar_o, (sc - 1) & 1, WAIT_LIMIT_NS);
-      if (__syncthreads_or(!got_o)) {
-        if (tid == 0) report_timeout(a.status, 0x701);
-        failed = true;
-        break;
-      }
-      tc_fence_after();
-      if (sc + 1 < nsub) {   // V buffer of sub-chunk sc-1 is free: V(sc+1) goes there
-        load_v(sc + 1, Vbuf((sc + 1) & 1), 2);
-        cp_async_commit();
-      }
-    }
-    if (sc + 2 < nsub) {   // K buffer bf is free once S(sc) is done; committed after V(sc+1)
-      load_k(sc + 2, Kbuf(bf), 2);
-      cp_async_commit();
-    }
     // The reference of the exponentials moves only when the row maximum has grown by more than
     // UA_RESCALE (log2 units): P stays below 2^UA_RESCALE, the sum and O are relative to the same
     // reference, and O / l is unchanged; O in tensor memory is rescaled only when a row's reference
     // moves, which after the first sub-chunks is rare.
     const float ref = (mx > m_run + UA_RESCALE) ? mx : m_run;
     const float corr = exp2f(m_run - ref);
+    const bool resc = sc > 0 && __any_sync(0xffffffffu, corr != 1.f);
+    // P buffer bf was last read by O += P V of sub-chunk sc - 2, complete since sub-chunk sc - 1
     float psum = 0.f;
-    uint8_t* prow = dsm + gm.p_off + (tid >> 3) * 128 + (tid & 7) * 16;   // P row, K-major [128 x 64]
+    uint8_t* prow = dsm + (bf ? gm.p_off1 : gm.p_off0) + (tid >> 3) * 128 + (tid & 7) * 16;   // K-major [128 x 64]
 #pragma unroll
     for (int kk = 0; kk < UA_SUB / 8; ++kk) {
       float p[8];
@@ -1251,7 +1264,9 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
     }
     l_run = l_run * corr + psum;
     m_run = ref;
-    if (sc > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
+    if (resc) {   // O(sc-1) complete before this warp's rows of O are rescaled
+      ok &= mbar_wait(&bar_o[bf ^ 1], ((sc - 1) >> 1) & 1, WAIT_LIMIT_NS);
+      tc_fence_after();
 #pragma unroll 1
       for (int c0 = 0; c0 < DH; c0 += 16) {
         uint32_t ov[16];
@@ -1263,21 +1278,34 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
       }
       tmem_wait_st();
     }
-    fence_proxy_async_smem();   // P (generic-proxy stores) -> visible to the tensor core
+    if (sc >= 2) {   // V(sc), committed in sub-chunk sc - 1 before K(sc + 2)
+      if (sc + 2 < nsub) cp_async_wait_one_pending();
+      else cp_async_wait_all();
+    }
+    fence_proxy_async_smem();   // P and V (generic-proxy / cp.async writes) -> visible to the tensor core
     tc_fence_before();
-    __syncthreads();
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) report_timeout(a.status, 0x700);
+      failed = true;
+      break;
+    }
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t pa = smem_u32(dsm + gm.p_off), va = smem_u32(Vbuf(bf));
+      const uint32_t pa = smem_u32(dsm + (bf ? gm.p_off1 : gm.p_off0)), va = smem_u32(Vbuf(bf));
 #pragma unroll
       for (int k = 0; k < UA_SUB / 16; ++k)
         mma_bf16(tO, smem_desc(pa + k * 2 * 2048, 2048, 128), smem_desc(va + k * 2 * (DH * 16), DH * 16, 128), IDESC_O,
                  (sc > 0 || k > 0) ? 1u : 0u);
-      mma_commit(&bar_o);
+      mma_commit(&bar_o[bf]);
+    }
+    if (sc >= 1 && sc + 1 < nsub) {   // O(sc-1) done: V buffer bf ^ 1 and P buffer bf ^ 1 are free
+      ok &= mbar_wait(&bar_o[bf ^ 1], ((sc - 1) >> 1) & 1, WAIT_LIMIT_NS);
+      load_v(sc + 1, Vbuf(bf ^ 1), 2);
+      cp_async_commit();
     }
   }
   if (!failed) {
-    const bool got = mbar_wait(&bar_o, (nsub - 1) & 1, WAIT_LIMIT_NS);
+    const bool got = ok && mbar_wait(&bar_o[(nsub - 1) & 1], ((nsub - 1) >> 1) & 1, WAIT_LIMIT_NS);
     if (__syncthreads_or(!got)) {
       if (tid == 0) report_timeout(a.status, 0x702);
       failed = true;
@@ -1380,6 +1408,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   }
   if (!mbar_wait(&stage_bar, 0, WAIT_LIMIT_NS) && tid == 0) report_timeout(a.status, 0x703);
   if (tid == 0) TL(4);
+  float* w_sh = reinterpret_cast<float*>(dsm + gm.w_off);   // [16][128]: merge weight of chunk s2, owned row
   const int nr = r_hi - r_lo;
   if (tid < nr) {
     float mv[16], lv[16];
@@ -1402,7 +1431,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
     for (int s2 = 0; s2 < 16; ++s2) {
       if (s2 < C) {
         const float e = exp2f(mv[s2] - M);
-        w_sh[s2][tid] = e;
+        w_sh[s2 * 128 + tid] = e;
         den += e * lv[s2];
       }
     }
@@ -1420,7 +1449,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
 #pragma unroll
     for (int s2 = 0; s2 < 16; ++s2)
       if (s2 < C) {
-        const float w = w_sh[s2][rq];
+        const float w = w_sh[s2 * 128 + rq];
         const float* src = stage + (static_cast<size_t>(s2) * RM + rq) * OLD + d0;
 #pragma unroll
         for (int e = 0; e < 16; e += 4) {
@@ -1625,8 +1654,9 @@ __global__ void k_wait_selftest(unsigned* status, unsigned long long limit_ns) {
 
 }  // namespace
 
-size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4, int epi, int H, int xb) {
-  return gemm_rope_off(Nt, stages, b_kind, fp8, S, nk, w4, epi) + gemm_stage_bytes(epi, fp8, Nt, S, H, xb);
+size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4, int epi, int H, int xb,
+                       int red_tok) {
+  return gemm_rope_off(Nt, stages, b_kind, fp8, S, nk, w4, epi, red_tok) + gemm_stage_bytes(epi, fp8, Nt, S, H, xb);
 }
 
 size_t gemm_scratch_bytes(int NT, int MB, int S, int Nt) {
@@ -1683,6 +1713,19 @@ int max_dynamic_smem() {
   return optin - static_cast<int>(fa.sharedSizeBytes);
 }
 
+int pair_dynamic_smem() {
+  int dev = 0, per_sm = 0, reserved = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  int stat = 0;
+  for (int epi : {EPI_QKV, EPI_RESID, EPI_GELU}) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, gemm_kernel(epi, 0, 0, 0)) == cudaSuccess) stat = std::max(stat, static_cast<int>(fa.sharedSizeBytes));
+  }
+  return per_sm / 2 - reserved - stat;
+}
+
 // One instantiation per (epilogue, operand type, B-operand kind, 4-bit weights) in use.
 const void* gemm_kernel(int epi, int fp8, int norm, int w4) {
   if (w4) {
@@ -1710,7 +1753,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int n_tiles, cudaStream_t s, bool 
   const void* f = gemm_kernel(a.epi, a.fp8, a.b_kind == B_NORM, a.w4);
   if (!f) return cudaErrorInvalidValue;
   return launch_ex(f, dim3(a.S, n_tiles, a.MB), dim3(GEMM_THREADS),
-                   gemm_smem_bytes(a.Nt, a.stages, a.b_kind, a.fp8, a.S, nk_max, a.w4, a.epi, a.H, a.xb_out != nullptr), s,
+                   gemm_smem_bytes(a.Nt, a.stages, a.b_kind, a.fp8, a.S, nk_max, a.w4, a.epi, a.H, a.xb_out != nullptr, a.red_tok), s,
                    pdl, a.S, args);
 }
 

@@ -124,6 +124,7 @@ struct GemmArgs {
   int NKC_u;
   const float* s_a_out;    // fp8: scale of the down-projection input
   int F;
+  int red_tok;             // S == 1: tokens per epilogue staging pass (Nt, or fewer so that two CTAs share an SM)
   // split-K exchange (S > 1): fp32 partial tiles [NT][MB][S][Nt][128], L2-resident scratch
   float* xscratch;
   unsigned* status;
@@ -223,7 +224,8 @@ cudaError_t launch_final_tc(const FinalArgs& a, cudaStream_t s, bool pdl);
 cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s);
 cudaError_t launch_to_bf16_t(const float* src, __nv_bfloat16* dst, int rows, int cols, cudaStream_t s);
 cudaError_t launch_wait_selftest(unsigned* status, unsigned long long limit_ns, cudaStream_t s);
-size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4, int epi, int H, int xb);
+size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4, int epi, int H, int xb,
+                       int red_tok);
 size_t gemm_scratch_bytes(int NT, int MB, int S, int Nt);
 size_t attn_scratch_bytes(int B, int Hq, int C, int H, int dh);
 size_t attn_smem_bytes(int H, int dh, int KC, int C, int umma);
@@ -231,6 +233,7 @@ const void* inproj_kernel_ptr();
 const void* final_kernel_ptr();
 cudaError_t tc_kernels_init();    // function attributes (smem opt-in, carveout, non-portable clusters)
 int max_dynamic_smem();           // dynamic shared memory a GEMM CTA may use
+int pair_dynamic_smem();          // dynamic shared memory of a GEMM CTA that shares its SM with another
 
 }  // namespace tc
 }  // namespace fr

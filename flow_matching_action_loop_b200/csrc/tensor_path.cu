@@ -58,6 +58,7 @@ ProjLayout make_layout(int rows, int K, int elem, int w4) {
 
 struct GemmPlan {
   int S = 1, stages = 1;
+  int red_tok = 0;   // S == 1: tokens per epilogue staging pass (0: the whole tile)
 };
 
 struct StepPlan {
@@ -91,6 +92,7 @@ struct TensorPath {
   TensorPathBuffers tb{};
   int nsm = 148;
   int max_dyn = 0;
+  int max_dyn2 = 0;              // dynamic shared memory of a GEMM CTA when two share an SM
   int fp8 = 0, elem = 2;
   int w4 = 0;                    // 4-bit weights dequantised in the GEMM (activations as bf16)
   int T_max = 0, T_pad = 0, MBd = 0, MB_rot = 0;
@@ -192,9 +194,28 @@ void init_sizes(TensorPath* tp, const fr_config& c) {
 // exchange, and weight chunks that must stream after the dependency wait.  Wider tiles are
 // throughput-bound: no split-K unless the tiles leave most SMs idle.
 GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, int epi, int H, int xb, int nsm,
-                     int max_dyn) {
+                     int max_dyn, int max_dyn2) {
   GemmPlan best;
+  auto smem = [&](int S, int stages, int chunks, int red_tok) {
+    return gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, epi, H, xb, red_tok);
+  };
   if (Nt > 64) {
+    // More than one wave of unsplit tiles: two CTAs per SM, so that one CTA's epilogue runs while
+    // the other's MMAs do (a ring of at least two slots; the accumulator staged in passes of half
+    // the tile when the whole tile does not fit).
+    if (tiles > nsm && max_dyn2 > 0) {
+      const int chunks = NKC;
+      for (int red_tok : {Nt, static_cast<int>(align_up(ceil_div(Nt, 2), 16))}) {
+        int stages = std::min(chunks, MAX_STAGES);
+        while (stages > 2 && smem(1, stages, chunks, red_tok) > static_cast<size_t>(max_dyn2)) --stages;
+        if (stages >= 2 && smem(1, stages, chunks, red_tok) <= static_cast<size_t>(max_dyn2)) {
+          best.S = 1;
+          best.stages = stages;
+          best.red_tok = red_tok;
+          return best;
+        }
+      }
+    }
     // throughput-bound tiles: split K in two only when the tiles leave most SMs idle; fall back to
     // the other split when the preferred one does not fit shared memory
     const int pref = (tiles * 2 <= nsm && NKC >= 2) ? 2 : 1;
@@ -202,11 +223,10 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, in
       if (S > NKC) continue;
       const int chunks = ceil_div(NKC, S);
       int stages = std::min(chunks, MAX_STAGES);
-      while (stages > 1 && gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, epi, H, xb) > static_cast<size_t>(max_dyn))
-        --stages;
+      while (stages > 1 && smem(S, stages, chunks, Nt) > static_cast<size_t>(max_dyn)) --stages;
       best.S = S;
       best.stages = stages;
-      if (gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, epi, H, xb) <= static_cast<size_t>(max_dyn)) return best;
+      if (smem(S, stages, chunks, Nt) <= static_cast<size_t>(max_dyn)) return best;
     }
     return best;   // nothing fits: the launch reports it
   }
@@ -215,8 +235,8 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, in
   for (int S = 1; S <= 16 && S <= NKC; ++S) {
     const int chunks = ceil_div(NKC, S);
     int stages = std::min(chunks, MAX_STAGES);
-    while (stages > 1 && gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, epi, H, xb) > cap) --stages;
-    if (gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, epi, H, xb) > static_cast<size_t>(max_dyn)) continue;
+    while (stages > 1 && smem(S, stages, chunks, Nt) > cap) --stages;
+    if (smem(S, stages, chunks, Nt) > static_cast<size_t>(max_dyn)) continue;
     const int waves = ceil_div(tiles * S, nsm);
     const double cost = waves * (1.0 + (S > 1 ? 1.0 : 0.0) + 0.3 * (chunks - stages) + 0.05 * chunks);
     if (cost < best_cost - 1e-9) {
@@ -241,13 +261,13 @@ StepPlan make_plan(const TensorPath* tp, int B, int P, int H) {
   p.Nt = static_cast<int>(align_up(ceil_div(p.T, p.NT), 16));
   const int norm_kind = tp->fp8 ? B_NORM : B_ROWS;   // bf16: the producer wrote bf16(h*gamma) already
   p.qkv = choose_plan(tp->qkv.MB * p.NT, tp->qkv.NKC, p.Nt, norm_kind, tp->fp8, tp->w4, EPI_QKV, H, 0, tp->nsm,
-                      tp->max_dyn);
+                      tp->max_dyn, tp->max_dyn2);
   p.o = choose_plan(tp->o.MB * p.NT, tp->o.NKC, p.Nt, B_ROWS, tp->fp8, tp->w4, EPI_RESID, H, !tp->fp8, tp->nsm,
-                    tp->max_dyn);
+                    tp->max_dyn, tp->max_dyn2);
   p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, norm_kind, tp->fp8, tp->w4, EPI_GELU, H, 0, tp->nsm,
-                     tp->max_dyn);
+                     tp->max_dyn, tp->max_dyn2);
   p.dn = choose_plan(tp->dn.MB * p.NT, tp->dn.NKC, p.Nt, B_ROWS, tp->fp8, tp->w4, EPI_RESID, H, !tp->fp8, tp->nsm,
-                     tp->max_dyn);
+                     tp->max_dyn, tp->max_dyn2);
   // the warp-MMA attention kernel holds at most 128 query rows per head: longer sequences take tcgen05
   p.attn_umma = attn_plan(P + H, attn_tiles(B, c.Hq, c.Hkv, H), tp->nsm, p.attn_C, p.attn_KC, H > 128);
   return p;
@@ -335,6 +355,7 @@ GemmArgs base_args(const TensorPath* tp, const StepPlan& p, const ProjLayout& L,
   a.Nout = L.rows;
   a.S = g.S;
   a.stages = g.stages;
+  a.red_tok = g.red_tok > 0 ? g.red_tok : p.Nt;
   a.fp8 = tp->fp8;
   a.w4 = tp->w4;
   a.Wscale = tp->w4 ? reinterpret_cast<const uint16_t*>(a.W + L.sc_off) : nullptr;
@@ -802,7 +823,7 @@ bool tensor_path_supports(const fr_config& c) {
   if (c.F % 64 != 0) return false;                            // gate/up pairs fill whole m-blocks
   if (c.D % 16 != 0 || (c.Hq * c.dh) % 16 != 0) return false; // 16-byte operand rows
   if (c.D > 2048) return false;                               // per-token kernels keep a row in registers
-  if (attn_smem_bytes(c.H, c.dh, 64, 1, 1) > 218 * 1024) return false;   // B200: 227 KB less the static part
+  if (attn_smem_bytes(c.H, c.dh, 64, 1, 1) > 226 * 1024) return false;   // B200: 227 KB less the static part
   if (c.role == FR_ROLE_PREFIX) return c.dtype != FR_DTYPE_FP8;   // longer sequences: tcgen05 attention
   if (c.H > 128) return false;                                // one attention row-group pass per warp
   if (c.A > 64) return false;
@@ -862,6 +883,7 @@ void device_params(TensorPath* tp) {
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&tp->nsm, cudaDevAttrMultiProcessorCount, dev);
   tc_kernels_init();
   tp->max_dyn = max_dynamic_smem();
+  tp->max_dyn2 = pair_dynamic_smem();
 }
 
 size_t tensor_path_bytes(const fr_config& c) {
@@ -899,6 +921,7 @@ int tensor_path_create(const fr_config& c, const TensorPathBuffers& b, TensorPat
     return cuda_fail(e, "tensor path init");
   }
   tp->max_dyn = max_dynamic_smem();
+  tp->max_dyn2 = pair_dynamic_smem();
   tp->gains_host.assign(static_cast<size_t>(c.L) * 2 * c.D, 1.f);
   *out = tp;
   return FR_OK;
