@@ -65,9 +65,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// two e4m3 codes (saturating, round to nearest even) in one conversion: a in the low byte
+__device__ __forceinline__ uint32_t pack_e4m3x2(float a, float b) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+
 __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
-  return static_cast<uint32_t>(to_e4m3(a)) | (static_cast<uint32_t>(to_e4m3(b)) << 8) |
-         (static_cast<uint32_t>(to_e4m3(c)) << 16) | (static_cast<uint32_t>(to_e4m3(d)) << 24);
+  return pack_e4m3x2(a, b) | (pack_e4m3x2(c, d) << 16);
 }
 
 

@@ -73,7 +73,6 @@ __device__ unsigned g_tl_cap = 0;
 #endif
 
 constexpr int CONV_THREADS = 192;                                  // warps 2-7
-constexpr int CONV_ITEMS = (NT_MAX * 8 + CONV_THREADS - 1) / CONV_THREADS;
 
 __device__ __forceinline__ void conv_sync() { asm volatile("bar.sync 1, 192;" ::: "memory"); }
 
@@ -109,9 +108,8 @@ __host__ __device__ __forceinline__ GemmGeom gemm_geom(int Nt, int stages, int b
                                                        int w4 = 0, int kc0 = 0) {
   GemmGeom g;
   g.a_bytes = BM * KCB;
-  g.raw_bytes = (b_kind == B_NORM) ? static_cast<uint32_t>(Nt) * 256u * (fp8 ? 2u : 1u) : 0u;
-  const uint32_t tile = static_cast<uint32_t>(Nt) * KCB;
-  g.breg = tile > g.raw_bytes ? tile : g.raw_bytes;
+  g.raw_bytes = 0;   // B_NORM converters read h from global memory straight into the operand tile
+  g.breg = static_cast<uint32_t>(Nt) * KCB;
   g.slot = g.a_bytes + g.breg;
   g.ring = g.slot * static_cast<uint32_t>(stages);
   g.TS = (Nt + S - 1) / S;
@@ -235,11 +233,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       auto issue_b = [&](int i) {
         const int s = i % stages;
         uint8_t* bdst = b_slot(s);
-        if (norm) {
-          const int kb = (kc0 + i) * (FP8 ? 2 : 1);
-          mbar_arrive_expect_tx(&sh.raw_b[s], gm.raw_bytes);
-          bulk_g2s(bdst, a.h + (static_cast<size_t>(nt) * a.KB + kb) * Nt * 64, gm.raw_bytes, &sh.raw_b[s]);
-        } else {
+        if (!norm) {   // B_NORM: the converters fill the slot
           const uint32_t tb = static_cast<uint32_t>(Nt) * KCB;
           mbar_arrive_expect_tx(&sh.full_b[s], tb);
           bulk_g2s(bdst, a.act + (static_cast<size_t>(nt) * a.NKC + kc0 + i) * tb, tb, &sh.full_b[s]);
@@ -298,7 +292,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         const int s = i % stages;
         const uint32_t par = (i / stages) & 1;
         if (!mbar_wait(W4 ? &sh.raw_a[s] : &sh.full_a[s], par, WAIT_LIMIT_NS) ||
-            !mbar_wait(norm ? &sh.raw_b[s] : &sh.full_b[s], par, WAIT_LIMIT_NS))
+            (!norm && !mbar_wait(&sh.full_b[s], par, WAIT_LIMIT_NS)))
           report_timeout(a.status, 0x101);
       }
     }
@@ -393,52 +387,49 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
     if (W4)
       for (int i = pre_a; i < nk; ++i) convert_a(i);
     const float inv_sa = (norm && FP8) ? 1.0f / *a.s_a : 1.0f;
+    // B_NORM (e4m3 operands): chunk i's operand tile e4m3(h * rstd * gamma / s_a) from the residual rows
+    // in global memory (just written by the previous kernel, in L2), CONV_BATCH 16-feature items per
+    // thread in flight; a slot is refilled once the MMAs of the chunk it held are done.
+    static_assert(!NORM || FP8, "the normalising B operand is the e4m3 one");
+    constexpr int CONV_BATCH = 4;
+    const int jt = st & 7;   // this thread's 16-feature piece of every token row (CONV_THREADS % 8 == 0)
     for (int i = 0; i < (norm ? nk : 0); ++i) {
       const int s = i % stages;
-      if (!mbar_wait(&sh.raw_b[s], (i / stages) & 1, WAIT_LIMIT_NS)) {
+      if (i >= stages && !mbar_wait(&sh.empty[s], ((i / stages) - 1) & 1, WAIT_LIMIT_NS)) {
         report_timeout(a.status, 0x300);
         break;
       }
       uint8_t* breg = b_slot(s);
-      const float* raw = reinterpret_cast<const float*>(breg);
-      const float* gch = gsm + i * kel;
-      uint4 res[CONV_ITEMS];
+      const int kb = (kc0 + i) * 2;   // two 64-feature blocks of h per 128-input chunk
+      const float* hsrc = a.h + ((static_cast<size_t>(nt) * a.KB + kb + (jt >> 2)) * Nt) * 64 + (jt & 3) * 16;
+      float4 gv[4];
 #pragma unroll
-      for (int q = 0; q < CONV_ITEMS; ++q) {
-        const int it = st + q * CONV_THREADS;
-        if (it < Nt * 8) {
-          const int r = it >> 3, j = it & 7;
-          const float rs = sh.rstd[r];
-          if (!FP8) {
-            const float* p = raw + static_cast<size_t>(r) * 64 + j * 8;
-            const float4 h0 = *reinterpret_cast<const float4*>(p), h1 = *reinterpret_cast<const float4*>(p + 4);
-            const float4 g0 = *reinterpret_cast<const float4*>(gch + j * 8);
-            const float4 g1 = *reinterpret_cast<const float4*>(gch + j * 8 + 4);
-            res[q] = make_uint4(pack_bf16x2(h0.x * rs * g0.x, h0.y * rs * g0.y),
-                                pack_bf16x2(h0.z * rs * g0.z, h0.w * rs * g0.w),
-                                pack_bf16x2(h1.x * rs * g1.x, h1.y * rs * g1.y),
-                                pack_bf16x2(h1.z * rs * g1.z, h1.w * rs * g1.w));
-          } else {
-            const float* p = raw + (static_cast<size_t>(j >> 2) * Nt + r) * 64 + (j & 3) * 16;
-            uint32_t w4[4];
+      for (int u = 0; u < 4; ++u) gv[u] = *reinterpret_cast<const float4*>(gsm + i * kel + jt * 16 + 4 * u);
+      for (int it0 = st; it0 < Nt * 8; it0 += CONV_BATCH * CONV_THREADS) {
+        float4 hv[CONV_BATCH][4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float4 hv = *reinterpret_cast<const float4*>(p + 4 * u);
-              const float4 gv = *reinterpret_cast<const float4*>(gch + j * 16 + 4 * u);
-              const float m = rs * inv_sa;
-              w4[u] = pack_e4m3x4(hv.x * gv.x * m, hv.y * gv.y * m, hv.z * gv.z * m, hv.w * gv.w * m);
-            }
-            res[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        for (int q = 0; q < CONV_BATCH; ++q) {
+          const int it = it0 + q * CONV_THREADS;
+          if (it < Nt * 8) {
+            const float4* p = reinterpret_cast<const float4*>(hsrc + static_cast<size_t>(it >> 3) * 64);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) hv[q][u] = p[u];
           }
         }
-      }
-      conv_sync();   // every raw value of this slot has been read before the tile overwrites it
 #pragma unroll
-      for (int q = 0; q < CONV_ITEMS; ++q) {
-        const int it = st + q * CONV_THREADS;
-        if (it < Nt * 8) {
-          const int r = it >> 3, j = it & 7;
-          *reinterpret_cast<uint4*>(breg + j * Nt * 16 + (r >> 3) * 128 + (r & 7) * 16) = res[q];
+        for (int q = 0; q < CONV_BATCH; ++q) {
+          const int it = it0 + q * CONV_THREADS;
+          if (it < Nt * 8) {
+            const int r = it >> 3;
+            const float m = sh.rstd[r] * inv_sa;
+            uint32_t w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              w[u] = pack_e4m3x4(hv[q][u].x * gv[u].x * m, hv[q][u].y * gv[u].y * m, hv[q][u].z * gv[u].z * m,
+                                 hv[q][u].w * gv[u].w * m);
+            *reinterpret_cast<uint4*>(breg + jt * Nt * 16 + (r >> 3) * 128 + (r & 7) * 16) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
       }
       fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core (async proxy)
@@ -638,7 +629,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         const size_t uo = btile_offset_nt(nt, tok, f, Nt, a.NKC_u);
         if (in_bounds(a.status, uo + 1, a.ext.ubuf, 0x9004))
           *reinterpret_cast<uint16_t*>(a.u_out + uo) =
-              static_cast<uint16_t>(to_e4m3(u0 * inv) | (static_cast<uint32_t>(to_e4m3(u1 * inv)) << 8));
+              static_cast<uint16_t>(pack_e4m3x2(u0 * inv, u1 * inv));
       } else {
         const size_t uo = btile_offset_nt(nt, tok, 2 * f, Nt, a.NKC_u);
         if (in_bounds(a.status, uo + 3, a.ext.ubuf, 0x9004))
@@ -1099,7 +1090,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   constexpr uint32_t IDESC_O = idesc_f32acc(FMT_BF16, 128, DH) | IDESC_B_MN_MAJOR;
   const UAttnGeom gm = uattn_geom(DH);
   const int c = blockIdx.x, y = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int G = a.Hq / a.Hkv;            // query heads per KV head (consecutive heads)
   const int R = G * a.H;                 // query rows of one KV group
   const int MT = (R + 127) >> 7;
@@ -1134,34 +1125,36 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t tS = tmem_base, tO = tmem_base + gm.o_col;
 
-  // K rows of sub-chunk sc into a K-major operand tile [64 keys x DH] (16-byte core columns
-  // of 64 x 16 B); which: 0 = prefix keys (and zero rows past the chunk), 1 = action keys, 2 = all.
-  auto load_k = [&](int sc, uint8_t* Kb, int which) {
-    const int kb0 = key0 + sc * UA_SUB;
-    for (int it = tid; it < UA_SUB * VPR; it += UA_THREADS) {
-      const int n = it % UA_SUB, j = it / UA_SUB;   // consecutive threads: consecutive keys
-      const int key = kb0 + n;
-      const bool valid = sc * UA_SUB + n < nkeys;
-      const bool mine = which == 2 || (which == 0 ? (key < a.P || !valid) : (key >= a.P && valid));
-      if (mine)
-        cp_async16(Kb + j * (UA_SUB * 16) + (n >> 3) * 128 + (n & 7) * 16,
-                   kg + static_cast<size_t>(valid ? key : 0) * DH + j * 8, valid);
-    }
+  // K and V rows of sub-chunk sc: thread t copies key t % 64 of the sub-chunk, its 16-byte columns
+  // t / 64, t / 64 + 2, ... (consecutive threads: consecutive keys), with per-thread base addresses and
+  // constant strides.  K lands as the K-major operand of S = Q K^T ([16-byte column][64 keys][16 B]);
+  // V as stored ([key][DH]) is the MN-major operand of O += P V (core matrices of 8 keys x 16 B, 8-key
+  // groups DH*16 bytes apart).  which: 0 = prefix keys (and zero rows past the chunk), 1 = action keys,
+  // 2 = all.
+  constexpr int CPT = UA_SUB * VPR / UA_THREADS;   // 16-byte copies per thread per sub-chunk and operand
+  const int kn = tid & (UA_SUB - 1), kj0 = tid / UA_SUB;
+  auto key_of = [&](int sc, int which, int& key, bool& valid) {
+    key = key0 + sc * UA_SUB + kn;
+    valid = sc * UA_SUB + kn < nkeys;
+    return which == 2 || (which == 0 ? (key < a.P || !valid) : (key >= a.P && valid));
   };
-  // V rows of sub-chunk sc as stored ([key][DH], DH contiguous): the MN-major B operand of
-  // O += P V, core matrices of 8 keys x 16 B; 8-key groups DH*16 bytes apart.
+  auto load_k = [&](int sc, uint8_t* Kb, int which) {
+    int key;
+    bool valid;
+    if (!key_of(sc, which, key, valid)) return;
+    uint8_t* dst = Kb + kj0 * (UA_SUB * 16) + kn * 16;
+    const __nv_bfloat16* src = kg + static_cast<size_t>(valid ? key : 0) * DH + kj0 * 8;
+#pragma unroll
+    for (int m = 0; m < CPT; ++m) cp_async16(dst + m * 2 * (UA_SUB * 16), src + m * 16, valid);
+  };
   auto load_v = [&](int sc, uint8_t* Vb, int which) {
-    const int kb0 = key0 + sc * UA_SUB;
-    for (int it = tid; it < UA_SUB * VPR; it += UA_THREADS) {
-      const int k8 = it & 7, j = (it >> 3) % VPR, kq = (it >> 3) / VPR;
-      const int n = kq * 8 + k8;
-      const int key = kb0 + n;
-      const bool valid = sc * UA_SUB + n < nkeys;
-      const bool mine = which == 2 || (which == 0 ? (key < a.P || !valid) : (key >= a.P && valid));
-      if (mine)
-        cp_async16(Vb + kq * (DH * 16) + j * 128 + k8 * 16, vg + static_cast<size_t>(valid ? key : 0) * DH + j * 8,
-                   valid);
-    }
+    int key;
+    bool valid;
+    if (!key_of(sc, which, key, valid)) return;
+    uint8_t* dst = Vb + (kn >> 3) * (DH * 16) + kj0 * 128 + (kn & 7) * 16;
+    const __nv_bfloat16* src = vg + static_cast<size_t>(valid ? key : 0) * DH + kj0 * 8;
+#pragma unroll
+    for (int m = 0; m < CPT; ++m) cp_async16(dst + m * 2 * 128, src + m * 16, valid);
   };
   auto Kbuf = [&](int bf) { return dsm + (bf ? gm.k_off1 : gm.k_off0); };
   auto Vbuf = [&](int bf) { return dsm + (bf ? gm.v_off1 : gm.v_off0); };
@@ -1182,10 +1175,12 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
     load_k(1, Kbuf(1), 1);
     load_v(1, Vbuf(1), 1);
   }
-  for (int it = tid; it < 128 * VPR; it += UA_THREADS) {   // Q tile, K-major [128 rows x DH]
-    const int r = it & 127, j = it >> 7;
-    cp_async16(dsm + gm.q_off + j * 2048 + (r >> 3) * 128 + (r & 7) * 16,
-               qg + static_cast<size_t>(r < Rv ? r : 0) * DH + j * 8, r < Rv);
+  {   // Q tile, K-major [16-byte column][128 rows][16 B]: thread t copies row t
+    const bool qv = tid < Rv;
+    uint8_t* dst = dsm + gm.q_off + tid * 16;
+    const __nv_bfloat16* src = qg + static_cast<size_t>(qv ? tid : 0) * DH;
+#pragma unroll
+    for (int j = 0; j < VPR; ++j) cp_async16(dst + j * 2048, src + j * 8, qv);
   }
   cp_async_commit();
   cp_async_wait_all();

@@ -190,7 +190,7 @@ void init_sizes(TensorPath* tp, const fr_config& c) {
 
 // Split-K / ring choice for one projection.  Batch-1-like tiles (Nt <= 64) are latency-bound:
 // at most one CTA per SM (so the next kernel's CTAs can become resident and prefetch their
-// weights next to it) and at most ~120 KB of shared memory; the cost counts waves, the split-K
+// weights next to it) and at most half an SM's shared memory; the cost counts waves, the split-K
 // exchange, and weight chunks that must stream after the dependency wait.  Wider tiles are
 // throughput-bound: no split-K unless the tiles leave most SMs idle.
 GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, int epi, int H, int xb, int nsm,
@@ -230,7 +230,8 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, in
     }
     return best;   // nothing fits: the launch reports it
   }
-  const size_t cap = std::min<size_t>(static_cast<size_t>(max_dyn), 120 * 1024);
+  // at most half an SM's shared memory, so that the next kernel's CTAs fit beside this one's
+  const size_t cap = std::min<size_t>(static_cast<size_t>(max_dyn), max_dyn2 > 0 ? static_cast<size_t>(max_dyn2) : 110 * 1024);
   double best_cost = 1e30;
   for (int S = 1; S <= 16 && S <= NKC; ++S) {
     const int chunks = ceil_div(NKC, S);
