@@ -60,6 +60,14 @@ __device__ __forceinline__ float gelu_tanh(float g) {
   return __fdividef(g, 1.f + __expf(t));
 }
 
+// 2^x by the multi-function unit's approximation (relative error about 2^-22, subnormal results
+// flushed to zero, 2^-inf = 0); softmax weights are rounded to bf16 right after.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -1050,7 +1050,9 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
 
 constexpr int UA_SUB = 64;        // keys per sub-chunk
 constexpr float UA_RESCALE = 8.f; // the softmax reference moves when the row maximum grows by more (log2 units)
-constexpr int UA_THREADS = 128;   // one thread per query row of the tile
+constexpr int UA_THREADS = 256;   // two per query row of the tile: warps w and w + 4 share the row's lane
+                                  // quadrant of tensor memory, each takes half of the keys' exponentials
+                                  // and half of the O columns
 
 struct UAttnGeom {
   uint32_t q_off, k_off0, k_off1, v_off0, v_off1, p_off0, p_off1, w_off, total, tcols, o_col;
@@ -1082,6 +1084,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   __shared__ uint64_t bar_s[2], bar_o[2], stage_bar;
   __shared__ uint32_t tmem_base;
   __shared__ float inv_den[128];
+  __shared__ float l_sh[2][128];         // the two halves' softmax sums of each row
   TL_DECL
   TL_BEGIN(20);
   constexpr int OLD = DH + 4;            // fp32 row stride of the partial-O rows
@@ -1091,6 +1094,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   const UAttnGeom gm = uattn_geom(DH);
   const int c = blockIdx.x, y = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int row = tid & 127, hh = tid >> 7;   // this thread's query row of the tile and half
   const int G = a.Hq / a.Hkv;            // query heads per KV head (consecutive heads)
   const int R = G * a.H;                 // query rows of one KV group
   const int MT = (R + 127) >> 7;
@@ -1122,16 +1126,17 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   __syncthreads();
   tc_fence_after();
   grid_dep_launch();
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   const uint32_t tS = tmem_base, tO = tmem_base + gm.o_col;
 
   // K and V rows of sub-chunk sc: thread t copies key t % 64 of the sub-chunk, its 16-byte columns
-  // t / 64, t / 64 + 2, ... (consecutive threads: consecutive keys), with per-thread base addresses and
+  // t / 64, t / 64 + 4, ... (consecutive threads: consecutive keys), with per-thread base addresses and
   // constant strides.  K lands as the K-major operand of S = Q K^T ([16-byte column][64 keys][16 B]);
   // V as stored ([key][DH]) is the MN-major operand of O += P V (core matrices of 8 keys x 16 B, 8-key
   // groups DH*16 bytes apart).  which: 0 = prefix keys (and zero rows past the chunk), 1 = action keys,
   // 2 = all.
   constexpr int CPT = UA_SUB * VPR / UA_THREADS;   // 16-byte copies per thread per sub-chunk and operand
+  constexpr int JS = UA_THREADS / UA_SUB;          // 16-byte column step between a thread's copies
   const int kn = tid & (UA_SUB - 1), kj0 = tid / UA_SUB;
   auto key_of = [&](int sc, int which, int& key, bool& valid) {
     key = key0 + sc * UA_SUB + kn;
@@ -1145,7 +1150,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
     uint8_t* dst = Kb + kj0 * (UA_SUB * 16) + kn * 16;
     const __nv_bfloat16* src = kg + static_cast<size_t>(valid ? key : 0) * DH + kj0 * 8;
 #pragma unroll
-    for (int m = 0; m < CPT; ++m) cp_async16(dst + m * 2 * (UA_SUB * 16), src + m * 16, valid);
+    for (int m = 0; m < CPT; ++m) cp_async16(dst + m * JS * (UA_SUB * 16), src + m * JS * 8, valid);
   };
   auto load_v = [&](int sc, uint8_t* Vb, int which) {
     int key;
@@ -1154,7 +1159,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
     uint8_t* dst = Vb + (kn >> 3) * (DH * 16) + kj0 * 128 + (kn & 7) * 16;
     const __nv_bfloat16* src = vg + static_cast<size_t>(valid ? key : 0) * DH + kj0 * 8;
 #pragma unroll
-    for (int m = 0; m < CPT; ++m) cp_async16(dst + m * 2 * 128, src + m * 16, valid);
+    for (int m = 0; m < CPT; ++m) cp_async16(dst + m * JS * 128, src + m * JS * 8, valid);
   };
   auto Kbuf = [&](int bf) { return dsm + (bf ? gm.k_off1 : gm.k_off0); };
   auto Vbuf = [&](int bf) { return dsm + (bf ? gm.v_off1 : gm.v_off0); };
@@ -1175,12 +1180,12 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
     load_k(1, Kbuf(1), 1);
     load_v(1, Vbuf(1), 1);
   }
-  {   // Q tile, K-major [16-byte column][128 rows][16 B]: thread t copies row t
-    const bool qv = tid < Rv;
-    uint8_t* dst = dsm + gm.q_off + tid * 16;
-    const __nv_bfloat16* src = qg + static_cast<size_t>(qv ? tid : 0) * DH;
+  {   // Q tile, K-major [16-byte column][128 rows][16 B]: the two threads of a row copy half of it each
+    const bool qv = row < Rv;
+    uint8_t* dst = dsm + gm.q_off + row * 16 + hh * (VPR / 2) * 2048;
+    const __nv_bfloat16* src = qg + static_cast<size_t>(qv ? row : 0) * DH + hh * (VPR / 2) * 8;
 #pragma unroll
-    for (int j = 0; j < VPR; ++j) cp_async16(dst + j * 2048, src + j * 8, qv);
+    for (int j = 0; j < VPR / 2; ++j) cp_async16(dst + j * 2048, src + j * 8, qv);
   }
   cp_async_commit();
   cp_async_wait_all();
@@ -1228,14 +1233,17 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
     for (int u = 0; u < UA_SUB / 16; ++u) tmem_ld16_nowait(tS + bf * UA_SUB + lane_base + 16 * u, sv + 16 * u);
     tmem_wait_ld();
     const int kb = sc * UA_SUB;
-    float mx = m_run;
+    // Both threads of a row take the maximum over all 64 raw scores (four independent chains: with
+    // few warps per scheduler the chains are the latency); the scale sl2 > 0 is applied after it
+    float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    if (kb + UA_SUB > nkeys) {   // the chunk's last sub-chunk: keys past it do not count
 #pragma unroll
-    for (int jj = 0; jj < UA_SUB; ++jj) {
-      float v = __uint_as_float(sv[jj]) * sl2;
-      if (kb + jj >= nkeys) v = -INFINITY;
-      sv[jj] = __float_as_uint(v);
-      mx = fmaxf(mx, v);
+      for (int jj = 0; jj < UA_SUB; ++jj)
+        if (kb + jj >= nkeys) sv[jj] = __float_as_uint(-INFINITY);
     }
+#pragma unroll
+    for (int jj = 0; jj < UA_SUB; ++jj) mq[jj & 3] = fmaxf(mq[jj & 3], __uint_as_float(sv[jj]));
+    const float mx = fmaxf(m_run, fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sl2);   // log2 units
     // The reference of the exponentials moves only when the row maximum has grown by more than
     // UA_RESCALE (log2 units): P stays below 2^UA_RESCALE, the sum and O are relative to the same
     // reference, and O / l is unchanged; O in tensor memory is rescaled only when a row's reference
@@ -1243,27 +1251,33 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
     const float ref = (mx > m_run + UA_RESCALE) ? mx : m_run;
     const float corr = exp2f(m_run - ref);
     const bool resc = sc > 0 && __any_sync(0xffffffffu, corr != 1.f);
-    // P buffer bf was last read by O += P V of sub-chunk sc - 2, complete since sub-chunk sc - 1
-    float psum = 0.f;
-    uint8_t* prow = dsm + (bf ? gm.p_off1 : gm.p_off0) + (tid >> 3) * 128 + (tid & 7) * 16;   // K-major [128 x 64]
+    // P buffer bf was last read by O += P V of sub-chunk sc - 2, complete since sub-chunk sc - 1; this
+    // thread writes keys 32*hh .. 32*hh + 31 of its row, 2^(s*sl2 - ref)
+    float ps[4] = {0.f, 0.f, 0.f, 0.f};
+    uint8_t* prow = dsm + (bf ? gm.p_off1 : gm.p_off0) + (row >> 3) * 128 + (row & 7) * 16;   // K-major [128 x 64]
+    auto expo = [&](auto half) {   // compile-time key range, so that sv stays in registers
+      constexpr int K0 = decltype(half)::value * (UA_SUB / 2);
 #pragma unroll
-    for (int kk = 0; kk < UA_SUB / 8; ++kk) {
-      float p[8];
+      for (int k2 = 0; k2 < UA_SUB / 16; ++k2) {
+        float p[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        p[e] = exp2f(__uint_as_float(sv[kk * 8 + e]) - ref);
-        psum += p[e];
+        for (int e = 0; e < 8; ++e) {
+          p[e] = ex2_approx(fmaf(__uint_as_float(sv[K0 + k2 * 8 + e]), sl2, -ref));
+          ps[e & 3] += p[e];
+        }
+        *reinterpret_cast<uint4*>(prow + (K0 / 8 + k2) * 2048) = make_uint4(
+            pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
       }
-      *reinterpret_cast<uint4*>(prow + kk * 2048) =
-          make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
-    }
-    l_run = l_run * corr + psum;
+    };
+    if (hh == 0) expo(std::integral_constant<int, 0>{});   // warp-uniform
+    else expo(std::integral_constant<int, 1>{});
+    l_run = l_run * corr + ((ps[0] + ps[1]) + (ps[2] + ps[3]));   // this half's keys
     m_run = ref;
     if (resc) {   // O(sc-1) complete before this warp's rows of O are rescaled
       ok &= mbar_wait(&bar_o[bf ^ 1], ((sc - 1) >> 1) & 1, WAIT_LIMIT_NS);
       tc_fence_after();
 #pragma unroll 1
-      for (int c0 = 0; c0 < DH; c0 += 16) {
+      for (int c0 = hh * (DH / 2); c0 < (hh + 1) * (DH / 2); c0 += 16) {   // this thread's half of O
         uint32_t ov[16];
         tmem_ld16_nowait(tO + lane_base + c0, ov);
         tmem_wait_ld();
@@ -1299,6 +1313,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
       cp_async_commit();
     }
   }
+  l_sh[hh][row] = l_run;
   if (!failed) {
     const bool got = ok && mbar_wait(&bar_o[(nsub - 1) & 1], ((nsub - 1) >> 1) & 1, WAIT_LIMIT_NS);
     if (__syncthreads_or(!got)) {
@@ -1310,8 +1325,10 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   tc_fence_after();
   if (tid == 0) TL(3);
 
-  const int rr = row0 + tid;                         // this thread's row of the group
-  const bool rv = tid < Rv && !failed;
+  __syncthreads();                                   // l_sh complete (also on the failure paths)
+  const float l_tot = l_sh[0][row] + l_sh[1][row];
+  const int rr = row0 + row;                         // this thread's row of the group
+  const bool rv = row < Rv && !failed;
   const int jq = g * G + rr / a.H, iq = rr % a.H;    // query head, action row
   const float inv_sa = (a.fp8 && a.s_a) ? 1.0f / *a.s_a : 1.0f;
   // writes 16 consecutive output features d0.. of row (token t, head jq)
@@ -1341,9 +1358,9 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   };
 
   if (C == 1) {
-    const float inv = 1.0f / l_run;
+    const float inv = 1.0f / l_tot;
 #pragma unroll 1
-    for (int c0 = 0; c0 < DH; c0 += 16) {
+    for (int c0 = hh * (DH / 2); c0 < (hh + 1) * (DH / 2); c0 += 16) {   // this thread's half of the row
       uint32_t ov[16];
       tmem_ld16_nowait(tO + lane_base + c0, ov);
       tmem_wait_ld();
@@ -1356,7 +1373,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
     // this chunk's (O, max, sum) row into the scratch, [B][Hq][C][H][OLD]
     float* xrow = a.xscratch + ((static_cast<size_t>(b) * a.Hq + jq) * C + c) * a.H * OLD + static_cast<size_t>(iq) * OLD;
 #pragma unroll 1
-    for (int c0 = 0; c0 < DH; c0 += 16) {
+    for (int c0 = hh * (DH / 2); c0 < (hh + 1) * (DH / 2); c0 += 16) {   // this thread's half of the row
       uint32_t ov[16];
       tmem_ld16_nowait(tO + lane_base + c0, ov);
       tmem_wait_ld();
@@ -1366,7 +1383,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
           *reinterpret_cast<float4*>(xrow + c0 + e) = make_float4(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1]),
                                                                   __uint_as_float(ov[e + 2]), __uint_as_float(ov[e + 3]));
     }
-    if (rv) *reinterpret_cast<float4*>(xrow + DH) = make_float4(m_run, l_run, 0.f, 0.f);
+    if (rv && hh == 0) *reinterpret_cast<float4*>(xrow + DH) = make_float4(m_run, l_tot, 0.f, 0.f);
     // the peers fetch these rows with bulk copies (async proxy): order this thread's generic-proxy
     // stores before them, ahead of the cluster barrier's release
     fence_proxy_async_global();

@@ -183,7 +183,7 @@ void init_sizes(TensorPath* tp, const fr_config& c) {
   tp->KB = ceil_div(c.D, BM) * 2;
   tp->ssq_ld = static_cast<int>(align_up(tp->MBd, 4));
   const int nt_max = ceil_div(tp->T_max, NT_MAX);
-  tp->tok_alloc = tp->T_max + 16 * nt_max;
+  tp->tok_alloc = tp->T_max + 32 * nt_max;   // n-tiles of a call: at most 2 * nt_max, each padded by < 16 tokens
   layouts(c, tp->elem, tp->w4, tp->qkv, tp->o, tp->gu, tp->dn);
   tp->layer_bytes = tp->qkv.bytes + tp->o.bytes + tp->gu.bytes + tp->dn.bytes;
 }
@@ -258,17 +258,46 @@ StepPlan make_plan(const TensorPath* tp, int B, int P, int H) {
   p.P = P;
   p.H = H;
   p.T = B * H;
-  p.NT = ceil_div(p.T, NT_MAX);
-  p.Nt = static_cast<int>(align_up(ceil_div(p.T, p.NT), 16));
   const int norm_kind = tp->fp8 ? B_NORM : B_ROWS;   // bf16: the producer wrote bf16(h*gamma) already
-  p.qkv = choose_plan(tp->qkv.MB * p.NT, tp->qkv.NKC, p.Nt, norm_kind, tp->fp8, tp->w4, EPI_QKV, H, 0, tp->nsm,
+  auto plan_gemms = [&](StepPlan& q) {
+    q.qkv = choose_plan(tp->qkv.MB * q.NT, tp->qkv.NKC, q.Nt, norm_kind, tp->fp8, tp->w4, EPI_QKV, H, 0, tp->nsm,
+                        tp->max_dyn, tp->max_dyn2);
+    q.o = choose_plan(tp->o.MB * q.NT, tp->o.NKC, q.Nt, B_ROWS, tp->fp8, tp->w4, EPI_RESID, H, !tp->fp8, tp->nsm,
                       tp->max_dyn, tp->max_dyn2);
-  p.o = choose_plan(tp->o.MB * p.NT, tp->o.NKC, p.Nt, B_ROWS, tp->fp8, tp->w4, EPI_RESID, H, !tp->fp8, tp->nsm,
-                    tp->max_dyn, tp->max_dyn2);
-  p.gu = choose_plan(tp->gu.MB * p.NT, tp->gu.NKC, p.Nt, norm_kind, tp->fp8, tp->w4, EPI_GELU, H, 0, tp->nsm,
-                     tp->max_dyn, tp->max_dyn2);
-  p.dn = choose_plan(tp->dn.MB * p.NT, tp->dn.NKC, p.Nt, B_ROWS, tp->fp8, tp->w4, EPI_RESID, H, !tp->fp8, tp->nsm,
-                     tp->max_dyn, tp->max_dyn2);
+    q.gu = choose_plan(tp->gu.MB * q.NT, tp->gu.NKC, q.Nt, norm_kind, tp->fp8, tp->w4, EPI_GELU, H, 0, tp->nsm,
+                       tp->max_dyn, tp->max_dyn2);
+    q.dn = choose_plan(tp->dn.MB * q.NT, tp->dn.NKC, q.Nt, B_ROWS, tp->fp8, tp->w4, EPI_RESID, H, !tp->fp8, tp->nsm,
+                       tp->max_dyn, tp->max_dyn2);
+  };
+  // Token tiling.  The fewest tiles of at most NT_MAX tokens, unless more tiles (up to twice as many,
+  // at least 160 tokens each: narrower tiles read their operands from shared memory about as fast as
+  // the tensor core consumes them) give the four GEMMs less work per SM: per GEMM, rounds of CTAs over
+  // the SMs x tokens x k-chunks per CTA, plus a fixed cost per round (prologue, exchange, epilogue) of
+  // 1800 token-chunks (about 2 us).  Batch-1-sized calls keep one tile.
+  const int nt0 = ceil_div(p.T, NT_MAX);
+  double best = 1e300;
+  for (int NT = nt0; NT <= 2 * nt0; ++NT) {
+    StepPlan q = p;
+    q.NT = NT;
+    q.Nt = static_cast<int>(align_up(ceil_div(q.T, NT), 16));
+    if (NT > nt0 && (q.Nt < 160 || ceil_div(q.T, q.Nt) != NT)) continue;
+    plan_gemms(q);
+    if (nt0 == 1) {
+      p = q;
+      break;
+    }
+    const ProjLayout* L[4] = {&tp->qkv, &tp->o, &tp->gu, &tp->dn};
+    const GemmPlan* G[4] = {&q.qkv, &q.o, &q.gu, &q.dn};
+    double cost = 0;
+    for (int i = 0; i < 4; ++i) {
+      const int rounds = ceil_div(L[i]->MB * NT * G[i]->S, tp->nsm);
+      cost += rounds * (static_cast<double>(q.Nt) * ceil_div(L[i]->NKC, G[i]->S) + 1800.0);
+    }
+    if (cost < best) {
+      best = cost;
+      p = q;
+    }
+  }
   // the warp-MMA attention kernel holds at most 128 query rows per head: longer sequences take tcgen05
   p.attn_umma = attn_plan(P + H, attn_tiles(B, c.Hq, c.Hkv, H), tp->nsm, p.attn_C, p.attn_KC, H > 128);
   return p;
