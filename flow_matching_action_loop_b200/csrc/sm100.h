@@ -73,6 +73,17 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint3
       "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// ------------------------------------------------------------------ tiled copies (TMA engine, tensor maps)
+// global -> shared through a tensor map held in a __grid_constant__ kernel parameter (generic address
+// of the parameter); box elements past the tensor's extents are written as zeros.  The innermost
+// coordinate times the element size must be a multiple of 16 bytes.  No cluster multicast.
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
 // L2 cache policy for data read once per pass (streamed weights): evicted first, so that the
 // activations, partials and the KV cache stay resident.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
@@ -182,6 +193,13 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1) << 46;   // descriptor version for sm_100
   return d;                              // base offset 0, absolute LBO mode, layout SWIZZLE_NONE
+}
+// The same for a 128-byte-swizzled operand (layout type 2): rows of 128 bytes in 1 KB atoms of 8 rows,
+// the 16-byte chunk c of row r stored at chunk c ^ (r % 8), atoms 1024-byte aligned (base offset 0).
+// K-major: SBO = 1024 (next 8 rows), LBO unused; a K step inside the 128-byte row moves the start
+// address.  MN-major: LBO = the stride between 64-element MN blocks, SBO = 1024 (next 8 K rows).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return smem_desc(saddr, lbo_bytes, sbo_bytes) | (static_cast<uint64_t>(2) << 61);
 }
 
 // Instruction descriptor: dense, fp32 accumulate, both operands K-major.

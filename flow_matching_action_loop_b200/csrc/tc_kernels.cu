@@ -20,7 +20,9 @@
 //   over 64-key sub-chunks; the chunks' (O, max, sum) rows are pushed to their owner CTA by
 //   bulk copies and merged with log-sum-exp weights in rank order.
 #include <algorithm>
+#include <mutex>
 #include <type_traits>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <math.h>
@@ -1041,18 +1043,21 @@ __global__ void __launch_bounds__(256) k_attn_tc(const __grid_constant__ AttnArg
 // One CTA per (sample b, KV head g, tile of 128 query rows, key chunk c); the rows of a tile
 // are the (query head, action row) pairs of every query head that reads KV head g, so the
 // chunk's K and V are staged once for the whole group.  Per 64-key sub-chunk:
+//   K, V               tensor-map copies (128-byte swizzle) by one thread of a copy / MMA warp
 //   S = Q K^T          tcgen05 (M = 128 rows, N = 64 keys, K = dh), fp32 in tensor memory
-//   online softmax     one thread per row: S row from tensor memory, running max / sum,
+//   online softmax     two threads per row: S row from tensor memory, running max / sum,
 //                      P = 2^(s - m) in bf16 into shared memory, O rescaled in tensor memory
 //   O += P V           tcgen05 (M = 128, N = dh, K = 64 keys), V read MN-major as stored
+// The softmax warps and the copy / MMA thread hand sub-chunks over through mbarriers only.
 // Chunks (a cluster when C > 1) are merged over (O, max, sum) rows in the L2 scratch with the
 // same rank-order log-sum-exp weights as the flash-decoding merge.
 
 constexpr int UA_SUB = 64;        // keys per sub-chunk
 constexpr float UA_RESCALE = 8.f; // the softmax reference moves when the row maximum grows by more (log2 units)
-constexpr int UA_THREADS = 256;   // two per query row of the tile: warps w and w + 4 share the row's lane
-                                  // quadrant of tensor memory, each takes half of the keys' exponentials
-                                  // and half of the O columns
+constexpr int UA_SOFTMAX = 256;   // softmax threads, two per query row of the tile: warps w and w + 4 share
+                                  // the row's lane quadrant of tensor memory, each takes half of the keys'
+                                  // exponentials and half of the O columns
+constexpr int UA_THREADS = UA_SOFTMAX + 32;   // + one warp whose lane 0 issues the copies and the MMAs
 
 struct UAttnGeom {
   uint32_t q_off, k_off0, k_off1, v_off0, v_off1, p_off0, p_off1, w_off, total, tcols, o_col;
@@ -1081,20 +1086,24 @@ __host__ __device__ __forceinline__ UAttnGeom uattn_geom(int dh) {
 template <int DH>
 __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_constant__ AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t dsm[];
-  __shared__ uint64_t bar_s[2], bar_o[2], stage_bar;
+  __shared__ uint64_t bar_s[2], bar_o[2], bar_p[2], kfull[2], vfull[2], stage_bar;
   __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;             // a wait gave up: the other role stops waiting too
   __shared__ float inv_den[128];
   __shared__ float l_sh[2][128];         // the two halves' softmax sums of each row
   TL_DECL
   TL_BEGIN(20);
   constexpr int OLD = DH + 4;            // fp32 row stride of the partial-O rows
-  constexpr int VPR = DH / 8;            // 16-byte vectors per K/V/Q row
+  constexpr int VPR = DH / 8;            // 16-byte vectors per Q row
+  constexpr int NBX = DH / 64;           // 64-feature boxes (128-byte rows) per K or V sub-chunk
   constexpr uint32_t IDESC_S = idesc_f32acc(FMT_BF16, 128, UA_SUB);
   constexpr uint32_t IDESC_O = idesc_f32acc(FMT_BF16, 128, DH) | IDESC_B_MN_MAJOR;
   const UAttnGeom gm = uattn_geom(DH);
   const int c = blockIdx.x, y = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int row = tid & 127, hh = tid >> 7;   // this thread's query row of the tile and half
+  const bool sm_thread = tid < UA_SOFTMAX;        // softmax warps 0-7: two threads per query row
+  const bool mma_thread = tid == UA_SOFTMAX;      // warp 8, lane 0: tensor-map copies and MMAs
+  const int row = tid & 127, hh = (tid >> 7) & 1; // a softmax thread's row of the tile and half
   const int G = a.Hq / a.Hkv;            // query heads per KV head (consecutive heads)
   const int R = G * a.H;                 // query rows of one KV group
   const int MT = (R + 127) >> 7;
@@ -1105,8 +1114,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   const int key0 = c * a.KC;
   const int nkeys = min(a.KC, S - key0);
   const int nsub = (nkeys + UA_SUB - 1) / UA_SUB;
-  const __nv_bfloat16* kg = a.kv_k + ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max) * DH;
-  const __nv_bfloat16* vg = a.kv_v + ((static_cast<size_t>(b) * a.Hkv + g) * a.S_max) * DH;
+  const int zkv = b * a.Hkv + g;         // K/V tensor-map plane of (sample, KV head)
   // the group's query rows are contiguous: heads g*G.. of sample b, H rows each
   const __nv_bfloat16* qg = a.q + ((static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G) * a.H + row0) * DH;
 
@@ -1114,8 +1122,12 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_s[i], 1);
       mbar_init(&bar_o[i], 1);
+      mbar_init(&bar_p[i], UA_SOFTMAX);
+      mbar_init(&kfull[i], 1);
+      mbar_init(&vfull[i], 1);
     }
     mbar_init(&stage_bar, 1);
+    abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -1128,207 +1140,201 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   grid_dep_launch();
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   const uint32_t tS = tmem_base, tO = tmem_base + gm.o_col;
-
-  // K and V rows of sub-chunk sc: thread t copies key t % 64 of the sub-chunk, its 16-byte columns
-  // t / 64, t / 64 + 4, ... (consecutive threads: consecutive keys), with per-thread base addresses and
-  // constant strides.  K lands as the K-major operand of S = Q K^T ([16-byte column][64 keys][16 B]);
-  // V as stored ([key][DH]) is the MN-major operand of O += P V (core matrices of 8 keys x 16 B, 8-key
-  // groups DH*16 bytes apart).  which: 0 = prefix keys (and zero rows past the chunk), 1 = action keys,
-  // 2 = all.
-  constexpr int CPT = UA_SUB * VPR / UA_THREADS;   // 16-byte copies per thread per sub-chunk and operand
-  constexpr int JS = UA_THREADS / UA_SUB;          // 16-byte column step between a thread's copies
-  const int kn = tid & (UA_SUB - 1), kj0 = tid / UA_SUB;
-  auto key_of = [&](int sc, int which, int& key, bool& valid) {
-    key = key0 + sc * UA_SUB + kn;
-    valid = sc * UA_SUB + kn < nkeys;
-    return which == 2 || (which == 0 ? (key < a.P || !valid) : (key >= a.P && valid));
-  };
-  auto load_k = [&](int sc, uint8_t* Kb, int which) {
-    int key;
-    bool valid;
-    if (!key_of(sc, which, key, valid)) return;
-    uint8_t* dst = Kb + kj0 * (UA_SUB * 16) + kn * 16;
-    const __nv_bfloat16* src = kg + static_cast<size_t>(valid ? key : 0) * DH + kj0 * 8;
-#pragma unroll
-    for (int m = 0; m < CPT; ++m) cp_async16(dst + m * JS * (UA_SUB * 16), src + m * JS * 8, valid);
-  };
-  auto load_v = [&](int sc, uint8_t* Vb, int which) {
-    int key;
-    bool valid;
-    if (!key_of(sc, which, key, valid)) return;
-    uint8_t* dst = Vb + (kn >> 3) * (DH * 16) + kj0 * 128 + (kn & 7) * 16;
-    const __nv_bfloat16* src = vg + static_cast<size_t>(valid ? key : 0) * DH + kj0 * 8;
-#pragma unroll
-    for (int m = 0; m < CPT; ++m) cp_async16(dst + m * JS * 128, src + m * JS * 8, valid);
-  };
   auto Kbuf = [&](int bf) { return dsm + (bf ? gm.k_off1 : gm.k_off0); };
   auto Vbuf = [&](int bf) { return dsm + (bf ? gm.v_off1 : gm.v_off0); };
+  auto Pbuf = [&](int bf) { return dsm + (bf ? gm.p_off1 : gm.p_off0); };
+  volatile int* abort_v = &abort_flag;
 
-  // prefix keys do not depend on the previous kernel: their loads go first
-  load_k(0, Kbuf(0), 0);
-  load_v(0, Vbuf(0), 0);
-  if (nsub > 1) {
-    load_k(1, Kbuf(1), 0);
-    load_v(1, Vbuf(1), 0);
-  }
-  cp_async_commit();
+  // K or V of sub-chunk j by tensor map (the MMA thread): NBX boxes of 64 keys x 64 features, each
+  // 64 rows of 128 bytes swizzled in 1 KB atoms, 8 KB apart.  Keys past the sequence read as zeros;
+  // keys past this chunk are real keys, masked in the softmax.
+  int k_issued = 0, v_issued = 0;
+  auto load_kv = [&](const CUtensorMap* tm, uint8_t* dst, uint64_t* bar, int j) {
+    mbar_arrive_expect_tx(bar, UA_SUB * DH * 2);
+    for (int x = 0; x < NBX; ++x) tma_load_3d(dst + x * (UA_SUB * 128), tm, x * 64, key0 + j * UA_SUB, zkv, bar);
+  };
+  auto load_k = [&](int j) {
+    load_kv(&a.tm_k, Kbuf(j & 1), &kfull[j & 1], j);
+    k_issued = j + 1;
+  };
+  auto load_v = [&](int j) {
+    load_kv(&a.tm_v, Vbuf(j & 1), &vfull[j & 1], j);
+    v_issued = j + 1;
+  };
+  // a sub-chunk whose 64 keys all precede the action rows does not depend on the previous kernel
+  auto prefix_only = [&](int j) { return key0 + (j + 1) * UA_SUB <= a.P; };
+  const int npro = nsub < 2 ? nsub : 2;
+  if (mma_thread)
+    for (int j = 0; j < npro; ++j)
+      if (prefix_only(j)) {
+        load_k(j);
+        load_v(j);
+      }
   grid_dep_wait();
   if (tid == 0) TL(1);
-  load_k(0, Kbuf(0), 1);
-  load_v(0, Vbuf(0), 1);
-  if (nsub > 1) {
-    load_k(1, Kbuf(1), 1);
-    load_v(1, Vbuf(1), 1);
-  }
-  {   // Q tile, K-major [16-byte column][128 rows][16 B]: the two threads of a row copy half of it each
+  if (mma_thread)
+    for (int j = 0; j < npro; ++j)
+      if (!prefix_only(j)) {
+        load_k(j);
+        load_v(j);
+      }
+  if (sm_thread) {   // Q tile, K-major [16-byte column][128 rows][16 B]: the two threads of a row copy half each
     const bool qv = row < Rv;
     uint8_t* dst = dsm + gm.q_off + row * 16 + hh * (VPR / 2) * 2048;
     const __nv_bfloat16* src = qg + static_cast<size_t>(qv ? row : 0) * DH + hh * (VPR / 2) * 8;
 #pragma unroll
     for (int j = 0; j < VPR / 2; ++j) cp_async16(dst + j * 2048, src + j * 8, qv);
+    cp_async_commit();
+    cp_async_wait_all();
+    fence_proxy_async_smem();   // cp.async writes -> visible to the tensor core
   }
-  cp_async_commit();
-  cp_async_wait_all();
-  fence_proxy_async_smem();   // cp.async writes -> visible to the tensor core
-  __syncthreads();
+  __syncthreads();   // Q in place
   if (tid == 0) TL(2);
 
-  const float sl2 = a.scale * 1.4426950408889634f;   // scores in log2 units
-  // S(j) = Q K(j)^T into score buffer j & 1 (thread 0; K(j) resident and made visible)
-  auto issue_s = [&](int j) {
-    tc_fence_after();
-    const uint32_t qa = smem_u32(dsm + gm.q_off), ka = smem_u32(Kbuf(j & 1));
-#pragma unroll
-    for (int k = 0; k < DH / 16; ++k)
-      mma_bf16(tS + (j & 1) * UA_SUB, smem_desc(qa + k * 2 * 2048, 2048, 128),
-               smem_desc(ka + k * 2 * (UA_SUB * 16), UA_SUB * 16, 128), IDESC_S, k > 0);
-    mma_commit(&bar_s[j & 1]);
-  };
-  if (tid == 0) {
-    issue_s(0);
-    if (nsub > 1) issue_s(1);
-  }
-  // Sub-chunk sc: the scores of sc + 1 are computed by the tensor core while the threads run the
-  // softmax of sc, and O += P(sc) V(sc) runs while they start on sc + 1 (P has two buffers).
-  // Copy groups in issue order: sub-chunk sc commits K(sc + 2), then V(sc + 1).
+  bool ok = true;
   float m_run = -INFINITY, l_run = 0.f;
-  bool ok = true, failed = false;
-  for (int sc = 0; sc < nsub; ++sc) {
-    const int bf = sc & 1;
-    if (sc >= 1 && sc + 1 < nsub) {   // K(sc+1) landed (V(sc), committed after it, may stay in flight)
-      if (sc >= 2) cp_async_wait_one_pending();
-      else cp_async_wait_all();
-      fence_proxy_async_smem();
-      __syncthreads();
-      if (tid == 0) issue_s(sc + 1);
-    }
-    ok &= mbar_wait(&bar_s[bf], (sc >> 1) & 1, WAIT_LIMIT_NS);
-    tc_fence_after();
-    if (sc + 2 < nsub) {   // S(sc) has read K buffer bf
-      load_k(sc + 2, Kbuf(bf), 2);
-      cp_async_commit();
-    }
-    uint32_t sv[UA_SUB];
+  if (mma_thread) {
+    // ---------------- copies and MMAs.  Per sub-chunk sc: K(sc+2) once S(sc) is done; O += P(sc) V(sc)
+    // once the softmax of sc has arrived; S(sc+2) into the score buffer that softmax just read; V(sc+2)
+    // once O(sc) is done.  The tensor core thus computes S(sc+1) while the softmax of sc runs.
+    auto issue_s = [&](int j) {   // S(j) = Q K(j)^T into score buffer j & 1 once K(j) has landed
+      if (!mbar_wait(&kfull[j & 1], (j >> 1) & 1, WAIT_LIMIT_NS)) return false;
+      tc_fence_after();
+      const uint32_t qa = smem_u32(dsm + gm.q_off), ka = smem_u32(Kbuf(j & 1));
 #pragma unroll
-    for (int u = 0; u < UA_SUB / 16; ++u) tmem_ld16_nowait(tS + bf * UA_SUB + lane_base + 16 * u, sv + 16 * u);
-    tmem_wait_ld();
-    const int kb = sc * UA_SUB;
-    // Both threads of a row take the maximum over all 64 raw scores (four independent chains: with
-    // few warps per scheduler the chains are the latency); the scale sl2 > 0 is applied after it
-    float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-    if (kb + UA_SUB > nkeys) {   // the chunk's last sub-chunk: keys past it do not count
-#pragma unroll
-      for (int jj = 0; jj < UA_SUB; ++jj)
-        if (kb + jj >= nkeys) sv[jj] = __float_as_uint(-INFINITY);
-    }
-#pragma unroll
-    for (int jj = 0; jj < UA_SUB; ++jj) mq[jj & 3] = fmaxf(mq[jj & 3], __uint_as_float(sv[jj]));
-    const float mx = fmaxf(m_run, fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sl2);   // log2 units
-    // The reference of the exponentials moves only when the row maximum has grown by more than
-    // UA_RESCALE (log2 units): P stays below 2^UA_RESCALE, the sum and O are relative to the same
-    // reference, and O / l is unchanged; O in tensor memory is rescaled only when a row's reference
-    // moves, which after the first sub-chunks is rare.
-    const float ref = (mx > m_run + UA_RESCALE) ? mx : m_run;
-    const float corr = exp2f(m_run - ref);
-    const bool resc = sc > 0 && __any_sync(0xffffffffu, corr != 1.f);
-    // P buffer bf was last read by O += P V of sub-chunk sc - 2, complete since sub-chunk sc - 1; this
-    // thread writes keys 32*hh .. 32*hh + 31 of its row, 2^(s*sl2 - ref)
-    float ps[4] = {0.f, 0.f, 0.f, 0.f};
-    uint8_t* prow = dsm + (bf ? gm.p_off1 : gm.p_off0) + (row >> 3) * 128 + (row & 7) * 16;   // K-major [128 x 64]
-    auto expo = [&](auto half) {   // compile-time key range, so that sv stays in registers
-      constexpr int K0 = decltype(half)::value * (UA_SUB / 2);
-#pragma unroll
-      for (int k2 = 0; k2 < UA_SUB / 16; ++k2) {
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = ex2_approx(fmaf(__uint_as_float(sv[K0 + k2 * 8 + e]), sl2, -ref));
-          ps[e & 3] += p[e];
-        }
-        *reinterpret_cast<uint4*>(prow + (K0 / 8 + k2) * 2048) = make_uint4(
-            pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
-      }
+      for (int k = 0; k < DH / 16; ++k)
+        mma_bf16(tS + (j & 1) * UA_SUB, smem_desc(qa + k * 2 * 2048, 2048, 128),
+                 smem_desc_sw128(ka + (k >> 2) * (UA_SUB * 128) + (k & 3) * 32, 16, 1024), IDESC_S, k > 0);
+      mma_commit(&bar_s[j & 1]);
+      return true;
     };
-    if (hh == 0) expo(std::integral_constant<int, 0>{});   // warp-uniform
-    else expo(std::integral_constant<int, 1>{});
-    l_run = l_run * corr + ((ps[0] + ps[1]) + (ps[2] + ps[3]));   // this half's keys
-    m_run = ref;
-    if (resc) {   // O(sc-1) complete before this warp's rows of O are rescaled
-      ok &= mbar_wait(&bar_o[bf ^ 1], ((sc - 1) >> 1) & 1, WAIT_LIMIT_NS);
-      tc_fence_after();
-#pragma unroll 1
-      for (int c0 = hh * (DH / 2); c0 < (hh + 1) * (DH / 2); c0 += 16) {   // this thread's half of O
-        uint32_t ov[16];
-        tmem_ld16_nowait(tO + lane_base + c0, ov);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-        tmem_st16(tO + lane_base + c0, ov);
+    ok = issue_s(0) && (nsub < 2 || issue_s(1));
+    for (int sc = 0; ok && sc < nsub; ++sc) {
+      const int bf = sc & 1;
+      if (sc + 2 < nsub) {
+        ok = mbar_wait(&bar_s[bf], (sc >> 1) & 1, WAIT_LIMIT_NS) && !*abort_v;
+        if (!ok) break;
+        load_k(sc + 2);
       }
-      tmem_wait_st();
-    }
-    if (sc >= 2) {   // V(sc), committed in sub-chunk sc - 1 before K(sc + 2)
-      if (sc + 2 < nsub) cp_async_wait_one_pending();
-      else cp_async_wait_all();
-    }
-    fence_proxy_async_smem();   // P and V (generic-proxy / cp.async writes) -> visible to the tensor core
-    tc_fence_before();
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) report_timeout(a.status, 0x700);
-      failed = true;
-      break;
-    }
-    if (tid == 0) {
+      ok = mbar_wait(&bar_p[bf], (sc >> 1) & 1, WAIT_LIMIT_NS) && mbar_wait(&vfull[bf], (sc >> 1) & 1, WAIT_LIMIT_NS) &&
+           !*abort_v;
+      if (!ok) break;
       tc_fence_after();
-      const uint32_t pa = smem_u32(dsm + (bf ? gm.p_off1 : gm.p_off0)), va = smem_u32(Vbuf(bf));
+      const uint32_t pa = smem_u32(Pbuf(bf)), va = smem_u32(Vbuf(bf));
 #pragma unroll
       for (int k = 0; k < UA_SUB / 16; ++k)
-        mma_bf16(tO, smem_desc(pa + k * 2 * 2048, 2048, 128), smem_desc(va + k * 2 * (DH * 16), DH * 16, 128), IDESC_O,
-                 (sc > 0 || k > 0) ? 1u : 0u);
+        mma_bf16(tO, smem_desc(pa + k * 2 * 2048, 2048, 128), smem_desc_sw128(va + k * 2 * 1024, UA_SUB * 128, 1024),
+                 IDESC_O, (sc > 0 || k > 0) ? 1u : 0u);
       mma_commit(&bar_o[bf]);
+      if (sc + 2 < nsub) {
+        ok = issue_s(sc + 2) && mbar_wait(&bar_o[bf], (sc >> 1) & 1, WAIT_LIMIT_NS);
+        if (!ok) break;
+        load_v(sc + 2);
+      }
     }
-    if (sc >= 1 && sc + 1 < nsub) {   // O(sc-1) done: V buffer bf ^ 1 and P buffer bf ^ 1 are free
-      ok &= mbar_wait(&bar_o[bf ^ 1], ((sc - 1) >> 1) & 1, WAIT_LIMIT_NS);
-      load_v(sc + 1, Vbuf(bf ^ 1), 2);
-      cp_async_commit();
+    if (!ok) {
+      *abort_v = 1;
+      report_timeout(a.status, 0x700);
+    }
+  } else if (sm_thread) {
+    // ---------------- online softmax (two threads per row, each half of the keys' exponentials)
+    const float sl2 = a.scale * 1.4426950408889634f;   // scores in log2 units
+    for (int sc = 0; sc < nsub; ++sc) {
+      const int bf = sc & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_s[bf], (sc >> 1) & 1, WAIT_LIMIT_NS) && !*abort_v)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv[UA_SUB];
+#pragma unroll
+      for (int u = 0; u < UA_SUB / 16; ++u) tmem_ld16_nowait(tS + bf * UA_SUB + lane_base + 16 * u, sv + 16 * u);
+      tmem_wait_ld();
+      const int kb = sc * UA_SUB;
+      // both threads of a row take the maximum over all 64 raw scores (four independent chains); the
+      // scale sl2 > 0 is applied after it
+      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (kb + UA_SUB > nkeys) {   // the chunk's last sub-chunk: keys past it do not count
+#pragma unroll
+        for (int jj = 0; jj < UA_SUB; ++jj)
+          if (kb + jj >= nkeys) sv[jj] = __float_as_uint(-INFINITY);
+      }
+#pragma unroll
+      for (int jj = 0; jj < UA_SUB; ++jj) mq[jj & 3] = fmaxf(mq[jj & 3], __uint_as_float(sv[jj]));
+      const float mx = fmaxf(m_run, fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sl2);   // log2 units
+      // The reference of the exponentials moves only when the row maximum has grown by more than
+      // UA_RESCALE (log2 units): P stays below 2^UA_RESCALE, the sum and O are relative to the same
+      // reference, and O / l is unchanged; O in tensor memory is rescaled only when a row's reference
+      // moves, which after the first sub-chunks is rare.
+      const float ref = (mx > m_run + UA_RESCALE) ? mx : m_run;
+      const float corr = exp2f(m_run - ref);
+      const bool resc = sc > 0 && __any_sync(0xffffffffu, corr != 1.f);
+      // P buffer bf was read by O += P V of sub-chunk sc - 2
+      if (sc >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar_o[bf], ((sc - 2) >> 1) & 1, WAIT_LIMIT_NS))) {
+        ok = false;
+        break;
+      }
+      // this thread writes keys 32*hh .. 32*hh + 31 of its row: 2^(s*sl2 - ref) in bf16
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+      uint8_t* prow = Pbuf(bf) + (row >> 3) * 128 + (row & 7) * 16;   // K-major [128 x 64]
+      auto expo = [&](auto half) {   // compile-time key range, so that sv stays in registers
+        constexpr int K0 = decltype(half)::value * (UA_SUB / 2);
+#pragma unroll
+        for (int k2 = 0; k2 < UA_SUB / 16; ++k2) {
+          float p[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            p[e] = ex2_approx(fmaf(__uint_as_float(sv[K0 + k2 * 8 + e]), sl2, -ref));
+            ps[e & 3] += p[e];
+          }
+          *reinterpret_cast<uint4*>(prow + (K0 / 8 + k2) * 2048) = make_uint4(
+              pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
+        }
+      };
+      if (hh == 0) expo(std::integral_constant<int, 0>{});   // warp-uniform
+      else expo(std::integral_constant<int, 1>{});
+      l_run = l_run * corr + ((ps[0] + ps[1]) + (ps[2] + ps[3]));   // this half's keys
+      m_run = ref;
+      if (resc) {   // O(sc-1) complete before this warp's rows of O are rescaled
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar_o[bf ^ 1], ((sc - 1) >> 1) & 1, WAIT_LIMIT_NS))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = hh * (DH / 2); c0 < (hh + 1) * (DH / 2); c0 += 16) {   // this thread's half of O
+          uint32_t ov[16];
+          tmem_ld16_nowait(tO + lane_base + c0, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+          tmem_st16(tO + lane_base + c0, ov);
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();   // P (generic-proxy stores) -> visible to the tensor core
+      tc_fence_before();          // S read and O rescaled before the MMA thread moves on
+      mbar_arrive(&bar_p[bf]);
+    }
+    if (!ok) *abort_v = 1;
+    l_sh[hh][row] = l_run;
+    if (ok && !__all_sync(0xffffffffu, mbar_wait(&bar_o[(nsub - 1) & 1], ((nsub - 1) >> 1) & 1, WAIT_LIMIT_NS))) {
+      ok = false;
+      *abort_v = 1;
+      if ((tid & 31) == 0) report_timeout(a.status, 0x702);
     }
   }
-  l_sh[hh][row] = l_run;
-  if (!failed) {
-    const bool got = ok && mbar_wait(&bar_o[(nsub - 1) & 1], ((nsub - 1) >> 1) & 1, WAIT_LIMIT_NS);
-    if (__syncthreads_or(!got)) {
-      if (tid == 0) report_timeout(a.status, 0x702);
-      failed = true;
-    }
+  const bool failed = __syncthreads_or(!ok);   // also: l_sh complete
+  if (mma_thread && failed) {   // copies issued and not consumed land before the buffers are reused
+    for (int j = (k_issued > 2 ? k_issued - 2 : 0); j < k_issued; ++j) mbar_wait(&kfull[j & 1], (j >> 1) & 1, WAIT_LIMIT_NS);
+    for (int j = (v_issued > 2 ? v_issued - 2 : 0); j < v_issued; ++j) mbar_wait(&vfull[j & 1], (j >> 1) & 1, WAIT_LIMIT_NS);
   }
-  cp_async_wait_all();
   tc_fence_after();
   if (tid == 0) TL(3);
 
-  __syncthreads();                                   // l_sh complete (also on the failure paths)
   const float l_tot = l_sh[0][row] + l_sh[1][row];
   const int rr = row0 + row;                         // this thread's row of the group
-  const bool rv = row < Rv && !failed;
+  const bool rv = sm_thread && row < Rv && !failed;
   const int jq = g * G + rr / a.H, iq = rr % a.H;    // query head, action row
   const float inv_sa = (a.fp8 && a.s_a) ? 1.0f / *a.s_a : 1.0f;
   // writes 16 consecutive output features d0.. of row (token t, head jq)
@@ -1357,7 +1363,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
     }
   };
 
-  if (C == 1) {
+  if (sm_thread && C == 1) {   // the copy / MMA warp holds no rows
     const float inv = 1.0f / l_tot;
 #pragma unroll 1
     for (int c0 = hh * (DH / 2); c0 < (hh + 1) * (DH / 2); c0 += 16) {   // this thread's half of the row
@@ -1369,7 +1375,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
       for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(ov[e]) * inv;
       if (rv) store16(b * a.H + iq, jq, c0, v);
     }
-  } else {
+  } else if (sm_thread) {
     // this chunk's (O, max, sum) row into the scratch, [B][Hq][C][H][OLD]
     float* xrow = a.xscratch + ((static_cast<size_t>(b) * a.Hq + jq) * C + c) * a.H * OLD + static_cast<size_t>(iq) * OLD;
 #pragma unroll 1
@@ -1769,11 +1775,50 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int n_tiles, cudaStream_t s, bool 
                    pdl, a.S, args);
 }
 
+namespace {
+
+// cuTensorMapEncodeTiled from the driver, found once through the runtime (no link-time dependency).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Tensor map of K or V ([planes][keys][dh] bf16, planes plane_bytes apart): boxes of 64 features
+// (128 bytes) x 64 keys x 1 plane, 128-byte swizzle; keys past `keys` read as zeros.
+bool encode_kv_map(CUtensorMap* m, const void* base, uint64_t dh, uint64_t keys, uint64_t planes,
+                   uint64_t plane_bytes) {
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (!fn || !base || (reinterpret_cast<uintptr_t>(base) & 15u) || keys == 0 || planes == 0 || dh % 64 != 0)
+    return false;
+  const cuuint64_t dims[3] = {dh, keys, planes};
+  const cuuint64_t strides[2] = {dh * 2, plane_bytes};
+  const cuuint32_t box[3] = {64u, 64u, 1u};
+  const cuuint32_t es[3] = {1u, 1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3u, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 cudaError_t launch_attention_tc(const AttnArgs& a, int B, cudaStream_t s, bool pdl) {
   AttnArgs copy = a;
   void* args[] = {&copy};
   const size_t smem = attn_smem_bytes(a.H, a.dh, a.KC, a.C, a.umma);
   if (a.umma) {
+    // K and V [B][Hkv][S_max][dh] as B*Hkv planes of this call's P + H keys (keys past them read as zeros)
+    const uint64_t dh = static_cast<uint64_t>(a.dh), keys = static_cast<uint64_t>(a.P + a.H);
+    const uint64_t planes = static_cast<uint64_t>(B) * a.Hkv, pb = static_cast<uint64_t>(a.S_max) * dh * 2;
+    if (!encode_kv_map(&copy.tm_k, a.kv_k, dh, keys, planes, pb) || !encode_kv_map(&copy.tm_v, a.kv_v, dh, keys, planes, pb))
+      return cudaErrorInvalidValue;
     const void* f = a.dh == 64 ? reinterpret_cast<const void*>(k_attn_umma<64>)
                   : a.dh == 128 ? reinterpret_cast<const void*>(k_attn_umma<128>)
                                 : reinterpret_cast<const void*>(k_attn_umma<256>);

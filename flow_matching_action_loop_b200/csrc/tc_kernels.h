@@ -20,6 +20,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -148,6 +149,9 @@ struct AttnArgs {
   unsigned* status;            // device status word (timeouts), or nullptr
   int umma;                    // 1: tcgen05 kernel over GQA-group tiles; 0: warp-MMA kernel per query head
   uint64_t o_extent;           // bytes of o (checked builds)
+  // tcgen05 kernel: tensor maps of this layer's K and V ([B*Hkv][P+H][dh], planes S_max rows apart),
+  // boxes of 64 features x 64 keys with 128-byte swizzle; written by launch_attention_tc
+  CUtensorMap tm_k, tm_v;
 };
 
 // Key chunks of the split-KV attention over S keys: at most 16 (one cluster), each a multiple
