@@ -717,6 +717,242 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   }
 }
 
+// ================================================================== persistent gate|up GEMM (wide tiles)
+//
+// One CTA per SM walks the (m-block, n-tile) tiles t = blockIdx.x, + gridDim.x, ... (consecutive t share
+// the m-block, so the CTAs running together read a weight tile from HBM once).  Warp 0 lane 0 copies
+// A and B chunks into the ring across tile boundaries, warp 1 lane 0 issues the MMAs into one of two
+// accumulators in tensor memory, and warps 2-9 drain the other: TMEM -> shared memory in passes of
+// PT_RED_TOK tokens, GeLU(gate) * up, the down projection's bf16 operand.  The epilogue of tile i thus
+// runs while the MMAs of tile i + 1 do.  bf16 operands, no split-K (multi-wave shapes only).
+
+constexpr int PT_THREADS = 320;   // warp 0: copies, warp 1: MMAs, warps 2-9: epilogue
+constexpr int PT_EPI = 256;       // epilogue threads
+constexpr int PT_RED_TOK = 64;    // tokens per epilogue staging pass
+
+struct PtSmem {
+  uint64_t full_a[MAX_STAGES], full_b[MAX_STAGES], empty[MAX_STAGES];
+  uint64_t tfull[2], tempty[2];   // accumulator a: MMAs done / drained by the epilogue
+  uint32_t tmem_base;
+  float rstd[NT_MAX];
+};
+
+__host__ __device__ __forceinline__ uint32_t pt_ring_bytes(int Nt, int stages) {
+  return static_cast<uint32_t>(stages) * (BM * KCB + static_cast<uint32_t>(Nt) * KCB);
+}
+
+__device__ __forceinline__ void pt_epi_sync() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
+
+__global__ void __launch_bounds__(PT_THREADS, 1) k_gemm_gelu_pt(const __grid_constant__ GemmArgs a) {
+  extern __shared__ __align__(1024) uint8_t dsm[];
+  __shared__ PtSmem sh;
+  __shared__ volatile int pt_fail;   // an epilogue wait gave up (all epilogue warps stop together)
+  TL_DECL
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  TL_BEGIN(13);
+  const int Nt = a.Nt, NTl = a.pt_nt, NKC = a.NKC, stages = a.stages;
+  const int tiles = a.MB * NTl;
+  const int my_tiles = (tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+  const uint32_t a_bytes = BM * KCB, b_bytes = static_cast<uint32_t>(Nt) * KCB;
+  auto a_slot = [&](int s) { return dsm + s * a_bytes; };
+  auto b_slot = [&](int s) { return dsm + stages * a_bytes + s * b_bytes; };
+  float* red = reinterpret_cast<float*>(dsm + pt_ring_bytes(Nt, stages));   // [PT_RED_TOK][RED_LD]
+  auto tile_of = [&](int i, int& mb, int& nt) {
+    const int t = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+    mb = t / NTl;
+    nt = t - mb * NTl;
+  };
+
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&sh.full_a[s], 1);
+      mbar_init(&sh.full_b[s], 1);
+      mbar_init(&sh.empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.tfull[i], 1);
+      mbar_init(&sh.tempty[i], PT_EPI);
+    }
+    pt_fail = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  grid_dep_launch();
+  const uint32_t tbase = sh.tmem_base;
+  const int total = my_tiles * NKC;   // chunks this CTA streams
+
+  if (warp == 0) {
+    // ---------------- copies: chunk q is chunk q % NKC of this CTA's tile q / NKC
+    if (lane == 0) {
+      auto issue_a = [&](int q) {
+        int mb, nt;
+        tile_of(q / NKC, mb, nt);
+        const int s = q % stages;
+        mbar_arrive_expect_tx(&sh.full_a[s], a_bytes);
+        bulk_g2s(a_slot(s), a.W + (static_cast<size_t>(mb) * NKC + q % NKC) * a_bytes, a_bytes, &sh.full_a[s]);
+      };
+      auto issue_b = [&](int q) {
+        int mb, nt;
+        tile_of(q / NKC, mb, nt);
+        const int s = q % stages;
+        mbar_arrive_expect_tx(&sh.full_b[s], b_bytes);
+        bulk_g2s(b_slot(s), a.act + (static_cast<size_t>(nt) * NKC + q % NKC) * b_bytes, b_bytes, &sh.full_b[s]);
+      };
+      const int pre = total < stages ? total : stages;
+      for (int q = 0; q < pre; ++q) issue_a(q);   // weights do not depend on the previous kernel
+      grid_dep_wait();
+      TL(1);
+      for (int q = 0; q < pre; ++q) issue_b(q);
+      int issued = pre;
+      for (int q = pre; q < total; ++q) {
+        const int s = q % stages;
+        if (!mbar_wait(&sh.empty[s], ((q / stages) - 1) & 1, WAIT_LIMIT_NS)) {
+          report_timeout(a.status, 0xB100);
+          break;
+        }
+        issue_a(q);
+        issue_b(q);
+        issued = q + 1;
+      }
+      // drain: every copy issued into this CTA's shared memory has landed before the CTA exits
+      for (int q = (issued > stages ? issued - stages : 0); q < issued; ++q) {
+        const int s = q % stages;
+        const uint32_t par = (q / stages) & 1;
+        if (!mbar_wait(&sh.full_a[s], par, WAIT_LIMIT_NS) || !mbar_wait(&sh.full_b[s], par, WAIT_LIMIT_NS))
+          report_timeout(a.status, 0xB101);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMAs: tile i into accumulator i & 1 once the epilogue has drained it (tile i - 2)
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f32acc(FMT_BF16, BM, Nt);
+      int q = 0;
+      bool ok = true;
+      for (int i = 0; ok && i < my_tiles; ++i) {
+        const int acc = i & 1;
+        if (i >= 2 && !mbar_wait(&sh.tempty[acc], ((i >> 1) - 1) & 1, WAIT_LIMIT_NS)) {
+          report_timeout(a.status, 0xB200);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tacc = tbase + static_cast<uint32_t>(acc) * 256u;
+        for (int c = 0; c < NKC; ++c, ++q) {
+          const int s = q % stages;
+          const uint32_t par = (q / stages) & 1;
+          if (!mbar_wait(&sh.full_a[s], par, WAIT_LIMIT_NS) || !mbar_wait(&sh.full_b[s], par, WAIT_LIMIT_NS)) {
+            report_timeout(a.status, 0xB201);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(a_slot(s)), b0 = smem_u32(b_slot(s));
+#pragma unroll
+          for (int k = 0; k < KCB / 32; ++k)
+            mma_bf16(tacc, smem_desc(a0 + k * 2 * BM * 16, BM * 16, 128), smem_desc(b0 + k * 2 * Nt * 16, Nt * 16, 128),
+                     idesc, (c | k) != 0);
+          mma_commit(&sh.empty[s]);
+        }
+        if (ok) mma_commit(&sh.tfull[acc]);
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2-9; warp w reads the TMEM lane quadrant w % 4, warps 2-5 the
+    // first half of a pass's token columns, warps 6-9 the rest; each warp then takes whole tokens,
+    // each lane two consecutive gate/up feature pairs)
+    const int ew = warp - 2, etid = tid - 64;
+    const int q4 = warp & 3, row = q4 * 32 + lane;
+    const int p = lane * 2;
+    grid_dep_wait();   // the Σh² partials and the operand buffer belong to the previous kernels
+    const float al = a.alpha ? *a.alpha : 1.0f;
+    for (int i = 0; i < my_tiles; ++i) {
+      const int acc = i & 1;
+      int mb, nt;
+      tile_of(i, mb, nt);
+      const int n0 = nt * Nt;
+      const uint32_t tacc = tbase + static_cast<uint32_t>(acc) * 256u;
+      if (!mbar_wait(&sh.tfull[acc], (i >> 1) & 1, WAIT_LIMIT_NS)) pt_fail = 1;   // MMAs of tile i done
+      pt_epi_sync();   // the previous tile's reads of rstd and of the staged rows are done; pt_fail agreed
+      if (pt_fail) {
+        if (etid == 0) report_timeout(a.status, 0xB300);
+        break;
+      }
+      if (a.rscale)
+        for (int r = etid; r < Nt; r += PT_EPI) {
+          const int t = n0 + r;
+          float rs = 0.f;
+          if (t < a.T) {
+            const float4* sp = reinterpret_cast<const float4*>(a.ssq + static_cast<size_t>(t) * a.ssq_ld);
+            float4 v[4];
+            const int nv = a.ssq_ld >> 2;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq)
+              if (qq < nv) v[qq] = sp[qq];
+            float ss = 0.f;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq)
+              if (qq < nv) ss += ((v[qq].x + v[qq].y) + v[qq].z) + v[qq].w;
+            rs = 1.0f / sqrtf(ss / a.D + a.eps);
+          }
+          sh.rstd[r] = rs;   // padded tokens become zero
+        }
+      tc_fence_after();
+      const int f = mb * 64 + p;   // F is a multiple of 64
+      float2 bg = make_float2(0.f, 0.f), bu = make_float2(0.f, 0.f);   // adaptive RMSNorm shift, W b
+      if (a.bias) {
+        bg = *reinterpret_cast<const float2*>(a.bias + f);
+        bu = *reinterpret_cast<const float2*>(a.bias + a.F + f);
+      }
+      for (int cb = 0; cb < Nt; cb += PT_RED_TOK) {
+        const int ce = min(Nt, cb + PT_RED_TOK);
+        if (cb > 0) pt_epi_sync();   // the previous pass's staged rows have been read
+        {
+          const int hc = (((ce - cb) >> 4) + 1) / 2 * 16;
+          const int cbeg = cb + (ew < 4 ? 0 : hc), cend = ew < 4 ? min(cb + hc, ce) : ce;
+          for (int c0 = cbeg; c0 < cend; c0 += 32) {   // up to 2 loads in flight, one wait
+            uint32_t v[2][16];
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+              if (c0 + 16 * u < cend) tmem_ld16_nowait(tacc + (static_cast<uint32_t>(q4 * 32) << 16) + c0 + 16 * u, v[u]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+              if (c0 + 16 * u < cend)
+#pragma unroll
+                for (int j = 0; j < 16; ++j) red[(c0 + 16 * u + j - cb) * RED_LD + row] = __uint_as_float(v[u][j]);
+          }
+        }
+        if (ce == Nt) {   // the accumulator is drained: the MMAs of tile i + 2 may use it
+          tc_fence_before();
+          mbar_arrive(&sh.tempty[acc]);
+        }
+        pt_epi_sync();   // this pass's rows are staged
+        for (int tok = cb + ew; tok < ce; tok += 8) {
+          const int t = n0 + tok;
+          if (t >= a.T) break;
+          const float sc = a.rscale ? al * sh.rstd[tok] : al;
+          const float* rr = red + (tok - cb) * RED_LD;
+          const float g0 = rr[p] * sc + bg.x, g1 = rr[p + 1] * sc + bg.y;
+          const float u0 = rr[p + 64] * sc + bu.x, u1 = rr[p + 65] * sc + bu.y;
+          const size_t uo = btile_offset_nt(nt, tok, 2 * f, Nt, a.NKC_u);
+          if (in_bounds(a.status, uo + 3, a.ext.ubuf, 0x9004))
+            *reinterpret_cast<uint32_t*>(a.u_out + uo) = pack_bf16x2(gelu_tanh(g0) * u0, gelu_tanh(g1) * u1);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
 // ================================================================== attention
 
 struct AttnGeom {
@@ -1672,6 +1908,8 @@ __global__ void k_wait_selftest(unsigned* status, unsigned long long limit_ns) {
 
 }  // namespace
 
+size_t pt_smem_bytes(int Nt, int stages) { return pt_ring_bytes(Nt, stages) + PT_RED_TOK * RED_LD * 4; }
+
 size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4, int epi, int H, int xb,
                        int red_tok) {
   return gemm_rope_off(Nt, stages, b_kind, fp8, S, nk, w4, epi, red_tok) + gemm_stage_bytes(epi, fp8, Nt, S, H, xb);
@@ -1708,7 +1946,8 @@ cudaError_t tc_kernels_init() {
                        reinterpret_cast<const void*>(k_attn_tc<128>), reinterpret_cast<const void*>(k_attn_tc<256>),
                        reinterpret_cast<const void*>(k_attn_umma<64>),
                        reinterpret_cast<const void*>(k_attn_umma<128>), reinterpret_cast<const void*>(k_attn_umma<256>),
-                       reinterpret_cast<const void*>(k_inproj_tc), reinterpret_cast<const void*>(k_final_tc)};
+                       reinterpret_cast<const void*>(k_inproj_tc), reinterpret_cast<const void*>(k_final_tc),
+                       reinterpret_cast<const void*>(k_gemm_gelu_pt)};
   for (const void* f : fns) {
     cudaFuncAttributes fa;
     if ((e = cudaFuncGetAttributes(&fa, f)) != cudaSuccess) return e;
@@ -1767,6 +2006,14 @@ const void* gemm_kernel(int epi, int fp8, int norm, int w4) {
 cudaError_t launch_gemm_tc(const GemmArgs& a, int n_tiles, cudaStream_t s, bool pdl) {
   GemmArgs copy = a;
   void* args[] = {&copy};
+  if (a.persist) {
+    if (a.epi != EPI_GELU || a.fp8 || a.w4 || a.b_kind != B_ROWS || a.S != 1 || a.pt_ctas < 1 ||
+        a.pt_ctas > a.MB * n_tiles || a.Nt > 256)
+      return cudaErrorInvalidValue;
+    copy.pt_nt = n_tiles;
+    return launch_ex(reinterpret_cast<const void*>(k_gemm_gelu_pt), dim3(a.pt_ctas), dim3(PT_THREADS),
+                     pt_smem_bytes(a.Nt, a.stages), s, pdl, 1, args);
+  }
   const int nk_max = (a.NKC + a.S - 1) / a.S;
   const void* f = gemm_kernel(a.epi, a.fp8, a.b_kind == B_NORM, a.w4);
   if (!f) return cudaErrorInvalidValue;

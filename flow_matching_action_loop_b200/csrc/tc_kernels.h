@@ -126,6 +126,8 @@ struct GemmArgs {
   const float* s_a_out;    // fp8: scale of the down-projection input
   int F;
   int red_tok;             // S == 1: tokens per epilogue staging pass (Nt, or fewer so that two CTAs share an SM)
+  int persist;             // 1: the persistent gate|up kernel (one CTA per SM over the tiles; bf16, S == 1)
+  int pt_ctas, pt_nt;      // persistent: CTAs of the launch, n-tiles
   // split-K exchange (S > 1): fp32 partial tiles [NT][MB][S][Nt][128], L2-resident scratch
   float* xscratch;
   unsigned* status;
@@ -238,6 +240,7 @@ const void* final_kernel_ptr();
 cudaError_t tc_kernels_init();    // function attributes (smem opt-in, carveout, non-portable clusters)
 int max_dynamic_smem();           // dynamic shared memory a GEMM CTA may use
 int pair_dynamic_smem();          // dynamic shared memory of a GEMM CTA that shares its SM with another
+size_t pt_smem_bytes(int Nt, int stages);   // dynamic shared memory of the persistent gate|up GEMM
 
 }  // namespace tc
 }  // namespace fr

@@ -59,6 +59,7 @@ ProjLayout make_layout(int rows, int K, int elem, int w4) {
 struct GemmPlan {
   int S = 1, stages = 1;
   int red_tok = 0;   // S == 1: tokens per epilogue staging pass (0: the whole tile)
+  int persist = 0;   // the persistent gate|up kernel
 };
 
 struct StepPlan {
@@ -200,6 +201,18 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, in
     return gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, epi, H, xb, red_tok);
   };
   if (Nt > 64) {
+    // The bf16 gate|up projection with at least two tiles per SM: the persistent kernel (one CTA per
+    // SM walks the tiles; the epilogue of one tile overlaps the MMAs of the next), deepest ring that fits.
+    if (epi == EPI_GELU && !fp8 && !w4 && b_kind == B_ROWS && tiles >= 2 * nsm) {
+      int stages = std::min(NKC, MAX_STAGES);
+      while (stages > 2 && pt_smem_bytes(Nt, stages) > static_cast<size_t>(max_dyn)) --stages;
+      if (stages >= 2 && pt_smem_bytes(Nt, stages) <= static_cast<size_t>(max_dyn)) {
+        best.S = 1;
+        best.stages = stages;
+        best.persist = 1;
+        return best;
+      }
+    }
     // More than one wave of unsplit tiles: two CTAs per SM, so that one CTA's epilogue runs while
     // the other's MMAs do (a ring of at least two slots; the accumulator staged in passes of half
     // the tile when the whole tile does not fit).
@@ -386,6 +399,9 @@ GemmArgs base_args(const TensorPath* tp, const StepPlan& p, const ProjLayout& L,
   a.S = g.S;
   a.stages = g.stages;
   a.red_tok = g.red_tok > 0 ? g.red_tok : p.Nt;
+  a.persist = g.persist;
+  a.pt_nt = p.NT;
+  a.pt_ctas = std::min(L.MB * p.NT, tp->nsm);
   a.fp8 = tp->fp8;
   a.w4 = tp->w4;
   a.Wscale = tp->w4 ? reinterpret_cast<const uint16_t*>(a.W + L.sc_off) : nullptr;
