@@ -729,6 +729,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
 constexpr int PT_THREADS = 320;   // warp 0: copies, warp 1: MMAs, warps 2-9: epilogue
 constexpr int PT_EPI = 256;       // epilogue threads
 constexpr int PT_RED_TOK = 64;    // tokens per epilogue staging pass
+constexpr int PT_KPS = 2;         // k-chunks per ring slot: two large copies per slot (the copy engine of an
+                                  // SM takes about a third of a microsecond per copy, one copy at a time)
 
 struct PtSmem {
   uint64_t full_a[MAX_STAGES], full_b[MAX_STAGES], empty[MAX_STAGES];
@@ -738,7 +740,7 @@ struct PtSmem {
 };
 
 __host__ __device__ __forceinline__ uint32_t pt_ring_bytes(int Nt, int stages) {
-  return static_cast<uint32_t>(stages) * (BM * KCB + static_cast<uint32_t>(Nt) * KCB);
+  return static_cast<uint32_t>(stages) * PT_KPS * (BM * KCB + static_cast<uint32_t>(Nt) * KCB);
 }
 
 __device__ __forceinline__ void pt_epi_sync() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
@@ -753,7 +755,8 @@ __global__ void __launch_bounds__(PT_THREADS, 1) k_gemm_gelu_pt(const __grid_con
   const int Nt = a.Nt, NTl = a.pt_nt, NKC = a.NKC, stages = a.stages;
   const int tiles = a.MB * NTl;
   const int my_tiles = (tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
-  const uint32_t a_bytes = BM * KCB, b_bytes = static_cast<uint32_t>(Nt) * KCB;
+  const uint32_t a_bytes = PT_KPS * BM * KCB, b_bytes = PT_KPS * static_cast<uint32_t>(Nt) * KCB;   // per slot
+  const int NSC = NKC / PT_KPS;   // slots of one tile (NKC is a multiple of PT_KPS)
   auto a_slot = [&](int s) { return dsm + s * a_bytes; };
   auto b_slot = [&](int s) { return dsm + stages * a_bytes + s * b_bytes; };
   float* red = reinterpret_cast<float*>(dsm + pt_ring_bytes(Nt, stages));   // [PT_RED_TOK][RED_LD]
@@ -785,24 +788,24 @@ __global__ void __launch_bounds__(PT_THREADS, 1) k_gemm_gelu_pt(const __grid_con
   tc_fence_after();
   grid_dep_launch();
   const uint32_t tbase = sh.tmem_base;
-  const int total = my_tiles * NKC;   // chunks this CTA streams
+  const int total = my_tiles * NSC;   // ring slots this CTA fills
 
   if (warp == 0) {
-    // ---------------- copies: chunk q is chunk q % NKC of this CTA's tile q / NKC
+    // ---------------- copies: slot fill q holds k-chunks PT_KPS * (q % NSC) .. of this CTA's tile q / NSC
     if (lane == 0) {
       auto issue_a = [&](int q) {
         int mb, nt;
-        tile_of(q / NKC, mb, nt);
+        tile_of(q / NSC, mb, nt);
         const int s = q % stages;
         mbar_arrive_expect_tx(&sh.full_a[s], a_bytes);
-        bulk_g2s(a_slot(s), a.W + (static_cast<size_t>(mb) * NKC + q % NKC) * a_bytes, a_bytes, &sh.full_a[s]);
+        bulk_g2s(a_slot(s), a.W + (static_cast<size_t>(mb) * NSC + q % NSC) * a_bytes, a_bytes, &sh.full_a[s]);
       };
       auto issue_b = [&](int q) {
         int mb, nt;
-        tile_of(q / NKC, mb, nt);
+        tile_of(q / NSC, mb, nt);
         const int s = q % stages;
         mbar_arrive_expect_tx(&sh.full_b[s], b_bytes);
-        bulk_g2s(b_slot(s), a.act + (static_cast<size_t>(nt) * NKC + q % NKC) * b_bytes, b_bytes, &sh.full_b[s]);
+        bulk_g2s(b_slot(s), a.act + (static_cast<size_t>(nt) * NSC + q % NSC) * b_bytes, b_bytes, &sh.full_b[s]);
       };
       const int pre = total < stages ? total : stages;
       for (int q = 0; q < pre; ++q) issue_a(q);   // weights do not depend on the previous kernel
@@ -842,7 +845,7 @@ __global__ void __launch_bounds__(PT_THREADS, 1) k_gemm_gelu_pt(const __grid_con
         }
         tc_fence_after();
         const uint32_t tacc = tbase + static_cast<uint32_t>(acc) * 256u;
-        for (int c = 0; c < NKC; ++c, ++q) {
+        for (int c = 0; c < NSC; ++c, ++q) {
           const int s = q % stages;
           const uint32_t par = (q / stages) & 1;
           if (!mbar_wait(&sh.full_a[s], par, WAIT_LIMIT_NS) || !mbar_wait(&sh.full_b[s], par, WAIT_LIMIT_NS)) {
@@ -851,11 +854,14 @@ __global__ void __launch_bounds__(PT_THREADS, 1) k_gemm_gelu_pt(const __grid_con
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(a_slot(s)), b0 = smem_u32(b_slot(s));
 #pragma unroll
-          for (int k = 0; k < KCB / 32; ++k)
-            mma_bf16(tacc, smem_desc(a0 + k * 2 * BM * 16, BM * 16, 128), smem_desc(b0 + k * 2 * Nt * 16, Nt * 16, 128),
-                     idesc, (c | k) != 0);
+          for (int c2 = 0; c2 < PT_KPS; ++c2) {   // the slot's k-chunks, each a [rows x 128 B] operand tile
+            const uint32_t a0 = smem_u32(a_slot(s) + c2 * BM * KCB), b0 = smem_u32(b_slot(s) + c2 * Nt * KCB);
+#pragma unroll
+            for (int k = 0; k < KCB / 32; ++k)
+              mma_bf16(tacc, smem_desc(a0 + k * 2 * BM * 16, BM * 16, 128), smem_desc(b0 + k * 2 * Nt * 16, Nt * 16, 128),
+                       idesc, (c | c2 | k) != 0);
+          }
           mma_commit(&sh.empty[s]);
         }
         if (ok) mma_commit(&sh.tfull[acc]);
@@ -1387,7 +1393,9 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
   int k_issued = 0, v_issued = 0;
   auto load_kv = [&](const CUtensorMap* tm, uint8_t* dst, uint64_t* bar, int j) {
     mbar_arrive_expect_tx(bar, UA_SUB * DH * 2);
-    for (int x = 0; x < NBX; ++x) tma_load_3d(dst + x * (UA_SUB * 128), tm, x * 64, key0 + j * UA_SUB, zkv, bar);
+    if (a.kv_boxes == 1) tma_load_4d(dst, tm, 0, key0 + j * UA_SUB, 0, zkv, bar);   // [feature block][key][128 B]
+    else
+      for (int x = 0; x < NBX; ++x) tma_load_3d(dst + x * (UA_SUB * 128), tm, x * 64, key0 + j * UA_SUB, zkv, bar);
   };
   auto load_k = [&](int j) {
     load_kv(&a.tm_k, Kbuf(j & 1), &kfull[j & 1], j);
@@ -2008,7 +2016,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int n_tiles, cudaStream_t s, bool 
   void* args[] = {&copy};
   if (a.persist) {
     if (a.epi != EPI_GELU || a.fp8 || a.w4 || a.b_kind != B_ROWS || a.S != 1 || a.pt_ctas < 1 ||
-        a.pt_ctas > a.MB * n_tiles || a.Nt > 256)
+        a.pt_ctas > a.MB * n_tiles || a.Nt > 256 || a.NKC % PT_KPS != 0)
       return cudaErrorInvalidValue;
     copy.pt_nt = n_tiles;
     return launch_ex(reinterpret_cast<const void*>(k_gemm_gelu_pt), dim3(a.pt_ctas), dim3(PT_THREADS),
@@ -2038,17 +2046,27 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// Tensor map of K or V ([planes][keys][dh] bf16, planes plane_bytes apart): boxes of 64 features
-// (128 bytes) x 64 keys x 1 plane, 128-byte swizzle; keys past `keys` read as zeros.
+// Tensor map of K or V ([planes][keys][dh] bf16, planes plane_bytes apart), 128-byte swizzle; keys past
+// `keys` read as zeros.  one_box: the 4-D view (64 features, keys, dh/64 feature blocks, planes) with
+// boxes of 64 x 64 x dh/64 x 1, which land as [feature block][key][128 B] in one copy; otherwise the
+// 3-D view (dh, keys, planes) with boxes of 64 features x 64 keys.
 bool encode_kv_map(CUtensorMap* m, const void* base, uint64_t dh, uint64_t keys, uint64_t planes,
-                   uint64_t plane_bytes) {
+                   uint64_t plane_bytes, bool one_box) {
   const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
   if (!fn || !base || (reinterpret_cast<uintptr_t>(base) & 15u) || keys == 0 || planes == 0 || dh % 64 != 0)
     return false;
+  const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+  if (one_box) {
+    const cuuint64_t dims[4] = {64, keys, dh / 64, planes};
+    const cuuint64_t strides[3] = {dh * 2, 128, plane_bytes};
+    const cuuint32_t box[4] = {64u, 64u, static_cast<cuuint32_t>(dh / 64), 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4u, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
   const cuuint64_t dims[3] = {dh, keys, planes};
   const cuuint64_t strides[2] = {dh * 2, plane_bytes};
   const cuuint32_t box[3] = {64u, 64u, 1u};
-  const cuuint32_t es[3] = {1u, 1u, 1u};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3u, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -2064,8 +2082,15 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int B, cudaStream_t s, bool p
     // K and V [B][Hkv][S_max][dh] as B*Hkv planes of this call's P + H keys (keys past them read as zeros)
     const uint64_t dh = static_cast<uint64_t>(a.dh), keys = static_cast<uint64_t>(a.P + a.H);
     const uint64_t planes = static_cast<uint64_t>(B) * a.Hkv, pb = static_cast<uint64_t>(a.S_max) * dh * 2;
-    if (!encode_kv_map(&copy.tm_k, a.kv_k, dh, keys, planes, pb) || !encode_kv_map(&copy.tm_v, a.kv_v, dh, keys, planes, pb))
-      return cudaErrorInvalidValue;
+    // one copy per sub-chunk where the driver accepts the 4-D view, else dh/64 copies
+    copy.kv_boxes = 1;
+    if (!encode_kv_map(&copy.tm_k, a.kv_k, dh, keys, planes, pb, true) ||
+        !encode_kv_map(&copy.tm_v, a.kv_v, dh, keys, planes, pb, true)) {
+      copy.kv_boxes = static_cast<int>(dh / 64);
+      if (!encode_kv_map(&copy.tm_k, a.kv_k, dh, keys, planes, pb, false) ||
+          !encode_kv_map(&copy.tm_v, a.kv_v, dh, keys, planes, pb, false))
+        return cudaErrorInvalidValue;
+    }
     const void* f = a.dh == 64 ? reinterpret_cast<const void*>(k_attn_umma<64>)
                   : a.dh == 128 ? reinterpret_cast<const void*>(k_attn_umma<128>)
                                 : reinterpret_cast<const void*>(k_attn_umma<256>);

@@ -152,8 +152,10 @@ struct AttnArgs {
   int umma;                    // 1: tcgen05 kernel over GQA-group tiles; 0: warp-MMA kernel per query head
   uint64_t o_extent;           // bytes of o (checked builds)
   // tcgen05 kernel: tensor maps of this layer's K and V ([B*Hkv][P+H][dh], planes S_max rows apart),
-  // boxes of 64 features x 64 keys with 128-byte swizzle; written by launch_attention_tc
+  // 128-byte swizzle; written by launch_attention_tc.  kv_boxes == 1: one box per 64-key sub-chunk
+  // (64 features x 64 keys x dh/64 feature blocks, a 4-D view); otherwise dh/64 boxes of 64 x 64
   CUtensorMap tm_k, tm_v;
+  int kv_boxes;
 };
 
 // Key chunks of the split-KV attention over S keys: at most 16 (one cluster), each a multiple

@@ -203,8 +203,8 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, in
   if (Nt > 64) {
     // The bf16 gate|up projection with at least two tiles per SM: the persistent kernel (one CTA per
     // SM walks the tiles; the epilogue of one tile overlaps the MMAs of the next), deepest ring that fits.
-    if (epi == EPI_GELU && !fp8 && !w4 && b_kind == B_ROWS && tiles >= 2 * nsm) {
-      int stages = std::min(NKC, MAX_STAGES);
+    if (epi == EPI_GELU && !fp8 && !w4 && b_kind == B_ROWS && tiles >= 2 * nsm && NKC % 2 == 0) {
+      int stages = std::min(NKC / 2, MAX_STAGES);   // ring slots of two k-chunks
       while (stages > 2 && pt_smem_bytes(Nt, stages) > static_cast<size_t>(max_dyn)) --stages;
       if (stages >= 2 && pt_smem_bytes(Nt, stages) <= static_cast<size_t>(max_dyn)) {
         best.S = 1;
