@@ -371,10 +371,15 @@ def main(argv=None):
     ap.add_argument("--workload", default="pi05_bf16_b1", help="a workload name, or 'all' (one line each)")
     ap.add_argument("--no-extra", action="store_true", help="headline workload only (no 'workloads' object)")
     ap.add_argument("--path", type=int, default=0, help="FR_PATH_* (0 auto, 1 stepwise, 2 tensor)")
+    ap.add_argument("--exec", dest="exec_mode", default="auto", choices=["auto", "graph", "persistent"],
+                    help="execution of fr_denoise (FR_EXEC_*): the library's choice, the CUDA graph, or the "
+                         "persistent kernel (batch-1-sized calls)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-steps", type=int, default=10, help="oracle Euler steps timed for cpu_baseline")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
+    if args.exec_mode == "persistent":   # the persistent kernel serves batch-1-sized calls only
+        args.no_extra = True
 
     import synthetic
     if args.workload in synthetic.PREFIX_CONFIGS:
@@ -424,6 +429,9 @@ def run_loop(cfg, args, world, rank, local, steps, warmup, cpu_steps):
     loop = ActionExpertLoop(cfg, device=local, path=args.path)
     if args.path == 0 and cfg.dtype != "f32" and loop.path != "tensor":
         raise SystemExit(f"{cfg.name}: the automatic kernel set is {loop.path!r}, expected the tensor path")
+    if args.exec_mode != "auto":
+        from flow_matching_action_loop_b200 import FR_EXEC_GRAPH, FR_EXEC_PERSISTENT
+        loop.set_exec_mode(FR_EXEC_GRAPH if args.exec_mode == "graph" else FR_EXEC_PERSISTENT)
     loop.load_weights(inp["weights"])
     if cfg.dtype == "fp8":
         obs = synthetic.make_observation(cfg, 1)
@@ -527,7 +535,7 @@ def run_loop(cfg, args, world, rank, local, steps, warmup, cpu_steps):
         "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded, random-init)",
         "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * world, "parallelism": f"replicas x{world}",
-                   "l2": l2_note, "path": loop.path, "kernel_digest": digest},
+                   "l2": l2_note, "path": loop.path, "exec": args.exec_mode, "kernel_digest": digest},
         "per_replica_us_per_chunk": round(ms_local * 1e3 / (steps * cfg.B), 2),
         "chunks_per_s": round(chunks / (ms * 1e-3), 1),
         "achieved_hbm_gbs": round(wb["per_chunk"] / (ms_per_step * 1e-3) / 1e9, 1),
