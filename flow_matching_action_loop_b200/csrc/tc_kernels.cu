@@ -107,11 +107,11 @@ constexpr uint32_t W4_CHUNK = BM * KCB / 4;   // 4-bit codes of one 128 x 64 wei
 __host__ __device__ __forceinline__ int w4_groups(int kc0, int nk) { return nk > 0 ? (kc0 + nk - 1) / 2 - kc0 / 2 + 1 : 0; }
 
 __host__ __device__ __forceinline__ GemmGeom gemm_geom(int Nt, int stages, int b_kind, int fp8, int S, int nk,
-                                                       int w4 = 0, int kc0 = 0) {
+                                                       int w4 = 0, int kc0 = 0, int kpu = 1) {
   GemmGeom g;
-  g.a_bytes = BM * KCB;
+  g.a_bytes = BM * KCB * static_cast<uint32_t>(kpu);   // one ring slot: kpu consecutive k-chunks
   g.raw_bytes = 0;   // B_NORM converters read h from global memory straight into the operand tile
-  g.breg = static_cast<uint32_t>(Nt) * KCB;
+  g.breg = static_cast<uint32_t>(Nt) * KCB * static_cast<uint32_t>(kpu);
   g.slot = g.a_bytes + g.breg;
   g.ring = g.slot * static_cast<uint32_t>(stages);
   g.TS = (Nt + S - 1) / S;
@@ -150,8 +150,8 @@ __host__ __device__ __forceinline__ int nk_max_of(const GemmArgs& a) { return (a
 // Bytes of the main loop and epilogue regions; the QKV epilogue's RoPE stage ([H][64] (cos, sin)
 // pairs of the m-block) follows them.
 __host__ __device__ __forceinline__ uint32_t gemm_rope_off(int Nt, int stages, int b_kind, int fp8, int S, int nk,
-                                                          int w4, int epi_kind, int red_tok) {
-  const GemmGeom g = gemm_geom(Nt, stages, b_kind, fp8, S, nk, w4, 1);   // kc0 odd: the larger group count
+                                                          int w4, int epi_kind, int red_tok, int kpu) {
+  const GemmGeom g = gemm_geom(Nt, stages, b_kind, fp8, S, nk, w4, 1, kpu);   // kc0 odd: the larger group count
   const uint32_t kel = fp8 ? KCB : KCB / 2;
   const uint32_t main = g.gamma_off + (b_kind == B_NORM ? static_cast<uint32_t>(nk) * kel * 4u : 0u);
   const uint32_t TS = (Nt + S - 1) / S;
@@ -176,11 +176,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   const int n0 = nt * Nt;
   const int S = a.S;
   const int kc0 = ks * a.NKC / S, kc1 = (ks + 1) * a.NKC / S;
-  const int nk = kc1 - kc0;
+  // KPU consecutive k-chunks per ring slot (two only without B_NORM and 4-bit weights, with every
+  // rank's chunk count even): one copy per operand and slot, fewer copies for the SM's copy engine
+  const int KPU = (NORM || W4) ? 1 : a.kpu;
+  const int nk = (kc1 - kc0) / KPU;   // ring slot fills of this CTA
   const int stages = a.stages;
   constexpr int norm = NORM;
   const int kel = FP8 ? KCB : KCB / 2;            // K elements per chunk
-  const GemmGeom gm = gemm_geom(Nt, stages, NORM ? B_NORM : B_ROWS, FP8, S, nk, W4, kc0);
+  const GemmGeom gm = gemm_geom(Nt, stages, NORM ? B_NORM : B_ROWS, FP8, S, nk, W4, kc0, KPU);
   const int g0 = kc0 / 2;                          // w4: first scale group of this CTA's k-range
   // ring slot addresses: B_NORM interleaves [A | raw h] per slot; otherwise the A slots come first and
   // the B slots follow contiguously, so that the B chunks resident before the main loop arrive in one copy
@@ -217,7 +220,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   const uint32_t tacc = sh.tmem_base;
   // QKV: (cos, sin) of this m-block's 64 rotate-half pairs at every action position, staged while
   // the previous kernel runs (the tables are static); read by the epilogue after the main loop
-  float2* rope_sh = reinterpret_cast<float2*>(dsm + gemm_rope_off(Nt, stages, NORM ? B_NORM : B_ROWS, FP8, S, nk_max_of(a), W4, EPI, a.red_tok));
+  float2* rope_sh = reinterpret_cast<float2*>(dsm + gemm_rope_off(Nt, stages, NORM ? B_NORM : B_ROWS, FP8, S, nk_max_of(a), W4, EPI, a.red_tok, KPU));
   if (EPI == EPI_QKV && mb < a.MB_rot && warp >= 2) {   // warps 2-7: the producer and MMA warps go on
     const int half = a.dh >> 1;
     const bool by_tok = rope_by_token(a.H, Nt);
@@ -231,14 +234,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   if (warp == 0) {
     // ---------------- bulk-copy producer
     if (lane == 0) {
-      const uint8_t* wsrc = a.W + (static_cast<size_t>(mb) * a.NKC + kc0) * gm.a_bytes;
+      const uint8_t* wsrc = a.W + (static_cast<size_t>(mb) * a.NKC + kc0) * (BM * KCB);
+      const uint32_t tb1 = static_cast<uint32_t>(Nt) * KCB;   // one k-chunk of B
       auto issue_b = [&](int i) {
         const int s = i % stages;
         uint8_t* bdst = b_slot(s);
         if (!norm) {   // B_NORM: the converters fill the slot
-          const uint32_t tb = static_cast<uint32_t>(Nt) * KCB;
-          mbar_arrive_expect_tx(&sh.full_b[s], tb);
-          bulk_g2s(bdst, a.act + (static_cast<size_t>(nt) * a.NKC + kc0 + i) * tb, tb, &sh.full_b[s]);
+          mbar_arrive_expect_tx(&sh.full_b[s], KPU * tb1);
+          bulk_g2s(bdst, a.act + (static_cast<size_t>(nt) * a.NKC + kc0 + i * KPU) * tb1, KPU * tb1, &sh.full_b[s]);
         }
       };
       const uint8_t* w4src = a.W + (static_cast<size_t>(mb) * a.NKC + kc0) * W4_CHUNK;
@@ -262,9 +265,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       grid_dep_wait();
       TL(1);
       if (!NORM && Nt <= 64) {   // batch-1 tiles: B chunks 0..pre-1 are contiguous in global and in shared memory: one copy
-        const uint32_t tb = static_cast<uint32_t>(Nt) * KCB;
+        const uint32_t tb = KPU * tb1;
         mbar_arrive_expect_tx(&sh.full_b[0], pre * tb);
-        bulk_g2s(b_slot(0), a.act + (static_cast<size_t>(nt) * a.NKC + kc0) * tb, pre * tb, &sh.full_b[0]);
+        bulk_g2s(b_slot(0), a.act + (static_cast<size_t>(nt) * a.NKC + kc0) * tb1, pre * tb, &sh.full_b[0]);
         for (int i = 1; i < pre; ++i) mbar_arrive(&sh.full_b[i]);   // their first fill is covered by slot 0's copy
       } else {
         for (int i = 0; i < pre; ++i) issue_b(i);
@@ -315,8 +318,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
         tc_fence_after();
         if (i == 0) TL(6);
         const uint32_t a0 = smem_u32(a_slot(s)), b0 = smem_u32(b_slot(s));
-#pragma unroll
-        for (int k = 0; k < KCB / 32; ++k) {
+        // the slot's KPU k-chunks continue the 16-byte core-matrix columns of the first (LBO apart)
+        for (int k = 0; k < KPU * (KCB / 32); ++k) {
           const uint64_t ad = smem_desc(a0 + k * 2 * BM * 16, BM * 16, 128);
           const uint64_t bd = smem_desc(b0 + k * 2 * Nt * 16, Nt * 16, 128);
           if (FP8) mma_e4m3(tacc, ad, bd, idesc, (i | k) != 0);
@@ -1919,8 +1922,8 @@ __global__ void k_wait_selftest(unsigned* status, unsigned long long limit_ns) {
 size_t pt_smem_bytes(int Nt, int stages) { return pt_ring_bytes(Nt, stages) + PT_RED_TOK * RED_LD * 4; }
 
 size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4, int epi, int H, int xb,
-                       int red_tok) {
-  return gemm_rope_off(Nt, stages, b_kind, fp8, S, nk, w4, epi, red_tok) + gemm_stage_bytes(epi, fp8, Nt, S, H, xb);
+                       int red_tok, int kpu) {
+  return gemm_rope_off(Nt, stages, b_kind, fp8, S, nk, w4, epi, red_tok, kpu) + gemm_stage_bytes(epi, fp8, Nt, S, H, xb);
 }
 
 size_t gemm_scratch_bytes(int NT, int MB, int S, int Nt) {
@@ -2026,7 +2029,8 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int n_tiles, cudaStream_t s, bool 
   const void* f = gemm_kernel(a.epi, a.fp8, a.b_kind == B_NORM, a.w4);
   if (!f) return cudaErrorInvalidValue;
   return launch_ex(f, dim3(a.S, n_tiles, a.MB), dim3(GEMM_THREADS),
-                   gemm_smem_bytes(a.Nt, a.stages, a.b_kind, a.fp8, a.S, nk_max, a.w4, a.epi, a.H, a.xb_out != nullptr, a.red_tok), s,
+                   gemm_smem_bytes(a.Nt, a.stages, a.b_kind, a.fp8, a.S, nk_max, a.w4, a.epi, a.H, a.xb_out != nullptr, a.red_tok,
+                                   a.kpu), s,
                    pdl, a.S, args);
 }
 

@@ -126,6 +126,7 @@ struct GemmArgs {
   const float* s_a_out;    // fp8: scale of the down-projection input
   int F;
   int red_tok;             // S == 1: tokens per epilogue staging pass (Nt, or fewer so that two CTAs share an SM)
+  int kpu;                 // k-chunks per ring slot (1, or 2 without B_NORM / 4-bit weights when every rank's count is even)
   int persist;             // 1: the persistent gate|up kernel (one CTA per SM over the tiles; bf16, S == 1)
   int pt_ctas, pt_nt;      // persistent: CTAs of the launch, n-tiles
   // split-K exchange (S > 1): fp32 partial tiles [NT][MB][S][Nt][128], L2-resident scratch
@@ -233,7 +234,7 @@ cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaS
 cudaError_t launch_to_bf16_t(const float* src, __nv_bfloat16* dst, int rows, int cols, cudaStream_t s);
 cudaError_t launch_wait_selftest(unsigned* status, unsigned long long limit_ns, cudaStream_t s);
 size_t gemm_smem_bytes(int Nt, int stages, int b_kind, int fp8, int S, int nk, int w4, int epi, int H, int xb,
-                       int red_tok);
+                       int red_tok, int kpu);
 size_t gemm_scratch_bytes(int NT, int MB, int S, int Nt);
 size_t attn_scratch_bytes(int B, int Hq, int C, int H, int dh);
 size_t attn_smem_bytes(int H, int dh, int KC, int C, int umma);

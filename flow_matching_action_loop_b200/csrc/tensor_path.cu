@@ -60,6 +60,7 @@ struct GemmPlan {
   int S = 1, stages = 1;
   int red_tok = 0;   // S == 1: tokens per epilogue staging pass (0: the whole tile)
   int persist = 0;   // the persistent gate|up kernel
+  int kpu = 1;       // k-chunks per ring slot
 };
 
 struct StepPlan {
@@ -197,8 +198,11 @@ void init_sizes(TensorPath* tp, const fr_config& c) {
 GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, int epi, int H, int xb, int nsm,
                      int max_dyn, int max_dyn2) {
   GemmPlan best;
+  // k-chunks per ring slot for split S: two when every rank's chunk count is even and the operands
+  // arrive by bulk copy (not B_NORM, not 4-bit weights) -- one copy per operand and slot
+  auto kpu_of = [&](int S) { return (b_kind == B_ROWS && !w4 && NKC % (2 * S) == 0) ? 2 : 1; };
   auto smem = [&](int S, int stages, int chunks, int red_tok) {
-    return gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, epi, H, xb, red_tok);
+    return gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, epi, H, xb, red_tok, kpu_of(S));
   };
   if (Nt > 64) {
     // The bf16 gate|up projection with at least two tiles per SM: the persistent kernel (one CTA per
@@ -217,14 +221,15 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, in
     // the other's MMAs do (a ring of at least two slots; the accumulator staged in passes of half
     // the tile when the whole tile does not fit).
     if (tiles > nsm && max_dyn2 > 0) {
-      const int chunks = NKC;
+      const int chunks = NKC, units = NKC / kpu_of(1);
       for (int red_tok : {Nt, static_cast<int>(align_up(ceil_div(Nt, 2), 16))}) {
-        int stages = std::min(chunks, MAX_STAGES);
+        int stages = std::min(units, MAX_STAGES);
         while (stages > 2 && smem(1, stages, chunks, red_tok) > static_cast<size_t>(max_dyn2)) --stages;
         if (stages >= 2 && smem(1, stages, chunks, red_tok) <= static_cast<size_t>(max_dyn2)) {
           best.S = 1;
           best.stages = stages;
           best.red_tok = red_tok;
+          best.kpu = kpu_of(1);
           return best;
         }
       }
@@ -234,11 +239,12 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, in
     const int pref = (tiles * 2 <= nsm && NKC >= 2) ? 2 : 1;
     for (int S : {pref, 3 - pref}) {
       if (S > NKC) continue;
-      const int chunks = ceil_div(NKC, S);
-      int stages = std::min(chunks, MAX_STAGES);
+      const int chunks = ceil_div(NKC, S), units = chunks / kpu_of(S);
+      int stages = std::min(units, MAX_STAGES);
       while (stages > 1 && smem(S, stages, chunks, Nt) > static_cast<size_t>(max_dyn)) --stages;
       best.S = S;
       best.stages = stages;
+      best.kpu = kpu_of(S);
       if (smem(S, stages, chunks, Nt) <= static_cast<size_t>(max_dyn)) return best;
     }
     return best;   // nothing fits: the launch reports it
@@ -247,16 +253,18 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, in
   const size_t cap = std::min<size_t>(static_cast<size_t>(max_dyn), max_dyn2 > 0 ? static_cast<size_t>(max_dyn2) : 110 * 1024);
   double best_cost = 1e30;
   for (int S = 1; S <= 16 && S <= NKC; ++S) {
-    const int chunks = ceil_div(NKC, S);
-    int stages = std::min(chunks, MAX_STAGES);
+    const int chunks = ceil_div(NKC, S), units = chunks / kpu_of(S);   // slot fills per CTA
+    int stages = std::min(units, MAX_STAGES);
     while (stages > 1 && smem(S, stages, chunks, Nt) > cap) --stages;
     if (smem(S, stages, chunks, Nt) > static_cast<size_t>(max_dyn)) continue;
     const int waves = ceil_div(tiles * S, nsm);
-    const double cost = waves * (1.0 + (S > 1 ? 1.0 : 0.0) + 0.3 * (chunks - stages) + 0.05 * chunks);
+    // streamed slots after the dependency wait; the copies in the cost count k-chunks
+    const double cost = waves * (1.0 + (S > 1 ? 1.0 : 0.0) + 0.3 * kpu_of(S) * (units - stages) + 0.05 * chunks);
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best.S = S;
       best.stages = stages;
+      best.kpu = kpu_of(S);
     }
   }
   return best;
@@ -400,6 +408,7 @@ GemmArgs base_args(const TensorPath* tp, const StepPlan& p, const ProjLayout& L,
   a.stages = g.stages;
   a.red_tok = g.red_tok > 0 ? g.red_tok : p.Nt;
   a.persist = g.persist;
+  a.kpu = g.kpu;
   a.pt_nt = p.NT;
   a.pt_ctas = std::min(L.MB * p.NT, tp->nsm);
   a.fp8 = tp->fp8;
