@@ -221,16 +221,22 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, in
     // the other's MMAs do (a ring of at least two slots; the accumulator staged in passes of half
     // the tile when the whole tile does not fit).
     if (tiles > nsm && max_dyn2 > 0) {
-      const int chunks = NKC, units = NKC / kpu_of(1);
-      for (int red_tok : {Nt, static_cast<int>(align_up(ceil_div(Nt, 2), 16))}) {
-        int stages = std::min(units, MAX_STAGES);
-        while (stages > 2 && smem(1, stages, chunks, red_tok) > static_cast<size_t>(max_dyn2)) --stages;
-        if (stages >= 2 && smem(1, stages, chunks, red_tok) <= static_cast<size_t>(max_dyn2)) {
-          best.S = 1;
-          best.stages = stages;
-          best.red_tok = red_tok;
-          best.kpu = kpu_of(1);
-          return best;
+      const int chunks = NKC;
+      // two-chunk slots where two of them still fit half an SM, else one-chunk slots: two CTAs per SM
+      // matter more than fewer copies
+      for (int kpu : {kpu_of(1), 1}) {
+        const int units = NKC / kpu;
+        for (int red_tok : {Nt, static_cast<int>(align_up(ceil_div(Nt, 2), 16))}) {
+          int stages = std::min(units, MAX_STAGES);
+          auto sm = [&](int st) { return gemm_smem_bytes(Nt, st, b_kind, fp8, 1, chunks, w4, epi, H, xb, red_tok, kpu); };
+          while (stages > 2 && sm(stages) > static_cast<size_t>(max_dyn2)) --stages;
+          if (stages >= 2 && sm(stages) <= static_cast<size_t>(max_dyn2)) {
+            best.S = 1;
+            best.stages = stages;
+            best.red_tok = red_tok;
+            best.kpu = kpu;
+            return best;
+          }
         }
       }
     }
