@@ -83,7 +83,6 @@ __device__ __forceinline__ void conv_sync() { asm volatile("bar.sync 1, 192;" ::
 struct GemmSmem {
   uint64_t full_a[MAX_STAGES];
   uint64_t full_b[MAX_STAGES];
-  uint64_t raw_b[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
   uint64_t done;
   uint64_t hbar;      // residual rows of this CTA's tokens (EPI_RESID, S > 1)
@@ -96,7 +95,7 @@ struct GemmSmem {
 };
 
 struct GemmGeom {
-  uint32_t a_bytes, breg, slot, raw_bytes, ring, gamma_off, recv_off;
+  uint32_t a_bytes, breg, slot, ring, gamma_off, recv_off;
   uint32_t rawa_off, scl_off;   // w4: raw 4-bit chunks [stages][4 KB], bf16 scales [groups][128]
   int TS;
 };
@@ -110,7 +109,7 @@ __host__ __device__ __forceinline__ GemmGeom gemm_geom(int Nt, int stages, int b
                                                        int w4 = 0, int kc0 = 0, int kpu = 1) {
   GemmGeom g;
   g.a_bytes = BM * KCB * static_cast<uint32_t>(kpu);   // one ring slot: kpu consecutive k-chunks
-  g.raw_bytes = 0;   // B_NORM converters read h from global memory straight into the operand tile
+  // (B_NORM: the converters read h from global memory straight into the B slot)
   g.breg = static_cast<uint32_t>(Nt) * KCB * static_cast<uint32_t>(kpu);
   g.slot = g.a_bytes + g.breg;
   g.ring = g.slot * static_cast<uint32_t>(stages);
@@ -185,7 +184,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
   const int kel = FP8 ? KCB : KCB / 2;            // K elements per chunk
   const GemmGeom gm = gemm_geom(Nt, stages, NORM ? B_NORM : B_ROWS, FP8, S, nk, W4, kc0, KPU);
   const int g0 = kc0 / 2;                          // w4: first scale group of this CTA's k-range
-  // ring slot addresses: B_NORM interleaves [A | raw h] per slot; otherwise the A slots come first and
+  // ring slot addresses: B_NORM interleaves [A | B] per slot; otherwise the A slots come first and
   // the B slots follow contiguously, so that the B chunks resident before the main loop arrive in one copy
   auto a_slot = [&](int s) -> uint8_t* { return dsm + (NORM ? s * gm.slot : s * gm.a_bytes); };
   auto b_slot = [&](int s) -> uint8_t* {
@@ -198,7 +197,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const __grid_consta
       mbar_init(&sh.full_a[s], W4 ? CONV_THREADS : 1);   // w4: the converters hand each chunk over
       mbar_init(&sh.raw_a[s], 1);
       mbar_init(&sh.full_b[s], norm ? CONV_THREADS : 1);
-      mbar_init(&sh.raw_b[s], 1);
       mbar_init(&sh.empty[s], 1);
     }
     mbar_init(&sh.done, 1);
