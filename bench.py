@@ -362,7 +362,8 @@ def run_prefix(args, cfg):
     return 0
 
 
-def main(argv=None):
+def parse_args(argv=None):
+    """Command-line options; --exec persistent times the headline batch-1 workload only."""
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
@@ -380,6 +381,11 @@ def main(argv=None):
     args.warmup = max(args.warmup, 3)
     if args.exec_mode == "persistent":   # the persistent kernel serves batch-1-sized calls only
         args.no_extra = True
+    return args
+
+
+def main(argv=None):
+    args = parse_args(argv)
 
     import synthetic
     if args.workload in synthetic.PREFIX_CONFIGS:

@@ -89,3 +89,16 @@ def test_reference_arm_is_silent_on_other_ranks(capsys, monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "2")
     assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"]) == 0
     assert capsys.readouterr().out.strip() == ""
+
+
+def test_options_warmup_floor_and_persistent_headline_only():
+    """At least three warm-up calls; `--exec persistent` times the batch-1 headline workload only (the
+    persistent kernel serves batch-1-sized calls), with no other workloads in the line."""
+    a = bench.parse_args(["--warmup", "1"])
+    assert a.warmup == 3 and a.exec_mode == "auto" and not a.no_extra
+    a = bench.parse_args(["--exec", "persistent"])
+    assert a.exec_mode == "persistent" and a.no_extra
+    a = bench.parse_args(["--exec", "graph", "--workload", "pi05_bf16_b32"])
+    assert a.exec_mode == "graph" and not a.no_extra and a.workload == "pi05_bf16_b32"
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--exec", "eager"])
