@@ -112,6 +112,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fr_set_wait_limit": (c_int, [H, ctypes.c_uint64]),
         "fr_device_checks": (c_int, []),
         "fr_debug_limit_extent": (c_int, [H, c_char_p, ctypes.c_uint64]),
+        "fr_debug_plan": (c_int, [ctypes.POINTER(FrConfig), c_int, c_int, c_int, c_int, c_int, ctypes.POINTER(c_int), c_int]),
         "fr_rope_tables": (c_int, [c_int, c_int, ctypes.c_double, _FP, _FP]),
         "fr_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                  c_void_p, ctypes.c_size_t, c_void_p]),
@@ -318,6 +319,22 @@ def fr_exec_mode(h, B: int) -> int:
 
 def fr_device_checks() -> bool:
     return load_library().fr_device_checks() == 1
+
+
+PLAN_GEMMS = ("qkv", "o", "gate_up", "down")
+PLAN_GEMM_FIELDS = ("S", "stages", "red_tok", "persist", "kpu", "smem", "tiles", "NKC")
+
+
+def fr_debug_plan(cfg, B: int, P: int, nsm: int, max_dyn: int, max_dyn2: int) -> dict:
+    """The tensor-core path's launch plan of one call, computed on the host (no device)."""
+    out = (ctypes.c_int * 64)()
+    n = _check(load_library().fr_debug_plan(ctypes.byref(cfg), B, P, nsm, max_dyn, max_dyn2, out, 64), "fr_debug_plan")
+    v = list(out[:n])
+    plan = {"NT": v[0], "Nt": v[1]}
+    for i, name in enumerate(PLAN_GEMMS):
+        plan[name] = dict(zip(PLAN_GEMM_FIELDS, v[2 + 8 * i: 10 + 8 * i]))
+    plan["attn_umma"], plan["attn_C"], plan["attn_KC"] = v[34:37]
+    return plan
 
 
 def fr_debug_limit_extent(h, buffer: str, elems: int) -> None:

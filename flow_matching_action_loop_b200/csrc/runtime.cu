@@ -1210,6 +1210,25 @@ int fr_device_checks(void) {
 #endif
 }
 
+int fr_debug_plan(const fr_config* cfg, int B, int P, int nsm, int max_dyn, int max_dyn2, int* out, int n_out) {
+  if (!cfg || !out || n_out < 0 || nsm < 1 || max_dyn < 1 || max_dyn2 < 0) {
+    set_error("fr_debug_plan: NULL or non-positive argument");
+    return FR_ERR_ARG;
+  }
+  int rc = validate(*cfg);
+  if (rc) return rc;
+  if (!tensor_path_supports(*cfg)) {
+    set_error("fr_debug_plan: the configuration is outside the tensor-core path (%s)", tensor_path_limits());
+    return FR_ERR_UNSUPPORTED;
+  }
+  const int p_max = cfg->role == FR_ROLE_PREFIX ? cfg->H : cfg->P_max;
+  if (B < 1 || B > cfg->B_max || P < 1 || P > p_max) {
+    set_error("fr_debug_plan: B must be in [1, B_max] and P in [1, %d]", p_max);
+    return FR_ERR_SHAPE;
+  }
+  return tensor_path_debug_plan(*cfg, B, P, nsm, max_dyn, max_dyn2, out, n_out);
+}
+
 int fr_debug_limit_extent(fr_handle* h, const char* buffer, uint64_t elems) {
   if (!h || !buffer) {
     set_error("fr_debug_limit_extent: NULL argument");

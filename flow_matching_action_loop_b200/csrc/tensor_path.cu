@@ -200,9 +200,17 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, in
   GemmPlan best;
   // k-chunks per ring slot for split S: two when every rank's chunk count is even and the operands
   // arrive by bulk copy (not B_NORM, not 4-bit weights) -- one copy per operand and slot
-  auto kpu_of = [&](int S) { return (b_kind == B_ROWS && !w4 && NKC % (2 * S) == 0) ? 2 : 1; };
-  auto smem = [&](int S, int stages, int chunks, int red_tok) {
-    return gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, epi, H, xb, red_tok, kpu_of(S));
+  auto kpu_ok = [&](int S) { return b_kind == B_ROWS && !w4 && NKC % (2 * S) == 0; };
+  auto smem_k = [&](int S, int stages, int chunks, int red_tok, int kpu) {
+    return gemm_smem_bytes(Nt, stages, b_kind, fp8, S, chunks, w4, epi, H, xb, red_tok, kpu);
+  };
+  // two-chunk slots only where the ring still double-buffers (or holds the whole k-range at once)
+  auto kpu_of = [&](int S, size_t limit) {
+    if (!kpu_ok(S)) return 1;
+    const int chunks = ceil_div(NKC, S), units = chunks / 2;
+    int stages = std::min(units, MAX_STAGES);
+    while (stages > 1 && smem_k(S, stages, chunks, Nt, 2) > limit) --stages;
+    return (stages >= 2 || stages == units) && smem_k(S, stages, chunks, Nt, 2) <= limit ? 2 : 1;
   };
   if (Nt > 64) {
     // The bf16 gate|up projection with at least two tiles per SM: the persistent kernel (one CTA per
@@ -224,7 +232,7 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, in
       const int chunks = NKC;
       // two-chunk slots where two of them still fit half an SM, else one-chunk slots: two CTAs per SM
       // matter more than fewer copies
-      for (int kpu : {kpu_of(1), 1}) {
+      for (int kpu : {kpu_ok(1) ? 2 : 1, 1}) {
         const int units = NKC / kpu;
         for (int red_tok : {Nt, static_cast<int>(align_up(ceil_div(Nt, 2), 16))}) {
           int stages = std::min(units, MAX_STAGES);
@@ -245,13 +253,14 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, in
     const int pref = (tiles * 2 <= nsm && NKC >= 2) ? 2 : 1;
     for (int S : {pref, 3 - pref}) {
       if (S > NKC) continue;
-      const int chunks = ceil_div(NKC, S), units = chunks / kpu_of(S);
+      const int kpu = kpu_of(S, static_cast<size_t>(max_dyn));
+      const int chunks = ceil_div(NKC, S), units = chunks / kpu;
       int stages = std::min(units, MAX_STAGES);
-      while (stages > 1 && smem(S, stages, chunks, Nt) > static_cast<size_t>(max_dyn)) --stages;
+      while (stages > 1 && smem_k(S, stages, chunks, Nt, kpu) > static_cast<size_t>(max_dyn)) --stages;
       best.S = S;
       best.stages = stages;
-      best.kpu = kpu_of(S);
-      if (smem(S, stages, chunks, Nt) <= static_cast<size_t>(max_dyn)) return best;
+      best.kpu = kpu;
+      if (smem_k(S, stages, chunks, Nt, kpu) <= static_cast<size_t>(max_dyn)) return best;
     }
     return best;   // nothing fits: the launch reports it
   }
@@ -259,18 +268,19 @@ GemmPlan choose_plan(int tiles, int NKC, int Nt, int b_kind, int fp8, int w4, in
   const size_t cap = std::min<size_t>(static_cast<size_t>(max_dyn), max_dyn2 > 0 ? static_cast<size_t>(max_dyn2) : 110 * 1024);
   double best_cost = 1e30;
   for (int S = 1; S <= 16 && S <= NKC; ++S) {
-    const int chunks = ceil_div(NKC, S), units = chunks / kpu_of(S);   // slot fills per CTA
+    const int kpu = kpu_of(S, cap);
+    const int chunks = ceil_div(NKC, S), units = chunks / kpu;   // slot fills per CTA
     int stages = std::min(units, MAX_STAGES);
-    while (stages > 1 && smem(S, stages, chunks, Nt) > cap) --stages;
-    if (smem(S, stages, chunks, Nt) > static_cast<size_t>(max_dyn)) continue;
+    while (stages > 1 && smem_k(S, stages, chunks, Nt, kpu) > cap) --stages;
+    if (smem_k(S, stages, chunks, Nt, kpu) > static_cast<size_t>(max_dyn)) continue;
     const int waves = ceil_div(tiles * S, nsm);
     // streamed slots after the dependency wait; the copies in the cost count k-chunks
-    const double cost = waves * (1.0 + (S > 1 ? 1.0 : 0.0) + 0.3 * kpu_of(S) * (units - stages) + 0.05 * chunks);
+    const double cost = waves * (1.0 + (S > 1 ? 1.0 : 0.0) + 0.3 * kpu * (units - stages) + 0.05 * chunks);
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best.S = S;
       best.stages = stages;
-      best.kpu = kpu_of(S);
+      best.kpu = kpu;
     }
   }
   return best;
@@ -893,6 +903,37 @@ bool tensor_path_supports(const fr_config& c) {
   attn_chunks(c.P_max + c.H, C, KC);
   if (attn_smem_bytes(c.H, c.dh, KC, C, 0) > 200 * 1024) return false;
   return true;
+}
+
+// The launch plan of one call for a device of nsm SMs and the given dynamic shared-memory limits, on the
+// host only (no device state): the token tiling, per projection (QKV, O, gate|up, down) the split, ring,
+// staging pass, kernel, k-chunks per slot, shared memory, tiles and k-chunks, then the attention kernel
+// and key split.  Returns the number of ints written.
+int tensor_path_debug_plan(const fr_config& c, int B, int P, int nsm, int max_dyn, int max_dyn2, int* out, int n_out) {
+  TensorPath tp;
+  init_sizes(&tp, c);
+  tp.nsm = nsm;
+  tp.max_dyn = max_dyn;
+  tp.max_dyn2 = max_dyn2;
+  const StepPlan p = c.role == FR_ROLE_PREFIX ? make_plan(&tp, B, 0, P) : make_plan(&tp, B, P);
+  std::vector<int> v = {p.NT, p.Nt};
+  const ProjLayout* L[4] = {&tp.qkv, &tp.o, &tp.gu, &tp.dn};
+  const GemmPlan* G[4] = {&p.qkv, &p.o, &p.gu, &p.dn};
+  const int epi[4] = {EPI_QKV, EPI_RESID, EPI_GELU, EPI_RESID};
+  for (int i = 0; i < 4; ++i) {
+    const GemmPlan& g = *G[i];
+    const int b_kind = (i == 0 || i == 2) && tp.fp8 ? B_NORM : B_ROWS;
+    const int xb = (i == 1 || i == 3) && !tp.fp8;
+    const size_t smem = g.persist ? pt_smem_bytes(p.Nt, g.stages)
+                                  : gemm_smem_bytes(p.Nt, g.stages, b_kind, tp.fp8, g.S, ceil_div(L[i]->NKC, g.S), tp.w4,
+                                                    epi[i], p.H, xb, g.red_tok > 0 ? g.red_tok : p.Nt, g.kpu);
+    v.insert(v.end(), {g.S, g.stages, g.red_tok > 0 ? g.red_tok : p.Nt, g.persist, g.kpu, static_cast<int>(smem),
+                       L[i]->MB * p.NT, L[i]->NKC});
+  }
+  v.insert(v.end(), {p.attn_umma, p.attn_C, p.attn_KC});
+  const int n = static_cast<int>(v.size()) < n_out ? static_cast<int>(v.size()) : n_out;
+  for (int i = 0; i < n; ++i) out[i] = v[i];
+  return static_cast<int>(v.size());
 }
 
 const char* tensor_path_limits() {

@@ -40,6 +40,7 @@ struct TensorPath;
 
 bool tensor_path_supports(const fr_config& c);
 const char* tensor_path_limits();
+int tensor_path_debug_plan(const fr_config& c, int B, int P, int nsm, int max_dyn, int max_dyn2, int* out, int n_out);
 size_t tensor_path_bytes(const fr_config& c);
 int tensor_path_create(const fr_config& c, const TensorPathBuffers& b, TensorPath** out);
 int tensor_path_pack_layer(TensorPath* tp, int layer, const fr_layer_weights& w, const double sw[4]);

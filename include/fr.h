@@ -286,6 +286,19 @@ int fr_set_wait_limit(fr_handle* h, uint64_t limit_ns);
  * No counterpart in the pages: it stands in for a memory checker in debugging. */
 int fr_device_checks(void);
 
+/* fr_debug_plan -- host only, no device: the tensor-core path's launch plan of one fr_denoise call of
+ * batch B and prefix length P (for an FR_ROLE_PREFIX config: the pass over P tokens) on a device with
+ * nsm SMs, max_dyn bytes of dynamic shared memory per CTA and max_dyn2 bytes per CTA when two share an
+ * SM.  No counterpart in the pages: it lets the host logic that sizes every launch be tested without a
+ * GPU.  out[0..n_out) receives: NT, Nt (token tiles, tokens per tile); then for the QKV, O, gate|up and
+ * down projections in turn eight ints each: split-K S, ring slots, tokens per epilogue staging pass,
+ * persistent kernel (0/1), k-chunks per ring slot, dynamic shared memory (bytes), tiles (m-blocks x NT),
+ * k-chunks of 64 bf16 / 128 e4m3 inputs; then the attention kernel (1: tcgen05), its key chunks and keys
+ * per chunk.  Returns the number of entries of the plan (37; fewer are written if n_out is smaller) or
+ * FR_ERR_ARG, the configuration errors of fr_create, FR_ERR_UNSUPPORTED (outside the tensor-core
+ * path), FR_ERR_SHAPE (B or P out of range). */
+int fr_debug_plan(const fr_config* cfg, int B, int P, int nsm, int max_dyn, int max_dyn2, int* out, int n_out);
+
 /* fr_debug_limit_extent -- checked builds: declare a smaller extent (elements of the buffer's type;
  * bytes for the tiled operands) for one of the handle's buffers "h", "q", "kv", "xbuf", "obuf",
  * "ubuf", "ssq" or "x" (0 restores the real one), so that the bounds checks can be exercised without
