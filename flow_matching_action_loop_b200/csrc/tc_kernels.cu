@@ -736,6 +736,7 @@ constexpr int PT_KPS = 2;         // k-chunks per ring slot: two large copies pe
 struct PtSmem {
   uint64_t full_a[MAX_STAGES], full_b[MAX_STAGES], empty[MAX_STAGES];
   uint64_t tfull[2], tempty[2];   // accumulator a: MMAs done / drained by the epilogue
+  uint64_t fin;                   // every MMA of the CTA done (before tensor memory is freed)
   uint32_t tmem_base;
   float rstd[NT_MAX];
 };
@@ -777,6 +778,7 @@ __global__ void __launch_bounds__(PT_THREADS, 1) k_gemm_gelu_pt(const __grid_con
       mbar_init(&sh.tfull[i], 1);
       mbar_init(&sh.tempty[i], PT_EPI);
     }
+    mbar_init(&sh.fin, 1);
     pt_fail = 0;
     fence_mbar_init();
   }
@@ -842,6 +844,7 @@ __global__ void __launch_bounds__(PT_THREADS, 1) k_gemm_gelu_pt(const __grid_con
         const int acc = i & 1;
         if (i >= 2 && !mbar_wait(&sh.tempty[acc], ((i >> 1) - 1) & 1, WAIT_LIMIT_NS)) {
           report_timeout(a.status, 0xB200);
+          ok = false;
           break;
         }
         tc_fence_after();
@@ -867,6 +870,10 @@ __global__ void __launch_bounds__(PT_THREADS, 1) k_gemm_gelu_pt(const __grid_con
         }
         if (ok) mma_commit(&sh.tfull[acc]);
       }
+      // every MMA issued has completed before the accumulators are freed, also when a wait gave up and
+      // no tile commit tracks the last ones (on the normal path the epilogue has waited for them already)
+      mma_commit(&sh.fin);
+      if (!mbar_wait(&sh.fin, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0xB202);
     }
   } else {
     // ---------------- epilogue (warps 2-9; warp w reads the TMEM lane quadrant w % 4, warps 2-5 the
@@ -1329,7 +1336,7 @@ __host__ __device__ __forceinline__ UAttnGeom uattn_geom(int dh) {
 template <int DH>
 __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_constant__ AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t dsm[];
-  __shared__ uint64_t bar_s[2], bar_o[2], bar_p[2], kfull[2], vfull[2], stage_bar;
+  __shared__ uint64_t bar_s[2], bar_o[2], bar_p[2], kfull[2], vfull[2], stage_bar, fin_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;             // a wait gave up: the other role stops waiting too
   __shared__ float inv_den[128];
@@ -1370,6 +1377,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
       mbar_init(&vfull[i], 1);
     }
     mbar_init(&stage_bar, 1);
+    mbar_init(&fin_bar, 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -1481,6 +1489,10 @@ __global__ void __launch_bounds__(UA_THREADS, 1) k_attn_umma(const __grid_consta
       *abort_v = 1;
       report_timeout(a.status, 0x700);
     }
+    // every MMA issued has completed before tensor memory is read back or freed, also after a give-up
+    // (on the normal path the softmax threads wait for the last O += P V as well)
+    mma_commit(&fin_bar);
+    if (!mbar_wait(&fin_bar, 0, WAIT_LIMIT_NS)) report_timeout(a.status, 0x705);
   } else if (sm_thread) {
     // ---------------- online softmax (two threads per row, each half of the keys' exponentials)
     const float sl2 = a.scale * 1.4426950408889634f;   // scores in log2 units
