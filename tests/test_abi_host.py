@@ -66,6 +66,9 @@ def test_invalid_configs_rejected_before_any_device_work(abi):
         (abi.make_config(base, path=7), abi.FR_ERR_ARG),
         (abi.make_config(base, path=abi.FR_PATH_TENSOR), abi.FR_ERR_UNSUPPORTED),   # f32 has no tensor path
     ]
+    # empty inputs: no Euler step, no action row or feature, an empty prefix or batch, no width
+    bad += [(abi.make_config(base.replace(**{f: 0})), abi.FR_ERR_ARG)
+            for f in ("K", "H", "A", "P", "B", "D", "F", "Hq", "Hkv", "time_dim")]
     for cfg, code in bad:
         with pytest.raises(abi.FrError) as ei:
             abi.fr_create(cfg, 0)
