@@ -45,10 +45,6 @@ __device__ __forceinline__ void report_timeout(unsigned* status, uint32_t where)
   }
 }
 
-__device__ __forceinline__ uint8_t to_e4m3(float v) {
-  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
-}
-
 // GeLU in its tanh form, 0.5·g·(1 + tanh z) with z = sqrt(2/pi)·(g + 0.044715·g³), evaluated as
 // g·σ(2z) = g / (1 + e^{-2z}) (the identity 1 + tanh z = 2 / (1 + e^{-2z})): one exponential and one
 // fast division instead of a full tanh. The exponent is capped at 80 so the denominator stays far
@@ -91,8 +87,6 @@ __device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc, bool va
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-// every committed group of this thread but the most recent one has completed
-__device__ __forceinline__ void cp_async_wait_one_pending() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
