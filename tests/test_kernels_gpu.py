@@ -3,8 +3,6 @@
 Tolerance per (sample, query head): relative L2 <= 1e-2 and cosine >= 0.9999 -- the output is
 rounded to bf16 and P is rounded to bf16 inside the kernel (flash-attention practice).
 """
-import math
-
 import numpy as np
 import pytest
 

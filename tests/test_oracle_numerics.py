@@ -8,7 +8,6 @@ import math
 import os
 
 import numpy as np
-import pytest
 import torch
 
 from oracle import oracle as O
