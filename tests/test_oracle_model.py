@@ -155,10 +155,10 @@ def _as_f64(w):
     return {k: (v if k == "layers" else np.asarray(v, np.float64)) for k, v in w.items()}
 
 
-def test_velocity_matches_loop_formulation():
+def _velocity_case():
+    """The micro workload with non-trivial gains and biases, so that their placement is exercised."""
     inp = synthetic.make_inputs(MICRO, seed=11)
     w = inp["weights"]
-    # non-trivial gains and biases so that their placement is exercised
     rng = np.random.default_rng(12)
     for key in ("b_in", "b_out", "b_t1", "b_t2"):
         w[key] = rng.standard_normal(w[key].shape).astype(np.float32)
@@ -166,15 +166,74 @@ def test_velocity_matches_loop_formulation():
     for lw in w["layers"]:
         lw["g1"] = (1 + 0.3 * rng.standard_normal(MICRO.D)).astype(np.float32)
         lw["g2"] = (1 + 0.3 * rng.standard_normal(MICRO.D)).astype(np.float32)
-    model = O.PreparedModel(MICRO, w)
-    b = 1
+    return inp, w
+
+
+def _velocity_pairs(inp, w_oracle, w_loops, b=1):
+    """(oracle, loop formulation) velocities of sample b at every step of the grid."""
+    model = O.PreparedModel(MICRO, w_oracle)
     kv_k, kv_v = O._sample_kv(model, inp["prefix_k"], inp["prefix_v"], b)
     x = np.asarray(inp["x0"][b], np.float64)
-    for k_step, t in enumerate(O.time_grid(MICRO.K)[0]):
-        got = O.velocity(model, x, k_step, t, kv_k, kv_v)
-        want = _velocity_loops(MICRO, w, x, t, inp["prefix_k"][:, b], inp["prefix_v"][:, b])
+    return [(O.velocity(model, x, k_step, t, kv_k, kv_v),
+             _velocity_loops(MICRO, w_loops, x, t, inp["prefix_k"][:, b], inp["prefix_v"][:, b]))
+            for k_step, t in enumerate(O.time_grid(MICRO.K)[0])]
+
+
+def test_velocity_matches_loop_formulation():
+    inp, w = _velocity_case()
+    for got, want in _velocity_pairs(inp, w, w):
         # the oracle's RoPE tables are rounded to float32 once; the loops use float64 angles
         assert np.allclose(got, want, rtol=1e-5, atol=1e-6), (got, want)
+
+
+def test_velocity_loop_pin_catches_planted_mistakes(monkeypatch):
+    """Mistakes planted in the oracle (CPU only) make the loop comparison above fail by far more
+    than its tolerance: the pin is not blind to a wrong sign, index, pairing, scale or operand."""
+    inp, w = _velocity_case()
+
+    def worst(w_oracle=w):
+        return max(float(np.linalg.norm(g - v) / np.linalg.norm(v)) for g, v in _velocity_pairs(inp, w_oracle, w))
+
+    assert worst() < 1e-5
+    real = {n: getattr(O, n) for n in ("rope_rotate", "attention", "_project", "sinusoidal_embedding", "gelu_tanh")}
+
+    def interleaved(z, c, s):   # RoPE on (2j, 2j+1) pairs instead of rotate-half (j, j + dh/2)
+        z = np.asarray(z, np.float64)
+        ev, od = z[..., 0::2], z[..., 1::2]
+        out = np.empty_like(z)
+        out[..., 0::2], out[..., 1::2] = ev * c - od * s, ev * s + od * c
+        return out
+
+    def kv_by_modulo(q, k, v):   # query head j reads KV head j mod Hkv instead of floor(j Hkv / Hq)
+        Hkv = k.shape[0]
+        return np.stack([real["attention"](q[j:j + 1], k[j % Hkv:j % Hkv + 1], v[j % Hkv:j % Hkv + 1])[0]
+                         for j in range(q.shape[0])])
+
+    def gate_up_swapped(model, l, which, a, ws, scales, record):
+        out = real["_project"](model, l, which, a, ws, scales, record)
+        return out[::-1] if which == "gu" else out
+
+    def cos_half_first(t, dim, base):
+        e = real["sinusoidal_embedding"](t, dim, base)
+        return np.concatenate([e[dim // 2:], e[:dim // 2]])
+
+    plants = {
+        "RoPE rotation sign": ("rope_rotate", lambda z, c, s: real["rope_rotate"](z, c, -s)),
+        "RoPE pairing": ("rope_rotate", interleaved),
+        "GQA head mapping": ("attention", kv_by_modulo),
+        "attention scale": ("attention", lambda q, k, v: real["attention"](q * math.sqrt(q.shape[-1]), k, v)),
+        "gate and up": ("_project", gate_up_swapped),
+        "time-embedding halves": ("sinusoidal_embedding", cos_half_first),
+        "MLP residual": ("gelu_tanh", lambda z: np.zeros_like(np.asarray(z, np.float64))),
+    }
+    for what, (name, fn) in plants.items():
+        monkeypatch.setattr(O, name, fn)
+        assert worst() > 1e-3, what
+        monkeypatch.setattr(O, name, real[name])
+    # gains in the wrong place: the pre-MLP norm with the pre-attention gain, the final norm with none
+    swapped = dict(w, layers=[dict(lw, g2=lw["g1"]) for lw in w["layers"]])
+    assert worst(swapped) > 1e-3
+    assert worst(dict(w, g_f=np.ones_like(w["g_f"]))) > 1e-3
 
 
 # ---------------------------------------------------------------- loop closed forms
