@@ -76,9 +76,9 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint3
 // ------------------------------------------------------------------ tiled copies (TMA engine, tensor maps)
 // global -> shared through a tensor map held in a __grid_constant__ kernel parameter (generic address
 // of the parameter); box elements past the tensor's extents are written as zeros.  The innermost
-// coordinate times the element size must be a multiple of 16 bytes.  No cluster multicast.  (On this
-// part the copy engine of an SM takes about a third of a microsecond per copy up to ~40 KB, one copy
-// at a time: few large copies, not many small ones.)
+// coordinate times the element size must be a multiple of 16 bytes.  Each copy fills this CTA's own
+// shared memory only.  (On this part the copy engine of an SM takes about a third of a microsecond per
+// copy up to ~40 KB, one copy at a time: few large copies, not many small ones.)
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, int x, int y, int z, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
