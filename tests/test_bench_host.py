@@ -102,3 +102,29 @@ def test_options_warmup_floor_and_persistent_headline_only():
     assert a.exec_mode == "graph" and not a.no_extra and a.workload == "pi05_bf16_b32"
     with pytest.raises(SystemExit):
         bench.parse_args(["--exec", "eager"])
+
+
+def test_peaks_come_from_the_measured_file_else_the_fallback(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.load_peaks() == (6650.0, 1590.0, 1400.0, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(
+        '{"hbm_gbs": 7012.5, "bf16_tflops": 1702.0, "bf16_tflops_sustained": 1455.5, "sm_mhz": 1965}')
+    assert bench.load_peaks() == (7012.5, 1702.0, 1455.5, "measured")
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 7012.5}')   # incomplete: not used
+    assert bench.load_peaks()[3] == "fallback"
+
+
+def test_clock_samples_summarise_median_max_and_active_reasons():
+    s = bench.ClockSampler(0)
+    # index, sm, max sm, power, active mask, hw_slowdown, hw_thermal, sw_thermal, sw_power_cap
+    s.lines = ["0, 1965, 1965, 702.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+               "0, 1800, 1965, 998.7, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+               "0, 1950, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+               "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",   # unparsable: skipped
+               "garbled"]
+    got = s.summary()
+    assert got == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    s.lines = ["0, 1200, 1965, 500.0, 0x0000000000000040, Active, Not Active, Active, Not Active"]
+    assert s.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    s.lines = []
+    assert s.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
