@@ -27,6 +27,9 @@ def test_every_header_function_is_exported(abi):
     lib = ctypes.CDLL(abi.LIB_PATH)
     for n in names:
         assert getattr(lib, n) is not None
+    # the binding declares every call's signature: no pointer or size goes through ctypes' default int
+    bound = abi.load_library()
+    assert [n for n in names if getattr(bound, n).argtypes is None] == []
 
 
 def test_rope_tables_byte_identical_to_oracle(abi):
