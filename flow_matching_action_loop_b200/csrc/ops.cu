@@ -147,6 +147,10 @@ int fr_ops_sync_status(fr_stream_t stream) {
     set_error("device wait gave up in an op (phase word 0x%08x, block %u)", st[1], st[2]);
     return FR_ERR_TIMEOUT;
   }
+  if (st[0] & ST_BOUNDS) {   // checked builds
+    set_error("device bounds check failed in an op (where 0x%08x, index %u)", st[1], st[2]);
+    return FR_ERR_DEVICE;
+  }
   return FR_OK;
 }
 

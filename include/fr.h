@@ -446,8 +446,10 @@ int fr_attention(const void* q, const void* k, const void* v, void* o, int B, in
 /*
  * fr_ops_sync_status -- synchronise `stream`, then read and clear the status word that the
  * stand-alone ops (fr_attention, fr_attention_noalloc) of the current device latch their
- * device-side failures in.  Returns FR_OK or FR_ERR_TIMEOUT (the message gives the wait's
- * where-code and block).  The word is one per device, shared by every op call on it.
+ * device-side failures in.  Returns FR_OK, FR_ERR_TIMEOUT (the message gives the wait's
+ * where-code and block) or, in a checked build, FR_ERR_DEVICE (a store's index failed its
+ * bounds check: where-code and index).  The word is one per device, shared by every op call
+ * on it.
  * Errors: FR_ERR_CUDA.
  */
 int fr_ops_sync_status(fr_stream_t stream);
