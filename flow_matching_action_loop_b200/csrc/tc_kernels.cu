@@ -1982,26 +1982,32 @@ cudaError_t tc_kernels_init() {
   return cudaSuccess;
 }
 
+// Dynamic shared memory a GEMM CTA may use alone on an SM; 0 when the device cannot be queried (the
+// plans then find that nothing fits and the launch reports it).
 int max_dynamic_smem() {
   int dev = 0, optin = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  cudaFuncAttributes fa;
-  cudaFuncGetAttributes(&fa, gemm_kernel(EPI_RESID, 0, 0, 0));
-  return optin - static_cast<int>(fa.sharedSizeBytes);
+  cudaFuncAttributes fa{};
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+      cudaFuncGetAttributes(&fa, gemm_kernel(EPI_RESID, 0, 0, 0)) != cudaSuccess)
+    return 0;
+  return std::max(0, optin - static_cast<int>(fa.sharedSizeBytes));
 }
 
+// ... and when two GEMM CTAs share an SM (0 as above).
 int pair_dynamic_smem() {
   int dev = 0, per_sm = 0, reserved = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-  cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+    return 0;
   int stat = 0;
   for (int epi : {EPI_QKV, EPI_RESID, EPI_GELU}) {
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, gemm_kernel(epi, 0, 0, 0)) == cudaSuccess) stat = std::max(stat, static_cast<int>(fa.sharedSizeBytes));
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, gemm_kernel(epi, 0, 0, 0)) != cudaSuccess) return 0;
+    stat = std::max(stat, static_cast<int>(fa.sharedSizeBytes));
   }
-  return per_sm / 2 - reserved - stat;
+  return std::max(0, per_sm / 2 - reserved - stat);
 }
 
 // One instantiation per (epilogue, operand type, B-operand kind, 4-bit weights) in use.
