@@ -880,7 +880,10 @@ int fr_set_graph_capacity(fr_handle* h, int capacity) {
     set_error("fr_set_graph_capacity: NULL handle or capacity < 1");
     return FR_ERR_ARG;
   }
-  if (h->tp) return tensor_path_set_graph_capacity(h->tp, capacity);
+  if (h->tp) {
+    FR_CUDA(cudaSetDevice(h->device));   // evicted graphs are destroyed on the handle's device
+    return tensor_path_set_graph_capacity(h->tp, capacity);
+  }
   return FR_OK;
 }
 
@@ -986,6 +989,7 @@ int fr_denoise(fr_handle* h, const float* x0_dev, float* x_out_dev, int B, fr_st
     set_error("fr_denoise: fp8 handle without activation scales (run fr_calibrate or fr_set_scales)");
     return FR_ERR_STATE;
   }
+  FR_CUDA(cudaSetDevice(h->device));   // the handle's buffers, graphs and kernels live there
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t xbytes = static_cast<size_t>(B) * c.H * c.A * sizeof(float);
   if (h->path == FR_PATH_TENSOR) {
@@ -1014,6 +1018,7 @@ int fr_calibrate(fr_handle* h, const float* x0_dev, const void* pk_dev, const vo
     set_error("fr_calibrate: no weights loaded");
     return FR_ERR_STATE;
   }
+  FR_CUDA(cudaSetDevice(h->device));
   int rc = fr_set_prefix_kv(h, pk_dev, pv_dev, B, P, 0, stream);
   if (rc) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -26,6 +26,9 @@
  *     call, device pointers until the work queued on `stream` has finished.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
  *     that take a stream are asynchronous unless stated otherwise.
+ *   - A call on a handle that does device work first makes the handle's device
+ *     (fr_create's `device`) the calling thread's current device, and leaves it
+ *     current; `stream` must belong to that device.
  *   - Device-side failures (a bounded wait that gave up, a device bounds check)
  *     are latched in a device status word; fr_sync_status() reads and clears it.
  */
