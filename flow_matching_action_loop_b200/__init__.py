@@ -57,6 +57,8 @@ class ActionExpertLoop:
         torch = self._torch
         if not isinstance(t, torch.Tensor) or t.device.type != "cuda" or t.dtype != dtype or not t.is_contiguous():
             raise FrError(FR_ERR_ARG, name, f"expected a contiguous {dtype} CUDA tensor")
+        if t.device.index != self.device:   # the kernels run on the handle's device
+            raise FrError(FR_ERR_ARG, name, f"expected a tensor on cuda:{self.device}, got {t.device}")
         if tuple(t.shape) != tuple(shape):
             raise FrError(FR_ERR_SHAPE, name, f"expected shape {tuple(shape)}, got {tuple(t.shape)}")
         return t.data_ptr()
@@ -214,6 +216,8 @@ class PrefixPass:
         if not isinstance(emb, torch.Tensor) or emb.device.type != "cuda" or emb.dtype != torch.bfloat16 \
                 or not emb.is_contiguous() or emb.dim() != 3 or emb.shape[2] != self.cfg.D:
             raise FrError(FR_ERR_ARG, "fr_prefill", "expected a contiguous bf16 CUDA tensor [B][P][D]")
+        if emb.device.index != self.device:
+            raise FrError(FR_ERR_ARG, "fr_prefill", f"expected a tensor on cuda:{self.device}, got {emb.device}")
         B, P = emb.shape[0], emb.shape[1]
         fr_prefill(self.h, emb.data_ptr(), B, P, expert.h if expert is not None else None, self._stream())
         if expert is not None:

@@ -919,6 +919,10 @@ int fr_prefill(fr_handle* bb, const void* emb_dev, int B, int P, fr_handle* ex, 
       set_error("fr_prefill: the destination is not an expert handle");
       return FR_ERR_STATE;
     }
+    if (ex->device != bb->device) {   // the copy kernel runs on the pass's device and writes the expert's cache
+      set_error("fr_prefill: the expert handle is on device %d, the prefix pass on device %d", ex->device, bb->device);
+      return FR_ERR_ARG;
+    }
     if (e.L != c.L || e.Hkv != c.Hkv || e.dh != c.dh || !ex->kv_bf || B > e.B_max || P > e.P_max) {
       set_error("fr_prefill: expert KV [L=%d Hkv=%d dh=%d, B_max=%d P_max=%d, %s] cannot take the pass's "
                 "[L=%d Hkv=%d dh=%d] for B=%d P=%d",

@@ -322,9 +322,9 @@ int fr_debug_limit_extent(fr_handle* h, const char* buffer, uint64_t elems);
  * KV for slots 0..B-1, which then holds (B, P) as after fr_set_prefix_kv with
  * FR_PREFIX_K_ROTATED; the expert needs the backbone's L, Hkv and dh and a bf16 KV cache.
  * Asynchronous on `stream`; allocates nothing.
- * Errors: FR_ERR_ARG (NULL), FR_ERR_STATE (not a prefix handle, no weights, expert not an
- * expert handle), FR_ERR_SHAPE (B > B_max, P > H of the backbone or P_max of the expert, KV
- * shapes differ), FR_ERR_CUDA.
+ * Errors: FR_ERR_ARG (NULL, expert handle on another device), FR_ERR_STATE (not a prefix
+ * handle, no weights, expert not an expert handle), FR_ERR_SHAPE (B > B_max, P > H of the
+ * backbone or P_max of the expert, KV shapes differ), FR_ERR_CUDA.
  */
 int fr_prefill(fr_handle* backbone, const void* emb_dev, int B, int P, fr_handle* expert, fr_stream_t stream);
 
