@@ -28,7 +28,8 @@
  *     that take a stream are asynchronous unless stated otherwise.
  *   - A call on a handle that does device work first makes the handle's device
  *     (fr_create's `device`) the calling thread's current device, and leaves it
- *     current; `stream` must belong to that device.
+ *     current; `stream` must belong to that device, and device pointers passed
+ *     in must point to its memory (the library does not enable peer access).
  *   - Device-side failures (a bounded wait that gave up, a device bounds check)
  *     are latched in a device status word; fr_sync_status() reads and clears it.
  */
