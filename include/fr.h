@@ -261,8 +261,8 @@ int fr_launches_per_call(const fr_handle* h, int B);
  * one unit).  FR_EXEC_PERSISTENT: one cooperative launch of a persistent kernel runs the whole
  * call, one CTA per SM, its phases handed over through bounded device-side waits; it serves bf16
  * handles without adaRMS whose calls have B*H <= 64 tokens.  FR_EXEC_GRAPH: one CUDA graph of
- * K*(2 + 5L) kernels chained by programmatic dependent launch (every other shape).  FR_EXEC_AUTO
- * (the default) takes the persistent kernel wherever it applies.
+ * K*(2 + 5L) kernels chained by programmatic dependent launch, for every shape.  FR_EXEC_AUTO
+ * (the default) replays the graph, which is the faster of the two as measured at pi0.5 batch 1.
  */
 enum { FR_EXEC_AUTO = 0, FR_EXEC_GRAPH = 1, FR_EXEC_PERSISTENT = 2 };
 
