@@ -108,6 +108,12 @@ int validate(const fr_config& c) {
     set_error("fr_create: bad dtype/path enum");
     return FR_ERR_ARG;
   }
+  // RMSNorm's eps, RoPE's theta and the time embedding's base: finite, and positive where a power is taken
+  if (!std::isfinite(c.eps) || c.eps < 0.f || !std::isfinite(c.rope_theta) || c.rope_theta <= 0.f ||
+      !std::isfinite(c.time_base) || c.time_base <= 0.f) {
+    set_error("fr_create: need eps >= 0, rope_theta > 0 and time_base > 0, all finite");
+    return FR_ERR_ARG;
+  }
   if ((c.dh & 1) || (c.time_dim & 1) || (c.Hq % c.Hkv)) {
     set_error("fr_create: dh and time_dim must be even and Hq a multiple of Hkv");
     return FR_ERR_UNSUPPORTED;

@@ -146,8 +146,9 @@ typedef struct fr_weights {
  * fr_create -- validate the config, make `device` current and allocate ALL
  * device memory of the handle: packed weights, the KV cache
  * [L][B_max][Hkv][P_max+H][dh], activations, workspaces and status words.
- * Errors: FR_ERR_ARG (NULL), FR_ERR_UNSUPPORTED (sizes the kernels do not
- * implement), FR_ERR_CUDA (allocation).  *out is NULL on error.
+ * Errors: FR_ERR_ARG (NULL, a size below 1, an unknown dtype, path or role),
+ * FR_ERR_UNSUPPORTED (sizes the kernels do not implement), FR_ERR_CUDA
+ * (allocation).  *out is NULL on error.
  */
 int fr_create(const fr_config* cfg, int device, fr_handle** out);
 
@@ -207,7 +208,9 @@ int fr_denoise(fr_handle* h, const float* x0_dev, float* x_out_dev, int B, fr_st
  * s_act: host [L][4] activation scales in the order (qkv input, o input,
  * gate|up input, down input); s_w: host [L][4] weight scales, same order
  * (may be NULL).  n must be L*4.  fr_set_scales also recomputes alpha.
- * Errors: FR_ERR_ARG, FR_ERR_STATE (not fp8, or scales not set for get).
+ * Errors: FR_ERR_ARG (NULL, a scale that is not positive and finite),
+ * FR_ERR_SHAPE (n != L*4), FR_ERR_STATE (not fp8, no weights for set, scales
+ * not set for get), FR_ERR_CUDA.
  */
 int fr_get_scales(const fr_handle* h, float* s_act, float* s_w, int n);
 int fr_set_scales(fr_handle* h, const float* s_act, int n);

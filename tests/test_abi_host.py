@@ -72,6 +72,10 @@ def test_invalid_configs_rejected_before_any_device_work(abi):
     # empty inputs: no Euler step, no action row or feature, an empty prefix or batch, no width
     bad += [(abi.make_config(base.replace(**{f: 0})), abi.FR_ERR_ARG)
             for f in ("K", "H", "A", "P", "B", "D", "F", "Hq", "Hkv", "time_dim")]
+    # constants that would give NaN tables: a negative eps, a non-positive or non-finite base
+    bad += [(abi.make_config(base.replace(**{f: v})), abi.FR_ERR_ARG)
+            for f, v in (("eps", -1e-6), ("eps", float("nan")), ("rope_theta", 0.0), ("rope_theta", float("inf")),
+                         ("time_base", -10000.0))]
     for cfg, code in bad:
         with pytest.raises(abi.FrError) as ei:
             abi.fr_create(cfg, 0)
