@@ -411,8 +411,8 @@ int fr_capsule_save(const fr_handle* h, void* cap_dev, size_t cap_bytes, int B, 
  * x_dev [B][H][A] receives the capsule's x of the same samples.  Asynchronous.
  * Errors: FR_ERR_ARG (NULL, not a capsule description, map entry out of range),
  * FR_ERR_SHAPE (capsule of a handle of another shape, B outside [1, B_max], desc->P >
- * P_max, B > desc->B without a map), FR_ERR_STATE (x_dev given, capsule without x),
- * FR_ERR_CUDA.
+ * P_max, B > desc->B without a map), FR_ERR_STATE (not an expert handle; x_dev given,
+ * capsule without x), FR_ERR_CUDA.
  */
 int fr_capsule_restore(fr_handle* h, const void* cap_dev, const fr_capsule* desc, const int* map, int B,
                        float* x_dev, fr_stream_t stream);
